@@ -1,0 +1,284 @@
+"""Pins of the fp64 oracle to facts fixed outside the oracle itself.
+
+Each test checks the oracle against something it cannot agree with by
+construction: a hand-derived worked example, counts printed by the pages,
+the bf16 format definition, a closed-form identity of the method, or a
+brute-force / naive-loop computation on tiny inputs.  Together they are
+chosen so that a dropped term, a flipped sign, a swapped index or a
+transposed operand anywhere in the oracle fails at least one of them.
+
+Method source: "MoVA: routing the value vectors, and why the KV cache does
+not notice", sections "Where the routing happens" and "So what does it
+cost?".
+"""
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+
+from oracle import mova_oracle as O
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _load(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+def _naive_silu(z):
+    return z / (1.0 + math.exp(-z))
+
+
+def _naive_matvec(W, x):
+    # W: list of rows (n x d), x: length d.  Plain loops, no numpy.
+    return [sum(W[r][j] * x[j] for j in range(len(x))) for r in range(len(W))]
+
+
+# ---------------------------------------------------------------------------
+# Worked examples derived by hand (tests/golden/worked_example.json)
+# ---------------------------------------------------------------------------
+
+
+@pytest.mark.parametrize("case", _load("worked_example.json")["cases"], ids=lambda c: c["name"])
+def test_worked_example(case):
+    ln3 = math.log(3.0)
+    p = np.array(case["p"], dtype=np.float64)
+    x = np.array(case["x"], dtype=np.float64)
+    # Router weight chosen so that logit_e = ln(p_e / (1 - p_e)) for x = [1].
+    Wr = np.log(p / (1.0 - p))[:, None]
+    br = np.array(case["br"], dtype=np.float64)
+    Wv = np.array(case["Wv_ln3"], dtype=np.float64) * ln3
+    v, r = O.value_routed(x, Wr, br, Wv, case["k"], case["scale"])
+    assert r["idx"].tolist() == case["idx"]
+    np.testing.assert_allclose(r["w"], np.array(case["w"]), rtol=0, atol=1e-14)
+    np.testing.assert_allclose(v, np.array(case["v_ln3"]) * ln3, rtol=0, atol=1e-14)
+
+
+def test_sigmoid_silu_closed_forms():
+    ln3 = math.log(3.0)
+    assert O.sigmoid(np.array(0.0)) == 0.5
+    np.testing.assert_allclose(O.sigmoid(np.array([ln3, -ln3])), [0.75, 0.25], atol=1e-15)
+    np.testing.assert_allclose(O.silu(np.array([0.0, ln3, -ln3])), [0.0, 0.75 * ln3, -0.25 * ln3],
+                               atol=1e-15)
+    # SiLU(-z) = SiLU(z) - z, and SiLU(z) -> z for large z.
+    z = np.linspace(-8, 8, 33)
+    np.testing.assert_allclose(O.silu(-z), O.silu(z) - z, atol=1e-14)
+    assert abs(O.silu(np.array(40.0)) - 40.0) < 1e-12
+
+
+# ---------------------------------------------------------------------------
+# Numbers printed by the pages (tests/golden/page_counts.json)
+# ---------------------------------------------------------------------------
+
+
+def test_page_counts():
+    g = _load("page_counts.json")
+    d, E, k = g["d_model"], g["n_experts"], g["top_k"]
+    n = g["heads"] * g["head_dim"]
+    assert n == 1024
+    per_layer = O.expert_params_per_layer(E, d, n)
+    assert round(per_layer / 1e6, 1) == g["expert_params_per_layer_rounded_M"]
+    assert per_layer * g["mova_layers"] == g["expert_params_all_layers"]
+    assert round(O.macs_per_token(d, n, k) / 1e6, 2) == g["macs_per_token_rounded_M"]
+    assert round(O.expert_params_per_layer(1, d, n) / 1e6, 2) == g["dense_v_proj_params_rounded_M"]
+    assert round(O.router_params(d, E) / 1e3) == g["router_params_rounded_K"]
+    assert O.flops_per_token(d, n, k) == 2 * 10_485_760
+
+
+def test_bf16_format():
+    for hexbits, val in _load("bf16_patterns.json")["patterns"]:
+        got = O.bf16_bits_to_f64(np.array([int(hexbits, 16)], dtype=np.uint16))[0]
+        assert got == val and math.copysign(1.0, got) == math.copysign(1.0, val), hexbits
+
+
+# ---------------------------------------------------------------------------
+# Identities of the method
+# ---------------------------------------------------------------------------
+
+
+def _rand_case(rng, T=5, d=12, E=8, n=6):
+    x = rng.standard_normal((T, d))
+    Wr = rng.standard_normal((E, d)) * 0.3
+    br = rng.standard_normal(E) * 0.1
+    Wv = rng.standard_normal((E, n, d)) / math.sqrt(d)
+    return x, Wr, br, Wv
+
+
+@pytest.mark.parametrize("k", [1, 2, 4])
+def test_identical_experts_give_scaled_silu(k):
+    """All experts equal W: the renormalised weights sum to 1, so
+    v = scale * SiLU(W x) whatever the routing (checked with naive loops)."""
+    rng = np.random.default_rng(1)
+    x, Wr, br, _ = _rand_case(rng)
+    d, E, n = x.shape[1], Wr.shape[0], 6
+    W = rng.standard_normal((n, d)) / math.sqrt(d)
+    Wv = np.broadcast_to(W, (E, n, d))
+    v, _ = O.value_routed(x, Wr, br, Wv, k, 2.5)
+    for t in range(x.shape[0]):
+        h = _naive_matvec(W.tolist(), x[t].tolist())
+        ref = [2.5 * _naive_silu(z) for z in h]
+        np.testing.assert_allclose(v[t], ref, rtol=1e-13, atol=1e-13)
+
+
+def test_single_expert_is_textbook_matvec():
+    """E = 1, k = 1: v = scale * SiLU(W x) for a non-square W (catches a
+    transposed expert operand)."""
+    rng = np.random.default_rng(2)
+    d, n = 7, 3
+    x = rng.standard_normal((4, d))
+    W = rng.standard_normal((1, n, d))
+    v, r = O.value_routed(x, rng.standard_normal((1, d)), np.zeros(1), W, 1, 2.5)
+    assert (r["idx"] == 0).all()
+    np.testing.assert_allclose(r["w"], 2.5)
+    for t in range(4):
+        h = _naive_matvec(W[0].tolist(), x[t].tolist())
+        np.testing.assert_allclose(v[t], [2.5 * _naive_silu(z) for z in h], rtol=1e-13)
+
+
+def test_k_equals_E_selection_irrelevant():
+    """k = E: every expert is selected, so the bias (which only steers the
+    selection) cannot change the output."""
+    rng = np.random.default_rng(3)
+    x, Wr, br, Wv = _rand_case(rng)
+    E = Wr.shape[0]
+    v1, _ = O.value_routed(x, Wr, br, Wv, E, 2.5)
+    v2, _ = O.value_routed(x, Wr, rng.standard_normal(E) * 5.0, Wv, E, 2.5)
+    np.testing.assert_allclose(v1, v2, rtol=1e-13, atol=1e-13)
+
+
+def test_weights_positive_and_sum_to_scale():
+    rng = np.random.default_rng(4)
+    x, Wr, br, _ = _rand_case(rng, T=50)
+    r = O.route(x, Wr, br, 4, 2.5)
+    assert (r["w"] > 0).all()
+    np.testing.assert_allclose(r["w"].sum(axis=1), 2.5, rtol=1e-14)
+    # Weights follow the unbiased sigmoid scores of the selected experts.
+    for t in range(x.shape[0]):
+        st = [1.0 / (1.0 + math.exp(-float(np.dot(x[t], Wr[e])))) for e in r["idx"][t]]
+        np.testing.assert_allclose(r["w"][t], [2.5 * s / sum(st) for s in st], rtol=1e-12)
+
+
+def test_bias_shift_invariance():
+    rng = np.random.default_rng(5)
+    x, Wr, br, Wv = _rand_case(rng, T=20)
+    v1, r1 = O.value_routed(x, Wr, br, Wv, 3, 2.5)
+    v2, r2 = O.value_routed(x, Wr, br + 0.37, Wv, 3, 2.5)
+    assert (r1["idx"] == r2["idx"]).all()
+    np.testing.assert_allclose(v1, v2, rtol=1e-13)
+
+
+# ---------------------------------------------------------------------------
+# Selection against brute force
+# ---------------------------------------------------------------------------
+
+
+def _brute_top_k(b_row, k):
+    """Best subset by sum of scores, lowest indices first among equals,
+    then ordered by descending score (ties: lower index first)."""
+    E = len(b_row)
+    best = None
+    for sub in itertools.combinations(range(E), k):
+        key = (sum(b_row[e] for e in sub), [-e for e in sub])
+        if best is None or key > best[0]:
+            best = (key, sub)
+    return sorted(best[1], key=lambda e: (-b_row[e], e))
+
+
+@pytest.mark.parametrize("E,k", [(6, 1), (6, 2), (6, 3), (7, 4), (8, 4)])
+def test_top_k_brute_force_random(E, k):
+    rng = np.random.default_rng(10 + E * 10 + k)
+    b = rng.standard_normal((40, E))
+    got = O.select_top_k(b, k)
+    for t in range(b.shape[0]):
+        assert got[t].tolist() == _brute_top_k(b[t].tolist(), k)
+
+
+@pytest.mark.parametrize("E,k", [(6, 2), (8, 4), (8, 3)])
+def test_top_k_brute_force_ties(E, k):
+    """Scores drawn from 3 values so that ties are everywhere: equal scores
+    go to the lower expert index."""
+    rng = np.random.default_rng(20 + E + k)
+    b = rng.integers(0, 3, size=(60, E)).astype(np.float64) * 0.5
+    got = O.select_top_k(b, k)
+    for t in range(b.shape[0]):
+        assert got[t].tolist() == _brute_top_k(b[t].tolist(), k)
+
+
+def test_route_brute_force_end_to_end():
+    """Tiny E, k: the whole route (logits by loops, sigmoid by math.exp,
+    best subset by enumeration) against the oracle."""
+    rng = np.random.default_rng(6)
+    T, d, E, k = 12, 5, 6, 2
+    x = rng.standard_normal((T, d))
+    Wr = rng.standard_normal((E, d))
+    br = rng.standard_normal(E) * 0.2
+    r = O.route(x, Wr, br, k, 2.5)
+    for t in range(T):
+        s = [1.0 / (1.0 + math.exp(-sum(x[t, j] * Wr[e, j] for j in range(d)))) for e in range(E)]
+        b = [s[e] + br[e] for e in range(E)]
+        sel = _brute_top_k(b, k)
+        assert r["idx"][t].tolist() == sel
+        tot = sum(s[e] for e in sel)
+        np.testing.assert_allclose(r["w"][t], [2.5 * s[e] / tot for e in sel], rtol=1e-12)
+
+
+def test_combine_naive_loops():
+    """The mixture against plain loops over tokens and slots, with the
+    routing given (also the routing-given mode's definition)."""
+    rng = np.random.default_rng(7)
+    T, d, E, n, k = 6, 5, 4, 3, 2
+    x = rng.standard_normal((T, d))
+    Wv = rng.standard_normal((E, n, d))
+    idx = np.array([rng.permutation(E)[:k] for _ in range(T)])
+    w = rng.random((T, k)) + 0.1
+    v = O.combine(x, idx, w, Wv)
+    for t in range(T):
+        acc = [0.0] * n
+        for slot in range(k):
+            h = _naive_matvec(Wv[idx[t, slot]].tolist(), x[t].tolist())
+            for c in range(n):
+                acc[c] += w[t, slot] * _naive_silu(h[c])
+        np.testing.assert_allclose(v[t], acc, rtol=1e-13, atol=1e-14)
+
+
+def test_gqa_shape_and_mapping():
+    v = np.arange(3 * 1024, dtype=np.float64).reshape(3, 1024)
+    g = O.as_gqa(v)
+    assert g.shape == (3, 8, 128)
+    for t, h, c in [(0, 0, 0), (1, 3, 5), (2, 7, 127)]:
+        assert g[t, h, c] == v[t, h * 128 + c]
+
+
+# ---------------------------------------------------------------------------
+# Grouping by expert against a pure-Python brute force
+# ---------------------------------------------------------------------------
+
+
+@pytest.mark.parametrize("T,E,k", [(1, 4, 1), (7, 5, 2), (33, 8, 4), (50, 64, 4)])
+def test_permutation_brute_force(T, E, k):
+    rng = np.random.default_rng(T * 100 + E)
+    idx = np.array([rng.permutation(E)[:k] for _ in range(T)])
+    p = O.permutation(idx, E)
+    flat = idx.reshape(-1).tolist()
+    perm = []
+    counts = []
+    for e in range(E):
+        mine = [f for f in range(len(flat)) if flat[f] == e]
+        counts.append(len(mine))
+        perm.extend(mine)
+    assert p["counts"].tolist() == counts
+    assert p["offsets"].tolist() == [sum(counts[:e]) for e in range(E + 1)]
+    assert p["perm"].tolist() == perm
+    for f in range(len(flat)):
+        assert perm[p["pos"][f]] == f
+
+
+def test_permutation_empty():
+    p = O.permutation(np.zeros((0, 4), dtype=np.int64), 8)
+    assert p["counts"].tolist() == [0] * 8
+    assert p["offsets"].tolist() == [0] * 9
+    assert p["perm"].size == 0 and p["pos"].size == 0
