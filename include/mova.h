@@ -1,0 +1,163 @@
+/*
+ * mova.h -- C ABI of the MoVA value path on NVIDIA B200 (sm_100a).
+ *
+ * MoVA (Mixture-of-Value Attention) replaces an attention layer's GQA value
+ * projection by a router over E value experts, each a full d -> n value
+ * projection.  For every token t with hidden state x[t] (length d):
+ *
+ *   logits[t,e] = sum_j x[t,j] * Wr[e,j]          (router, no bias, fp32)
+ *   s[t,e]      = sigmoid(logits[t,e])
+ *   idx[t,:]    = the k experts with the largest s[t,e] + br[e]
+ *                 (descending; equal scores -> lower expert index first)
+ *   w[t,slot]   = scale * s[t,idx[t,slot]] / sum_slots s[t,idx[t,slot']]
+ *   v[t,:]      = sum_{slot = 0..k-1, ascending} w[t,slot] * SiLU(Wv[idx[t,slot]] x[t])
+ *
+ * and v, of shape (T, n) = (T, heads, head_dim), is exactly the tensor a
+ * GQA v_proj would have produced.  Source: "MoVA: routing the value vectors,
+ * and why the KV cache does not notice" (ai.thesatyajit.com), section
+ * "Where the routing happens" (router call, gate with the bias handed
+ * separately, top-4, scale 2.5, SiLU mixture, reshape to 128-wide heads);
+ * section "So what does it cost?" (64 experts of 2560 x 1024 per layer).
+ * The routing-given entry point recomputes v from a stored x and its routing
+ * as in the compact cache of "IFM K2 Horizon Deep Dive ...", Section 4,
+ * Option B.
+ *
+ * Conventions for every entry point:
+ *  - All tensor pointers are DEVICE pointers owned by the caller, row-major
+ *    and contiguous, 16-byte aligned.  The library never allocates.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *    stream).  Every compute call is asynchronous on it; outputs are valid
+ *    once the stream has reached that point.
+ *  - Argument errors are detected on the host before anything is enqueued
+ *    and returned synchronously; nothing is written then.
+ *  - Errors that only the device can see (an expert index out of range in
+ *    routing-given mode, a bounded wait that ran out) are recorded in a
+ *    status word at the start of the workspace; read it with
+ *    mova_get_status().  Offending entries are clamped so that no access
+ *    leaves its buffer.
+ *  - T == 0 is a valid no-op and returns MOVA_OK.
+ *  - Supported on the GPU: 1 <= E <= 64, 1 <= k <= min(E, 8), d % 64 == 0,
+ *    n % 128 == 0, T < 2^24; dtypes x/Wv/v all fp32, or all bf16 (router
+ *    Wr/br always fp32).  Anything else returns MOVA_ERR_UNSUPPORTED; there
+ *    is no fallback path.
+ */
+#ifndef MOVA_H_
+#define MOVA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MOVA_OK = 0,
+  MOVA_ERR_INVALID_ARG = 1,   /* null pointer, bad size, misalignment, workspace too small */
+  MOVA_ERR_UNSUPPORTED = 2,   /* valid arguments this build does not implement */
+  MOVA_ERR_CUDA = 3,          /* a CUDA runtime call or a launch failed */
+  MOVA_ERR_TIMEOUT = 4,       /* a bounded device-side wait ran out (status word) */
+  MOVA_ERR_DEVICE_CHECK = 5   /* a device-side input check failed (status word) */
+} mova_status;
+
+typedef enum {
+  MOVA_F32 = 0,
+  MOVA_BF16 = 1,
+  MOVA_F16 = 2,
+  MOVA_I32 = 3,
+  MOVA_I8 = 4
+} mova_dtype;
+
+/* Which expert kernel runs.  AUTO picks the weight-streaming kernel for
+ * small token counts (and for fp32) and the tcgen05 grouped GEMM for bf16
+ * batches above a threshold.  STREAM and TENSOR force one (TENSOR requires
+ * bf16; otherwise MOVA_ERR_UNSUPPORTED). */
+typedef enum {
+  MOVA_PATH_AUTO = 0,
+  MOVA_PATH_STREAM = 1,
+  MOVA_PATH_TENSOR = 2
+} mova_path;
+
+/* Human-readable name of a status code (static storage, never NULL). */
+const char* mova_status_str(mova_status s);
+
+/* Bytes of device workspace the value entry points need for these sizes
+ * (0 when T == 0).  The workspace holds the status word, the routing, the
+ * grouping by expert and the per-(token, slot) expert outputs; it may be
+ * reused across calls on the same stream.  Returns 0 for invalid sizes. */
+size_t mova_workspace_size(int T, int d, int E, int k, int n);
+
+/* Router: sigmoid gate, bias-assisted top-k, renormalise, scale.
+ *   x    (T, d)  x_dt in {MOVA_F32, MOVA_BF16}
+ *   Wr   (E, d)  fp32 router weight;  br (E) fp32 router bias (selection only)
+ *   idx  (T, k)  int32 out: selected experts, slot 0 = highest biased score
+ *   w    (T, k)  fp32 out: scale * s / sum(s) over the k selected
+ * Logits are accumulated in fp32.  Source: "Where the routing happens". */
+mova_status mova_route(const void* x, mova_dtype x_dt, const float* Wr, const float* br,
+                       int T, int d, int E, int k, float scale,
+                       int32_t* idx, float* w, void* stream);
+
+/* Grouping of the flat (token, slot) pairs f = t*k + slot by expert: a
+ * stable counting sort.
+ *   idx     (T, k) int32 in [0, E)
+ *   counts  (E)    int32 out: pairs per expert
+ *   offsets (E+1)  int32 out: exclusive prefix sum of counts
+ *   perm    (T*k)  int32 out: the pair at each position of the order sorted
+ *                  by (expert, f)
+ *   pos     (T*k)  int32 out: inverse of perm
+ * Bit-exact and deterministic.  An index outside [0, E) is clamped and
+ * raises MOVA_ERR_DEVICE_CHECK in the status word held by `ws`
+ * (ws_bytes >= mova_workspace_size(T, 64, E, k, 128) suffices). */
+mova_status mova_permute(const int32_t* idx, int T, int E, int k,
+                         int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* pos,
+                         void* ws, size_t ws_bytes, void* stream);
+
+/* Routing-given mixture (compact-cache recompute):
+ *   v[t] = sum_{slot ascending} w[t,slot] * SiLU(Wv[idx[t,slot]] x[t])
+ *   x   (T, d)    x_dt in {MOVA_F32, MOVA_BF16}
+ *   idx (T, k)    idx_dt in {MOVA_I32, MOVA_I8}
+ *   w   (T, k)    w_dt in {MOVA_F32, MOVA_F16}; used as given (no renormalisation)
+ *   Wv  (E, n, d) wv_dt == x_dt; expert e's weight is output-major (n rows of d)
+ *   v   (T, n)    same dtype as x; equals (T, n/128, 128) GQA value heads
+ *   ws  device workspace of ws_bytes >= mova_workspace_size(T, d, E, k, n) */
+mova_status mova_value(const void* x, mova_dtype x_dt, const void* idx, mova_dtype idx_dt,
+                       const void* w, mova_dtype w_dt, const void* Wv, mova_dtype wv_dt,
+                       int T, int d, int E, int k, int n, void* v,
+                       void* ws, size_t ws_bytes, void* stream);
+
+/* Full value path: route, group, expert projections with SiLU x weight,
+ * fixed-order combine.  Arguments as in mova_route and mova_value; idx_out
+ * (T, k) int32 and w_out (T, k) fp32 are optional copies of the routing
+ * (pass NULL to skip). */
+mova_status mova_value_routed(const void* x, mova_dtype x_dt, const float* Wr, const float* br,
+                              const void* Wv, mova_dtype wv_dt,
+                              int T, int d, int E, int k, int n, float scale, void* v,
+                              int32_t* idx_out, float* w_out,
+                              void* ws, size_t ws_bytes, void* stream);
+
+/* As mova_value / mova_value_routed, with the expert kernel chosen by
+ * `path` instead of automatically. */
+mova_status mova_value_ex(const void* x, mova_dtype x_dt, const void* idx, mova_dtype idx_dt,
+                          const void* w, mova_dtype w_dt, const void* Wv, mova_dtype wv_dt,
+                          int T, int d, int E, int k, int n, void* v,
+                          void* ws, size_t ws_bytes, mova_path path, void* stream);
+mova_status mova_value_routed_ex(const void* x, mova_dtype x_dt, const float* Wr, const float* br,
+                                 const void* Wv, mova_dtype wv_dt,
+                                 int T, int d, int E, int k, int n, float scale, void* v,
+                                 int32_t* idx_out, float* w_out,
+                                 void* ws, size_t ws_bytes, mova_path path, void* stream);
+
+/* Synchronises `stream`, then returns and clears the device status word
+ * held in `ws` (MOVA_OK if no device-side check fired since the last read).
+ * `detail_out` (nullable) receives the first offending item (e.g. the flat
+ * pair index of a bad expert index). */
+mova_status mova_get_status(void* ws, int32_t* detail_out, void* stream);
+
+/* The path AUTO would pick for these sizes and dtype (for tests/benches). */
+mova_path mova_auto_path(int T, mova_dtype x_dt);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOVA_H_ */

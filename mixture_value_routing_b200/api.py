@@ -1,0 +1,172 @@
+"""Python face of the MoVA value path: the C ABI of libmova.so, called with
+torch CUDA tensors (torch only provides device memory and the stream).
+
+    v = value_routed(x, Wr, br, Wv)            # (T, 1024) -> view (T, 8, 128)
+    idx, w = route(x, Wr, br)
+    v = value(x, idx, w, Wv)                    # routing given (compact cache)
+
+Every function enqueues on torch's current CUDA stream and returns without
+synchronising.  Device-side checks are read with get_status().
+"""
+from __future__ import annotations
+
+import ctypes
+from typing import Optional
+
+import torch
+
+from . import _lib
+
+_DT = {torch.float32: _lib.F32, torch.bfloat16: _lib.BF16, torch.float16: _lib.F16,
+       torch.int32: _lib.I32, torch.int8: _lib.I8}
+_PATH = {"auto": _lib.PATH_AUTO, "stream": _lib.PATH_STREAM, "tensor": _lib.PATH_TENSOR}
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _need(t: torch.Tensor, name: str, dtypes=None, ndim=None):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtypes is not None and t.dtype not in dtypes:
+        raise ValueError(f"{name}: dtype {t.dtype} not in {dtypes}")
+    if ndim is not None and t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dims")
+
+
+class Workspace:
+    """A device workspace that grows on demand (one per device)."""
+
+    def __init__(self):
+        self.buf: Optional[torch.Tensor] = None
+
+    def get(self, nbytes: int, device) -> torch.Tensor:
+        if self.buf is None or self.buf.numel() < nbytes or self.buf.device != torch.device(device):
+            self.buf = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
+        return self.buf
+
+
+_WS = {}
+
+
+def _devkey(device) -> torch.device:
+    dev = torch.device(device)
+    if dev.index is None:
+        dev = torch.device(dev.type, torch.cuda.current_device())
+    return dev
+
+
+def _workspace(nbytes: int, device) -> torch.Tensor:
+    dev = _devkey(device)
+    if dev not in _WS:
+        _WS[dev] = Workspace()
+    return _WS[dev].get(nbytes, dev)
+
+
+def workspace_size(T: int, d: int, E: int, k: int, n: int) -> int:
+    return int(_lib.load().mova_workspace_size(T, d, E, k, n))
+
+
+def auto_path(T: int, dtype: torch.dtype) -> str:
+    code = _lib.load().mova_auto_path(T, _DT[dtype])
+    return {v: k for k, v in _PATH.items()}[code]
+
+
+def route(x: torch.Tensor, Wr: torch.Tensor, br: torch.Tensor, k: int = 4, scale: float = 2.5):
+    """(idx (T, k) int32, w (T, k) fp32)."""
+    _need(x, "x", (torch.float32, torch.bfloat16), 2)
+    _need(Wr, "Wr", (torch.float32,), 2)
+    _need(br, "br", (torch.float32,), 1)
+    T, d = x.shape
+    E = Wr.shape[0]
+    idx = torch.empty((T, k), dtype=torch.int32, device=x.device)
+    w = torch.empty((T, k), dtype=torch.float32, device=x.device)
+    lib = _lib.load()
+    _lib.check(lib.mova_route(_ptr(x), _DT[x.dtype], _ptr(Wr), _ptr(br), T, d, E, k, float(scale),
+                              _ptr(idx), _ptr(w), _stream()), "mova_route")
+    return idx, w
+
+
+def permute(idx: torch.Tensor, E: int):
+    """Stable grouping of the (token, slot) pairs by expert:
+    dict(counts (E), offsets (E+1), perm (T*k), pos (T*k)), all int32."""
+    _need(idx, "idx", (torch.int32,), 2)
+    T, k = idx.shape
+    dev = idx.device
+    counts = torch.empty(E, dtype=torch.int32, device=dev)
+    offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    perm = torch.empty(T * k, dtype=torch.int32, device=dev)
+    pos = torch.empty(T * k, dtype=torch.int32, device=dev)
+    nbytes = workspace_size(T, 64, E, k, 128)
+    ws = _workspace(nbytes, dev)
+    lib = _lib.load()
+    _lib.check(lib.mova_permute(_ptr(idx), T, E, k, _ptr(counts), _ptr(offsets), _ptr(perm),
+                                _ptr(pos), _ptr(ws), ws.numel(), _stream()), "mova_permute")
+    return dict(counts=counts, offsets=offsets, perm=perm, pos=pos, ws=ws)
+
+
+def value(x: torch.Tensor, idx: torch.Tensor, w: torch.Tensor, Wv: torch.Tensor,
+          path: str = "auto", ws: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Routing-given mixture: v (T, n) in x's dtype."""
+    _need(x, "x", (torch.float32, torch.bfloat16), 2)
+    _need(idx, "idx", (torch.int32, torch.int8), 2)
+    _need(w, "w", (torch.float32, torch.float16), 2)
+    _need(Wv, "Wv", (x.dtype,), 3)
+    T, d = x.shape
+    E, n, _ = Wv.shape
+    k = idx.shape[1]
+    v = torch.empty((T, n), dtype=x.dtype, device=x.device)
+    nbytes = workspace_size(T, d, E, k, n)
+    if ws is None:
+        ws = _workspace(nbytes, x.device)
+    lib = _lib.load()
+    _lib.check(lib.mova_value_ex(_ptr(x), _DT[x.dtype], _ptr(idx), _DT[idx.dtype], _ptr(w),
+                                 _DT[w.dtype], _ptr(Wv), _DT[Wv.dtype], T, d, E, k, n, _ptr(v),
+                                 _ptr(ws), ws.numel(), _PATH[path], _stream()), "mova_value")
+    return v
+
+
+def value_routed(x: torch.Tensor, Wr: torch.Tensor, br: torch.Tensor, Wv: torch.Tensor,
+                 k: int = 4, scale: float = 2.5, return_routing: bool = False,
+                 path: str = "auto", ws: Optional[torch.Tensor] = None,
+                 out: Optional[torch.Tensor] = None):
+    """Full value path: v (T, n) in x's dtype [, idx (T, k) int32, w (T, k) fp32]."""
+    _need(x, "x", (torch.float32, torch.bfloat16), 2)
+    _need(Wr, "Wr", (torch.float32,), 2)
+    _need(br, "br", (torch.float32,), 1)
+    _need(Wv, "Wv", (x.dtype,), 3)
+    T, d = x.shape
+    E, n, _ = Wv.shape
+    dev = x.device
+    v = out if out is not None else torch.empty((T, n), dtype=x.dtype, device=dev)
+    idx = w = None
+    if return_routing:
+        idx = torch.empty((T, k), dtype=torch.int32, device=dev)
+        w = torch.empty((T, k), dtype=torch.float32, device=dev)
+    nbytes = workspace_size(T, d, E, k, n)
+    if ws is None:
+        ws = _workspace(nbytes, dev)
+    lib = _lib.load()
+    _lib.check(lib.mova_value_routed_ex(_ptr(x), _DT[x.dtype], _ptr(Wr), _ptr(br), _ptr(Wv),
+                                        _DT[Wv.dtype], T, d, E, k, n, float(scale), _ptr(v),
+                                        _ptr(idx), _ptr(w), _ptr(ws), ws.numel(), _PATH[path],
+                                        _stream()), "mova_value_routed")
+    if return_routing:
+        return v, idx, w
+    return v
+
+
+def get_status(ws: Optional[torch.Tensor] = None, device=None):
+    """(status name, detail) of the last value call on this workspace."""
+    if ws is None:
+        ws = _WS[_devkey(device if device is not None else "cuda")].buf
+    detail = ctypes.c_int32(0)
+    code = _lib.load().mova_get_status(_ptr(ws), ctypes.byref(detail), _stream())
+    return _lib.STATUS_NAMES.get(code, str(code)), int(detail.value)

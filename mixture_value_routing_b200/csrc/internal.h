@@ -1,0 +1,46 @@
+// Host-side launchers shared between the translation units of the library.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/mova.h"
+
+namespace mova {
+
+struct StatusBlock;
+
+// Largest number of (token, slot) pairs the single-CTA grouping handles.
+constexpr int kMaxPairs = 131072;
+
+cudaError_t launch_router(const void* x, mova_dtype x_dt, const float* Wr, const float* br, int T,
+                          int d, int E, int k, float scale, int32_t* idx, float* w,
+                          cudaStream_t stream);
+
+// Stable counting sort of the pairs by expert.  idx_in has dtype idx_dt
+// (int32 or int8); when w_in is given (w_dt fp32 or fp16) it is converted to
+// fp32 into w32, and idx_in to int32 into idx32 (routing-given mode).
+cudaError_t launch_permute(const void* idx_in, mova_dtype idx_dt, const void* w_in,
+                           mova_dtype w_dt, int N, int E, int32_t* idx32, float* w32,
+                           int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* pos,
+                           int32_t* active, StatusBlock* sb, cudaStream_t stream);
+
+// Weight-streaming expert kernel: P[p, :] = w * SiLU(Wv[e] x[t]) for every
+// pair p (fp32 rows in grouped order).
+cudaError_t launch_stream_experts(const void* x, const void* Wv, mova_dtype dt, const int32_t* counts,
+                                  const int32_t* offsets, const int32_t* perm, const float* w32,
+                                  const int32_t* active, const StatusBlock* sb, int d, int n, int k,
+                                  int E, float* P, cudaStream_t stream);
+
+// tcgen05 grouped GEMM (bf16): P[p, :] = w * SiLU(Wv[e] x[t]) as bf16 rows.
+cudaError_t launch_tensor_experts(const void* x, const void* Wv, const int32_t* counts,
+                                  const int32_t* offsets, const int32_t* perm, const float* w32,
+                                  StatusBlock* sb, int T, int d, int n, int k, int E,
+                                  __nv_bfloat16* P, cudaStream_t stream);
+
+// v[t, :] = sum over slots (ascending) of P[pos[t*k + slot], :].
+cudaError_t launch_combine(const void* P, bool p_bf16, const int32_t* pos, int T, int k, int n,
+                           void* v, mova_dtype v_dt, cudaStream_t stream);
+
+}  // namespace mova

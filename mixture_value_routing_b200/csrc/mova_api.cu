@@ -1,0 +1,220 @@
+// C ABI entry points of the MoVA value path: argument checks, workspace
+// layout, and the enqueueing of the kernels on the caller's stream.
+//
+// Call sequence of mova_value_routed (the pages' forward, "MoVA: routing the
+// value vectors, and why the KV cache does not notice", section "Where the
+// routing happens"):
+//   router  -> idx, w                     (fp32 logits, sigmoid, biased top-k)
+//   permute -> counts, offsets, perm, pos (stable grouping by expert)
+//   experts -> P rows = w * SiLU(Wv[e] x) (weight streaming or tcgen05 GEMM)
+//   combine -> v = sum of each token's rows in ascending slot order
+#include <stdio.h>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace mova {
+namespace {
+
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+struct Workspace {
+  StatusBlock* sb;
+  int32_t* idx;
+  float* w;
+  int32_t* counts;
+  int32_t* offsets;
+  int32_t* active;
+  int32_t* perm;
+  int32_t* pos;
+  void* P;
+  size_t bytes;
+};
+
+// Byte layout of the workspace (every part 256-byte aligned).
+Workspace layout(void* base, int T, int k, int n) {
+  const size_t pairs = static_cast<size_t>(T) * k;
+  char* b = static_cast<char*>(base);
+  size_t o = 0;
+  Workspace w{};
+  w.sb = reinterpret_cast<StatusBlock*>(b + o);      o += 256;
+  w.idx = reinterpret_cast<int32_t*>(b + o);         o += align256(pairs * 4);
+  w.w = reinterpret_cast<float*>(b + o);             o += align256(pairs * 4);
+  w.counts = reinterpret_cast<int32_t*>(b + o);      o += 256;
+  w.offsets = reinterpret_cast<int32_t*>(b + o);     o += 512;
+  w.active = reinterpret_cast<int32_t*>(b + o);      o += 256;
+  w.perm = reinterpret_cast<int32_t*>(b + o);        o += align256(pairs * 4);
+  w.pos = reinterpret_cast<int32_t*>(b + o);         o += align256(pairs * 4);
+  w.P = b + o;                                       o += align256(pairs * static_cast<size_t>(n) * 4);
+  w.bytes = o;
+  return w;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+mova_status check_dims(int T, int d, int E, int k, int n) {
+  if (T < 0 || d <= 0 || E <= 0 || k <= 0 || n <= 0) return MOVA_ERR_INVALID_ARG;
+  if (k > E) return MOVA_ERR_INVALID_ARG;
+  if (E > 64 || k > 8 || d % 64 != 0 || n % 128 != 0) return MOVA_ERR_UNSUPPORTED;
+  if (static_cast<long long>(T) * k > kMaxPairs) return MOVA_ERR_UNSUPPORTED;
+  return MOVA_OK;
+}
+
+mova_status from_cuda(cudaError_t e) {
+  if (e == cudaSuccess) return MOVA_OK;
+  fprintf(stderr, "mova: CUDA error %s\n", cudaGetErrorString(e));
+  return MOVA_ERR_CUDA;
+}
+
+bool valid_act_dtype(mova_dtype dt) { return dt == MOVA_F32 || dt == MOVA_BF16; }
+
+// Experts and combine, shared by both value entry points.
+mova_status run_experts_and_combine(const void* x, mova_dtype dt, const void* Wv,
+                                    const Workspace& ws, const int32_t* idx, const float* w32,
+                                    int T, int d, int E, int k, int n, void* v, mova_path path,
+                                    cudaStream_t stream) {
+  (void)idx;
+  if (path == MOVA_PATH_AUTO) path = mova_auto_path(T, dt);
+  if (path == MOVA_PATH_TENSOR) return MOVA_ERR_UNSUPPORTED;
+  cudaError_t err = launch_stream_experts(x, Wv, dt, ws.counts, ws.offsets, ws.perm, w32,
+                                          ws.active, ws.sb, d, n, k, E,
+                                          static_cast<float*>(ws.P), stream);
+  if (err != cudaSuccess) return from_cuda(err);
+  return from_cuda(launch_combine(ws.P, false, ws.pos, T, k, n, v, dt, stream));
+}
+
+}  // namespace
+}  // namespace mova
+
+using namespace mova;
+
+extern "C" {
+
+const char* mova_status_str(mova_status s) {
+  switch (s) {
+    case MOVA_OK: return "MOVA_OK";
+    case MOVA_ERR_INVALID_ARG: return "MOVA_ERR_INVALID_ARG";
+    case MOVA_ERR_UNSUPPORTED: return "MOVA_ERR_UNSUPPORTED";
+    case MOVA_ERR_CUDA: return "MOVA_ERR_CUDA";
+    case MOVA_ERR_TIMEOUT: return "MOVA_ERR_TIMEOUT";
+    case MOVA_ERR_DEVICE_CHECK: return "MOVA_ERR_DEVICE_CHECK";
+  }
+  return "MOVA_ERR_UNKNOWN";
+}
+
+size_t mova_workspace_size(int T, int d, int E, int k, int n) {
+  if (check_dims(T, d, E, k, n) != MOVA_OK) return 0;
+  if (T == 0) return 0;
+  return layout(nullptr, T, k, n).bytes;
+}
+
+mova_path mova_auto_path(int T, mova_dtype x_dt) {
+  (void)T;
+  (void)x_dt;
+  return MOVA_PATH_STREAM;
+}
+
+mova_status mova_route(const void* x, mova_dtype x_dt, const float* Wr, const float* br, int T,
+                       int d, int E, int k, float scale, int32_t* idx, float* w, void* stream) {
+  mova_status st = check_dims(T, d, E, k, 128);
+  if (st != MOVA_OK) return st;
+  if (!valid_act_dtype(x_dt)) return MOVA_ERR_UNSUPPORTED;
+  if (T == 0) return MOVA_OK;
+  if (!x || !Wr || !br || !idx || !w) return MOVA_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(Wr)) return MOVA_ERR_INVALID_ARG;
+  return from_cuda(launch_router(x, x_dt, Wr, br, T, d, E, k, scale, idx, w,
+                                 static_cast<cudaStream_t>(stream)));
+}
+
+mova_status mova_permute(const int32_t* idx, int T, int E, int k, int32_t* counts,
+                         int32_t* offsets, int32_t* perm, int32_t* pos, void* ws, size_t ws_bytes,
+                         void* stream) {
+  mova_status st = check_dims(T, 64, E, k, 128);
+  if (st != MOVA_OK) return st;
+  if (T == 0) return MOVA_OK;
+  if (!idx || !counts || !offsets || !perm || !pos || !ws) return MOVA_ERR_INVALID_ARG;
+  const Workspace w = layout(ws, T, k, 128);
+  if (ws_bytes < w.bytes || (reinterpret_cast<uintptr_t>(ws) & 255) != 0) return MOVA_ERR_INVALID_ARG;
+  return from_cuda(launch_permute(idx, MOVA_I32, nullptr, MOVA_F32, T * k, E, nullptr, nullptr,
+                                  counts, offsets, perm, pos, w.active, w.sb,
+                                  static_cast<cudaStream_t>(stream)));
+}
+
+mova_status mova_value_ex(const void* x, mova_dtype x_dt, const void* idx, mova_dtype idx_dt,
+                          const void* wgt, mova_dtype w_dt, const void* Wv, mova_dtype wv_dt, int T,
+                          int d, int E, int k, int n, void* v, void* ws, size_t ws_bytes,
+                          mova_path path, void* stream) {
+  mova_status st = check_dims(T, d, E, k, n);
+  if (st != MOVA_OK) return st;
+  if (!valid_act_dtype(x_dt) || wv_dt != x_dt) return MOVA_ERR_UNSUPPORTED;
+  if (idx_dt != MOVA_I32 && idx_dt != MOVA_I8) return MOVA_ERR_UNSUPPORTED;
+  if (w_dt != MOVA_F32 && w_dt != MOVA_F16) return MOVA_ERR_UNSUPPORTED;
+  if (path != MOVA_PATH_AUTO && path != MOVA_PATH_STREAM && path != MOVA_PATH_TENSOR)
+    return MOVA_ERR_INVALID_ARG;
+  if (T == 0) return MOVA_OK;
+  if (!x || !idx || !wgt || !Wv || !v || !ws) return MOVA_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(Wv) || !aligned16(v)) return MOVA_ERR_INVALID_ARG;
+  const Workspace w = layout(ws, T, k, n);
+  if (ws_bytes < w.bytes || (reinterpret_cast<uintptr_t>(ws) & 255) != 0) return MOVA_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t err = launch_permute(idx, idx_dt, wgt, w_dt, T * k, E, w.idx, w.w, w.counts,
+                                   w.offsets, w.perm, w.pos, w.active, w.sb, s);
+  if (err != cudaSuccess) return from_cuda(err);
+  return run_experts_and_combine(x, x_dt, Wv, w, w.idx, w.w, T, d, E, k, n, v, path, s);
+}
+
+mova_status mova_value(const void* x, mova_dtype x_dt, const void* idx, mova_dtype idx_dt,
+                       const void* wgt, mova_dtype w_dt, const void* Wv, mova_dtype wv_dt, int T,
+                       int d, int E, int k, int n, void* v, void* ws, size_t ws_bytes,
+                       void* stream) {
+  return mova_value_ex(x, x_dt, idx, idx_dt, wgt, w_dt, Wv, wv_dt, T, d, E, k, n, v, ws, ws_bytes,
+                       MOVA_PATH_AUTO, stream);
+}
+
+mova_status mova_value_routed_ex(const void* x, mova_dtype x_dt, const float* Wr, const float* br,
+                                 const void* Wv, mova_dtype wv_dt, int T, int d, int E, int k,
+                                 int n, float scale, void* v, int32_t* idx_out, float* w_out,
+                                 void* ws, size_t ws_bytes, mova_path path, void* stream) {
+  mova_status st = check_dims(T, d, E, k, n);
+  if (st != MOVA_OK) return st;
+  if (!valid_act_dtype(x_dt) || wv_dt != x_dt) return MOVA_ERR_UNSUPPORTED;
+  if (path != MOVA_PATH_AUTO && path != MOVA_PATH_STREAM && path != MOVA_PATH_TENSOR)
+    return MOVA_ERR_INVALID_ARG;
+  if (T == 0) return MOVA_OK;
+  if (!x || !Wr || !br || !Wv || !v || !ws) return MOVA_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(Wr) || !aligned16(Wv) || !aligned16(v))
+    return MOVA_ERR_INVALID_ARG;
+  const Workspace w = layout(ws, T, k, n);
+  if (ws_bytes < w.bytes || (reinterpret_cast<uintptr_t>(ws) & 255) != 0) return MOVA_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int32_t* idx = idx_out ? idx_out : w.idx;
+  float* wgt = w_out ? w_out : w.w;
+  cudaError_t err = launch_router(x, x_dt, Wr, br, T, d, E, k, scale, idx, wgt, s);
+  if (err != cudaSuccess) return from_cuda(err);
+  err = launch_permute(idx, MOVA_I32, nullptr, MOVA_F32, T * k, E, nullptr, nullptr, w.counts,
+                       w.offsets, w.perm, w.pos, w.active, w.sb, s);
+  if (err != cudaSuccess) return from_cuda(err);
+  return run_experts_and_combine(x, x_dt, Wv, w, idx, wgt, T, d, E, k, n, v, path, s);
+}
+
+mova_status mova_value_routed(const void* x, mova_dtype x_dt, const float* Wr, const float* br,
+                              const void* Wv, mova_dtype wv_dt, int T, int d, int E, int k, int n,
+                              float scale, void* v, int32_t* idx_out, float* w_out, void* ws,
+                              size_t ws_bytes, void* stream) {
+  return mova_value_routed_ex(x, x_dt, Wr, br, Wv, wv_dt, T, d, E, k, n, scale, v, idx_out, w_out,
+                              ws, ws_bytes, MOVA_PATH_AUTO, stream);
+}
+
+mova_status mova_get_status(void* ws, int32_t* detail_out, void* stream) {
+  if (!ws) return MOVA_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t err = cudaStreamSynchronize(s);
+  if (err != cudaSuccess) return from_cuda(err);
+  StatusBlock sb{};
+  err = cudaMemcpy(&sb, ws, sizeof(sb), cudaMemcpyDeviceToHost);
+  if (err != cudaSuccess) return from_cuda(err);
+  if (detail_out) *detail_out = sb.detail;
+  return static_cast<mova_status>(sb.code);
+}
+
+}  // extern "C"

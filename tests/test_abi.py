@@ -1,0 +1,95 @@
+"""The C-ABI library: it builds, loads without a GPU, exports every entry point
+include/mova.h declares, and rejects bad arguments on the host (no compute
+call is made here)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from mixture_value_routing_b200 import _lib, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "mova.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return _lib.load()
+
+
+def _declared():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(mova_[a-z_]+)\s*\(", src)))
+
+
+def test_header_declares_the_boundary():
+    names = _declared()
+    for must in ["mova_route", "mova_value", "mova_value_routed", "mova_permute",
+                 "mova_workspace_size", "mova_get_status", "mova_status_str"]:
+        assert must in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in _declared():
+        assert hasattr(lib, name), name
+    assert set(_declared()) == set(_lib.SIGNATURES)
+
+
+def test_status_strings(lib):
+    for code, name in _lib.STATUS_NAMES.items():
+        assert lib.mova_status_str(code).decode() == name
+    assert lib.mova_status_str(99).decode() == "MOVA_ERR_UNKNOWN"
+
+
+def test_workspace_size(lib):
+    assert lib.mova_workspace_size(0, 2560, 64, 4, 1024) == 0
+    a = lib.mova_workspace_size(8, 2560, 64, 4, 1024)
+    b = lib.mova_workspace_size(4096, 2560, 64, 4, 1024)
+    assert a > 0 and b > a and b % 256 == 0
+    # P rows dominate: T*k*n fp32
+    assert b >= 4096 * 4 * 1024 * 4
+    # unsupported or invalid sizes give 0
+    assert lib.mova_workspace_size(8, 2560, 65, 4, 1024) == 0
+    assert lib.mova_workspace_size(8, 2561, 64, 4, 1024) == 0
+    assert lib.mova_workspace_size(8, 2560, 64, 9, 1024) == 0
+    assert lib.mova_workspace_size(8, 2560, 64, 4, 1000) == 0
+    assert lib.mova_workspace_size(-1, 2560, 64, 4, 1024) == 0
+    assert lib.mova_workspace_size(8, 2560, 4, 5, 1024) == 0
+    assert lib.mova_workspace_size(40000, 2560, 64, 4, 1024) == 0  # above the pair limit
+
+
+def test_host_side_validation(lib):
+    """Errors found on the host return before anything touches a GPU."""
+    fake = ctypes.c_void_p(4096)  # never dereferenced: every call below fails validation first
+    st = lib.mova_route(None, _lib.BF16, None, None, 0, 2560, 64, 4, 2.5, None, None, None)
+    assert st == _lib.OK  # T == 0 is a no-op
+    st = lib.mova_route(None, _lib.BF16, None, None, 8, 2560, 64, 4, 2.5, None, None, None)
+    assert st == _lib.ERR_INVALID_ARG
+    st = lib.mova_route(fake, _lib.F16, fake, fake, 8, 2560, 64, 4, 2.5, fake, fake, None)
+    assert st == _lib.ERR_UNSUPPORTED
+    st = lib.mova_route(fake, _lib.BF16, fake, fake, 8, 2560, 64, 65, 2.5, fake, fake, None)
+    assert st == _lib.ERR_INVALID_ARG
+    # misaligned x
+    st = lib.mova_route(ctypes.c_void_p(4098), _lib.BF16, fake, fake, 8, 2560, 64, 4, 2.5, fake,
+                        fake, None)
+    assert st == _lib.ERR_INVALID_ARG
+    # value: wv dtype must equal x dtype; workspace too small
+    st = lib.mova_value_routed(fake, _lib.BF16, fake, fake, fake, _lib.F32, 8, 2560, 64, 4, 1024,
+                               2.5, fake, None, None, fake, 1 << 30, None)
+    assert st == _lib.ERR_UNSUPPORTED
+    st = lib.mova_value_routed(fake, _lib.BF16, fake, fake, fake, _lib.BF16, 8, 2560, 64, 4, 1024,
+                               2.5, fake, None, None, fake, 16, None)
+    assert st == _lib.ERR_INVALID_ARG
+    st = lib.mova_value(fake, _lib.BF16, fake, _lib.F32, fake, _lib.F16, fake, _lib.BF16, 8, 2560,
+                        64, 4, 1024, fake, fake, 1 << 30, None)
+    assert st == _lib.ERR_UNSUPPORTED  # idx must be int32 or int8
+    st = lib.mova_value_ex(fake, _lib.BF16, fake, _lib.I8, fake, _lib.F16, fake, _lib.BF16, 8, 2560,
+                           64, 4, 1024, fake, fake, 1 << 30, 7, None)
+    assert st == _lib.ERR_INVALID_ARG  # unknown path
+    st = lib.mova_permute(None, 0, 64, 4, None, None, None, None, None, 0, None)
+    assert st == _lib.OK
+    st = lib.mova_get_status(None, None, None)
+    assert st == _lib.ERR_INVALID_ARG

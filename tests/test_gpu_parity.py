@@ -1,0 +1,207 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle on the
+same seeded inputs.  Comparison rules are in tests/_parity.py."""
+import numpy as np
+import pytest
+import torch
+
+import mova_inputs as MI
+from oracle import mova_oracle as O
+from tests import _parity as P
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def api():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    from mixture_value_routing_b200 import build
+    build.build()
+    from mixture_value_routing_b200 import api as A
+    return A
+
+
+def _layer(seed, d, E, n, dtype, bias="normal"):
+    return MI.make_layer(seed, 0, d=d, E=E, n=n, wv_dtype=dtype, bias=bias)
+
+
+def _routing_ref(bat, lay, k, scale=2.5):
+    x = O.to_f64(bat.x, bat.x_dtype)
+    return x, O.route(x, lay.Wr.astype(np.float64), lay.br.astype(np.float64), k, scale)
+
+
+# ---------------------------------------------------------------------------
+# Router
+# ---------------------------------------------------------------------------
+
+ROUTE_CASES = [
+    # T, d, E, k, dtype
+    (1, 256, 8, 1, "f32"),
+    (3, 512, 64, 4, "bf16"),
+    (8, 2560, 64, 4, "bf16"),
+    (31, 256, 8, 8, "f32"),
+    (33, 2560, 64, 4, "bf16"),
+    (65, 1024, 17, 3, "f32"),
+    (128, 2560, 64, 4, "f32"),
+    (300, 2560, 64, 4, "bf16"),
+    (4096, 2560, 64, 4, "bf16"),
+]
+
+
+@pytest.mark.parametrize("T,d,E,k,dtype", ROUTE_CASES)
+def test_route(api, T, d, E, k, dtype):
+    lay = _layer(11, d, E, 128, dtype)
+    bat = MI.make_batch(T, 11, dtype=dtype, d=d)
+    _, ref = _routing_ref(bat, lay, k)
+    idx, w = api.route(P.dev(bat.x, dtype), P.dev(lay.Wr, "f32"), P.dev(lay.br, "f32"), k, 2.5)
+    torch.cuda.synchronize()
+    P.check_routing(idx.cpu().numpy(), w.cpu().numpy().astype(np.float64), ref, k, 2.5)
+
+
+def test_route_ties_go_to_lower_index(api):
+    """Identical router rows and zero bias: all scores tie exactly, so the
+    selection must be experts 0..k-1 in order."""
+    d, E, k, T = 256, 16, 4, 5
+    Wr = np.tile(np.random.default_rng(0).standard_normal(d).astype(np.float32) * 0.02, (E, 1))
+    br = np.zeros(E, np.float32)
+    x = np.random.default_rng(1).standard_normal((T, d)).astype(np.float32)
+    idx, w = api.route(P.dev(x, "f32"), P.dev(Wr, "f32"), P.dev(br, "f32"), k, 2.5)
+    assert (idx.cpu().numpy() == np.arange(k)[None, :]).all()
+    np.testing.assert_allclose(w.cpu().numpy(), 2.5 / k, rtol=1e-6)
+
+
+# ---------------------------------------------------------------------------
+# Grouping by expert
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("T,E,k,kind", [
+    (1, 64, 4, "distinct"), (7, 5, 2, "distinct"), (33, 64, 8, "distinct"),
+    (1000, 64, 4, "distinct"), (4096, 64, 4, "distinct"), (32768, 64, 4, "distinct"),
+    (3000, 64, 4, "skewed"), (2000, 3, 3, "duplicates"), (999, 1, 1, "distinct"),
+])
+def test_permute(api, T, E, k, kind):
+    rng = np.random.default_rng(T + E + k)
+    if kind == "distinct":
+        idx = np.argsort(rng.random((T, E)), axis=1)[:, :k].astype(np.int32)
+    elif kind == "skewed":
+        p = 1.0 / np.arange(1, E + 1) ** 2.0
+        idx = rng.choice(E, size=(T, k), p=p / p.sum()).astype(np.int32)
+    else:
+        idx = rng.integers(0, E, size=(T, k)).astype(np.int32)
+    got = api.permute(P.dev(idx, "i32"), E)
+    torch.cuda.synchronize()
+    P.check_permutation(got, idx, E)
+
+
+def test_permute_rejects_bad_index(api):
+    idx = np.array([[0, 1], [2, 7], [1, 0]], np.int32)  # 7 >= E = 4
+    got = api.permute(P.dev(idx, "i32"), 4)
+    status, detail = api.get_status(got["ws"])
+    assert status == "MOVA_ERR_DEVICE_CHECK" and detail == 3
+    assert got["offsets"].cpu().numpy()[-1] == 6  # every pair still placed, none out of bounds
+
+
+# ---------------------------------------------------------------------------
+# Routing-given mixture (compact-cache recompute)
+# ---------------------------------------------------------------------------
+
+GIVEN_CASES = [
+    # T, d, E, k, n, dtype, idx dtype, w dtype, path
+    (5, 256, 8, 2, 128, "f32", "i32", "f32", "stream"),
+    (5, 256, 8, 2, 128, "bf16", "i8", "f16", "stream"),
+    (8, 2560, 64, 4, 1024, "bf16", "i8", "f16", "stream"),
+    (37, 512, 4, 4, 256, "bf16", "i32", "f32", "stream"),
+    (128, 2560, 64, 4, 1024, "f32", "i8", "f16", "stream"),
+    (1, 64, 1, 1, 128, "f32", "i32", "f32", "stream"),
+]
+
+
+@pytest.mark.parametrize("T,d,E,k,n,dtype,idt,wdt,path", GIVEN_CASES)
+def test_value_given(api, T, d, E, k, n, dtype, idt, wdt, path):
+    lay = _layer(5, d, E, n, dtype)
+    rng = np.random.default_rng(T * 7 + E)
+    idx = np.argsort(rng.random((T, E)), axis=1)[:, :k]
+    g = rng.exponential(1.0, size=(T, k))
+    w = (2.5 * g / g.sum(axis=1, keepdims=True))
+    w = w.astype(np.float16 if wdt == "f16" else np.float32)
+    bat = MI.make_batch(T, 5, dtype=dtype, d=d)
+    v = api.value(P.dev(bat.x, dtype), P.dev(idx, idt), P.dev(w, wdt), P.dev(lay.Wv, dtype),
+                  path=path)
+    torch.cuda.synchronize()
+    status, _ = api.get_status()
+    assert status == "MOVA_OK"
+    x = O.to_f64(bat.x, dtype)
+    v_ref = O.combine(x, idx, w.astype(np.float64), lay.Wv, dtype)
+    assert v.shape == (T, n) and v.dtype == (torch.bfloat16 if dtype == "bf16" else torch.float32)
+    P.check_values(P.host_f64(v), v_ref, dtype)
+
+
+def test_value_given_bad_index_is_flagged(api):
+    d, E, k, n, T = 256, 8, 2, 128, 4
+    lay = _layer(6, d, E, n, "bf16")
+    bat = MI.make_batch(T, 6, dtype="bf16", d=d)
+    idx = np.array([[0, 1], [2, 3], [4, -1], [6, 7]], np.int8)
+    w = np.full((T, k), 1.25, np.float16)
+    v = api.value(P.dev(bat.x, "bf16"), P.dev(idx, "i8"), P.dev(w, "f16"), P.dev(lay.Wv, "bf16"))
+    status, detail = api.get_status()
+    assert status == "MOVA_ERR_DEVICE_CHECK" and detail == 5
+    assert torch.isfinite(v.float()).all()
+
+
+# ---------------------------------------------------------------------------
+# Full path
+# ---------------------------------------------------------------------------
+
+def _full(api, T, d, E, k, n, dtype, seed=0, bias="normal", sample=None, path="auto"):
+    lay = _layer(seed, d, E, n, dtype, bias)
+    bat = MI.make_batch(T, seed, dtype=dtype, d=d)
+    x, ref = _routing_ref(bat, lay, k)
+    v, idx, w = api.value_routed(P.dev(bat.x, dtype), P.dev(lay.Wr, "f32"), P.dev(lay.br, "f32"),
+                                 P.dev(lay.Wv, dtype), k, 2.5, return_routing=True, path=path)
+    torch.cuda.synchronize()
+    idx_g = idx.cpu().numpy().astype(np.int64)
+    P.check_routing(idx_g, w.cpu().numpy().astype(np.float64), ref, k, 2.5)
+    rows = np.arange(T) if sample is None else np.sort(
+        np.random.default_rng(seed + 99).choice(T, size=min(sample, T), replace=False))
+    # Values of the GPU's (validated) selection with the oracle's weights.
+    w_ref = O.weights_for(ref["s"][rows], idx_g[rows], 2.5)
+    v_ref = O.combine(x[rows], idx_g[rows], w_ref, lay.Wv, dtype)
+    return P.check_values(P.host_f64(v)[rows], v_ref, dtype), v, idx
+
+
+def test_full_pr1_fp32(api):
+    """T=128, all fp32, d=2560, 64 experts, top-4 (every output element)."""
+    _full(api, 128, 2560, 64, 4, 1024, "f32")
+
+
+def test_full_decode_bf16(api):
+    """T=8 bf16 decode step at full dimensions (every output element)."""
+    _full(api, 8, 2560, 64, 4, 1024, "bf16")
+
+
+@pytest.mark.parametrize("T,E,k,n", [(1, 64, 4, 1024), (2, 8, 8, 128), (3, 1, 1, 256),
+                                     (17, 16, 4, 384)])
+def test_full_edge_shapes(api, T, E, k, n):
+    _full(api, T, 256, E, k, n, "bf16", seed=T)
+
+
+def test_full_zero_tokens(api):
+    lay = _layer(0, 256, 8, 128, "bf16")
+    x = torch.empty((0, 256), dtype=torch.bfloat16, device="cuda")
+    v = api.value_routed(x, P.dev(lay.Wr, "f32"), P.dev(lay.br, "f32"), P.dev(lay.Wv, "bf16"))
+    assert v.shape == (0, 128)
+
+
+def test_full_gqa_view(api):
+    _, v, _ = _full(api, 8, 2560, 64, 4, 1024, "bf16", seed=3)
+    g = v.view(8, 8, 128)
+    assert torch.equal(g[2, 5], v[2, 5 * 128:6 * 128])
+
+
+def test_deterministic(api):
+    lay = _layer(2, 2560, 64, 1024, "bf16")
+    bat = MI.make_batch(8, 2, dtype="bf16")
+    args = (P.dev(bat.x, "bf16"), P.dev(lay.Wr, "f32"), P.dev(lay.br, "f32"),
+            P.dev(lay.Wv, "bf16"))
+    first = api.value_routed(*args).clone()
+    for _ in range(9):
+        assert torch.equal(api.value_routed(*args), first)
