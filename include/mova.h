@@ -37,9 +37,10 @@
  *    leaves its buffer.
  *  - T == 0 is a valid no-op and returns MOVA_OK.
  *  - Supported on the GPU: 1 <= E <= 64, 1 <= k <= min(E, 8), d % 64 == 0,
- *    n % 128 == 0, T < 2^24; dtypes x/Wv/v all fp32, or all bf16 (router
- *    Wr/br always fp32).  Anything else returns MOVA_ERR_UNSUPPORTED; there
- *    is no fallback path.
+ *    n % 128 == 0, T * k <= 131072; dtypes x/Wv/v all fp32, or all bf16
+ *    (router Wr/br always fp32).  The weight-streaming expert kernel also
+ *    needs d <= 6400 (bf16) or d <= 3200 (fp32).  Anything else returns
+ *    MOVA_ERR_UNSUPPORTED; there is no fallback path.
  */
 #ifndef MOVA_H_
 #define MOVA_H_
@@ -136,16 +137,25 @@ mova_status mova_value_routed(const void* x, mova_dtype x_dt, const float* Wr, c
                               void* ws, size_t ws_bytes, void* stream);
 
 /* As mova_value / mova_value_routed, with the expert kernel chosen by
- * `path` instead of automatically. */
+ * `path` instead of automatically, and optional stage timing: `events`
+ * (nullable) points to MOVA_STAGE_EVENTS cudaEvent_t handles (passed as
+ * void*, created by the caller) that are recorded on `stream` at the stage
+ * boundaries: [0] start, [1] after routing, [2] after grouping, [3] after the
+ * expert kernel, [4] after the combine (mova_value_ex records [0] and [1]
+ * together, as its routing is given).  They are recorded with
+ * cudaEventRecordExternal, so they also work inside CUDA graph capture. */
+#define MOVA_STAGE_EVENTS 5
 mova_status mova_value_ex(const void* x, mova_dtype x_dt, const void* idx, mova_dtype idx_dt,
                           const void* w, mova_dtype w_dt, const void* Wv, mova_dtype wv_dt,
                           int T, int d, int E, int k, int n, void* v,
-                          void* ws, size_t ws_bytes, mova_path path, void* stream);
+                          void* ws, size_t ws_bytes, mova_path path, void* const* events,
+                          void* stream);
 mova_status mova_value_routed_ex(const void* x, mova_dtype x_dt, const float* Wr, const float* br,
                                  const void* Wv, mova_dtype wv_dt,
                                  int T, int d, int E, int k, int n, float scale, void* v,
                                  int32_t* idx_out, float* w_out,
-                                 void* ws, size_t ws_bytes, mova_path path, void* stream);
+                                 void* ws, size_t ws_bytes, mova_path path, void* const* events,
+                                 void* stream);
 
 /* Synchronises `stream`, then returns and clears the device status word
  * held in `ws` (MOVA_OK if no device-side check fired since the last read).

@@ -20,6 +20,9 @@ STATUS_NAMES = {OK: "MOVA_OK", ERR_INVALID_ARG: "MOVA_ERR_INVALID_ARG",
 F32, BF16, F16, I32, I8 = range(5)
 # mova_path
 PATH_AUTO, PATH_STREAM, PATH_TENSOR = range(3)
+# stage events recorded by the _ex entry points
+STAGE_EVENTS = 5
+STAGES = ("route", "group", "experts", "combine")
 
 _vp = ctypes.c_void_p
 _i = ctypes.c_int
@@ -34,11 +37,11 @@ SIGNATURES = {
     "mova_permute": (_i, [_vp, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "mova_value": (_i, [_vp, _i, _vp, _i, _vp, _i, _vp, _i, _i, _i, _i, _i, _i, _vp, _vp, _sz, _vp]),
     "mova_value_ex": (_i, [_vp, _i, _vp, _i, _vp, _i, _vp, _i, _i, _i, _i, _i, _i, _vp, _vp, _sz,
-                           _i, _vp]),
+                           _i, _vp, _vp]),
     "mova_value_routed": (_i, [_vp, _i, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _vp, _vp, _vp,
                                _vp, _sz, _vp]),
     "mova_value_routed_ex": (_i, [_vp, _i, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _vp, _vp,
-                                  _vp, _vp, _sz, _i, _vp]),
+                                  _vp, _vp, _sz, _i, _vp, _vp]),
     "mova_get_status": (_i, [_vp, _vp, _vp]),
 }
 

@@ -112,8 +112,17 @@ def permute(idx: torch.Tensor, E: int):
     return dict(counts=counts, offsets=offsets, perm=perm, pos=pos, ws=ws)
 
 
+def _events(events):
+    """Array of raw cudaEvent_t handles (or None) for the _ex entry points."""
+    if events is None:
+        return None
+    assert len(events) == _lib.STAGE_EVENTS
+    return (ctypes.c_void_p * _lib.STAGE_EVENTS)(*[ctypes.c_void_p(e.cuda_event) for e in events])
+
+
 def value(x: torch.Tensor, idx: torch.Tensor, w: torch.Tensor, Wv: torch.Tensor,
-          path: str = "auto", ws: Optional[torch.Tensor] = None) -> torch.Tensor:
+          path: str = "auto", ws: Optional[torch.Tensor] = None,
+          events=None) -> torch.Tensor:
     """Routing-given mixture: v (T, n) in x's dtype."""
     _need(x, "x", (torch.float32, torch.bfloat16), 2)
     _need(idx, "idx", (torch.int32, torch.int8), 2)
@@ -129,14 +138,15 @@ def value(x: torch.Tensor, idx: torch.Tensor, w: torch.Tensor, Wv: torch.Tensor,
     lib = _lib.load()
     _lib.check(lib.mova_value_ex(_ptr(x), _DT[x.dtype], _ptr(idx), _DT[idx.dtype], _ptr(w),
                                  _DT[w.dtype], _ptr(Wv), _DT[Wv.dtype], T, d, E, k, n, _ptr(v),
-                                 _ptr(ws), ws.numel(), _PATH[path], _stream()), "mova_value")
+                                 _ptr(ws), ws.numel(), _PATH[path], _events(events), _stream()),
+               "mova_value")
     return v
 
 
 def value_routed(x: torch.Tensor, Wr: torch.Tensor, br: torch.Tensor, Wv: torch.Tensor,
                  k: int = 4, scale: float = 2.5, return_routing: bool = False,
                  path: str = "auto", ws: Optional[torch.Tensor] = None,
-                 out: Optional[torch.Tensor] = None):
+                 out: Optional[torch.Tensor] = None, events=None):
     """Full value path: v (T, n) in x's dtype [, idx (T, k) int32, w (T, k) fp32]."""
     _need(x, "x", (torch.float32, torch.bfloat16), 2)
     _need(Wr, "Wr", (torch.float32,), 2)
@@ -157,7 +167,7 @@ def value_routed(x: torch.Tensor, Wr: torch.Tensor, br: torch.Tensor, Wv: torch.
     _lib.check(lib.mova_value_routed_ex(_ptr(x), _DT[x.dtype], _ptr(Wr), _ptr(br), _ptr(Wv),
                                         _DT[Wv.dtype], T, d, E, k, n, float(scale), _ptr(v),
                                         _ptr(idx), _ptr(w), _ptr(ws), ws.numel(), _PATH[path],
-                                        _stream()), "mova_value_routed")
+                                        _events(events), _stream()), "mova_value_routed")
     if return_routing:
         return v, idx, w
     return v

@@ -39,6 +39,7 @@ template <typename PT, typename OT>
 __global__ void __launch_bounds__(kThreads)
 combine_kernel(const PT* __restrict__ P, const int32_t* __restrict__ pos, int T, int k, int n,
                OT* __restrict__ v) {
+  pdl_wait();  // the expert rows of this call are complete and visible
   const int per_tok = n / 8;
   const long long total = static_cast<long long>(T) * per_tok;
   for (long long i = static_cast<long long>(blockIdx.x) * kThreads + threadIdx.x; i < total;
@@ -62,17 +63,13 @@ combine_kernel(const PT* __restrict__ P, const int32_t* __restrict__ pos, int T,
 template <typename PT, typename OT>
 cudaError_t launch_t(const void* P, const int32_t* pos, int T, int k, int n, void* v,
                      cudaStream_t stream) {
-  int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const long long total = static_cast<long long>(T) * (n / 8);
   long long blocks = (total + kThreads - 1) / kThreads;
-  const long long cap = static_cast<long long>(sms) * 8;
+  const long long cap = static_cast<long long>(sm_count()) * 8;
   if (blocks > cap) blocks = cap;
   if (blocks < 1) blocks = 1;
-  combine_kernel<PT, OT><<<static_cast<int>(blocks), kThreads, 0, stream>>>(
-      static_cast<const PT*>(P), pos, T, k, n, static_cast<OT*>(v));
-  return cudaGetLastError();
+  return launch_pdl(combine_kernel<PT, OT>, dim3(static_cast<unsigned>(blocks)), dim3(kThreads), 0,
+                    stream, static_cast<const PT*>(P), pos, T, k, n, static_cast<OT*>(v));
 }
 
 }  // namespace

@@ -83,6 +83,14 @@ __device__ __forceinline__ void load8_stream(const float* p, float out[8]) {
   out[6] = __uint_as_float(b.z); out[7] = __uint_as_float(b.w);
 }
 
+// Programmatic dependent launch: wait for the predecessor grid (no-op when
+// the kernel was launched without the attribute), and let the successor
+// start its launch early.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // Logistic function and SiLU in fp32 (IEEE expf and division).
 __device__ __forceinline__ float sigmoidf_(float z) { return 1.0f / (1.0f + expf(-z)); }
 __device__ __forceinline__ float siluf_(float h) { return h / (1.0f + expf(-h)); }

@@ -13,10 +13,48 @@ struct StatusBlock;
 
 // Largest number of (token, slot) pairs the single-CTA grouping handles.
 constexpr int kMaxPairs = 131072;
+// Token counts up to this run the fused decode router (routing + grouping in
+// one kernel).
+constexpr int kFusedRouterMaxT = 8;
 
+// Outputs of the grouping by expert (see launch_permute).
+struct GroupOut {
+  int32_t* counts;
+  int32_t* offsets;
+  int32_t* perm;
+  int32_t* pos;
+  int32_t* active;
+  StatusBlock* sb;
+};
+
+// Router.  When g is non-null and T <= kFusedRouterMaxT the same kernel also
+// writes the grouping (and *grouped is set); otherwise the caller runs
+// launch_permute next.
 cudaError_t launch_router(const void* x, mova_dtype x_dt, const float* Wr, const float* br, int T,
                           int d, int E, int k, float scale, int32_t* idx, float* w,
-                          cudaStream_t stream);
+                          const GroupOut* g, bool* grouped, cudaStream_t stream);
+
+// Launch with programmatic dependent launch enabled: the kernel may start
+// while its predecessor on the stream finishes, and waits for it with
+// griddepcontrol.wait before touching its outputs.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t stream, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
+// Per-device SM count (cached).
+int sm_count();
 
 // Stable counting sort of the pairs by expert.  idx_in has dtype idx_dt
 // (int32 or int8); when w_in is given (w_dt fp32 or fp16) it is converted to
@@ -30,8 +68,12 @@ cudaError_t launch_permute(const void* idx_in, mova_dtype idx_dt, const void* w_
 // pair p (fp32 rows in grouped order).
 cudaError_t launch_stream_experts(const void* x, const void* Wv, mova_dtype dt, const int32_t* counts,
                                   const int32_t* offsets, const int32_t* perm, const float* w32,
-                                  const int32_t* active, const StatusBlock* sb, int d, int n, int k,
+                                  const int32_t* active, StatusBlock* sb, int d, int n, int k,
                                   int E, float* P, cudaStream_t stream);
+
+// Shared memory the streaming kernel needs for rows of d elements (0 if d is
+// too long for two 8-row stages).
+size_t stream_experts_smem(int d, mova_dtype dt, int* stages_out);
 
 // tcgen05 grouped GEMM (bf16): P[p, :] = w * SiLU(Wv[e] x[t]) as bf16 rows.
 cudaError_t launch_tensor_experts(const void* x, const void* Wv, const int32_t* counts,

@@ -14,6 +14,20 @@
 #include "internal.h"
 
 namespace mova {
+
+int sm_count() {
+  static int cached[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (cached[dev] == 0) {
+    int sms = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
+      sms = 148;
+    cached[dev] = sms;
+  }
+  return cached[dev];
+}
+
 namespace {
 
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
@@ -68,19 +82,29 @@ mova_status from_cuda(cudaError_t e) {
 
 bool valid_act_dtype(mova_dtype dt) { return dt == MOVA_F32 || dt == MOVA_BF16; }
 
+// Records stage event i (if events were given); external so that it also
+// becomes an event node under stream capture.
+cudaError_t mark(void* const* events, int i, cudaStream_t s) {
+  if (events == nullptr || events[i] == nullptr) return cudaSuccess;
+  return cudaEventRecordWithFlags(static_cast<cudaEvent_t>(events[i]), s, cudaEventRecordExternal);
+}
+
 // Experts and combine, shared by both value entry points.
 mova_status run_experts_and_combine(const void* x, mova_dtype dt, const void* Wv,
                                     const Workspace& ws, const int32_t* idx, const float* w32,
                                     int T, int d, int E, int k, int n, void* v, mova_path path,
-                                    cudaStream_t stream) {
+                                    void* const* events, cudaStream_t stream) {
   (void)idx;
   if (path == MOVA_PATH_AUTO) path = mova_auto_path(T, dt);
   if (path == MOVA_PATH_TENSOR) return MOVA_ERR_UNSUPPORTED;
+  if (stream_experts_smem(d, dt, nullptr) == 0) return MOVA_ERR_UNSUPPORTED;
   cudaError_t err = launch_stream_experts(x, Wv, dt, ws.counts, ws.offsets, ws.perm, w32,
                                           ws.active, ws.sb, d, n, k, E,
                                           static_cast<float*>(ws.P), stream);
-  if (err != cudaSuccess) return from_cuda(err);
-  return from_cuda(launch_combine(ws.P, false, ws.pos, T, k, n, v, dt, stream));
+  if (err == cudaSuccess) err = mark(events, 3, stream);
+  if (err == cudaSuccess) err = launch_combine(ws.P, false, ws.pos, T, k, n, v, dt, stream);
+  if (err == cudaSuccess) err = mark(events, 4, stream);
+  return from_cuda(err);
 }
 
 }  // namespace
@@ -122,7 +146,7 @@ mova_status mova_route(const void* x, mova_dtype x_dt, const float* Wr, const fl
   if (T == 0) return MOVA_OK;
   if (!x || !Wr || !br || !idx || !w) return MOVA_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(Wr)) return MOVA_ERR_INVALID_ARG;
-  return from_cuda(launch_router(x, x_dt, Wr, br, T, d, E, k, scale, idx, w,
+  return from_cuda(launch_router(x, x_dt, Wr, br, T, d, E, k, scale, idx, w, nullptr, nullptr,
                                  static_cast<cudaStream_t>(stream)));
 }
 
@@ -143,7 +167,7 @@ mova_status mova_permute(const int32_t* idx, int T, int E, int k, int32_t* count
 mova_status mova_value_ex(const void* x, mova_dtype x_dt, const void* idx, mova_dtype idx_dt,
                           const void* wgt, mova_dtype w_dt, const void* Wv, mova_dtype wv_dt, int T,
                           int d, int E, int k, int n, void* v, void* ws, size_t ws_bytes,
-                          mova_path path, void* stream) {
+                          mova_path path, void* const* events, void* stream) {
   mova_status st = check_dims(T, d, E, k, n);
   if (st != MOVA_OK) return st;
   if (!valid_act_dtype(x_dt) || wv_dt != x_dt) return MOVA_ERR_UNSUPPORTED;
@@ -157,10 +181,14 @@ mova_status mova_value_ex(const void* x, mova_dtype x_dt, const void* idx, mova_
   const Workspace w = layout(ws, T, k, n);
   if (ws_bytes < w.bytes || (reinterpret_cast<uintptr_t>(ws) & 255) != 0) return MOVA_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  cudaError_t err = launch_permute(idx, idx_dt, wgt, w_dt, T * k, E, w.idx, w.w, w.counts,
-                                   w.offsets, w.perm, w.pos, w.active, w.sb, s);
+  cudaError_t err = mark(events, 0, s);
+  if (err == cudaSuccess) err = mark(events, 1, s);
+  if (err == cudaSuccess)
+    err = launch_permute(idx, idx_dt, wgt, w_dt, T * k, E, w.idx, w.w, w.counts, w.offsets, w.perm,
+                         w.pos, w.active, w.sb, s);
+  if (err == cudaSuccess) err = mark(events, 2, s);
   if (err != cudaSuccess) return from_cuda(err);
-  return run_experts_and_combine(x, x_dt, Wv, w, w.idx, w.w, T, d, E, k, n, v, path, s);
+  return run_experts_and_combine(x, x_dt, Wv, w, w.idx, w.w, T, d, E, k, n, v, path, events, s);
 }
 
 mova_status mova_value(const void* x, mova_dtype x_dt, const void* idx, mova_dtype idx_dt,
@@ -168,13 +196,14 @@ mova_status mova_value(const void* x, mova_dtype x_dt, const void* idx, mova_dty
                        int d, int E, int k, int n, void* v, void* ws, size_t ws_bytes,
                        void* stream) {
   return mova_value_ex(x, x_dt, idx, idx_dt, wgt, w_dt, Wv, wv_dt, T, d, E, k, n, v, ws, ws_bytes,
-                       MOVA_PATH_AUTO, stream);
+                       MOVA_PATH_AUTO, nullptr, stream);
 }
 
 mova_status mova_value_routed_ex(const void* x, mova_dtype x_dt, const float* Wr, const float* br,
                                  const void* Wv, mova_dtype wv_dt, int T, int d, int E, int k,
                                  int n, float scale, void* v, int32_t* idx_out, float* w_out,
-                                 void* ws, size_t ws_bytes, mova_path path, void* stream) {
+                                 void* ws, size_t ws_bytes, mova_path path, void* const* events,
+                                 void* stream) {
   mova_status st = check_dims(T, d, E, k, n);
   if (st != MOVA_OK) return st;
   if (!valid_act_dtype(x_dt) || wv_dt != x_dt) return MOVA_ERR_UNSUPPORTED;
@@ -189,12 +218,18 @@ mova_status mova_value_routed_ex(const void* x, mova_dtype x_dt, const float* Wr
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   int32_t* idx = idx_out ? idx_out : w.idx;
   float* wgt = w_out ? w_out : w.w;
-  cudaError_t err = launch_router(x, x_dt, Wr, br, T, d, E, k, scale, idx, wgt, s);
+  const GroupOut g{w.counts, w.offsets, w.perm, w.pos, w.active, w.sb};
+  bool grouped = false;
+  cudaError_t err = mark(events, 0, s);
+  if (err == cudaSuccess)
+    err = launch_router(x, x_dt, Wr, br, T, d, E, k, scale, idx, wgt, &g, &grouped, s);
+  if (err == cudaSuccess) err = mark(events, 1, s);
+  if (err == cudaSuccess && !grouped)
+    err = launch_permute(idx, MOVA_I32, nullptr, MOVA_F32, T * k, E, nullptr, nullptr, w.counts,
+                         w.offsets, w.perm, w.pos, w.active, w.sb, s);
+  if (err == cudaSuccess) err = mark(events, 2, s);
   if (err != cudaSuccess) return from_cuda(err);
-  err = launch_permute(idx, MOVA_I32, nullptr, MOVA_F32, T * k, E, nullptr, nullptr, w.counts,
-                       w.offsets, w.perm, w.pos, w.active, w.sb, s);
-  if (err != cudaSuccess) return from_cuda(err);
-  return run_experts_and_combine(x, x_dt, Wv, w, idx, wgt, T, d, E, k, n, v, path, s);
+  return run_experts_and_combine(x, x_dt, Wv, w, idx, wgt, T, d, E, k, n, v, path, events, s);
 }
 
 mova_status mova_value_routed(const void* x, mova_dtype x_dt, const float* Wr, const float* br,
@@ -202,7 +237,7 @@ mova_status mova_value_routed(const void* x, mova_dtype x_dt, const float* Wr, c
                               float scale, void* v, int32_t* idx_out, float* w_out, void* ws,
                               size_t ws_bytes, void* stream) {
   return mova_value_routed_ex(x, x_dt, Wr, br, Wv, wv_dt, T, d, E, k, n, scale, v, idx_out, w_out,
-                              ws, ws_bytes, MOVA_PATH_AUTO, stream);
+                              ws, ws_bytes, MOVA_PATH_AUTO, nullptr, stream);
 }
 
 mova_status mova_get_status(void* ws, int32_t* detail_out, void* stream) {

@@ -43,6 +43,7 @@ permute_kernel(const IT* __restrict__ idx_in, const WT* __restrict__ w_in, int N
   if (tid == 0) {
     sb->code = 0;
     sb->detail = 0;
+    sb->work_next = 0;
   }
   __syncthreads();
 

@@ -6,145 +6,325 @@
 // notice", section "Where the routing happens" (each selected expert's
 // projection passes through SiLU and is weighted by its renormalised score).
 //
-// At a few tokens per expert the work is a matrix-vector product per active
-// expert and HBM-bound: the kernel streams each active expert's n x d weight
-// exactly once.  A warp owns a task of two weight rows of one active expert
-// and all the tokens routed to it (in chunks of 8): each lane reads 16-byte
-// vectors of the rows (no L1 allocation, evict-first in L2, since each row is
-// read once) and multiplies them with the matching x vectors (L1/L2 hits).
-// Partial sums are reduced by a transposing butterfly, so lane l ends with
-// one (row, token) dot product and applies SiLU x weight.  Tasks are spread
-// round-robin over all warps of a grid sized to the SM count, so the whole
-// GPU streams every active expert in parallel.  Every sum runs in a fixed
-// order: results are deterministic.
+// At a few tokens per expert this is a matrix-vector product per active
+// expert and HBM-bound: each active expert's n x d weight is read exactly
+// once.  The rows of all active experts, concatenated, are split evenly over
+// one persistent CTA per SM.  In each CTA a producer warp streams 8-row slabs
+// (contiguous bytes of one or two experts) into a ring of shared-memory
+// stages with 1-D bulk (TMA) copies completing on mbarriers, so each SM keeps
+// ~160 KB of weights in flight without spending registers on it; eight
+// consumer warps take one row of each slab, dot it with the x rows of the
+// expert's tokens (L1 hits), reduce across lanes in a fixed butterfly order
+// and write w * SiLU(h).  Every wait is bounded; a wait that runs out sets
+// MOVA_ERR_TIMEOUT in the status block and the CTA drains its copies and
+// exits.
 #include "common.cuh"
 #include "internal.h"
+
+#include "sm100.cuh"
 
 namespace mova {
 
 namespace {
 
-constexpr int kThreads = 256;
-constexpr int kRows = 2;   // weight rows per warp task
-constexpr int kTok = 8;    // tokens per chunk
+constexpr int kConsumerWarps = 8;
+constexpr int kThreads = (kConsumerWarps + 1) * 32;  // warp 8 produces
+constexpr int kRowsPerStage = kConsumerWarps;
+constexpr int kTok = 8;
+constexpr int kMaxStages = 8;
 
-// Transposing butterfly over 16 values per lane: at each step a lane keeps
-// one half of its values and trades the other half with its partner, so after
-// four steps lane l holds the sum over lanes of value index (l >> 1) & 15 (a
-// fifth exchange adds the halves held by lanes l and l ^ 1).
-template <int V>
-__device__ __forceinline__ float transpose_reduce(float (&v)[V], int lane) {
-  static_assert(V == 16, "lane-to-index map assumes 16 values");
-  int cnt = V;
-  int s = 16;
+template <typename DT> struct Vec;
+template <> struct Vec<__nv_bfloat16> { static constexpr int EL = 8; };
+template <> struct Vec<float> { static constexpr int EL = 4; };
+
+__device__ __forceinline__ void unpack(const uint4& u, const __nv_bfloat16*, float out[8]) {
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
 #pragma unroll
-  for (int step = V; step > 1; step >>= 1) {
-    const bool upper = (lane & s) != 0;
-    const int half = step >> 1;
-#pragma unroll
-    for (int i = 0; i < half; ++i) {
-      const float send = upper ? v[i] : v[i + half];
-      const float keep = upper ? v[i + half] : v[i];
-      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, s);
-    }
-    s >>= 1;
-    cnt = half;
+  for (int i = 0; i < 4; ++i) {
+    float2 f = __bfloat1622float2(h[i]);
+    out[2 * i] = f.x;
+    out[2 * i + 1] = f.y;
   }
-  (void)cnt;
-  for (; s >= 1; s >>= 1) v[0] += __shfl_xor_sync(0xffffffffu, v[0], s);
-  return v[0];
+}
+__device__ __forceinline__ void unpack(const uint4& u, const float*, float out[4]) {
+  out[0] = __uint_as_float(u.x); out[1] = __uint_as_float(u.y);
+  out[2] = __uint_as_float(u.z); out[3] = __uint_as_float(u.w);
+}
+__device__ __forceinline__ void load_x(const __nv_bfloat16* p, float out[8]) { load8(p, out); }
+__device__ __forceinline__ void load_x(const float* p, float out[4]) {
+  const float4 a = *reinterpret_cast<const float4*>(p);
+  out[0] = a.x; out[1] = a.y; out[2] = a.z; out[3] = a.w;
+}
+
+// ---- bf16 consumers: legacy mma.sync m16n8k16 fragments ------------------
+// A = 8 weight rows (rows 8..15 of the fragment are zero), B = up to 8
+// tokens' x, both read with ldmatrix from row-padded shared memory (pitch =
+// row bytes + 16, so the 8 rows of an 8x8 matrix hit distinct banks).  The 8
+// consumer warps split K; partial 8x8 tiles meet in shared memory and are
+// summed in warp order.
+
+__device__ __forceinline__ void ldsm_x2(uint32_t addr, uint32_t& r0, uint32_t& r1) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0, %1}, [%2];"
+               : "=r"(r0), "=r"(r1)
+               : "r"(addr));
+}
+
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a2, uint32_t b0,
+                                               uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1));
+}
+
+// Consumer-group barrier (the 8 consumer warps only; the producer warp never
+// joins it).
+__device__ __forceinline__ void consumers_sync() {
+  asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");
 }
 
 template <typename DT>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, 1)
 stream_experts_kernel(const DT* __restrict__ x, const DT* __restrict__ Wv,
                       const int32_t* __restrict__ counts, const int32_t* __restrict__ offsets,
                       const int32_t* __restrict__ perm, const float* __restrict__ w32,
-                      const int32_t* __restrict__ active, const StatusBlock* __restrict__ sb,
-                      int d, int n, int k, float* __restrict__ P) {
-  const int nact = sb->num_active;
-  const int tasks_per_expert = n / kRows;
-  const long long total = static_cast<long long>(nact) * tasks_per_expert;
-  const int lane = threadIdx.x & 31;
-  const long long gw = (static_cast<long long>(blockIdx.x) * kThreads + threadIdx.x) >> 5;
-  const long long nw = (static_cast<long long>(gridDim.x) * kThreads) >> 5;
+                      const int32_t* __restrict__ active, StatusBlock* __restrict__ sb, int d,
+                      int n, int k, float* __restrict__ P, int NS) {
+  constexpr bool kMma = sizeof(DT) == 2;
+  constexpr int EL = Vec<DT>::EL;
+  extern __shared__ __align__(128) uint8_t smem[];
+  const size_t row_bytes = static_cast<size_t>(d) * sizeof(DT);
+  const size_t pitch = row_bytes + 16;
+  const size_t stage_bytes = pitch * kRowsPerStage;
+  uint8_t* stages = smem;
+  uint8_t* xs = smem + NS * stage_bytes;                    // bf16: kTok padded x rows
+  float* red = reinterpret_cast<float*>(xs + (kMma ? kTok * pitch : 0));  // [warps][8][8]
+  uint64_t* full = reinterpret_cast<uint64_t*>(red + (kMma ? kConsumerWarps * 64 : 0));
+  uint64_t* empty = full + kMaxStages;
+  int* act = reinterpret_cast<int*>(empty + kMaxStages);
+  volatile int* abort_flag = act + 64;
+  int* issued = act + 65;
 
-  for (long long task = gw; task < total; task += nw) {
-    const int a = static_cast<int>(task / tasks_per_expert);
-    const int row0 = static_cast<int>(task % tasks_per_expert) * kRows;
-    const int e = active[a];
-    const int cnt = counts[e];
-    const int off = offsets[e];
-    const DT* wr0 = Wv + (static_cast<size_t>(e) * n + row0) * d;
-    const DT* wr1 = wr0 + d;
-    for (int c0 = 0; c0 < cnt; c0 += kTok) {
-      const int nt = min(kTok, cnt - c0);
-      const DT* xr[kTok];
-#pragma unroll
-      for (int j = 0; j < kTok; ++j) {
-        const int f = perm[off + c0 + min(j, nt - 1)];
-        xr[j] = x + static_cast<size_t>(f / k) * d;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kConsumerWarps);
+    }
+    *abort_flag = 0;
+    *issued = 0;
+    fence_barrier_init();
+  }
+  pdl_wait();  // routing and grouping of this call are complete and visible
+  const int nact = sb->num_active;
+  if (threadIdx.x < 64) act[threadIdx.x] = (threadIdx.x < nact) ? active[threadIdx.x] : 0;
+  __syncthreads();
+  pdl_trigger();
+
+  // Rows of all active experts, in units of whole stages (n % 8 == 0, so a
+  // stage never straddles two experts), split evenly over the CTAs.
+  const int units_per_expert = n / kRowsPerStage;
+  const int units = nact * units_per_expert;
+  const int u0 = static_cast<int>(static_cast<long long>(units) * blockIdx.x / gridDim.x);
+  const int u1 = static_cast<int>(static_cast<long long>(units) * (blockIdx.x + 1) / gridDim.x);
+  const int nstages = u1 - u0;
+
+  if (warp == kConsumerWarps) {
+    if (lane == 0) {
+      const uint64_t pol = policy_evict_first();
+      int j = 0;
+      for (; j < nstages; ++j) {
+        const int s = j % NS;
+        if (j >= NS && !mbar_wait(&empty[s], ((j / NS) - 1) & 1)) {
+          raise_status(sb, MOVA_ERR_TIMEOUT, blockIdx.x);
+          *abort_flag = 1;
+          break;
+        }
+        if (*abort_flag) break;
+        const int u = u0 + j;
+        const int a = u / units_per_expert;
+        const int r = (u - a * units_per_expert) * kRowsPerStage;
+        const DT* src = Wv + (static_cast<size_t>(act[a]) * n + r) * d;
+        mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(kRowsPerStage * row_bytes));
+        uint8_t* dst = stages + s * stage_bytes;
+#pragma unroll 1
+        for (int i = 0; i < kRowsPerStage; ++i)
+          bulk_g2s(dst + i * pitch, src + static_cast<size_t>(i) * d,
+                   static_cast<uint32_t>(row_bytes), &full[s], pol);
       }
-      float acc[kRows * kTok];
-#pragma unroll
-      for (int i = 0; i < kRows * kTok; ++i) acc[i] = 0.f;
-#pragma unroll 2
-      for (int kk = lane * 8; kk < d; kk += 256) {
-        float wa[8], wb[8];
-        load8_stream(wr0 + kk, wa);
-        load8_stream(wr1 + kk, wb);
-#pragma unroll
-        for (int j = 0; j < kTok; ++j) {
-          if (j < nt) {
-            float xv[8];
-            load8(xr[j] + kk, xv);
-#pragma unroll
-            for (int q = 0; q < 8; ++q) {
-              acc[j] = fmaf(wa[q], xv[q], acc[j]);
-              acc[kTok + j] = fmaf(wb[q], xv[q], acc[kTok + j]);
+      *issued = j;
+    }
+  } else {
+    int cur_a = -1, cnt = 0, off = 0;
+    int staged_a = -1, staged_c0 = -1;  // whose x rows the x tile holds
+    for (int j = 0; j < nstages; ++j) {
+      const int s = j % NS;
+      if (*abort_flag) break;
+      if (!mbar_wait(&full[s], (j / NS) & 1)) {
+        raise_status(sb, MOVA_ERR_TIMEOUT, blockIdx.x);
+        *abort_flag = 1;
+        break;
+      }
+      const int u = u0 + j;
+      const int a = u / units_per_expert;
+      const int r0 = (u - a * units_per_expert) * kRowsPerStage;
+      if (a != cur_a) {
+        cur_a = a;
+        cnt = counts[act[a]];
+        off = offsets[act[a]];
+      }
+      const uint8_t* wst = stages + s * stage_bytes;
+      for (int c0 = 0; c0 < cnt; c0 += kTok) {
+        const int nt = min(kTok, cnt - c0);
+        if constexpr (kMma) {
+          // Stage this chunk's x rows (once per expert and chunk; rows
+          // beyond nt repeat the last token and are never stored).
+          if (a != staged_a || c0 != staged_c0) {
+            staged_a = a;
+            staged_c0 = c0;
+            consumers_sync();
+            const int vec_per_row = static_cast<int>(row_bytes / 16);
+            for (int i = threadIdx.x; i < kTok * vec_per_row; i += kConsumerWarps * 32) {
+              const int t = i / vec_per_row;
+              const int v = i - t * vec_per_row;
+              const int f = perm[off + c0 + min(t, nt - 1)];
+              const uint4* srow = reinterpret_cast<const uint4*>(x + static_cast<size_t>(f / k) * d);
+              *reinterpret_cast<uint4*>(xs + t * pitch + v * 16) = srow[v];
             }
+            consumers_sync();
+          }
+          // This warp's K slice, in 16-element steps.
+          const int ksteps = d / 16;
+          const int kb = ksteps * warp / kConsumerWarps;
+          const int ke = ksteps * (warp + 1) / kConsumerWarps;
+          float acc[4] = {0.f, 0.f, 0.f, 0.f};
+          const int lr = lane & 7;
+          const int lk = (lane >> 3) & 1;
+          const uint32_t a_base = smem_u32(wst) + lr * static_cast<uint32_t>(pitch) + lk * 16;
+          const uint32_t b_base = smem_u32(xs) + lr * static_cast<uint32_t>(pitch) + lk * 16;
+#pragma unroll 4
+          for (int ks = kb; ks < ke; ++ks) {
+            uint32_t a0, a2, b0, b1;
+            ldsm_x2(a_base + ks * 32, a0, a2);
+            ldsm_x2(b_base + ks * 32, b0, b1);
+            mma_bf16_16816(acc, a0, a2, b0, b1);
+          }
+          // acc[0], acc[1]: weight row lane/4, tokens 2*(lane%4) + {0, 1}.
+          const int g = lane >> 2;
+          const int tc = (lane & 3) * 2;
+          red[(warp * 8 + g) * 8 + tc] = acc[0];
+          red[(warp * 8 + g) * 8 + tc + 1] = acc[1];
+          consumers_sync();
+          if (threadIdx.x < 64) {
+            const int row = threadIdx.x >> 3;
+            const int t = threadIdx.x & 7;
+            if (t < nt) {
+              float h = 0.f;
+#pragma unroll
+              for (int w = 0; w < kConsumerWarps; ++w) h += red[(w * 8 + row) * 8 + t];
+              const int p = off + c0 + t;
+              P[static_cast<size_t>(p) * n + r0 + row] = w32[perm[p]] * siluf_(h);
+            }
+          }
+          consumers_sync();
+        } else {
+          // fp32 weights: CUDA-core dot products, one row per warp.
+          const int f_last = nt - 1;
+          const DT* xr[kTok];
+#pragma unroll
+          for (int t = 0; t < kTok; ++t) {
+            const int f = perm[off + c0 + min(t, f_last)];
+            xr[t] = x + static_cast<size_t>(f / k) * d;
+          }
+          const uint8_t* wrow = wst + warp * pitch;
+          float acc[kTok];
+#pragma unroll
+          for (int t = 0; t < kTok; ++t) acc[t] = 0.f;
+          for (int kk = lane * EL; kk < d; kk += 32 * EL) {
+            const uint4 uu = *reinterpret_cast<const uint4*>(wrow + kk * sizeof(DT));
+            float wv[EL];
+            unpack(uu, static_cast<const DT*>(nullptr), wv);
+#pragma unroll
+            for (int t = 0; t < kTok; ++t) {
+              if (t < nt) {
+                float xv[EL];
+                load_x(xr[t] + kk, xv);
+#pragma unroll
+                for (int q = 0; q < EL; ++q) acc[t] = fmaf(wv[q], xv[q], acc[t]);
+              }
+            }
+          }
+          float mine = 0.f;
+#pragma unroll
+          for (int t = 0; t < kTok; ++t) {
+            if (t < nt) {
+#pragma unroll
+              for (int o = 16; o >= 1; o >>= 1) acc[t] += __shfl_xor_sync(0xffffffffu, acc[t], o);
+              if (lane == t) mine = acc[t];
+            }
+          }
+          if (lane < nt) {
+            const int p = off + c0 + lane;
+            P[static_cast<size_t>(p) * n + r0 + warp] = w32[perm[p]] * siluf_(mine);
           }
         }
       }
-      const float h = transpose_reduce<kRows * kTok>(acc, lane);
-      const int vi = (lane >> 1) & 15;
-      const int r = vi / kTok;
-      const int j = vi % kTok;
-      if ((lane & 1) == 0 && j < nt) {
-        const int p = off + c0 + j;
-        const int f = perm[p];
-        P[static_cast<size_t>(p) * n + row0 + r] = w32[f] * siluf_(h);
-      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);
     }
+  }
+  __syncthreads();
+  // No bulk copy may still be writing this CTA's shared memory at exit: wait
+  // (bounded) for the last phase issued into every stage.
+  if (threadIdx.x == kConsumerWarps * 32) {
+    const int done = *issued;
+    for (int j = max(0, done - NS); j < done; ++j) mbar_wait(&full[j % NS], (j / NS) & 1);
   }
 }
 
 }  // namespace
 
+size_t stream_experts_smem(int d, mova_dtype dt, int* stages_out) {
+  const bool mma = dt == MOVA_BF16;
+  const size_t pitch = static_cast<size_t>(d) * (mma ? 2 : 4) + 16;
+  const size_t stage_bytes = pitch * kRowsPerStage;
+  const size_t fixed = (mma ? kTok * pitch + kConsumerWarps * 64 * sizeof(float) : 0) +
+                       2 * kMaxStages * sizeof(uint64_t) + 66 * sizeof(int);
+  const size_t budget = 220 * 1024;
+  int NS = fixed < budget ? static_cast<int>((budget - fixed) / stage_bytes) : 0;
+  if (NS > kMaxStages) NS = kMaxStages;
+  if (stages_out) *stages_out = NS;
+  if (NS < 2) return 0;
+  return NS * stage_bytes + fixed;
+}
+
 cudaError_t launch_stream_experts(const void* x, const void* Wv, mova_dtype dt, const int32_t* counts,
                                   const int32_t* offsets, const int32_t* perm, const float* w32,
-                                  const int32_t* active, const StatusBlock* sb, int d, int n, int k,
+                                  const int32_t* active, StatusBlock* sb, int d, int n, int k,
                                   int E, float* P, cudaStream_t stream) {
-  int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  // Upper bound of tasks (all E experts active); the kernel reads the real
-  // count of active experts from the status block.
-  const long long max_tasks = static_cast<long long>(E) * (n / kRows);
-  long long blocks = (max_tasks * 32 + kThreads - 1) / kThreads;
-  const long long cap = static_cast<long long>(sms) * 4;
-  if (blocks > cap) blocks = cap;
-  if (blocks < 1) blocks = 1;
+  (void)E;
+  int NS = 0;
+  const size_t smem = stream_experts_smem(d, dt, &NS);
+  if (smem == 0) return cudaErrorInvalidValue;
+  const dim3 grid(sm_count());
   if (dt == MOVA_BF16) {
-    stream_experts_kernel<__nv_bfloat16><<<static_cast<int>(blocks), kThreads, 0, stream>>>(
-        static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(Wv), counts,
-        offsets, perm, w32, active, sb, d, n, k, P);
-  } else {
-    stream_experts_kernel<float><<<static_cast<int>(blocks), kThreads, 0, stream>>>(
-        static_cast<const float*>(x), static_cast<const float*>(Wv), counts, offsets, perm, w32,
-        active, sb, d, n, k, P);
+    auto kern = stream_experts_kernel<__nv_bfloat16>;
+    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           static_cast<int>(smem));
+    if (err != cudaSuccess) return err;
+    return launch_pdl(kern, grid, dim3(kThreads), smem, stream,
+                      static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(Wv),
+                      counts, offsets, perm, w32, active, sb, d, n, k, P, NS);
   }
-  return cudaGetLastError();
+  auto kern = stream_experts_kernel<float>;
+  cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+  if (err != cudaSuccess) return err;
+  return launch_pdl(kern, grid, dim3(kThreads), smem, stream, static_cast<const float*>(x),
+                    static_cast<const float*>(Wv), counts, offsets, perm, w32, active, sb, d, n, k,
+                    P, NS);
 }
 
 }  // namespace mova

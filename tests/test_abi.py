@@ -87,7 +87,7 @@ def test_host_side_validation(lib):
                         64, 4, 1024, fake, fake, 1 << 30, None)
     assert st == _lib.ERR_UNSUPPORTED  # idx must be int32 or int8
     st = lib.mova_value_ex(fake, _lib.BF16, fake, _lib.I8, fake, _lib.F16, fake, _lib.BF16, 8, 2560,
-                           64, 4, 1024, fake, fake, 1 << 30, 7, None)
+                           64, 4, 1024, fake, fake, 1 << 30, 7, None, None)
     assert st == _lib.ERR_INVALID_ARG  # unknown path
     st = lib.mova_permute(None, 0, 64, 4, None, None, None, None, None, 0, None)
     assert st == _lib.OK

@@ -184,6 +184,12 @@ def test_full_edge_shapes(api, T, E, k, n):
     _full(api, T, 256, E, k, n, "bf16", seed=T)
 
 
+@pytest.mark.parametrize("T", [24, 64])
+def test_full_stream_mid(api, T):
+    """Weight-streaming path with more than 8 tokens on some experts."""
+    _full(api, T, 2560, 64, 4, 1024, "bf16", seed=T, path="stream")
+
+
 def test_full_zero_tokens(api):
     lay = _layer(0, 256, 8, 128, "bf16")
     x = torch.empty((0, 256), dtype=torch.bfloat16, device="cuda")
