@@ -68,8 +68,8 @@ cudaError_t launch_permute(const void* idx_in, mova_dtype idx_dt, const void* w_
 // pair p (fp32 rows in grouped order).
 cudaError_t launch_stream_experts(const void* x, const void* Wv, mova_dtype dt, const int32_t* counts,
                                   const int32_t* offsets, const int32_t* perm, const float* w32,
-                                  const int32_t* active, StatusBlock* sb, int d, int n, int k,
-                                  int E, float* P, cudaStream_t stream);
+                                  const int32_t* active, StatusBlock* sb, int T, int d, int n,
+                                  int k, int E, float* P, cudaStream_t stream);
 
 // Shared memory the streaming kernel needs for rows of d elements (0 if d is
 // too long for two 8-row stages).

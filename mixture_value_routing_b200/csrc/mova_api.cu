@@ -99,7 +99,7 @@ mova_status run_experts_and_combine(const void* x, mova_dtype dt, const void* Wv
   if (path == MOVA_PATH_TENSOR) return MOVA_ERR_UNSUPPORTED;
   if (stream_experts_smem(d, dt, nullptr) == 0) return MOVA_ERR_UNSUPPORTED;
   cudaError_t err = launch_stream_experts(x, Wv, dt, ws.counts, ws.offsets, ws.perm, w32,
-                                          ws.active, ws.sb, d, n, k, E,
+                                          ws.active, ws.sb, T, d, n, k, E,
                                           static_cast<float*>(ws.P), stream);
   if (err == cudaSuccess) err = mark(events, 3, stream);
   if (err == cudaSuccess) err = launch_combine(ws.P, false, ws.pos, T, k, n, v, dt, stream);

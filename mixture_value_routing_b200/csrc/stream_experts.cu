@@ -89,8 +89,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 stream_experts_kernel(const DT* __restrict__ x, const DT* __restrict__ Wv,
                       const int32_t* __restrict__ counts, const int32_t* __restrict__ offsets,
                       const int32_t* __restrict__ perm, const float* __restrict__ w32,
-                      const int32_t* __restrict__ active, StatusBlock* __restrict__ sb, int d,
-                      int n, int k, float* __restrict__ P, int NS) {
+                      const int32_t* __restrict__ active, StatusBlock* __restrict__ sb, int T,
+                      int d, int n, int k, float* __restrict__ P, int NS) {
   constexpr bool kMma = sizeof(DT) == 2;
   constexpr int EL = Vec<DT>::EL;
   extern __shared__ __align__(128) uint8_t smem[];
@@ -99,8 +99,17 @@ stream_experts_kernel(const DT* __restrict__ x, const DT* __restrict__ Wv,
   const size_t stage_bytes = pitch * kRowsPerStage;
   uint8_t* stages = smem;
   uint8_t* xs = smem + NS * stage_bytes;                    // bf16: kTok padded x rows
-  float* red = reinterpret_cast<float*>(xs + (kMma ? kTok * pitch : 0));  // [warps][8][8]
-  uint64_t* full = reinterpret_cast<uint64_t*>(red + (kMma ? kConsumerWarps * 64 : 0));
+  float* red = reinterpret_cast<float*>(xs + (kMma ? kTok * pitch : 0));  // [2][warps][8][8]
+  float* tok_w = red + (kMma ? 2 * kConsumerWarps * 64 : 0);  // weights of the staged pairs
+  int* tok_p = reinterpret_cast<int*>(tok_w + kTok);           // their grouped positions
+  // Resident mode (bf16, T <= 8): every token's x row stays in the x tile for
+  // the whole kernel, and the pair tables below replace all global loads of
+  // the grouping in the loop.
+  int* pair_tok = tok_p + kTok;          // [64] token of each grouped position
+  float* pair_w = reinterpret_cast<float*>(pair_tok + 64);  // [64] its weight
+  int* act_cnt = reinterpret_cast<int*>(pair_w + 64);       // [64] pairs per active expert
+  int* act_off = act_cnt + 64;                              // [64] first position
+  uint64_t* full = reinterpret_cast<uint64_t*>(act_off + 64);
   uint64_t* empty = full + kMaxStages;
   int* act = reinterpret_cast<int*>(empty + kMaxStages);
   volatile int* abort_flag = act + 64;
@@ -122,6 +131,7 @@ stream_experts_kernel(const DT* __restrict__ x, const DT* __restrict__ Wv,
   if (threadIdx.x < 64) act[threadIdx.x] = (threadIdx.x < nact) ? active[threadIdx.x] : 0;
   __syncthreads();
   pdl_trigger();
+  const bool resident = kMma && T <= kTok;
 
   // Rows of all active experts, in units of whole stages (n % 8 == 0, so a
   // stage never straddles two experts), split evenly over the CTAs.
@@ -159,6 +169,28 @@ stream_experts_kernel(const DT* __restrict__ x, const DT* __restrict__ Wv,
   } else {
     int cur_a = -1, cnt = 0, off = 0;
     int staged_a = -1, staged_c0 = -1;  // whose x rows the x tile holds
+    int rbuf = 0;
+    if (resident) {
+      // Overlaps the producer's first bulk copies.
+      const int vec_per_row = static_cast<int>(row_bytes / 16);
+      for (int i = threadIdx.x; i < T * vec_per_row; i += kConsumerWarps * 32) {
+        const int t = i / vec_per_row;
+        const int v = i - t * vec_per_row;
+        *reinterpret_cast<uint4*>(xs + t * pitch + v * 16) =
+            reinterpret_cast<const uint4*>(x + static_cast<size_t>(t) * d)[v];
+      }
+      const int N = T * k;
+      if (threadIdx.x < N) {
+        const int f = perm[threadIdx.x];
+        pair_tok[threadIdx.x] = f / k;
+        pair_w[threadIdx.x] = w32[f];
+      }
+      if (threadIdx.x < nact) {
+        act_cnt[threadIdx.x] = counts[act[threadIdx.x]];
+        act_off[threadIdx.x] = offsets[act[threadIdx.x]];
+      }
+      consumers_sync();
+    }
     for (int j = 0; j < nstages; ++j) {
       const int s = j % NS;
       if (*abort_flag) break;
@@ -172,8 +204,8 @@ stream_experts_kernel(const DT* __restrict__ x, const DT* __restrict__ Wv,
       const int r0 = (u - a * units_per_expert) * kRowsPerStage;
       if (a != cur_a) {
         cur_a = a;
-        cnt = counts[act[a]];
-        off = offsets[act[a]];
+        cnt = resident ? act_cnt[a] : counts[act[a]];
+        off = resident ? act_off[a] : offsets[act[a]];
       }
       const uint8_t* wst = stages + s * stage_bytes;
       for (int c0 = 0; c0 < cnt; c0 += kTok) {
@@ -181,7 +213,7 @@ stream_experts_kernel(const DT* __restrict__ x, const DT* __restrict__ Wv,
         if constexpr (kMma) {
           // Stage this chunk's x rows (once per expert and chunk; rows
           // beyond nt repeat the last token and are never stored).
-          if (a != staged_a || c0 != staged_c0) {
+          if (!resident && (a != staged_a || c0 != staged_c0)) {
             staged_a = a;
             staged_c0 = c0;
             consumers_sync();
@@ -193,6 +225,12 @@ stream_experts_kernel(const DT* __restrict__ x, const DT* __restrict__ Wv,
               const uint4* srow = reinterpret_cast<const uint4*>(x + static_cast<size_t>(f / k) * d);
               *reinterpret_cast<uint4*>(xs + t * pitch + v * 16) = srow[v];
             }
+            if (threadIdx.x < kTok) {
+              const int t = threadIdx.x;
+              const int p = off + c0 + min(t, nt - 1);
+              tok_p[t] = p;
+              tok_w[t] = w32[perm[p]];
+            }
             consumers_sync();
           }
           // This warp's K slice, in 16-element steps.
@@ -203,7 +241,8 @@ stream_experts_kernel(const DT* __restrict__ x, const DT* __restrict__ Wv,
           const int lr = lane & 7;
           const int lk = (lane >> 3) & 1;
           const uint32_t a_base = smem_u32(wst) + lr * static_cast<uint32_t>(pitch) + lk * 16;
-          const uint32_t b_base = smem_u32(xs) + lr * static_cast<uint32_t>(pitch) + lk * 16;
+          const int b_row = resident ? pair_tok[off + c0 + min(lr, nt - 1)] : lr;
+          const uint32_t b_base = smem_u32(xs) + b_row * static_cast<uint32_t>(pitch) + lk * 16;
 #pragma unroll 4
           for (int ks = kb; ks < ke; ++ks) {
             uint32_t a0, a2, b0, b1;
@@ -212,10 +251,15 @@ stream_experts_kernel(const DT* __restrict__ x, const DT* __restrict__ Wv,
             mma_bf16_16816(acc, a0, a2, b0, b1);
           }
           // acc[0], acc[1]: weight row lane/4, tokens 2*(lane%4) + {0, 1}.
+          // Two reduction buffers alternate, so one barrier per tile
+          // suffices: a warp can only overwrite a buffer after every thread
+          // has passed the next barrier, i.e. finished reading it.
+          float* rb = red + (rbuf & 1) * (kConsumerWarps * 64);
+          ++rbuf;
           const int g = lane >> 2;
           const int tc = (lane & 3) * 2;
-          red[(warp * 8 + g) * 8 + tc] = acc[0];
-          red[(warp * 8 + g) * 8 + tc + 1] = acc[1];
+          rb[(warp * 8 + g) * 8 + tc] = acc[0];
+          rb[(warp * 8 + g) * 8 + tc + 1] = acc[1];
           consumers_sync();
           if (threadIdx.x < 64) {
             const int row = threadIdx.x >> 3;
@@ -223,12 +267,12 @@ stream_experts_kernel(const DT* __restrict__ x, const DT* __restrict__ Wv,
             if (t < nt) {
               float h = 0.f;
 #pragma unroll
-              for (int w = 0; w < kConsumerWarps; ++w) h += red[(w * 8 + row) * 8 + t];
-              const int p = off + c0 + t;
-              P[static_cast<size_t>(p) * n + r0 + row] = w32[perm[p]] * siluf_(h);
+              for (int w = 0; w < kConsumerWarps; ++w) h += rb[(w * 8 + row) * 8 + t];
+              const int p = resident ? off + c0 + t : tok_p[t];
+              const float wp = resident ? pair_w[off + c0 + t] : tok_w[t];
+              P[static_cast<size_t>(p) * n + r0 + row] = wp * siluf_(h);
             }
           }
-          consumers_sync();
         } else {
           // fp32 weights: CUDA-core dot products, one row per warp.
           const int f_last = nt - 1;
@@ -290,7 +334,8 @@ size_t stream_experts_smem(int d, mova_dtype dt, int* stages_out) {
   const bool mma = dt == MOVA_BF16;
   const size_t pitch = static_cast<size_t>(d) * (mma ? 2 : 4) + 16;
   const size_t stage_bytes = pitch * kRowsPerStage;
-  const size_t fixed = (mma ? kTok * pitch + kConsumerWarps * 64 * sizeof(float) : 0) +
+  const size_t fixed = (mma ? kTok * pitch + 2 * kConsumerWarps * 64 * sizeof(float) : 0) +
+                       2 * kTok * sizeof(float) + 4 * 64 * sizeof(int) +
                        2 * kMaxStages * sizeof(uint64_t) + 66 * sizeof(int);
   const size_t budget = 220 * 1024;
   int NS = fixed < budget ? static_cast<int>((budget - fixed) / stage_bytes) : 0;
@@ -302,8 +347,8 @@ size_t stream_experts_smem(int d, mova_dtype dt, int* stages_out) {
 
 cudaError_t launch_stream_experts(const void* x, const void* Wv, mova_dtype dt, const int32_t* counts,
                                   const int32_t* offsets, const int32_t* perm, const float* w32,
-                                  const int32_t* active, StatusBlock* sb, int d, int n, int k,
-                                  int E, float* P, cudaStream_t stream) {
+                                  const int32_t* active, StatusBlock* sb, int T, int d, int n,
+                                  int k, int E, float* P, cudaStream_t stream) {
   (void)E;
   int NS = 0;
   const size_t smem = stream_experts_smem(d, dt, &NS);
@@ -316,15 +361,15 @@ cudaError_t launch_stream_experts(const void* x, const void* Wv, mova_dtype dt, 
     if (err != cudaSuccess) return err;
     return launch_pdl(kern, grid, dim3(kThreads), smem, stream,
                       static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(Wv),
-                      counts, offsets, perm, w32, active, sb, d, n, k, P, NS);
+                      counts, offsets, perm, w32, active, sb, T, d, n, k, P, NS);
   }
   auto kern = stream_experts_kernel<float>;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
   if (err != cudaSuccess) return err;
   return launch_pdl(kern, grid, dim3(kThreads), smem, stream, static_cast<const float*>(x),
-                    static_cast<const float*>(Wv), counts, offsets, perm, w32, active, sb, d, n, k,
-                    P, NS);
+                    static_cast<const float*>(Wv), counts, offsets, perm, w32, active, sb, T, d, n,
+                    k, P, NS);
 }
 
 }  // namespace mova

@@ -135,6 +135,22 @@ def test_value_given(api, T, d, E, k, n, dtype, idt, wdt, path):
     P.check_values(P.host_f64(v), v_ref, dtype)
 
 
+def test_value_given_duplicate_experts(api):
+    """A stored routing may name one expert in several slots of a token: every
+    pair still counts once (here one expert receives all 6 x 4 pairs)."""
+    d, E, k, n, T = 512, 8, 4, 256, 6
+    lay = _layer(8, d, E, n, "bf16")
+    bat = MI.make_batch(T, 8, dtype="bf16", d=d)
+    idx = np.full((T, k), 3, np.int32)
+    idx[0, 1] = 5
+    w = np.random.default_rng(3).random((T, k)).astype(np.float32)
+    v = api.value(P.dev(bat.x, "bf16"), P.dev(idx, "i32"), P.dev(w, "f32"), P.dev(lay.Wv, "bf16"),
+                  path="stream")
+    torch.cuda.synchronize()
+    v_ref = O.combine(O.to_f64(bat.x, "bf16"), idx, w.astype(np.float64), lay.Wv, "bf16")
+    P.check_values(P.host_f64(v), v_ref, "bf16")
+
+
 def test_value_given_bad_index_is_flagged(api):
     d, E, k, n, T = 256, 8, 2, 128, 4
     lay = _layer(6, d, E, n, "bf16")
