@@ -1,0 +1,368 @@
+// Grouped expert GEMM on 5th-generation tensor cores (tcgen05), bf16 -> fp32.
+//
+// For every active expert e and every (token, slot) pair p routed to it:
+//   P[p, r] = w[p] * SiLU( sum_j Wv[e, r, j] * x[t(p), j] )
+// i.e. the k selected value projections of "MoVA: routing the value vectors,
+// and why the KV cache does not notice" (section "Where the routing happens"),
+// each passed through SiLU and weighted by its renormalised score; the
+// fixed-order sum over slots happens in the combine kernel.
+//
+// Tiles ("swap AB"): the MMA's M side is 128 weight rows of one expert, its N
+// side up to 256 of the expert's pairs (ragged: rounded up to 16), K runs
+// over d in 64-element steps.  An expert with c pairs is cut into ceil(c/256)
+// near-equal token tiles, each combined with the n/128 weight-row tiles, so
+// tail waste is below 16 columns per tile.
+//
+// One persistent CTA per SM, warp-specialised:
+//   warp 0      TMA producer: weight tile (128 x 64) by a 2-D tensor-map load
+//               with 128-byte swizzle;
+//   warps 1-4   gather producers: the tile's token rows of x (rows chosen by
+//               the grouping), 16-byte cp.async into the same swizzled K-major
+//               layout, completing on the stage's mbarrier;
+//   warp 5      MMA issuer (one thread): 4 x tcgen05.mma (K = 16) per stage
+//               into a tensor-memory accumulator; tcgen05.commit frees the
+//               stage and, per tile, hands the accumulator to the epilogue;
+//   warps 6-9   epilogue: tcgen05.ld of their 32 TMEM lanes, SiLU x weight,
+//               bf16 round, store.
+// Shared memory holds 4 stages of 48 KB; tensor memory holds two 256-column
+// fp32 accumulators, so the epilogue of one tile overlaps the MMAs of the
+// next.  Tiles are dealt round-robin over the CTAs in (expert, token tile,
+// weight-row tile) order, so concurrently running CTAs share weight and x
+// tiles in L2.  Every wait is bounded; a wait that runs out sets
+// MOVA_ERR_TIMEOUT, every role leaves its loop, in-flight copies are drained
+// and tensor memory is freed before the CTA exits.
+#include <cuda.h>
+
+#include "common.cuh"
+#include "internal.h"
+#include "sm100.cuh"
+
+namespace mova {
+
+namespace {
+
+constexpr int BM = 128;
+constexpr int BN = 256;
+constexpr int BK = 64;
+constexpr int kStages = 4;
+constexpr int kABytes = BM * BK * 2;
+constexpr int kBBytes = BN * BK * 2;
+constexpr int kStageBytes = kABytes + kBBytes;
+constexpr int kWarpTma = 0;
+constexpr int kWarpGather0 = 1;
+constexpr int kGatherThreads = 128;
+constexpr int kWarpMma = 5;
+constexpr int kWarpEpi0 = 6;
+constexpr int kEpiThreads = 128;
+constexpr int kThreads = 10 * 32;
+constexpr uint32_t kTmemCols = 512;
+
+struct __align__(1024) Smem {
+  uint8_t stage[kStages][kStageBytes];
+  uint64_t full[kStages];
+  uint64_t empty[kStages];
+  uint64_t tmem_full[2];
+  uint64_t tmem_empty[2];
+  uint32_t tmem_base;
+  int abort;
+  int ntiles;
+  int nact;
+  int act_e[64];
+  int act_cnt[64];
+  int act_off[64];
+  int act_ntt[64];
+  int tile_base[65];
+};
+
+struct Tile {
+  int e, mt, tok0, valid, N, off;
+};
+
+__device__ __forceinline__ Tile decode_tile(const Smem& S, int t, int mtiles) {
+  int a = 0;
+  while (a + 1 < S.nact && S.tile_base[a + 1] <= t) ++a;
+  const int local = t - S.tile_base[a];
+  const int tt = local / mtiles;
+  const int cnt = S.act_cnt[a];
+  const int ntt = S.act_ntt[a];
+  Tile r;
+  r.e = S.act_e[a];
+  r.mt = local - tt * mtiles;
+  r.tok0 = static_cast<int>(static_cast<long long>(tt) * cnt / ntt);
+  r.valid = static_cast<int>(static_cast<long long>(tt + 1) * cnt / ntt) - r.tok0;
+  r.N = (r.valid + 15) & ~15;
+  r.off = S.act_off[a];
+  return r;
+}
+
+__device__ __forceinline__ bool aborted(const Smem& S) {
+  return *reinterpret_cast<const volatile int*>(&S.abort) != 0;
+}
+
+__device__ __forceinline__ void fail(Smem& S, StatusBlock* sb) {
+  raise_status(sb, MOVA_ERR_TIMEOUT, static_cast<int32_t>(blockIdx.x));
+  *reinterpret_cast<volatile int*>(&S.abort) = 1;
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_w, const __nv_bfloat16* __restrict__ x,
+                    const int32_t* __restrict__ counts, const int32_t* __restrict__ offsets,
+                    const int32_t* __restrict__ perm, const float* __restrict__ w32,
+                    const int32_t* __restrict__ active, StatusBlock* __restrict__ sb, int d,
+                    int n, int k, __nv_bfloat16* __restrict__ P) {
+  extern __shared__ uint8_t smem_raw[];
+  Smem& S = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int mtiles = n / BM;
+  const int nk = d / BK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&S.full[s], 1 + kGatherThreads);  // TMA arrive.expect_tx + one per gatherer
+      mbar_init(&S.empty[s], 1);                   // tcgen05.commit of the MMA thread
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&S.tmem_full[i], 1);
+      mbar_init(&S.tmem_empty[i], kEpiThreads / 32);
+    }
+    S.abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == kWarpMma) {
+    tmem_alloc(&S.tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  pdl_wait();  // grouping of this call is complete and visible
+  if (threadIdx.x < 32) {
+    // Active experts, their pair counts and token-tile counts; tile prefix.
+    const int nact = sb->num_active;
+    int ntt0 = 0, ntt1 = 0;
+    const int a0 = lane, a1 = lane + 32;
+    if (a0 < nact) {
+      const int e = active[a0];
+      const int c = counts[e];
+      S.act_e[a0] = e; S.act_cnt[a0] = c; S.act_off[a0] = offsets[e];
+      ntt0 = (c + BN - 1) / BN;
+      S.act_ntt[a0] = ntt0;
+    }
+    if (a1 < nact) {
+      const int e = active[a1];
+      const int c = counts[e];
+      S.act_e[a1] = e; S.act_cnt[a1] = c; S.act_off[a1] = offsets[e];
+      ntt1 = (c + BN - 1) / BN;
+      S.act_ntt[a1] = ntt1;
+    }
+    int v0 = ntt0 * mtiles, v1 = ntt1 * mtiles;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y0 = __shfl_up_sync(0xffffffffu, v0, o);
+      const int y1 = __shfl_up_sync(0xffffffffu, v1, o);
+      if (lane >= o) { v0 += y0; v1 += y1; }
+    }
+    const int tot0 = __shfl_sync(0xffffffffu, v0, 31);
+    S.tile_base[a0 + 1] = v0;
+    S.tile_base[a1 + 1] = tot0 + v1;
+    if (lane == 0) {
+      S.tile_base[0] = 0;
+      S.nact = nact;
+    }
+    if (lane == 31) S.ntiles = tot0 + v1;  // tiles beyond nact contribute 0
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  pdl_trigger();
+  const int ntiles = S.ntiles;
+
+  if (warp == kWarpTma) {
+    if (lane == 0) {
+      int it = 0;
+      for (int t = blockIdx.x; t < ntiles && !aborted(S); t += gridDim.x) {
+        const Tile tl = decode_tile(S, t, mtiles);
+        const int row = tl.e * n + tl.mt * BM;
+        for (int kb = 0; kb < nk; ++kb, ++it) {
+          const int s = it % kStages;
+          if (it >= kStages && !mbar_wait(&S.empty[s], ((it / kStages) - 1) & 1)) { fail(S, sb); break; }
+          mbar_arrive_expect_tx(&S.full[s], kABytes);
+          tma_load_2d_nohint(S.stage[s], &tmap_w, kb * BK, row, &S.full[s]);
+        }
+      }
+    }
+  } else if (warp >= kWarpGather0 && warp < kWarpGather0 + 4) {
+    const int g = threadIdx.x - kWarpGather0 * 32;
+    int it = 0;
+    for (int t = blockIdx.x; t < ntiles && !aborted(S); t += gridDim.x) {
+      const Tile tl = decode_tile(S, t, mtiles);
+      const __nv_bfloat16* src[2];
+      bool have[2];
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        const int r = g + i * kGatherThreads;
+        have[i] = r < tl.N;
+        const int pr = tl.off + tl.tok0 + min(r, tl.valid - 1);
+        src[i] = x + static_cast<size_t>(perm[pr] / k) * d;
+      }
+      bool ok = true;
+      for (int kb = 0; kb < nk; ++kb, ++it) {
+        const int s = it % kStages;
+        if (it >= kStages && !mbar_wait(&S.empty[s], ((it / kStages) - 1) & 1)) {
+          fail(S, sb);
+          ok = false;
+          break;
+        }
+        uint8_t* bs = S.stage[s] + kABytes;
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+          if (have[i]) {
+            const int r = g + i * kGatherThreads;
+            const __nv_bfloat16* sp = src[i] + kb * BK;
+            uint8_t* drow = bs + r * 128;
+#pragma unroll
+            for (int c = 0; c < 8; ++c) cp_async_16(drow + ((c ^ (r & 7)) << 4), sp + c * 8);
+          }
+        }
+        cp_async_arrive_noinc(&S.full[s]);
+      }
+      if (!ok) break;
+    }
+    cp_async_wait_all();
+  } else if (warp == kWarpMma) {
+    if (lane == 0) {
+      int it = 0, titer = 0;
+      for (int t = blockIdx.x; t < ntiles && !aborted(S); t += gridDim.x, ++titer) {
+        const Tile tl = decode_tile(S, t, mtiles);
+        const int acc = titer & 1;
+        if (titer >= 2 && !mbar_wait(&S.tmem_empty[acc], ((titer / 2) - 1) & 1)) { fail(S, sb); break; }
+        tc_fence_after();
+        const uint32_t d_tmem = S.tmem_base + static_cast<uint32_t>(acc * BN);
+        const uint32_t idesc = idesc_bf16_f32(BM, tl.N);
+        bool ok = true;
+        for (int kb = 0; kb < nk; ++kb, ++it) {
+          const int s = it % kStages;
+          if (!mbar_wait(&S.full[s], (it / kStages) & 1)) { fail(S, sb); ok = false; break; }
+          tc_fence_after();
+          fence_proxy_async_smem();  // gathered rows were written by cp.async
+          const uint32_t a0 = smem_u32(S.stage[s]);
+          const uint32_t b0 = a0 + kABytes;
+#pragma unroll
+          for (int k16 = 0; k16 < BK / 16; ++k16)
+            tc_mma_bf16(d_tmem, smem_desc_sw128(a0 + k16 * 32), smem_desc_sw128(b0 + k16 * 32), idesc,
+                        (kb | k16) != 0);
+          tc_commit(&S.empty[s]);
+        }
+        if (!ok) break;
+        tc_commit(&S.tmem_full[acc]);
+      }
+    }
+  } else if (warp >= kWarpEpi0) {
+    // No block-level barrier in this role: each warp fetches the pair
+    // weights itself (lane l holds columns l, l+32, ...), so a warp that
+    // gives up on a wait can never leave the others stuck at a barrier.
+    const int lg = warp & 3;  // this warp may access TMEM lanes 32*lg .. 32*lg+31
+    int titer = 0;
+    for (int t = blockIdx.x; t < ntiles && !aborted(S); t += gridDim.x, ++titer) {
+      const Tile tl = decode_tile(S, t, mtiles);
+      const int acc = titer & 1;
+      float wreg[BN / 32];
+#pragma unroll
+      for (int q = 0; q < BN / 32; ++q) {
+        const int col = q * 32 + lane;
+        wreg[q] = (col < tl.valid) ? w32[perm[tl.off + tl.tok0 + col]] : 0.f;
+      }
+      if (!mbar_wait(&S.tmem_full[acc], (titer / 2) & 1)) { fail(S, sb); break; }
+      tc_fence_after();
+      const int row = tl.mt * BM + lg * 32 + lane;
+      const uint32_t tbase = S.tmem_base + static_cast<uint32_t>(acc * BN) +
+                             (static_cast<uint32_t>(lg * 32) << 16);
+      __nv_bfloat16* prow = P + static_cast<size_t>(tl.off + tl.tok0) * n + row;
+#pragma unroll
+      for (int q = 0; q < BN / 32; ++q) {
+        if (q * 32 < tl.N) {
+          uint32_t r[32];
+          tmem_ld_32(tbase + q * 32, r);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const float wj = __shfl_sync(0xffffffffu, wreg[q], j);
+            const int col = q * 32 + j;
+            if (col < tl.valid) {
+              const float h = __uint_as_float(r[j]);
+              prow[static_cast<size_t>(col) * n] = __float2bfloat16_rn(wj * siluf_(h));
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&S.tmem_empty[acc]);
+    }
+  }
+
+  __syncthreads();
+  if (S.abort) {
+    // Let every copy and MMA this CTA issued finish before its shared and
+    // tensor memory are released (bounded: a dead wait just gives up).
+    if (threadIdx.x == 0) {
+      for (int s = 0; s < kStages; ++s) {
+        mbar_wait(&S.full[s], 0);
+        mbar_wait(&S.empty[s], 0);
+      }
+    }
+    __syncthreads();
+  }
+  if (warp == kWarpMma) {
+    tc_fence_after();
+    tmem_dealloc(S.tmem_base, kTmemCols);
+  }
+}
+
+using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                 const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                 const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                 CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiled encoder() {
+  static EncodeTiled fn = nullptr;
+  if (fn == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiled>(p);
+  }
+  return fn;
+}
+
+}  // namespace
+
+size_t tensor_experts_smem() { return sizeof(Smem) + 1024; }
+
+cudaError_t launch_tensor_experts(const void* x, const void* Wv, const int32_t* counts,
+                                  const int32_t* offsets, const int32_t* perm, const float* w32,
+                                  const int32_t* active, StatusBlock* sb, int T, int d, int n, int k,
+                                  int E, __nv_bfloat16* P, cudaStream_t stream) {
+  (void)T;
+  EncodeTiled enc = encoder();
+  if (enc == nullptr) return cudaErrorNotSupported;
+  // The experts as one (E*n) x d row-major bf16 matrix; boxes of 128 rows x
+  // 64 columns (128 bytes) with 128-byte swizzle.
+  CUtensorMap tmap;
+  const cuuint64_t gdim[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(E) * n};
+  const cuuint64_t gstride[1] = {static_cast<cuuint64_t>(d) * 2};
+  const cuuint32_t box[2] = {BK, BM};
+  const cuuint32_t estride[2] = {1, 1};
+  if (enc(&tmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(Wv), gdim, gstride, box,
+          estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
+  const size_t smem = tensor_experts_smem();
+  cudaError_t err = cudaFuncSetAttribute(grouped_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+  if (err != cudaSuccess) return err;
+  return launch_pdl(grouped_gemm_kernel, dim3(sm_count()), dim3(kThreads), smem, stream, tmap,
+                    static_cast<const __nv_bfloat16*>(x), counts, offsets, perm, w32, active, sb, d, n,
+                    k, P);
+}
+
+}  // namespace mova

@@ -78,8 +78,9 @@ size_t stream_experts_smem(int d, mova_dtype dt, int* stages_out);
 // tcgen05 grouped GEMM (bf16): P[p, :] = w * SiLU(Wv[e] x[t]) as bf16 rows.
 cudaError_t launch_tensor_experts(const void* x, const void* Wv, const int32_t* counts,
                                   const int32_t* offsets, const int32_t* perm, const float* w32,
-                                  StatusBlock* sb, int T, int d, int n, int k, int E,
-                                  __nv_bfloat16* P, cudaStream_t stream);
+                                  const int32_t* active, StatusBlock* sb, int T, int d, int n, int k,
+                                  int E, __nv_bfloat16* P, cudaStream_t stream);
+size_t tensor_experts_smem();
 
 // v[t, :] = sum over slots (ascending) of P[pos[t*k + slot], :].
 cudaError_t launch_combine(const void* P, bool p_bf16, const int32_t* pos, int T, int k, int n,

@@ -30,6 +30,9 @@ int sm_count() {
 
 namespace {
 
+// AUTO: bf16 batches above this many tokens use the tcgen05 grouped GEMM.
+constexpr int kStreamMaxTokens = 64;
+
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 struct Workspace {
@@ -96,13 +99,19 @@ mova_status run_experts_and_combine(const void* x, mova_dtype dt, const void* Wv
                                     void* const* events, cudaStream_t stream) {
   (void)idx;
   if (path == MOVA_PATH_AUTO) path = mova_auto_path(T, dt);
-  if (path == MOVA_PATH_TENSOR) return MOVA_ERR_UNSUPPORTED;
-  if (stream_experts_smem(d, dt, nullptr) == 0) return MOVA_ERR_UNSUPPORTED;
-  cudaError_t err = launch_stream_experts(x, Wv, dt, ws.counts, ws.offsets, ws.perm, w32,
-                                          ws.active, ws.sb, T, d, n, k, E,
-                                          static_cast<float*>(ws.P), stream);
+  cudaError_t err;
+  const bool tensor = path == MOVA_PATH_TENSOR;
+  if (tensor) {
+    if (dt != MOVA_BF16) return MOVA_ERR_UNSUPPORTED;
+    err = launch_tensor_experts(x, Wv, ws.counts, ws.offsets, ws.perm, w32, ws.active, ws.sb, T, d,
+                                n, k, E, static_cast<__nv_bfloat16*>(ws.P), stream);
+  } else {
+    if (stream_experts_smem(d, dt, nullptr) == 0) return MOVA_ERR_UNSUPPORTED;
+    err = launch_stream_experts(x, Wv, dt, ws.counts, ws.offsets, ws.perm, w32, ws.active, ws.sb, T,
+                                d, n, k, E, static_cast<float*>(ws.P), stream);
+  }
   if (err == cudaSuccess) err = mark(events, 3, stream);
-  if (err == cudaSuccess) err = launch_combine(ws.P, false, ws.pos, T, k, n, v, dt, stream);
+  if (err == cudaSuccess) err = launch_combine(ws.P, tensor, ws.pos, T, k, n, v, dt, stream);
   if (err == cudaSuccess) err = mark(events, 4, stream);
   return from_cuda(err);
 }
@@ -133,9 +142,7 @@ size_t mova_workspace_size(int T, int d, int E, int k, int n) {
 }
 
 mova_path mova_auto_path(int T, mova_dtype x_dt) {
-  (void)T;
-  (void)x_dt;
-  return MOVA_PATH_STREAM;
+  return (x_dt == MOVA_BF16 && T > kStreamMaxTokens) ? MOVA_PATH_TENSOR : MOVA_PATH_STREAM;
 }
 
 mova_status mova_route(const void* x, mova_dtype x_dt, const float* Wr, const float* br, int T,

@@ -206,6 +206,67 @@ def test_full_stream_mid(api, T):
     _full(api, T, 2560, 64, 4, 1024, "bf16", seed=T, path="stream")
 
 
+# ---------------------------------------------------------------------------
+# tcgen05 grouped GEMM (bf16)
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("T,d,E,k,n", [(1, 256, 8, 4, 128), (3, 512, 64, 4, 256), (40, 256, 4, 2, 384),
+                                       (300, 2560, 64, 4, 1024), (700, 512, 2, 2, 128)])
+def test_full_tensor_path(api, T, d, E, k, n):
+    """The tcgen05 path at small and ragged sizes (one token, tiles of 16,
+    several tiles per expert, 700 x 2 pairs over 2 experts = 3 token tiles)."""
+    _full(api, T, d, E, k, n, "bf16", seed=T + 1, path="tensor")
+
+
+def test_tensor_given(api):
+    d, E, k, n, T = 512, 8, 4, 256, 333
+    lay = _layer(9, d, E, n, "bf16")
+    bat = MI.make_batch(T, 9, dtype="bf16", d=d, mode="given", E=E, k=k)
+    v = api.value(P.dev(bat.x, "bf16"), P.dev(bat.idx, "i8"), P.dev(bat.w, "f16"),
+                  P.dev(lay.Wv, "bf16"), path="tensor")
+    torch.cuda.synchronize()
+    assert api.get_status()[0] == "MOVA_OK"
+    v_ref = O.combine(O.to_f64(bat.x, "bf16"), bat.idx.astype(np.int64), bat.w.astype(np.float64),
+                      lay.Wv, "bf16")
+    P.check_values(P.host_f64(v), v_ref, "bf16")
+
+
+def test_full_prefill_4096(api):
+    """Prefill workload at full size (T=4096): routing of every token, values
+    of 256 sampled tokens."""
+    _full(api, 4096, 2560, 64, 4, 1024, "bf16", sample=256)
+
+
+def test_full_skewed_16384(api):
+    """Skewed prefill (router bias 2 ln Zipf(1.2)), T=16384, sampled values."""
+    _full(api, 16384, 2560, 64, 4, 1024, "bf16", bias="zipf", sample=128)
+
+
+def test_given_32768(api):
+    """Routing-given recompute at L=32768 (int8 indices, fp16 weights),
+    sampled values."""
+    lay = _layer(0, 2560, 64, 1024, "bf16")
+    bat = MI.make_batch(32768, 0, dtype="bf16", mode="given")
+    v = api.value(P.dev(bat.x, "bf16"), P.dev(bat.idx, "i8"), P.dev(bat.w, "f16"),
+                  P.dev(lay.Wv, "bf16"))
+    torch.cuda.synchronize()
+    assert api.get_status()[0] == "MOVA_OK"
+    rows = np.sort(np.random.default_rng(5).choice(32768, 128, replace=False))
+    v_ref = O.combine(O.to_f64(bat.x[rows], "bf16"), bat.idx[rows].astype(np.int64),
+                      bat.w[rows].astype(np.float64), lay.Wv, "bf16")
+    P.check_values(P.host_f64(v)[rows], v_ref, "bf16")
+
+
+def test_tensor_deterministic(api):
+    lay = _layer(4, 2560, 64, 1024, "bf16")
+    bat = MI.make_batch(512, 4, dtype="bf16")
+    args = (P.dev(bat.x, "bf16"), P.dev(lay.Wr, "f32"), P.dev(lay.br, "f32"),
+            P.dev(lay.Wv, "bf16"))
+    first = api.value_routed(*args, path="tensor").clone()
+    for _ in range(4):
+        assert torch.equal(api.value_routed(*args, path="tensor"), first)
+
+
 def test_full_zero_tokens(api):
     lay = _layer(0, 256, 8, 128, "bf16")
     x = torch.empty((0, 256), dtype=torch.bfloat16, device="cuda")
