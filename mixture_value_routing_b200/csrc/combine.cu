@@ -1,10 +1,10 @@
 // Fixed-order gather-combine.
 //
-//   v[t, :] = sum over slot = 0..k-1 (ascending) of P[pos[t*k + slot], :]
+//   v[t, :] = sum over slot = 0..k-1 (ascending) of w[t*k + slot] * P[pos[t*k + slot], :]
 //
-// P already holds w * SiLU(Wv[e] x[t]) per (token, slot) pair, in grouped
-// order; this sums each token's k rows in ascending slot order in fp32 and
-// rounds once at the store.  The (T, n) result, n = heads x 128, is the GQA
+// P holds SiLU(Wv[e] x[t]) per (token, slot) pair, in grouped order; this
+// weights each token's k rows by their routing weights and sums them in
+// ascending slot order in fp32, rounding once at the store.  The (T, n) result, n = heads x 128, is the GQA
 // value tensor ("MoVA: routing the value vectors, and why the KV cache does
 // not notice", section "Where the routing happens": the mixture is reshaped
 // into 8 heads of 128 and is exactly what a GQA v_proj produces).
@@ -37,8 +37,8 @@ __device__ __forceinline__ void store8(__nv_bfloat16* p, const float v[8]) {
 
 template <typename PT, typename OT>
 __global__ void __launch_bounds__(kThreads)
-combine_kernel(const PT* __restrict__ P, const int32_t* __restrict__ pos, int T, int k, int n,
-               OT* __restrict__ v) {
+combine_kernel(const PT* __restrict__ P, const int32_t* __restrict__ pos,
+               const float* __restrict__ w32, int T, int k, int n, OT* __restrict__ v) {
   pdl_wait();  // the expert rows of this call are complete and visible
   const int per_tok = n / 8;
   const long long total = static_cast<long long>(T) * per_tok;
@@ -51,38 +51,39 @@ combine_kernel(const PT* __restrict__ P, const int32_t* __restrict__ pos, int T,
     for (int q = 0; q < 8; ++q) acc[q] = 0.f;
     for (int s = 0; s < k; ++s) {
       const int p = pos[static_cast<size_t>(t) * k + s];
+      const float ws = w32[static_cast<size_t>(t) * k + s];
       float pv[8];
       load8_p(P + static_cast<size_t>(p) * n + c, pv);
 #pragma unroll
-      for (int q = 0; q < 8; ++q) acc[q] += pv[q];
+      for (int q = 0; q < 8; ++q) acc[q] = fmaf(ws, pv[q], acc[q]);
     }
     store8(v + static_cast<size_t>(t) * n + c, acc);
   }
 }
 
 template <typename PT, typename OT>
-cudaError_t launch_t(const void* P, const int32_t* pos, int T, int k, int n, void* v,
-                     cudaStream_t stream) {
+cudaError_t launch_t(const void* P, const int32_t* pos, const float* w32, int T, int k, int n,
+                     void* v, cudaStream_t stream) {
   const long long total = static_cast<long long>(T) * (n / 8);
   long long blocks = (total + kThreads - 1) / kThreads;
   const long long cap = static_cast<long long>(sm_count()) * 8;
   if (blocks > cap) blocks = cap;
   if (blocks < 1) blocks = 1;
   return launch_pdl(combine_kernel<PT, OT>, dim3(static_cast<unsigned>(blocks)), dim3(kThreads), 0,
-                    stream, static_cast<const PT*>(P), pos, T, k, n, static_cast<OT*>(v));
+                    stream, static_cast<const PT*>(P), pos, w32, T, k, n, static_cast<OT*>(v));
 }
 
 }  // namespace
 
-cudaError_t launch_combine(const void* P, bool p_bf16, const int32_t* pos, int T, int k, int n,
-                           void* v, mova_dtype v_dt, cudaStream_t stream) {
+cudaError_t launch_combine(const void* P, bool p_bf16, const int32_t* pos, const float* w32, int T,
+                           int k, int n, void* v, mova_dtype v_dt, cudaStream_t stream) {
   if (T <= 0) return cudaSuccess;
   if (p_bf16) {
-    if (v_dt == MOVA_BF16) return launch_t<__nv_bfloat16, __nv_bfloat16>(P, pos, T, k, n, v, stream);
-    return launch_t<__nv_bfloat16, float>(P, pos, T, k, n, v, stream);
+    if (v_dt == MOVA_BF16) return launch_t<__nv_bfloat16, __nv_bfloat16>(P, pos, w32, T, k, n, v, stream);
+    return launch_t<__nv_bfloat16, float>(P, pos, w32, T, k, n, v, stream);
   }
-  if (v_dt == MOVA_BF16) return launch_t<float, __nv_bfloat16>(P, pos, T, k, n, v, stream);
-  return launch_t<float, float>(P, pos, T, k, n, v, stream);
+  if (v_dt == MOVA_BF16) return launch_t<float, __nv_bfloat16>(P, pos, w32, T, k, n, v, stream);
+  return launch_t<float, float>(P, pos, w32, T, k, n, v, stream);
 }
 
 }  // namespace mova

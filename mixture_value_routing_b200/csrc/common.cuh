@@ -94,5 +94,8 @@ __device__ __forceinline__ void pdl_trigger() {
 // Logistic function and SiLU in fp32 (IEEE expf and division).
 __device__ __forceinline__ float sigmoidf_(float z) { return 1.0f / (1.0f + expf(-z)); }
 __device__ __forceinline__ float siluf_(float h) { return h / (1.0f + expf(-h)); }
+// SiLU with the fast exponential and division intrinsics (relative error
+// ~1e-6): used where the result is rounded to bf16 anyway.
+__device__ __forceinline__ float silu_fast(float h) { return __fdividef(h, 1.0f + __expf(-h)); }
 
 }  // namespace mova

@@ -1,11 +1,11 @@
 // Grouped expert GEMM on 5th-generation tensor cores (tcgen05), bf16 -> fp32.
 //
 // For every active expert e and every (token, slot) pair p routed to it:
-//   P[p, r] = w[p] * SiLU( sum_j Wv[e, r, j] * x[t(p), j] )
+//   P[p, r] = SiLU( sum_j Wv[e, r, j] * x[t(p), j] )
 // i.e. the k selected value projections of "MoVA: routing the value vectors,
 // and why the KV cache does not notice" (section "Where the routing happens"),
-// each passed through SiLU and weighted by its renormalised score; the
-// fixed-order sum over slots happens in the combine kernel.
+// each passed through SiLU; the combine kernel weights them by their
+// renormalised scores and sums the slots in fixed order.
 //
 // Tiles ("swap AB"): the MMA's M side is 128 weight rows of one expert, its N
 // side up to 256 of the expert's pairs (ragged: rounded up to 16), K runs
@@ -22,8 +22,8 @@
 //   warp 5      MMA issuer (one thread): 4 x tcgen05.mma (K = 16) per stage
 //               into a tensor-memory accumulator; tcgen05.commit frees the
 //               stage and, per tile, hands the accumulator to the epilogue;
-//   warps 6-9   epilogue: tcgen05.ld of their 32 TMEM lanes, SiLU x weight,
-//               bf16 round, store.
+//   warps 6-9   epilogue: tcgen05.ld of their 32 TMEM lanes, SiLU, bf16
+//               round, store.
 // Shared memory holds 4 stages of 48 KB; tensor memory holds two 256-column
 // fp32 accumulators, so the epilogue of one tile overlaps the MMAs of the
 // next.  Tiles are dealt round-robin over the CTAs in (expert, token tile,
@@ -72,6 +72,7 @@ struct __align__(1024) Smem {
   int act_off[64];
   int act_ntt[64];
   int tile_base[65];
+  int gather_tok[4][64];  // token of each row a gather warp copies
 };
 
 struct Tile {
@@ -190,19 +191,26 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_w, const __nv_bfloa
       }
     }
   } else if (warp >= kWarpGather0 && warp < kWarpGather0 + 4) {
-    const int g = threadIdx.x - kWarpGather0 * 32;
+    // Each gather warp owns 64 rows of the token tile.  Lane l copies 16-byte
+    // chunk (l & 7) of rows (l >> 3) + 4i, so one warp instruction moves 4
+    // whole 128-byte rows (coalesced); the chunk lands at its 128-byte-swizzle
+    // position (chunk ^ (row & 7)).
+    const int gw = warp - kWarpGather0;
+    int* rows = S.gather_tok[gw];
+    const int chunk = lane & 7;
+    const int sub = lane >> 3;
     int it = 0;
     for (int t = blockIdx.x; t < ntiles && !aborted(S); t += gridDim.x) {
       const Tile tl = decode_tile(S, t, mtiles);
-      const __nv_bfloat16* src[2];
-      bool have[2];
+      __syncwarp();
 #pragma unroll
       for (int i = 0; i < 2; ++i) {
-        const int r = g + i * kGatherThreads;
-        have[i] = r < tl.N;
+        const int r = gw * 64 + i * 32 + lane;
         const int pr = tl.off + tl.tok0 + min(r, tl.valid - 1);
-        src[i] = x + static_cast<size_t>(perm[pr] / k) * d;
+        rows[i * 32 + lane] = perm[pr] / k;
       }
+      __syncwarp();
+      const int nrows = min(64, max(0, tl.N - gw * 64));
       bool ok = true;
       for (int kb = 0; kb < nk; ++kb, ++it) {
         const int s = it % kStages;
@@ -212,14 +220,12 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_w, const __nv_bfloa
           break;
         }
         uint8_t* bs = S.stage[s] + kABytes;
-#pragma unroll
-        for (int i = 0; i < 2; ++i) {
-          if (have[i]) {
-            const int r = g + i * kGatherThreads;
-            const __nv_bfloat16* sp = src[i] + kb * BK;
-            uint8_t* drow = bs + r * 128;
-#pragma unroll
-            for (int c = 0; c < 8; ++c) cp_async_16(drow + ((c ^ (r & 7)) << 4), sp + c * 8);
+        for (int i = 0; i < 16; ++i) {
+          const int lr = sub + 4 * i;  // row within this warp's 64
+          if (lr < nrows) {
+            const int r = gw * 64 + lr;
+            const __nv_bfloat16* sp = x + static_cast<size_t>(rows[lr]) * d + kb * BK + chunk * 8;
+            cp_async_16(bs + r * 128 + ((chunk ^ (r & 7)) << 4), sp);
           }
         }
         cp_async_arrive_noinc(&S.full[s]);
@@ -256,41 +262,28 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_w, const __nv_bfloa
       }
     }
   } else if (warp >= kWarpEpi0) {
-    // No block-level barrier in this role: each warp fetches the pair
-    // weights itself (lane l holds columns l, l+32, ...), so a warp that
-    // gives up on a wait can never leave the others stuck at a barrier.
+    // No block-level barrier in this role, so a warp that gives up on a wait
+    // can never leave the others stuck.  Thread = one weight row; columns =
+    // the tile's pairs.
     const int lg = warp & 3;  // this warp may access TMEM lanes 32*lg .. 32*lg+31
     int titer = 0;
     for (int t = blockIdx.x; t < ntiles && !aborted(S); t += gridDim.x, ++titer) {
       const Tile tl = decode_tile(S, t, mtiles);
       const int acc = titer & 1;
-      float wreg[BN / 32];
-#pragma unroll
-      for (int q = 0; q < BN / 32; ++q) {
-        const int col = q * 32 + lane;
-        wreg[q] = (col < tl.valid) ? w32[perm[tl.off + tl.tok0 + col]] : 0.f;
-      }
       if (!mbar_wait(&S.tmem_full[acc], (titer / 2) & 1)) { fail(S, sb); break; }
       tc_fence_after();
       const int row = tl.mt * BM + lg * 32 + lane;
       const uint32_t tbase = S.tmem_base + static_cast<uint32_t>(acc * BN) +
                              (static_cast<uint32_t>(lg * 32) << 16);
       __nv_bfloat16* prow = P + static_cast<size_t>(tl.off + tl.tok0) * n + row;
+      for (int c0 = 0; c0 < tl.N; c0 += 32) {
+        uint32_t r[32];
+        tmem_ld_32(tbase + c0, r);
+        tmem_ld_wait();
 #pragma unroll
-      for (int q = 0; q < BN / 32; ++q) {
-        if (q * 32 < tl.N) {
-          uint32_t r[32];
-          tmem_ld_32(tbase + q * 32, r);
-          tmem_ld_wait();
-#pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const float wj = __shfl_sync(0xffffffffu, wreg[q], j);
-            const int col = q * 32 + j;
-            if (col < tl.valid) {
-              const float h = __uint_as_float(r[j]);
-              prow[static_cast<size_t>(col) * n] = __float2bfloat16_rn(wj * siluf_(h));
-            }
-          }
+        for (int j = 0; j < 32; ++j) {
+          if (c0 + j < tl.valid)
+            prow[static_cast<size_t>(c0 + j) * n] = __float2bfloat16_rn(silu_fast(__uint_as_float(r[j])));
         }
       }
       tc_fence_before();

@@ -64,7 +64,7 @@ cudaError_t launch_permute(const void* idx_in, mova_dtype idx_dt, const void* w_
                            int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* pos,
                            int32_t* active, StatusBlock* sb, cudaStream_t stream);
 
-// Weight-streaming expert kernel: P[p, :] = w * SiLU(Wv[e] x[t]) for every
+// Weight-streaming expert kernel: P[p, :] = SiLU(Wv[e] x[t]) for every
 // pair p (fp32 rows in grouped order).
 cudaError_t launch_stream_experts(const void* x, const void* Wv, mova_dtype dt, const int32_t* counts,
                                   const int32_t* offsets, const int32_t* perm, const float* w32,
@@ -75,15 +75,15 @@ cudaError_t launch_stream_experts(const void* x, const void* Wv, mova_dtype dt, 
 // too long for two 8-row stages).
 size_t stream_experts_smem(int d, mova_dtype dt, int* stages_out);
 
-// tcgen05 grouped GEMM (bf16): P[p, :] = w * SiLU(Wv[e] x[t]) as bf16 rows.
+// tcgen05 grouped GEMM (bf16): P[p, :] = SiLU(Wv[e] x[t]) as bf16 rows.
 cudaError_t launch_tensor_experts(const void* x, const void* Wv, const int32_t* counts,
                                   const int32_t* offsets, const int32_t* perm, const float* w32,
                                   const int32_t* active, StatusBlock* sb, int T, int d, int n, int k,
                                   int E, __nv_bfloat16* P, cudaStream_t stream);
 size_t tensor_experts_smem();
 
-// v[t, :] = sum over slots (ascending) of P[pos[t*k + slot], :].
-cudaError_t launch_combine(const void* P, bool p_bf16, const int32_t* pos, int T, int k, int n,
-                           void* v, mova_dtype v_dt, cudaStream_t stream);
+// v[t, :] = sum over slots (ascending) of w[t*k + slot] * P[pos[t*k + slot], :].
+cudaError_t launch_combine(const void* P, bool p_bf16, const int32_t* pos, const float* w32, int T,
+                           int k, int n, void* v, mova_dtype v_dt, cudaStream_t stream);
 
 }  // namespace mova

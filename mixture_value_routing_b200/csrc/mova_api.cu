@@ -6,8 +6,8 @@
 // routing happens"):
 //   router  -> idx, w                     (fp32 logits, sigmoid, biased top-k)
 //   permute -> counts, offsets, perm, pos (stable grouping by expert)
-//   experts -> P rows = w * SiLU(Wv[e] x) (weight streaming or tcgen05 GEMM)
-//   combine -> v = sum of each token's rows in ascending slot order
+//   experts -> P rows = SiLU(Wv[e] x)     (weight streaming or tcgen05 GEMM)
+//   combine -> v = sum of w x row over each token's slots, ascending
 #include <stdio.h>
 
 #include "common.cuh"
@@ -111,7 +111,7 @@ mova_status run_experts_and_combine(const void* x, mova_dtype dt, const void* Wv
                                 d, n, k, E, static_cast<float*>(ws.P), stream);
   }
   if (err == cudaSuccess) err = mark(events, 3, stream);
-  if (err == cudaSuccess) err = launch_combine(ws.P, tensor, ws.pos, T, k, n, v, dt, stream);
+  if (err == cudaSuccess) err = launch_combine(ws.P, tensor, ws.pos, w32, T, k, n, v, dt, stream);
   if (err == cudaSuccess) err = mark(events, 4, stream);
   return from_cuda(err);
 }

@@ -1,10 +1,11 @@
 // Weight-streaming expert kernel for decode-sized batches (and the fp32 path).
 //
 // Computes, for every (token, slot) pair p routed to expert e,
-//   P[p, :] = w[p] * SiLU(Wv[e] x[t])
+//   P[p, :] = SiLU(Wv[e] x[t])
 // as in "MoVA: routing the value vectors, and why the KV cache does not
 // notice", section "Where the routing happens" (each selected expert's
-// projection passes through SiLU and is weighted by its renormalised score).
+// projection passes through SiLU; the combine kernel weights it by its
+// renormalised score and sums the slots).
 //
 // At a few tokens per expert this is a matrix-vector product per active
 // expert and HBM-bound: each active expert's n x d weight is read exactly
@@ -269,8 +270,7 @@ stream_experts_kernel(const DT* __restrict__ x, const DT* __restrict__ Wv,
 #pragma unroll
               for (int w = 0; w < kConsumerWarps; ++w) h += rb[(w * 8 + row) * 8 + t];
               const int p = resident ? off + c0 + t : tok_p[t];
-              const float wp = resident ? pair_w[off + c0 + t] : tok_w[t];
-              P[static_cast<size_t>(p) * n + r0 + row] = wp * siluf_(h);
+              P[static_cast<size_t>(p) * n + r0 + row] = siluf_(h);
             }
           }
         } else {
@@ -311,7 +311,7 @@ stream_experts_kernel(const DT* __restrict__ x, const DT* __restrict__ Wv,
           }
           if (lane < nt) {
             const int p = off + c0 + lane;
-            P[static_cast<size_t>(p) * n + r0 + warp] = w32[perm[p]] * siluf_(mine);
+            P[static_cast<size_t>(p) * n + r0 + warp] = siluf_(mine);
           }
         }
       }
