@@ -315,18 +315,6 @@ using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, 
                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
-EncodeTiled encoder() {
-  static EncodeTiled fn = nullptr;
-  if (fn == nullptr) {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiled>(p);
-  }
-  return fn;
-}
-
 }  // namespace
 
 size_t tensor_experts_smem() { return sizeof(Smem) + 1024; }
@@ -336,8 +324,9 @@ cudaError_t launch_tensor_experts(const void* x, const void* Wv, const int32_t* 
                                   const int32_t* active, StatusBlock* sb, int T, int d, int n, int k,
                                   int E, __nv_bfloat16* P, cudaStream_t stream) {
   (void)T;
-  EncodeTiled enc = encoder();
-  if (enc == nullptr) return cudaErrorNotSupported;
+  void* fp = encode_tiled_fn();
+  if (fp == nullptr) return cudaErrorNotSupported;
+  EncodeTiled enc = reinterpret_cast<EncodeTiled>(fp);
   // The experts as one (E*n) x d row-major bf16 matrix; boxes of 128 rows x
   // 64 columns (128 bytes) with 128-byte swizzle.
   CUtensorMap tmap;

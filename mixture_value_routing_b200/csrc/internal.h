@@ -56,6 +56,18 @@ cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t sme
 // Per-device SM count (cached).
 int sm_count();
 
+// cuTensorMapEncodeTiled from the driver (cached; nullptr if unavailable).
+void* encode_tiled_fn();
+
+// Tensor-core router (bf16 x): splits Wr into three bf16 planes (in
+// `planes`, router_planes_bytes(d) bytes), then one CTA per 128 tokens
+// computes the logits with tcgen05 and selects; tile_counts (nullable)
+// receives each 128-token tile's expert histogram.
+size_t router_planes_bytes(int d);
+cudaError_t launch_router_tc(const void* x, const float* Wr, const float* br, int T, int d, int E,
+                             int k, float scale, int32_t* idx, float* w, int32_t* tile_counts,
+                             __nv_bfloat16* planes, StatusBlock* sb, cudaStream_t stream);
+
 // Stable counting sort of the pairs by expert.  idx_in has dtype idx_dt
 // (int32 or int8); when w_in is given (w_dt fp32 or fp16) it is converted to
 // fp32 into w32, and idx_in to int32 into idx32 (routing-given mode).
@@ -63,6 +75,20 @@ cudaError_t launch_permute(const void* idx_in, mova_dtype idx_dt, const void* w_
                            mova_dtype w_dt, int N, int E, int32_t* idx32, float* w32,
                            int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* pos,
                            int32_t* active, StatusBlock* sb, cudaStream_t stream);
+
+// Multi-CTA grouping (batches above kSmallGroupT tokens).  Tiles of 128
+// tokens; tile_counts holds group_tiles(T) x 64 ints.  launch_tile_hist
+// fills tile_counts (and, in routing-given mode, idx32/w32 with the range
+// check); launch_tile_group scans and scatters.
+constexpr int kSmallGroupT = 512;
+int group_tiles(int T);
+cudaError_t launch_tile_hist(const void* idx_in, mova_dtype idx_dt, const void* w_in,
+                             mova_dtype w_dt, int T, int E, int k, int32_t* idx32, float* w32,
+                             int32_t* tile_counts, StatusBlock* sb, cudaStream_t stream);
+cudaError_t launch_tile_group(const int32_t* idx32, int T, int E, int k, int32_t* tile_counts,
+                              int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* pos,
+                              int32_t* active, StatusBlock* sb, bool reset_status,
+                              cudaStream_t stream);
 
 // Weight-streaming expert kernel: P[p, :] = SiLU(Wv[e] x[t]) for every
 // pair p (fp32 rows in grouped order).

@@ -15,6 +15,18 @@
 
 namespace mova {
 
+void* encode_tiled_fn() {
+  static void* fn = nullptr;
+  if (fn == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = p;
+  }
+  return fn;
+}
+
 int sm_count() {
   static int cached[64] = {0};
   int dev = 0;
@@ -32,6 +44,8 @@ namespace {
 
 // AUTO: bf16 batches above this many tokens use the tcgen05 grouped GEMM.
 constexpr int kStreamMaxTokens = 64;
+// bf16 batches above this many tokens use the tensor-core router.
+constexpr int kTcRouterMinT = 64;
 
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
@@ -44,25 +58,29 @@ struct Workspace {
   int32_t* active;
   int32_t* perm;
   int32_t* pos;
+  int32_t* tile_counts;
+  __nv_bfloat16* planes;
   void* P;
   size_t bytes;
 };
 
 // Byte layout of the workspace (every part 256-byte aligned).
-Workspace layout(void* base, int T, int k, int n) {
+Workspace layout(void* base, int T, int d, int k, int n) {
   const size_t pairs = static_cast<size_t>(T) * k;
   char* b = static_cast<char*>(base);
   size_t o = 0;
   Workspace w{};
-  w.sb = reinterpret_cast<StatusBlock*>(b + o);      o += 256;
-  w.idx = reinterpret_cast<int32_t*>(b + o);         o += align256(pairs * 4);
-  w.w = reinterpret_cast<float*>(b + o);             o += align256(pairs * 4);
-  w.counts = reinterpret_cast<int32_t*>(b + o);      o += 256;
-  w.offsets = reinterpret_cast<int32_t*>(b + o);     o += 512;
-  w.active = reinterpret_cast<int32_t*>(b + o);      o += 256;
-  w.perm = reinterpret_cast<int32_t*>(b + o);        o += align256(pairs * 4);
-  w.pos = reinterpret_cast<int32_t*>(b + o);         o += align256(pairs * 4);
-  w.P = b + o;                                       o += align256(pairs * static_cast<size_t>(n) * 4);
+  w.sb = reinterpret_cast<StatusBlock*>(b + o);       o += 256;
+  w.idx = reinterpret_cast<int32_t*>(b + o);          o += align256(pairs * 4);
+  w.w = reinterpret_cast<float*>(b + o);              o += align256(pairs * 4);
+  w.counts = reinterpret_cast<int32_t*>(b + o);       o += 256;
+  w.offsets = reinterpret_cast<int32_t*>(b + o);      o += 512;
+  w.active = reinterpret_cast<int32_t*>(b + o);       o += 256;
+  w.perm = reinterpret_cast<int32_t*>(b + o);         o += align256(pairs * 4);
+  w.pos = reinterpret_cast<int32_t*>(b + o);          o += align256(pairs * 4);
+  w.tile_counts = reinterpret_cast<int32_t*>(b + o);  o += align256(static_cast<size_t>(group_tiles(T)) * 64 * 4);
+  w.planes = reinterpret_cast<__nv_bfloat16*>(b + o); o += align256(router_planes_bytes(d));
+  w.P = b + o;                                        o += align256(pairs * static_cast<size_t>(n) * 4);
   w.bytes = o;
   return w;
 }
@@ -138,7 +156,7 @@ const char* mova_status_str(mova_status s) {
 size_t mova_workspace_size(int T, int d, int E, int k, int n) {
   if (check_dims(T, d, E, k, n) != MOVA_OK) return 0;
   if (T == 0) return 0;
-  return layout(nullptr, T, k, n).bytes;
+  return layout(nullptr, T, d, k, n).bytes;
 }
 
 mova_path mova_auto_path(int T, mova_dtype x_dt) {
@@ -164,11 +182,19 @@ mova_status mova_permute(const int32_t* idx, int T, int E, int k, int32_t* count
   if (st != MOVA_OK) return st;
   if (T == 0) return MOVA_OK;
   if (!idx || !counts || !offsets || !perm || !pos || !ws) return MOVA_ERR_INVALID_ARG;
-  const Workspace w = layout(ws, T, k, 128);
+  const Workspace w = layout(ws, T, 64, k, 128);
   if (ws_bytes < w.bytes || (reinterpret_cast<uintptr_t>(ws) & 255) != 0) return MOVA_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (T > kSmallGroupT) {
+    cudaError_t err = launch_tile_hist(idx, MOVA_I32, nullptr, MOVA_F32, T, E, k, nullptr, nullptr,
+                                       w.tile_counts, w.sb, s);
+    if (err == cudaSuccess)
+      err = launch_tile_group(idx, T, E, k, w.tile_counts, counts, offsets, perm, pos, w.active, w.sb,
+                              false, s);
+    return from_cuda(err);
+  }
   return from_cuda(launch_permute(idx, MOVA_I32, nullptr, MOVA_F32, T * k, E, nullptr, nullptr,
-                                  counts, offsets, perm, pos, w.active, w.sb,
-                                  static_cast<cudaStream_t>(stream)));
+                                  counts, offsets, perm, pos, w.active, w.sb, s));
 }
 
 mova_status mova_value_ex(const void* x, mova_dtype x_dt, const void* idx, mova_dtype idx_dt,
@@ -185,14 +211,22 @@ mova_status mova_value_ex(const void* x, mova_dtype x_dt, const void* idx, mova_
   if (T == 0) return MOVA_OK;
   if (!x || !idx || !wgt || !Wv || !v || !ws) return MOVA_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(Wv) || !aligned16(v)) return MOVA_ERR_INVALID_ARG;
-  const Workspace w = layout(ws, T, k, n);
+  const Workspace w = layout(ws, T, d, k, n);
   if (ws_bytes < w.bytes || (reinterpret_cast<uintptr_t>(ws) & 255) != 0) return MOVA_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t err = mark(events, 0, s);
   if (err == cudaSuccess) err = mark(events, 1, s);
-  if (err == cudaSuccess)
-    err = launch_permute(idx, idx_dt, wgt, w_dt, T * k, E, w.idx, w.w, w.counts, w.offsets, w.perm,
-                         w.pos, w.active, w.sb, s);
+  if (err == cudaSuccess) {
+    if (T > kSmallGroupT) {
+      err = launch_tile_hist(idx, idx_dt, wgt, w_dt, T, E, k, w.idx, w.w, w.tile_counts, w.sb, s);
+      if (err == cudaSuccess)
+        err = launch_tile_group(w.idx, T, E, k, w.tile_counts, w.counts, w.offsets, w.perm, w.pos,
+                                w.active, w.sb, false, s);
+    } else {
+      err = launch_permute(idx, idx_dt, wgt, w_dt, T * k, E, w.idx, w.w, w.counts, w.offsets, w.perm,
+                           w.pos, w.active, w.sb, s);
+    }
+  }
   if (err == cudaSuccess) err = mark(events, 2, s);
   if (err != cudaSuccess) return from_cuda(err);
   return run_experts_and_combine(x, x_dt, Wv, w, w.idx, w.w, T, d, E, k, n, v, path, events, s);
@@ -220,7 +254,7 @@ mova_status mova_value_routed_ex(const void* x, mova_dtype x_dt, const float* Wr
   if (!x || !Wr || !br || !Wv || !v || !ws) return MOVA_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(Wr) || !aligned16(Wv) || !aligned16(v))
     return MOVA_ERR_INVALID_ARG;
-  const Workspace w = layout(ws, T, k, n);
+  const Workspace w = layout(ws, T, d, k, n);
   if (ws_bytes < w.bytes || (reinterpret_cast<uintptr_t>(ws) & 255) != 0) return MOVA_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   int32_t* idx = idx_out ? idx_out : w.idx;
@@ -228,12 +262,31 @@ mova_status mova_value_routed_ex(const void* x, mova_dtype x_dt, const float* Wr
   const GroupOut g{w.counts, w.offsets, w.perm, w.pos, w.active, w.sb};
   bool grouped = false;
   cudaError_t err = mark(events, 0, s);
-  if (err == cudaSuccess)
-    err = launch_router(x, x_dt, Wr, br, T, d, E, k, scale, idx, wgt, &g, &grouped, s);
+  // bf16 batches above the decode range route on the tensor cores and group
+  // with the tile kernels (the router writes the per-tile histograms).
+  const bool tc_router = x_dt == MOVA_BF16 && T > kTcRouterMinT;
+  if (err == cudaSuccess) {
+    if (tc_router)
+      err = launch_router_tc(x, Wr, br, T, d, E, k, scale, idx, wgt, w.tile_counts, w.planes, w.sb, s);
+    else
+      err = launch_router(x, x_dt, Wr, br, T, d, E, k, scale, idx, wgt, &g, &grouped, s);
+  }
   if (err == cudaSuccess) err = mark(events, 1, s);
-  if (err == cudaSuccess && !grouped)
-    err = launch_permute(idx, MOVA_I32, nullptr, MOVA_F32, T * k, E, nullptr, nullptr, w.counts,
-                         w.offsets, w.perm, w.pos, w.active, w.sb, s);
+  if (err == cudaSuccess && !grouped) {
+    if (tc_router) {
+      err = launch_tile_group(idx, T, E, k, w.tile_counts, w.counts, w.offsets, w.perm, w.pos, w.active,
+                              w.sb, true, s);
+    } else if (T > kSmallGroupT) {
+      err = launch_tile_hist(idx, MOVA_I32, nullptr, MOVA_F32, T, E, k, nullptr, nullptr, w.tile_counts,
+                             w.sb, s);
+      if (err == cudaSuccess)
+        err = launch_tile_group(idx, T, E, k, w.tile_counts, w.counts, w.offsets, w.perm, w.pos,
+                                w.active, w.sb, false, s);
+    } else {
+      err = launch_permute(idx, MOVA_I32, nullptr, MOVA_F32, T * k, E, nullptr, nullptr, w.counts,
+                           w.offsets, w.perm, w.pos, w.active, w.sb, s);
+    }
+  }
   if (err == cudaSuccess) err = mark(events, 2, s);
   if (err != cudaSuccess) return from_cuda(err);
   return run_experts_and_combine(x, x_dt, Wv, w, idx, wgt, T, d, E, k, n, v, path, events, s);

@@ -145,6 +145,158 @@ cudaError_t launch_t(const void* idx_in, const void* w_in, int N, int E, int32_t
   return cudaGetLastError();
 }
 
+// ---------------------------------------------------------------------------
+// Multi-CTA grouping for large batches: per-tile histograms, one scan, a
+// stable scatter per tile.  A tile is 128 tokens (128 * k pairs, in pair
+// order), so the tile order is the pair order and the result is the same
+// stable sort as above.
+// ---------------------------------------------------------------------------
+
+constexpr int kTileTok = 128;
+
+// Histogram of each tile's pairs; in routing-given mode also the int32 / fp32
+// copies of the routing and the range check.
+template <typename IT, typename WT>
+__global__ void __launch_bounds__(256)
+tile_hist_kernel(const IT* __restrict__ idx_in, const WT* __restrict__ w_in, int N, int E, int k,
+                 int32_t* __restrict__ idx32, float* __restrict__ w32,
+                 int32_t* __restrict__ tile_counts, StatusBlock* sb) {
+  __shared__ int hist[64];
+  if (threadIdx.x < 64) hist[threadIdx.x] = 0;
+  __syncthreads();
+  const int per = kTileTok * k;
+  const int f0 = blockIdx.x * per;
+  const int f1 = min(N, f0 + per);
+  for (int f = f0 + threadIdx.x; f < f1; f += blockDim.x) {
+    int e = static_cast<int>(idx_in[f]);
+    if (e < 0 || e >= E) {
+      raise_status(sb, MOVA_ERR_DEVICE_CHECK, f);
+      e = 0;
+    }
+    if (idx32 != nullptr) idx32[f] = e;
+    if (w32 != nullptr) w32[f] = to_f32(w_in[f]);
+    atomicAdd(&hist[e], 1);
+  }
+  __syncthreads();
+  if (threadIdx.x < 64) tile_counts[blockIdx.x * 64 + threadIdx.x] = hist[threadIdx.x];
+}
+
+// One CTA: tile_counts[t][e] becomes the first grouped position of tile t's
+// pairs of expert e; writes counts, offsets, the active list and resets the
+// status block for this call.
+__global__ void __launch_bounds__(64)
+tile_scan_kernel(int32_t* __restrict__ tile_counts, int ntiles, int E, int32_t* __restrict__ counts,
+                 int32_t* __restrict__ offsets, int32_t* __restrict__ active, StatusBlock* sb,
+                 int N, bool reset_status) {
+  pdl_wait();
+  __shared__ int tot[64];
+  __shared__ int off[65];
+  const int e = threadIdx.x;
+  int s = 0;
+  if (e < E)
+    for (int t = 0; t < ntiles; ++t) s += tile_counts[t * 64 + e];
+  tot[e] = (e < E) ? s : 0;
+  __syncthreads();
+  if (e == 0) {
+    int acc = 0;
+    for (int q = 0; q < E; ++q) {
+      off[q] = acc;
+      acc += tot[q];
+    }
+    off[E] = acc;
+  }
+  __syncthreads();
+  if (e < E) {
+    int base = off[e];
+    for (int t = 0; t < ntiles; ++t) {
+      const int c = tile_counts[t * 64 + e];
+      tile_counts[t * 64 + e] = base;
+      base += c;
+    }
+    counts[e] = tot[e];
+    offsets[e] = off[e];
+  }
+  if (e == 0) offsets[E] = off[E];
+  const int lane = e & 31;
+  const unsigned lt = (1u << lane) - 1u;
+  const bool a = e < E && tot[e] > 0;
+  __shared__ unsigned m[2];
+  const unsigned mm = __ballot_sync(0xffffffffu, a);
+  if (lane == 0) m[e >> 5] = mm;
+  __syncthreads();
+  const int before = (e >= 32) ? __popc(m[0]) : 0;
+  if (a) active[before + __popc(mm & lt)] = e;
+  if (e == 0) {
+    if (reset_status) {
+      sb->code = 0;
+      sb->detail = 0;
+    }
+    sb->num_active = __popc(m[0]) + __popc(m[1]);
+    sb->work_next = 0;
+  }
+  (void)N;
+}
+
+// Stable scatter of one tile: 4 warps own consecutive segments of the tile's
+// pairs; per-warp histograms are scanned in warp order on top of the tile's
+// first positions, then each warp ranks 32 pairs at a time (earlier lanes with
+// the same expert come first).
+__global__ void __launch_bounds__(128)
+tile_scatter_kernel(const int32_t* __restrict__ idx32, int N, int k,
+                    const int32_t* __restrict__ tile_base, int32_t* __restrict__ perm,
+                    int32_t* __restrict__ pos) {
+  pdl_wait();
+  __shared__ int hist[4][64];
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  for (int i = threadIdx.x; i < 4 * 64; i += 128) (&hist[0][0])[i] = 0;
+  __syncthreads();
+  const int per = kTileTok * k;
+  const int t0 = blockIdx.x * per;
+  const int t1 = min(N, t0 + per);
+  const int seg = (per + 3) / 4;
+  const int f_begin = min(t1, t0 + warp * seg);
+  const int f_end = min(t1, f_begin + seg);
+  for (int f = f_begin + lane; f < f_end; f += 32) atomicAdd(&hist[warp][idx32[f]], 1);
+  __syncthreads();
+  if (threadIdx.x < 64) {
+    int b = tile_base[blockIdx.x * 64 + threadIdx.x];
+    for (int w = 0; w < 4; ++w) {
+      const int c = hist[w][threadIdx.x];
+      hist[w][threadIdx.x] = b;
+      b += c;
+    }
+  }
+  __syncthreads();
+  const unsigned lt_mask = (1u << lane) - 1u;
+  for (int c0 = f_begin; c0 < f_end; c0 += 32) {
+    const int f = c0 + lane;
+    const bool valid = f < f_end;
+    const int e = valid ? idx32[f] : 0;
+    const unsigned grp = __match_any_sync(0xffffffffu, valid ? e : 256 + lane);
+    const int rank = __popc(grp & lt_mask);
+    const int size = __popc(grp);
+    if (valid) {
+      const int p = hist[warp][e] + rank;
+      perm[p] = f;
+      pos[f] = p;
+    }
+    __syncwarp();
+    if (valid && rank == size - 1) hist[warp][e] += size;
+    __syncwarp();
+  }
+}
+
+template <typename IT, typename WT>
+cudaError_t launch_hist_t(const void* idx_in, const void* w_in, int N, int E, int k, int32_t* idx32,
+                          float* w32, int32_t* tile_counts, StatusBlock* sb, cudaStream_t stream) {
+  const int ntiles = (N + kTileTok * k - 1) / (kTileTok * k);
+  tile_hist_kernel<IT, WT><<<ntiles, 256, 0, stream>>>(static_cast<const IT*>(idx_in),
+                                                       static_cast<const WT*>(w_in), N, E, k, idx32,
+                                                       w32, tile_counts, sb);
+  return cudaGetLastError();
+}
+
 }  // namespace
 
 cudaError_t launch_permute(const void* idx_in, mova_dtype idx_dt, const void* w_in,
@@ -165,6 +317,44 @@ cudaError_t launch_permute(const void* idx_in, mova_dtype idx_dt, const void* w_
                                      active, sb, stream);
   return launch_t<int32_t, float>(idx_in, w_in, N, E, idx32, w32, counts, offsets, perm, pos,
                                   active, sb, stream);
+}
+
+}  // namespace mova
+
+namespace mova {
+
+int group_tiles(int T) { return (T + kTileTok - 1) / kTileTok; }
+
+cudaError_t launch_tile_hist(const void* idx_in, mova_dtype idx_dt, const void* w_in,
+                             mova_dtype w_dt, int T, int E, int k, int32_t* idx32, float* w32,
+                             int32_t* tile_counts, StatusBlock* sb, cudaStream_t stream) {
+  const int N = T * k;
+  if (w_in == nullptr) w32 = nullptr;
+  // The status word is reset by the first kernel of the call that may raise it.
+  cudaError_t err = cudaMemsetAsync(sb, 0, 8, stream);
+  if (err != cudaSuccess) return err;
+  if (idx_dt == MOVA_I8) {
+    return w_dt == MOVA_F16
+               ? launch_hist_t<int8_t, __half>(idx_in, w_in, N, E, k, idx32, w32, tile_counts, sb, stream)
+               : launch_hist_t<int8_t, float>(idx_in, w_in, N, E, k, idx32, w32, tile_counts, sb, stream);
+  }
+  return w_dt == MOVA_F16
+             ? launch_hist_t<int32_t, __half>(idx_in, w_in, N, E, k, idx32, w32, tile_counts, sb, stream)
+             : launch_hist_t<int32_t, float>(idx_in, w_in, N, E, k, idx32, w32, tile_counts, sb, stream);
+}
+
+cudaError_t launch_tile_group(const int32_t* idx32, int T, int E, int k, int32_t* tile_counts,
+                              int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* pos,
+                              int32_t* active, StatusBlock* sb, bool reset_status,
+                              cudaStream_t stream) {
+  const int N = T * k;
+  const int ntiles = group_tiles(T);
+  cudaError_t err = launch_pdl(tile_scan_kernel, dim3(1), dim3(64), 0, stream, tile_counts, ntiles,
+                               E, counts, offsets, active, sb, N, reset_status);
+  if (err != cudaSuccess) return err;
+  return launch_pdl(tile_scatter_kernel, dim3(ntiles), dim3(128), 0, stream,
+                    static_cast<const int32_t*>(idx32), N, k,
+                    static_cast<const int32_t*>(tile_counts), perm, pos);
 }
 
 }  // namespace mova

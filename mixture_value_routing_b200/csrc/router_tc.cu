@@ -1,0 +1,269 @@
+// Tensor-core router for large bf16 batches.
+//
+// "MoVA: routing the value vectors, and why the KV cache does not notice",
+// section "Where the routing happens": logits = x Wr^T (no bias), sigmoid
+// gate, the bias steers a top-k selection, the k scores are renormalised and
+// scaled.  At prefill sizes the logits are a dense T x 2560 x 64 contraction,
+// so they run on tcgen05 tensor cores with fp32 accumulation:
+//
+//   * x is bf16, so every product x_j * Wr[e, j] is formed exactly if Wr is
+//     bf16 too.  The fp32 router weight is therefore split exactly into three
+//     bf16 planes, Wr = hi + mid + lo (8 + 8 + 8 significand bits cover fp32's
+//     24; each plane is the round-to-nearest bf16 of what the previous ones
+//     left), and the router runs as one GEMM against the 3E = 192 plane rows.
+//     logits[e] = (acc_hi[e] + acc_mid[e]) + acc_lo[e]: the same products as
+//     an fp32 dot product, accumulated in fp32 in another order.
+//   * One CTA per 128 tokens: a TMA warp streams 128 x 64 token tiles and
+//     192 x 64 plane tiles (128-byte swizzle) through 4 stages; one thread
+//     issues tcgen05.mma (M = 128, N = 192, K = 16) into tensor memory; four
+//     epilogue warps read one token per thread (all 192 columns), form the
+//     64 logits, the sigmoid scores and the biased selection in registers and
+//     write idx / w, plus the tile's expert histogram for the grouping.
+// Every wait is bounded (MOVA_ERR_TIMEOUT, then drain and free).
+#include <cuda.h>
+
+#include "common.cuh"
+#include "internal.h"
+#include "sm100.cuh"
+
+namespace mova {
+
+namespace {
+
+constexpr int RM = 128;  // tokens per CTA
+constexpr int RN = 192;  // 3 planes x 64 experts
+constexpr int RK = 64;
+constexpr int kRStages = 4;
+constexpr int kRABytes = RM * RK * 2;
+constexpr int kRBBytes = RN * RK * 2;
+constexpr int kRStageBytes = kRABytes + kRBBytes;
+constexpr int kRThreads = 6 * 32;  // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
+constexpr uint32_t kRTmemCols = 256;
+
+struct __align__(1024) RSmem {
+  uint8_t stage[kRStages][kRStageBytes];
+  uint64_t full[kRStages];
+  uint64_t empty[kRStages];
+  uint64_t tmem_full;
+  uint32_t tmem_base;
+  int abort;
+  int hist[64];
+  float br[64];
+};
+
+// Exact split of an fp32 value into three bf16 values summing to it.
+__global__ void __launch_bounds__(256)
+split_router_kernel(const float* __restrict__ Wr, int E, int d, __nv_bfloat16* __restrict__ W3) {
+  const long long total = 64LL * d;
+  for (long long i = blockIdx.x * 256LL + threadIdx.x; i < total; i += 256LL * gridDim.x) {
+    const int e = static_cast<int>(i / d);
+    const int j = static_cast<int>(i - static_cast<long long>(e) * d);
+    float v = (e < E) ? Wr[i] : 0.f;
+    const __nv_bfloat16 hi = __float2bfloat16_rn(v);
+    v -= __bfloat162float(hi);
+    const __nv_bfloat16 mid = __float2bfloat16_rn(v);
+    v -= __bfloat162float(mid);
+    const __nv_bfloat16 lo = __float2bfloat16_rn(v);
+    W3[static_cast<size_t>(e) * d + j] = hi;
+    W3[static_cast<size_t>(64 + e) * d + j] = mid;
+    W3[static_cast<size_t>(128 + e) * d + j] = lo;
+  }
+}
+
+__global__ void __launch_bounds__(kRThreads, 1)
+router_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
+                 const float* __restrict__ br, int T, int d, int E, int k, float scale,
+                 int32_t* __restrict__ idx_out, float* __restrict__ w_out,
+                 int32_t* __restrict__ tile_counts, StatusBlock* __restrict__ sb) {
+  extern __shared__ uint8_t smem_raw[];
+  RSmem& S = *reinterpret_cast<RSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int nk = d / RK;
+  const int t0 = blockIdx.x * RM;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kRStages; ++s) {
+      mbar_init(&S.full[s], 1);
+      mbar_init(&S.empty[s], 1);
+    }
+    mbar_init(&S.tmem_full, 1);
+    S.abort = 0;
+    fence_barrier_init();
+  }
+  if (threadIdx.x < 64) {
+    S.hist[threadIdx.x] = 0;
+    S.br[threadIdx.x] = (threadIdx.x < E) ? br[threadIdx.x] : 0.f;
+  }
+  if (warp == 1) {
+    tmem_alloc(&S.tmem_base, kRTmemCols);
+    tmem_relinquish();
+  }
+  pdl_wait();  // the plane split of this call is complete
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+
+  if (warp == 0) {
+    if (lane == 0) {
+      for (int kb = 0; kb < nk; ++kb) {
+        const int s = kb % kRStages;
+        if (kb >= kRStages && !mbar_wait(&S.empty[s], ((kb / kRStages) - 1) & 1)) {
+          raise_status(sb, MOVA_ERR_TIMEOUT, blockIdx.x);
+          S.abort = 1;
+          break;
+        }
+        mbar_arrive_expect_tx(&S.full[s], kRStageBytes);
+        tma_load_2d_nohint(S.stage[s], &tmap_x, kb * RK, t0, &S.full[s]);
+        tma_load_2d_nohint(S.stage[s] + kRABytes, &tmap_w, kb * RK, 0, &S.full[s]);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16_f32(RM, RN);
+      bool ok = true;
+      for (int kb = 0; kb < nk; ++kb) {
+        const int s = kb % kRStages;
+        if (!mbar_wait(&S.full[s], (kb / kRStages) & 1)) {
+          raise_status(sb, MOVA_ERR_TIMEOUT, blockIdx.x);
+          S.abort = 1;
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t a0 = smem_u32(S.stage[s]);
+        const uint32_t b0 = a0 + kRABytes;
+#pragma unroll
+        for (int k16 = 0; k16 < RK / 16; ++k16)
+          tc_mma_bf16(S.tmem_base, smem_desc_sw128(a0 + k16 * 32), smem_desc_sw128(b0 + k16 * 32), idesc,
+                      (kb | k16) != 0);
+        tc_commit(&S.empty[s]);
+      }
+      if (ok) tc_commit(&S.tmem_full);
+    }
+  } else {
+    // Epilogue: thread = token (TMEM lane).
+    const int lg = warp & 3;
+    const int t = t0 + lg * 32 + lane;
+    if (mbar_wait(&S.tmem_full, 0)) {
+      tc_fence_after();
+      const uint32_t tb = S.tmem_base + (static_cast<uint32_t>(lg * 32) << 16);
+      float logit[64];
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        uint32_t hi[32], mid[32], lo[32];
+        tmem_ld_32(tb + c * 32, hi);
+        tmem_ld_32(tb + 64 + c * 32, mid);
+        tmem_ld_32(tb + 128 + c * 32, lo);
+        tmem_ld_wait();
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          logit[c * 32 + j] = (__uint_as_float(hi[j]) + __uint_as_float(mid[j])) + __uint_as_float(lo[j]);
+      }
+      tc_fence_before();
+      if (t < T) {
+        // Sigmoid scores (in place); the biased score s + br steers the
+        // selection only, NaN never wins.
+#pragma unroll
+        for (int e = 0; e < 64; ++e) logit[e] = sigmoidf_(logit[e]);
+        uint64_t taken = 0;
+        float ssum = 0.f;
+        int sel[8];
+        float ssel[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          if (j < k) {
+            // Highest biased score among live experts; ties to the lower
+            // index (strict comparison in ascending expert order).
+            int be = -1;
+            float bb = 0.f, bsv = 0.f;
+#pragma unroll
+            for (int e = 0; e < 64; ++e) {
+              float b = logit[e] + S.br[e];
+              if (!(b == b)) b = -INFINITY;
+              const bool live = e < E && !((taken >> e) & 1ull);
+              if (live && (be < 0 || b > bb)) {
+                be = e;
+                bb = b;
+                bsv = logit[e];
+              }
+            }
+            taken |= 1ull << be;
+            sel[j] = be;
+            ssel[j] = bsv;
+            ssum += bsv;
+          }
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          if (j < k) {
+            idx_out[static_cast<size_t>(t) * k + j] = sel[j];
+            w_out[static_cast<size_t>(t) * k + j] = scale * ssel[j] / ssum;
+            atomicAdd(&S.hist[sel[j]], 1);
+          }
+        }
+      }
+    } else {
+      raise_status(sb, MOVA_ERR_TIMEOUT, blockIdx.x);
+      S.abort = 1;
+    }
+  }
+  __syncthreads();
+  if (tile_counts != nullptr && threadIdx.x < 64)
+    tile_counts[blockIdx.x * 64 + threadIdx.x] = S.hist[threadIdx.x];
+  if (S.abort && threadIdx.x == 0) {
+    for (int s = 0; s < kRStages; ++s) {
+      mbar_wait(&S.full[s], 0);
+      mbar_wait(&S.empty[s], 0);
+    }
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(S.tmem_base, kRTmemCols);
+  }
+}
+
+using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                 const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                 const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                 CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+}  // namespace
+
+size_t router_planes_bytes(int d) { return static_cast<size_t>(RN) * d * 2; }
+
+cudaError_t launch_router_tc(const void* x, const float* Wr, const float* br, int T, int d, int E,
+                             int k, float scale, int32_t* idx, float* w, int32_t* tile_counts,
+                             __nv_bfloat16* planes, StatusBlock* sb, cudaStream_t stream) {
+  void* fp = encode_tiled_fn();
+  if (fp == nullptr) return cudaErrorNotSupported;
+  EncodeTiled enc = reinterpret_cast<EncodeTiled>(fp);
+  split_router_kernel<<<2 * sm_count(), 256, 0, stream>>>(Wr, E, d, planes);
+  cudaError_t err = cudaGetLastError();
+  if (err != cudaSuccess) return err;
+  CUtensorMap tx, tw;
+  const cuuint64_t xdim[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(T)};
+  const cuuint64_t wdim[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(RN)};
+  const cuuint64_t stride[1] = {static_cast<cuuint64_t>(d) * 2};
+  const cuuint32_t xbox[2] = {RK, RM};
+  const cuuint32_t wbox[2] = {RK, RN};
+  const cuuint32_t es[2] = {1, 1};
+  if (enc(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(x), xdim, stride, xbox, es,
+          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
+  if (enc(&tw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, planes, wdim, stride, wbox, es,
+          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
+  const size_t smem = sizeof(RSmem) + 1024;
+  err = cudaFuncSetAttribute(router_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem));
+  if (err != cudaSuccess) return err;
+  const int grid = (T + RM - 1) / RM;
+  return launch_pdl(router_tc_kernel, dim3(grid), dim3(kRThreads), smem, stream, tx, tw, br, T, d, E,
+                    k, scale, idx, w, tile_counts, sb);
+}
+
+}  // namespace mova

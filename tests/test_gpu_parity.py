@@ -267,6 +267,14 @@ def test_tensor_deterministic(api):
         assert torch.equal(api.value_routed(*args, path="tensor"), first)
 
 
+@pytest.mark.parametrize("T,d,E,k", [(65, 2560, 64, 4), (130, 512, 17, 3), (777, 256, 64, 8)])
+def test_tensor_router_and_tile_grouping(api, T, d, E, k):
+    """bf16 batches above 64 tokens route on the tensor cores (exact three-way
+    bf16 split of the fp32 router) and group with the tile kernels; the
+    expert step is forced onto the streaming kernel to isolate them."""
+    _full(api, T, d, E, k, 256, "bf16", seed=T, path="stream")
+
+
 def test_full_zero_tokens(api):
     lay = _layer(0, 256, 8, 128, "bf16")
     x = torch.empty((0, 256), dtype=torch.bfloat16, device="cuda")
