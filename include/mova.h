@@ -166,6 +166,38 @@ mova_status mova_get_status(void* ws, int32_t* detail_out, void* stream);
 /* The path AUTO would pick for these sizes and dtype (for tests/benches). */
 mova_path mova_auto_path(int T, mova_dtype x_dt);
 
+/* Size of the workspace array built into the library for
+ * mova_value_routed_noalloc. */
+#define MOVA_NOALLOC_SCRATCH_BYTES (2u << 20)
+
+/* mova_value_routed without a caller-provided workspace, for callers that
+ * cannot allocate device memory where they run the value projection: code
+ * inside a stream capture that must not add allocation nodes, programs whose
+ * memory pool owns all of the device memory, or plug-ins that are handed only
+ * the tensors they compute on.  (The MoVA pages have no counterpart: this is
+ * a deployment convenience, not part of the method.)
+ *
+ * Arguments, layouts, results and errors are those of mova_value_routed
+ * (automatic kernel choice, no routing copies).  The workspace is a
+ * MOVA_NOALLOC_SCRATCH_BYTES array compiled into the library; every GPU that
+ * loads the library holds it until the process exits.  Nothing is allocated
+ * or freed: no cudaMalloc, cudaFree or allocating library routine is called.
+ *  - Sizes whose mova_workspace_size exceeds MOVA_NOALLOC_SCRATCH_BYTES are
+ *    rejected with MOVA_ERR_UNSUPPORTED (and a message on stderr); at
+ *    d = 2560, E = 64, k = 4, n = 1024 that admits batches up to T = 67.
+ *  - The first call on each device looks up the array's device address
+ *    (cudaGetSymbolAddress, with that device current); make that first call
+ *    before any stream capture.
+ *  - All calls share the one array and it keeps the last call's contents;
+ *    each call's first kernel resets the status fields it relies on, and
+ *    every other part is fully rewritten.  Calls that overlap on the GPU
+ *    (different streams, or other devices' work is unaffected) race: order
+ *    them on one stream.  The device status word is not exposed. */
+mova_status mova_value_routed_noalloc(const void* x, mova_dtype x_dt, const float* Wr,
+                                      const float* br, const void* Wv, mova_dtype wv_dt,
+                                      int T, int d, int E, int k, int n, float scale, void* v,
+                                      void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -43,6 +43,8 @@ SIGNATURES = {
     "mova_value_routed_ex": (_i, [_vp, _i, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _vp, _vp,
                                   _vp, _vp, _sz, _i, _vp, _vp]),
     "mova_get_status": (_i, [_vp, _vp, _vp]),
+    "mova_value_routed_noalloc": (_i, [_vp, _i, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _vp,
+                                       _vp]),
 }
 
 _lib = None
