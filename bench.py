@@ -87,6 +87,16 @@ def init_dist(world, backend):
     return world > 1
 
 
+def rank_batch_seed(seed, rank):
+    """Each rank draws its own tokens; every rank holds the same layer weights."""
+    return seed + 7919 * rank
+
+
+def job_value(world, tokens_per_rank_step, steps, ms_max):
+    """Whole-job throughput: all ranks' tokens over the slowest rank's time."""
+    return world * tokens_per_rank_step * steps / (ms_max / 1e3)
+
+
 def barrier(on):
     if on:
         import torch.distributed as dist
@@ -254,7 +264,8 @@ def run_mova(a):
                        dev_of(lay.Wv, wdt, device)))
         del lay
     # One batch per layer position; every rank has its own tokens.
-    batches = [MI.make_batch(T, a.seed + 7919 * rank, step=l, dtype=dtype, mode=mode) for l in range(L)]
+    batches = [MI.make_batch(T, rank_batch_seed(a.seed, rank), step=l, dtype=dtype, mode=mode)
+               for l in range(L)]
     xs = [dev_of(b.x, dtype, device) for b in batches]
     routing = None
     if mode == "given":
@@ -345,7 +356,7 @@ def run_mova(a):
 
     peaks, peak_src = load_peaks()
     ms_per_step = ms / K
-    value = world * T * K / (ms / 1e3)
+    value = job_value(world, T, K, ms)
 
     # Roofline of the dominant kernel (the expert kernel at these sizes).
     xs_b = 2 if dtype == "bf16" else 4
@@ -411,7 +422,7 @@ def run_mova(a):
         torch.cuda.synchronize()
         barrier(dist_on)
         ems = allmax(e0.elapsed_time(e1), dist_on, device)
-        e2e = {"value": round(world * T * Ke / (ems / 1e3), 1), "unit": "tokens/s",
+        e2e = {"value": round(job_value(world, T, Ke, ems), 1), "unit": "tokens/s",
                "h2d_bytes_per_step": int(xs[0].numel() * xs[0].element_size()),
                "d2h_bytes_per_step": int(vh.numel() * vh.element_size()), "steps": Ke,
                "ms_per_step": round(ems / Ke, 5)}

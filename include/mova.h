@@ -163,6 +163,14 @@ mova_status mova_value_routed_ex(const void* x, mova_dtype x_dt, const float* Wr
  * pair index of a bad expert index). */
 mova_status mova_get_status(void* ws, int32_t* detail_out, void* stream);
 
+/* Self-test of the device-side failure detection: launches one thread that
+ * waits on a barrier nothing arrives at, with the same bounded wait every
+ * pipeline kernel uses but a limit of `limit_cycles` clock cycles (at most
+ * about one second's worth); it then records MOVA_ERR_TIMEOUT in the status
+ * word of `ws` (256 bytes suffice), readable with mova_get_status.  The
+ * context stays usable afterwards.  Not part of the method. */
+mova_status mova_selftest_wait_timeout(void* ws, long long limit_cycles, void* stream);
+
 /* The path AUTO would pick for these sizes and dtype (for tests/benches). */
 mova_path mova_auto_path(int T, mova_dtype x_dt);
 

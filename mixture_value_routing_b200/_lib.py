@@ -43,6 +43,7 @@ SIGNATURES = {
     "mova_value_routed_ex": (_i, [_vp, _i, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _vp, _vp,
                                   _vp, _vp, _sz, _i, _vp, _vp]),
     "mova_get_status": (_i, [_vp, _vp, _vp]),
+    "mova_selftest_wait_timeout": (_i, [_vp, ctypes.c_longlong, _vp]),
     "mova_value_routed_noalloc": (_i, [_vp, _i, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _vp,
                                        _vp]),
 }

@@ -12,6 +12,7 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "sm100.cuh"
 
 namespace mova {
 
@@ -132,6 +133,20 @@ mova_status run_experts_and_combine(const void* x, mova_dtype dt, const void* Wv
   if (err == cudaSuccess) err = launch_combine(ws.P, tensor, ws.pos, w32, T, k, n, v, dt, stream);
   if (err == cudaSuccess) err = mark(events, 4, stream);
   return from_cuda(err);
+}
+
+// Self-test of the bounded waits: one thread waits on an mbarrier that
+// nothing will ever arrive at, gives up after `limit` cycles and reports
+// MOVA_ERR_TIMEOUT in the status block, as every pipeline wait does.
+__global__ void selftest_wait_kernel(StatusBlock* sb, long long limit) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    sb->code = 0;
+    sb->detail = 0;
+    mbar_init(&bar, 1);
+    fence_barrier_init();
+    if (!mbar_wait_for(&bar, 0, limit)) raise_status(sb, MOVA_ERR_TIMEOUT, 1);
+  }
 }
 
 }  // namespace
@@ -298,6 +313,13 @@ mova_status mova_value_routed(const void* x, mova_dtype x_dt, const float* Wr, c
                               size_t ws_bytes, void* stream) {
   return mova_value_routed_ex(x, x_dt, Wr, br, Wv, wv_dt, T, d, E, k, n, scale, v, idx_out, w_out,
                               ws, ws_bytes, MOVA_PATH_AUTO, nullptr, stream);
+}
+
+mova_status mova_selftest_wait_timeout(void* ws, long long limit_cycles, void* stream) {
+  if (!ws || limit_cycles <= 0 || limit_cycles > kWaitLimitCycles) return MOVA_ERR_INVALID_ARG;
+  selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<StatusBlock*>(ws), limit_cycles);
+  return from_cuda(cudaGetLastError());
 }
 
 mova_status mova_get_status(void* ws, int32_t* detail_out, void* stream) {

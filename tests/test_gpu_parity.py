@@ -1,5 +1,7 @@
 """GPU parity: the CUDA path (through the C ABI) against the fp64 oracle on the
 same seeded inputs.  Comparison rules are in tests/_parity.py."""
+import ctypes
+
 import numpy as np
 import pytest
 import torch
@@ -273,6 +275,19 @@ def test_tensor_router_and_tile_grouping(api, T, d, E, k):
     bf16 split of the fp32 router) and group with the tile kernels; the
     expert step is forced onto the streaming kernel to isolate them."""
     _full(api, T, d, E, k, 256, "bf16", seed=T, path="stream")
+
+
+def test_bounded_wait_reports_timeout(api):
+    """A device wait that can never complete gives up after its limit and
+    reports MOVA_ERR_TIMEOUT; the context stays usable for a normal call."""
+    from mixture_value_routing_b200 import _lib
+    ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    lib = _lib.load()
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    assert lib.mova_selftest_wait_timeout(ctypes.c_void_p(ws.data_ptr()), 2_000_000, stream) == _lib.OK
+    status, _ = api.get_status(ws)
+    assert status == "MOVA_ERR_TIMEOUT"
+    _full(api, 8, 256, 8, 2, 128, "bf16", seed=77)
 
 
 def test_full_zero_tokens(api):
