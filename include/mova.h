@@ -70,13 +70,15 @@ typedef enum {
 } mova_dtype;
 
 /* Which expert kernel runs.  AUTO picks the weight-streaming kernel for
- * small token counts (and for fp32) and the tcgen05 grouped GEMM for bf16
- * batches above a threshold.  STREAM and TENSOR force one (TENSOR requires
- * bf16; otherwise MOVA_ERR_UNSUPPORTED). */
+ * small token counts (and for fp32) and the tcgen05 grouped GEMM on SM pairs
+ * for bf16 batches above a threshold.  STREAM and TENSOR force one;
+ * TENSOR_1CTA forces the single-CTA variant of the grouped GEMM (TENSOR*
+ * require bf16; otherwise MOVA_ERR_UNSUPPORTED). */
 typedef enum {
   MOVA_PATH_AUTO = 0,
   MOVA_PATH_STREAM = 1,
-  MOVA_PATH_TENSOR = 2
+  MOVA_PATH_TENSOR = 2,
+  MOVA_PATH_TENSOR_1CTA = 3
 } mova_path;
 
 /* Human-readable name of a status code (static storage, never NULL). */
@@ -192,7 +194,7 @@ mova_path mova_auto_path(int T, mova_dtype x_dt);
  * or freed: no cudaMalloc, cudaFree or allocating library routine is called.
  *  - Sizes whose mova_workspace_size exceeds MOVA_NOALLOC_SCRATCH_BYTES are
  *    rejected with MOVA_ERR_UNSUPPORTED (and a message on stderr); at
- *    d = 2560, E = 64, k = 4, n = 1024 that admits batches up to T = 67.
+ *    d = 2560, E = 64, k = 4, n = 1024 that admits batches up to T = 30.
  *  - The first call on each device looks up the array's device address
  *    (cudaGetSymbolAddress, with that device current); make that first call
  *    before any stream capture.

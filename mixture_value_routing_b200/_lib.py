@@ -19,7 +19,7 @@ STATUS_NAMES = {OK: "MOVA_OK", ERR_INVALID_ARG: "MOVA_ERR_INVALID_ARG",
 # mova_dtype
 F32, BF16, F16, I32, I8 = range(5)
 # mova_path
-PATH_AUTO, PATH_STREAM, PATH_TENSOR = range(3)
+PATH_AUTO, PATH_STREAM, PATH_TENSOR, PATH_TENSOR_1CTA = range(4)
 # stage events recorded by the _ex entry points
 STAGE_EVENTS = 5
 STAGES = ("route", "group", "experts", "combine")

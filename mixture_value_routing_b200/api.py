@@ -19,7 +19,8 @@ from . import _lib
 
 _DT = {torch.float32: _lib.F32, torch.bfloat16: _lib.BF16, torch.float16: _lib.F16,
        torch.int32: _lib.I32, torch.int8: _lib.I8}
-_PATH = {"auto": _lib.PATH_AUTO, "stream": _lib.PATH_STREAM, "tensor": _lib.PATH_TENSOR}
+_PATH = {"auto": _lib.PATH_AUTO, "stream": _lib.PATH_STREAM, "tensor": _lib.PATH_TENSOR,
+         "tensor_1cta": _lib.PATH_TENSOR_1CTA}
 
 
 def _ptr(t: Optional[torch.Tensor]):

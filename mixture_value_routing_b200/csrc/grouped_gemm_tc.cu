@@ -13,16 +13,20 @@
 // near-equal token tiles, each combined with the n/128 weight-row tiles, so
 // tail waste is below 16 columns per tile.
 //
-// One persistent CTA per SM, warp-specialised:
-//   warp 0      TMA producer: weight tile (128 x 64) by a 2-D tensor-map load
-//               with 128-byte swizzle;
-//   warps 1-4   gather producers: the tile's token rows of x (rows chosen by
-//               the grouping), 16-byte cp.async into the same swizzled K-major
-//               layout, completing on the stage's mbarrier;
-//   warp 5      MMA issuer (one thread): 4 x tcgen05.mma (K = 16) per stage
+// First, gather_pairs_kernel copies each pair's x row into grouped order
+// (xp[p] = x[token of pair p]), one bandwidth-bound pass, so that every
+// token tile of the GEMM is a run of consecutive rows that TMA loads as
+// plain 2-D boxes (token rows are read n/128 times, from L2, by TMA instead
+// of 16-byte gathers through the load/store units).
+//
+// Then one persistent CTA per SM, warp-specialised:
+//   warp 0      TMA producer: per 64-wide K step the weight tile (128 rows) and
+//               the token tile (up to 256 rows of xp, in boxes of 32 rows),
+//               both with 128-byte swizzle, completing on the stage mbarrier;
+//   warp 1      MMA issuer (one thread): 4 x tcgen05.mma (K = 16) per stage
 //               into a tensor-memory accumulator; tcgen05.commit frees the
 //               stage and, per tile, hands the accumulator to the epilogue;
-//   warps 6-9   epilogue: tcgen05.ld of their 32 TMEM lanes, SiLU, bf16
+//   warps 2-5   epilogue: tcgen05.ld of their 32 TMEM lanes, SiLU, bf16
 //               round, store.
 // Shared memory holds 4 stages of 48 KB; tensor memory holds two 256-column
 // fp32 accumulators, so the epilogue of one tile overlaps the MMAs of the
@@ -48,13 +52,12 @@ constexpr int kStages = 4;
 constexpr int kABytes = BM * BK * 2;
 constexpr int kBBytes = BN * BK * 2;
 constexpr int kStageBytes = kABytes + kBBytes;
+constexpr int kBoxRows = 32;  // token rows per TMA box
 constexpr int kWarpTma = 0;
-constexpr int kWarpGather0 = 1;
-constexpr int kGatherThreads = 128;
-constexpr int kWarpMma = 5;
-constexpr int kWarpEpi0 = 6;
+constexpr int kWarpMma = 1;
+constexpr int kWarpEpi0 = 2;
 constexpr int kEpiThreads = 128;
-constexpr int kThreads = 10 * 32;
+constexpr int kThreads = 6 * 32;
 constexpr uint32_t kTmemCols = 512;
 
 struct __align__(1024) Smem {
@@ -72,7 +75,6 @@ struct __align__(1024) Smem {
   int act_off[64];
   int act_ntt[64];
   int tile_base[65];
-  int gather_tok[4][64];  // token of each row a gather warp copies
 };
 
 struct Tile {
@@ -106,11 +108,10 @@ __device__ __forceinline__ void fail(Smem& S, StatusBlock* sb) {
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
-grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_w, const __nv_bfloat16* __restrict__ x,
+grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_xp,
                     const int32_t* __restrict__ counts, const int32_t* __restrict__ offsets,
-                    const int32_t* __restrict__ perm, const float* __restrict__ w32,
                     const int32_t* __restrict__ active, StatusBlock* __restrict__ sb, int d,
-                    int n, int k, __nv_bfloat16* __restrict__ P) {
+                    int n, __nv_bfloat16* __restrict__ P) {
   extern __shared__ uint8_t smem_raw[];
   Smem& S = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5;
@@ -120,7 +121,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_w, const __nv_bfloa
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(&S.full[s], 1 + kGatherThreads);  // TMA arrive.expect_tx + one per gatherer
+      mbar_init(&S.full[s], 1);                    // TMA arrive.expect_tx
       mbar_init(&S.empty[s], 1);                   // tcgen05.commit of the MMA thread
     }
     for (int i = 0; i < 2; ++i) {
@@ -134,7 +135,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_w, const __nv_bfloa
     tmem_alloc(&S.tmem_base, kTmemCols);
     tmem_relinquish();
   }
-  pdl_wait();  // grouping of this call is complete and visible
+  pdl_wait();  // grouping and gathered rows of this call are complete and visible
   if (threadIdx.x < 32) {
     // Active experts, their pair counts and token-tile counts; tile prefix.
     const int nact = sb->num_active;
@@ -182,57 +183,19 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_w, const __nv_bfloa
       for (int t = blockIdx.x; t < ntiles && !aborted(S); t += gridDim.x) {
         const Tile tl = decode_tile(S, t, mtiles);
         const int row = tl.e * n + tl.mt * BM;
+        const int nbox = (tl.N + kBoxRows - 1) / kBoxRows;
+        const uint32_t bytes = kABytes + nbox * kBoxRows * BK * 2;
         for (int kb = 0; kb < nk; ++kb, ++it) {
           const int s = it % kStages;
           if (it >= kStages && !mbar_wait(&S.empty[s], ((it / kStages) - 1) & 1)) { fail(S, sb); break; }
-          mbar_arrive_expect_tx(&S.full[s], kABytes);
+          mbar_arrive_expect_tx(&S.full[s], bytes);
           tma_load_2d_nohint(S.stage[s], &tmap_w, kb * BK, row, &S.full[s]);
+          for (int b = 0; b < nbox; ++b)
+            tma_load_2d_nohint(S.stage[s] + kABytes + b * kBoxRows * 128, &tmap_xp, kb * BK,
+                               tl.off + tl.tok0 + b * kBoxRows, &S.full[s]);
         }
       }
     }
-  } else if (warp >= kWarpGather0 && warp < kWarpGather0 + 4) {
-    // Each gather warp owns 64 rows of the token tile.  Lane l copies 16-byte
-    // chunk (l & 7) of rows (l >> 3) + 4i, so one warp instruction moves 4
-    // whole 128-byte rows (coalesced); the chunk lands at its 128-byte-swizzle
-    // position (chunk ^ (row & 7)).
-    const int gw = warp - kWarpGather0;
-    int* rows = S.gather_tok[gw];
-    const int chunk = lane & 7;
-    const int sub = lane >> 3;
-    int it = 0;
-    for (int t = blockIdx.x; t < ntiles && !aborted(S); t += gridDim.x) {
-      const Tile tl = decode_tile(S, t, mtiles);
-      __syncwarp();
-#pragma unroll
-      for (int i = 0; i < 2; ++i) {
-        const int r = gw * 64 + i * 32 + lane;
-        const int pr = tl.off + tl.tok0 + min(r, tl.valid - 1);
-        rows[i * 32 + lane] = perm[pr] / k;
-      }
-      __syncwarp();
-      const int nrows = min(64, max(0, tl.N - gw * 64));
-      bool ok = true;
-      for (int kb = 0; kb < nk; ++kb, ++it) {
-        const int s = it % kStages;
-        if (it >= kStages && !mbar_wait(&S.empty[s], ((it / kStages) - 1) & 1)) {
-          fail(S, sb);
-          ok = false;
-          break;
-        }
-        uint8_t* bs = S.stage[s] + kABytes;
-        for (int i = 0; i < 16; ++i) {
-          const int lr = sub + 4 * i;  // row within this warp's 64
-          if (lr < nrows) {
-            const int r = gw * 64 + lr;
-            const __nv_bfloat16* sp = x + static_cast<size_t>(rows[lr]) * d + kb * BK + chunk * 8;
-            cp_async_16(bs + r * 128 + ((chunk ^ (r & 7)) << 4), sp);
-          }
-        }
-        cp_async_arrive_noinc(&S.full[s]);
-      }
-      if (!ok) break;
-    }
-    cp_async_wait_all();
   } else if (warp == kWarpMma) {
     if (lane == 0) {
       int it = 0, titer = 0;
@@ -248,7 +211,6 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_w, const __nv_bfloa
           const int s = it % kStages;
           if (!mbar_wait(&S.full[s], (it / kStages) & 1)) { fail(S, sb); ok = false; break; }
           tc_fence_after();
-          fence_proxy_async_smem();  // gathered rows were written by cp.async
           const uint32_t a0 = smem_u32(S.stage[s]);
           const uint32_t b0 = a0 + kABytes;
 #pragma unroll
@@ -310,6 +272,22 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_w, const __nv_bfloa
   }
 }
 
+// xp[p, :] = x[perm[p] / k, :] for every pair p: one warp per row, 16-byte
+// vectors (HBM/L2-bound copy).
+__global__ void __launch_bounds__(256)
+gather_pairs_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ perm, int k, int vec_per_row,
+                    int N, uint4* __restrict__ xp) {
+  pdl_wait();
+  const int lane = threadIdx.x & 31;
+  const long long gw = (static_cast<long long>(blockIdx.x) * 256 + threadIdx.x) >> 5;
+  const long long nw = (static_cast<long long>(gridDim.x) * 256) >> 5;
+  for (long long p = gw; p < N; p += nw) {
+    const uint4* src = x + static_cast<size_t>(perm[p] / k) * vec_per_row;
+    uint4* dst = xp + static_cast<size_t>(p) * vec_per_row;
+    for (int v = lane; v < vec_per_row; v += 32) dst[v] = src[v];
+  }
+}
+
 using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
@@ -319,32 +297,53 @@ using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, 
 
 size_t tensor_experts_smem() { return sizeof(Smem) + 1024; }
 
+cudaError_t launch_gather_pairs(const void* x, const int32_t* perm, int T, int d, int k,
+                                __nv_bfloat16* xp, cudaStream_t stream) {
+  const int N = T * k;
+  const int vec_per_row = d / 8;
+  long long blocks = (static_cast<long long>(N) * 32 + 255) / 256;
+  const long long cap = static_cast<long long>(sm_count()) * 8;
+  if (blocks > cap) blocks = cap;
+  return launch_pdl(gather_pairs_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, stream,
+                    static_cast<const uint4*>(x), perm, k, vec_per_row, N, reinterpret_cast<uint4*>(xp));
+}
+
 cudaError_t launch_tensor_experts(const void* x, const void* Wv, const int32_t* counts,
                                   const int32_t* offsets, const int32_t* perm, const float* w32,
                                   const int32_t* active, StatusBlock* sb, int T, int d, int n, int k,
-                                  int E, __nv_bfloat16* P, cudaStream_t stream) {
-  (void)T;
+                                  int E, __nv_bfloat16* xp, __nv_bfloat16* P, cudaStream_t stream) {
+  (void)w32;
   void* fp = encode_tiled_fn();
   if (fp == nullptr) return cudaErrorNotSupported;
   EncodeTiled enc = reinterpret_cast<EncodeTiled>(fp);
+  const int N = T * k;
+  // Rows of x in grouped order.
+  cudaError_t err = launch_gather_pairs(x, perm, T, d, k, xp, stream);
+  if (err != cudaSuccess) return err;
   // The experts as one (E*n) x d row-major bf16 matrix; boxes of 128 rows x
-  // 64 columns (128 bytes) with 128-byte swizzle.
-  CUtensorMap tmap;
+  // 64 columns (128 bytes) with 128-byte swizzle.  The gathered rows: N x d,
+  // boxes of 32 rows.
+  CUtensorMap tmap_w, tmap_xp;
   const cuuint64_t gdim[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(E) * n};
+  const cuuint64_t xdim[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N)};
   const cuuint64_t gstride[1] = {static_cast<cuuint64_t>(d) * 2};
   const cuuint32_t box[2] = {BK, BM};
+  const cuuint32_t xbox[2] = {BK, kBoxRows};
   const cuuint32_t estride[2] = {1, 1};
-  if (enc(&tmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(Wv), gdim, gstride, box,
+  if (enc(&tmap_w, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(Wv), gdim, gstride, box,
           estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
+  if (enc(&tmap_xp, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, xp, xdim, gstride, xbox, estride,
+          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
   const size_t smem = tensor_experts_smem();
-  cudaError_t err = cudaFuncSetAttribute(grouped_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
+  err = cudaFuncSetAttribute(grouped_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem));
   if (err != cudaSuccess) return err;
-  return launch_pdl(grouped_gemm_kernel, dim3(sm_count()), dim3(kThreads), smem, stream, tmap,
-                    static_cast<const __nv_bfloat16*>(x), counts, offsets, perm, w32, active, sb, d, n,
-                    k, P);
+  return launch_pdl(grouped_gemm_kernel, dim3(sm_count()), dim3(kThreads), smem, stream, tmap_w, tmap_xp,
+                    counts, offsets, active, sb, d, n, P);
 }
 
 }  // namespace mova

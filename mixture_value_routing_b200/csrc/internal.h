@@ -102,11 +102,21 @@ cudaError_t launch_stream_experts(const void* x, const void* Wv, mova_dtype dt, 
 size_t stream_experts_smem(int d, mova_dtype dt, int* stages_out);
 
 // tcgen05 grouped GEMM (bf16): P[p, :] = SiLU(Wv[e] x[t]) as bf16 rows.
+// xp: T*k x d bf16 scratch for the pairs' x rows in grouped order.
 cudaError_t launch_tensor_experts(const void* x, const void* Wv, const int32_t* counts,
                                   const int32_t* offsets, const int32_t* perm, const float* w32,
                                   const int32_t* active, StatusBlock* sb, int T, int d, int n, int k,
-                                  int E, __nv_bfloat16* P, cudaStream_t stream);
+                                  int E, __nv_bfloat16* xp, __nv_bfloat16* P, cudaStream_t stream);
 size_t tensor_experts_smem();
+// xp[p] = x[perm[p] / k] for the T*k pairs.
+cudaError_t launch_gather_pairs(const void* x, const int32_t* perm, int T, int d, int k,
+                                __nv_bfloat16* xp, cudaStream_t stream);
+// The same grouped GEMM on SM pairs (tcgen05 cta_group::2), reading the
+// already gathered rows xp.
+cudaError_t launch_tensor_experts_pair(const void* Wv, const int32_t* counts, const int32_t* offsets,
+                                       const int32_t* active, StatusBlock* sb, int T, int d, int n,
+                                       int k, int E, const __nv_bfloat16* xp, __nv_bfloat16* P,
+                                       cudaStream_t stream);
 
 // v[t, :] = sum over slots (ascending) of w[t*k + slot] * P[pos[t*k + slot], :].
 cudaError_t launch_combine(const void* P, bool p_bf16, const int32_t* pos, const float* w32, int T,

@@ -61,6 +61,7 @@ struct Workspace {
   int32_t* pos;
   int32_t* tile_counts;
   __nv_bfloat16* planes;
+  __nv_bfloat16* xp;
   void* P;
   size_t bytes;
 };
@@ -81,6 +82,7 @@ Workspace layout(void* base, int T, int d, int k, int n) {
   w.pos = reinterpret_cast<int32_t*>(b + o);          o += align256(pairs * 4);
   w.tile_counts = reinterpret_cast<int32_t*>(b + o);  o += align256(static_cast<size_t>(group_tiles(T)) * 64 * 4);
   w.planes = reinterpret_cast<__nv_bfloat16*>(b + o); o += align256(router_planes_bytes(d));
+  w.xp = reinterpret_cast<__nv_bfloat16*>(b + o);     o += align256(pairs * static_cast<size_t>(d) * 2);
   w.P = b + o;                                        o += align256(pairs * static_cast<size_t>(n) * 4);
   w.bytes = o;
   return w;
@@ -119,11 +121,18 @@ mova_status run_experts_and_combine(const void* x, mova_dtype dt, const void* Wv
   (void)idx;
   if (path == MOVA_PATH_AUTO) path = mova_auto_path(T, dt);
   cudaError_t err;
-  const bool tensor = path == MOVA_PATH_TENSOR;
+  const bool tensor = path == MOVA_PATH_TENSOR || path == MOVA_PATH_TENSOR_1CTA;
   if (tensor) {
     if (dt != MOVA_BF16) return MOVA_ERR_UNSUPPORTED;
-    err = launch_tensor_experts(x, Wv, ws.counts, ws.offsets, ws.perm, w32, ws.active, ws.sb, T, d,
-                                n, k, E, static_cast<__nv_bfloat16*>(ws.P), stream);
+    if (path == MOVA_PATH_TENSOR && sm_count() >= 2) {
+      err = launch_gather_pairs(x, ws.perm, T, d, k, ws.xp, stream);
+      if (err == cudaSuccess)
+        err = launch_tensor_experts_pair(Wv, ws.counts, ws.offsets, ws.active, ws.sb, T, d, n, k, E, ws.xp,
+                                         static_cast<__nv_bfloat16*>(ws.P), stream);
+    } else {
+      err = launch_tensor_experts(x, Wv, ws.counts, ws.offsets, ws.perm, w32, ws.active, ws.sb, T, d,
+                                  n, k, E, ws.xp, static_cast<__nv_bfloat16*>(ws.P), stream);
+    }
   } else {
     if (stream_experts_smem(d, dt, nullptr) == 0) return MOVA_ERR_UNSUPPORTED;
     err = launch_stream_experts(x, Wv, dt, ws.counts, ws.offsets, ws.perm, w32, ws.active, ws.sb, T,
@@ -221,7 +230,8 @@ mova_status mova_value_ex(const void* x, mova_dtype x_dt, const void* idx, mova_
   if (!valid_act_dtype(x_dt) || wv_dt != x_dt) return MOVA_ERR_UNSUPPORTED;
   if (idx_dt != MOVA_I32 && idx_dt != MOVA_I8) return MOVA_ERR_UNSUPPORTED;
   if (w_dt != MOVA_F32 && w_dt != MOVA_F16) return MOVA_ERR_UNSUPPORTED;
-  if (path != MOVA_PATH_AUTO && path != MOVA_PATH_STREAM && path != MOVA_PATH_TENSOR)
+  if (path != MOVA_PATH_AUTO && path != MOVA_PATH_STREAM && path != MOVA_PATH_TENSOR &&
+      path != MOVA_PATH_TENSOR_1CTA)
     return MOVA_ERR_INVALID_ARG;
   if (T == 0) return MOVA_OK;
   if (!x || !idx || !wgt || !Wv || !v || !ws) return MOVA_ERR_INVALID_ARG;
@@ -263,7 +273,8 @@ mova_status mova_value_routed_ex(const void* x, mova_dtype x_dt, const float* Wr
   mova_status st = check_dims(T, d, E, k, n);
   if (st != MOVA_OK) return st;
   if (!valid_act_dtype(x_dt) || wv_dt != x_dt) return MOVA_ERR_UNSUPPORTED;
-  if (path != MOVA_PATH_AUTO && path != MOVA_PATH_STREAM && path != MOVA_PATH_TENSOR)
+  if (path != MOVA_PATH_AUTO && path != MOVA_PATH_STREAM && path != MOVA_PATH_TENSOR &&
+      path != MOVA_PATH_TENSOR_1CTA)
     return MOVA_ERR_INVALID_ARG;
   if (T == 0) return MOVA_OK;
   if (!x || !Wr || !br || !Wv || !v || !ws) return MOVA_ERR_INVALID_ARG;

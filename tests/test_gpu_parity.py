@@ -214,10 +214,13 @@ def test_full_stream_mid(api, T):
 
 @pytest.mark.parametrize("T,d,E,k,n", [(1, 256, 8, 4, 128), (3, 512, 64, 4, 256), (40, 256, 4, 2, 384),
                                        (300, 2560, 64, 4, 1024), (700, 512, 2, 2, 128)])
-def test_full_tensor_path(api, T, d, E, k, n):
-    """The tcgen05 path at small and ragged sizes (one token, tiles of 16,
-    several tiles per expert, 700 x 2 pairs over 2 experts = 3 token tiles)."""
-    _full(api, T, d, E, k, n, "bf16", seed=T + 1, path="tensor")
+@pytest.mark.parametrize("path", ["tensor", "tensor_1cta"])
+def test_full_tensor_path(api, T, d, E, k, n, path):
+    """The tcgen05 paths (SM-pair and single-CTA grouped GEMM) at small and
+    ragged sizes: one token, tiles of 16, n not a multiple of 256 (the odd
+    CTA's weight rows run past the expert), several token tiles per expert
+    (700 x 2 pairs over 2 experts = 3 token tiles)."""
+    _full(api, T, d, E, k, n, "bf16", seed=T + 1, path=path)
 
 
 def test_tensor_given(api):
@@ -233,10 +236,11 @@ def test_tensor_given(api):
     P.check_values(P.host_f64(v), v_ref, "bf16")
 
 
-def test_full_prefill_4096(api):
+@pytest.mark.parametrize("path", ["auto", "tensor_1cta"])
+def test_full_prefill_4096(api, path):
     """Prefill workload at full size (T=4096): routing of every token, values
     of 256 sampled tokens."""
-    _full(api, 4096, 2560, 64, 4, 1024, "bf16", sample=256)
+    _full(api, 4096, 2560, 64, 4, 1024, "bf16", sample=256, path=path)
 
 
 def test_full_skewed_16384(api):
