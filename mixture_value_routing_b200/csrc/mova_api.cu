@@ -120,12 +120,17 @@ mova_status run_experts_and_combine(const void* x, mova_dtype dt, const void* Wv
                                     void* const* events, cudaStream_t stream) {
   (void)idx;
   if (path == MOVA_PATH_AUTO) path = mova_auto_path(T, dt);
-  cudaError_t err;
+  cudaError_t err = cudaSuccess;
+  if (path != MOVA_PATH_TENSOR || sm_count() < 2) err = mark(events, 2, stream);
+  if (err != cudaSuccess) return from_cuda(err);
   const bool tensor = path == MOVA_PATH_TENSOR || path == MOVA_PATH_TENSOR_1CTA;
   if (tensor) {
     if (dt != MOVA_BF16) return MOVA_ERR_UNSUPPORTED;
     if (path == MOVA_PATH_TENSOR && sm_count() >= 2) {
+      // The gathered rows are part of the grouping: the stage mark for
+      // "grouped" follows them, so the expert stage times the GEMM alone.
       err = launch_gather_pairs(x, ws.perm, T, d, k, ws.xp, stream);
+      if (err == cudaSuccess) err = mark(events, 2, stream);
       if (err == cudaSuccess)
         err = launch_tensor_experts_pair(Wv, ws.counts, ws.offsets, ws.active, ws.sb, T, d, n, k, E, ws.xp,
                                          static_cast<__nv_bfloat16*>(ws.P), stream);
@@ -252,7 +257,6 @@ mova_status mova_value_ex(const void* x, mova_dtype x_dt, const void* idx, mova_
                            w.pos, w.active, w.sb, s);
     }
   }
-  if (err == cudaSuccess) err = mark(events, 2, s);
   if (err != cudaSuccess) return from_cuda(err);
   return run_experts_and_combine(x, x_dt, Wv, w, w.idx, w.w, T, d, E, k, n, v, path, events, s);
 }
@@ -313,7 +317,6 @@ mova_status mova_value_routed_ex(const void* x, mova_dtype x_dt, const float* Wr
                            w.offsets, w.perm, w.pos, w.active, w.sb, s);
     }
   }
-  if (err == cudaSuccess) err = mark(events, 2, s);
   if (err != cudaSuccess) return from_cuda(err);
   return run_experts_and_combine(x, x_dt, Wv, w, idx, wgt, T, d, E, k, n, v, path, events, s);
 }
