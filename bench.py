@@ -42,8 +42,9 @@ DEFAULT_STEPS = {"decode": 2000, "prefill": 300, "skewed": 60, "given": 30, "pr1
 METRIC = "MoVA value-path tokens/s at T=8 & T=4096; % of HBM / bf16 tensor roofline"
 STAGES = ("route", "group", "experts", "combine")
 KERNEL_SOURCES = {
-    "route": ["router.cu"], "group": ["permute.cu"], "experts_stream": ["stream_experts.cu"],
-    "experts_tensor": ["grouped_gemm_tc.cu"], "combine": ["combine.cu"],
+    "route": ["router.cu"], "group": ["permute.cu"],
+    "experts_stream": ["stream_experts.cu", "sm100.cuh"],
+    "experts_tensor": ["grouped_gemm_pair.cu", "sm100.cuh"], "combine": ["combine.cu"],
 }
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
