@@ -39,7 +39,7 @@
  *  - Supported on the GPU: 1 <= E <= 64, 1 <= k <= min(E, 8), d % 64 == 0,
  *    n % 128 == 0, T * k <= 131072; dtypes x/Wv/v all fp32, or all bf16
  *    (router Wr/br always fp32).  The weight-streaming expert kernel also
- *    needs d <= 6400 (bf16) or d <= 3200 (fp32).  Anything else returns
+ *    needs d <= 4544 (bf16) or d <= 3456 (fp32).  Anything else returns
  *    MOVA_ERR_UNSUPPORTED; there is no fallback path.
  */
 #ifndef MOVA_H_
@@ -175,6 +175,12 @@ mova_status mova_selftest_wait_timeout(void* ws, long long limit_cycles, void* s
 
 /* The path AUTO would pick for these sizes and dtype (for tests/benches). */
 mova_path mova_auto_path(int T, mova_dtype x_dt);
+
+/* Number of kernel launches this library has enqueued in this process so far
+ * (all devices and threads; a launch enqueued into a stream capture counts
+ * once, however often the graph is replayed).  The difference across a call
+ * is the number of kernels that call issues.  Never fails. */
+unsigned long long mova_launch_count(void);
 
 /* Size of the workspace array built into the library for
  * mova_value_routed_noalloc. */

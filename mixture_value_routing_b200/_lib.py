@@ -33,6 +33,7 @@ SIGNATURES = {
     "mova_status_str": (ctypes.c_char_p, [_i]),
     "mova_workspace_size": (_sz, [_i, _i, _i, _i, _i]),
     "mova_auto_path": (_i, [_i, _i]),
+    "mova_launch_count": (ctypes.c_ulonglong, []),
     "mova_route": (_i, [_vp, _i, _vp, _vp, _i, _i, _i, _i, _f, _vp, _vp, _vp]),
     "mova_permute": (_i, [_vp, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "mova_value": (_i, [_vp, _i, _vp, _i, _vp, _i, _vp, _i, _i, _i, _i, _i, _i, _vp, _vp, _sz, _vp]),

@@ -80,6 +80,11 @@ def auto_path(T: int, dtype: torch.dtype) -> str:
     return {v: k for k, v in _PATH.items()}[code]
 
 
+def launch_count() -> int:
+    """Kernel launches the library has enqueued in this process so far."""
+    return int(_lib.load().mova_launch_count())
+
+
 def route(x: torch.Tensor, Wr: torch.Tensor, br: torch.Tensor, k: int = 4, scale: float = 2.5):
     """(idx (T, k) int32, w (T, k) fp32)."""
     _need(x, "x", (torch.float32, torch.bfloat16), 2)

@@ -25,14 +25,32 @@ struct GroupOut {
   int32_t* pos;
   int32_t* active;
   StatusBlock* sb;
+  int32_t* tickets;  // per-row-block completion counters of the fused combine, zeroed
+  int ntickets;
+  float* logits;     // decode routing: kMaxLogitSplits x 8 x 64 partial logits
 };
 
-// Router.  When g is non-null and T <= kFusedRouterMaxT the same kernel also
-// writes the grouping (and *grouped is set); otherwise the caller runs
-// launch_permute next.
+// Router.  When g (with its logits scratch) is non-null and T <=
+// kFusedRouterMaxT, the decode kernels also write the grouping (and *grouped
+// is set); otherwise the caller runs launch_permute next.
 cudaError_t launch_router(const void* x, mova_dtype x_dt, const float* Wr, const float* br, int T,
                           int d, int E, int k, float scale, int32_t* idx, float* w,
                           const GroupOut* g, bool* grouped, cudaStream_t stream);
+
+// Decode routing in parts (T <= 8): the partial logits part[s][t][e] over S
+// K ranges (S chosen here, returned in *S_out; at most 4), which also starts
+// the call's status afresh and zeroes the tickets; then selection and
+// grouping by one CTA.  The weight-streaming kernel can take the place of
+// the second part (RouteIn).
+constexpr int kMaxLogitSplits = 4;
+cudaError_t launch_router_logits(const void* x, mova_dtype x_dt, const float* Wr, int T, int d, int E,
+                                 float* part, int* S_out, int32_t* tickets, int ntickets, StatusBlock* sb,
+                                 cudaStream_t stream);
+cudaError_t launch_select_group(const float* part, int S, const float* br, int T, int E, int k, float scale,
+                                int32_t* idx, float* w, const GroupOut* g, cudaStream_t stream);
+
+// Every kernel launch the library enqueues is counted (mova_launch_count).
+void note_launch();
 
 // Launch with programmatic dependent launch enabled: the kernel may start
 // while its predecessor on the stream finishes, and waits for it with
@@ -50,6 +68,7 @@ cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t sme
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  note_launch();
   return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
 }
 
@@ -74,7 +93,8 @@ cudaError_t launch_router_tc(const void* x, const float* Wr, const float* br, in
 cudaError_t launch_permute(const void* idx_in, mova_dtype idx_dt, const void* w_in,
                            mova_dtype w_dt, int N, int E, int32_t* idx32, float* w32,
                            int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* pos,
-                           int32_t* active, StatusBlock* sb, cudaStream_t stream);
+                           int32_t* active, StatusBlock* sb, int32_t* tickets, int ntickets,
+                           cudaStream_t stream);
 
 // Multi-CTA grouping (batches above kSmallGroupT tokens).  Tiles of 128
 // tokens; tile_counts holds group_tiles(T) x 64 ints.  launch_tile_hist
@@ -92,14 +112,35 @@ cudaError_t launch_tile_group(const int32_t* idx32, int T, int E, int k, int32_t
 
 // Weight-streaming expert kernel: P[p, :] = SiLU(Wv[e] x[t]) for every
 // pair p (fp32 rows in grouped order).
+// Routing done by the weight-streaming kernel itself (resident decode
+// batches): every CTA sums the partial logits, selects and groups in shared
+// memory; CTA 0 also writes idx_out / w_out.
+struct RouteIn {
+  const float* part;  // S x 8 x 64 partial logits (launch_router_logits); null: routing given
+  int S;
+  const float* br;
+  int E;
+  float scale;
+  int32_t* idx_out;
+  float* w_out;
+};
+
+// With tickets and v given (bf16, T <= 8 only), the kernel also performs
+// the combine: the CTA that completes a block of 8 output columns computes v
+// there; the caller then skips launch_combine.  tickets: n / 8 counters,
+// zeroed by the grouping of the same call.
 cudaError_t launch_stream_experts(const void* x, const void* Wv, mova_dtype dt, const int32_t* counts,
                                   const int32_t* offsets, const int32_t* perm, const float* w32,
                                   const int32_t* active, StatusBlock* sb, int T, int d, int n,
-                                  int k, int E, float* P, cudaStream_t stream);
+                                  int k, int E, float* P, int32_t* tickets, void* v,
+                                  const RouteIn& route, cudaStream_t stream);
 
 // Shared memory the streaming kernel needs for rows of d elements (0 if d is
 // too long for two 8-row stages).
-size_t stream_experts_smem(int d, mova_dtype dt, int* stages_out);
+size_t stream_experts_smem(int d, mova_dtype dt, int T, int* stages_out);
+// Whether the weight-streaming kernel keeps x in registers for this batch
+// (the mode in which it can also perform the combine).
+bool stream_resident(int T, int d, mova_dtype dt);
 
 // tcgen05 grouped GEMM (bf16): P[p, :] = SiLU(Wv[e] x[t]) as bf16 rows.
 // xp: T*k x d bf16 scratch for the pairs' x rows in grouped order.

@@ -8,6 +8,7 @@
 //   permute -> counts, offsets, perm, pos (stable grouping by expert)
 //   experts -> P rows = SiLU(Wv[e] x)     (weight streaming or tcgen05 GEMM)
 //   combine -> v = sum of w x row over each token's slots, ascending
+#include <atomic>
 #include <stdio.h>
 
 #include "common.cuh"
@@ -28,6 +29,12 @@ void* encode_tiled_fn() {
   return fn;
 }
 
+namespace {
+std::atomic<unsigned long long> g_launches{0};
+}  // namespace
+
+void note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+
 int sm_count() {
   static int cached[64] = {0};
   int dev = 0;
@@ -47,6 +54,9 @@ namespace {
 constexpr int kStreamMaxTokens = 64;
 // bf16 batches above this many tokens use the tensor-core router.
 constexpr int kTcRouterMinT = 64;
+// bf16 batches up to this many tokens run the combine inside the
+// weight-streaming kernel (the x rows stay resident there).
+constexpr int kFusedCombineMaxT = 8;
 
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
@@ -59,6 +69,8 @@ struct Workspace {
   int32_t* active;
   int32_t* perm;
   int32_t* pos;
+  int32_t* tickets;
+  float* logits;
   int32_t* tile_counts;
   __nv_bfloat16* planes;
   __nv_bfloat16* xp;
@@ -80,6 +92,8 @@ Workspace layout(void* base, int T, int d, int k, int n) {
   w.active = reinterpret_cast<int32_t*>(b + o);       o += 256;
   w.perm = reinterpret_cast<int32_t*>(b + o);         o += align256(pairs * 4);
   w.pos = reinterpret_cast<int32_t*>(b + o);          o += align256(pairs * 4);
+  w.tickets = reinterpret_cast<int32_t*>(b + o);      o += align256(static_cast<size_t>(n / 8) * 4);
+  w.logits = reinterpret_cast<float*>(b + o);         o += static_cast<size_t>(kMaxLogitSplits) * 8 * 64 * 4;
   w.tile_counts = reinterpret_cast<int32_t*>(b + o);  o += align256(static_cast<size_t>(group_tiles(T)) * 64 * 4);
   w.planes = reinterpret_cast<__nv_bfloat16*>(b + o); o += align256(router_planes_bytes(d));
   w.xp = reinterpret_cast<__nv_bfloat16*>(b + o);     o += align256(pairs * static_cast<size_t>(d) * 2);
@@ -121,6 +135,7 @@ mova_status run_experts_and_combine(const void* x, mova_dtype dt, const void* Wv
   (void)idx;
   if (path == MOVA_PATH_AUTO) path = mova_auto_path(T, dt);
   cudaError_t err = cudaSuccess;
+  bool fused_combine = false;
   if (path != MOVA_PATH_TENSOR || sm_count() < 2) err = mark(events, 2, stream);
   if (err != cudaSuccess) return from_cuda(err);
   const bool tensor = path == MOVA_PATH_TENSOR || path == MOVA_PATH_TENSOR_1CTA;
@@ -134,17 +149,22 @@ mova_status run_experts_and_combine(const void* x, mova_dtype dt, const void* Wv
       if (err == cudaSuccess)
         err = launch_tensor_experts_pair(Wv, ws.counts, ws.offsets, ws.active, ws.sb, T, d, n, k, E, ws.xp,
                                          static_cast<__nv_bfloat16*>(ws.P), stream);
+      if (err == cudaSuccess) note_launch();  // the pair GEMM's one launch
     } else {
       err = launch_tensor_experts(x, Wv, ws.counts, ws.offsets, ws.perm, w32, ws.active, ws.sb, T, d,
                                   n, k, E, ws.xp, static_cast<__nv_bfloat16*>(ws.P), stream);
     }
   } else {
-    if (stream_experts_smem(d, dt, nullptr) == 0) return MOVA_ERR_UNSUPPORTED;
+    if (stream_experts_smem(d, dt, T, nullptr) == 0) return MOVA_ERR_UNSUPPORTED;
+    // Decode-sized bf16 batches fold the combine into the expert kernel.
+    fused_combine = T <= kFusedCombineMaxT && stream_resident(T, d, dt);
     err = launch_stream_experts(x, Wv, dt, ws.counts, ws.offsets, ws.perm, w32, ws.active, ws.sb, T,
-                                d, n, k, E, static_cast<float*>(ws.P), stream);
+                                d, n, k, E, static_cast<float*>(ws.P), fused_combine ? ws.tickets : nullptr,
+                                fused_combine ? v : nullptr, RouteIn{}, stream);
   }
   if (err == cudaSuccess) err = mark(events, 3, stream);
-  if (err == cudaSuccess) err = launch_combine(ws.P, tensor, ws.pos, w32, T, k, n, v, dt, stream);
+  if (err == cudaSuccess && !fused_combine)
+    err = launch_combine(ws.P, tensor, ws.pos, w32, T, k, n, v, dt, stream);
   if (err == cudaSuccess) err = mark(events, 4, stream);
   return from_cuda(err);
 }
@@ -188,6 +208,8 @@ size_t mova_workspace_size(int T, int d, int E, int k, int n) {
   return layout(nullptr, T, d, k, n).bytes;
 }
 
+unsigned long long mova_launch_count(void) { return mova::g_launches.load(); }
+
 mova_path mova_auto_path(int T, mova_dtype x_dt) {
   return (x_dt == MOVA_BF16 && T > kStreamMaxTokens) ? MOVA_PATH_TENSOR : MOVA_PATH_STREAM;
 }
@@ -223,7 +245,7 @@ mova_status mova_permute(const int32_t* idx, int T, int E, int k, int32_t* count
     return from_cuda(err);
   }
   return from_cuda(launch_permute(idx, MOVA_I32, nullptr, MOVA_F32, T * k, E, nullptr, nullptr,
-                                  counts, offsets, perm, pos, w.active, w.sb, s));
+                                  counts, offsets, perm, pos, w.active, w.sb, nullptr, 0, s));
 }
 
 mova_status mova_value_ex(const void* x, mova_dtype x_dt, const void* idx, mova_dtype idx_dt,
@@ -254,7 +276,7 @@ mova_status mova_value_ex(const void* x, mova_dtype x_dt, const void* idx, mova_
                                 w.active, w.sb, false, s);
     } else {
       err = launch_permute(idx, idx_dt, wgt, w_dt, T * k, E, w.idx, w.w, w.counts, w.offsets, w.perm,
-                           w.pos, w.active, w.sb, s);
+                           w.pos, w.active, w.sb, w.tickets, n / 8, s);
     }
   }
   if (err != cudaSuccess) return from_cuda(err);
@@ -289,9 +311,27 @@ mova_status mova_value_routed_ex(const void* x, mova_dtype x_dt, const float* Wr
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   int32_t* idx = idx_out ? idx_out : w.idx;
   float* wgt = w_out ? w_out : w.w;
-  const GroupOut g{w.counts, w.offsets, w.perm, w.pos, w.active, w.sb};
+  const GroupOut g{w.counts, w.offsets, w.perm, w.pos, w.active, w.sb, w.tickets, n / 8, w.logits};
   bool grouped = false;
   cudaError_t err = mark(events, 0, s);
+  // Decode batches on the weight-streaming path: the router computes the
+  // logits only; the streaming kernel selects, groups and combines.
+  const mova_path rp = path == MOVA_PATH_AUTO ? mova_auto_path(T, x_dt) : path;
+  if (rp == MOVA_PATH_STREAM && T <= kFusedCombineMaxT && stream_resident(T, d, x_dt) &&
+      stream_experts_smem(d, x_dt, T, nullptr) != 0) {
+    int S = 0;
+    if (err == cudaSuccess)
+      err = launch_router_logits(x, x_dt, Wr, T, d, E, w.logits, &S, w.tickets, n / 8, w.sb, s);
+    if (err == cudaSuccess) err = mark(events, 1, s);
+    if (err == cudaSuccess) err = mark(events, 2, s);
+    const RouteIn ri{w.logits, S, br, E, scale, idx, wgt};
+    if (err == cudaSuccess)
+      err = launch_stream_experts(x, Wv, x_dt, w.counts, w.offsets, w.perm, wgt, w.active, w.sb, T, d, n, k,
+                                  E, static_cast<float*>(w.P), w.tickets, v, ri, s);
+    if (err == cudaSuccess) err = mark(events, 3, s);
+    if (err == cudaSuccess) err = mark(events, 4, s);
+    return from_cuda(err);
+  }
   // bf16 batches above the decode range route on the tensor cores and group
   // with the tile kernels (the router writes the per-tile histograms).
   const bool tc_router = x_dt == MOVA_BF16 && T > kTcRouterMinT;
@@ -314,7 +354,7 @@ mova_status mova_value_routed_ex(const void* x, mova_dtype x_dt, const float* Wr
                                 w.active, w.sb, false, s);
     } else {
       err = launch_permute(idx, MOVA_I32, nullptr, MOVA_F32, T * k, E, nullptr, nullptr, w.counts,
-                           w.offsets, w.perm, w.pos, w.active, w.sb, s);
+                           w.offsets, w.perm, w.pos, w.active, w.sb, w.tickets, n / 8, s);
     }
   }
   if (err != cudaSuccess) return from_cuda(err);
@@ -331,6 +371,7 @@ mova_status mova_value_routed(const void* x, mova_dtype x_dt, const float* Wr, c
 
 mova_status mova_selftest_wait_timeout(void* ws, long long limit_cycles, void* stream) {
   if (!ws || limit_cycles <= 0 || limit_cycles > kWaitLimitCycles) return MOVA_ERR_INVALID_ARG;
+  note_launch();
   selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
       static_cast<StatusBlock*>(ws), limit_cycles);
   return from_cuda(cudaGetLastError());

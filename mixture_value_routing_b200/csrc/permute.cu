@@ -28,7 +28,8 @@ __global__ void __launch_bounds__(kPermThreads)
 permute_kernel(const IT* __restrict__ idx_in, const WT* __restrict__ w_in, int N, int E,
                int32_t* __restrict__ idx32, float* __restrict__ w32, int32_t* __restrict__ counts,
                int32_t* __restrict__ offsets, int32_t* __restrict__ perm, int32_t* __restrict__ pos,
-               int32_t* __restrict__ active, StatusBlock* sb) {
+               int32_t* __restrict__ active, StatusBlock* sb, int32_t* __restrict__ tickets,
+               int ntickets) {
   extern __shared__ uint8_t codes[];  // N expert codes
   __shared__ int hist[kPermWarps][64];
   __shared__ int tot[64];
@@ -45,6 +46,7 @@ permute_kernel(const IT* __restrict__ idx_in, const WT* __restrict__ w_in, int N
     sb->detail = 0;
     sb->work_next = 0;
   }
+  for (int i = tid; i < ntickets; i += kPermThreads) tickets[i] = 0;
   __syncthreads();
 
   const int seg = (N + kPermWarps - 1) / kPermWarps;
@@ -133,15 +135,18 @@ permute_kernel(const IT* __restrict__ idx_in, const WT* __restrict__ w_in, int N
 template <typename IT, typename WT>
 cudaError_t launch_t(const void* idx_in, const void* w_in, int N, int E, int32_t* idx32, float* w32,
                      int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* pos,
-                     int32_t* active, StatusBlock* sb, cudaStream_t stream) {
+                     int32_t* active, StatusBlock* sb, int32_t* tickets, int ntickets,
+                     cudaStream_t stream) {
   auto kern = permute_kernel<IT, WT>;
   const size_t smem = static_cast<size_t>(N);
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(kMaxPairs));
   if (err != cudaSuccess) return err;
+  note_launch();
   kern<<<1, kPermThreads, smem, stream>>>(static_cast<const IT*>(idx_in),
                                           static_cast<const WT*>(w_in), N, E, idx32, w32, counts,
-                                          offsets, perm, pos, active, sb);
+                                          offsets, perm, pos, active, sb, tickets,
+                                          tickets ? ntickets : 0);
   return cudaGetLastError();
 }
 
@@ -291,6 +296,7 @@ template <typename IT, typename WT>
 cudaError_t launch_hist_t(const void* idx_in, const void* w_in, int N, int E, int k, int32_t* idx32,
                           float* w32, int32_t* tile_counts, StatusBlock* sb, cudaStream_t stream) {
   const int ntiles = (N + kTileTok * k - 1) / (kTileTok * k);
+  note_launch();
   tile_hist_kernel<IT, WT><<<ntiles, 256, 0, stream>>>(static_cast<const IT*>(idx_in),
                                                        static_cast<const WT*>(w_in), N, E, k, idx32,
                                                        w32, tile_counts, sb);
@@ -302,21 +308,22 @@ cudaError_t launch_hist_t(const void* idx_in, const void* w_in, int N, int E, in
 cudaError_t launch_permute(const void* idx_in, mova_dtype idx_dt, const void* w_in,
                            mova_dtype w_dt, int N, int E, int32_t* idx32, float* w32,
                            int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* pos,
-                           int32_t* active, StatusBlock* sb, cudaStream_t stream) {
+                           int32_t* active, StatusBlock* sb, int32_t* tickets, int ntickets,
+                           cudaStream_t stream) {
   if (N <= 0 || N > kMaxPairs) return cudaErrorInvalidValue;
   if (w_in == nullptr) w32 = nullptr;
   if (idx_dt == MOVA_I8) {
     if (w_dt == MOVA_F16)
       return launch_t<int8_t, __half>(idx_in, w_in, N, E, idx32, w32, counts, offsets, perm, pos,
-                                      active, sb, stream);
+                                      active, sb, tickets, ntickets, stream);
     return launch_t<int8_t, float>(idx_in, w_in, N, E, idx32, w32, counts, offsets, perm, pos,
-                                   active, sb, stream);
+                                   active, sb, tickets, ntickets, stream);
   }
   if (w_dt == MOVA_F16)
     return launch_t<int32_t, __half>(idx_in, w_in, N, E, idx32, w32, counts, offsets, perm, pos,
-                                     active, sb, stream);
+                                     active, sb, tickets, ntickets, stream);
   return launch_t<int32_t, float>(idx_in, w_in, N, E, idx32, w32, counts, offsets, perm, pos,
-                                  active, sb, stream);
+                                  active, sb, tickets, ntickets, stream);
 }
 
 }  // namespace mova

@@ -13,9 +13,12 @@
 // one warp per token holds two experts per lane, forms the biased scores in
 // registers and runs k rounds of a warp arg-max (ties -> lower index).
 #include <cooperative_groups.h>
+#include <cuda.h>
 
 #include "common.cuh"
 #include "internal.h"
+#include "route_select.cuh"
+#include "sm100.cuh"
 
 namespace cg = cooperative_groups;
 
@@ -35,63 +38,6 @@ __device__ __forceinline__ float4 load4(const __nv_bfloat16* p) {
 constexpr int kRouterThreads = 128;
 constexpr int kRouterKC = 32;  // K elements per shared-memory chunk
 
-// Gate and selection of one token by one warp.  lg: the token's E logits (in
-// shared memory).  Lane l holds experts l and l + 32.  A candidate is (biased
-// score, key); the key is the expert index, plus 64 once the expert is taken
-// or does not exist, so such candidates lose every tie against a live expert
-// (NaN scores are mapped to -inf and can never displace a finite one).  k
-// rounds of a warp arg-max under the total order (score descending, key
-// ascending) pick the experts: ties go to the lower index.  On return every
-// lane holds the same sel_e / sel_s (unbiased sigmoid scores) for j < k.
-__device__ __forceinline__ void select_top_k(const float* lg, const float* __restrict__ br, int E,
-                                             int k, int lane, int (&sel_e)[8], float (&sel_s)[8]) {
-  const float NEG = -INFINITY;
-  const int e0 = lane, e1 = lane + 32;
-  float s0 = 0.f, s1 = 0.f, b0 = NEG, b1 = NEG;
-  int key0 = e0 + 64, key1 = e1 + 64;
-  if (e0 < E) {
-    s0 = sigmoidf_(lg[e0]);
-    b0 = s0 + br[e0];
-    if (!(b0 == b0)) b0 = NEG;
-    key0 = e0;
-  }
-  if (e1 < E) {
-    s1 = sigmoidf_(lg[e1]);
-    b1 = s1 + br[e1];
-    if (!(b1 == b1)) b1 = NEG;
-    key1 = e1;
-  }
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    if (j < k) {
-      float bb = b0, bs = s0;
-      int be = key0;
-      if (b1 > b0 || (b1 == b0 && key1 < key0)) { bb = b1; bs = s1; be = key1; }
-#pragma unroll
-      for (int off = 16; off >= 1; off >>= 1) {
-        const float ob = __shfl_xor_sync(0xffffffffu, bb, off);
-        const float os = __shfl_xor_sync(0xffffffffu, bs, off);
-        const int oe = __shfl_xor_sync(0xffffffffu, be, off);
-        if (ob > bb || (ob == bb && oe < be)) { bb = ob; bs = os; be = oe; }
-      }
-      be &= 63;  // always a live expert: k <= E
-      sel_e[j] = be;
-      sel_s[j] = bs;
-      if (be == e0) { b0 = NEG; key0 = e0 + 64; }
-      if (be == e1) { b1 = NEG; key1 = e1 + 64; }
-    }
-  }
-}
-
-// Sum of the k selected scores in slot order.
-__device__ __forceinline__ float sum_k(const float (&s)[8], int k) {
-  float acc = 0.f;
-#pragma unroll
-  for (int j = 0; j < 8; ++j)
-    if (j < k) acc += s[j];
-  return acc;
-}
-
 template <typename XT, int TT>
 __global__ void __launch_bounds__(kRouterThreads)
 router_kernel(const XT* __restrict__ x, const float* __restrict__ Wr, const float* __restrict__ br,
@@ -102,6 +48,7 @@ router_kernel(const XT* __restrict__ x, const float* __restrict__ Wr, const floa
   __shared__ __align__(16) float xs[TT][KC + 4];
   __shared__ __align__(16) float wsm[64][KC + 4];
   __shared__ __align__(16) float part[TT * 64];
+  __shared__ float brs[64];
 
   cg::cluster_group cluster = cg::this_cluster();
   const int tid = threadIdx.x;
@@ -113,6 +60,7 @@ router_kernel(const XT* __restrict__ x, const float* __restrict__ Wr, const floa
   const int c_end = (rank + 1) * nchunks / ks;
   const int tg = tid >> 4;
   const int eg = tid & 15;
+  if (tid < 64) brs[tid] = tid < E ? br[tid] : 0.f;
 
   float acc[TPT][4];
 #pragma unroll
@@ -181,7 +129,7 @@ router_kernel(const XT* __restrict__ x, const float* __restrict__ Wr, const floa
     if (t >= T) break;
     int sel_e[8];
     float sel_s[8];
-    select_top_k(&part[tt * 64], br, E, k, lane, sel_e, sel_s);
+    select_top_k(&part[tt * 64], brs, E, k, lane, sel_e, sel_s);
     const float ssum = sum_k(sel_s, k);
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
@@ -194,192 +142,144 @@ router_kernel(const XT* __restrict__ x, const float* __restrict__ Wr, const floa
 }
 
 // ---------------------------------------------------------------------------
-// Decode router (T <= 8): one cluster of 8 CTAs x 8 warps, one warp per
-// expert.  Each warp issues its whole router row (d fp32) as 16-byte loads at
-// once and dots it with every token's x (L1/L2 hits), so the 655 KB router
-// read is spread over 64 warps with all loads in flight.  Partial sums are
-// reduced across lanes in a fixed butterfly order; each warp writes its
-// expert's T logits into CTA rank 0's shared memory (distributed shared
-// memory).  Rank 0 then selects per token (warp per token) and, as T*k <= 64
-// pairs, also groups the pairs by expert in the same kernel (stable counting
-// sort by one warp), so a decode step needs no separate grouping launch.
+// Decode router (T <= 8), in two parts.
+//
+// router_logits_kernel: one CTA per (expert, K range), S ranges per expert
+// (E * S CTAs, S <= 4).  Each thread takes 8-element chunks of the range:
+// the chunk of the expert's router row (requested before
+// griddepcontrol.wait: no kernel writes router weights), then the same
+// chunk of every token's x, 8 FMAs per token in ascending k.  A transposing
+// warp butterfly leaves each token's warp sum in one lane group; the warps'
+// sums are added in warp order and stored as part[s][t][e].  Every step has a
+// fixed order, so the logits do not depend on timing.  The CTA of (expert 0,
+// range 0) also starts the call's status afresh and zeroes the fused
+// combine's row-block tickets.
+//
+// The selection and grouping that follow (select_token, group_pairs_warp)
+// run either in select_group_kernel (one CTA) or at the start of the
+// weight-streaming kernel, which then needs no grouping launch at all.
 // ---------------------------------------------------------------------------
-constexpr int kSmallT = 8;
-constexpr int kSmallWarps = 8;
-constexpr size_t kSmallRouterSmem = 160 * 1024;  // largest staged x tile
-
-constexpr int kSmallQ = 4;                        // warps per expert (K quarters)
-constexpr int kSmallThreads = kSmallWarps * kSmallQ * 32;
-constexpr int kSmallCH = 5;                       // float4 loads in flight per lane and pass
+constexpr int kDecT = 8;
+constexpr int kLogitThreads = 256;
 
 template <typename XT>
-__global__ void __launch_bounds__(kSmallThreads)
-router_small_kernel(const XT* __restrict__ x, const float* __restrict__ Wr,
-                    const float* __restrict__ br, int T, int d, int E, int k, float scale,
-                    int32_t* __restrict__ idx_out, float* __restrict__ w_out,
-                    GroupOut g) {
-  extern __shared__ __align__(16) uint8_t xsm[];  // the T x d tokens, as stored
-  __shared__ float logits[kSmallT][64];
-  __shared__ float part[kSmallQ][kSmallWarps][kSmallT];
-  __shared__ int sel[kSmallT * 8];
-  cg::cluster_group cluster = cg::this_cluster();
-  const XT* xs = reinterpret_cast<const XT*>(xsm);
-  const int rank = blockIdx.x;  // 8 CTAs per cluster, 8 experts per CTA
-  const int warp = threadIdx.x >> 5;
-  const int lane = threadIdx.x & 31;
-  const int el = warp >> 2;     // expert within the CTA
-  const int q = warp & 3;       // K quarter
-  const int e = rank * kSmallWarps + el;
-  float* rlog = cluster.map_shared_rank(&logits[0][0], 0);
-  // Every CTA of the cluster must have started before shared memory of
-  // another CTA is written: arrive now, wait just before the remote stores.
-  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+__global__ void __launch_bounds__(kLogitThreads)
+router_logits_kernel(const float* __restrict__ Wr, const XT* __restrict__ x, int T, int d, int E,
+                     float* __restrict__ part, int32_t* __restrict__ tickets, int ntickets,
+                     StatusBlock* __restrict__ sb) {
+  __shared__ float red[kLogitThreads / 32][kDecT];
+  const int e = blockIdx.x % E;
+  const int s = blockIdx.x / E;
+  const int S = gridDim.x / E;
+  const int chunks = d / 8;
+  const int cb = chunks * s / S;
+  const int ce = chunks * (s + 1) / S;
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
+  const float* wrow = Wr + static_cast<size_t>(e) * d;
 
-  // K is cut into chunks of 128 (32 lanes x float4); quarter q owns a
-  // contiguous run of chunks.
-  const int nchunk = (d + 127) / 128;
-  const int cb = nchunk * q / kSmallQ;
-  const int ce = nchunk * (q + 1) / kSmallQ;
-  const float* wrow = Wr + static_cast<size_t>(min(e, E - 1)) * d;
-  float4 wv[kSmallCH];
-#pragma unroll
-  for (int i = 0; i < kSmallCH; ++i) {
-    const int kk = (cb + i) * 128 + lane * 4;
-    wv[i] = (cb + i < ce && kk < d) ? __ldg(reinterpret_cast<const float4*>(wrow + kk))
-                                    : make_float4(0.f, 0.f, 0.f, 0.f);
+  // The first chunk's router weights, in flight during the wait.
+  const int c0 = cb + tid;
+  float w0[8];
+  if (c0 < ce) load8(wrow + 8 * c0, w0);
+  pdl_wait();  // x may come from the previous kernel; every output is written after this
+  pdl_trigger();
+  if (blockIdx.x == 0) {
+    if (tid == 0 && sb != nullptr) {
+      sb->code = 0;
+      sb->detail = 0;
+      sb->work_next = 0;
+    }
+    for (int i = tid; i < ntickets; i += kLogitThreads) tickets[i] = 0;
   }
-  {
-    const int nvec = static_cast<int>(static_cast<size_t>(T) * d * sizeof(XT) / 16);
-    const uint4* src = reinterpret_cast<const uint4*>(x);
-    uint4* dst = reinterpret_cast<uint4*>(xsm);
-    for (int i = threadIdx.x; i < nvec; i += kSmallThreads) dst[i] = src[i];
-  }
-  __syncthreads();
 
-  float acc[kSmallT];
+  float acc[kDecT];
 #pragma unroll
-  for (int t = 0; t < kSmallT; ++t) acc[t] = 0.f;
-  for (int c0 = cb; c0 < ce; c0 += kSmallCH) {
-    if (c0 > cb) {
+  for (int t = 0; t < kDecT; ++t) acc[t] = 0.f;
+  for (int c = c0; c < ce; c += kLogitThreads) {
+    float w[8];
+    if (c == c0) {
 #pragma unroll
-      for (int i = 0; i < kSmallCH; ++i) {
-        const int kk = (c0 + i) * 128 + lane * 4;
-        wv[i] = (c0 + i < ce && kk < d) ? __ldg(reinterpret_cast<const float4*>(wrow + kk))
-                                        : make_float4(0.f, 0.f, 0.f, 0.f);
-      }
+      for (int q = 0; q < 8; ++q) w[q] = w0[q];
+    } else {
+      load8(wrow + 8 * c, w);
     }
 #pragma unroll
-    for (int t = 0; t < kSmallT; ++t) {
+    for (int t = 0; t < kDecT; ++t) {
       if (t < T) {
+        float xv[8];
+        load8(x + static_cast<size_t>(t) * d + 8 * c, xv);
 #pragma unroll
-        for (int i = 0; i < kSmallCH; ++i) {
-          const int kk = (c0 + i) * 128 + lane * 4;
-          if (c0 + i < ce && kk < d) {
-            const float4 xv = load4(xs + static_cast<size_t>(t) * d + kk);
-            acc[t] = fmaf(xv.x, wv[i].x, acc[t]);
-            acc[t] = fmaf(xv.y, wv[i].y, acc[t]);
-            acc[t] = fmaf(xv.z, wv[i].z, acc[t]);
-            acc[t] = fmaf(xv.w, wv[i].w, acc[t]);
-          }
-        }
+        for (int q = 0; q < 8; ++q) acc[t] = fmaf(w[q], xv[q], acc[t]);
       }
     }
   }
+
+  // Transposing butterfly over the 8 token sums: after the steps with
+  // offsets 16, 8, 4 lane l holds token 4*b4 + 2*b3 + b2 (bits of l) summed
+  // over its 8-lane group pattern; offsets 2 and 1 finish the warp sum.
+  {
+    const bool u16 = (lane & 16) != 0;
 #pragma unroll
-  for (int t = 0; t < kSmallT; ++t) {
+    for (int i = 0; i < 4; ++i) {
+      const float send = u16 ? acc[i] : acc[i + 4];
+      const float keep = u16 ? acc[i + 4] : acc[i];
+      acc[i] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
+    }
+    const bool u8 = (lane & 8) != 0;
 #pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) acc[t] += __shfl_xor_sync(0xffffffffu, acc[t], off);
+    for (int i = 0; i < 2; ++i) {
+      const float send = u8 ? acc[i] : acc[i + 2];
+      const float keep = u8 ? acc[i + 2] : acc[i];
+      acc[i] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+    }
+    const bool u4 = (lane & 4) != 0;
+    const float send = u4 ? acc[0] : acc[1];
+    const float keep = u4 ? acc[1] : acc[0];
+    acc[0] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
+    acc[0] += __shfl_xor_sync(0xffffffffu, acc[0], 2);
+    acc[0] += __shfl_xor_sync(0xffffffffu, acc[0], 1);
   }
-  if (lane == 0) {
+  if ((lane & 3) == 0) red[warp][((lane >> 4) & 1) * 4 + ((lane >> 3) & 1) * 2 + ((lane >> 2) & 1)] = acc[0];
+  __syncthreads();
+  if (tid < kDecT) {
+    float v = red[0][tid];
 #pragma unroll
-    for (int t = 0; t < kSmallT; ++t) part[q][el][t] = acc[t];
+    for (int w = 1; w < kLogitThreads / 32; ++w) v += red[w][tid];
+    part[(s * kDecT + tid) * 64 + e] = v;
+  }
+}
+
+// Selection and grouping of a decode batch by one CTA, from the S partial
+// logits: warp t selects token t, warp 0 then groups the pairs.
+__global__ void __launch_bounds__(kLogitThreads)
+select_group_kernel(const float* __restrict__ part, int S, const float* __restrict__ br, int T, int E,
+                    int k, float scale, int32_t* __restrict__ idx_out, float* __restrict__ w_out,
+                    GroupOut g) {
+  __shared__ float lg[kDecT * 64];
+  __shared__ float brs[64];
+  __shared__ int sel[kDecT * 8];
+  __shared__ float wsel[kDecT * 8];
+  __shared__ int scratch[128];
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
+  if (tid < 64) brs[tid] = tid < E ? br[tid] : 0.f;
+  pdl_wait();
+  for (int j = tid; j < T * 64; j += kLogitThreads) {
+    float v = part[j];
+    for (int r = 1; r < S; ++r) v += part[r * kDecT * 64 + j];
+    lg[j] = v;
   }
   __syncthreads();
-  asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
-  // The four K quarters of each expert, summed in order, go to rank 0.
-  if (threadIdx.x < kSmallWarps * kSmallT) {
-    const int ee = threadIdx.x / kSmallT;
-    const int t = threadIdx.x % kSmallT;
-    const int eg = rank * kSmallWarps + ee;
-    if (eg < E) {
-      float v = part[0][ee][t];
-#pragma unroll
-      for (int qq = 1; qq < kSmallQ; ++qq) v += part[qq][ee][t];
-      rlog[t * 64 + eg] = v;
-    }
-  }
-  cluster.sync();
-  if (rank != 0) return;
-
-  // Selection: warp t handles token t.
-  if (warp < T) {
-    const int t = warp;
-    float ws_[8];
-    int es_[8];
-    select_top_k(&logits[t][0], br, E, k, lane, es_, ws_);
-    const float ssum = sum_k(ws_, k);
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      if (j < k && lane == j) {
-        idx_out[t * k + j] = es_[j];
-        w_out[t * k + j] = scale * ws_[j] / ssum;
-        sel[t * k + j] = es_[j];
-      }
-    }
-  }
+  if (warp < T) select_token(&lg[warp * 64], brs, E, k, scale, warp, lane, sel, wsel, idx_out, w_out);
   if (g.counts == nullptr) return;
   __syncthreads();
-  if (warp != 0) return;
-  // Grouping of the N = T*k <= 64 pairs by one warp (stable counting sort).
-  const int N = T * k;
-  const int f0 = lane, f1 = lane + 32;
-  const int ef0 = (f0 < N) ? sel[f0] : -1;
-  const int ef1 = (f1 < N) ? sel[f1] : -1;
-  int rank0 = 0, rank1 = 0, cnt0 = 0, cnt1 = 0;
-  for (int f = 0; f < N; ++f) {
-    const int ef = sel[f];
-    rank0 += (f < f0 && ef == ef0);
-    rank1 += (f < f1 && ef == ef1);
-    cnt0 += (ef == lane);
-    cnt1 += (ef == lane + 32);
-  }
-  // Exclusive scan of the counts over experts lane, lane+32.
-  int inc0 = cnt0;
-#pragma unroll
-  for (int off = 1; off < 32; off <<= 1) {
-    const int y = __shfl_up_sync(0xffffffffu, inc0, off);
-    if (lane >= off) inc0 += y;
-  }
-  const int tot0 = __shfl_sync(0xffffffffu, inc0, 31);
-  int inc1 = cnt1;
-#pragma unroll
-  for (int off = 1; off < 32; off <<= 1) {
-    const int y = __shfl_up_sync(0xffffffffu, inc1, off);
-    if (lane >= off) inc1 += y;
-  }
-  const int ex0 = inc0 - cnt0;
-  const int ex1 = tot0 + inc1 - cnt1;
-  if (lane < E) { g.counts[lane] = cnt0; g.offsets[lane] = ex0; }
-  if (lane + 32 < E) { g.counts[lane + 32] = cnt1; g.offsets[lane + 32] = ex1; }
-  if (lane == 0) g.offsets[E] = N;
-  __shared__ int offs[64];
-  offs[lane] = ex0;
-  offs[lane + 32] = ex1;
-  __syncwarp();
-  if (f0 < N) { const int p = offs[ef0] + rank0; g.pos[f0] = p; g.perm[p] = f0; }
-  if (f1 < N) { const int p = offs[ef1] + rank1; g.pos[f1] = p; g.perm[p] = f1; }
-  const bool a0 = lane < E && cnt0 > 0;
-  const bool a1 = lane + 32 < E && cnt1 > 0;
-  const unsigned m0 = __ballot_sync(0xffffffffu, a0);
-  const unsigned m1 = __ballot_sync(0xffffffffu, a1);
-  const unsigned lt = (1u << lane) - 1u;
-  if (a0) g.active[__popc(m0 & lt)] = lane;
-  if (a1) g.active[__popc(m0) + __popc(m1 & lt)] = lane + 32;
-  if (lane == 0) {
-    g.sb->code = 0;
-    g.sb->detail = 0;
-    g.sb->num_active = __popc(m0) + __popc(m1);
-    g.sb->work_next = 0;
+  if (warp == 0) {
+    const int nact = group_pairs_warp(sel, T * k, E, lane, scratch, g.counts, g.offsets, g.pos, g.perm,
+                                      g.active);
+    if (lane == 0) g.sb->num_active = nact;
   }
 }
 
@@ -400,35 +300,16 @@ cudaError_t launch_router_t(const void* x, const float* Wr, const float* br, int
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  note_launch();
   return cudaLaunchKernelEx(&cfg, router_kernel<XT, TT>, static_cast<const XT*>(x), Wr, br, T, d,
                             E, k, scale, idx, w);
 }
 
 template <typename XT>
-cudaError_t launch_router_small(const void* x, const float* Wr, const float* br, int T, int d,
-                                int E, int k, float scale, int32_t* idx, float* w, GroupOut g,
-                                cudaStream_t stream) {
-  const size_t smem = static_cast<size_t>(T) * d * sizeof(XT);
-  if (smem > 48 * 1024) {
-    cudaError_t err = cudaFuncSetAttribute(router_small_kernel<XT>,
-                                           cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           static_cast<int>(kSmallRouterSmem));
-    if (err != cudaSuccess) return err;
-  }
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(8, 1, 1);
-  cfg.blockDim = dim3(kSmallThreads, 1, 1);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 8;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, router_small_kernel<XT>, static_cast<const XT*>(x), Wr, br, T,
-                            d, E, k, scale, idx, w, g);
+cudaError_t launch_logits_t(const void* x, const float* Wr, int T, int d, int E, int S, float* part,
+                            int32_t* tickets, int ntickets, StatusBlock* sb, cudaStream_t stream) {
+  return launch_pdl(router_logits_kernel<XT>, dim3(static_cast<unsigned>(E * S)), dim3(kLogitThreads), 0,
+                    stream, Wr, static_cast<const XT*>(x), T, d, E, part, tickets, ntickets, sb);
 }
 
 }  // namespace
@@ -438,14 +319,13 @@ cudaError_t launch_router(const void* x, mova_dtype x_dt, const float* Wr, const
                           const GroupOut* g, bool* grouped, cudaStream_t stream) {
   if (grouped) *grouped = false;
   if (T <= 0) return cudaSuccess;
-  const size_t xbytes = static_cast<size_t>(T) * d * (x_dt == MOVA_BF16 ? 2 : 4);
-  if (T <= kFusedRouterMaxT && xbytes <= kSmallRouterSmem) {
-    GroupOut go{};
-    if (g != nullptr) go = *g;
-    if (grouped) *grouped = (g != nullptr);
-    return x_dt == MOVA_BF16
-               ? launch_router_small<__nv_bfloat16>(x, Wr, br, T, d, E, k, scale, idx, w, go, stream)
-               : launch_router_small<float>(x, Wr, br, T, d, E, k, scale, idx, w, go, stream);
+  if (T <= kFusedRouterMaxT && g != nullptr && g->logits != nullptr) {
+    int S = 0;
+    cudaError_t err = launch_router_logits(x, x_dt, Wr, T, d, E, g->logits, &S, g->tickets, g->ntickets,
+                                           g->sb, stream);
+    if (err != cudaSuccess) return err;
+    if (grouped) *grouped = true;
+    return launch_select_group(g->logits, S, br, T, E, k, scale, idx, w, g, stream);
   }
   const bool small = T <= 64;
   const int TT = small ? 8 : 32;
@@ -461,6 +341,30 @@ cudaError_t launch_router(const void* x, mova_dtype x_dt, const float* Wr, const
   }
   return small ? launch_router_t<float, 8>(x, Wr, br, T, d, E, k, scale, idx, w, ks, stream)
                : launch_router_t<float, 32>(x, Wr, br, T, d, E, k, scale, idx, w, ks, stream);
+}
+
+int logit_splits(int d, int E) {
+  int S = 1;
+  while (S < kMaxLogitSplits && E * S * 2 <= sm_count() && d / 8 >= 2 * S * kLogitThreads / 4) S *= 2;
+  return S;
+}
+
+cudaError_t launch_router_logits(const void* x, mova_dtype x_dt, const float* Wr, int T, int d, int E,
+                                 float* part, int* S_out, int32_t* tickets, int ntickets, StatusBlock* sb,
+                                 cudaStream_t stream) {
+  if (T <= 0 || T > kDecT) return cudaErrorInvalidValue;
+  const int S = logit_splits(d, E);
+  *S_out = S;
+  return x_dt == MOVA_BF16 ? launch_logits_t<__nv_bfloat16>(x, Wr, T, d, E, S, part, tickets, ntickets, sb, stream)
+                           : launch_logits_t<float>(x, Wr, T, d, E, S, part, tickets, ntickets, sb, stream);
+}
+
+cudaError_t launch_select_group(const float* part, int S, const float* br, int T, int E, int k, float scale,
+                                int32_t* idx, float* w, const GroupOut* g, cudaStream_t stream) {
+  GroupOut go{};
+  if (g != nullptr) go = *g;
+  return launch_pdl(select_group_kernel, dim3(1), dim3(kLogitThreads), 0, stream, part, S, br, T, E, k, scale,
+                    idx, w, go);
 }
 
 }  // namespace mova

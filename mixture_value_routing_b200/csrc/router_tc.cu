@@ -239,6 +239,7 @@ cudaError_t launch_router_tc(const void* x, const float* Wr, const float* br, in
   void* fp = encode_tiled_fn();
   if (fp == nullptr) return cudaErrorNotSupported;
   EncodeTiled enc = reinterpret_cast<EncodeTiled>(fp);
+  note_launch();
   split_router_kernel<<<2 * sm_count(), 256, 0, stream>>>(Wr, E, d, planes);
   cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess) return err;

@@ -21,6 +21,7 @@
 // exits.
 #include "common.cuh"
 #include "internal.h"
+#include "route_select.cuh"
 
 #include "sm100.cuh"
 
@@ -33,6 +34,13 @@ constexpr int kThreads = (kConsumerWarps + 1) * 32;  // warp 8 produces
 constexpr int kRowsPerStage = kConsumerWarps;
 constexpr int kTok = 8;
 constexpr int kMaxStages = 8;
+// More stages than this do not raise the streaming rate: the extra requests
+// in flight only queue in the memory system.
+constexpr int kStreamStages = 4;
+
+// Resident mode (bf16, T <= 8): the x rows of all tokens stay in shared
+// memory for the whole kernel.
+__host__ __device__ constexpr bool is_resident(bool mma, int T) { return mma && T <= kTok; }
 
 template <typename DT> struct Vec;
 template <> struct Vec<__nv_bfloat16> { static constexpr int EL = 8; };
@@ -91,30 +99,37 @@ stream_experts_kernel(const DT* __restrict__ x, const DT* __restrict__ Wv,
                       const int32_t* __restrict__ counts, const int32_t* __restrict__ offsets,
                       const int32_t* __restrict__ perm, const float* __restrict__ w32,
                       const int32_t* __restrict__ active, StatusBlock* __restrict__ sb, int T,
-                      int d, int n, int k, float* __restrict__ P, int NS) {
+                      int d, int n, int k, float* __restrict__ P, int NS,
+                      int32_t* __restrict__ tickets, DT* __restrict__ v, RouteIn route) {
   constexpr bool kMma = sizeof(DT) == 2;
   constexpr int EL = Vec<DT>::EL;
   extern __shared__ __align__(128) uint8_t smem[];
   const size_t row_bytes = static_cast<size_t>(d) * sizeof(DT);
   const size_t pitch = row_bytes + 16;
   const size_t stage_bytes = pitch * kRowsPerStage;
+  const bool resident = is_resident(kMma, T);
   uint8_t* stages = smem;
-  uint8_t* xs = smem + NS * stage_bytes;                    // bf16: kTok padded x rows
+  uint8_t* xs = smem + NS * stage_bytes;  // bf16: kTok padded x rows
   float* red = reinterpret_cast<float*>(xs + (kMma ? kTok * pitch : 0));  // [2][warps][8][8]
   float* tok_w = red + (kMma ? 2 * kConsumerWarps * 64 : 0);  // weights of the staged pairs
   int* tok_p = reinterpret_cast<int*>(tok_w + kTok);           // their grouped positions
-  // Resident mode (bf16, T <= 8): every token's x row stays in the x tile for
-  // the whole kernel, and the pair tables below replace all global loads of
-  // the grouping in the loop.
+  // Resident mode: every token's x row stays in the x tile for the whole
+  // kernel (the mma computes all 8 token columns for every expert; each pair
+  // reads its token's column), and the pair tables below replace all global
+  // loads of the grouping in the loop.
   int* pair_tok = tok_p + kTok;          // [64] token of each grouped position
   float* pair_w = reinterpret_cast<float*>(pair_tok + 64);  // [64] its weight
   int* act_cnt = reinterpret_cast<int*>(pair_w + 64);       // [64] pairs per active expert
   int* act_off = act_cnt + 64;                              // [64] first position
-  uint64_t* full = reinterpret_cast<uint64_t*>(act_off + 64);
+  int* slot_pos = act_off + 64;                             // [64] grouped position of pair f
+  float* slot_w = reinterpret_cast<float*>(slot_pos + 64);  // [64] weight of pair f
+  uint64_t* full = reinterpret_cast<uint64_t*>(slot_w + 64);
   uint64_t* empty = full + kMaxStages;
-  int* act = reinterpret_cast<int*>(empty + kMaxStages);
+  uint64_t* xbar = empty + kMaxStages;  // resident x rows landed
+  int* act = reinterpret_cast<int*>(xbar + 2);
   volatile int* abort_flag = act + 64;
   int* issued = act + 65;
+  int* blk_tick = act + 66;  // [64] completion counts of this CTA's row blocks (fused combine)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -123,19 +138,66 @@ stream_experts_kernel(const DT* __restrict__ x, const DT* __restrict__ Wv,
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], kConsumerWarps);
     }
+    mbar_init(xbar, 1);
     *abort_flag = 0;
     *issued = 0;
     fence_barrier_init();
   }
   pdl_wait();  // routing and grouping of this call are complete and visible
-  const int nact = sb->num_active;
-  if (threadIdx.x < 64) act[threadIdx.x] = (threadIdx.x < nact) ? active[threadIdx.x] : 0;
+  if (resident && threadIdx.x == 0) {
+    // The resident x tile: one bulk copy per token row, issued at once so its
+    // latency overlaps the first weight stages.
+    const uint32_t row_bytes_x = static_cast<uint32_t>(row_bytes);
+    mbar_arrive_expect_tx(xbar, static_cast<uint32_t>(T) * row_bytes_x);
+    for (int t = 0; t < T; ++t)
+      bulk_g2s(xs + t * pitch, x + static_cast<size_t>(t) * d, row_bytes_x, xbar, policy_evict_last());
+  }
+  // Route mode: the consumer warps select and group the batch from the
+  // partial logits (every CTA the same, in the same fixed order).
+  __shared__ float r_lg[kTok * 64];
+  __shared__ float r_br[64];
+  __shared__ int r_sel[kTok * 8];
+  __shared__ float r_w[kTok * 8];
+  __shared__ int r_scratch[128];
+  __shared__ int32_t r_cnt[64], r_off[65], r_pos[64], r_perm[64];
+  __shared__ int r_nact;
+  const bool routing = route.part != nullptr;
+  if (routing) {
+    if (threadIdx.x < kConsumerWarps * 32) {
+      for (int j = threadIdx.x; j < T * 64; j += kConsumerWarps * 32) {
+        float lv = route.part[j];
+        for (int r = 1; r < route.S; ++r) lv += route.part[r * kTok * 64 + j];
+        r_lg[j] = lv;
+      }
+      if (threadIdx.x < 64) r_br[threadIdx.x] = threadIdx.x < route.E ? route.br[threadIdx.x] : 0.f;
+      consumers_sync();
+      if (warp < T)
+        select_token(&r_lg[warp * 64], r_br, route.E, k, route.scale, warp, lane, r_sel, r_w,
+                     blockIdx.x == 0 ? route.idx_out : nullptr, route.w_out);
+      consumers_sync();
+      if (warp == 0) {
+        const int na = group_pairs_warp(r_sel, T * k, route.E, lane, r_scratch, r_cnt, r_off, r_pos,
+                                        r_perm, act);
+        if (lane == 0) r_nact = na;
+      }
+    }
+  } else {
+    const int na = sb->num_active;
+    if (threadIdx.x < 64) act[threadIdx.x] = (threadIdx.x < na) ? active[threadIdx.x] : 0;
+  }
   __syncthreads();
+  const int nact = routing ? r_nact : sb->num_active;
   pdl_trigger();
-  const bool resident = kMma && T <= kTok;
 
   // Rows of all active experts, in units of whole stages (n % 8 == 0, so a
-  // stage never straddles two experts), split evenly over the CTAs.
+  // stage never straddles two experts), split evenly over the CTAs.  With
+  // the combine fused in (v given; only in resident mode), units run
+  // row-block-major -- unit u is row block u / nact of active expert
+  // u % nact -- so a row block's units sit in one or two neighbouring CTAs
+  // and the one that completes it last also combines it: it owns every
+  // slot's expert row for those 8 output columns.  Otherwise units run
+  // expert-major, so the staged x rows change only with the expert.
+  const bool fused = v != nullptr;
   const int units_per_expert = n / kRowsPerStage;
   const int units = nact * units_per_expert;
   const int u0 = static_cast<int>(static_cast<long long>(units) * blockIdx.x / gridDim.x);
@@ -155,8 +217,8 @@ stream_experts_kernel(const DT* __restrict__ x, const DT* __restrict__ Wv,
         }
         if (*abort_flag) break;
         const int u = u0 + j;
-        const int a = u / units_per_expert;
-        const int r = (u - a * units_per_expert) * kRowsPerStage;
+        const int a = fused ? u % nact : u / units_per_expert;
+        const int r = (fused ? u / nact : u - a * units_per_expert) * kRowsPerStage;
         const DT* src = Wv + (static_cast<size_t>(act[a]) * n + r) * d;
         mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(kRowsPerStage * row_bytes));
         uint8_t* dst = stages + s * stage_bytes;
@@ -171,24 +233,27 @@ stream_experts_kernel(const DT* __restrict__ x, const DT* __restrict__ Wv,
     int cur_a = -1, cnt = 0, off = 0;
     int staged_a = -1, staged_c0 = -1;  // whose x rows the x tile holds
     int rbuf = 0;
+    const int ksteps = d / 16;
+    const int kb = ksteps * warp / kConsumerWarps;
+    const int ke = ksteps * (warp + 1) / kConsumerWarps;
     if (resident) {
-      // Overlaps the producer's first bulk copies.
-      const int vec_per_row = static_cast<int>(row_bytes / 16);
-      for (int i = threadIdx.x; i < T * vec_per_row; i += kConsumerWarps * 32) {
-        const int t = i / vec_per_row;
-        const int v = i - t * vec_per_row;
-        *reinterpret_cast<uint4*>(xs + t * pitch + v * 16) =
-            reinterpret_cast<const uint4*>(x + static_cast<size_t>(t) * d)[v];
-      }
+      // Pair tables, while x and the first weight stages are in flight.
       const int N = T * k;
       if (threadIdx.x < N) {
-        const int f = perm[threadIdx.x];
+        const int f = routing ? r_perm[threadIdx.x] : perm[threadIdx.x];
+        const float wf = routing ? r_w[f] : w32[f];
         pair_tok[threadIdx.x] = f / k;
-        pair_w[threadIdx.x] = w32[f];
+        pair_w[threadIdx.x] = wf;
+        slot_pos[f] = threadIdx.x;
+        slot_w[f] = wf;
       }
       if (threadIdx.x < nact) {
-        act_cnt[threadIdx.x] = counts[act[threadIdx.x]];
-        act_off[threadIdx.x] = offsets[act[threadIdx.x]];
+        act_cnt[threadIdx.x] = routing ? r_cnt[act[threadIdx.x]] : counts[act[threadIdx.x]];
+        act_off[threadIdx.x] = routing ? r_off[act[threadIdx.x]] : offsets[act[threadIdx.x]];
+      }
+      if (!mbar_wait(xbar, 0)) {
+        raise_status(sb, MOVA_ERR_TIMEOUT, blockIdx.x);
+        *abort_flag = 1;
       }
       consumers_sync();
     }
@@ -201,8 +266,8 @@ stream_experts_kernel(const DT* __restrict__ x, const DT* __restrict__ Wv,
         break;
       }
       const int u = u0 + j;
-      const int a = u / units_per_expert;
-      const int r0 = (u - a * units_per_expert) * kRowsPerStage;
+      const int a = fused ? u % nact : u / units_per_expert;
+      const int r0 = (fused ? u / nact : u - a * units_per_expert) * kRowsPerStage;
       if (a != cur_a) {
         cur_a = a;
         cnt = resident ? act_cnt[a] : counts[act[a]];
@@ -235,15 +300,11 @@ stream_experts_kernel(const DT* __restrict__ x, const DT* __restrict__ Wv,
             consumers_sync();
           }
           // This warp's K slice, in 16-element steps.
-          const int ksteps = d / 16;
-          const int kb = ksteps * warp / kConsumerWarps;
-          const int ke = ksteps * (warp + 1) / kConsumerWarps;
           float acc[4] = {0.f, 0.f, 0.f, 0.f};
           const int lr = lane & 7;
           const int lk = (lane >> 3) & 1;
           const uint32_t a_base = smem_u32(wst) + lr * static_cast<uint32_t>(pitch) + lk * 16;
-          const int b_row = resident ? pair_tok[off + c0 + min(lr, nt - 1)] : lr;
-          const uint32_t b_base = smem_u32(xs) + b_row * static_cast<uint32_t>(pitch) + lk * 16;
+          const uint32_t b_base = smem_u32(xs) + lr * static_cast<uint32_t>(pitch) + lk * 16;
 #pragma unroll 4
           for (int ks = kb; ks < ke; ++ks) {
             uint32_t a0, a2, b0, b1;
@@ -266,9 +327,10 @@ stream_experts_kernel(const DT* __restrict__ x, const DT* __restrict__ Wv,
             const int row = threadIdx.x >> 3;
             const int t = threadIdx.x & 7;
             if (t < nt) {
+              const int col = resident ? pair_tok[off + c0 + t] : t;  // the pair's token column
               float h = 0.f;
 #pragma unroll
-              for (int w = 0; w < kConsumerWarps; ++w) h += rb[(w * 8 + row) * 8 + t];
+              for (int w = 0; w < kConsumerWarps; ++w) h += rb[(w * 8 + row) * 8 + col];
               const int p = resident ? off + c0 + t : tok_p[t];
               P[static_cast<size_t>(p) * n + r0 + row] = siluf_(h);
             }
@@ -318,6 +380,42 @@ stream_experts_kernel(const DT* __restrict__ x, const DT* __restrict__ Wv,
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[s]);
     }
+    if (fused && nstages > 0 && !*abort_flag) {
+      // Fused combine.  This CTA's rows of P are complete: publish them, then
+      // count them on the tickets of the row blocks they belong to; the CTA
+      // that completes a block's count sums the slots of every token for its
+      // 8 columns,
+      //   v[t, r] = sum over slots (ascending) of w[t, slot] * P[pos[t, slot], r].
+      // Done once at the end, so the weight stream never waits for it.
+      __threadfence();
+      consumers_sync();
+      const int jb = u0 / nact;
+      const int je = (u1 - 1) / nact;
+      for (int j0 = jb; j0 <= je; j0 += 64) {
+        const int nb = min(64, je - j0 + 1);
+        if (threadIdx.x < nb) {
+          const int jj = j0 + threadIdx.x;
+          const int done = min(u1, (jj + 1) * nact) - max(u0, jj * nact);
+          blk_tick[threadIdx.x] = atomicAdd(&tickets[jj], done) + done;
+        }
+        consumers_sync();
+        __threadfence();
+        for (int i = threadIdx.x; i < nb * kTok * kRowsPerStage; i += kConsumerWarps * 32) {
+          const int bi = i / (kTok * kRowsPerStage);
+          const int t = (i / kRowsPerStage) % kTok;
+          const int row = i % kRowsPerStage;
+          if (blk_tick[bi] != nact || t >= T) continue;
+          const int col = (j0 + bi) * kRowsPerStage + row;
+          float acc = 0.f;
+          for (int sl = 0; sl < k; ++sl) {
+            const float pv = __ldcg(P + static_cast<size_t>(slot_pos[t * k + sl]) * n + col);
+            acc = fmaf(slot_w[t * k + sl], pv, acc);
+          }
+          v[static_cast<size_t>(t) * n + col] = from_f32<DT>(acc);
+        }
+        consumers_sync();
+      }
+    }
   }
   __syncthreads();
   // No bulk copy may still be writing this CTA's shared memory at exit: wait
@@ -325,33 +423,41 @@ stream_experts_kernel(const DT* __restrict__ x, const DT* __restrict__ Wv,
   if (threadIdx.x == kConsumerWarps * 32) {
     const int done = *issued;
     for (int j = max(0, done - NS); j < done; ++j) mbar_wait(&full[j % NS], (j / NS) & 1);
+    if (resident) mbar_wait(xbar, 0);
   }
 }
 
 }  // namespace
 
-size_t stream_experts_smem(int d, mova_dtype dt, int* stages_out) {
+size_t stream_experts_smem(int d, mova_dtype dt, int T, int* stages_out) {
   const bool mma = dt == MOVA_BF16;
+  (void)T;
   const size_t pitch = static_cast<size_t>(d) * (mma ? 2 : 4) + 16;
   const size_t stage_bytes = pitch * kRowsPerStage;
   const size_t fixed = (mma ? kTok * pitch + 2 * kConsumerWarps * 64 * sizeof(float) : 0) +
-                       2 * kTok * sizeof(float) + 4 * 64 * sizeof(int) +
-                       2 * kMaxStages * sizeof(uint64_t) + 66 * sizeof(int);
+                       2 * kTok * sizeof(float) + 6 * 64 * sizeof(int) +
+                       (2 * kMaxStages + 2) * sizeof(uint64_t) + 130 * sizeof(int);
   const size_t budget = 220 * 1024;
   int NS = fixed < budget ? static_cast<int>((budget - fixed) / stage_bytes) : 0;
-  if (NS > kMaxStages) NS = kMaxStages;
+  if (NS > kStreamStages) NS = kStreamStages;
   if (stages_out) *stages_out = NS;
   if (NS < 2) return 0;
   return NS * stage_bytes + fixed;
 }
 
+bool stream_resident(int T, int d, mova_dtype dt) {
+  (void)d;
+  return is_resident(dt == MOVA_BF16, T);
+}
+
 cudaError_t launch_stream_experts(const void* x, const void* Wv, mova_dtype dt, const int32_t* counts,
                                   const int32_t* offsets, const int32_t* perm, const float* w32,
                                   const int32_t* active, StatusBlock* sb, int T, int d, int n,
-                                  int k, int E, float* P, cudaStream_t stream) {
+                                  int k, int E, float* P, int32_t* tickets, void* v,
+                                  const RouteIn& route, cudaStream_t stream) {
   (void)E;
   int NS = 0;
-  const size_t smem = stream_experts_smem(d, dt, &NS);
+  const size_t smem = stream_experts_smem(d, dt, T, &NS);
   if (smem == 0) return cudaErrorInvalidValue;
   const dim3 grid(sm_count());
   if (dt == MOVA_BF16) {
@@ -361,7 +467,8 @@ cudaError_t launch_stream_experts(const void* x, const void* Wv, mova_dtype dt, 
     if (err != cudaSuccess) return err;
     return launch_pdl(kern, grid, dim3(kThreads), smem, stream,
                       static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(Wv),
-                      counts, offsets, perm, w32, active, sb, T, d, n, k, P, NS);
+                      counts, offsets, perm, w32, active, sb, T, d, n, k, P, NS, tickets,
+                      static_cast<__nv_bfloat16*>(v), route);
   }
   auto kern = stream_experts_kernel<float>;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -369,7 +476,7 @@ cudaError_t launch_stream_experts(const void* x, const void* Wv, mova_dtype dt, 
   if (err != cudaSuccess) return err;
   return launch_pdl(kern, grid, dim3(kThreads), smem, stream, static_cast<const float*>(x),
                     static_cast<const float*>(Wv), counts, offsets, perm, w32, active, sb, T, d, n,
-                    k, P, NS);
+                    k, P, NS, tickets, static_cast<float*>(v), route);
 }
 
 }  // namespace mova

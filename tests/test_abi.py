@@ -93,3 +93,12 @@ def test_host_side_validation(lib):
     assert st == _lib.OK
     st = lib.mova_get_status(None, None, None)
     assert st == _lib.ERR_INVALID_ARG
+
+
+def test_launch_counter_ignores_rejected_calls(lib):
+    # A call rejected on the host enqueues nothing, so the counter is unchanged.
+    before = lib.mova_launch_count()
+    st = lib.mova_value_routed(None, _lib.BF16, None, None, None, _lib.BF16, 8, 2560, 64, 4, 1024,
+                               ctypes.c_float(2.5), None, None, None, None, 0, None)
+    assert st == _lib.ERR_INVALID_ARG
+    assert lib.mova_launch_count() == before

@@ -202,6 +202,13 @@ def test_full_edge_shapes(api, T, E, k, n):
     _full(api, T, 256, E, k, n, "bf16", seed=T)
 
 
+@pytest.mark.parametrize("T,d", [(8, 3072), (4, 4096), (3, 4544)])
+def test_full_stream_resident_boundary(api, T, d):
+    """Decode batches at and near the widest rows the weight-streaming
+    kernel holds (two stages of 8 rows plus the resident x tile)."""
+    _full(api, T, d, 16, 4, 256, "bf16", seed=d, path="stream")
+
+
 @pytest.mark.parametrize("T", [24, 64])
 def test_full_stream_mid(api, T):
     """Weight-streaming path with more than 8 tokens on some experts."""
@@ -315,3 +322,19 @@ def test_deterministic(api):
     first = api.value_routed(*args).clone()
     for _ in range(9):
         assert torch.equal(api.value_routed(*args), first)
+
+
+def test_decode_step_kernel_count(api):
+    """A bf16 decode step is two kernels: the router logits and the
+    weight-streaming experts (which also select, group and combine); fp32
+    runs selection/grouping and the combine as kernels of their own."""
+    for dtype, want in (("bf16", 2), ("f32", 4)):
+        lay = _layer(5, 2560, 64, 1024, dtype)
+        bat = MI.make_batch(8, 5, dtype=dtype)
+        args = (P.dev(bat.x, dtype), P.dev(lay.Wr, "f32"), P.dev(lay.br, "f32"), P.dev(lay.Wv, dtype))
+        api.value_routed(*args)
+        torch.cuda.synchronize()
+        before = api.launch_count()
+        api.value_routed(*args)
+        assert api.launch_count() - before == want, dtype
+    torch.cuda.synchronize()
