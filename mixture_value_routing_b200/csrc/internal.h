@@ -82,6 +82,7 @@ void* encode_tiled_fn();
 // `planes`, router_planes_bytes(d) bytes), then one CTA per 128 tokens
 // computes the logits with tcgen05 and selects; tile_counts (nullable)
 // receives each 128-token tile's expert histogram.
+constexpr int kTcRouterMinT = 64;  // bf16 batches above this many tokens use it
 size_t router_planes_bytes(int d);
 cudaError_t launch_router_tc(const void* x, const float* Wr, const float* br, int T, int d, int E,
                              int k, float scale, int32_t* idx, float* w, int32_t* tile_counts,

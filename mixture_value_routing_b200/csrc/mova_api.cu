@@ -52,8 +52,6 @@ namespace {
 
 // AUTO: bf16 batches above this many tokens use the tcgen05 grouped GEMM.
 constexpr int kStreamMaxTokens = 64;
-// bf16 batches above this many tokens use the tensor-core router.
-constexpr int kTcRouterMinT = 64;
 // bf16 batches up to this many tokens run the combine inside the
 // weight-streaming kernel (the x rows stay resident there).
 constexpr int kFusedCombineMaxT = 8;
@@ -93,9 +91,11 @@ Workspace layout(void* base, int T, int d, int k, int n) {
   w.perm = reinterpret_cast<int32_t*>(b + o);         o += align256(pairs * 4);
   w.pos = reinterpret_cast<int32_t*>(b + o);          o += align256(pairs * 4);
   w.tickets = reinterpret_cast<int32_t*>(b + o);      o += align256(static_cast<size_t>(n / 8) * 4);
-  w.logits = reinterpret_cast<float*>(b + o);         o += static_cast<size_t>(kMaxLogitSplits) * 8 * 64 * 4;
   w.tile_counts = reinterpret_cast<int32_t*>(b + o);  o += align256(static_cast<size_t>(group_tiles(T)) * 64 * 4);
   w.planes = reinterpret_cast<__nv_bfloat16*>(b + o); o += align256(router_planes_bytes(d));
+  // The decode partial logits (T <= 8, kMaxLogitSplits x 8 x 64 floats <= 192 * d * 2 bytes for
+  // d >= 64) share the router planes' bytes: the planes exist only for T > 64.
+  w.logits = reinterpret_cast<float*>(w.planes);
   w.xp = reinterpret_cast<__nv_bfloat16*>(b + o);     o += align256(pairs * static_cast<size_t>(d) * 2);
   w.P = b + o;                                        o += align256(pairs * static_cast<size_t>(n) * 4);
   w.bytes = o;

@@ -186,75 +186,71 @@ tile_hist_kernel(const IT* __restrict__ idx_in, const WT* __restrict__ w_in, int
   if (threadIdx.x < 64) tile_counts[blockIdx.x * 64 + threadIdx.x] = hist[threadIdx.x];
 }
 
-// One CTA: tile_counts[t][e] becomes the first grouped position of tile t's
-// pairs of expert e; writes counts, offsets, the active list and resets the
-// status block for this call.
-__global__ void __launch_bounds__(64)
-tile_scan_kernel(int32_t* __restrict__ tile_counts, int ntiles, int E, int32_t* __restrict__ counts,
-                 int32_t* __restrict__ offsets, int32_t* __restrict__ active, StatusBlock* sb,
-                 int N, bool reset_status) {
-  pdl_wait();
-  __shared__ int tot[64];
-  __shared__ int off[65];
-  const int e = threadIdx.x;
-  int s = 0;
-  if (e < E)
-    for (int t = 0; t < ntiles; ++t) s += tile_counts[t * 64 + e];
-  tot[e] = (e < E) ? s : 0;
-  __syncthreads();
-  if (e == 0) {
-    int acc = 0;
-    for (int q = 0; q < E; ++q) {
-      off[q] = acc;
-      acc += tot[q];
-    }
-    off[E] = acc;
-  }
-  __syncthreads();
-  if (e < E) {
-    int base = off[e];
-    for (int t = 0; t < ntiles; ++t) {
-      const int c = tile_counts[t * 64 + e];
-      tile_counts[t * 64 + e] = base;
-      base += c;
-    }
-    counts[e] = tot[e];
-    offsets[e] = off[e];
-  }
-  if (e == 0) offsets[E] = off[E];
-  const int lane = e & 31;
-  const unsigned lt = (1u << lane) - 1u;
-  const bool a = e < E && tot[e] > 0;
-  __shared__ unsigned m[2];
-  const unsigned mm = __ballot_sync(0xffffffffu, a);
-  if (lane == 0) m[e >> 5] = mm;
-  __syncthreads();
-  const int before = (e >= 32) ? __popc(m[0]) : 0;
-  if (a) active[before + __popc(mm & lt)] = e;
-  if (e == 0) {
-    if (reset_status) {
-      sb->code = 0;
-      sb->detail = 0;
-    }
-    sb->num_active = __popc(m[0]) + __popc(m[1]);
-    sb->work_next = 0;
-  }
-  (void)N;
-}
-
-// Stable scatter of one tile: 4 warps own consecutive segments of the tile's
-// pairs; per-warp histograms are scanned in warp order on top of the tile's
-// first positions, then each warp ranks 32 pairs at a time (earlier lanes with
-// the same expert come first).
+// Stable scatter of one tile.  Each CTA first derives, from every tile's
+// histogram, the expert totals, their exclusive prefix (the expert offsets)
+// and the number of its expert's pairs in earlier tiles, i.e. the first
+// grouped position of each of its experts (CTA 0 also writes counts,
+// offsets, the active list and the status fields).  Then 4 warps own
+// consecutive segments of the tile's pairs; per-warp histograms are scanned
+// in warp order on top of those positions, and each warp ranks 32 pairs at a
+// time (earlier lanes with the same expert come first).
 __global__ void __launch_bounds__(128)
-tile_scatter_kernel(const int32_t* __restrict__ idx32, int N, int k,
-                    const int32_t* __restrict__ tile_base, int32_t* __restrict__ perm,
-                    int32_t* __restrict__ pos) {
+tile_scatter_kernel(const int32_t* __restrict__ idx32, int N, int k, int E,
+                    const int32_t* __restrict__ tile_counts, int ntiles, int32_t* __restrict__ counts,
+                    int32_t* __restrict__ offsets, int32_t* __restrict__ active, StatusBlock* sb,
+                    bool reset_status, int32_t* __restrict__ perm, int32_t* __restrict__ pos) {
   pdl_wait();
   __shared__ int hist[4][64];
+  __shared__ int base[64];
+  __shared__ int tot_s[64];
+  __shared__ unsigned amask[2];
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   for (int i = threadIdx.x; i < 4 * 64; i += 128) (&hist[0][0])[i] = 0;
+  const unsigned lt_mask = (1u << lane) - 1u;
+  if (threadIdx.x < 64) {
+    // Thread e: the expert's total and its count in the tiles before this one.
+    const int e = threadIdx.x;
+    int tot = 0, before = 0;
+    if (e < E) {
+      for (int t = 0; t < ntiles; ++t) {
+        const int c = tile_counts[t * 64 + e];
+        tot += c;
+        before += (t < static_cast<int>(blockIdx.x)) ? c : 0;
+      }
+    }
+    // Exclusive prefix of the totals over experts (two warps).
+    int inc = tot;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, inc, o);
+      if (lane >= o) inc += y;
+    }
+    tot_s[e] = inc;  // inclusive within the warp
+    const unsigned am = __ballot_sync(0xffffffffu, e < E && tot > 0);
+    if (lane == 0) amask[warp] = am;
+    asm volatile("bar.sync 1, 64;" ::: "memory");  // the two scanning warps
+    const int warp0_total = tot_s[31];
+    const int off = inc - tot + (warp == 1 ? warp0_total : 0);
+    base[e] = off + before;
+    if (blockIdx.x == 0) {
+      if (e < E) {
+        counts[e] = tot;
+        offsets[e] = off;
+      }
+      if (e == E - 1) offsets[E] = off + tot;
+      const int nbefore = (warp == 1) ? __popc(amask[0]) : 0;
+      if (e < E && tot > 0) active[nbefore + __popc(am & lt_mask)] = e;
+      if (e == 0) {
+        if (reset_status) {
+          sb->code = 0;
+          sb->detail = 0;
+        }
+        sb->num_active = __popc(amask[0]) + __popc(amask[1]);
+        sb->work_next = 0;
+      }
+    }
+  }
   __syncthreads();
   const int per = kTileTok * k;
   const int t0 = blockIdx.x * per;
@@ -265,7 +261,7 @@ tile_scatter_kernel(const int32_t* __restrict__ idx32, int N, int k,
   for (int f = f_begin + lane; f < f_end; f += 32) atomicAdd(&hist[warp][idx32[f]], 1);
   __syncthreads();
   if (threadIdx.x < 64) {
-    int b = tile_base[blockIdx.x * 64 + threadIdx.x];
+    int b = base[threadIdx.x];
     for (int w = 0; w < 4; ++w) {
       const int c = hist[w][threadIdx.x];
       hist[w][threadIdx.x] = b;
@@ -273,7 +269,6 @@ tile_scatter_kernel(const int32_t* __restrict__ idx32, int N, int k,
     }
   }
   __syncthreads();
-  const unsigned lt_mask = (1u << lane) - 1u;
   for (int c0 = f_begin; c0 < f_end; c0 += 32) {
     const int f = c0 + lane;
     const bool valid = f < f_end;
@@ -356,12 +351,9 @@ cudaError_t launch_tile_group(const int32_t* idx32, int T, int E, int k, int32_t
                               cudaStream_t stream) {
   const int N = T * k;
   const int ntiles = group_tiles(T);
-  cudaError_t err = launch_pdl(tile_scan_kernel, dim3(1), dim3(64), 0, stream, tile_counts, ntiles,
-                               E, counts, offsets, active, sb, N, reset_status);
-  if (err != cudaSuccess) return err;
-  return launch_pdl(tile_scatter_kernel, dim3(ntiles), dim3(128), 0, stream,
-                    static_cast<const int32_t*>(idx32), N, k,
-                    static_cast<const int32_t*>(tile_counts), perm, pos);
+  return launch_pdl(tile_scatter_kernel, dim3(ntiles), dim3(128), 0, stream, idx32, N, k, E,
+                    static_cast<const int32_t*>(tile_counts), ntiles, counts, offsets, active, sb,
+                    reset_status, perm, pos);
 }
 
 }  // namespace mova

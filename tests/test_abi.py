@@ -102,3 +102,11 @@ def test_launch_counter_ignores_rejected_calls(lib):
                                ctypes.c_float(2.5), None, None, None, None, 0, None)
     assert st == _lib.ERR_INVALID_ARG
     assert lib.mova_launch_count() == before
+
+
+def test_noalloc_scratch_admits_the_documented_batch(lib):
+    # include/mova.h: the built-in 2 MiB workspace admits T <= 30 at the
+    # decode dimensions (d = 2560, E = 64, k = 4, n = 1024).
+    scratch = 2 << 20
+    assert lib.mova_workspace_size(30, 2560, 64, 4, 1024) <= scratch
+    assert lib.mova_workspace_size(31, 2560, 64, 4, 1024) > scratch
