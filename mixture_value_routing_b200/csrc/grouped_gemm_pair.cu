@@ -23,6 +23,12 @@
 //     accumulator with a remote arrive on the even CTA's barrier.
 //   * Warps: 0 TMA, 1 MMA (even CTA), 2-5 epilogue (SiLU, bf16, store; rows
 //     beyond the expert's n are skipped).
+//   * One persistent pair per two SMs takes tiles from a global counter as
+//     it goes (the even CTA's producer fetches the id and publishes it to
+//     every role of both CTAs through a ring of mbarrier-guarded slots), so
+//     unequal tile sizes do not leave some pairs a whole tile behind.  Tile
+//     ids run expert by expert with the 4 weight-row tiles of a token tile
+//     adjacent, so pairs working at the same time share the token rows in L2.
 // Every mbarrier wait is bounded (MOVA_ERR_TIMEOUT); both CTAs meet at a
 // cluster barrier before tensor memory is freed.
 #include <cuda.h>
@@ -39,6 +45,11 @@ constexpr int PM = 128;          // weight rows per CTA (256 per pair)
 constexpr int PN = 256;          // pairs per tile
 constexpr int PK = 64;
 constexpr int kPStages = 6;
+// Tile ids handed out dynamically pass through a ring in both CTAs'
+// shared memory.  A role can lag the leader's producer by at most 8 tiles:
+// the producer leads the MMA by at most kPStages k-steps (so at most 6
+// tiles), the MMA leads the epilogues by the 2 accumulators.
+constexpr int kTileRing = 16;
 constexpr int kPABytes = PM * PK * 2;
 constexpr int kPBBytes = (PN / 2) * PK * 2;
 constexpr int kPStageBytes = kPABytes + kPBBytes;
@@ -52,6 +63,8 @@ struct __align__(1024) PSmem {
   uint64_t empty[kPStages];  // both CTAs: the pair's MMAs on the stage are done
   uint64_t tmem_full[2];     // both CTAs
   uint64_t tmem_empty[2];    // even CTA: 4 epilogue warps x 2 CTAs
+  uint64_t tq_full[kTileRing];  // both CTAs: tile id i of this cluster published
+  int tq[kTileRing];
   uint32_t tmem_base;
   int abort;
   int ntiles;
@@ -84,6 +97,14 @@ __device__ __forceinline__ PTile decode_ptile(const PSmem& S, int t, int mtiles)
   return r;
 }
 
+// The cluster's i-th tile id (waits until the even CTA's producer has
+// published it; ntiles or more means no more tiles).  -1 if the wait ran out.
+__device__ __forceinline__ int next_tile(PSmem& S, int i) {
+  const int slot = i % kTileRing;
+  if (!mbar_wait(&S.tq_full[slot], (i / kTileRing) & 1)) return -1;
+  return *reinterpret_cast<volatile int*>(&S.tq[slot]);
+}
+
 __device__ __forceinline__ bool p_aborted(const PSmem& S) {
   return *reinterpret_cast<const volatile int*>(&S.abort) != 0;
 }
@@ -102,8 +123,6 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_w, const __gri
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const uint32_t rank = cluster_rank();
-  const int cid = blockIdx.x >> 1;
-  const int nclusters = gridDim.x >> 1;
   const int mtiles = (n + 2 * PM - 1) / (2 * PM);
   const int nk = d / PK;
 
@@ -116,6 +135,7 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_w, const __gri
       mbar_init(&S.tmem_full[i], 1);
       mbar_init(&S.tmem_empty[i], 8);
     }
+    for (int i = 0; i < kTileRing; ++i) mbar_init(&S.tq_full[i], 1);
     S.abort = 0;
     fence_barrier_init();
   }
@@ -167,7 +187,27 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_w, const __gri
   if (warp == 0) {
     if (lane == 0) {
       int it = 0;
-      for (int t = cid; t < ntiles && !p_aborted(S); t += nclusters) {
+      // Tiles are handed out one at a time from a counter (zeroed by the
+      // grouping of this call), so the clusters finish together however the
+      // tile sizes fall.  The even CTA's producer takes each id and publishes
+      // it to both CTAs; it requests the following id while it loads a tile.
+      int next = (rank == 0) ? atomicAdd(&sb->work_next, 1) : 0;
+      for (int i = 0;; ++i) {
+        int t;
+        if (rank == 0) {
+          t = p_aborted(S) ? ntiles : next;
+          const int slot = i % kTileRing;
+          S.tq[slot] = t;
+          st_cluster_u32(mapa_shared(smem_u32(&S.tq[slot]), 1), static_cast<uint32_t>(t));
+          mbar_arrive_cluster(mapa_shared(smem_u32(&S.tq_full[slot]), 1));
+          mbar_arrive(&S.tq_full[slot]);
+          if (t >= ntiles) break;
+          next = atomicAdd(&sb->work_next, 1);
+        } else {
+          t = next_tile(S, i);
+          if (t < 0) { p_fail(S, sb); break; }
+          if (t >= ntiles) break;
+        }
         const PTile tl = decode_ptile(S, t, mtiles);
         const int arow = tl.e * n + tl.mt * 2 * PM + static_cast<int>(rank) * PM;
         const int half = tl.N / 2;
@@ -187,30 +227,58 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_w, const __gri
       }
     }
   } else if (warp == 1) {
-    if (rank == 0 && lane == 0) {
-      int it = 0, titer = 0;
-      for (int t = cid; t < ntiles && !p_aborted(S); t += nclusters, ++titer) {
+    if (rank == 0) {
+      // The whole warp runs the loop (so its state stays warp-uniform); one
+      // elected lane issues the MMAs and commits.  Stage descriptors are
+      // built once and advanced by adding offsets (start address in 16-byte
+      // units), which keeps the issue cost below the MMA time even at
+      // N = 144.
+      const uint64_t adesc0 = smem_desc_sw128(smem_u32(S.stage[0]));
+      const uint64_t bdesc0 = smem_desc_sw128(smem_u32(S.stage[0]) + kPABytes);
+      constexpr uint32_t kStageDesc = kPStageBytes >> 4;
+      int s = 0;
+      uint32_t phase = 0;
+      for (int titer = 0;; ++titer) {
+        const int t = next_tile(S, titer);
+        if (t < 0) {
+          if (lane == 0) p_fail(S, sb);
+          break;
+        }
+        if (t >= ntiles || p_aborted(S)) break;
         const PTile tl = decode_ptile(S, t, mtiles);
         const int acc = titer & 1;
-        if (titer >= 2 && !mbar_wait(&S.tmem_empty[acc], ((titer / 2) - 1) & 1)) { p_fail(S, sb); break; }
+        if (titer >= 2 && !__all_sync(0xffffffffu, mbar_wait(&S.tmem_empty[acc], ((titer / 2) - 1) & 1))) {
+          if (lane == 0) p_fail(S, sb);
+          break;
+        }
         tc_fence_after();
         const uint32_t d_tmem = S.tmem_base + static_cast<uint32_t>(acc * PN);
         const uint32_t idesc = idesc_bf16_f32(2 * PM, tl.N);
         bool ok = true;
-        for (int kb = 0; kb < nk; ++kb, ++it) {
-          const int s = it % kPStages;
-          if (!mbar_wait(&S.full[s], (it / kPStages) & 1)) { p_fail(S, sb); ok = false; break; }
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!__all_sync(0xffffffffu, mbar_wait(&S.full[s], phase))) {
+            if (lane == 0) p_fail(S, sb);
+            ok = false;
+            break;
+          }
           tc_fence_after();
-          const uint32_t a0 = smem_u32(S.stage[s]);
-          const uint32_t b0 = a0 + kPABytes;
+          const uint64_t da = adesc0 + static_cast<uint64_t>(s) * kStageDesc;
+          const uint64_t db = bdesc0 + static_cast<uint64_t>(s) * kStageDesc;
+          if (elect_one()) {
 #pragma unroll
-          for (int k16 = 0; k16 < PK / 16; ++k16)
-            tc_mma_bf16_pair(d_tmem, smem_desc_sw128(a0 + k16 * 32), smem_desc_sw128(b0 + k16 * 32), idesc,
-                             (kb | k16) != 0);
-          tc_commit_pair_both(&S.empty[s]);
+            for (int k16 = 0; k16 < PK / 16; ++k16)
+              tc_mma_bf16_pair(d_tmem, da + 2 * k16, db + 2 * k16, idesc, (kb | k16) != 0);
+            tc_commit_pair_both(&S.empty[s]);
+          }
+          __syncwarp();
+          if (++s == kPStages) {
+            s = 0;
+            phase ^= 1;
+          }
         }
         if (!ok) break;
-        tc_commit_pair_both(&S.tmem_full[acc]);
+        if (elect_one()) tc_commit_pair_both(&S.tmem_full[acc]);
+        __syncwarp();
       }
     }
   } else {
@@ -218,7 +286,10 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_w, const __gri
     const uint32_t empty0 = mapa_shared(smem_u32(&S.tmem_empty[0]), 0);
     const uint32_t empty1 = mapa_shared(smem_u32(&S.tmem_empty[1]), 0);
     int titer = 0;
-    for (int t = cid; t < ntiles && !p_aborted(S); t += nclusters, ++titer) {
+    for (;; ++titer) {
+      const int t = next_tile(S, titer);
+      if (t < 0) { p_fail(S, sb); break; }
+      if (t >= ntiles || p_aborted(S)) break;
       const PTile tl = decode_ptile(S, t, mtiles);
       const int acc = titer & 1;
       if (!mbar_wait(&S.tmem_full[acc], (titer / 2) & 1)) { p_fail(S, sb); break; }

@@ -119,28 +119,37 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_consta
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      const uint32_t idesc = idesc_bf16_f32(RM, RN);
-      bool ok = true;
-      for (int kb = 0; kb < nk; ++kb) {
-        const int s = kb % kRStages;
-        if (!mbar_wait(&S.full[s], (kb / kRStages) & 1)) {
+    // The whole warp runs the loop; one elected lane issues the MMAs.  Stage
+    // descriptors are built once and advanced by adding offsets (16-byte
+    // units), so issuing stays cheaper than the MMAs themselves.
+    const uint32_t idesc = idesc_bf16_f32(RM, RN);
+    const uint64_t adesc0 = smem_desc_sw128(smem_u32(S.stage[0]));
+    const uint64_t bdesc0 = smem_desc_sw128(smem_u32(S.stage[0]) + kRABytes);
+    constexpr uint32_t kStageDesc = kRStageBytes >> 4;
+    bool ok = true;
+    for (int kb = 0; kb < nk; ++kb) {
+      const int s = kb % kRStages;
+      if (!__all_sync(0xffffffffu, mbar_wait(&S.full[s], (kb / kRStages) & 1))) {
+        if (lane == 0) {
           raise_status(sb, MOVA_ERR_TIMEOUT, blockIdx.x);
           S.abort = 1;
-          ok = false;
-          break;
         }
-        tc_fence_after();
-        const uint32_t a0 = smem_u32(S.stage[s]);
-        const uint32_t b0 = a0 + kRABytes;
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint64_t da = adesc0 + static_cast<uint64_t>(s) * kStageDesc;
+      const uint64_t db = bdesc0 + static_cast<uint64_t>(s) * kStageDesc;
+      if (elect_one()) {
 #pragma unroll
         for (int k16 = 0; k16 < RK / 16; ++k16)
-          tc_mma_bf16(S.tmem_base, smem_desc_sw128(a0 + k16 * 32), smem_desc_sw128(b0 + k16 * 32), idesc,
-                      (kb | k16) != 0);
+          tc_mma_bf16(S.tmem_base, da + 2 * k16, db + 2 * k16, idesc, (kb | k16) != 0);
         tc_commit(&S.empty[s]);
       }
-      if (ok) tc_commit(&S.tmem_full);
+      __syncwarp();
     }
+    if (ok && elect_one()) tc_commit(&S.tmem_full);
+    __syncwarp();
   } else {
     // Epilogue: thread = token (TMEM lane).
     const int lg = warp & 3;

@@ -193,6 +193,22 @@ __device__ __forceinline__ void tma_load_2d_pair_hint(void* dst, const void* tma
       : "memory");
 }
 
+// True in exactly one lane of the (fully active) warp: the lane that issues
+// the warp's tensor-core or copy instructions while the whole warp runs the
+// loop around them, so loop state stays warp-uniform.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred = 0;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\telect.sync _|p, 0xffffffff;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(pred));
+  return pred != 0;
+}
+
+// 32-bit store into another CTA's shared memory (cluster address).
+__device__ __forceinline__ void st_cluster_u32(uint32_t addr_cluster, uint32_t v) {
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr_cluster), "r"(v) : "memory");
+}
+
 // Plain arrive on an mbarrier of another CTA of the cluster.
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar_cluster) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster)

@@ -164,12 +164,28 @@ stream_experts_kernel(const DT* __restrict__ x, const DT* __restrict__ Wv,
   const bool routing = route.part != nullptr;
   if (routing) {
     if (threadIdx.x < kConsumerWarps * 32) {
-      for (int j = threadIdx.x; j < T * 64; j += kConsumerWarps * 32) {
-        float lv = route.part[j];
-        for (int r = 1; r < route.S; ++r) lv += route.part[r * kTok * 64 + j];
-        r_lg[j] = lv;
+      // Every load of the partials and biases is issued before the first is
+      // used (one L2 round trip): thread i sums logits i and i + 256 over the
+      // S <= kMaxLogitSplits ranges in range order.
+      constexpr int kC = kConsumerWarps * 32;
+      static_assert(kTok * 64 == 2 * kC, "two logits per consumer thread");
+      float pv[2][kMaxLogitSplits];
+#pragma unroll
+      for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int r = 0; r < kMaxLogitSplits; ++r)
+          pv[h][r] = (r < route.S && threadIdx.x + h * kC < T * 64)
+                         ? route.part[r * kTok * 64 + threadIdx.x + h * kC] : 0.f;
+      const float bv = threadIdx.x < route.E ? route.br[threadIdx.x] : 0.f;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        float lv = pv[h][0];
+#pragma unroll
+        for (int r = 1; r < kMaxLogitSplits; ++r)
+          if (r < route.S) lv += pv[h][r];
+        r_lg[threadIdx.x + h * kC] = lv;
       }
-      if (threadIdx.x < 64) r_br[threadIdx.x] = threadIdx.x < route.E ? route.br[threadIdx.x] : 0.f;
+      if (threadIdx.x < 64) r_br[threadIdx.x] = bv;
       consumers_sync();
       if (warp < T)
         select_token(&r_lg[warp * 64], r_br, route.E, k, route.scale, warp, lane, r_sel, r_w,
