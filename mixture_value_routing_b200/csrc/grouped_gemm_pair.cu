@@ -185,46 +185,75 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_w, const __gri
   const int ntiles = S.ntiles;
 
   if (warp == 0) {
-    if (lane == 0) {
-      int it = 0;
-      // Tiles are handed out one at a time from a counter (zeroed by the
-      // grouping of this call), so the clusters finish together however the
-      // tile sizes fall.  The even CTA's producer takes each id and publishes
-      // it to both CTAs; it requests the following id while it loads a tile.
-      int next = (rank == 0) ? atomicAdd(&sb->work_next, 1) : 0;
-      for (int i = 0;; ++i) {
-        int t;
-        if (rank == 0) {
-          t = p_aborted(S) ? ntiles : next;
+    // The whole warp runs the loop (warp-uniform state); one elected lane
+    // issues the copies.  Stage and barrier addresses are computed once.
+    // Tiles are handed out one at a time from a counter (zeroed by the
+    // grouping of this call), so the clusters finish together however the
+    // tile sizes fall.  The even CTA's producer takes each id and publishes it
+    // to both CTAs; it requests the following id while it loads a tile.
+    const uint32_t full0_cl = mapa_shared(smem_u32(&S.full[0]), 0);  // even CTA's barriers
+    int s = 0;
+    uint32_t phase = 0;
+    bool started = false;
+    int next = 0;
+    if (rank == 0) {
+      if (lane == 0) next = atomicAdd(&sb->work_next, 1);
+      next = __shfl_sync(0xffffffffu, next, 0);
+    }
+    for (int i = 0;; ++i) {
+      int t;
+      if (rank == 0) {
+        t = p_aborted(S) ? ntiles : next;
+        if (elect_one()) {
           const int slot = i % kTileRing;
           S.tq[slot] = t;
           st_cluster_u32(mapa_shared(smem_u32(&S.tq[slot]), 1), static_cast<uint32_t>(t));
           mbar_arrive_cluster(mapa_shared(smem_u32(&S.tq_full[slot]), 1));
           mbar_arrive(&S.tq_full[slot]);
-          if (t >= ntiles) break;
-          next = atomicAdd(&sb->work_next, 1);
-        } else {
-          t = next_tile(S, i);
-          if (t < 0) { p_fail(S, sb); break; }
-          if (t >= ntiles) break;
         }
-        const PTile tl = decode_ptile(S, t, mtiles);
-        const int arow = tl.e * n + tl.mt * 2 * PM + static_cast<int>(rank) * PM;
-        const int half = tl.N / 2;
-        const int brow = tl.off + tl.tok0 + static_cast<int>(rank) * half;
-        const int nbox = (half + kPBoxRows - 1) / kPBoxRows;
-        const uint32_t bytes = 2u * static_cast<uint32_t>(kPABytes + nbox * kPBoxRows * PK * 2);
-        for (int kb = 0; kb < nk; ++kb, ++it) {
-          const int s = it % kPStages;
-          if (it >= kPStages && !mbar_wait(&S.empty[s], ((it / kPStages) - 1) & 1)) { p_fail(S, sb); break; }
-          const uint32_t full0 = mapa_shared(smem_u32(&S.full[s]), 0);
+        __syncwarp();
+        if (t >= ntiles) break;
+        if (lane == 0) next = atomicAdd(&sb->work_next, 1);  // read back at the next tile
+        next = __shfl_sync(0xffffffffu, next, 0);
+      } else {
+        t = next_tile(S, i);
+        if (t < 0) {
+          if (lane == 0) p_fail(S, sb);
+          break;
+        }
+        if (t >= ntiles) break;
+      }
+      const PTile tl = decode_ptile(S, t, mtiles);
+      const int arow = tl.e * n + tl.mt * 2 * PM + static_cast<int>(rank) * PM;
+      const int half = tl.N / 2;
+      const int brow = tl.off + tl.tok0 + static_cast<int>(rank) * half;
+      const int nbox = (half + kPBoxRows - 1) / kPBoxRows;
+      const uint32_t bytes = 2u * static_cast<uint32_t>(kPABytes + nbox * kPBoxRows * PK * 2);
+      bool ok = true;
+      for (int kb = 0; kb < nk; ++kb) {
+        // Slot s was used before (from the second pass over the ring on):
+        // wait until the MMAs reading it have completed.
+        if (started && !__all_sync(0xffffffffu, mbar_wait(&S.empty[s], phase ^ 1))) {
+          if (lane == 0) p_fail(S, sb);
+          ok = false;
+          break;
+        }
+        if (elect_one()) {
+          const uint32_t full_cl = full0_cl + static_cast<uint32_t>(s) * 8u;
           if (rank == 0) mbar_arrive_expect_tx(&S.full[s], bytes);
-          tma_load_2d_pair(S.stage[s], &tmap_w, kb * PK, arow, full0);
+          uint8_t* st = S.stage[s];
+          tma_load_2d_pair(st, &tmap_w, kb * PK, arow, full_cl);
           for (int b = 0; b < nbox; ++b)
-            tma_load_2d_pair(S.stage[s] + kPABytes + b * kPBoxRows * 128, &tmap_xp, kb * PK,
-                             brow + b * kPBoxRows, full0);
+            tma_load_2d_pair(st + kPABytes + b * kPBoxRows * 128, &tmap_xp, kb * PK, brow + b * kPBoxRows, full_cl);
+        }
+        __syncwarp();
+        if (++s == kPStages) {
+          s = 0;
+          phase ^= 1;
+          started = true;
         }
       }
+      if (!ok) break;
     }
   } else if (warp == 1) {
     if (rank == 0) {
