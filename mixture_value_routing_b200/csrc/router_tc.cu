@@ -105,17 +105,26 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_consta
   tc_fence_after();
 
   if (warp == 0) {
-    if (lane == 0) {
-      for (int kb = 0; kb < nk; ++kb) {
-        const int s = kb % kRStages;
-        if (kb >= kRStages && !mbar_wait(&S.empty[s], ((kb / kRStages) - 1) & 1)) {
+    // The whole warp runs the loop; one elected lane issues the copies.
+    int s = 0;
+    uint32_t phase = 0;
+    for (int kb = 0; kb < nk; ++kb) {
+      if (kb >= kRStages && !__all_sync(0xffffffffu, mbar_wait(&S.empty[s], phase ^ 1))) {
+        if (lane == 0) {
           raise_status(sb, MOVA_ERR_TIMEOUT, blockIdx.x);
           S.abort = 1;
-          break;
         }
+        break;
+      }
+      if (elect_one()) {
         mbar_arrive_expect_tx(&S.full[s], kRStageBytes);
         tma_load_2d_nohint(S.stage[s], &tmap_x, kb * RK, t0, &S.full[s]);
         tma_load_2d_nohint(S.stage[s] + kRABytes, &tmap_w, kb * RK, 0, &S.full[s]);
+      }
+      __syncwarp();
+      if (++s == kRStages) {
+        s = 0;
+        phase ^= 1;
       }
     }
   } else if (warp == 1) {
@@ -127,9 +136,10 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_consta
     const uint64_t bdesc0 = smem_desc_sw128(smem_u32(S.stage[0]) + kRABytes);
     constexpr uint32_t kStageDesc = kRStageBytes >> 4;
     bool ok = true;
+    int s = 0;
+    uint32_t phase = 0;
     for (int kb = 0; kb < nk; ++kb) {
-      const int s = kb % kRStages;
-      if (!__all_sync(0xffffffffu, mbar_wait(&S.full[s], (kb / kRStages) & 1))) {
+      if (!__all_sync(0xffffffffu, mbar_wait(&S.full[s], phase))) {
         if (lane == 0) {
           raise_status(sb, MOVA_ERR_TIMEOUT, blockIdx.x);
           S.abort = 1;
@@ -147,6 +157,10 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_consta
         tc_commit(&S.empty[s]);
       }
       __syncwarp();
+      if (++s == kRStages) {
+        s = 0;
+        phase ^= 1;
+      }
     }
     if (ok && elect_one()) tc_commit(&S.tmem_full);
     __syncwarp();

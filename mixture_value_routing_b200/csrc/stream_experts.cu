@@ -221,30 +221,40 @@ stream_experts_kernel(const DT* __restrict__ x, const DT* __restrict__ Wv,
   const int nstages = u1 - u0;
 
   if (warp == kConsumerWarps) {
-    if (lane == 0) {
-      const uint64_t pol = policy_evict_first();
-      int j = 0;
-      for (; j < nstages; ++j) {
-        const int s = j % NS;
-        if (j >= NS && !mbar_wait(&empty[s], ((j / NS) - 1) & 1)) {
+    // The producer warp runs the loop together; lane 0 declares each stage's
+    // bytes, then lanes 0-7 issue one row copy each, so a stage's eight
+    // copies leave at once.  The unit's expert and row advance incrementally.
+    const uint64_t pol = policy_evict_first();
+    int a = fused ? u0 % max(nact, 1) : u0 / units_per_expert;
+    int rb = fused ? u0 / max(nact, 1) : u0 - a * units_per_expert;  // row block
+    int s = 0;
+    uint32_t phase = 0;
+    int j = 0;
+    for (; j < nstages; ++j) {
+      if (j >= NS && !__all_sync(0xffffffffu, mbar_wait(&empty[s], phase ^ 1))) {
+        if (lane == 0) {
           raise_status(sb, MOVA_ERR_TIMEOUT, blockIdx.x);
           *abort_flag = 1;
-          break;
         }
-        if (*abort_flag) break;
-        const int u = u0 + j;
-        const int a = fused ? u % nact : u / units_per_expert;
-        const int r = (fused ? u / nact : u - a * units_per_expert) * kRowsPerStage;
-        const DT* src = Wv + (static_cast<size_t>(act[a]) * n + r) * d;
-        mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(kRowsPerStage * row_bytes));
-        uint8_t* dst = stages + s * stage_bytes;
-#pragma unroll 1
-        for (int i = 0; i < kRowsPerStage; ++i)
-          bulk_g2s(dst + i * pitch, src + static_cast<size_t>(i) * d,
-                   static_cast<uint32_t>(row_bytes), &full[s], pol);
+        break;
       }
-      *issued = j;
+      if (*abort_flag) break;
+      const DT* src = Wv + (static_cast<size_t>(act[a]) * n + rb * kRowsPerStage) * d;
+      uint8_t* dst = stages + s * stage_bytes;
+      if (lane == 0) mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(kRowsPerStage * row_bytes));
+      __syncwarp();
+      if (lane < kRowsPerStage)
+        bulk_g2s(dst + lane * pitch, src + static_cast<size_t>(lane) * d, static_cast<uint32_t>(row_bytes),
+                 &full[s], pol);
+      __syncwarp();
+      if (fused) {
+        if (++a == nact) { a = 0; ++rb; }
+      } else {
+        if (++rb == units_per_expert) { rb = 0; ++a; }
+      }
+      if (++s == NS) { s = 0; phase ^= 1; }
     }
+    if (lane == 0) *issued = j;
   } else {
     int cur_a = -1, cnt = 0, off = 0;
     int staged_a = -1, staged_c0 = -1;  // whose x rows the x tile holds
