@@ -22,7 +22,9 @@
 //     accumulators to the epilogues.  The odd CTA's epilogue releases an
 //     accumulator with a remote arrive on the even CTA's barrier.
 //   * Warps: 0 TMA, 1 MMA (even CTA), 2-5 epilogue (SiLU, bf16, store; rows
-//     beyond the expert's n are skipped).
+//     beyond the expert's n are skipped).  The epilogue reads the whole
+//     accumulator into registers (bf16 pairs) and hands it back before it
+//     stores, so the MMA of the tile after next never waits for the stores.
 //   * One persistent pair per two SMs takes tiles from a global counter as
 //     it goes (the even CTA's producer fetches the id and publishes it to
 //     every role of both CTAs through a ring of mbarrier-guarded slots), so
@@ -326,23 +328,43 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_w, const __gri
       const int rloc = tl.mt * 2 * PM + static_cast<int>(rank) * PM + lg * 32 + lane;
       const uint32_t tbase = S.tmem_base + static_cast<uint32_t>(acc * PN) +
                              (static_cast<uint32_t>(lg * 32) << 16);
-      __nv_bfloat16* prow = P + static_cast<size_t>(tl.off + tl.tok0) * n + rloc;
+      unsigned short* prow =
+          reinterpret_cast<unsigned short*>(P + static_cast<size_t>(tl.off + tl.tok0) * n + rloc);
       const bool live = rloc < n;
-      for (int c0 = 0; c0 < tl.N; c0 += 32) {
-        uint32_t r[32];
-        tmem_ld_32(tbase + c0, r);
-        tmem_ld_wait();
-        if (live) {
+      // All of the tile's columns go to registers first (SiLU, rounded to
+      // bf16, two per word), so the accumulator is handed back to the MMA
+      // before the stores start.
+      uint32_t pk[PN / 32][16];
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            if (c0 + j < tl.valid)
-              prow[static_cast<size_t>(c0 + j) * n] = __float2bfloat16_rn(silu_fast(__uint_as_float(r[j])));
+      for (int c = 0; c < PN / 32; ++c) {
+        if (c * 32 < tl.N) {
+          uint32_t r[32];
+          tmem_ld_32(tbase + c * 32, r);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const __nv_bfloat162 h = __floats2bfloat162_rn(silu_fast(__uint_as_float(r[2 * j])),
+                                                           silu_fast(__uint_as_float(r[2 * j + 1])));
+            pk[c][j] = *reinterpret_cast<const uint32_t*>(&h);
           }
         }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(acc == 0 ? empty0 : empty1);
+      if (live) {
+#pragma unroll
+        for (int c = 0; c < PN / 32; ++c) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const int col = c * 32 + j;
+            if (col < tl.valid) {
+              const uint32_t wv = pk[c][j >> 1];
+              prow[static_cast<size_t>(col) * n] = static_cast<unsigned short>((j & 1) ? (wv >> 16) : (wv & 0xFFFFu));
+            }
+          }
+        }
+      }
     }
   }
 
