@@ -39,6 +39,9 @@ template <typename PT, typename OT>
 __global__ void __launch_bounds__(kThreads)
 combine_kernel(const PT* __restrict__ P, const int32_t* __restrict__ pos,
                const float* __restrict__ w32, int T, int k, int n, OT* __restrict__ v) {
+  // The next call's plane split may start now: it touches nothing this
+  // kernel reads, and waits for this grid before it ends.
+  pdl_trigger();
   pdl_wait();  // the expert rows of this call are complete and visible
   const int per_tok = n / 8;
   const long long total = static_cast<long long>(T) * per_tok;

@@ -14,7 +14,7 @@
 //     logits[e] = (acc_hi[e] + acc_mid[e]) + acc_lo[e]: the same products as
 //     an fp32 dot product, accumulated in fp32 in another order.
 //   * One CTA per 128 tokens: a TMA warp streams 128 x 64 token tiles and
-//     192 x 64 plane tiles (128-byte swizzle) through 4 stages; one thread
+//     192 x 64 plane tiles (128-byte swizzle) through 5 stages; one thread
 //     issues tcgen05.mma (M = 128, N = 192, K = 16) into tensor memory; four
 //     epilogue warps read one token per thread (all 192 columns), form the
 //     64 logits, the sigmoid scores and the biased selection in registers and
@@ -33,7 +33,7 @@ namespace {
 constexpr int RM = 128;  // tokens per CTA
 constexpr int RN = 192;  // 3 planes x 64 experts
 constexpr int RK = 64;
-constexpr int kRStages = 4;
+constexpr int kRStages = 5;
 constexpr int kRABytes = RM * RK * 2;
 constexpr int kRBBytes = RN * RK * 2;
 constexpr int kRStageBytes = kRABytes + kRBBytes;
@@ -68,6 +68,11 @@ split_router_kernel(const float* __restrict__ Wr, int E, int d, __nv_bfloat16* _
     W3[static_cast<size_t>(64 + e) * d + j] = mid;
     W3[static_cast<size_t>(128 + e) * d + j] = lo;
   }
+  // Launched with programmatic dependent launch, this kernel overlaps the
+  // previous kernel (which never reads the planes: their last reader is the
+  // previous call's router, long complete).  It ends only after that kernel
+  // has, so everything launched after it still follows the previous kernel.
+  pdl_wait();
 }
 
 __global__ void __launch_bounds__(kRThreads, 1)
@@ -262,9 +267,7 @@ cudaError_t launch_router_tc(const void* x, const float* Wr, const float* br, in
   void* fp = encode_tiled_fn();
   if (fp == nullptr) return cudaErrorNotSupported;
   EncodeTiled enc = reinterpret_cast<EncodeTiled>(fp);
-  note_launch();
-  split_router_kernel<<<2 * sm_count(), 256, 0, stream>>>(Wr, E, d, planes);
-  cudaError_t err = cudaGetLastError();
+  cudaError_t err = launch_pdl(split_router_kernel, dim3(2 * sm_count()), dim3(256), 0, stream, Wr, E, d, planes);
   if (err != cudaSuccess) return err;
   CUtensorMap tx, tw;
   const cuuint64_t xdim[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(T)};
