@@ -13,8 +13,9 @@ struct StatusBlock;
 
 // Largest number of (token, slot) pairs the single-CTA grouping handles.
 constexpr int kMaxPairs = 131072;
-// Token counts up to this run the fused decode router (routing + grouping in
-// one kernel).
+// Token counts up to this take the decode routing: a logits kernel over
+// many CTAs, then selection and grouping by one CTA or inside the
+// weight-streaming kernel.
 constexpr int kFusedRouterMaxT = 8;
 
 // Outputs of the grouping by expert (see launch_permute).

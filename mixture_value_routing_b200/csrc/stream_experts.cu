@@ -4,21 +4,27 @@
 //   P[p, :] = SiLU(Wv[e] x[t])
 // as in "MoVA: routing the value vectors, and why the KV cache does not
 // notice", section "Where the routing happens" (each selected expert's
-// projection passes through SiLU; the combine kernel weights it by its
-// renormalised score and sums the slots).
+// projection passes through SiLU; the combine weights it by its renormalised
+// score and sums the slots).
 //
 // At a few tokens per expert this is a matrix-vector product per active
 // expert and HBM-bound: each active expert's n x d weight is read exactly
 // once.  The rows of all active experts, concatenated, are split evenly over
 // one persistent CTA per SM.  In each CTA a producer warp streams 8-row slabs
-// (contiguous bytes of one or two experts) into a ring of shared-memory
-// stages with 1-D bulk (TMA) copies completing on mbarriers, so each SM keeps
-// ~160 KB of weights in flight without spending registers on it; eight
-// consumer warps take one row of each slab, dot it with the x rows of the
-// expert's tokens (L1 hits), reduce across lanes in a fixed butterfly order
-// and write w * SiLU(h).  Every wait is bounded; a wait that runs out sets
-// MOVA_ERR_TIMEOUT in the status block and the CTA drains its copies and
-// exits.
+// (contiguous bytes of one expert) into a ring of 4 shared-memory stages with
+// 1-D bulk (TMA) copies completing on mbarriers (lanes 0-7 issue a stage's
+// eight row copies together), so each SM keeps ~160 KB of weights in flight
+// without spending registers on it.  Eight consumer warps split K, run
+// mma.sync m16n8k16 on (8 weight rows) x (8 token columns), and reduce the
+// partial tiles in warp order; a slab's 8 x 8 results go to P.
+//
+// Decode batches (bf16, T <= 8) keep every token's x in shared memory, and
+// with RouteIn the kernel also routes them itself: each CTA sums the router's
+// partial logits, selects (route_select.cuh) and groups in shared memory.
+// With the combine fused in, slabs run row-block-major and the CTA that
+// completes a block of 8 output columns (per-block tickets) writes v there.
+// Every wait is bounded; a wait that runs out sets MOVA_ERR_TIMEOUT in the
+// status block and the CTA drains its copies and exits.
 #include "common.cuh"
 #include "internal.h"
 #include "route_select.cuh"
