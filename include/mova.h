@@ -55,7 +55,7 @@ extern "C" {
 typedef enum {
   MOVA_OK = 0,
   MOVA_ERR_INVALID_ARG = 1,   /* null pointer, bad size, misalignment, workspace too small */
-  MOVA_ERR_UNSUPPORTED = 2,   /* valid arguments this build does not implement */
+  MOVA_ERR_UNSUPPORTED = 2,   /* valid arguments the library does not implement */
   MOVA_ERR_CUDA = 3,          /* a CUDA runtime call or a launch failed */
   MOVA_ERR_TIMEOUT = 4,       /* a bounded device-side wait ran out (status word) */
   MOVA_ERR_DEVICE_CHECK = 5   /* a device-side input check failed (status word) */
