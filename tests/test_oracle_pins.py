@@ -95,6 +95,14 @@ def test_bf16_format():
         assert got == val and math.copysign(1.0, got) == math.copysign(1.0, val), hexbits
 
 
+def test_f16_format():
+    # Routing-given mode stores the weights in fp16 and uses them as they are.
+    for hexbits, val in _load("f16_patterns.json")["patterns"]:
+        a = np.array([int(hexbits, 16)], dtype=np.uint16).view(np.float16)
+        got = O.to_f64(a, "f16")[0]
+        assert got == val and math.copysign(1.0, got) == math.copysign(1.0, val), hexbits
+
+
 # ---------------------------------------------------------------------------
 # Identities of the method
 # ---------------------------------------------------------------------------
@@ -160,6 +168,27 @@ def test_weights_positive_and_sum_to_scale():
     for t in range(x.shape[0]):
         st = [1.0 / (1.0 + math.exp(-float(np.dot(x[t], Wr[e])))) for e in r["idx"][t]]
         np.testing.assert_allclose(r["w"][t], [2.5 * s / sum(st) for s in st], rtol=1e-12)
+
+
+def test_weights_for_another_selection():
+    # weights_for serves the parity tests when a near-tie admits a second
+    # valid selection.  On the router's own selection it must give the
+    # router's weights; on any selection, positive weights summing to the
+    # scale, in the ratio of the selected unbiased scores.
+    rng = np.random.default_rng(5)
+    x, Wr, br, _ = _rand_case(rng, T=20)
+    r = O.route(x, Wr, br, 4, 2.5)
+    np.testing.assert_array_equal(O.weights_for(r["s"], r["idx"], 2.5), r["w"])
+    alt = r["idx"].copy()
+    alt[:, 3] = np.argsort(-r["b"], axis=1, kind="stable")[:, 4]  # the 5th expert instead of the 4th
+    w = O.weights_for(r["s"], alt, 2.5)
+    assert (w > 0).all()
+    np.testing.assert_allclose(w.sum(axis=1), 2.5, rtol=1e-14)
+    for t in range(x.shape[0]):
+        s0 = 1.0 / (1.0 + math.exp(-float(np.dot(x[t], Wr[alt[t, 0]]))))
+        for j in range(1, 4):
+            sj = 1.0 / (1.0 + math.exp(-float(np.dot(x[t], Wr[alt[t, j]]))))
+            assert math.isclose(w[t, j] / w[t, 0], sj / s0, rel_tol=1e-12)
 
 
 def test_bias_shift_invariance():
