@@ -480,9 +480,10 @@ def _oracle_tokens(O, lay, bat, rows, mode, wv_dt, dtype):
     return v
 
 
-def cpu_baseline(a, budget_s=12.0, steps=None):
+def cpu_baseline(a, budget_s=12.0, steps=None, warmup=0):
     """Time the oracle, as it stands, on seeded batches of the same workload:
-    whole steps when they fit the budget, else a sample of tokens per step."""
+    whole steps when they fit the budget, else a sample of tokens per step.
+    `warmup` untimed steps (of at most 8 tokens each) run first."""
     from oracle import mova_oracle as O
     cfg = MI.WORKLOADS[a.workload]
     T, dtype, mode = cfg["T"], cfg["dtype"], cfg["mode"]
@@ -500,6 +501,8 @@ def cpu_baseline(a, budget_s=12.0, steps=None):
         rows_per = T if per_tok * T * steps <= budget_s else max(1, int(budget_s / steps / per_tok))
         nsteps = steps
     rng = np.random.default_rng(1234)
+    for _ in range(warmup):
+        _oracle_tokens(O, lay, bat, np.arange(min(T, rows_per, 8)), mode, wdt, dtype)
     done = 0
     i = 0
     t0 = time.perf_counter()
@@ -515,7 +518,8 @@ def cpu_baseline(a, budget_s=12.0, steps=None):
     return {"value": round(done / el, 3), "unit": "tokens/s", "cores": _blas_threads(),
             "kind": "oracle",
             "sample": f"{i} oracle steps of {rows_per} of the {T} tokens of a seeded "
-                      f"{a.workload} batch ({done} tokens, {el:.1f} s, numpy fp64)",
+                      f"{a.workload} batch ({done} tokens, {el:.1f} s, numpy fp64)"
+                      + (f", after {warmup} untimed warm-up steps of up to 8 tokens" if warmup else ""),
             "steps_timed": i, "seconds": round(el, 2)}
 
 
@@ -524,7 +528,7 @@ def run_reference(a):
     if rank != 0:
         return
     budget = 150.0
-    cb = cpu_baseline(a, budget_s=budget, steps=a.steps)
+    cb = cpu_baseline(a, budget_s=budget, steps=a.steps, warmup=a.warmup)
     line = {"impl": "reference", "metric": METRIC, "value": cb["value"], "unit": "tokens/s",
             "n_gpus": world, "steps": a.steps, "warmup": a.warmup,
             "ms_per_step": round(1e3 * cb["seconds"] / max(1, cb["steps_timed"]), 3),
