@@ -159,6 +159,23 @@ mova_status mova_value_routed_ex(const void* x, mova_dtype x_dt, const float* Wr
                                  void* ws, size_t ws_bytes, mova_path path, void* const* events,
                                  void* stream);
 
+/* Where a value call leaves its routing and grouping inside the workspace.
+ * Writes MOVA_WS_PARTS byte offsets, relative to the start of a workspace
+ * laid out for these sizes, of:
+ *   [0] idx     (T, k)  int32  the routing the expert kernels used, unless the
+ *   [1] w       (T, k)  fp32   call wrote it to caller-given idx_out / w_out
+ *   [2] counts  (E)     int32  pairs per expert
+ *   [3] offsets (E+1)   int32  exclusive prefix sum of counts
+ *   [4] perm    (T*k)   int32  pair f = t*k + slot at each grouped position
+ *   [5] pos     (T*k)   int32  inverse of perm
+ * (the arrays mova_permute defines).  Every value entry point fills [2]-[5]
+ * with the grouping its expert kernels ran on, so a caller (or a test) can
+ * read it back once the stream has passed the call.  Host-only; returns
+ * MOVA_ERR_INVALID_ARG / MOVA_ERR_UNSUPPORTED as mova_workspace_size would
+ * return 0, and for T == 0 (no workspace). */
+#define MOVA_WS_PARTS 6
+mova_status mova_workspace_parts(int T, int d, int E, int k, int n, size_t* offsets);
+
 /* Synchronises `stream`, then returns and clears the device status word
  * held in `ws` (MOVA_OK if no device-side check fired since the last read).
  * `detail_out` (nullable) receives the first offending item (e.g. the flat
@@ -172,6 +189,17 @@ mova_status mova_get_status(void* ws, int32_t* detail_out, void* stream);
  * word of `ws` (256 bytes suffice), readable with mova_get_status.  The
  * context stays usable afterwards.  Not part of the method. */
 mova_status mova_selftest_wait_timeout(void* ws, long long limit_cycles, void* stream);
+
+/* Self-test of the weight-streaming kernel's failure handling: arms the
+ * next weight-streaming launch in this process so that its first CTA stops
+ * issuing weight copies at stage `stall_stage`, and its pipeline waits give
+ * up after `limit_cycles` clock cycles (at most about one second's worth).
+ * That launch then records MOVA_ERR_TIMEOUT in the status word, every warp
+ * leaves, the copies already issued are drained, and the context stays
+ * usable.  The arming is consumed by that one launch.  Not part of the
+ * method; returns MOVA_ERR_INVALID_ARG for a negative stage or a limit out of
+ * range. */
+mova_status mova_selftest_arm_stream_stall(int stall_stage, long long limit_cycles);
 
 /* The path AUTO would pick for these sizes and dtype (for tests/benches). */
 mova_path mova_auto_path(int T, mova_dtype x_dt);
@@ -203,7 +231,11 @@ unsigned long long mova_launch_count(void);
  *    d = 2560, E = 64, k = 4, n = 1024 that admits batches up to T = 30.
  *  - The first call on each device looks up the array's device address
  *    (cudaGetSymbolAddress, with that device current); make that first call
- *    before any stream capture.
+ *    before any stream capture.  The address is kept per device and context
+ *    (keyed on the context's process-unique id); after cudaDeviceReset, or
+ *    with another context current, the next call looks it up again, so make
+ *    that call outside a capture too.  If the driver cannot report context
+ *    ids, every call looks the address up.
  *  - All calls share the one array and it keeps the last call's contents;
  *    each call's first kernel resets the status fields it relies on, and
  *    every other part is fully rewritten.  Calls that overlap on the GPU

@@ -20,6 +20,8 @@ STATUS_NAMES = {OK: "MOVA_OK", ERR_INVALID_ARG: "MOVA_ERR_INVALID_ARG",
 F32, BF16, F16, I32, I8 = range(5)
 # mova_path
 PATH_AUTO, PATH_STREAM, PATH_TENSOR, PATH_TENSOR_1CTA = range(4)
+# parts of the workspace (mova_workspace_parts)
+WS_PARTS = ("idx", "w", "counts", "offsets", "perm", "pos")
 # stage events recorded by the _ex entry points
 STAGE_EVENTS = 5
 STAGES = ("route", "group", "experts", "combine")
@@ -45,6 +47,8 @@ SIGNATURES = {
                                   _vp, _vp, _sz, _i, _vp, _vp]),
     "mova_get_status": (_i, [_vp, _vp, _vp]),
     "mova_selftest_wait_timeout": (_i, [_vp, ctypes.c_longlong, _vp]),
+    "mova_selftest_arm_stream_stall": (_i, [_i, ctypes.c_longlong]),
+    "mova_workspace_parts": (_i, [_i, _i, _i, _i, _i, _vp]),
     "mova_value_routed_noalloc": (_i, [_vp, _i, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _vp,
                                        _vp]),
 }

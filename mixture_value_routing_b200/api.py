@@ -179,6 +179,35 @@ def value_routed(x: torch.Tensor, Wr: torch.Tensor, br: torch.Tensor, Wv: torch.
     return v
 
 
+def workspace_parts(T: int, d: int, E: int, k: int, n: int) -> dict:
+    """Byte offsets of the routing and grouping a value call leaves in its
+    workspace: dict(idx, w, counts, offsets, perm, pos) -> offset."""
+    offs = (ctypes.c_size_t * len(_lib.WS_PARTS))()
+    _lib.check(_lib.load().mova_workspace_parts(T, d, E, k, n, offs), "mova_workspace_parts")
+    return dict(zip(_lib.WS_PARTS, (int(o) for o in offs)))
+
+
+def grouping(ws: torch.Tensor, T: int, d: int, E: int, k: int, n: int) -> dict:
+    """The grouping by expert (counts, offsets, perm, pos; int32 copies) that
+    the last value call with these sizes ran on, read from its workspace
+    (call after the stream has passed that call)."""
+    offs = workspace_parts(T, d, E, k, n)
+    size = {"counts": E, "offsets": E + 1, "perm": T * k, "pos": T * k}
+    out = {}
+    for name, count in size.items():
+        o = offs[name]
+        out[name] = ws[o:o + 4 * count].view(torch.int32).clone()
+    return out
+
+
+def arm_stream_stall(stall_stage: int, limit_cycles: int) -> None:
+    """Test hook: the next weight-streaming launch stops issuing weight copies
+    in its first CTA at `stall_stage` and gives up waiting after
+    `limit_cycles`, reporting MOVA_ERR_TIMEOUT (mova_selftest_arm_stream_stall)."""
+    _lib.check(_lib.load().mova_selftest_arm_stream_stall(int(stall_stage), int(limit_cycles)),
+               "mova_selftest_arm_stream_stall")
+
+
 def get_status(ws: Optional[torch.Tensor] = None, device=None):
     """(status name, detail) of the last value call on this workspace."""
     if ws is None:

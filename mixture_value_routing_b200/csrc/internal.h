@@ -125,7 +125,26 @@ struct RouteIn {
   float scale;
   int32_t* idx_out;
   float* w_out;
+  // The grouping CTA 0 computes (also written to global memory, so that it
+  // can be read back from the workspace): counts (E), offsets (E+1), perm and
+  // pos (T*k), the active list and the status block's active count.
+  int32_t* counts_out;
+  int32_t* offsets_out;
+  int32_t* perm_out;
+  int32_t* pos_out;
+  int32_t* active_out;
 };
+
+// Test-only fault injection for the weight-streaming kernel
+// (mova_selftest_arm_stream_stall): the limit of its pipeline waits in clock
+// cycles, and the stage at which CTA 0's producer stops issuing weight
+// copies (-1: never).  take_stream_fault() returns the armed values once and
+// disarms them; unarmed it returns {kWaitLimitCycles, -1}.
+struct StreamFault {
+  long long wait_limit;
+  int stall_stage;
+};
+StreamFault take_stream_fault();
 
 // With tickets and v given (bf16, T <= 8 only), the kernel also performs
 // the combine: the CTA that completes a block of 8 output columns computes v

@@ -31,9 +31,19 @@ void* encode_tiled_fn() {
 
 namespace {
 std::atomic<unsigned long long> g_launches{0};
+// Armed by mova_selftest_arm_stream_stall for the next weight-streaming launch.
+std::atomic<int> g_fault_stage{-1};
+std::atomic<long long> g_fault_limit{0};
 }  // namespace
 
 void note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+
+StreamFault take_stream_fault() {
+  const int stage = g_fault_stage.exchange(-1);
+  const long long limit = g_fault_limit.exchange(0);
+  if (stage < 0 || limit <= 0) return StreamFault{kWaitLimitCycles, -1};
+  return StreamFault{limit, stage};
+}
 
 int sm_count() {
   static int cached[64] = {0};
@@ -324,7 +334,7 @@ mova_status mova_value_routed_ex(const void* x, mova_dtype x_dt, const float* Wr
       err = launch_router_logits(x, x_dt, Wr, T, d, E, w.logits, &S, w.tickets, n / 8, w.sb, s);
     if (err == cudaSuccess) err = mark(events, 1, s);
     if (err == cudaSuccess) err = mark(events, 2, s);
-    const RouteIn ri{w.logits, S, br, E, scale, idx, wgt};
+    const RouteIn ri{w.logits, S, br, E, scale, idx, wgt, w.counts, w.offsets, w.perm, w.pos, w.active};
     if (err == cudaSuccess)
       err = launch_stream_experts(x, Wv, x_dt, w.counts, w.offsets, w.perm, wgt, w.active, w.sb, T, d, n, k,
                                   E, static_cast<float*>(w.P), w.tickets, v, ri, s);
@@ -375,6 +385,24 @@ mova_status mova_selftest_wait_timeout(void* ws, long long limit_cycles, void* s
   selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
       static_cast<StatusBlock*>(ws), limit_cycles);
   return from_cuda(cudaGetLastError());
+}
+
+mova_status mova_selftest_arm_stream_stall(int stall_stage, long long limit_cycles) {
+  if (stall_stage < 0 || limit_cycles <= 0 || limit_cycles > kWaitLimitCycles) return MOVA_ERR_INVALID_ARG;
+  g_fault_limit.store(limit_cycles);
+  g_fault_stage.store(stall_stage);
+  return MOVA_OK;
+}
+
+mova_status mova_workspace_parts(int T, int d, int E, int k, int n, size_t* offsets) {
+  if (offsets == nullptr) return MOVA_ERR_INVALID_ARG;
+  const mova_status st = check_dims(T, d, E, k, n);
+  if (st != MOVA_OK) return st;
+  if (T == 0) return MOVA_ERR_INVALID_ARG;
+  const Workspace w = layout(nullptr, T, d, k, n);
+  const void* parts[MOVA_WS_PARTS] = {w.idx, w.w, w.counts, w.offsets, w.perm, w.pos};
+  for (int i = 0; i < MOVA_WS_PARTS; ++i) offsets[i] = reinterpret_cast<uintptr_t>(parts[i]);
+  return MOVA_OK;
 }
 
 mova_status mova_get_status(void* ws, int32_t* detail_out, void* stream) {

@@ -52,27 +52,59 @@ struct __align__(1024) RSmem {
 };
 
 // Exact split of an fp32 value into three bf16 values summing to it.
+// Each thread handles up to kSplitPer elements of Wr (8 consecutive floats
+// per step).  The router weights are read and split while the previous
+// kernel on the stream may still run (launched with programmatic dependent
+// launch; no kernel writes router weights), but the planes are stored only
+// after griddepcontrol.wait: they live in the caller's workspace, where the
+// previous call's kernels may still be reading other data at the same
+// offsets (the workspace layout depends on the call's sizes).
+constexpr int kSplitPer = 2;  // 8-element groups per thread
 __global__ void __launch_bounds__(256)
 split_router_kernel(const float* __restrict__ Wr, int E, int d, __nv_bfloat16* __restrict__ W3) {
-  const long long total = 64LL * d;
-  for (long long i = blockIdx.x * 256LL + threadIdx.x; i < total; i += 256LL * gridDim.x) {
-    const int e = static_cast<int>(i / d);
-    const int j = static_cast<int>(i - static_cast<long long>(e) * d);
-    float v = (e < E) ? Wr[i] : 0.f;
-    const __nv_bfloat16 hi = __float2bfloat16_rn(v);
-    v -= __bfloat162float(hi);
-    const __nv_bfloat16 mid = __float2bfloat16_rn(v);
-    v -= __bfloat162float(mid);
-    const __nv_bfloat16 lo = __float2bfloat16_rn(v);
-    W3[static_cast<size_t>(e) * d + j] = hi;
-    W3[static_cast<size_t>(64 + e) * d + j] = mid;
-    W3[static_cast<size_t>(128 + e) * d + j] = lo;
+  const int groups = 64 * d / 8;
+  uint4 hi[kSplitPer], mid[kSplitPer], lo[kSplitPer];
+  int gi[kSplitPer];
+#pragma unroll
+  for (int q = 0; q < kSplitPer; ++q) {
+    const int g = (blockIdx.x * kSplitPer + q) * 256 + threadIdx.x;
+    gi[q] = g;
+    if (g >= groups) continue;
+    const int e = g * 8 / d;
+    float v[8];
+    if (e < E) {
+      load8(Wr + static_cast<size_t>(g) * 8, v);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) v[i] = 0.f;
+    }
+    __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&hi[q]);
+    __nv_bfloat162* m = reinterpret_cast<__nv_bfloat162*>(&mid[q]);
+    __nv_bfloat162* l = reinterpret_cast<__nv_bfloat162*>(&lo[q]);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      float a = v[2 * i], b = v[2 * i + 1];
+      const __nv_bfloat162 ha = __floats2bfloat162_rn(a, b);
+      a -= __low2float(ha);
+      b -= __high2float(ha);
+      const __nv_bfloat162 ma = __floats2bfloat162_rn(a, b);
+      a -= __low2float(ma);
+      b -= __high2float(ma);
+      h[i] = ha;
+      m[i] = ma;
+      l[i] = __floats2bfloat162_rn(a, b);
+    }
   }
-  // Launched with programmatic dependent launch, this kernel overlaps the
-  // previous kernel (which never reads the planes: their last reader is the
-  // previous call's router, long complete).  It ends only after that kernel
-  // has, so everything launched after it still follows the previous kernel.
-  pdl_wait();
+  pdl_wait();  // every kernel before this one on the stream has completed
+  const size_t plane = static_cast<size_t>(64) * d / 8;  // uint4 per plane
+  uint4* W = reinterpret_cast<uint4*>(W3);
+#pragma unroll
+  for (int q = 0; q < kSplitPer; ++q) {
+    if (gi[q] >= groups) continue;
+    W[gi[q]] = hi[q];
+    W[plane + gi[q]] = mid[q];
+    W[2 * plane + gi[q]] = lo[q];
+  }
 }
 
 __global__ void __launch_bounds__(kRThreads, 1)
@@ -267,7 +299,8 @@ cudaError_t launch_router_tc(const void* x, const float* Wr, const float* br, in
   void* fp = encode_tiled_fn();
   if (fp == nullptr) return cudaErrorNotSupported;
   EncodeTiled enc = reinterpret_cast<EncodeTiled>(fp);
-  cudaError_t err = launch_pdl(split_router_kernel, dim3(2 * sm_count()), dim3(256), 0, stream, Wr, E, d, planes);
+  const int split_blocks = (64 * d / 8 + 256 * kSplitPer - 1) / (256 * kSplitPer);
+  cudaError_t err = launch_pdl(split_router_kernel, dim3(split_blocks), dim3(256), 0, stream, Wr, E, d, planes);
   if (err != cudaSuccess) return err;
   CUtensorMap tx, tw;
   const cuuint64_t xdim[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(T)};

@@ -64,6 +64,18 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   return mbar_wait_for(bar, parity, kWaitLimitCycles);
 }
 
+// As mbar_wait_for, but also gives up as soon as *abort is non-zero (another
+// role of the CTA has already failed, so nothing is worth waiting for).
+__device__ __forceinline__ bool mbar_wait_or_abort(uint64_t* bar, uint32_t parity,
+                                                   const volatile int* abort, long long limit) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long start = clock64();
+  while (!mbar_try_wait(bar, parity)) {
+    if (*abort != 0 || clock64() - start > limit) return false;
+  }
+  return true;
+}
+
 // 1-D bulk copy global -> shared (this CTA), completion counted in bytes on
 // `bar`.  dst, src 16-byte aligned; bytes a multiple of 16.
 __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar,

@@ -99,6 +99,18 @@ __device__ __forceinline__ void consumers_sync() {
   asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");
 }
 
+// Consumer-group barrier that also ORs a predicate over the group's threads.
+__device__ __forceinline__ bool consumers_any(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.or.pred q, 1, %2, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(v)), "n"(kConsumerWarps * 32)
+      : "memory");
+  return r != 0;
+}
+
 template <typename DT>
 __global__ void __launch_bounds__(kThreads, 1)
 stream_experts_kernel(const DT* __restrict__ x, const DT* __restrict__ Wv,
@@ -106,7 +118,8 @@ stream_experts_kernel(const DT* __restrict__ x, const DT* __restrict__ Wv,
                       const int32_t* __restrict__ perm, const float* __restrict__ w32,
                       const int32_t* __restrict__ active, StatusBlock* __restrict__ sb, int T,
                       int d, int n, int k, float* __restrict__ P, int NS,
-                      int32_t* __restrict__ tickets, DT* __restrict__ v, RouteIn route) {
+                      int32_t* __restrict__ tickets, DT* __restrict__ v, RouteIn route,
+                      StreamFault fault) {
   constexpr bool kMma = sizeof(DT) == 2;
   constexpr int EL = Vec<DT>::EL;
   extern __shared__ __align__(128) uint8_t smem[];
@@ -201,6 +214,24 @@ stream_experts_kernel(const DT* __restrict__ x, const DT* __restrict__ Wv,
         const int na = group_pairs_warp(r_sel, T * k, route.E, lane, r_scratch, r_cnt, r_off, r_pos,
                                         r_perm, act);
         if (lane == 0) r_nact = na;
+        if (blockIdx.x == 0 && route.counts_out != nullptr) {
+          // Every CTA groups the batch identically; CTA 0 also leaves the
+          // result in global memory (counts, offsets, perm, pos, active).
+          __syncwarp();
+          for (int i = lane; i < route.E; i += 32) {
+            route.counts_out[i] = r_cnt[i];
+            route.offsets_out[i] = r_off[i];
+          }
+          if (lane == 0) {
+            route.offsets_out[route.E] = r_off[route.E];
+            sb->num_active = na;
+          }
+          for (int i = lane; i < T * k; i += 32) {
+            route.perm_out[i] = r_perm[i];
+            route.pos_out[i] = r_pos[i];
+          }
+          for (int i = lane; i < na; i += 32) route.active_out[i] = act[i];
+        }
       }
     }
   } else {
@@ -237,14 +268,18 @@ stream_experts_kernel(const DT* __restrict__ x, const DT* __restrict__ Wv,
     uint32_t phase = 0;
     int j = 0;
     for (; j < nstages; ++j) {
-      if (j >= NS && !__all_sync(0xffffffffu, mbar_wait(&empty[s], phase ^ 1))) {
-        if (lane == 0) {
+      if (j >= NS &&
+          !__all_sync(0xffffffffu, mbar_wait_or_abort(&empty[s], phase ^ 1, abort_flag, fault.wait_limit))) {
+        if (lane == 0 && *abort_flag == 0) {
           raise_status(sb, MOVA_ERR_TIMEOUT, blockIdx.x);
           *abort_flag = 1;
         }
         break;
       }
-      if (*abort_flag) break;
+      if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
+      // Test-only injection: CTA 0 stops issuing here, so the consumers'
+      // wait for this stage must run out.
+      if (j == fault.stall_stage && blockIdx.x == 0) break;
       const DT* src = Wv + (static_cast<size_t>(act[a]) * n + rb * kRowsPerStage) * d;
       uint8_t* dst = stages + s * stage_bytes;
       if (lane == 0) mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(kRowsPerStage * row_bytes));
@@ -283,20 +318,28 @@ stream_experts_kernel(const DT* __restrict__ x, const DT* __restrict__ Wv,
         act_cnt[threadIdx.x] = routing ? r_cnt[act[threadIdx.x]] : counts[act[threadIdx.x]];
         act_off[threadIdx.x] = routing ? r_off[act[threadIdx.x]] : offsets[act[threadIdx.x]];
       }
-      if (!mbar_wait(xbar, 0)) {
+      if (!mbar_wait_or_abort(xbar, 0, abort_flag, fault.wait_limit)) {
         raise_status(sb, MOVA_ERR_TIMEOUT, blockIdx.x);
         *abort_flag = 1;
       }
       consumers_sync();
     }
+    // Every consumer warp runs every stage of the loop and meets the others
+    // at the same barriers, whatever happens: after a failed wait (or an
+    // abort raised by another role) a warp skips the stage's arithmetic but
+    // not its barriers, so no warp can be left waiting at one.  `ok` is
+    // warp-uniform (the mma.sync path needs the whole warp).
     for (int j = 0; j < nstages; ++j) {
       const int s = j % NS;
-      if (*abort_flag) break;
-      if (!mbar_wait(&full[s], (j / NS) & 1)) {
-        raise_status(sb, MOVA_ERR_TIMEOUT, blockIdx.x);
-        *abort_flag = 1;
-        break;
+      bool ok = *abort_flag == 0;
+      if (ok && !mbar_wait_or_abort(&full[s], (j / NS) & 1, abort_flag, fault.wait_limit)) {
+        ok = false;
+        if (*abort_flag == 0) {
+          raise_status(sb, MOVA_ERR_TIMEOUT, blockIdx.x);
+          *abort_flag = 1;
+        }
       }
+      ok = __all_sync(0xffffffffu, ok);
       const int u = u0 + j;
       const int a = fused ? u % nact : u / units_per_expert;
       const int r0 = (fused ? u / nact : u - a * units_per_expert) * kRowsPerStage;
@@ -337,12 +380,14 @@ stream_experts_kernel(const DT* __restrict__ x, const DT* __restrict__ Wv,
           const int lk = (lane >> 3) & 1;
           const uint32_t a_base = smem_u32(wst) + lr * static_cast<uint32_t>(pitch) + lk * 16;
           const uint32_t b_base = smem_u32(xs) + lr * static_cast<uint32_t>(pitch) + lk * 16;
+          if (ok) {
 #pragma unroll 4
-          for (int ks = kb; ks < ke; ++ks) {
-            uint32_t a0, a2, b0, b1;
-            ldsm_x2(a_base + ks * 32, a0, a2);
-            ldsm_x2(b_base + ks * 32, b0, b1);
-            mma_bf16_16816(acc, a0, a2, b0, b1);
+            for (int ks = kb; ks < ke; ++ks) {
+              uint32_t a0, a2, b0, b1;
+              ldsm_x2(a_base + ks * 32, a0, a2);
+              ldsm_x2(b_base + ks * 32, b0, b1);
+              mma_bf16_16816(acc, a0, a2, b0, b1);
+            }
           }
           // acc[0], acc[1]: weight row lane/4, tokens 2*(lane%4) + {0, 1}.
           // Two reduction buffers alternate, so one barrier per tile
@@ -367,7 +412,7 @@ stream_experts_kernel(const DT* __restrict__ x, const DT* __restrict__ Wv,
               P[static_cast<size_t>(p) * n + r0 + row] = siluf_(h);
             }
           }
-        } else {
+        } else if (ok) {
           // fp32 weights: CUDA-core dot products, one row per warp.
           const int f_last = nt - 1;
           const DT* xr[kTok];
@@ -412,7 +457,9 @@ stream_experts_kernel(const DT* __restrict__ x, const DT* __restrict__ Wv,
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[s]);
     }
-    if (fused && nstages > 0 && !*abort_flag) {
+    // The consumer warps agree (one bar.red) on whether any role failed: if
+    // so, nothing is combined; otherwise every warp takes the same path.
+    if (fused && nstages > 0 && !consumers_any(*abort_flag != 0)) {
       // Fused combine.  This CTA's rows of P are complete: publish them, then
       // count them on the tickets of the row blocks they belong to; the CTA
       // that completes a block's count sums the slots of every token for its
@@ -492,6 +539,7 @@ cudaError_t launch_stream_experts(const void* x, const void* Wv, mova_dtype dt, 
   const size_t smem = stream_experts_smem(d, dt, T, &NS);
   if (smem == 0) return cudaErrorInvalidValue;
   const dim3 grid(sm_count());
+  const StreamFault fault = take_stream_fault();
   if (dt == MOVA_BF16) {
     auto kern = stream_experts_kernel<__nv_bfloat16>;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -500,7 +548,7 @@ cudaError_t launch_stream_experts(const void* x, const void* Wv, mova_dtype dt, 
     return launch_pdl(kern, grid, dim3(kThreads), smem, stream,
                       static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(Wv),
                       counts, offsets, perm, w32, active, sb, T, d, n, k, P, NS, tickets,
-                      static_cast<__nv_bfloat16*>(v), route);
+                      static_cast<__nv_bfloat16*>(v), route, fault);
   }
   auto kern = stream_experts_kernel<float>;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -508,7 +556,7 @@ cudaError_t launch_stream_experts(const void* x, const void* Wv, mova_dtype dt, 
   if (err != cudaSuccess) return err;
   return launch_pdl(kern, grid, dim3(kThreads), smem, stream, static_cast<const float*>(x),
                     static_cast<const float*>(Wv), counts, offsets, perm, w32, active, sb, T, d, n,
-                    k, P, NS, tickets, static_cast<float*>(v), route);
+                    k, P, NS, tickets, static_cast<float*>(v), route, fault);
 }
 
 }  // namespace mova

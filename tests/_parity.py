@@ -14,6 +14,8 @@ Comparison rules (all written here, in one place):
 """
 from __future__ import annotations
 
+from typing import NamedTuple
+
 import numpy as np
 import torch
 
@@ -44,11 +46,16 @@ def host_f64(t: torch.Tensor) -> np.ndarray:
     return t.detach().float().cpu().numpy().astype(np.float64)
 
 
+class RoutingCheck(NamedTuple):
+    differ: np.ndarray  # tokens whose GPU selection differs from the oracle's (inside the band)
+    near: np.ndarray    # every token with a near tie
+
+
 def check_routing(idx_gpu: np.ndarray, w_gpu: np.ndarray, ref: dict, k: int, scale: float,
-                  log=print):
-    """Compare the GPU's routing with the oracle's.  Returns the tokens whose
-    selection differs inside the near-tie band (their value references must
-    use the GPU's selection)."""
+                  log=print) -> RoutingCheck:
+    """Compare the GPU's routing with the oracle's.  Returns the near-tie
+    tokens and those whose selection differs inside the near-tie band (their
+    value references must use the GPU's selection)."""
     b = ref["b"]
     T, E = b.shape
     order = np.argsort(-b, axis=1, kind="stable")
@@ -76,7 +83,9 @@ def check_routing(idx_gpu: np.ndarray, w_gpu: np.ndarray, ref: dict, k: int, sca
         if t not in set(differ.tolist()):
             log(f"near-tie token {t} (same choice): gap45={member_gap[t]:.3e} "
                 f"gap_slots={slot_gap[t]:.3e}")
-    return differ
+    log(f"routing of {T} tokens: {near_all.size} near-tie tokens, {differ.size} chosen differently "
+        f"inside the band")
+    return RoutingCheck(differ=differ, near=near_all)
 
 
 def check_values(v_gpu: np.ndarray, v_ref: np.ndarray, dtype: str, what: str = "v"):

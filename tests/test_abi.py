@@ -110,3 +110,40 @@ def test_noalloc_scratch_admits_the_documented_batch(lib):
     scratch = 2 << 20
     assert lib.mova_workspace_size(30, 2560, 64, 4, 1024) <= scratch
     assert lib.mova_workspace_size(31, 2560, 64, 4, 1024) > scratch
+
+
+def test_noalloc_validates_like_the_regular_entry_point(lib):
+    """The no-allocation entry point checks its arguments exactly as
+    mova_value_routed does; T == 0 is a no-op only for valid sizes."""
+    for args in ((0, 2560, 64, 4, 1024), (0, -1, 64, 4, 1024), (0, 2560, 65, 4, 1024),
+                 (8, 2561, 64, 4, 1024), (8, 2560, 64, 9, 1024)):
+        want = lib.mova_value_routed(None, _lib.BF16, None, None, None, _lib.BF16, *args,
+                                     ctypes.c_float(2.5), None, None, None, None, 0, None)
+        got = lib.mova_value_routed_noalloc(None, _lib.BF16, None, None, None, _lib.BF16, *args,
+                                            ctypes.c_float(2.5), None, None)
+        assert got == want, (args, got, want)
+
+
+def test_workspace_parts(lib):
+    """The routing and grouping parts of the workspace lie inside it, in
+    order, 256-byte aligned and large enough for their arrays."""
+    T, d, E, k, n = 4096, 2560, 64, 4, 1024
+    offs = (ctypes.c_size_t * len(_lib.WS_PARTS))()
+    assert lib.mova_workspace_parts(T, d, E, k, n, offs) == _lib.OK
+    o = dict(zip(_lib.WS_PARTS, offs))
+    size = dict(idx=T * k * 4, w=T * k * 4, counts=E * 4, offsets=(E + 1) * 4, perm=T * k * 4,
+                pos=T * k * 4)
+    total = lib.mova_workspace_size(T, d, E, k, n)
+    names = list(_lib.WS_PARTS)
+    for a, b in zip(names, names[1:]):
+        assert o[a] % 256 == 0 and o[a] + size[a] <= o[b]
+    assert o["pos"] + size["pos"] <= total
+    assert lib.mova_workspace_parts(0, d, E, k, n, offs) == _lib.ERR_INVALID_ARG
+    assert lib.mova_workspace_parts(T, d, 65, k, n, offs) == _lib.ERR_UNSUPPORTED
+    assert lib.mova_workspace_parts(T, d, E, k, n, None) == _lib.ERR_INVALID_ARG
+
+
+def test_stream_stall_arming_is_validated(lib):
+    assert lib.mova_selftest_arm_stream_stall(-1, 1000) == _lib.ERR_INVALID_ARG
+    assert lib.mova_selftest_arm_stream_stall(2, 0) == _lib.ERR_INVALID_ARG
+    assert lib.mova_selftest_arm_stream_stall(2, 1 << 40) == _lib.ERR_INVALID_ARG

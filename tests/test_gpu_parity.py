@@ -169,21 +169,34 @@ def test_value_given_bad_index_is_flagged(api):
 # Full path
 # ---------------------------------------------------------------------------
 
-def _full(api, T, d, E, k, n, dtype, seed=0, bias="normal", sample=None, path="auto"):
+def _full(api, T, d, E, k, n, dtype, seed=0, bias="normal", sample=None, path="auto", record=None):
+    """The whole path through mova_value_routed: routing against the oracle's
+    (near-tie rule), the grouping the expert kernels actually ran on (read back
+    from the workspace) bit-exact against the oracle's stable counting sort of
+    the GPU's routing, and the values (every token, or a seeded sample)."""
     lay = _layer(seed, d, E, n, dtype, bias)
     bat = MI.make_batch(T, seed, dtype=dtype, d=d)
     x, ref = _routing_ref(bat, lay, k)
+    ws = torch.empty(api.workspace_size(T, d, E, k, n), dtype=torch.uint8, device="cuda")
     v, idx, w = api.value_routed(P.dev(bat.x, dtype), P.dev(lay.Wr, "f32"), P.dev(lay.br, "f32"),
-                                 P.dev(lay.Wv, dtype), k, 2.5, return_routing=True, path=path)
+                                 P.dev(lay.Wv, dtype), k, 2.5, return_routing=True, path=path, ws=ws)
     torch.cuda.synchronize()
+    assert api.get_status(ws)[0] == "MOVA_OK"
     idx_g = idx.cpu().numpy().astype(np.int64)
-    P.check_routing(idx_g, w.cpu().numpy().astype(np.float64), ref, k, 2.5)
+    rc = P.check_routing(idx_g, w.cpu().numpy().astype(np.float64), ref, k, 2.5)
+    P.check_permutation(api.grouping(ws, T, d, E, k, n), idx_g, E)
     rows = np.arange(T) if sample is None else np.sort(
         np.random.default_rng(seed + 99).choice(T, size=min(sample, T), replace=False))
     # Values of the GPU's (validated) selection with the oracle's weights.
     w_ref = O.weights_for(ref["s"][rows], idx_g[rows], 2.5)
     v_ref = O.combine(x[rows], idx_g[rows], w_ref, lay.Wv, dtype)
-    return P.check_values(P.host_f64(v)[rows], v_ref, dtype), v, idx
+    err = P.check_values(P.host_f64(v)[rows], v_ref, dtype)
+    if record is not None:
+        record("near_tie_tokens", int(rc.near.size))
+        record("differently_chosen_near_ties", int(rc.differ.size))
+        record("value_rows_checked", int(rows.size))
+        record("max_abs_err", err)
+    return err, v, idx
 
 
 def test_full_pr1_fp32(api):
@@ -244,30 +257,60 @@ def test_tensor_given(api):
 
 
 @pytest.mark.parametrize("path", ["auto", "tensor_1cta"])
-def test_full_prefill_4096(api, path):
-    """Prefill workload at full size (T=4096): routing of every token, values
-    of 256 sampled tokens."""
-    _full(api, 4096, 2560, 64, 4, 1024, "bf16", sample=256, path=path)
+def test_full_prefill_4096(api, path, record_property):
+    """Prefill workload at full size (T=4096): routing, grouping and the value
+    of every token, element by element."""
+    _full(api, 4096, 2560, 64, 4, 1024, "bf16", path=path, record=record_property)
 
 
-def test_full_skewed_16384(api):
-    """Skewed prefill (router bias 2 ln Zipf(1.2)), T=16384, sampled values."""
-    _full(api, 16384, 2560, 64, 4, 1024, "bf16", bias="zipf", sample=128)
+def test_full_skewed_16384(api, record_property):
+    """Skewed prefill (router bias 2 ln Zipf(1.2)), T=16384: routing and
+    grouping of every token, values of 1024 sampled tokens."""
+    _full(api, 16384, 2560, 64, 4, 1024, "bf16", bias="zipf", sample=1024, record=record_property)
 
 
 def test_given_32768(api):
-    """Routing-given recompute at L=32768 (int8 indices, fp16 weights),
-    sampled values."""
-    lay = _layer(0, 2560, 64, 1024, "bf16")
-    bat = MI.make_batch(32768, 0, dtype="bf16", mode="given")
+    """Routing-given recompute at L=32768 (int8 indices, fp16 weights): the
+    grouping of every pair bit-exact, values of 1024 sampled rows."""
+    L, d, E, k, n = 32768, 2560, 64, 4, 1024
+    lay = _layer(0, d, E, n, "bf16")
+    bat = MI.make_batch(L, 0, dtype="bf16", mode="given")
+    ws = torch.empty(api.workspace_size(L, d, E, k, n), dtype=torch.uint8, device="cuda")
     v = api.value(P.dev(bat.x, "bf16"), P.dev(bat.idx, "i8"), P.dev(bat.w, "f16"),
-                  P.dev(lay.Wv, "bf16"))
+                  P.dev(lay.Wv, "bf16"), ws=ws)
     torch.cuda.synchronize()
-    assert api.get_status()[0] == "MOVA_OK"
-    rows = np.sort(np.random.default_rng(5).choice(32768, 128, replace=False))
+    assert api.get_status(ws)[0] == "MOVA_OK"
+    P.check_permutation(api.grouping(ws, L, d, E, k, n), bat.idx.astype(np.int64), E)
+    rows = np.sort(np.random.default_rng(5).choice(L, 1024, replace=False))
     v_ref = O.combine(O.to_f64(bat.x[rows], "bf16"), bat.idx[rows].astype(np.int64),
                       bat.w[rows].astype(np.float64), lay.Wv, "bf16")
     P.check_values(P.host_f64(v)[rows], v_ref, "bf16")
+
+
+def test_back_to_back_sizes_share_a_workspace(api):
+    """A large bf16 call followed, with no synchronisation, by a smaller one on
+    the same stream and the same workspace: the second call's kernels start
+    while the first call's last kernels may still run (programmatic dependent
+    launch), and the workspace offsets of the two layouts overlap.  Both
+    results must match the oracle."""
+    d, E, k, n = 2560, 64, 4, 1024
+    lay = _layer(31, d, E, n, "bf16")
+    ws = torch.empty(api.workspace_size(4096, d, E, k, n), dtype=torch.uint8, device="cuda")
+    args = (P.dev(lay.Wr, "f32"), P.dev(lay.br, "f32"), P.dev(lay.Wv, "bf16"))
+    outs = []
+    for T, seed in ((4096, 31), (128, 32), (8, 33), (4096, 34)):
+        bat = MI.make_batch(T, seed, dtype="bf16", d=d)
+        v, idx, _ = api.value_routed(P.dev(bat.x, "bf16"), *args, k, 2.5, return_routing=True, ws=ws)
+        outs.append((bat, v, idx))
+    torch.cuda.synchronize()
+    assert api.get_status(ws)[0] == "MOVA_OK"
+    for bat, v, idx in outs:
+        x, ref = _routing_ref(bat, lay, k)
+        idx_g = idx.cpu().numpy().astype(np.int64)
+        rows = np.arange(min(bat.x.shape[0], 512))
+        P.check_values(P.host_f64(v)[rows],
+                       O.combine(x[rows], idx_g[rows], O.weights_for(ref["s"][rows], idx_g[rows], 2.5),
+                                 lay.Wv, "bf16"), "bf16")
 
 
 def test_tensor_deterministic(api):
@@ -299,6 +342,23 @@ def test_bounded_wait_reports_timeout(api):
     status, _ = api.get_status(ws)
     assert status == "MOVA_ERR_TIMEOUT"
     _full(api, 8, 256, 8, 2, 128, "bf16", seed=77)
+
+
+def test_stream_stall_reports_timeout_and_recovers(api):
+    """Failure detection in the weight-streaming kernel itself: the first CTA
+    stops issuing weight copies at stage 2 and the waits are limited to about
+    a millisecond, so its consumers' wait must run out.  The call reports
+    MOVA_ERR_TIMEOUT, every warp leaves (the call completes), and the next
+    call on the same context gives correct values."""
+    lay = _layer(41, 2560, 64, 1024, "bf16")
+    bat = MI.make_batch(8, 41, dtype="bf16")
+    args = (P.dev(bat.x, "bf16"), P.dev(lay.Wr, "f32"), P.dev(lay.br, "f32"), P.dev(lay.Wv, "bf16"))
+    ws = torch.empty(api.workspace_size(8, 2560, 64, 4, 1024), dtype=torch.uint8, device="cuda")
+    api.arm_stream_stall(2, 2_000_000)
+    api.value_routed(*args, ws=ws)
+    status, detail = api.get_status(ws)
+    assert status == "MOVA_ERR_TIMEOUT" and detail == 0  # the first CTA gave up
+    _full(api, 8, 2560, 64, 4, 1024, "bf16", seed=41)
 
 
 def test_full_zero_tokens(api):
