@@ -9,9 +9,14 @@ A step is one pass of the whole value path over one batch of synthetic tokens
 steps, launched once between a barrier + synchronize on both sides; the expert
 weights rotate over several layers (each layer's weights are read once per
 step, as in a real forward pass), so the weights a step reads are far larger
-than L2.  Per-kernel durations come from stage events recorded inside the
-same graph.  Rank 0 prints one JSON line.  Multi-GPU: one process per GPU,
-each on its own batch (weak scaling, no collective in the data path).
+than L2.  Per-kernel durations come from a second replay with stage events
+recorded inside the graph, less the measured cost of an empty event pair.
+Rank 0 prints one JSON line: the headline workload (--workload, decode T=8 by
+default) and, as sub-records of the same line, the other workloads of the
+metric and scope (--also: prefill T=4096, skewed prefill T=16384,
+routing-given L=32768), each with its own steps, roofline, end-to-end rate and
+CPU baseline.  Multi-GPU: one process per GPU, each on its own batch (weak
+scaling, no collective in the data path).
 """
 from __future__ import annotations
 
@@ -60,8 +65,14 @@ def parse(argv=None):
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="oracle sample budget")
+    ap.add_argument("--cpu-seconds", type=float, default=8.0, help="oracle sample budget")
+    ap.add_argument("--also", default="prefill,skewed,given",
+                    help="workloads measured as sub-records of the same line (comma list; '=' for none)")
     a = ap.parse_args(argv)
+    a.also = [w for w in a.also.split(",") if w and w != "="]
+    for w in a.also:
+        if w not in WORKLOAD_TEXT:
+            ap.error(f"--also: unknown workload {w}")
     if a.steps is None:
         a.steps = DEFAULT_STEPS[a.workload]
     if a.warmup < 3:
@@ -243,28 +254,51 @@ def ncu_traffic(kernel_key, units_per_launch):
 # The CUDA arm
 # ---------------------------------------------------------------------------
 
-def run_mova(a):
+class _Layers:
+    """The L rotated layers' weights on the device (shared by the workloads;
+    the skewed workload swaps in its Zipf router bias)."""
+
+    def __init__(self, a, device, wdt):
+        self.L = max(1, a.layers)
+        self.items = []
+        for l in range(self.L):
+            lay = MI.make_layer(a.seed, l, wv_dtype=wdt)
+            self.items.append((dev_of(lay.Wr, "f32", device), dev_of(lay.br, "f32", device),
+                               dev_of(lay.Wv, wdt, device)))
+            del lay
+        self.zipf = dev_of(MI.zipf_bias(), "f32", device)
+
+    def get(self, l, bias):
+        Wr, br, Wv = self.items[l % self.L]
+        return Wr, (self.zipf if bias == "zipf" else br), Wv
+
+
+def _replay_for(graph, seconds, step_s, K):
+    """Replay `graph` (K steps) back to back for about `seconds` (untimed
+    load around the timed replay, so that the clock sampler sees the GPU
+    under the same load)."""
+    import torch
+    reps = max(1, int(seconds / max(step_s * K, 1e-6)))
+    for _ in range(reps):
+        graph.replay()
+    torch.cuda.synchronize()
+    return reps
+
+
+def measure_workload(a, name, K, layers, device, dist_on, world, rank, peaks, peak_src):
+    """One workload: W warm-up steps, then exactly K steps in one CUDA graph
+    timed with CUDA events between barrier + synchronize (max over ranks);
+    per-kernel durations from a second replay with stage events; the
+    end-to-end rate through the Python API with host buffers."""
     import torch
 
     from mixture_value_routing_b200 import api
 
-    rank, local, world = dist_env()
-    torch.cuda.set_device(local)
-    device = torch.device("cuda", local)
-    dist_on = init_dist(world, "nccl")
-    cfg = MI.WORKLOADS[a.workload]
+    cfg = MI.WORKLOADS[name]
     T, dtype, mode = cfg["T"], cfg["dtype"], cfg["mode"]
     d, E, k, n = MI.D_MODEL, MI.N_EXPERTS, MI.TOP_K, MI.N_OUT
-    L = max(1, a.layers)
-    wdt = "f32" if dtype == "f32" else "bf16"
-
-    layers = []
-    for l in range(L):
-        lay = MI.make_layer(a.seed, l, wv_dtype=wdt, bias=cfg["bias"])
-        layers.append((dev_of(lay.Wr, "f32", device), dev_of(lay.br, "f32", device),
-                       dev_of(lay.Wv, wdt, device)))
-        del lay
-    # One batch per layer position; every rank has its own tokens.
+    L = layers.L
+    xs_b = 2 if dtype == "bf16" else 4
     batches = [MI.make_batch(T, rank_batch_seed(a.seed, rank), step=l, dtype=dtype, mode=mode)
                for l in range(L)]
     xs = [dev_of(b.x, dtype, device) for b in batches]
@@ -279,27 +313,29 @@ def run_mova(a):
 
     def step(i, events=None):
         l = i % L
-        Wr, br, Wv = layers[l]
+        Wr, br, Wv = layers.get(l, cfg["bias"])
         if routing is None:
             api.value_routed(xs[l], Wr, br, Wv, k, MI.SCALE, out=v, ws=ws, events=events)
         else:
             idx, w = routing[l]
             api.value(xs[l], idx, w, Wv, ws=ws, events=events)
 
-    # Distinct experts each layer's step streams (for the decode byte count).
-    distinct = []
+    # Distinct experts each layer's step streams, and the busiest expert's load.
+    distinct, max_load = [], []
     for l in range(L):
         if routing is None:
-            _, idx_l, _ = api.value_routed(xs[l], *layers[l], k, MI.SCALE, return_routing=True)
+            _, idx_l, _ = api.value_routed(xs[l], *layers.get(l, cfg["bias"]), k, MI.SCALE,
+                                           return_routing=True)
         else:
             idx_l = routing[l][0]
-        distinct.append(int(torch.unique(idx_l.long()).numel()))
+        cnt = torch.bincount(idx_l.long().flatten(), minlength=E)
+        distinct.append(int((cnt > 0).sum().item()))
+        max_load.append(int(cnt.max().item()))
 
     for i in range(a.warmup):
         step(i)
     torch.cuda.synchronize()
 
-    K = a.steps
     cap = torch.cuda.Stream()
     cap.wait_stream(torch.cuda.current_stream())
     # The timed graph: K steps back to back, nothing between the kernels (so
@@ -311,11 +347,12 @@ def run_mova(a):
         for i in range(K):
             step(i)
     launches = api.launch_count() - launches0  # kernels the timed graph holds
-    # The same K steps with stage events between the kernels: the per-kernel
-    # durations.  Events serialise the kernels, so this replay is not the
-    # headline number.
+    # The same K steps with stage events between the kernels, plus one empty
+    # event pair per step: stage events serialise the kernels and each event
+    # node costs time of its own, which the empty pair measures.
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(K)]
-    for row in evs:  # torch creates the CUDA event on its first record
+    empty = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)] for _ in range(K)]
+    for row in evs + empty:  # torch creates the CUDA event on its first record
         for e in row:
             e.record()
     torch.cuda.synchronize()
@@ -323,6 +360,8 @@ def run_mova(a):
     with torch.cuda.graph(pgraph, stream=cap):
         for i in range(K):
             step(i, events=evs[i])
+            empty[i][0].record()
+            empty[i][1].record()
     torch.cuda.synchronize()
     graph.replay()  # untimed warm-up replays
     pgraph.replay()
@@ -330,14 +369,20 @@ def run_mova(a):
 
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
-    barrier(dist_on)
+    w0 = time.perf_counter()
+    graph.replay()
     torch.cuda.synchronize()
+    est_step_s = (time.perf_counter() - w0) / K
     with ClockSampler(device) as clk:
+        _replay_for(graph, 0.25, est_step_s, K)
+        barrier(dist_on)
+        torch.cuda.synchronize()
         t0.record()
         graph.replay()
         t1.record()
         torch.cuda.synchronize()
-    barrier(dist_on)
+        barrier(dist_on)
+        _replay_for(graph, 0.25, est_step_s, K)
     ms_local = t0.elapsed_time(t1)
     ms = allmax(ms_local, dist_on, device)
     status, _ = api.get_status(ws)
@@ -349,110 +394,178 @@ def run_mova(a):
     p1.record()
     torch.cuda.synchronize()
     prof_ms = p0.elapsed_time(p1)
-
     stage_ms = {s: 0.0 for s in STAGES}
+    empty_ms = 0.0
     for i in range(K):
         for j, s in enumerate(STAGES):
             stage_ms[s] += evs[i][j].elapsed_time(evs[i][j + 1])
+        empty_ms += empty[i][0].elapsed_time(empty[i][1])
     stage_avg_us = {s: 1e3 * stage_ms[s] / K for s in STAGES}
+    empty_us = 1e3 * empty_ms / K
     del graph, pgraph
 
-    peaks, peak_src = load_peaks()
     ms_per_step = ms / K
     value = job_value(world, T, K, ms)
+    roof = roofline(name, path, T, d, E, k, n, xs_b, distinct, stage_avg_us, empty_us, ms_per_step,
+                    peaks, peak_src)
 
-    # Roofline of the dominant kernel (the expert kernel at these sizes).
-    xs_b = 2 if dtype == "bf16" else 4
-    dom = max(stage_avg_us, key=stage_avg_us.get)
-    if path == "stream" or dom != "experts":
-        Dm = statistics.mean(distinct)
-        expert_bytes = Dm * n * d * xs_b + T * d * xs_b + T * k * n * 4
-        alg = {"route": E * d * 4 + E * 4 + T * d * xs_b + T * k * 8,
-               "group": 3 * T * k * 4 + (2 * E + 1) * 4,
-               "experts": expert_bytes,
-               "combine": T * k * n * 4 + T * n * xs_b + T * k * 4}
-        dur = stage_avg_us[dom] * 1e-6
-        achieved = alg[dom] / dur / 1e9
-        peak = float(peaks["hbm_gbs"])
-        key = {"experts": "experts_stream"}.get(dom, dom)
-        roof = {"kernel": dom, "bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
-                "unit": "GB/s", "frac": round(achieved / peak, 4),
-                "traffic": ncu_traffic(key, Dm if key == "experts_stream" else 1),
-                "algorithmic_bytes_per_launch": int(alg[dom]),
-                "peak_source": f"{peak_src} (hbm_gbs, copy)"}
-    else:
-        flops = 2.0 * T * k * d * n
-        dur = stage_avg_us["experts"] * 1e-6
-        achieved = flops / dur / 1e12
-        peak = float(peaks["bf16_tflops"])
-        roof = {"kernel": "experts", "bound": "tensor", "achieved": round(achieved, 1),
-                "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
-                "traffic": ncu_traffic("experts_tensor", T * k),
-                "algorithmic_flops_per_launch": flops,
-                "peak_source": f"{peak_src} (bf16_tflops, burst)"}
-
-    # End to end through the public API with host buffers.
     e2e = None
     if not a.no_e2e:
-        xh = [torch.empty_like(x, device="cpu").pin_memory() for x in xs]
-        for i, x in enumerate(xs):
-            xh[i].copy_(x)
-        vh = torch.empty((T, n), dtype=tdt).pin_memory()
-        xd = torch.empty_like(xs[0])
-        Ke = min(K, 500)
+        e2e = measure_e2e(a, T, L, xs, routing, layers, cfg, v, ws, k, n, tdt, dist_on, world, device)
 
-        def e2e_step(i):
-            l = i % L
-            xd.copy_(xh[l], non_blocking=True)
-            Wr, br, Wv = layers[l]
-            if routing is None:
-                out = api.value_routed(xd, Wr, br, Wv, k, MI.SCALE, ws=ws)
-            else:
-                out = api.value(xd, routing[l][0], routing[l][1], Wv, ws=ws)
-            vh.copy_(out, non_blocking=True)
-
-        for i in range(a.warmup):
-            e2e_step(i)
-        torch.cuda.synchronize()
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        barrier(dist_on)
-        torch.cuda.synchronize()
-        e0.record()
-        for i in range(Ke):
-            e2e_step(i)
-        e1.record()
-        torch.cuda.synchronize()
-        barrier(dist_on)
-        ems = allmax(e0.elapsed_time(e1), dist_on, device)
-        e2e = {"value": round(job_value(world, T, Ke, ems), 1), "unit": "tokens/s",
-               "h2d_bytes_per_step": int(xs[0].numel() * xs[0].element_size()),
-               "d2h_bytes_per_step": int(vh.numel() * vh.element_size()), "steps": Ke,
-               "ms_per_step": round(ems / Ke, 5)}
-
-    line = {
-        "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
-        "steps": K, "warmup": a.warmup, "ms_per_step": round(ms_per_step, 5),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": dtype,
-        "data": "synthetic (seeded; mova_inputs)",
-        "config": {"workload": WORKLOAD_TEXT[a.workload], "tokens_per_step_per_gpu": T,
+    rec = {
+        "value": round(value, 1), "unit": "tokens/s", "steps": K, "warmup": a.warmup,
+        "ms_per_step": round(ms_per_step, 5), "dtype": dtype,
+        "config": {"workload": WORKLOAD_TEXT[name], "tokens_per_step_per_gpu": T,
                    "layers_rotated": L, "expert_path": path,
                    "l2": f"weights rotate over {L} layers ({L * E * n * d * xs_b / 1e9:.2f} GB) "
                          f"> 126 MB L2; no flush",
-                   "distinct_experts_per_step": distinct, "timing": "one CUDA graph of the K steps, replayed once",
-                   "parallelism": f"dp{world} (independent batches, no collective)"},
+                   "distinct_experts_per_step": distinct, "max_expert_load_per_step": max_load,
+                   "timing": "one CUDA graph of the K steps, replayed once between barrier + "
+                             "synchronize; CUDA events on the replaying stream"},
         "stage_us": {s: round(u, 3) for s, u in stage_avg_us.items()},
-        "stage_timing": f"second replay of the K steps with stage events ({prof_ms / K * 1e3:.2f} us/step)",
+        "event_pair_us": round(empty_us, 3),
+        "stage_timing": f"second replay of the K steps with stage events ({prof_ms / K * 1e3:.2f} us/step); "
+                        f"a kernel's duration = its stage time minus the measured empty event pair",
         "roofline": roof,
         "e2e": e2e,
         "gpu_launches": int(launches),
-        "clocks": clk.summary(),
+        "clocks": dict(clk.summary(), window="sampled from 0.25 s of the same graph replayed before "
+                                             "the timed replay, through it, to 0.25 s after"),
     }
-    if rank == 0 and world == 1 and not a.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(a, budget_s=a.cpu_seconds)
+    return rec
+
+
+def roofline(name, path, T, d, E, k, n, xs_b, distinct, stage_us, empty_us, ms_per_step, peaks,
+             peak_src):
+    """Roofline of the dominant kernel (duration = stage time minus the event
+    pair) and of the whole step (duration = ms_per_step)."""
+    Dm = statistics.mean(distinct)
+    dom = max(stage_us, key=stage_us.get)
+    dur_us = max(stage_us[dom] - empty_us, 1e-3)
+    if path == "stream":
+        kernel_bytes = Dm * n * d * xs_b + T * d * xs_b + T * n * xs_b
+        step_bytes = Dm * n * d * xs_b + E * d * 4 + E * 4 + T * d * xs_b + T * n * xs_b
+        peak = float(peaks["hbm_gbs"])
+        achieved = kernel_bytes / (dur_us * 1e-6) / 1e9
+        step_achieved = step_bytes / (ms_per_step * 1e-3) / 1e9
+        key = "experts_stream"
+        return {"kernel": "stream_experts_kernel (route, group, stream, combine)" if dom == "experts" else dom,
+                "bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                "frac": round(achieved / peak, 4),
+                "frac_of_nominal_8000": round(achieved / 8000.0, 4),
+                "traffic": ncu_traffic(key, Dm) if dom == "experts" else None,
+                "kernel_us": round(dur_us, 3),
+                "algorithmic_bytes_per_launch": int(kernel_bytes),
+                "step": {"achieved": round(step_achieved, 1), "frac": round(step_achieved / peak, 4),
+                         "frac_of_nominal_8000": round(step_achieved / 8000.0, 4),
+                         "algorithmic_bytes_per_step": int(step_bytes)},
+                "peak_source": f"{peak_src} (hbm_gbs, copy)"}
+    flops = 2.0 * T * k * d * n
+    peak = float(peaks["bf16_tflops"])
+    achieved = flops / (dur_us * 1e-6) / 1e12
+    step_achieved = flops / (ms_per_step * 1e-3) / 1e12
+    return {"kernel": "grouped_gemm_pair_kernel" if dom == "experts" else dom,
+            "bound": "tensor", "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
+            "frac": round(achieved / peak, 4), "frac_of_nominal_2250": round(achieved / 2250.0, 4),
+            "traffic": ncu_traffic("experts_tensor", T * k) if dom == "experts" else None,
+            "kernel_us": round(dur_us, 3), "algorithmic_flops_per_launch": flops,
+            "step": {"achieved": round(step_achieved, 1), "frac": round(step_achieved / peak, 4),
+                     "frac_of_nominal_2250": round(step_achieved / 2250.0, 4)},
+            "peak_source": f"{peak_src} (bf16_tflops, burst)"}
+
+
+def measure_e2e(a, T, L, xs, routing, layers, cfg, v, ws, k, n, tdt, dist_on, world, device):
+    """The same metric through the public API with host buffers: per step, the
+    pinned host->device copy of that step's inputs (x, and the stored routing
+    in routing-given mode), the call, and the device->host copy of v."""
+    import torch
+
+    from mixture_value_routing_b200 import api
+    xh = [torch.empty_like(x, device="cpu").pin_memory() for x in xs]
+    for i, x in enumerate(xs):
+        xh[i].copy_(x)
+    rh = None
+    if routing is not None:
+        rh = [(i.cpu().pin_memory(), w.cpu().pin_memory()) for i, w in routing]
+        rd = [torch.empty_like(routing[0][0]), torch.empty_like(routing[0][1])]
+    vh = torch.empty((T, n), dtype=tdt).pin_memory()
+    xd = torch.empty_like(xs[0])
+    Ke = max(3, min(500, int(0.2 / max(1e-6, 2.5e-8 * T * 20))))
+
+    def e2e_step(i):
+        l = i % L
+        xd.copy_(xh[l], non_blocking=True)
+        Wr, br, Wv = layers.get(l, cfg["bias"])
+        if rh is None:
+            out = api.value_routed(xd, Wr, br, Wv, k, MI.SCALE, ws=ws)
+        else:
+            rd[0].copy_(rh[l][0], non_blocking=True)
+            rd[1].copy_(rh[l][1], non_blocking=True)
+            out = api.value(xd, rd[0], rd[1], Wv, ws=ws)
+        vh.copy_(out, non_blocking=True)
+
+    for i in range(a.warmup):
+        e2e_step(i)
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    barrier(dist_on)
+    torch.cuda.synchronize()
+    e0.record()
+    for i in range(Ke):
+        e2e_step(i)
+    e1.record()
+    torch.cuda.synchronize()
+    barrier(dist_on)
+    ems = allmax(e0.elapsed_time(e1), dist_on, device)
+    h2d = xs[0].numel() * xs[0].element_size()
+    if routing is not None:
+        h2d += sum(t.numel() * t.element_size() for t in routing[0])
+    return {"value": round(job_value(world, T, Ke, ems), 1), "unit": "tokens/s",
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(vh.numel() * vh.element_size()),
+            "steps": Ke, "ms_per_step": round(ems / Ke, 5)}
+
+
+def run_mova(a):
+    import torch
+
+    rank, local, world = dist_env()
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    dist_on = init_dist(world, "nccl")
+    peaks, peak_src = load_peaks()
+    head = a.workload
+    wdt = "f32" if MI.WORKLOADS[head]["dtype"] == "f32" else "bf16"
+    layers = _Layers(a, device, wdt)
+    # The headline workload with --steps; the other workloads of the metric
+    # and of the scope (prefill, skewed prefill, routing-given recompute) as
+    # sub-records of the same line, each with its own step count.
+    extras = [w for w in a.also if w != head and MI.WORKLOADS[w]["dtype"] == MI.WORKLOADS[head]["dtype"]]
+    recs = {}
+    for name in [head] + extras:
+        K = a.steps if name == head else DEFAULT_STEPS[name]
+        recs[name] = measure_workload(a, name, K, layers, device, dist_on, world, rank, peaks, peak_src)
+        if rank == 0 and world == 1 and not a.no_cpu_baseline:
+            budget = a.cpu_seconds if name == head or name == "prefill" else a.cpu_seconds / 2
+            recs[name]["cpu_baseline"] = cpu_baseline(a, name, budget_s=budget)
     if dist_on:
         import torch.distributed as dist
         dist.destroy_process_group()
+    h = recs[head]
+    line = {
+        "metric": METRIC, "value": h["value"], "unit": "tokens/s", "n_gpus": world,
+        "steps": a.steps, "warmup": a.warmup, "ms_per_step": h["ms_per_step"],
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": h["dtype"],
+        "data": "synthetic (seeded; mova_inputs)",
+        "config": dict(h["config"], parallelism=f"dp{world} (independent batches, no collective)"),
+        "stage_us": h["stage_us"], "event_pair_us": h["event_pair_us"], "stage_timing": h["stage_timing"],
+        "roofline": h["roofline"], "e2e": h["e2e"], "gpu_launches": h["gpu_launches"], "clocks": h["clocks"],
+    }
+    if "cpu_baseline" in h:
+        line["cpu_baseline"] = h["cpu_baseline"]
+    for name in extras:
+        line[name] = recs[name]
     if rank == 0:
         print(json.dumps(line), flush=True)
 
@@ -480,27 +593,21 @@ def _oracle_tokens(O, lay, bat, rows, mode, wv_dt, dtype):
     return v
 
 
-def cpu_baseline(a, budget_s=12.0, steps=None, warmup=0):
-    """Time the oracle, as it stands, on seeded batches of the same workload:
-    whole steps when they fit the budget, else a sample of tokens per step.
-    `warmup` untimed steps (of at most 8 tokens each) run first."""
-    from oracle import mova_oracle as O
-    cfg = MI.WORKLOADS[a.workload]
-    T, dtype, mode = cfg["T"], cfg["dtype"], cfg["mode"]
-    wdt = "f32" if dtype == "f32" else "bf16"
-    lay = MI.make_layer(a.seed, 0, wv_dtype=wdt, bias=cfg["bias"])
-    bat = MI.make_batch(T, a.seed, dtype=dtype, mode=mode)
-    # Estimate the per-token cost on a small sample first.
-    t = time.perf_counter()
-    _oracle_tokens(O, lay, bat, np.arange(min(T, 4)), mode, wdt, dtype)
-    per_tok = (time.perf_counter() - t) / min(T, 4)
-    if steps is None:
-        rows_per = T if per_tok * T <= budget_s / 3 else max(1, int(budget_s / 3 / per_tok))
-        nsteps = None
-    else:
-        rows_per = T if per_tok * T * steps <= budget_s else max(1, int(budget_s / steps / per_tok))
-        nsteps = steps
-    rng = np.random.default_rng(1234)
+def _cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
+
+
+def _oracle_rate(O, lay, bat, T, mode, wdt, dtype, budget_s, steps, warmup, rows_per, rng):
+    """Tokens/s of the oracle over seeded token samples (whole steps when
+    rows_per == T); runs `steps` steps, or until `budget_s` when steps is None."""
     for _ in range(warmup):
         _oracle_tokens(O, lay, bat, np.arange(min(T, rows_per, 8)), mode, wdt, dtype)
     done = 0
@@ -512,15 +619,53 @@ def cpu_baseline(a, budget_s=12.0, steps=None, warmup=0):
         done += rows.size
         i += 1
         el = time.perf_counter() - t0
-        if (nsteps is not None and i >= nsteps) or (nsteps is None and el >= budget_s):
+        if (steps is not None and i >= steps) or (steps is None and el >= budget_s):
             break
     el = time.perf_counter() - t0
-    return {"value": round(done / el, 3), "unit": "tokens/s", "cores": _blas_threads(),
-            "kind": "oracle",
-            "sample": f"{i} oracle steps of {rows_per} of the {T} tokens of a seeded "
-                      f"{a.workload} batch ({done} tokens, {el:.1f} s, numpy fp64)"
-                      + (f", after {warmup} untimed warm-up steps of up to 8 tokens" if warmup else ""),
-            "steps_timed": i, "seconds": round(el, 2)}
+    return done / el, i, done, el
+
+
+def cpu_baseline(a, name=None, budget_s=8.0, steps=None, warmup=0, one_core=True):
+    """Time the oracle, as it stands, on seeded batches of a workload: whole
+    steps when they fit the budget, else a seeded sample of tokens per step;
+    on all the BLAS threads, then (one_core) on one.  `warmup` untimed steps
+    (of at most 8 tokens each) run first."""
+    from oracle import mova_oracle as O
+    name = name or a.workload
+    cfg = MI.WORKLOADS[name]
+    T, dtype, mode = cfg["T"], cfg["dtype"], cfg["mode"]
+    wdt = "f32" if dtype == "f32" else "bf16"
+    lay = MI.make_layer(a.seed, 0, wv_dtype=wdt, bias=cfg["bias"])
+    bat = MI.make_batch(T, a.seed, dtype=dtype, mode=mode)
+    # Estimate the per-token cost on a small sample first.
+    t = time.perf_counter()
+    _oracle_tokens(O, lay, bat, np.arange(min(T, 4)), mode, wdt, dtype)
+    per_tok = (time.perf_counter() - t) / min(T, 4)
+    share = budget_s / 2 if one_core else budget_s
+    if steps is None:
+        rows_per = T if per_tok * T <= share / 3 else max(1, int(share / 3 / per_tok))
+    else:
+        rows_per = T if per_tok * T * steps <= share else max(1, int(share / steps / per_tok))
+    rate, i, done, el = _oracle_rate(O, lay, bat, T, mode, wdt, dtype, share, steps, warmup, rows_per,
+                                     np.random.default_rng(1234))
+    out = {"value": round(rate, 3), "unit": "tokens/s", "cores": _blas_threads(),
+           "cpu_model": _cpu_model(), "host_cpus": os.cpu_count(),
+           "kind": "oracle",
+           "sample": f"{i} oracle steps of {rows_per} of the {T} tokens of a seeded "
+                     f"{name} batch ({done} tokens, {el:.1f} s, numpy fp64)"
+                     + (f", after {warmup} untimed warm-up steps of up to 8 tokens" if warmup else ""),
+           "steps_timed": i, "seconds": round(el, 2)}
+    if one_core:
+        try:
+            from threadpoolctl import threadpool_limits
+            with threadpool_limits(limits=1):
+                r1, i1, d1, e1 = _oracle_rate(O, lay, bat, T, mode, wdt, dtype, share, None, 0,
+                                              rows_per, np.random.default_rng(4321))
+            out["one_core"] = {"value": round(r1, 3), "unit": "tokens/s", "cores": 1,
+                               "sample": f"{i1} oracle steps of {rows_per} tokens ({d1} tokens, {e1:.1f} s)"}
+        except Exception as e:  # threadpoolctl unavailable: say so
+            out["one_core"] = {"value": None, "note": f"not measured: {e}"}
+    return out
 
 
 def run_reference(a):
@@ -528,7 +673,7 @@ def run_reference(a):
     if rank != 0:
         return
     budget = 150.0
-    cb = cpu_baseline(a, budget_s=budget, steps=a.steps, warmup=a.warmup)
+    cb = cpu_baseline(a, a.workload, budget_s=budget, steps=a.steps, warmup=a.warmup, one_core=False)
     line = {"impl": "reference", "metric": METRIC, "value": cb["value"], "unit": "tokens/s",
             "n_gpus": world, "steps": a.steps, "warmup": a.warmup,
             "ms_per_step": round(1e3 * cb["seconds"] / max(1, cb["steps_timed"]), 3),

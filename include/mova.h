@@ -176,6 +176,63 @@ mova_status mova_value_routed_ex(const void* x, mova_dtype x_dt, const float* Wr
 #define MOVA_WS_PARTS 6
 mova_status mova_workspace_parts(int T, int d, int E, int k, int n, size_t* offsets);
 
+/* Options of the _opts entry points (zero-initialise, then set what is
+ * needed; a NULL options pointer means all defaults).
+ *
+ *  path, events       as for mova_value_ex / mova_value_routed_ex.
+ *
+ *  wv_expert_stride   rows of Wv from one expert's first row to the next
+ *                     expert's (0 means n: the dense (E, n, d) layout).  With
+ *                     a stride the call reads only rows [0, n) of each
+ *                     expert, so a head-parallel rank computes its slice of
+ *                     the value heads straight from a full (E, n_total, d)
+ *                     tensor: pass Wv + row0 * d, n = its rows, stride =
+ *                     n_total.  v then holds that rank's (T, n) slice, i.e.
+ *                     its n / 128 heads.  This is the tensor-parallel serving
+ *                     layout of "IFM/K2-Horizon-MoVA-36B-A4B" (paperfeed.app),
+ *                     "What's actually there, and maturity" (2 GPUs, TP = 2):
+ *                     the router is replicated, every rank routes the same
+ *                     tokens identically, and no collective is needed because
+ *                     the heads stay on their rank.  Must be >= n (else
+ *                     MOVA_ERR_INVALID_ARG); the start of every expert's rows
+ *                     must stay 16-byte aligned.
+ *
+ *  router_partitions  0 or 1: each logit is one fp32 sum over d, in an order
+ *                     the kernels choose.  2: the router's reduction over d
+ *                     runs as two halves, j < d/2 and j >= d/2, each summed in
+ *                     fp32, and the two fp32 partial sums are then added
+ *                     (first + second).  This reproduces a router GEMM split
+ *                     into two K partitions, the setting the serving recipes
+ *                     pass to keep a checkpoint's router numerics
+ *                     ("xllm_source_router_gemm_partitions: 2";
+ *                     "Mixture of Value Attention" (robotsatlas.com),
+ *                     "Implementation pitfalls").  Where partial sums cancel,
+ *                     the rounding of each half to fp32 decides the logit, and
+ *                     so the selection.  Needs d % 128 == 0; other values
+ *                     return MOVA_ERR_UNSUPPORTED. */
+typedef struct mova_options {
+  mova_path path;
+  void* const* events;
+  long long wv_expert_stride;
+  int router_partitions;
+} mova_options;
+
+/* mova_route with options (only router_partitions applies). */
+mova_status mova_route_opts(const void* x, mova_dtype x_dt, const float* Wr, const float* br,
+                            int T, int d, int E, int k, float scale, int32_t* idx, float* w,
+                            const mova_options* opts, void* stream);
+/* mova_value with options (path, events, wv_expert_stride). */
+mova_status mova_value_opts(const void* x, mova_dtype x_dt, const void* idx, mova_dtype idx_dt,
+                            const void* w, mova_dtype w_dt, const void* Wv, mova_dtype wv_dt,
+                            int T, int d, int E, int k, int n, void* v,
+                            void* ws, size_t ws_bytes, const mova_options* opts, void* stream);
+/* mova_value_routed with options (all of them). */
+mova_status mova_value_routed_opts(const void* x, mova_dtype x_dt, const float* Wr, const float* br,
+                                   const void* Wv, mova_dtype wv_dt,
+                                   int T, int d, int E, int k, int n, float scale, void* v,
+                                   int32_t* idx_out, float* w_out,
+                                   void* ws, size_t ws_bytes, const mova_options* opts, void* stream);
+
 /* Synchronises `stream`, then returns and clears the device status word
  * held in `ws` (MOVA_OK if no device-side check fired since the last read).
  * `detail_out` (nullable) receives the first offending item (e.g. the flat

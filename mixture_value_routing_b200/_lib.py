@@ -31,6 +31,13 @@ _i = ctypes.c_int
 _f = ctypes.c_float
 _sz = ctypes.c_size_t
 
+
+class Options(ctypes.Structure):
+    """mova_options (include/mova.h)."""
+    _fields_ = [("path", ctypes.c_int), ("events", ctypes.c_void_p),
+                ("wv_expert_stride", ctypes.c_longlong), ("router_partitions", ctypes.c_int)]
+
+
 SIGNATURES = {
     "mova_status_str": (ctypes.c_char_p, [_i]),
     "mova_workspace_size": (_sz, [_i, _i, _i, _i, _i]),
@@ -51,6 +58,11 @@ SIGNATURES = {
     "mova_workspace_parts": (_i, [_i, _i, _i, _i, _i, _vp]),
     "mova_value_routed_noalloc": (_i, [_vp, _i, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _vp,
                                        _vp]),
+    "mova_route_opts": (_i, [_vp, _i, _vp, _vp, _i, _i, _i, _i, _f, _vp, _vp, _vp, _vp]),
+    "mova_value_opts": (_i, [_vp, _i, _vp, _i, _vp, _i, _vp, _i, _i, _i, _i, _i, _i, _vp, _vp, _sz,
+                             _vp, _vp]),
+    "mova_value_routed_opts": (_i, [_vp, _i, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _vp, _vp,
+                                    _vp, _vp, _sz, _vp, _vp]),
 }
 
 _lib = None

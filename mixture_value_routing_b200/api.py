@@ -85,8 +85,18 @@ def launch_count() -> int:
     return int(_lib.load().mova_launch_count())
 
 
-def route(x: torch.Tensor, Wr: torch.Tensor, br: torch.Tensor, k: int = 4, scale: float = 2.5):
-    """(idx (T, k) int32, w (T, k) fp32)."""
+def _opts(path="auto", events=None, wv_stride=0, partitions=0):
+    """A mova_options value (kept alive by the caller for the call)."""
+    ev = _events(events)
+    o = _lib.Options(_PATH[path], ctypes.cast(ev, ctypes.c_void_p) if ev is not None else None,
+                     int(wv_stride), int(partitions))
+    return o, ev
+
+
+def route(x: torch.Tensor, Wr: torch.Tensor, br: torch.Tensor, k: int = 4, scale: float = 2.5,
+          partitions: int = 0):
+    """(idx (T, k) int32, w (T, k) fp32).  partitions=2 sums the router's two
+    halves of d separately in fp32 and then adds them (mova_options)."""
     _need(x, "x", (torch.float32, torch.bfloat16), 2)
     _need(Wr, "Wr", (torch.float32,), 2)
     _need(br, "br", (torch.float32,), 1)
@@ -95,8 +105,9 @@ def route(x: torch.Tensor, Wr: torch.Tensor, br: torch.Tensor, k: int = 4, scale
     idx = torch.empty((T, k), dtype=torch.int32, device=x.device)
     w = torch.empty((T, k), dtype=torch.float32, device=x.device)
     lib = _lib.load()
-    _lib.check(lib.mova_route(_ptr(x), _DT[x.dtype], _ptr(Wr), _ptr(br), T, d, E, k, float(scale),
-                              _ptr(idx), _ptr(w), _stream()), "mova_route")
+    o, _ = _opts(partitions=partitions)
+    _lib.check(lib.mova_route_opts(_ptr(x), _DT[x.dtype], _ptr(Wr), _ptr(br), T, d, E, k, float(scale),
+                                   _ptr(idx), _ptr(w), ctypes.byref(o), _stream()), "mova_route")
     return idx, w
 
 
@@ -126,25 +137,55 @@ def _events(events):
     return (ctypes.c_void_p * _lib.STAGE_EVENTS)(*[ctypes.c_void_p(e.cuda_event) for e in events])
 
 
+def _expert_view(Wv: torch.Tensor, rows: Optional[tuple]):
+    """(E, n, stride in rows, base tensor) of the experts' rows a call reads:
+    all of Wv, or rows = (row0, count) of every expert (head-parallel slice)."""
+    E, n_total, _ = Wv.shape
+    if rows is None:
+        return E, n_total, 0, Wv
+    row0, count = rows
+    if not (0 <= row0 and count > 0 and row0 + count <= n_total):
+        raise ValueError(f"rows {rows} outside the {n_total} rows of each expert")
+    return E, count, n_total, Wv[:, row0:, :]
+
+
+def head_slice(n_total: int, world: int, rank: int, head_dim: int = 128) -> tuple:
+    """(row0, count) of the expert rows -- whole value heads -- that rank
+    `rank` of `world` head-parallel ranks computes: the heads are dealt in
+    contiguous blocks, the first n_heads % world ranks taking one extra."""
+    if n_total % head_dim != 0:
+        raise ValueError("n_total must be whole heads")
+    heads = n_total // head_dim
+    if not 0 <= rank < world or world > heads:
+        raise ValueError(f"rank {rank} of {world} over {heads} heads")
+    base, extra = divmod(heads, world)
+    h0 = rank * base + min(rank, extra)
+    nh = base + (1 if rank < extra else 0)
+    return h0 * head_dim, nh * head_dim
+
+
 def value(x: torch.Tensor, idx: torch.Tensor, w: torch.Tensor, Wv: torch.Tensor,
           path: str = "auto", ws: Optional[torch.Tensor] = None,
-          events=None) -> torch.Tensor:
-    """Routing-given mixture: v (T, n) in x's dtype."""
+          events=None, rows: Optional[tuple] = None) -> torch.Tensor:
+    """Routing-given mixture: v (T, n) in x's dtype.  rows=(row0, count)
+    computes only rows [row0, row0+count) of every expert (v is (T, count)),
+    reading them in place from the full Wv."""
     _need(x, "x", (torch.float32, torch.bfloat16), 2)
     _need(idx, "idx", (torch.int32, torch.int8), 2)
     _need(w, "w", (torch.float32, torch.float16), 2)
     _need(Wv, "Wv", (x.dtype,), 3)
     T, d = x.shape
-    E, n, _ = Wv.shape
+    E, n, stride, Wb = _expert_view(Wv, rows)
     k = idx.shape[1]
     v = torch.empty((T, n), dtype=x.dtype, device=x.device)
     nbytes = workspace_size(T, d, E, k, n)
     if ws is None:
         ws = _workspace(nbytes, x.device)
     lib = _lib.load()
-    _lib.check(lib.mova_value_ex(_ptr(x), _DT[x.dtype], _ptr(idx), _DT[idx.dtype], _ptr(w),
-                                 _DT[w.dtype], _ptr(Wv), _DT[Wv.dtype], T, d, E, k, n, _ptr(v),
-                                 _ptr(ws), ws.numel(), _PATH[path], _events(events), _stream()),
+    o, _ev = _opts(path, events, stride)
+    _lib.check(lib.mova_value_opts(_ptr(x), _DT[x.dtype], _ptr(idx), _DT[idx.dtype], _ptr(w),
+                                   _DT[w.dtype], _ptr(Wb), _DT[Wv.dtype], T, d, E, k, n, _ptr(v),
+                                   _ptr(ws), ws.numel(), ctypes.byref(o), _stream()),
                "mova_value")
     return v
 
@@ -152,14 +193,17 @@ def value(x: torch.Tensor, idx: torch.Tensor, w: torch.Tensor, Wv: torch.Tensor,
 def value_routed(x: torch.Tensor, Wr: torch.Tensor, br: torch.Tensor, Wv: torch.Tensor,
                  k: int = 4, scale: float = 2.5, return_routing: bool = False,
                  path: str = "auto", ws: Optional[torch.Tensor] = None,
-                 out: Optional[torch.Tensor] = None, events=None):
-    """Full value path: v (T, n) in x's dtype [, idx (T, k) int32, w (T, k) fp32]."""
+                 out: Optional[torch.Tensor] = None, events=None, rows: Optional[tuple] = None,
+                 partitions: int = 0):
+    """Full value path: v (T, n) in x's dtype [, idx (T, k) int32, w (T, k) fp32].
+    rows=(row0, count): only those rows of every expert (a head-parallel
+    slice, v is (T, count)); partitions=2: the router's two-partition sum."""
     _need(x, "x", (torch.float32, torch.bfloat16), 2)
     _need(Wr, "Wr", (torch.float32,), 2)
     _need(br, "br", (torch.float32,), 1)
     _need(Wv, "Wv", (x.dtype,), 3)
     T, d = x.shape
-    E, n, _ = Wv.shape
+    E, n, stride, Wb = _expert_view(Wv, rows)
     dev = x.device
     v = out if out is not None else torch.empty((T, n), dtype=x.dtype, device=dev)
     idx = w = None
@@ -170,10 +214,11 @@ def value_routed(x: torch.Tensor, Wr: torch.Tensor, br: torch.Tensor, Wv: torch.
     if ws is None:
         ws = _workspace(nbytes, dev)
     lib = _lib.load()
-    _lib.check(lib.mova_value_routed_ex(_ptr(x), _DT[x.dtype], _ptr(Wr), _ptr(br), _ptr(Wv),
-                                        _DT[Wv.dtype], T, d, E, k, n, float(scale), _ptr(v),
-                                        _ptr(idx), _ptr(w), _ptr(ws), ws.numel(), _PATH[path],
-                                        _events(events), _stream()), "mova_value_routed")
+    o, _ev = _opts(path, events, stride, partitions)
+    _lib.check(lib.mova_value_routed_opts(_ptr(x), _DT[x.dtype], _ptr(Wr), _ptr(br), _ptr(Wb),
+                                          _DT[Wv.dtype], T, d, E, k, n, float(scale), _ptr(v),
+                                          _ptr(idx), _ptr(w), _ptr(ws), ws.numel(), ctypes.byref(o),
+                                          _stream()), "mova_value_routed")
     if return_routing:
         return v, idx, w
     return v

@@ -1,38 +1,45 @@
 // Grouped expert GEMM on an SM pair (tcgen05 cta_group::2), bf16 -> fp32.
 //
-// Same computation as grouped_gemm_tc.cu -- for every pair p routed to
-// expert e, P[p, r] = SiLU(Wv[e, r, :] . x[t(p), :]) ("MoVA: routing the
-// value vectors, and why the KV cache does not notice", section "Where the
-// routing happens"; the combine weights and sums the slots) -- with the MMA's
-// M side spread over a cluster of two CTAs on neighbouring SMs:
+// For every pair p = (token t, slot) routed to expert e,
+//   P[p, r] = SiLU(Wv[e, r, :] . x[t, :])
+// ("MoVA: routing the value vectors, and why the KV cache does not notice",
+// section "Where the routing happens": each selected expert's projection
+// passes through SiLU; the combine weights it and sums the slots).  At
+// prefill sizes this is a dense contraction -- 2 T k d n flop, 85.9 GFLOP
+// at T = 4096 ("So what does it cost?": 10.49M multiply-accumulates per
+// token) -- so it runs on the tensor cores:
 //
-//   * a tile is 256 weight rows x up to 256 pairs of one expert; the even CTA
-//     holds weight rows 0..127 and the first half of the pairs, the odd CTA
-//     rows 128..255 and the second half; one tcgen05.mma.cta_group::2 (M =
-//     256, N <= 256, K = 16) reads both CTAs' shared memory and accumulates
-//     into both CTAs' tensor memory (each its own 128 rows).
-//   * Each CTA therefore loads per 64-wide K step only 16 KB of weights and
-//     16 KB of token rows (vs 16 + 32 KB for one CTA doing half the work), and
-//     the token tile is read n/256 instead of n/128 times.  Six 32 KB stages.
-//   * Each CTA's TMA warp loads its own halves with 2-D tensor-map loads (no
-//     multicast); completion is counted on the even CTA's stage barrier, for
-//     which the even CTA alone declares the byte count of both halves.
-//   * The even CTA's MMA thread issues the MMAs; tcgen05.commit with a
-//     two-CTA multicast frees the stage in both CTAs and hands both
-//     accumulators to the epilogues.  The odd CTA's epilogue releases an
-//     accumulator with a remote arrive on the even CTA's barrier.
-//   * Warps: 0 TMA, 1 MMA (even CTA), 2-5 epilogue (SiLU, bf16, store; rows
-//     beyond the expert's n are skipped).  The epilogue reads the whole
-//     accumulator into registers (bf16 pairs) and hands it back before it
-//     stores, so the MMA of the tile after next never waits for the stores.
-//   * One persistent pair per two SMs takes tiles from a global counter as
-//     it goes (the even CTA's producer fetches the id and publishes it to
-//     every role of both CTAs through a ring of mbarrier-guarded slots), so
-//     unequal tile sizes do not leave some pairs a whole tile behind.  Tile
-//     ids run expert by expert with the 4 weight-row tiles of a token tile
-//     adjacent, so pairs working at the same time share the token rows in L2.
-// Every mbarrier wait is bounded (MOVA_ERR_TIMEOUT); both CTAs meet at a
-// cluster barrier before tensor memory is freed.
+//   * A tile is 256 weight rows of one expert (the MMA's M side, 128 rows in
+//     each CTA of a two-CTA cluster) against up to 512 of that expert's
+//     pairs (the N side, in two tensor-memory accumulators of up to 256
+//     columns).  At ~256 pairs per expert every expert's weights are then
+//     read once per 256-row block, and its pairs' token rows once per block.
+//   * The token rows come from xp, the pairs' rows of x already gathered into
+//     grouped order, so each CTA's share of a tile is two runs of consecutive
+//     rows that 2-D TMA boxes of 32 rows load (TMA tile::gather4 straight from
+//     x was measured at ~18 GB/s per SM, too slow to feed the MMA).
+//   * Per 64-wide K step a CTA loads 16 KB of weights (one 2-D box) and up to
+//     32 KB of token rows (its half of the tile's pairs: accumulator 0's rows
+//     at the start of the stage's B area, accumulator 1's 16 KB further);
+//     four 48 KB stages.
+//     Both CTAs' copies complete on the even CTA's stage barrier (no
+//     multicast).  The even CTA's MMA warp issues tcgen05.mma.cta_group::2
+//     (M = 256, N = 16..256, K = 16) into accumulator 0 (pairs 0..255 of the
+//     tile) and accumulator 1 (pairs 256..511); tcgen05.commit multicast
+//     frees the stage in both CTAs.
+//   * Eight epilogue warps: four per accumulator, one per tensor-memory lane
+//     quarter.  Each reads its accumulator's columns into registers (SiLU,
+//     bf16) in two halves, storing the first half before reading the second,
+//     and hands the accumulator back right after its last read, so the next
+//     tile's MMAs wait for the reads and one half's stores only.
+//   * One persistent pair per two SMs takes tiles from a global counter;
+//     tiles are numbered largest expert first (then token tile, then the
+//     four weight-row blocks of a token tile next to each other, so pairs
+//     working at the same time share the token rows in L2), so the last
+//     tiles handed out are the smallest.
+// Every mbarrier wait is bounded (MOVA_ERR_TIMEOUT); on a failed wait every
+// role leaves its loop, the copies and MMAs in flight are drained and tensor
+// memory is freed.  Both CTAs meet at a cluster barrier before exiting.
 #include <cuda.h>
 
 #include "common.cuh"
@@ -43,43 +50,44 @@ namespace mova {
 
 namespace {
 
-constexpr int PM = 128;          // weight rows per CTA (256 per pair)
-constexpr int PN = 256;          // pairs per tile
+constexpr int PM = 128;         // weight rows per CTA (256 per pair)
+constexpr int NA = 256;         // pairs per accumulator
+constexpr int NT = 2 * NA;      // pairs per tile
 constexpr int PK = 64;
-constexpr int kPStages = 6;
-// Tile ids handed out dynamically pass through a ring in both CTAs'
-// shared memory.  A role can lag the leader's producer by at most 8 tiles:
-// the producer leads the MMA by at most kPStages k-steps (so at most 6
-// tiles), the MMA leads the epilogues by the 2 accumulators.
+constexpr int kPStages = 4;
 constexpr int kTileRing = 16;
-constexpr int kPABytes = PM * PK * 2;
-constexpr int kPBBytes = (PN / 2) * PK * 2;
+constexpr int kPABytes = PM * PK * 2;           // 16 KB of weights per stage
+constexpr int kPBBytes = (NT / 2) * PK * 2;     // up to 32 KB of token rows
 constexpr int kPStageBytes = kPABytes + kPBBytes;
-constexpr int kPBoxRows = 32;
-constexpr int kPThreads = 6 * 32;
+constexpr int kEpiWarps = 8;
+constexpr int kPThreads = (2 + kEpiWarps) * 32;  // warp 0 TMA, warp 1 MMA, 2-9 epilogue
 constexpr uint32_t kPTmemCols = 512;
 
 struct __align__(1024) PSmem {
   uint8_t stage[kPStages][kPStageBytes];
-  uint64_t full[kPStages];   // even CTA: both halves of the stage landed
-  uint64_t empty[kPStages];  // both CTAs: the pair's MMAs on the stage are done
-  uint64_t tmem_full[2];     // both CTAs
-  uint64_t tmem_empty[2];    // even CTA: 4 epilogue warps x 2 CTAs
+  uint64_t full[kPStages];      // even CTA: both CTAs' copies of the stage landed
+  uint64_t empty[kPStages];     // both CTAs: the pair's MMAs on the stage are done
+  uint64_t tmem_full;           // both CTAs: the tile's accumulators are complete
+  uint64_t acc_empty[2];        // even CTA: accumulator a read by 4 warps x 2 CTAs
   uint64_t tq_full[kTileRing];  // both CTAs: tile id i of this cluster published
   int tq[kTileRing];
   uint32_t tmem_base;
   int abort;
   int ntiles;
   int nact;
+  // Active experts in tile order (largest pair count first).
   int act_e[64];
   int act_cnt[64];
   int act_off[64];
   int act_ntt[64];
   int tile_base[65];
+  // Scratch of the ordering: the active experts in ascending order.
+  int raw_e[64];
+  int raw_cnt[64];
 };
 
 struct PTile {
-  int e, mt, tok0, valid, N, off;
+  int e, mt, tok0, valid, N0, N1, off;
 };
 
 __device__ __forceinline__ PTile decode_ptile(const PSmem& S, int t, int mtiles) {
@@ -94,7 +102,9 @@ __device__ __forceinline__ PTile decode_ptile(const PSmem& S, int t, int mtiles)
   r.mt = local - tt * mtiles;
   r.tok0 = static_cast<int>(static_cast<long long>(tt) * cnt / ntt);
   r.valid = static_cast<int>(static_cast<long long>(tt + 1) * cnt / ntt) - r.tok0;
-  r.N = (r.valid + 15) & ~15;
+  const int N = (r.valid + 15) & ~15;
+  r.N0 = min(N, NA);
+  r.N1 = N - r.N0;
   r.off = S.act_off[a];
   return r;
 }
@@ -115,11 +125,14 @@ __device__ __forceinline__ void p_fail(PSmem& S, StatusBlock* sb) {
   *reinterpret_cast<volatile int*>(&S.abort) = 1;
 }
 
+constexpr int kBoxRows = 32;                    // token rows per TMA box
+constexpr int kAcc1Rows = NA / 2;               // accumulator 1's rows start here in B
+
 __global__ void __launch_bounds__(kPThreads, 1)
 grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_xp,
                          const int32_t* __restrict__ counts, const int32_t* __restrict__ offsets,
                          const int32_t* __restrict__ active, StatusBlock* __restrict__ sb, int d, int n,
-                         __nv_bfloat16* __restrict__ P) {
+                         int ldw, __nv_bfloat16* __restrict__ P) {
   extern __shared__ uint8_t smem_raw[];
   PSmem& S = *reinterpret_cast<PSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5;
@@ -133,10 +146,8 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_w, const __gri
       mbar_init(&S.full[s], 1);
       mbar_init(&S.empty[s], 1);
     }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&S.tmem_full[i], 1);
-      mbar_init(&S.tmem_empty[i], 8);
-    }
+    mbar_init(&S.tmem_full, 1);
+    for (int i = 0; i < 2; ++i) mbar_init(&S.acc_empty[i], 4 * 2);
     for (int i = 0; i < kTileRing; ++i) mbar_init(&S.tq_full[i], 1);
     S.abort = 0;
     fence_barrier_init();
@@ -145,26 +156,36 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_w, const __gri
     tmem_alloc_pair(&S.tmem_base, kPTmemCols);
     tmem_relinquish_pair();
   }
-  pdl_wait();  // grouping and gathered rows of this call are complete and visible
+  pdl_wait();  // the grouping of this call is complete and visible
   if (threadIdx.x < 32) {
+    // Active experts, then their order by pair count (descending; equal
+    // counts keep ascending expert order), then the tile prefix.
     const int nact = sb->num_active;
-    int ntt0 = 0, ntt1 = 0;
+    for (int a = lane; a < 64; a += 32) {
+      if (a < nact) {
+        const int e = active[a];
+        S.raw_e[a] = e;
+        S.raw_cnt[a] = counts[e];
+      }
+    }
+    __syncwarp();
+    for (int a = lane; a < nact; a += 32) {
+      const int c = S.raw_cnt[a];
+      int rk = 0;
+      for (int b = 0; b < nact; ++b) {
+        const int cb = S.raw_cnt[b];
+        rk += (cb > c || (cb == c && b < a)) ? 1 : 0;
+      }
+      const int e = S.raw_e[a];
+      S.act_e[rk] = e;
+      S.act_cnt[rk] = c;
+      S.act_off[rk] = offsets[e];
+      S.act_ntt[rk] = (c + NT - 1) / NT;
+    }
+    __syncwarp();
     const int a0 = lane, a1 = lane + 32;
-    if (a0 < nact) {
-      const int e = active[a0];
-      const int c = counts[e];
-      S.act_e[a0] = e; S.act_cnt[a0] = c; S.act_off[a0] = offsets[e];
-      ntt0 = (c + PN - 1) / PN;
-      S.act_ntt[a0] = ntt0;
-    }
-    if (a1 < nact) {
-      const int e = active[a1];
-      const int c = counts[e];
-      S.act_e[a1] = e; S.act_cnt[a1] = c; S.act_off[a1] = offsets[e];
-      ntt1 = (c + PN - 1) / PN;
-      S.act_ntt[a1] = ntt1;
-    }
-    int v0 = ntt0 * mtiles, v1 = ntt1 * mtiles;
+    int v0 = a0 < nact ? S.act_ntt[a0] * mtiles : 0;
+    int v1 = a1 < nact ? S.act_ntt[a1] * mtiles : 0;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const int y0 = __shfl_up_sync(0xffffffffu, v0, o);
@@ -181,18 +202,16 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_w, const __gri
     if (lane == 31) S.ntiles = tot0 + v1;
   }
   tc_fence_before();
-  cluster_sync_all();  // barriers and tensor memory of both CTAs are ready
+  cluster_sync_all();  // barriers, expert order and tensor memory of both CTAs are ready
   tc_fence_after();
   pdl_trigger();
   const int ntiles = S.ntiles;
 
   if (warp == 0) {
     // The whole warp runs the loop (warp-uniform state); one elected lane
-    // issues the copies.  Stage and barrier addresses are computed once.
-    // Tiles are handed out one at a time from a counter (zeroed by the
-    // grouping of this call), so the clusters finish together however the
-    // tile sizes fall.  The even CTA's producer takes each id and publishes it
-    // to both CTAs; it requests the following id while it loads a tile.
+    // declares the stage's bytes and issues the copies.  The even CTA's
+    // producer takes the tile ids from the global counter (zeroed by this
+    // call's grouping) and publishes each to both CTAs.
     const uint32_t full0_cl = mapa_shared(smem_u32(&S.full[0]), 0);  // even CTA's barriers
     int s = 0;
     uint32_t phase = 0;
@@ -226,11 +245,18 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_w, const __gri
         if (t >= ntiles) break;
       }
       const PTile tl = decode_ptile(S, t, mtiles);
-      const int arow = tl.e * n + tl.mt * 2 * PM + static_cast<int>(rank) * PM;
-      const int half = tl.N / 2;
-      const int brow = tl.off + tl.tok0 + static_cast<int>(rank) * half;
-      const int nbox = (half + kPBoxRows - 1) / kPBoxRows;
-      const uint32_t bytes = 2u * static_cast<uint32_t>(kPABytes + nbox * kPBoxRows * PK * 2);
+      const int arow = tl.e * ldw + tl.mt * 2 * PM + static_cast<int>(rank) * PM;
+      // This CTA's B rows: the first half (rank 0) or second half (rank 1)
+      // of accumulator 0's pairs, then likewise of accumulator 1's, each a
+      // run of consecutive xp rows.  Boxes of 32 rows may read past a run's
+      // end (rows of the next pairs, or zeros past the last pair): those rows
+      // land inside the run's 16 KB of B and no MMA reads them.
+      const int h0 = tl.N0 / 2, h1 = tl.N1 / 2;
+      const int row0 = tl.off + tl.tok0 + static_cast<int>(rank) * h0;
+      const int row1 = tl.off + tl.tok0 + tl.N0 + static_cast<int>(rank) * h1;
+      const int nb0 = (h0 + kBoxRows - 1) / kBoxRows;
+      const int nb1 = (h1 + kBoxRows - 1) / kBoxRows;
+      const uint32_t bytes = 2u * static_cast<uint32_t>(kPABytes + (nb0 + nb1) * kBoxRows * PK * 2);
       bool ok = true;
       for (int kb = 0; kb < nk; ++kb) {
         // Slot s was used before (from the second pass over the ring on):
@@ -240,13 +266,17 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_w, const __gri
           ok = false;
           break;
         }
+        const uint32_t full_cl = full0_cl + static_cast<uint32_t>(s) * 8u;
+        uint8_t* st = S.stage[s];
         if (elect_one()) {
-          const uint32_t full_cl = full0_cl + static_cast<uint32_t>(s) * 8u;
           if (rank == 0) mbar_arrive_expect_tx(&S.full[s], bytes);
-          uint8_t* st = S.stage[s];
           tma_load_2d_pair(st, &tmap_w, kb * PK, arow, full_cl);
-          for (int b = 0; b < nbox; ++b)
-            tma_load_2d_pair(st + kPABytes + b * kPBoxRows * 128, &tmap_xp, kb * PK, brow + b * kPBoxRows, full_cl);
+          uint8_t* bt = st + kPABytes;
+          for (int b = 0; b < nb0; ++b)
+            tma_load_2d_pair(bt + b * kBoxRows * 128, &tmap_xp, kb * PK, row0 + b * kBoxRows, full_cl);
+          for (int b = 0; b < nb1; ++b)
+            tma_load_2d_pair(bt + (kAcc1Rows + b * kBoxRows) * 128, &tmap_xp, kb * PK, row1 + b * kBoxRows,
+                             full_cl);
         }
         __syncwarp();
         if (++s == kPStages) {
@@ -259,11 +289,9 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_w, const __gri
     }
   } else if (warp == 1) {
     if (rank == 0) {
-      // The whole warp runs the loop (so its state stays warp-uniform); one
-      // elected lane issues the MMAs and commits.  Stage descriptors are
-      // built once and advanced by adding offsets (start address in 16-byte
-      // units), which keeps the issue cost below the MMA time even at
-      // N = 144.
+      // The whole warp runs the loop; one elected lane issues the MMAs and
+      // commits.  Stage descriptors are built once and advanced by adding
+      // offsets (start address in 16-byte units).
       const uint64_t adesc0 = smem_desc_sw128(smem_u32(S.stage[0]));
       const uint64_t bdesc0 = smem_desc_sw128(smem_u32(S.stage[0]) + kPABytes);
       constexpr uint32_t kStageDesc = kPStageBytes >> 4;
@@ -277,16 +305,23 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_w, const __gri
         }
         if (t >= ntiles || p_aborted(S)) break;
         const PTile tl = decode_ptile(S, t, mtiles);
-        const int acc = titer & 1;
-        if (titer >= 2 && !__all_sync(0xffffffffu, mbar_wait(&S.tmem_empty[acc], ((titer / 2) - 1) & 1))) {
-          if (lane == 0) p_fail(S, sb);
-          break;
-        }
-        tc_fence_after();
-        const uint32_t d_tmem = S.tmem_base + static_cast<uint32_t>(acc * PN);
-        const uint32_t idesc = idesc_bf16_f32(2 * PM, tl.N);
+        const uint32_t idesc0 = idesc_bf16_f32(2 * PM, tl.N0);
+        const uint32_t idesc1 = idesc_bf16_f32(2 * PM, tl.N1 > 0 ? tl.N1 : 16);
+        // Accumulator 1's B rows start kAcc1Rows rows into each CTA's B area.
+        const uint64_t b1off = static_cast<uint64_t>(kAcc1Rows * PK * 2) >> 4;
         bool ok = true;
         for (int kb = 0; kb < nk; ++kb) {
+          if (kb == 0 && titer > 0) {
+            // Both accumulators must have been read out by the previous
+            // tile's epilogues (every tile's epilogues release both).
+            const uint32_t par = (titer - 1) & 1;
+            if (!__all_sync(0xffffffffu, mbar_wait(&S.acc_empty[0], par) && mbar_wait(&S.acc_empty[1], par))) {
+              if (lane == 0) p_fail(S, sb);
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+          }
           if (!__all_sync(0xffffffffu, mbar_wait(&S.full[s], phase))) {
             if (lane == 0) p_fail(S, sb);
             ok = false;
@@ -298,7 +333,13 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_w, const __gri
           if (elect_one()) {
 #pragma unroll
             for (int k16 = 0; k16 < PK / 16; ++k16)
-              tc_mma_bf16_pair(d_tmem, da + 2 * k16, db + 2 * k16, idesc, (kb | k16) != 0);
+              tc_mma_bf16_pair(S.tmem_base, da + 2 * k16, db + 2 * k16, idesc0, (kb | k16) != 0);
+            if (tl.N1 > 0) {
+#pragma unroll
+              for (int k16 = 0; k16 < PK / 16; ++k16)
+                tc_mma_bf16_pair(S.tmem_base + NA, da + 2 * k16, db + b1off + 2 * k16, idesc1,
+                                 (kb | k16) != 0);
+            }
             tc_commit_pair_both(&S.empty[s]);
           }
           __syncwarp();
@@ -308,59 +349,71 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_w, const __gri
           }
         }
         if (!ok) break;
-        if (elect_one()) tc_commit_pair_both(&S.tmem_full[acc]);
+        if (elect_one()) tc_commit_pair_both(&S.tmem_full);
         __syncwarp();
       }
     }
   } else {
-    const int lg = warp & 3;  // this warp may access TMEM lanes 32*lg .. 32*lg+31
-    const uint32_t empty0 = mapa_shared(smem_u32(&S.tmem_empty[0]), 0);
-    const uint32_t empty1 = mapa_shared(smem_u32(&S.tmem_empty[1]), 0);
-    int titer = 0;
-    for (;; ++titer) {
+    // Epilogue: warp w reads tensor-memory lanes 32 * (w % 4) .. +31 (its
+    // CTA's weight rows) of accumulator (w - 2) / 4.
+    const int q = warp & 3;
+    const int acc = (warp - 2) / 4;
+    const uint32_t empty_cl = mapa_shared(smem_u32(&S.acc_empty[acc]), 0);
+    for (int titer = 0;; ++titer) {
       const int t = next_tile(S, titer);
       if (t < 0) { p_fail(S, sb); break; }
       if (t >= ntiles || p_aborted(S)) break;
       const PTile tl = decode_ptile(S, t, mtiles);
-      const int acc = titer & 1;
-      if (!mbar_wait(&S.tmem_full[acc], (titer / 2) & 1)) { p_fail(S, sb); break; }
+      if (!mbar_wait(&S.tmem_full, titer & 1)) { p_fail(S, sb); break; }
       tc_fence_after();
-      const int rloc = tl.mt * 2 * PM + static_cast<int>(rank) * PM + lg * 32 + lane;
-      const uint32_t tbase = S.tmem_base + static_cast<uint32_t>(acc * PN) +
-                             (static_cast<uint32_t>(lg * 32) << 16);
+      const int N = acc == 0 ? tl.N0 : tl.N1;
+      const int j0 = acc == 0 ? 0 : tl.N0;  // the tile's pair of this accumulator's column 0
+      const int nvalid = min(N, tl.valid - j0);
+      const int rloc = tl.mt * 2 * PM + static_cast<int>(rank) * PM + q * 32 + lane;
+      const uint32_t tbase = S.tmem_base + static_cast<uint32_t>(acc * NA) + (static_cast<uint32_t>(q * 32) << 16);
+      // The accumulator's columns are read in two halves of 128 (SiLU,
+      // rounded to bf16, two per word): the first half is read and stored,
+      // then the second half is read, the accumulator is handed back to the
+      // MMA, and the second half is stored.  (Three of the ten warps share a
+      // sub-partition's 16K registers, so a thread cannot hold all 256
+      // columns at once.)
       unsigned short* prow =
-          reinterpret_cast<unsigned short*>(P + static_cast<size_t>(tl.off + tl.tok0) * n + rloc);
+          reinterpret_cast<unsigned short*>(P + static_cast<size_t>(tl.off + tl.tok0 + j0) * n + rloc);
       const bool live = rloc < n;
-      // All of the tile's columns go to registers first (SiLU, rounded to
-      // bf16, two per word), so the accumulator is handed back to the MMA
-      // before the stores start.
-      uint32_t pk[PN / 32][16];
 #pragma unroll
-      for (int c = 0; c < PN / 32; ++c) {
-        if (c * 32 < tl.N) {
-          uint32_t r[32];
-          tmem_ld_32(tbase + c * 32, r);
-          tmem_ld_wait();
+      for (int h = 0; h < 2; ++h) {
+        uint32_t pk[4][16];
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const __nv_bfloat162 h = __floats2bfloat162_rn(silu_fast(__uint_as_float(r[2 * j])),
-                                                           silu_fast(__uint_as_float(r[2 * j + 1])));
-            pk[c][j] = *reinterpret_cast<const uint32_t*>(&h);
+        for (int c = 0; c < 4; ++c) {
+          const int cc = 4 * h + c;
+          if (cc * 32 < N) {
+            uint32_t r[32];
+            tmem_ld_32(tbase + cc * 32, r);
+            tmem_ld_wait();
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              const __nv_bfloat162 v2 = __floats2bfloat162_rn(silu_fast(__uint_as_float(r[2 * j])),
+                                                              silu_fast(__uint_as_float(r[2 * j + 1])));
+              pk[c][j] = *reinterpret_cast<const uint32_t*>(&v2);
+            }
           }
         }
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(acc == 0 ? empty0 : empty1);
-      if (live) {
+        if (h == 1) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive_cluster(empty_cl);
+        }
+        if (live) {
 #pragma unroll
-        for (int c = 0; c < PN / 32; ++c) {
+          for (int c = 0; c < 4; ++c) {
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const int col = c * 32 + j;
-            if (col < tl.valid) {
-              const uint32_t wv = pk[c][j >> 1];
-              prow[static_cast<size_t>(col) * n] = static_cast<unsigned short>((j & 1) ? (wv >> 16) : (wv & 0xFFFFu));
+            for (int j = 0; j < 32; ++j) {
+              const int col = (4 * h + c) * 32 + j;
+              if (col < nvalid) {
+                const uint32_t wv = pk[c][j >> 1];
+                prow[static_cast<size_t>(col) * n] =
+                    static_cast<unsigned short>((j & 1) ? (wv >> 16) : (wv & 0xFFFFu));
+              }
             }
           }
         }
@@ -387,28 +440,32 @@ using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, 
 
 }  // namespace
 
-cudaError_t launch_tensor_experts_pair(const void* Wv, const int32_t* counts, const int32_t* offsets,
-                                       const int32_t* active, StatusBlock* sb, int T, int d, int n,
-                                       int k, int E, const __nv_bfloat16* xp, __nv_bfloat16* P,
+cudaError_t launch_tensor_experts_pair(const void* Wv, long long ldw, const int32_t* counts,
+                                       const int32_t* offsets, const int32_t* active, StatusBlock* sb, int T,
+                                       int d, int n, int k, int E, const __nv_bfloat16* xp, __nv_bfloat16* P,
                                        cudaStream_t stream) {
   void* fp = encode_tiled_fn();
   if (fp == nullptr) return cudaErrorNotSupported;
   EncodeTiled enc = reinterpret_cast<EncodeTiled>(fp);
-  const int N = T * k;
   CUtensorMap tmap_w, tmap_xp;
-  const cuuint64_t gdim[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(E) * n};
-  const cuuint64_t xdim[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N)};
+  // The experts' rows as one matrix: expert e's row r is row e * ldw + r;
+  // rows between n and ldw (another rank's slice) are read by a weight tile
+  // that runs past n but never stored.
+  const cuuint64_t gdim[2] = {static_cast<cuuint64_t>(d),
+                              static_cast<cuuint64_t>(E - 1) * static_cast<cuuint64_t>(ldw) + n};
+  const cuuint64_t xdim[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(T) * k};
   const cuuint64_t gstride[1] = {static_cast<cuuint64_t>(d) * 2};
   const cuuint32_t box[2] = {PK, PM};
-  const cuuint32_t xbox[2] = {PK, kPBoxRows};
+  const cuuint32_t xbox[2] = {PK, kBoxRows};
   const cuuint32_t estride[2] = {1, 1};
   if (enc(&tmap_w, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(Wv), gdim, gstride, box,
           estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
-  if (enc(&tmap_xp, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<__nv_bfloat16*>(xp), xdim, gstride,
-          xbox, estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+  if (enc(&tmap_xp, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<__nv_bfloat16*>(xp), xdim, gstride, xbox,
+          estride,
+          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
   const size_t smem = sizeof(PSmem) + 1024;
   cudaError_t err = cudaFuncSetAttribute(grouped_gemm_pair_kernel,
@@ -437,8 +494,9 @@ cudaError_t launch_tensor_experts_pair(const void* Wv, const int32_t* counts, co
     max_clusters = c;
   }
   cfg.gridDim = dim3(2 * max_clusters);
-  return cudaLaunchKernelEx(&cfg, grouped_gemm_pair_kernel, tmap_w, tmap_xp, counts, offsets, active, sb,
-                            d, n, P);
+  note_launch();
+  return cudaLaunchKernelEx(&cfg, grouped_gemm_pair_kernel, tmap_w, tmap_xp, counts, offsets, active, sb, d, n,
+                            static_cast<int>(ldw), P);
 }
 
 }  // namespace mova

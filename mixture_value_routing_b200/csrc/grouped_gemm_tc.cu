@@ -111,7 +111,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_xp,
                     const int32_t* __restrict__ counts, const int32_t* __restrict__ offsets,
                     const int32_t* __restrict__ active, StatusBlock* __restrict__ sb, int d,
-                    int n, __nv_bfloat16* __restrict__ P) {
+                    int n, int ldw, __nv_bfloat16* __restrict__ P) {
   extern __shared__ uint8_t smem_raw[];
   Smem& S = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5;
@@ -182,7 +182,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_con
       int it = 0;
       for (int t = blockIdx.x; t < ntiles && !aborted(S); t += gridDim.x) {
         const Tile tl = decode_tile(S, t, mtiles);
-        const int row = tl.e * n + tl.mt * BM;
+        const int row = tl.e * ldw + tl.mt * BM;
         const int nbox = (tl.N + kBoxRows - 1) / kBoxRows;
         const uint32_t bytes = kABytes + nbox * kBoxRows * BK * 2;
         for (int kb = 0; kb < nk; ++kb, ++it) {
@@ -308,7 +308,7 @@ cudaError_t launch_gather_pairs(const void* x, const int32_t* perm, int T, int d
                     static_cast<const uint4*>(x), perm, k, vec_per_row, N, reinterpret_cast<uint4*>(xp));
 }
 
-cudaError_t launch_tensor_experts(const void* x, const void* Wv, const int32_t* counts,
+cudaError_t launch_tensor_experts(const void* x, const void* Wv, long long ldw, const int32_t* counts,
                                   const int32_t* offsets, const int32_t* perm, const float* w32,
                                   const int32_t* active, StatusBlock* sb, int T, int d, int n, int k,
                                   int E, __nv_bfloat16* xp, __nv_bfloat16* P, cudaStream_t stream) {
@@ -324,7 +324,8 @@ cudaError_t launch_tensor_experts(const void* x, const void* Wv, const int32_t* 
   // 64 columns (128 bytes) with 128-byte swizzle.  The gathered rows: N x d,
   // boxes of 32 rows.
   CUtensorMap tmap_w, tmap_xp;
-  const cuuint64_t gdim[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(E) * n};
+  const cuuint64_t gdim[2] = {static_cast<cuuint64_t>(d),
+                              static_cast<cuuint64_t>(E - 1) * static_cast<cuuint64_t>(ldw) + n};
   const cuuint64_t xdim[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N)};
   const cuuint64_t gstride[1] = {static_cast<cuuint64_t>(d) * 2};
   const cuuint32_t box[2] = {BK, BM};
@@ -343,7 +344,7 @@ cudaError_t launch_tensor_experts(const void* x, const void* Wv, const int32_t* 
                              static_cast<int>(smem));
   if (err != cudaSuccess) return err;
   return launch_pdl(grouped_gemm_kernel, dim3(sm_count()), dim3(kThreads), smem, stream, tmap_w, tmap_xp,
-                    counts, offsets, active, sb, d, n, P);
+                    counts, offsets, active, sb, d, n, static_cast<int>(ldw), P);
 }
 
 }  // namespace mova

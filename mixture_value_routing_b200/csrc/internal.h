@@ -34,9 +34,11 @@ struct GroupOut {
 // Router.  When g (with its logits scratch) is non-null and T <=
 // kFusedRouterMaxT, the decode kernels also write the grouping (and *grouped
 // is set); otherwise the caller runs launch_permute next.
+// partitions: 1 (one fp32 sum per logit, any order) or 2 (the halves j < d/2
+// and j >= d/2 summed separately in fp32, then added first + second).
 cudaError_t launch_router(const void* x, mova_dtype x_dt, const float* Wr, const float* br, int T,
                           int d, int E, int k, float scale, int32_t* idx, float* w,
-                          const GroupOut* g, bool* grouped, cudaStream_t stream);
+                          const GroupOut* g, bool* grouped, int partitions, cudaStream_t stream);
 
 // Decode routing in parts (T <= 8): the partial logits part[s][t][e] over S
 // K ranges (S chosen here, returned in *S_out; at most 4), which also starts
@@ -45,8 +47,8 @@ cudaError_t launch_router(const void* x, mova_dtype x_dt, const float* Wr, const
 // the second part (RouteIn).
 constexpr int kMaxLogitSplits = 4;
 cudaError_t launch_router_logits(const void* x, mova_dtype x_dt, const float* Wr, int T, int d, int E,
-                                 float* part, int* S_out, int32_t* tickets, int ntickets, StatusBlock* sb,
-                                 cudaStream_t stream);
+                                 int partitions, float* part, int* S_out, int32_t* tickets, int ntickets,
+                                 StatusBlock* sb, cudaStream_t stream);
 cudaError_t launch_select_group(const float* part, int S, const float* br, int T, int E, int k, float scale,
                                 int32_t* idx, float* w, const GroupOut* g, cudaStream_t stream);
 
@@ -86,8 +88,9 @@ void* encode_tiled_fn();
 constexpr int kTcRouterMinT = 64;  // bf16 batches above this many tokens use it
 size_t router_planes_bytes(int d);
 cudaError_t launch_router_tc(const void* x, const float* Wr, const float* br, int T, int d, int E,
-                             int k, float scale, int32_t* idx, float* w, int32_t* tile_counts,
-                             __nv_bfloat16* planes, StatusBlock* sb, cudaStream_t stream);
+                             int k, float scale, int partitions, int32_t* idx, float* w,
+                             int32_t* tile_counts, __nv_bfloat16* planes, StatusBlock* sb,
+                             cudaStream_t stream);
 
 // Stable counting sort of the pairs by expert.  idx_in has dtype idx_dt
 // (int32 or int8); when w_in is given (w_dt fp32 or fp16) it is converted to
@@ -109,8 +112,15 @@ cudaError_t launch_tile_hist(const void* idx_in, mova_dtype idx_dt, const void* 
                              int32_t* tile_counts, StatusBlock* sb, cudaStream_t stream);
 cudaError_t launch_tile_group(const int32_t* idx32, int T, int E, int k, int32_t* tile_counts,
                               int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* pos,
-                              int32_t* active, StatusBlock* sb, bool reset_status,
-                              cudaStream_t stream);
+                              int32_t* active, StatusBlock* sb, bool reset_status, int32_t* tickets,
+                              int ntickets, cudaStream_t stream);
+
+// Combine tickets a value call needs (zeroed by its grouping): one per
+// 8-column block, for the weight-streaming kernel's fused combine.
+inline int combine_tickets(int T, int n) {
+  (void)T;
+  return n / 8;
+}
 
 // Weight-streaming expert kernel: P[p, :] = SiLU(Wv[e] x[t]) for every
 // pair p (fp32 rows in grouped order).
@@ -150,7 +160,9 @@ StreamFault take_stream_fault();
 // the combine: the CTA that completes a block of 8 output columns computes v
 // there; the caller then skips launch_combine.  tickets: n / 8 counters,
 // zeroed by the grouping of the same call.
-cudaError_t launch_stream_experts(const void* x, const void* Wv, mova_dtype dt, const int32_t* counts,
+// ldw: rows of Wv between consecutive experts' first rows (>= n).
+cudaError_t launch_stream_experts(const void* x, const void* Wv, long long ldw, mova_dtype dt,
+                                  const int32_t* counts,
                                   const int32_t* offsets, const int32_t* perm, const float* w32,
                                   const int32_t* active, StatusBlock* sb, int T, int d, int n,
                                   int k, int E, float* P, int32_t* tickets, void* v,
@@ -165,7 +177,7 @@ bool stream_resident(int T, int d, mova_dtype dt);
 
 // tcgen05 grouped GEMM (bf16): P[p, :] = SiLU(Wv[e] x[t]) as bf16 rows.
 // xp: T*k x d bf16 scratch for the pairs' x rows in grouped order.
-cudaError_t launch_tensor_experts(const void* x, const void* Wv, const int32_t* counts,
+cudaError_t launch_tensor_experts(const void* x, const void* Wv, long long ldw, const int32_t* counts,
                                   const int32_t* offsets, const int32_t* perm, const float* w32,
                                   const int32_t* active, StatusBlock* sb, int T, int d, int n, int k,
                                   int E, __nv_bfloat16* xp, __nv_bfloat16* P, cudaStream_t stream);
@@ -173,11 +185,12 @@ size_t tensor_experts_smem();
 // xp[p] = x[perm[p] / k] for the T*k pairs.
 cudaError_t launch_gather_pairs(const void* x, const int32_t* perm, int T, int d, int k,
                                 __nv_bfloat16* xp, cudaStream_t stream);
-// The same grouped GEMM on SM pairs (tcgen05 cta_group::2), reading the
-// already gathered rows xp.
-cudaError_t launch_tensor_experts_pair(const void* Wv, const int32_t* counts, const int32_t* offsets,
-                                       const int32_t* active, StatusBlock* sb, int T, int d, int n,
-                                       int k, int E, const __nv_bfloat16* xp, __nv_bfloat16* P,
+// The grouped GEMM on SM pairs (tcgen05 cta_group::2), reading the pairs'
+// token rows already gathered into grouped order (xp, launch_gather_pairs);
+// tiles of up to 512 pairs on two accumulators.
+cudaError_t launch_tensor_experts_pair(const void* Wv, long long ldw, const int32_t* counts,
+                                       const int32_t* offsets, const int32_t* active, StatusBlock* sb, int T,
+                                       int d, int n, int k, int E, const __nv_bfloat16* xp, __nv_bfloat16* P,
                                        cudaStream_t stream);
 
 // v[t, :] = sum over slots (ascending) of w[t*k + slot] * P[pos[t*k + slot], :].

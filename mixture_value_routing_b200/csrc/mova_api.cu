@@ -100,7 +100,7 @@ Workspace layout(void* base, int T, int d, int k, int n) {
   w.active = reinterpret_cast<int32_t*>(b + o);       o += 256;
   w.perm = reinterpret_cast<int32_t*>(b + o);         o += align256(pairs * 4);
   w.pos = reinterpret_cast<int32_t*>(b + o);          o += align256(pairs * 4);
-  w.tickets = reinterpret_cast<int32_t*>(b + o);      o += align256(static_cast<size_t>(n / 8) * 4);
+  w.tickets = reinterpret_cast<int32_t*>(b + o);      o += align256(static_cast<size_t>(combine_tickets(T, n)) * 4);
   w.tile_counts = reinterpret_cast<int32_t*>(b + o);  o += align256(static_cast<size_t>(group_tiles(T)) * 64 * 4);
   w.planes = reinterpret_cast<__nv_bfloat16*>(b + o); o += align256(router_planes_bytes(d));
   // The decode partial logits (T <= 8, kMaxLogitSplits x 8 x 64 floats <= 192 * d * 2 bytes for
@@ -130,6 +130,33 @@ mova_status from_cuda(cudaError_t e) {
 
 bool valid_act_dtype(mova_dtype dt) { return dt == MOVA_F32 || dt == MOVA_BF16; }
 
+// Options with their defaults filled in.
+struct Opts {
+  mova_path path = MOVA_PATH_AUTO;
+  void* const* events = nullptr;
+  long long ldw = 0;   // rows between experts in Wv (n if 0 was given)
+  int partitions = 1;  // router reduction halves (1 or 2)
+};
+
+mova_status read_opts(const mova_options* o, int d, int n, Opts* out) {
+  Opts r;
+  if (o != nullptr) {
+    r.path = o->path;
+    r.events = o->events;
+    r.ldw = o->wv_expert_stride;
+    r.partitions = o->router_partitions == 0 ? 1 : o->router_partitions;
+  }
+  if (r.path != MOVA_PATH_AUTO && r.path != MOVA_PATH_STREAM && r.path != MOVA_PATH_TENSOR &&
+      r.path != MOVA_PATH_TENSOR_1CTA)
+    return MOVA_ERR_INVALID_ARG;
+  if (r.ldw == 0) r.ldw = n;
+  if (r.ldw < n || r.ldw > (1LL << 24)) return MOVA_ERR_INVALID_ARG;
+  if (r.partitions < 0) return MOVA_ERR_INVALID_ARG;
+  if (r.partitions > 2 || (r.partitions == 2 && d % 128 != 0)) return MOVA_ERR_UNSUPPORTED;
+  *out = r;
+  return MOVA_OK;
+}
+
 // Records stage event i (if events were given); external so that it also
 // becomes an event node under stream capture.
 cudaError_t mark(void* const* events, int i, cudaStream_t s) {
@@ -138,7 +165,7 @@ cudaError_t mark(void* const* events, int i, cudaStream_t s) {
 }
 
 // Experts and combine, shared by both value entry points.
-mova_status run_experts_and_combine(const void* x, mova_dtype dt, const void* Wv,
+mova_status run_experts_and_combine(const void* x, mova_dtype dt, const void* Wv, long long ldw,
                                     const Workspace& ws, const int32_t* idx, const float* w32,
                                     int T, int d, int E, int k, int n, void* v, mova_path path,
                                     void* const* events, cudaStream_t stream) {
@@ -146,31 +173,30 @@ mova_status run_experts_and_combine(const void* x, mova_dtype dt, const void* Wv
   if (path == MOVA_PATH_AUTO) path = mova_auto_path(T, dt);
   cudaError_t err = cudaSuccess;
   bool fused_combine = false;
-  if (path != MOVA_PATH_TENSOR || sm_count() < 2) err = mark(events, 2, stream);
-  if (err != cudaSuccess) return from_cuda(err);
   const bool tensor = path == MOVA_PATH_TENSOR || path == MOVA_PATH_TENSOR_1CTA;
+  if (tensor && dt != MOVA_BF16) return MOVA_ERR_UNSUPPORTED;
+  const bool pair = tensor && path == MOVA_PATH_TENSOR && sm_count() >= 2;
+  // The pair GEMM's token rows are gathered first; the gather belongs to the
+  // grouping stage, so the expert stage times the GEMM alone.
+  if (pair) err = launch_gather_pairs(x, ws.perm, T, d, k, ws.xp, stream);
+  if (err == cudaSuccess) err = mark(events, 2, stream);
+  if (err != cudaSuccess) return from_cuda(err);
   if (tensor) {
-    if (dt != MOVA_BF16) return MOVA_ERR_UNSUPPORTED;
-    if (path == MOVA_PATH_TENSOR && sm_count() >= 2) {
-      // The gathered rows are part of the grouping: the stage mark for
-      // "grouped" follows them, so the expert stage times the GEMM alone.
-      err = launch_gather_pairs(x, ws.perm, T, d, k, ws.xp, stream);
-      if (err == cudaSuccess) err = mark(events, 2, stream);
-      if (err == cudaSuccess)
-        err = launch_tensor_experts_pair(Wv, ws.counts, ws.offsets, ws.active, ws.sb, T, d, n, k, E, ws.xp,
-                                         static_cast<__nv_bfloat16*>(ws.P), stream);
-      if (err == cudaSuccess) note_launch();  // the pair GEMM's one launch
+    if (pair) {
+      err = launch_tensor_experts_pair(Wv, ldw, ws.counts, ws.offsets, ws.active, ws.sb, T, d, n, k, E, ws.xp,
+                                       static_cast<__nv_bfloat16*>(ws.P), stream);
     } else {
-      err = launch_tensor_experts(x, Wv, ws.counts, ws.offsets, ws.perm, w32, ws.active, ws.sb, T, d,
-                                  n, k, E, ws.xp, static_cast<__nv_bfloat16*>(ws.P), stream);
+      err = launch_tensor_experts(x, Wv, ldw, ws.counts, ws.offsets, ws.perm, w32, ws.active, ws.sb, T,
+                                  d, n, k, E, ws.xp, static_cast<__nv_bfloat16*>(ws.P), stream);
     }
   } else {
     if (stream_experts_smem(d, dt, T, nullptr) == 0) return MOVA_ERR_UNSUPPORTED;
     // Decode-sized bf16 batches fold the combine into the expert kernel.
     fused_combine = T <= kFusedCombineMaxT && stream_resident(T, d, dt);
-    err = launch_stream_experts(x, Wv, dt, ws.counts, ws.offsets, ws.perm, w32, ws.active, ws.sb, T,
-                                d, n, k, E, static_cast<float*>(ws.P), fused_combine ? ws.tickets : nullptr,
-                                fused_combine ? v : nullptr, RouteIn{}, stream);
+    err = launch_stream_experts(x, Wv, ldw, dt, ws.counts, ws.offsets, ws.perm, w32, ws.active, ws.sb,
+                                T, d, n, k, E, static_cast<float*>(ws.P),
+                                fused_combine ? ws.tickets : nullptr, fused_combine ? v : nullptr,
+                                RouteIn{}, stream);
   }
   if (err == cudaSuccess) err = mark(events, 3, stream);
   if (err == cudaSuccess && !fused_combine)
@@ -224,16 +250,25 @@ mova_path mova_auto_path(int T, mova_dtype x_dt) {
   return (x_dt == MOVA_BF16 && T > kStreamMaxTokens) ? MOVA_PATH_TENSOR : MOVA_PATH_STREAM;
 }
 
-mova_status mova_route(const void* x, mova_dtype x_dt, const float* Wr, const float* br, int T,
-                       int d, int E, int k, float scale, int32_t* idx, float* w, void* stream) {
+mova_status mova_route_opts(const void* x, mova_dtype x_dt, const float* Wr, const float* br, int T,
+                            int d, int E, int k, float scale, int32_t* idx, float* w,
+                            const mova_options* opts, void* stream) {
   mova_status st = check_dims(T, d, E, k, 128);
+  if (st != MOVA_OK) return st;
+  Opts o;
+  st = read_opts(opts, d, 128, &o);
   if (st != MOVA_OK) return st;
   if (!valid_act_dtype(x_dt)) return MOVA_ERR_UNSUPPORTED;
   if (T == 0) return MOVA_OK;
   if (!x || !Wr || !br || !idx || !w) return MOVA_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(Wr)) return MOVA_ERR_INVALID_ARG;
   return from_cuda(launch_router(x, x_dt, Wr, br, T, d, E, k, scale, idx, w, nullptr, nullptr,
-                                 static_cast<cudaStream_t>(stream)));
+                                 o.partitions, static_cast<cudaStream_t>(stream)));
+}
+
+mova_status mova_route(const void* x, mova_dtype x_dt, const float* Wr, const float* br, int T,
+                       int d, int E, int k, float scale, int32_t* idx, float* w, void* stream) {
+  return mova_route_opts(x, x_dt, Wr, br, T, d, E, k, scale, idx, w, nullptr, stream);
 }
 
 mova_status mova_permute(const int32_t* idx, int T, int E, int k, int32_t* counts,
@@ -251,28 +286,33 @@ mova_status mova_permute(const int32_t* idx, int T, int E, int k, int32_t* count
                                        w.tile_counts, w.sb, s);
     if (err == cudaSuccess)
       err = launch_tile_group(idx, T, E, k, w.tile_counts, counts, offsets, perm, pos, w.active, w.sb,
-                              false, s);
+                              false, nullptr, 0, s);
     return from_cuda(err);
   }
   return from_cuda(launch_permute(idx, MOVA_I32, nullptr, MOVA_F32, T * k, E, nullptr, nullptr,
                                   counts, offsets, perm, pos, w.active, w.sb, nullptr, 0, s));
 }
 
-mova_status mova_value_ex(const void* x, mova_dtype x_dt, const void* idx, mova_dtype idx_dt,
-                          const void* wgt, mova_dtype w_dt, const void* Wv, mova_dtype wv_dt, int T,
-                          int d, int E, int k, int n, void* v, void* ws, size_t ws_bytes,
-                          mova_path path, void* const* events, void* stream) {
+mova_status mova_value_opts(const void* x, mova_dtype x_dt, const void* idx, mova_dtype idx_dt,
+                            const void* wgt, mova_dtype w_dt, const void* Wv, mova_dtype wv_dt, int T,
+                            int d, int E, int k, int n, void* v, void* ws, size_t ws_bytes,
+                            const mova_options* opts, void* stream) {
   mova_status st = check_dims(T, d, E, k, n);
   if (st != MOVA_OK) return st;
+  Opts o;
+  st = read_opts(opts, d, n, &o);
+  if (st != MOVA_OK) return st;
+  const mova_path path = o.path;
+  void* const* events = o.events;
   if (!valid_act_dtype(x_dt) || wv_dt != x_dt) return MOVA_ERR_UNSUPPORTED;
+  if ((path == MOVA_PATH_TENSOR || path == MOVA_PATH_TENSOR_1CTA) && x_dt != MOVA_BF16)
+    return MOVA_ERR_UNSUPPORTED;  // the tensor-core kernels take bf16 only
   if (idx_dt != MOVA_I32 && idx_dt != MOVA_I8) return MOVA_ERR_UNSUPPORTED;
   if (w_dt != MOVA_F32 && w_dt != MOVA_F16) return MOVA_ERR_UNSUPPORTED;
-  if (path != MOVA_PATH_AUTO && path != MOVA_PATH_STREAM && path != MOVA_PATH_TENSOR &&
-      path != MOVA_PATH_TENSOR_1CTA)
-    return MOVA_ERR_INVALID_ARG;
   if (T == 0) return MOVA_OK;
   if (!x || !idx || !wgt || !Wv || !v || !ws) return MOVA_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(Wv) || !aligned16(v)) return MOVA_ERR_INVALID_ARG;
+  if ((o.ldw * d * (x_dt == MOVA_BF16 ? 2 : 4)) % 16 != 0) return MOVA_ERR_INVALID_ARG;
   const Workspace w = layout(ws, T, d, k, n);
   if (ws_bytes < w.bytes || (reinterpret_cast<uintptr_t>(ws) & 255) != 0) return MOVA_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -283,14 +323,23 @@ mova_status mova_value_ex(const void* x, mova_dtype x_dt, const void* idx, mova_
       err = launch_tile_hist(idx, idx_dt, wgt, w_dt, T, E, k, w.idx, w.w, w.tile_counts, w.sb, s);
       if (err == cudaSuccess)
         err = launch_tile_group(w.idx, T, E, k, w.tile_counts, w.counts, w.offsets, w.perm, w.pos,
-                                w.active, w.sb, false, s);
+                                w.active, w.sb, false, w.tickets, combine_tickets(T, n), s);
     } else {
       err = launch_permute(idx, idx_dt, wgt, w_dt, T * k, E, w.idx, w.w, w.counts, w.offsets, w.perm,
-                           w.pos, w.active, w.sb, w.tickets, n / 8, s);
+                           w.pos, w.active, w.sb, w.tickets, combine_tickets(T, n), s);
     }
   }
   if (err != cudaSuccess) return from_cuda(err);
-  return run_experts_and_combine(x, x_dt, Wv, w, w.idx, w.w, T, d, E, k, n, v, path, events, s);
+  return run_experts_and_combine(x, x_dt, Wv, o.ldw, w, w.idx, w.w, T, d, E, k, n, v, path, events, s);
+}
+
+mova_status mova_value_ex(const void* x, mova_dtype x_dt, const void* idx, mova_dtype idx_dt,
+                          const void* wgt, mova_dtype w_dt, const void* Wv, mova_dtype wv_dt, int T,
+                          int d, int E, int k, int n, void* v, void* ws, size_t ws_bytes,
+                          mova_path path, void* const* events, void* stream) {
+  const mova_options o{path, events, 0, 0};
+  return mova_value_opts(x, x_dt, idx, idx_dt, wgt, w_dt, Wv, wv_dt, T, d, E, k, n, v, ws, ws_bytes, &o,
+                         stream);
 }
 
 mova_status mova_value(const void* x, mova_dtype x_dt, const void* idx, mova_dtype idx_dt,
@@ -301,27 +350,32 @@ mova_status mova_value(const void* x, mova_dtype x_dt, const void* idx, mova_dty
                        MOVA_PATH_AUTO, nullptr, stream);
 }
 
-mova_status mova_value_routed_ex(const void* x, mova_dtype x_dt, const float* Wr, const float* br,
-                                 const void* Wv, mova_dtype wv_dt, int T, int d, int E, int k,
-                                 int n, float scale, void* v, int32_t* idx_out, float* w_out,
-                                 void* ws, size_t ws_bytes, mova_path path, void* const* events,
-                                 void* stream) {
+mova_status mova_value_routed_opts(const void* x, mova_dtype x_dt, const float* Wr, const float* br,
+                                   const void* Wv, mova_dtype wv_dt, int T, int d, int E, int k,
+                                   int n, float scale, void* v, int32_t* idx_out, float* w_out,
+                                   void* ws, size_t ws_bytes, const mova_options* opts,
+                                   void* stream) {
   mova_status st = check_dims(T, d, E, k, n);
   if (st != MOVA_OK) return st;
+  Opts o;
+  st = read_opts(opts, d, n, &o);
+  if (st != MOVA_OK) return st;
+  const mova_path path = o.path;
+  void* const* events = o.events;
   if (!valid_act_dtype(x_dt) || wv_dt != x_dt) return MOVA_ERR_UNSUPPORTED;
-  if (path != MOVA_PATH_AUTO && path != MOVA_PATH_STREAM && path != MOVA_PATH_TENSOR &&
-      path != MOVA_PATH_TENSOR_1CTA)
-    return MOVA_ERR_INVALID_ARG;
+  if ((path == MOVA_PATH_TENSOR || path == MOVA_PATH_TENSOR_1CTA) && x_dt != MOVA_BF16)
+    return MOVA_ERR_UNSUPPORTED;  // the tensor-core kernels take bf16 only
   if (T == 0) return MOVA_OK;
   if (!x || !Wr || !br || !Wv || !v || !ws) return MOVA_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(Wr) || !aligned16(Wv) || !aligned16(v))
     return MOVA_ERR_INVALID_ARG;
+  if ((o.ldw * d * (x_dt == MOVA_BF16 ? 2 : 4)) % 16 != 0) return MOVA_ERR_INVALID_ARG;
   const Workspace w = layout(ws, T, d, k, n);
   if (ws_bytes < w.bytes || (reinterpret_cast<uintptr_t>(ws) & 255) != 0) return MOVA_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   int32_t* idx = idx_out ? idx_out : w.idx;
   float* wgt = w_out ? w_out : w.w;
-  const GroupOut g{w.counts, w.offsets, w.perm, w.pos, w.active, w.sb, w.tickets, n / 8, w.logits};
+  const GroupOut g{w.counts, w.offsets, w.perm, w.pos, w.active, w.sb, w.tickets, combine_tickets(T, n), w.logits};
   bool grouped = false;
   cudaError_t err = mark(events, 0, s);
   // Decode batches on the weight-streaming path: the router computes the
@@ -331,13 +385,13 @@ mova_status mova_value_routed_ex(const void* x, mova_dtype x_dt, const float* Wr
       stream_experts_smem(d, x_dt, T, nullptr) != 0) {
     int S = 0;
     if (err == cudaSuccess)
-      err = launch_router_logits(x, x_dt, Wr, T, d, E, w.logits, &S, w.tickets, n / 8, w.sb, s);
+      err = launch_router_logits(x, x_dt, Wr, T, d, E, o.partitions, w.logits, &S, w.tickets, combine_tickets(T, n), w.sb, s);
     if (err == cudaSuccess) err = mark(events, 1, s);
     if (err == cudaSuccess) err = mark(events, 2, s);
     const RouteIn ri{w.logits, S, br, E, scale, idx, wgt, w.counts, w.offsets, w.perm, w.pos, w.active};
     if (err == cudaSuccess)
-      err = launch_stream_experts(x, Wv, x_dt, w.counts, w.offsets, w.perm, wgt, w.active, w.sb, T, d, n, k,
-                                  E, static_cast<float*>(w.P), w.tickets, v, ri, s);
+      err = launch_stream_experts(x, Wv, o.ldw, x_dt, w.counts, w.offsets, w.perm, wgt, w.active, w.sb, T, d,
+                                  n, k, E, static_cast<float*>(w.P), w.tickets, v, ri, s);
     if (err == cudaSuccess) err = mark(events, 3, s);
     if (err == cudaSuccess) err = mark(events, 4, s);
     return from_cuda(err);
@@ -347,28 +401,39 @@ mova_status mova_value_routed_ex(const void* x, mova_dtype x_dt, const float* Wr
   const bool tc_router = x_dt == MOVA_BF16 && T > kTcRouterMinT;
   if (err == cudaSuccess) {
     if (tc_router)
-      err = launch_router_tc(x, Wr, br, T, d, E, k, scale, idx, wgt, w.tile_counts, w.planes, w.sb, s);
+      err = launch_router_tc(x, Wr, br, T, d, E, k, scale, o.partitions, idx, wgt, w.tile_counts, w.planes,
+                             w.sb, s);
     else
-      err = launch_router(x, x_dt, Wr, br, T, d, E, k, scale, idx, wgt, &g, &grouped, s);
+      err = launch_router(x, x_dt, Wr, br, T, d, E, k, scale, idx, wgt, &g, &grouped, o.partitions, s);
   }
   if (err == cudaSuccess) err = mark(events, 1, s);
   if (err == cudaSuccess && !grouped) {
     if (tc_router) {
       err = launch_tile_group(idx, T, E, k, w.tile_counts, w.counts, w.offsets, w.perm, w.pos, w.active,
-                              w.sb, true, s);
+                              w.sb, true, w.tickets, combine_tickets(T, n), s);
     } else if (T > kSmallGroupT) {
       err = launch_tile_hist(idx, MOVA_I32, nullptr, MOVA_F32, T, E, k, nullptr, nullptr, w.tile_counts,
                              w.sb, s);
       if (err == cudaSuccess)
         err = launch_tile_group(idx, T, E, k, w.tile_counts, w.counts, w.offsets, w.perm, w.pos,
-                                w.active, w.sb, false, s);
+                                w.active, w.sb, false, w.tickets, combine_tickets(T, n), s);
     } else {
       err = launch_permute(idx, MOVA_I32, nullptr, MOVA_F32, T * k, E, nullptr, nullptr, w.counts,
-                           w.offsets, w.perm, w.pos, w.active, w.sb, w.tickets, n / 8, s);
+                           w.offsets, w.perm, w.pos, w.active, w.sb, w.tickets, combine_tickets(T, n), s);
     }
   }
   if (err != cudaSuccess) return from_cuda(err);
-  return run_experts_and_combine(x, x_dt, Wv, w, idx, wgt, T, d, E, k, n, v, path, events, s);
+  return run_experts_and_combine(x, x_dt, Wv, o.ldw, w, idx, wgt, T, d, E, k, n, v, path, events, s);
+}
+
+mova_status mova_value_routed_ex(const void* x, mova_dtype x_dt, const float* Wr, const float* br,
+                                 const void* Wv, mova_dtype wv_dt, int T, int d, int E, int k,
+                                 int n, float scale, void* v, int32_t* idx_out, float* w_out,
+                                 void* ws, size_t ws_bytes, mova_path path, void* const* events,
+                                 void* stream) {
+  const mova_options o{path, events, 0, 0};
+  return mova_value_routed_opts(x, x_dt, Wr, br, Wv, wv_dt, T, d, E, k, n, scale, v, idx_out, w_out, ws,
+                                ws_bytes, &o, stream);
 }
 
 mova_status mova_value_routed(const void* x, mova_dtype x_dt, const float* Wr, const float* br,

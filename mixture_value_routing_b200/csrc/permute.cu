@@ -198,8 +198,11 @@ __global__ void __launch_bounds__(128)
 tile_scatter_kernel(const int32_t* __restrict__ idx32, int N, int k, int E,
                     const int32_t* __restrict__ tile_counts, int ntiles, int32_t* __restrict__ counts,
                     int32_t* __restrict__ offsets, int32_t* __restrict__ active, StatusBlock* sb,
-                    bool reset_status, int32_t* __restrict__ perm, int32_t* __restrict__ pos) {
+                    bool reset_status, int32_t* __restrict__ perm, int32_t* __restrict__ pos,
+                    int32_t* __restrict__ tickets, int ntickets) {
   pdl_wait();
+  // The combine tickets of this call start at zero.
+  for (int i = blockIdx.x * 128 + threadIdx.x; i < ntickets; i += gridDim.x * 128) tickets[i] = 0;
   __shared__ int hist[4][64];
   __shared__ int base[64];
   __shared__ int tot_s[64];
@@ -347,13 +350,13 @@ cudaError_t launch_tile_hist(const void* idx_in, mova_dtype idx_dt, const void* 
 
 cudaError_t launch_tile_group(const int32_t* idx32, int T, int E, int k, int32_t* tile_counts,
                               int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* pos,
-                              int32_t* active, StatusBlock* sb, bool reset_status,
-                              cudaStream_t stream) {
+                              int32_t* active, StatusBlock* sb, bool reset_status, int32_t* tickets,
+                              int ntickets, cudaStream_t stream) {
   const int N = T * k;
   const int ntiles = group_tiles(T);
   return launch_pdl(tile_scatter_kernel, dim3(ntiles), dim3(128), 0, stream, idx32, N, k, E,
                     static_cast<const int32_t*>(tile_counts), ntiles, counts, offsets, active, sb,
-                    reset_status, perm, pos);
+                    reset_status, perm, pos, tickets, tickets ? ntickets : 0);
 }
 
 }  // namespace mova

@@ -316,13 +316,13 @@ cudaError_t launch_logits_t(const void* x, const float* Wr, int T, int d, int E,
 
 cudaError_t launch_router(const void* x, mova_dtype x_dt, const float* Wr, const float* br, int T,
                           int d, int E, int k, float scale, int32_t* idx, float* w,
-                          const GroupOut* g, bool* grouped, cudaStream_t stream) {
+                          const GroupOut* g, bool* grouped, int partitions, cudaStream_t stream) {
   if (grouped) *grouped = false;
   if (T <= 0) return cudaSuccess;
   if (T <= kFusedRouterMaxT && g != nullptr && g->logits != nullptr) {
     int S = 0;
-    cudaError_t err = launch_router_logits(x, x_dt, Wr, T, d, E, g->logits, &S, g->tickets, g->ntickets,
-                                           g->sb, stream);
+    cudaError_t err = launch_router_logits(x, x_dt, Wr, T, d, E, partitions, g->logits, &S, g->tickets,
+                                           g->ntickets, g->sb, stream);
     if (err != cudaSuccess) return err;
     if (grouped) *grouped = true;
     return launch_select_group(g->logits, S, br, T, E, k, scale, idx, w, g, stream);
@@ -335,6 +335,9 @@ cudaError_t launch_router(const void* x, mova_dtype x_dt, const float* Wr, const
   if (ks > 8) ks = 8;
   if (ks < 1) ks = 1;
   if (ks > d / kRouterKC) ks = d / kRouterKC;
+  // Two router partitions: exactly two ranks, rank 0 summing j < d/2 and
+  // rank 1 the rest; rank 0 adds rank 1's fp32 partial to its own.
+  if (partitions == 2) ks = 2;
   if (x_dt == MOVA_BF16) {
     return small ? launch_router_t<__nv_bfloat16, 8>(x, Wr, br, T, d, E, k, scale, idx, w, ks, stream)
                  : launch_router_t<__nv_bfloat16, 32>(x, Wr, br, T, d, E, k, scale, idx, w, ks, stream);
@@ -350,10 +353,12 @@ int logit_splits(int d, int E) {
 }
 
 cudaError_t launch_router_logits(const void* x, mova_dtype x_dt, const float* Wr, int T, int d, int E,
-                                 float* part, int* S_out, int32_t* tickets, int ntickets, StatusBlock* sb,
-                                 cudaStream_t stream) {
+                                 int partitions, float* part, int* S_out, int32_t* tickets, int ntickets,
+                                 StatusBlock* sb, cudaStream_t stream) {
   if (T <= 0 || T > kDecT) return cudaErrorInvalidValue;
-  const int S = logit_splits(d, E);
+  // Two router partitions: exactly two K ranges, the halves of d; the
+  // selection adds their fp32 partial logits in range order.
+  const int S = partitions == 2 ? 2 : logit_splits(d, E);
   *S_out = S;
   return x_dt == MOVA_BF16 ? launch_logits_t<__nv_bfloat16>(x, Wr, T, d, E, S, part, tickets, ntickets, sb, stream)
                            : launch_logits_t<float>(x, Wr, T, d, E, S, part, tickets, ntickets, sb, stream);

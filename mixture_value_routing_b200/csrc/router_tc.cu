@@ -111,7 +111,7 @@ __global__ void __launch_bounds__(kRThreads, 1)
 router_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
                  const float* __restrict__ br, int T, int d, int E, int k, float scale,
                  int32_t* __restrict__ idx_out, float* __restrict__ w_out,
-                 int32_t* __restrict__ tile_counts, StatusBlock* __restrict__ sb) {
+                 int32_t* __restrict__ tile_counts, StatusBlock* __restrict__ sb, int parts) {
   extern __shared__ uint8_t smem_raw[];
   RSmem& S = *reinterpret_cast<RSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5;
@@ -132,8 +132,11 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_consta
     S.hist[threadIdx.x] = 0;
     S.br[threadIdx.x] = (threadIdx.x < E) ? br[threadIdx.x] : 0.f;
   }
+  // Two router partitions keep a second accumulator (columns 256..447) for
+  // the second half of d.
+  const uint32_t tmem_cols = parts == 2 ? 2 * kRTmemCols : kRTmemCols;
   if (warp == 1) {
-    tmem_alloc(&S.tmem_base, kRTmemCols);
+    tmem_alloc(&S.tmem_base, tmem_cols);
     tmem_relinquish();
   }
   pdl_wait();  // the plane split of this call is complete
@@ -175,6 +178,7 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_consta
     bool ok = true;
     int s = 0;
     uint32_t phase = 0;
+    const int khalf = parts == 2 ? nk / 2 : nk;
     for (int kb = 0; kb < nk; ++kb) {
       if (!__all_sync(0xffffffffu, mbar_wait(&S.full[s], phase))) {
         if (lane == 0) {
@@ -187,10 +191,13 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_consta
       tc_fence_after();
       const uint64_t da = adesc0 + static_cast<uint64_t>(s) * kStageDesc;
       const uint64_t db = bdesc0 + static_cast<uint64_t>(s) * kStageDesc;
+      const bool second = kb >= khalf;
+      const uint32_t d_tmem = S.tmem_base + (second ? kRTmemCols : 0u);
+      const int kl = second ? kb - khalf : kb;  // k-step within its partition
       if (elect_one()) {
 #pragma unroll
         for (int k16 = 0; k16 < RK / 16; ++k16)
-          tc_mma_bf16(S.tmem_base, da + 2 * k16, db + 2 * k16, idesc, (kb | k16) != 0);
+          tc_mma_bf16(d_tmem, da + 2 * k16, db + 2 * k16, idesc, (kl | k16) != 0);
         tc_commit(&S.empty[s]);
       }
       __syncwarp();
@@ -219,6 +226,17 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_consta
 #pragma unroll
         for (int j = 0; j < 32; ++j)
           logit[c * 32 + j] = (__uint_as_float(hi[j]) + __uint_as_float(mid[j])) + __uint_as_float(lo[j]);
+        if (parts == 2) {
+          // Second partition: its own fp32 partial, added after the first.
+          tmem_ld_32(tb + kRTmemCols + c * 32, hi);
+          tmem_ld_32(tb + kRTmemCols + 64 + c * 32, mid);
+          tmem_ld_32(tb + kRTmemCols + 128 + c * 32, lo);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            logit[c * 32 + j] +=
+                (__uint_as_float(hi[j]) + __uint_as_float(mid[j])) + __uint_as_float(lo[j]);
+        }
       }
       tc_fence_before();
       if (t < T) {
@@ -280,7 +298,7 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_consta
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(S.tmem_base, kRTmemCols);
+    tmem_dealloc(S.tmem_base, tmem_cols);
   }
 }
 
@@ -294,8 +312,9 @@ using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, 
 size_t router_planes_bytes(int d) { return static_cast<size_t>(RN) * d * 2; }
 
 cudaError_t launch_router_tc(const void* x, const float* Wr, const float* br, int T, int d, int E,
-                             int k, float scale, int32_t* idx, float* w, int32_t* tile_counts,
-                             __nv_bfloat16* planes, StatusBlock* sb, cudaStream_t stream) {
+                             int k, float scale, int partitions, int32_t* idx, float* w,
+                             int32_t* tile_counts, __nv_bfloat16* planes, StatusBlock* sb,
+                             cudaStream_t stream) {
   void* fp = encode_tiled_fn();
   if (fp == nullptr) return cudaErrorNotSupported;
   EncodeTiled enc = reinterpret_cast<EncodeTiled>(fp);
@@ -323,7 +342,7 @@ cudaError_t launch_router_tc(const void* x, const float* Wr, const float* br, in
   if (err != cudaSuccess) return err;
   const int grid = (T + RM - 1) / RM;
   return launch_pdl(router_tc_kernel, dim3(grid), dim3(kRThreads), smem, stream, tx, tw, br, T, d, E,
-                    k, scale, idx, w, tile_counts, sb);
+                    k, scale, idx, w, tile_counts, sb, partitions == 2 ? 2 : 1);
 }
 
 }  // namespace mova

@@ -36,7 +36,11 @@ namespace mova {
 namespace {
 
 constexpr int kConsumerWarps = 8;
-constexpr int kThreads = (kConsumerWarps + 1) * 32;  // warp 8 produces
+// Warp 8 produces; warp 9 reduces the consumers' partial tiles in resident
+// (decode) mode.
+constexpr int kProducerWarp = kConsumerWarps;
+constexpr int kReducerWarp = kConsumerWarps + 1;
+constexpr int kThreads = (kConsumerWarps + 2) * 32;
 constexpr int kRowsPerStage = kConsumerWarps;
 constexpr int kTok = 8;
 constexpr int kMaxStages = 8;
@@ -95,6 +99,10 @@ __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint3
 
 // Consumer-group barrier (the 8 consumer warps only; the producer warp never
 // joins it).
+// Partial-tile buffers of the consumer warps: one per stage slot (resident
+// mode), at least the two that alternate otherwise.
+__host__ __device__ constexpr int red_slots(int NS) { return NS > 2 ? NS : 2; }
+
 __device__ __forceinline__ void consumers_sync() {
   asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");
 }
@@ -119,7 +127,7 @@ stream_experts_kernel(const DT* __restrict__ x, const DT* __restrict__ Wv,
                       const int32_t* __restrict__ active, StatusBlock* __restrict__ sb, int T,
                       int d, int n, int k, float* __restrict__ P, int NS,
                       int32_t* __restrict__ tickets, DT* __restrict__ v, RouteIn route,
-                      StreamFault fault) {
+                      StreamFault fault, long long ldw) {
   constexpr bool kMma = sizeof(DT) == 2;
   constexpr int EL = Vec<DT>::EL;
   extern __shared__ __align__(128) uint8_t smem[];
@@ -129,8 +137,10 @@ stream_experts_kernel(const DT* __restrict__ x, const DT* __restrict__ Wv,
   const bool resident = is_resident(kMma, T);
   uint8_t* stages = smem;
   uint8_t* xs = smem + NS * stage_bytes;  // bf16: kTok padded x rows
-  float* red = reinterpret_cast<float*>(xs + (kMma ? kTok * pitch : 0));  // [2][warps][8][8]
-  float* tok_w = red + (kMma ? 2 * kConsumerWarps * 64 : 0);  // weights of the staged pairs
+  // Partial tiles of the consumer warps: one [warps][8][8] buffer per stage
+  // slot in resident mode, two alternating ones otherwise.
+  float* red = reinterpret_cast<float*>(xs + (kMma ? kTok * pitch : 0));
+  float* tok_w = red + (kMma ? red_slots(NS) * kConsumerWarps * 64 : 0);  // weights of the staged pairs
   int* tok_p = reinterpret_cast<int*>(tok_w + kTok);           // their grouped positions
   // Resident mode: every token's x row stays in the x tile for the whole
   // kernel (the mma computes all 8 token columns for every expert; each pair
@@ -145,7 +155,9 @@ stream_experts_kernel(const DT* __restrict__ x, const DT* __restrict__ Wv,
   uint64_t* full = reinterpret_cast<uint64_t*>(slot_w + 64);
   uint64_t* empty = full + kMaxStages;
   uint64_t* xbar = empty + kMaxStages;  // resident x rows landed
-  int* act = reinterpret_cast<int*>(xbar + 2);
+  uint64_t* partb = xbar + 2;           // [kMaxStages] resident: a stage's 8 partial tiles are in red
+  float* hred = reinterpret_cast<float*>(partb + kMaxStages);  // [8][8] the reducer's summed tile
+  int* act = reinterpret_cast<int*>(hred + 64);
   volatile int* abort_flag = act + 64;
   int* issued = act + 65;
   int* blk_tick = act + 66;  // [64] completion counts of this CTA's row blocks (fused combine)
@@ -155,7 +167,9 @@ stream_experts_kernel(const DT* __restrict__ x, const DT* __restrict__ Wv,
   if (threadIdx.x == 0) {
     for (int s = 0; s < NS; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], kConsumerWarps);
+      // Resident mode: the reducer frees a stage; otherwise the consumers.
+      mbar_init(&empty[s], resident ? 1 : kConsumerWarps);
+      mbar_init(&partb[s], kConsumerWarps);
     }
     mbar_init(xbar, 1);
     *abort_flag = 0;
@@ -257,7 +271,7 @@ stream_experts_kernel(const DT* __restrict__ x, const DT* __restrict__ Wv,
   const int u1 = static_cast<int>(static_cast<long long>(units) * (blockIdx.x + 1) / gridDim.x);
   const int nstages = u1 - u0;
 
-  if (warp == kConsumerWarps) {
+  if (warp == kProducerWarp) {
     // The producer warp runs the loop together; lane 0 declares each stage's
     // bytes, then lanes 0-7 issue one row copy each, so a stage's eight
     // copies leave at once.  The unit's expert and row advance incrementally.
@@ -280,7 +294,7 @@ stream_experts_kernel(const DT* __restrict__ x, const DT* __restrict__ Wv,
       // Test-only injection: CTA 0 stops issuing here, so the consumers'
       // wait for this stage must run out.
       if (j == fault.stall_stage && blockIdx.x == 0) break;
-      const DT* src = Wv + (static_cast<size_t>(act[a]) * n + rb * kRowsPerStage) * d;
+      const DT* src = Wv + (static_cast<size_t>(act[a]) * ldw + rb * kRowsPerStage) * d;
       uint8_t* dst = stages + s * stage_bytes;
       if (lane == 0) mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(kRowsPerStage * row_bytes));
       __syncwarp();
@@ -296,6 +310,60 @@ stream_experts_kernel(const DT* __restrict__ x, const DT* __restrict__ Wv,
       if (++s == NS) { s = 0; phase ^= 1; }
     }
     if (lane == 0) *issued = j;
+  } else if (warp == kReducerWarp) {
+    if (resident) {
+      // Resident mode: the consumer warps hand each stage's partial tiles
+      // (their K slices of 8 weight rows x 8 token columns) over through an
+      // mbarrier instead of meeting at a block barrier; this warp sums them
+      // in warp order, applies SiLU, stores the rows of every pair of the
+      // stage's expert, and frees the stage.  It takes every stage, even
+      // after a failure (then storing nothing), so the stage ring stays in
+      // step.
+      int cur_a = -1, cnt = 0, off = 0;
+      for (int j = 0; j < nstages; ++j) {
+        const int s = j % NS;
+        bool ok = *abort_flag == 0;
+        if (ok && !mbar_wait_or_abort(&partb[s], (j / NS) & 1, abort_flag, fault.wait_limit)) {
+          ok = false;
+          if (*abort_flag == 0) {
+            raise_status(sb, MOVA_ERR_TIMEOUT, blockIdx.x);
+            *abort_flag = 1;
+          }
+        }
+        ok = __all_sync(0xffffffffu, ok);
+        const int u = u0 + j;
+        const int a = fused ? u % nact : u / units_per_expert;
+        const int r0 = (fused ? u / nact : u - a * units_per_expert) * kRowsPerStage;
+        if (a != cur_a) {
+          cur_a = a;
+          cnt = act_cnt[a];
+          off = act_off[a];
+        }
+        if (ok) {
+          const float* rb = red + s * (kConsumerWarps * 64);
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int e = lane + 32 * h;  // row e / 8, token column e % 8
+            float acc = 0.f;
+#pragma unroll
+            for (int w = 0; w < kConsumerWarps; ++w) acc += rb[w * 64 + e];
+            hred[e] = siluf_(acc);
+          }
+          __syncwarp();
+          for (int e = lane; e < cnt * kRowsPerStage; e += 32) {
+            const int p = off + e / kRowsPerStage;
+            const int row = e % kRowsPerStage;
+            P[static_cast<size_t>(p) * n + r0 + row] = hred[row * 8 + pair_tok[p]];
+          }
+          __syncwarp();
+        }
+        if (lane == 0) mbar_arrive(&empty[s]);
+      }
+      // This warp's rows of P are complete: the consumers' fused combine
+      // reads them after the barrier below.
+      __threadfence();
+      asm volatile("bar.sync 2, %0;" ::"n"((kConsumerWarps + 1) * 32) : "memory");
+    }
   } else {
     int cur_a = -1, cnt = 0, off = 0;
     int staged_a = -1, staged_c0 = -1;  // whose x rows the x tile holds
@@ -349,6 +417,52 @@ stream_experts_kernel(const DT* __restrict__ x, const DT* __restrict__ Wv,
         off = resident ? act_off[a] : offsets[act[a]];
       }
       const uint8_t* wst = stages + s * stage_bytes;
+      if constexpr (kMma) {
+        if (resident) {
+          // The stage's (8 weight rows) x (8 token columns) tile over this
+          // warp's K slice, with four independent accumulators fed by four
+          // k-steps of loads at a time (summed in a fixed order at the end),
+          // handed to the reducer warp.
+          float acc[4] = {0.f, 0.f, 0.f, 0.f};
+          if (ok) {
+            const int lr = lane & 7;
+            const int lk = (lane >> 3) & 1;
+            const uint32_t a_base = smem_u32(wst) + lr * static_cast<uint32_t>(pitch) + lk * 16;
+            const uint32_t b_base = smem_u32(xs) + lr * static_cast<uint32_t>(pitch) + lk * 16;
+            float c1[4] = {0.f, 0.f, 0.f, 0.f}, c2[4] = {0.f, 0.f, 0.f, 0.f}, c3[4] = {0.f, 0.f, 0.f, 0.f};
+            int ks = kb;
+            for (; ks + 3 < ke; ks += 4) {
+              uint32_t a0[4], a2[4], b0[4], b1[4];
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                ldsm_x2(a_base + (ks + q) * 32, a0[q], a2[q]);
+                ldsm_x2(b_base + (ks + q) * 32, b0[q], b1[q]);
+              }
+              mma_bf16_16816(acc, a0[0], a2[0], b0[0], b1[0]);
+              mma_bf16_16816(c1, a0[1], a2[1], b0[1], b1[1]);
+              mma_bf16_16816(c2, a0[2], a2[2], b0[2], b1[2]);
+              mma_bf16_16816(c3, a0[3], a2[3], b0[3], b1[3]);
+            }
+            for (; ks < ke; ++ks) {
+              uint32_t a0, a2, b0, b1;
+              ldsm_x2(a_base + ks * 32, a0, a2);
+              ldsm_x2(b_base + ks * 32, b0, b1);
+              mma_bf16_16816(acc, a0, a2, b0, b1);
+            }
+#pragma unroll
+            for (int q = 0; q < 4; ++q) acc[q] = (acc[q] + c1[q]) + (c2[q] + c3[q]);
+          }
+          // acc[0], acc[1]: weight row lane / 4, token columns 2 * (lane % 4) + {0, 1}.
+          float* rb = red + s * (kConsumerWarps * 64);
+          const int g = lane >> 2;
+          const int tc = (lane & 3) * 2;
+          rb[warp * 64 + g * 8 + tc] = acc[0];
+          rb[warp * 64 + g * 8 + tc + 1] = acc[1];
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&partb[s]);
+          continue;  // the reducer frees the stage
+        }
+      }
       for (int c0 = 0; c0 < cnt; c0 += kTok) {
         const int nt = min(kTok, cnt - c0);
         if constexpr (kMma) {
@@ -457,6 +571,8 @@ stream_experts_kernel(const DT* __restrict__ x, const DT* __restrict__ Wv,
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[s]);
     }
+    // Resident mode: wait until the reducer has stored this CTA's rows of P.
+    if (resident) asm volatile("bar.sync 2, %0;" ::"n"((kConsumerWarps + 1) * 32) : "memory");
     // The consumer warps agree (one bar.red) on whether any role failed: if
     // so, nothing is combined; otherwise every warp takes the same path.
     if (fused && nstages > 0 && !consumers_any(*abort_flag != 0)) {
@@ -499,7 +615,7 @@ stream_experts_kernel(const DT* __restrict__ x, const DT* __restrict__ Wv,
   __syncthreads();
   // No bulk copy may still be writing this CTA's shared memory at exit: wait
   // (bounded) for the last phase issued into every stage.
-  if (threadIdx.x == kConsumerWarps * 32) {
+  if (threadIdx.x == kProducerWarp * 32) {
     const int done = *issued;
     for (int j = max(0, done - NS); j < done; ++j) mbar_wait(&full[j % NS], (j / NS) & 1);
     if (resident) mbar_wait(xbar, 0);
@@ -513,15 +629,20 @@ size_t stream_experts_smem(int d, mova_dtype dt, int T, int* stages_out) {
   (void)T;
   const size_t pitch = static_cast<size_t>(d) * (mma ? 2 : 4) + 16;
   const size_t stage_bytes = pitch * kRowsPerStage;
-  const size_t fixed = (mma ? kTok * pitch + 2 * kConsumerWarps * 64 * sizeof(float) : 0) +
-                       2 * kTok * sizeof(float) + 6 * 64 * sizeof(int) +
-                       (2 * kMaxStages + 2) * sizeof(uint64_t) + 130 * sizeof(int);
   const size_t budget = 220 * 1024;
-  int NS = fixed < budget ? static_cast<int>((budget - fixed) / stage_bytes) : 0;
-  if (NS > kStreamStages) NS = kStreamStages;
-  if (stages_out) *stages_out = NS;
-  if (NS < 2) return 0;
-  return NS * stage_bytes + fixed;
+  // The most stages (up to kStreamStages) that fit next to the fixed parts,
+  // whose partial-tile buffers grow with the stage count.
+  for (int NS = kStreamStages; NS >= 2; --NS) {
+    const size_t fixed = (mma ? kTok * pitch + red_slots(NS) * kConsumerWarps * 64 * sizeof(float) : 0) +
+                         2 * kTok * sizeof(float) + 6 * 64 * sizeof(int) +
+                         (3 * kMaxStages + 2) * sizeof(uint64_t) + 64 * sizeof(float) + 130 * sizeof(int);
+    if (NS * stage_bytes + fixed <= budget) {
+      if (stages_out) *stages_out = NS;
+      return NS * stage_bytes + fixed;
+    }
+  }
+  if (stages_out) *stages_out = 0;
+  return 0;
 }
 
 bool stream_resident(int T, int d, mova_dtype dt) {
@@ -529,7 +650,8 @@ bool stream_resident(int T, int d, mova_dtype dt) {
   return is_resident(dt == MOVA_BF16, T);
 }
 
-cudaError_t launch_stream_experts(const void* x, const void* Wv, mova_dtype dt, const int32_t* counts,
+cudaError_t launch_stream_experts(const void* x, const void* Wv, long long ldw, mova_dtype dt,
+                                  const int32_t* counts,
                                   const int32_t* offsets, const int32_t* perm, const float* w32,
                                   const int32_t* active, StatusBlock* sb, int T, int d, int n,
                                   int k, int E, float* P, int32_t* tickets, void* v,
@@ -548,7 +670,7 @@ cudaError_t launch_stream_experts(const void* x, const void* Wv, mova_dtype dt, 
     return launch_pdl(kern, grid, dim3(kThreads), smem, stream,
                       static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(Wv),
                       counts, offsets, perm, w32, active, sb, T, d, n, k, P, NS, tickets,
-                      static_cast<__nv_bfloat16*>(v), route, fault);
+                      static_cast<__nv_bfloat16*>(v), route, fault, ldw);
   }
   auto kern = stream_experts_kernel<float>;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -556,7 +678,7 @@ cudaError_t launch_stream_experts(const void* x, const void* Wv, mova_dtype dt, 
   if (err != cudaSuccess) return err;
   return launch_pdl(kern, grid, dim3(kThreads), smem, stream, static_cast<const float*>(x),
                     static_cast<const float*>(Wv), counts, offsets, perm, w32, active, sb, T, d, n,
-                    k, P, NS, tickets, static_cast<float*>(v), route, fault);
+                    k, P, NS, tickets, static_cast<float*>(v), route, fault, ldw);
 }
 
 }  // namespace mova

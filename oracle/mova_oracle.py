@@ -67,6 +67,28 @@ def router_logits(x: np.ndarray, Wr: np.ndarray) -> np.ndarray:
     return x @ Wr.T
 
 
+def router_logits_partitioned(x: np.ndarray, Wr: np.ndarray, partitions: int) -> np.ndarray:
+    """Router logits with the reduction over d split into `partitions`
+    equal consecutive ranges, as a router GEMM partitioned along K computes
+    them: each range's dot product is formed (exactly, in fp64) and rounded
+    once to fp32, and the fp32 partial sums are added in range order with
+    fp32 rounding.  "Mixture of Value Attention" (robotsatlas.com),
+    "Implementation pitfalls", names keeping the router's numerics through
+    its GEMM partitioning; the serving recipe of "IFM/K2-Horizon-MoVA-36B-A4B"
+    (paperfeed.app) sets two partitions.  The reading -- halves of d, each
+    rounded to fp32, then added first + second -- is this oracle's.
+    x: (T, d) fp64, Wr: (E, d) fp64, d divisible by `partitions`
+    -> (T, E) fp64 holding fp32 values."""
+    d = x.shape[1]
+    assert d % partitions == 0
+    step = d // partitions
+    acc = None
+    for p in range(partitions):
+        part = (x[:, p * step:(p + 1) * step] @ Wr[:, p * step:(p + 1) * step].T).astype(np.float32)
+        acc = part if acc is None else (acc + part).astype(np.float32)
+    return acc.astype(np.float64)
+
+
 def sigmoid(z: np.ndarray) -> np.ndarray:
     """Logistic function 1 / (1 + exp(-z)), in fp64."""
     return 1.0 / (1.0 + np.exp(-z))
@@ -81,14 +103,16 @@ def select_top_k(b: np.ndarray, k: int) -> np.ndarray:
     return order[:, :k]
 
 
-def route(x: np.ndarray, Wr: np.ndarray, br: np.ndarray, k: int, scale: float):
+def route(x: np.ndarray, Wr: np.ndarray, br: np.ndarray, k: int, scale: float,
+          partitions: int = 1):
     """Sigmoid gate, bias-assisted top-k, renormalise, scale.
 
     s = sigmoid(logits); b = s + br (selection only); idx = top-k of b;
     w[t, slot] = scale * s[t, idx] / sum over the k slots of s[t, idx].
+    partitions > 1 takes the logits of router_logits_partitioned.
     Returns dict(idx (T,k) int64, w (T,k), s (T,E), b (T,E), logits (T,E)).
     """
-    logits = router_logits(x, Wr)
+    logits = router_logits(x, Wr) if partitions == 1 else router_logits_partitioned(x, Wr, partitions)
     s = sigmoid(logits)
     b = s + br[None, :]
     idx = select_top_k(b, k)

@@ -398,3 +398,138 @@ def test_decode_step_kernel_count(api):
         api.value_routed(*args)
         assert api.launch_count() - before == want, dtype
     torch.cuda.synchronize()
+
+
+# ---------------------------------------------------------------------------
+# Router partitions (mova_options.router_partitions = 2)
+# ---------------------------------------------------------------------------
+
+def _cancel_inputs(T, d, E, dtype):
+    """Every token: expert 0's first half of d sums to 2^25 and its second
+    half to -2^25 + 1, which fp32 rounds to -2^25 (a tie, to even): the
+    partitioned logit is 0, the exact one 1.  Other experts' logits are 0."""
+    x = np.zeros((T, d), np.float32)
+    Wr = np.zeros((E, d), np.float32)
+    h = d // 2
+    x[:, 0] = x[:, h] = 2.0 ** 12
+    x[:, h + 1] = 1.0
+    Wr[0, 0], Wr[0, h], Wr[0, h + 1] = 2.0 ** 13, -2.0 ** 13, 1.0
+    br = np.full(E, -1.0, np.float32)
+    br[0], br[1] = 0.0, 0.1
+    xs = MI.f32_to_bf16_bits(x) if dtype == "bf16" else x
+    return xs, Wr, br
+
+
+@pytest.mark.parametrize("T,dtype", [(1, "bf16"), (8, "bf16"), (8, "f32"), (16, "f32"), (40, "bf16")])
+def test_route_partitions_cancellation(api, T, dtype):
+    """The fp32 CUDA-core routers in two-partition mode (the tiled router of
+    mova_route, and for decode batches of the full path the logits kernel)
+    take the selection the partitioned oracle takes, which differs from the
+    exact one.  (The tensor-core router is checked on random inputs below:
+    how its accumulator rounds a 16-product block sum is not specified, so
+    this exact tie is not asked of it.)"""
+    d, E, k = 128, 8, 2
+    xs, Wr, br = _cancel_inputs(T, d, E, dtype)
+    x64 = O.to_f64(xs, dtype)
+    ref = O.route(x64, Wr.astype(np.float64), br.astype(np.float64), k, 2.5, partitions=2)
+    exact = O.route(x64, Wr.astype(np.float64), br.astype(np.float64), k, 2.5)
+    assert (ref["idx"] == [1, 0]).all() and (exact["idx"] == [0, 1]).all()
+    idx, w = api.route(P.dev(xs, dtype), P.dev(Wr, "f32"), P.dev(br, "f32"), k, 2.5, partitions=2)
+    torch.cuda.synchronize()
+    assert (idx.cpu().numpy() == ref["idx"]).all()
+    np.testing.assert_allclose(w.cpu().numpy(), 1.25, rtol=1e-6)
+    if dtype == "bf16" and T <= 8:
+        # The decode batches of the full path route in the logits kernel.
+        Wv = _layer(3, d, E, 128, "bf16").Wv
+        _, idx2, w2 = api.value_routed(P.dev(xs, dtype), P.dev(Wr, "f32"), P.dev(br, "f32"),
+                                       P.dev(Wv, "bf16"), k, 2.5, return_routing=True, partitions=2)
+        torch.cuda.synchronize()
+        assert (idx2.cpu().numpy() == ref["idx"]).all()
+        np.testing.assert_allclose(w2.cpu().numpy(), 1.25, rtol=1e-6)
+
+
+@pytest.mark.parametrize("T,d,dtype", [(8, 2560, "bf16"), (33, 2560, "bf16"), (130, 2560, "bf16"),
+                                       (4096, 2560, "bf16"), (128, 2560, "f32")])
+def test_route_partitions_random(api, T, d, dtype):
+    """Two-partition routing on random inputs, every router kernel (decode
+    logits, tiled SIMT, tensor-core with two accumulators), against the
+    partitioned oracle under the near-tie rule."""
+    E, k = 64, 4
+    lay = _layer(13, d, E, 128, dtype)
+    bat = MI.make_batch(T, 13, dtype=dtype, d=d)
+    x = O.to_f64(bat.x, dtype)
+    ref = O.route(x, lay.Wr.astype(np.float64), lay.br.astype(np.float64), k, 2.5, partitions=2)
+    idx, w = api.route(P.dev(bat.x, dtype), P.dev(lay.Wr, "f32"), P.dev(lay.br, "f32"), k, 2.5,
+                       partitions=2)
+    torch.cuda.synchronize()
+    P.check_routing(idx.cpu().numpy(), w.cpu().numpy().astype(np.float64), ref, k, 2.5)
+
+
+@pytest.mark.parametrize("T", [8, 300])
+def test_value_routed_partitions(api, T):
+    """The whole path in two-partition mode: routing as the partitioned
+    oracle's, values of the GPU's selection."""
+    d, E, k, n = 2560, 64, 4, 1024
+    lay = _layer(17, d, E, n, "bf16")
+    bat = MI.make_batch(T, 17, dtype="bf16", d=d)
+    x = O.to_f64(bat.x, "bf16")
+    ref = O.route(x, lay.Wr.astype(np.float64), lay.br.astype(np.float64), k, 2.5, partitions=2)
+    v, idx, w = api.value_routed(P.dev(bat.x, "bf16"), P.dev(lay.Wr, "f32"), P.dev(lay.br, "f32"),
+                                 P.dev(lay.Wv, "bf16"), k, 2.5, return_routing=True, partitions=2)
+    torch.cuda.synchronize()
+    idx_g = idx.cpu().numpy().astype(np.int64)
+    P.check_routing(idx_g, w.cpu().numpy().astype(np.float64), ref, k, 2.5)
+    rows = np.arange(min(T, 128))
+    v_ref = O.combine(x[rows], idx_g[rows], O.weights_for(ref["s"][rows], idx_g[rows], 2.5), lay.Wv, "bf16")
+    P.check_values(P.host_f64(v)[rows], v_ref, "bf16")
+
+
+def test_partitions_unsupported_width(api):
+    from mixture_value_routing_b200 import _lib
+    x = torch.zeros((4, 192), dtype=torch.bfloat16, device="cuda")  # 192 % 128 != 0
+    with pytest.raises(_lib.MovaError) as e:
+        api.route(x, torch.zeros((8, 192), device="cuda"), torch.zeros(8, device="cuda"), 2, 2.5,
+                  partitions=2)
+    assert e.value.code == _lib.ERR_UNSUPPORTED
+
+
+# ---------------------------------------------------------------------------
+# Head-parallel slices (mova_options.wv_expert_stride)
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("T,path", [(8, "auto"), (24, "auto"), (300, "auto"), (300, "tensor_1cta"),
+                                    (4096, "auto")])
+def test_head_parallel_slices(api, T, path):
+    """Two ranks' halves of the 8 value heads (rows 0..511 and 512..1023 of
+    every expert, read in place from the full Wv): each equals the oracle's
+    columns and, concatenated, the full call bit for bit (the same dot
+    products in the same order)."""
+    d, E, k, n = 2560, 64, 4, 1024
+    lay = _layer(23, d, E, n, "bf16")
+    bat = MI.make_batch(T, 23, dtype="bf16", d=d)
+    args = (P.dev(bat.x, "bf16"), P.dev(lay.Wr, "f32"), P.dev(lay.br, "f32"), P.dev(lay.Wv, "bf16"))
+    full, idx, _ = api.value_routed(*args, return_routing=True, path=path)
+    halves = [api.value_routed(*args, path=path, rows=(r * 512, 512)) for r in range(2)]
+    torch.cuda.synchronize()
+    for h in halves:
+        assert h.shape == (T, 512)
+    assert torch.equal(torch.cat(halves, dim=1), full)
+    x, ref = _routing_ref(bat, lay, k)
+    idx_g = idx.cpu().numpy().astype(np.int64)
+    rows = np.arange(min(T, 256))
+    v_ref = O.combine(x[rows], idx_g[rows], O.weights_for(ref["s"][rows], idx_g[rows], 2.5), lay.Wv, "bf16")
+    for r, h in enumerate(halves):
+        P.check_values(P.host_f64(h)[rows], v_ref[:, r * 512:(r + 1) * 512], "bf16")
+
+
+def test_head_parallel_given(api):
+    """Routing-given recompute of one head slice (rows 256..639, three heads)."""
+    d, E, k, n, T = 512, 8, 4, 1024, 333
+    lay = _layer(9, d, E, n, "bf16")
+    bat = MI.make_batch(T, 9, dtype="bf16", d=d, mode="given", E=E, k=k)
+    v = api.value(P.dev(bat.x, "bf16"), P.dev(bat.idx, "i8"), P.dev(bat.w, "f16"), P.dev(lay.Wv, "bf16"),
+                  rows=(256, 384))
+    torch.cuda.synchronize()
+    v_ref = O.combine(O.to_f64(bat.x, "bf16"), bat.idx.astype(np.int64), bat.w.astype(np.float64),
+                      lay.Wv, "bf16")
+    P.check_values(P.host_f64(v), v_ref[:, 256:640], "bf16")

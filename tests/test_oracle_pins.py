@@ -311,3 +311,68 @@ def test_permutation_empty():
     assert p["counts"].tolist() == [0] * 8
     assert p["offsets"].tolist() == [0] * 9
     assert p["perm"].size == 0 and p["pos"].size == 0
+
+
+# ---------------------------------------------------------------------------
+# Router partitions ("Implementation pitfalls": router numerics through the
+# GEMM partitioning)
+# ---------------------------------------------------------------------------
+
+
+def _cancel_case(layout):
+    """Expert 0's partial sums cancel; the rest have zero logits.  Returns
+    (x (1, 8), Wr (3, 8), br (3,)) in fp64; values exactly representable."""
+    x = np.zeros((1, 8))
+    Wr = np.zeros((3, 8))
+    for j, xv, wv in layout:
+        x[0, j] = xv
+        Wr[0, j] = wv
+    br = np.array([0.0, 0.1, -1.0])
+    return x, Wr, br
+
+
+def test_partitioned_logits_round_each_half():
+    """2^25 lands in the first half and -2^25 + 1 in the second: the second
+    half's fp32 sum rounds -(2^25 - 1) to -2^25 (a tie, to even), so the
+    partitioned logit is 0 while the exact one is 1 -- and the selection
+    follows (expert 1's biased score 0.6 beats sigmoid(0) = 0.5 but not
+    sigmoid(1) = 0.731)."""
+    x, Wr, br = _cancel_case([(0, 2.0 ** 12, 2.0 ** 13), (4, 2.0 ** 12, -2.0 ** 13), (5, 1.0, 1.0)])
+    assert O.router_logits(x, Wr)[0].tolist() == [1.0, 0.0, 0.0]
+    assert O.router_logits_partitioned(x, Wr, 2)[0].tolist() == [0.0, 0.0, 0.0]
+    plain = O.route(x, Wr, br, 2, 2.5)
+    part = O.route(x, Wr, br, 2, 2.5, partitions=2)
+    assert plain["idx"].tolist() == [[0, 1]]
+    assert part["idx"].tolist() == [[1, 0]]
+    np.testing.assert_allclose(part["w"], [[1.25, 1.25]], rtol=0, atol=1e-15)
+    s1 = 1.0 / (1.0 + math.exp(-1.0))
+    np.testing.assert_allclose(plain["w"], [[2.5 * s1 / (s1 + 0.5), 2.5 * 0.5 / (s1 + 0.5)]], rtol=1e-15)
+
+
+def test_partitioned_logits_split_at_the_middle():
+    """2^25 and -2^25 both in the first half, +1 in its last place: the first
+    half sums exactly to 1, so the partitioned logit is 1; a split after two
+    elements would round 1 - 2^25 to -2^25 and give 0."""
+    x, Wr, br = _cancel_case([(0, 2.0 ** 12, 2.0 ** 13), (2, 2.0 ** 12, -2.0 ** 13), (3, 1.0, 1.0)])
+    assert O.router_logits_partitioned(x, Wr, 2)[0].tolist() == [1.0, 0.0, 0.0]
+    quarters = (np.float32(x[0, :2] @ Wr[0, :2]) + np.float32(x[0, 2:4] @ Wr[0, 2:4]))
+    assert float(quarters) == 0.0  # the wrong split point gives another answer
+
+
+def test_partitioned_logits_are_fp32_within_rounding():
+    """On random inputs the partitioned logits are fp32 numbers within the
+    three roundings of the exact logits (each half, then their sum)."""
+    rng = np.random.default_rng(5)
+    x = rng.standard_normal((16, 256)).astype(np.float32).astype(np.float64)
+    Wr = (rng.standard_normal((8, 256)) * 0.02).astype(np.float32).astype(np.float64)
+    exact = O.router_logits(x, Wr)
+    part = O.router_logits_partitioned(x, Wr, 2)
+    assert (part.astype(np.float32).astype(np.float64) == part).all()
+    h0 = np.abs(x[:, :128] @ Wr[:, :128].T)
+    h1 = np.abs(x[:, 128:] @ Wr[:, 128:].T)
+    eps = 2.0 ** -24
+    bound = eps * (h0 + h1) + eps * np.abs(part) + 1e-300
+    assert (np.abs(part - exact) <= bound * 1.0000001).all()
+    assert not (part == exact).all()  # the rounding is really there
+    np.testing.assert_array_equal(O.route(x, Wr, np.zeros(8), 2, 2.5)["logits"], exact)
+    np.testing.assert_array_equal(O.route(x, Wr, np.zeros(8), 2, 2.5, partitions=2)["logits"], part)
