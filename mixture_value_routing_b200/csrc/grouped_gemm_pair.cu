@@ -27,11 +27,13 @@
 //     (M = 256, N = 16..256, K = 16) into accumulator 0 (pairs 0..255 of the
 //     tile) and accumulator 1 (pairs 256..511); tcgen05.commit multicast
 //     frees the stage in both CTAs.
-//   * Eight epilogue warps: four per accumulator, one per tensor-memory lane
-//     quarter.  Each reads its accumulator's columns into registers (SiLU,
-//     bf16) in two halves, storing the first half before reading the second,
-//     and hands the accumulator back right after its last read, so the next
-//     tile's MMAs wait for the reads and one half's stores only.
+//   * Tensor memory holds two 256-column accumulator regions.  A tile of at
+//     most 256 pairs uses one, alternating, so its epilogue overlaps the next
+//     tile's MMAs; a larger tile uses both.  Eight epilogue warps: four per
+//     region, one per tensor-memory lane quarter.  Each reads the region's
+//     columns into registers (SiLU, bf16) in two halves, storing the first
+//     half before reading the second, and hands the region back right after
+//     its last read.
 //   * One persistent pair per two SMs takes tiles from a global counter;
 //     tiles are numbered largest expert first (then token tile, then the
 //     four weight-row blocks of a token tile next to each other, so pairs
@@ -67,8 +69,8 @@ struct __align__(1024) PSmem {
   uint8_t stage[kPStages][kPStageBytes];
   uint64_t full[kPStages];      // even CTA: both CTAs' copies of the stage landed
   uint64_t empty[kPStages];     // both CTAs: the pair's MMAs on the stage are done
-  uint64_t tmem_full;           // both CTAs: the tile's accumulators are complete
-  uint64_t acc_empty[2];        // even CTA: accumulator a read by 4 warps x 2 CTAs
+  uint64_t reg_full[2];         // both CTAs: tensor-memory region r holds a finished accumulator
+  uint64_t reg_empty[2];        // even CTA: region r read out by its 4 epilogue warps x 2 CTAs
   uint64_t tq_full[kTileRing];  // both CTAs: tile id i of this cluster published
   int tq[kTileRing];
   uint32_t tmem_base;
@@ -109,6 +111,32 @@ __device__ __forceinline__ PTile decode_ptile(const PSmem& S, int t, int mtiles)
   return r;
 }
 
+// Tensor memory holds two accumulator regions of 256 columns.  A tile of at
+// most 256 pairs takes one region, alternating between the two, so its
+// epilogue overlaps the next tile's MMAs; a larger tile takes both (pairs
+// 0..255 in the next region, the rest in the other).  Every role walks the
+// cluster's tile sequence and applies this rule, so they agree on which
+// region holds what, and on each region's use count (its barrier parity).
+struct Regions {
+  int next = 0;
+  int uses0 = 0, uses1 = 0;
+  __device__ __forceinline__ int uses(int r) const { return r == 0 ? uses0 : uses1; }
+  __device__ __forceinline__ void used(int r) {
+    if (r == 0) ++uses0; else ++uses1;
+  }
+  // Regions of a tile: r0 for its first accumulator, r1 for its second (-1
+  // if none).
+  __device__ __forceinline__ void take(const PTile& tl, int& r0, int& r1) {
+    r0 = next;
+    if (tl.N1 > 0) {
+      r1 = next ^ 1;
+    } else {
+      r1 = -1;
+      next ^= 1;
+    }
+  }
+};
+
 // The cluster's i-th tile id (waits until the even CTA's producer has
 // published it; ntiles or more means no more tiles).  -1 if the wait ran out.
 __device__ __forceinline__ int next_tile(PSmem& S, int i) {
@@ -146,8 +174,10 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_w, const __gri
       mbar_init(&S.full[s], 1);
       mbar_init(&S.empty[s], 1);
     }
-    mbar_init(&S.tmem_full, 1);
-    for (int i = 0; i < 2; ++i) mbar_init(&S.acc_empty[i], 4 * 2);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&S.reg_full[i], 1);
+      mbar_init(&S.reg_empty[i], 4 * 2);
+    }
     for (int i = 0; i < kTileRing; ++i) mbar_init(&S.tq_full[i], 1);
     S.abort = 0;
     fence_barrier_init();
@@ -297,6 +327,7 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_w, const __gri
       constexpr uint32_t kStageDesc = kPStageBytes >> 4;
       int s = 0;
       uint32_t phase = 0;
+      Regions reg;
       for (int titer = 0;; ++titer) {
         const int t = next_tile(S, titer);
         if (t < 0) {
@@ -305,17 +336,23 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_w, const __gri
         }
         if (t >= ntiles || p_aborted(S)) break;
         const PTile tl = decode_ptile(S, t, mtiles);
+        int r0, r1;
+        reg.take(tl, r0, r1);
+        const uint32_t d0 = S.tmem_base + static_cast<uint32_t>(r0 * NA);
+        const uint32_t d1 = S.tmem_base + static_cast<uint32_t>((r1 < 0 ? 0 : r1) * NA);
         const uint32_t idesc0 = idesc_bf16_f32(2 * PM, tl.N0);
         const uint32_t idesc1 = idesc_bf16_f32(2 * PM, tl.N1 > 0 ? tl.N1 : 16);
         // Accumulator 1's B rows start kAcc1Rows rows into each CTA's B area.
         const uint64_t b1off = static_cast<uint64_t>(kAcc1Rows * PK * 2) >> 4;
         bool ok = true;
         for (int kb = 0; kb < nk; ++kb) {
-          if (kb == 0 && titer > 0) {
-            // Both accumulators must have been read out by the previous
-            // tile's epilogues (every tile's epilogues release both).
-            const uint32_t par = (titer - 1) & 1;
-            if (!__all_sync(0xffffffffu, mbar_wait(&S.acc_empty[0], par) && mbar_wait(&S.acc_empty[1], par))) {
+          if (kb == 0) {
+            // The regions this tile writes must have been read out by the
+            // epilogues of their previous uses.
+            bool got = true;
+            if (reg.uses(r0) > 0) got = mbar_wait(&S.reg_empty[r0], (reg.uses(r0) - 1) & 1);
+            if (got && r1 >= 0 && reg.uses(r1) > 0) got = mbar_wait(&S.reg_empty[r1], (reg.uses(r1) - 1) & 1);
+            if (!__all_sync(0xffffffffu, got)) {
               if (lane == 0) p_fail(S, sb);
               ok = false;
               break;
@@ -333,12 +370,11 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_w, const __gri
           if (elect_one()) {
 #pragma unroll
             for (int k16 = 0; k16 < PK / 16; ++k16)
-              tc_mma_bf16_pair(S.tmem_base, da + 2 * k16, db + 2 * k16, idesc0, (kb | k16) != 0);
+              tc_mma_bf16_pair(d0, da + 2 * k16, db + 2 * k16, idesc0, (kb | k16) != 0);
             if (tl.N1 > 0) {
 #pragma unroll
               for (int k16 = 0; k16 < PK / 16; ++k16)
-                tc_mma_bf16_pair(S.tmem_base + NA, da + 2 * k16, db + b1off + 2 * k16, idesc1,
-                                 (kb | k16) != 0);
+                tc_mma_bf16_pair(d1, da + 2 * k16, db + b1off + 2 * k16, idesc1, (kb | k16) != 0);
             }
             tc_commit_pair_both(&S.empty[s]);
           }
@@ -349,28 +385,39 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_w, const __gri
           }
         }
         if (!ok) break;
-        if (elect_one()) tc_commit_pair_both(&S.tmem_full);
+        if (elect_one()) {
+          tc_commit_pair_both(&S.reg_full[r0]);
+          if (r1 >= 0) tc_commit_pair_both(&S.reg_full[r1]);
+        }
         __syncwarp();
+        reg.used(r0);
+        if (r1 >= 0) reg.used(r1);
       }
     }
   } else {
     // Epilogue: warp w reads tensor-memory lanes 32 * (w % 4) .. +31 (its
-    // CTA's weight rows) of accumulator (w - 2) / 4.
+    // CTA's weight rows) of region (w - 2) / 4, for every tile that uses it.
     const int q = warp & 3;
-    const int acc = (warp - 2) / 4;
-    const uint32_t empty_cl = mapa_shared(smem_u32(&S.acc_empty[acc]), 0);
+    const int myreg = (warp - 2) / 4;
+    const uint32_t empty_cl = mapa_shared(smem_u32(&S.reg_empty[myreg]), 0);
+    Regions reg;
     for (int titer = 0;; ++titer) {
       const int t = next_tile(S, titer);
       if (t < 0) { p_fail(S, sb); break; }
       if (t >= ntiles || p_aborted(S)) break;
       const PTile tl = decode_ptile(S, t, mtiles);
-      if (!mbar_wait(&S.tmem_full, titer & 1)) { p_fail(S, sb); break; }
+      int r0, r1;
+      reg.take(tl, r0, r1);
+      if (myreg != r0 && myreg != r1) continue;  // this tile leaves the region alone
+      const int acc = myreg == r0 ? 0 : 1;       // which of the tile's accumulators it holds
+      if (!mbar_wait(&S.reg_full[myreg], reg.uses(myreg) & 1)) { p_fail(S, sb); break; }
+      reg.used(myreg);
       tc_fence_after();
       const int N = acc == 0 ? tl.N0 : tl.N1;
       const int j0 = acc == 0 ? 0 : tl.N0;  // the tile's pair of this accumulator's column 0
       const int nvalid = min(N, tl.valid - j0);
       const int rloc = tl.mt * 2 * PM + static_cast<int>(rank) * PM + q * 32 + lane;
-      const uint32_t tbase = S.tmem_base + static_cast<uint32_t>(acc * NA) + (static_cast<uint32_t>(q * 32) << 16);
+      const uint32_t tbase = S.tmem_base + static_cast<uint32_t>(myreg * NA) + (static_cast<uint32_t>(q * 32) << 16);
       // The accumulator's columns are read in two halves of 128 (SiLU,
       // rounded to bf16, two per word): the first half is read and stored,
       // then the second half is read, the accumulator is handed back to the

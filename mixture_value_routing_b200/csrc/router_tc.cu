@@ -13,12 +13,16 @@
 //     left), and the router runs as one GEMM against the 3E = 192 plane rows.
 //     logits[e] = (acc_hi[e] + acc_mid[e]) + acc_lo[e]: the same products as
 //     an fp32 dot product, accumulated in fp32 in another order.
-//   * One CTA per 128 tokens: a TMA warp streams 128 x 64 token tiles and
-//     192 x 64 plane tiles (128-byte swizzle) through 5 stages; one thread
-//     issues tcgen05.mma (M = 128, N = 192, K = 16) into tensor memory; four
-//     epilogue warps read one token per thread (all 192 columns), form the
-//     64 logits, the sigmoid scores and the biased selection in registers and
-//     write idx / w, plus the tile's expert histogram for the grouping.
+//   * One SM pair (a two-CTA cluster) per 256 tokens: each CTA's TMA warp
+//     streams its 128 x 64 token tile and its half (96 rows) of the 192 x 64
+//     plane tile (128-byte swizzle) through 7 stages of 28 KB, so a CTA
+//     streams 30% fewer bytes than with all plane rows in every CTA; the even
+//     CTA issues tcgen05.mma.cta_group::2 (M = 256 tokens, N = 192, K = 16),
+//     which accumulates each CTA's 128 tokens in its own tensor memory.  Four
+//     epilogue warps per CTA read one token per thread (all 192 columns),
+//     form the 64 logits, the sigmoid scores and the biased selection in
+//     registers and write idx / w, plus the 128-token tile's expert histogram
+//     for the grouping.
 // Every wait is bounded (MOVA_ERR_TIMEOUT, then drain and free).
 #include <cuda.h>
 
@@ -30,12 +34,12 @@ namespace mova {
 
 namespace {
 
-constexpr int RM = 128;  // tokens per CTA
-constexpr int RN = 192;  // 3 planes x 64 experts
+constexpr int RM = 128;  // tokens per CTA (256 per SM pair)
+constexpr int RN = 192;  // 3 planes x 64 experts (96 plane rows in each CTA of the pair)
 constexpr int RK = 64;
-constexpr int kRStages = 5;
+constexpr int kRStages = 7;
 constexpr int kRABytes = RM * RK * 2;
-constexpr int kRBBytes = RN * RK * 2;
+constexpr int kRBBytes = (RN / 2) * RK * 2;
 constexpr int kRStageBytes = kRABytes + kRBBytes;
 constexpr int kRThreads = 6 * 32;  // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
 constexpr uint32_t kRTmemCols = 256;
@@ -116,8 +120,9 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_consta
   RSmem& S = *reinterpret_cast<RSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();
   const int nk = d / RK;
-  const int t0 = blockIdx.x * RM;
+  const int t0 = blockIdx.x * RM;  // this CTA's 128 tokens (the pair's M = 256)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kRStages; ++s) {
@@ -136,16 +141,19 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_consta
   // the second half of d.
   const uint32_t tmem_cols = parts == 2 ? 2 * kRTmemCols : kRTmemCols;
   if (warp == 1) {
-    tmem_alloc(&S.tmem_base, tmem_cols);
-    tmem_relinquish();
+    tmem_alloc_pair(&S.tmem_base, tmem_cols);
+    tmem_relinquish_pair();
   }
   pdl_wait();  // the plane split of this call is complete
   tc_fence_before();
-  __syncthreads();
+  cluster_sync_all();  // barriers and tensor memory of both CTAs are ready
   tc_fence_after();
 
   if (warp == 0) {
-    // The whole warp runs the loop; one elected lane issues the copies.
+    // The whole warp runs the loop; one elected lane issues the copies: this
+    // CTA's 128 token rows and its half of the 192 plane rows, completing on
+    // the even CTA's stage barrier (which declares both CTAs' bytes).
+    const uint32_t full0_cl = mapa_shared(smem_u32(&S.full[0]), 0);
     int s = 0;
     uint32_t phase = 0;
     for (int kb = 0; kb < nk; ++kb) {
@@ -157,9 +165,10 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_consta
         break;
       }
       if (elect_one()) {
-        mbar_arrive_expect_tx(&S.full[s], kRStageBytes);
-        tma_load_2d_nohint(S.stage[s], &tmap_x, kb * RK, t0, &S.full[s]);
-        tma_load_2d_nohint(S.stage[s] + kRABytes, &tmap_w, kb * RK, 0, &S.full[s]);
+        const uint32_t full_cl = full0_cl + static_cast<uint32_t>(s) * 8u;
+        if (rank == 0) mbar_arrive_expect_tx(&S.full[s], 2 * kRStageBytes);
+        tma_load_2d_pair(S.stage[s], &tmap_x, kb * RK, t0, full_cl);
+        tma_load_2d_pair(S.stage[s] + kRABytes, &tmap_w, kb * RK, static_cast<int>(rank) * (RN / 2), full_cl);
       }
       __syncwarp();
       if (++s == kRStages) {
@@ -168,48 +177,50 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_consta
       }
     }
   } else if (warp == 1) {
-    // The whole warp runs the loop; one elected lane issues the MMAs.  Stage
-    // descriptors are built once and advanced by adding offsets (16-byte
-    // units), so issuing stays cheaper than the MMAs themselves.
-    const uint32_t idesc = idesc_bf16_f32(RM, RN);
-    const uint64_t adesc0 = smem_desc_sw128(smem_u32(S.stage[0]));
-    const uint64_t bdesc0 = smem_desc_sw128(smem_u32(S.stage[0]) + kRABytes);
-    constexpr uint32_t kStageDesc = kRStageBytes >> 4;
-    bool ok = true;
-    int s = 0;
-    uint32_t phase = 0;
-    const int khalf = parts == 2 ? nk / 2 : nk;
-    for (int kb = 0; kb < nk; ++kb) {
-      if (!__all_sync(0xffffffffu, mbar_wait(&S.full[s], phase))) {
-        if (lane == 0) {
-          raise_status(sb, MOVA_ERR_TIMEOUT, blockIdx.x);
-          S.abort = 1;
+    if (rank == 0) {
+      // The whole warp runs the loop; one elected lane issues the pair's
+      // MMAs (M = 256 tokens, N = 192 plane rows: 96 from each CTA) and
+      // commits to both CTAs' barriers.
+      const uint32_t idesc = idesc_bf16_f32(2 * RM, RN);
+      const uint64_t adesc0 = smem_desc_sw128(smem_u32(S.stage[0]));
+      const uint64_t bdesc0 = smem_desc_sw128(smem_u32(S.stage[0]) + kRABytes);
+      constexpr uint32_t kStageDesc = kRStageBytes >> 4;
+      bool ok = true;
+      int s = 0;
+      uint32_t phase = 0;
+      const int khalf = parts == 2 ? nk / 2 : nk;
+      for (int kb = 0; kb < nk; ++kb) {
+        if (!__all_sync(0xffffffffu, mbar_wait(&S.full[s], phase))) {
+          if (lane == 0) {
+            raise_status(sb, MOVA_ERR_TIMEOUT, blockIdx.x);
+            S.abort = 1;
+          }
+          ok = false;
+          break;
         }
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      const uint64_t da = adesc0 + static_cast<uint64_t>(s) * kStageDesc;
-      const uint64_t db = bdesc0 + static_cast<uint64_t>(s) * kStageDesc;
-      const bool second = kb >= khalf;
-      const uint32_t d_tmem = S.tmem_base + (second ? kRTmemCols : 0u);
-      const int kl = second ? kb - khalf : kb;  // k-step within its partition
-      if (elect_one()) {
+        tc_fence_after();
+        const uint64_t da = adesc0 + static_cast<uint64_t>(s) * kStageDesc;
+        const uint64_t db = bdesc0 + static_cast<uint64_t>(s) * kStageDesc;
+        const bool second = kb >= khalf;
+        const uint32_t d_tmem = S.tmem_base + (second ? kRTmemCols : 0u);
+        const int kl = second ? kb - khalf : kb;  // k-step within its partition
+        if (elect_one()) {
 #pragma unroll
-        for (int k16 = 0; k16 < RK / 16; ++k16)
-          tc_mma_bf16(d_tmem, da + 2 * k16, db + 2 * k16, idesc, (kl | k16) != 0);
-        tc_commit(&S.empty[s]);
+          for (int k16 = 0; k16 < RK / 16; ++k16)
+            tc_mma_bf16_pair(d_tmem, da + 2 * k16, db + 2 * k16, idesc, (kl | k16) != 0);
+          tc_commit_pair_both(&S.empty[s]);
+        }
+        __syncwarp();
+        if (++s == kRStages) {
+          s = 0;
+          phase ^= 1;
+        }
       }
+      if (ok && elect_one()) tc_commit_pair_both(&S.tmem_full);
       __syncwarp();
-      if (++s == kRStages) {
-        s = 0;
-        phase ^= 1;
-      }
     }
-    if (ok && elect_one()) tc_commit(&S.tmem_full);
-    __syncwarp();
   } else {
-    // Epilogue: thread = token (TMEM lane).
+    // Epilogue: thread = token (TMEM lane of this CTA).
     const int lg = warp & 3;
     const int t = t0 + lg * 32 + lane;
     if (mbar_wait(&S.tmem_full, 0)) {
@@ -287,18 +298,17 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_consta
     }
   }
   __syncthreads();
-  if (tile_counts != nullptr && threadIdx.x < 64)
+  if (tile_counts != nullptr && threadIdx.x < 64 && t0 < T)
     tile_counts[blockIdx.x * 64 + threadIdx.x] = S.hist[threadIdx.x];
+  tc_fence_before();
+  cluster_sync_all();  // neither CTA leaves while the pair may still touch its memory
   if (S.abort && threadIdx.x == 0) {
-    for (int s = 0; s < kRStages; ++s) {
-      mbar_wait(&S.full[s], 0);
-      mbar_wait(&S.empty[s], 0);
-    }
+    for (int s = 0; s < kRStages; ++s) mbar_wait(&S.empty[s], 0);
   }
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(S.tmem_base, tmem_cols);
+    tmem_dealloc_pair(S.tmem_base, tmem_cols);
   }
 }
 
@@ -326,7 +336,7 @@ cudaError_t launch_router_tc(const void* x, const float* Wr, const float* br, in
   const cuuint64_t wdim[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(RN)};
   const cuuint64_t stride[1] = {static_cast<cuuint64_t>(d) * 2};
   const cuuint32_t xbox[2] = {RK, RM};
-  const cuuint32_t wbox[2] = {RK, RN};
+  const cuuint32_t wbox[2] = {RK, RN / 2};
   const cuuint32_t es[2] = {1, 1};
   if (enc(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(x), xdim, stride, xbox, es,
           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -340,9 +350,26 @@ cudaError_t launch_router_tc(const void* x, const float* Wr, const float* br, in
   err = cudaFuncSetAttribute(router_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem));
   if (err != cudaSuccess) return err;
-  const int grid = (T + RM - 1) / RM;
-  return launch_pdl(router_tc_kernel, dim3(grid), dim3(kRThreads), smem, stream, tx, tw, br, T, d, E,
-                    k, scale, idx, w, tile_counts, sb, partitions == 2 ? 2 : 1);
+  // One SM pair per 256 tokens (the last pair's odd CTA may hold none: its
+  // token rows are read as zeros and nothing of it is stored).
+  const int grid = 2 * ((T + 2 * RM - 1) / (2 * RM));
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kRThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  note_launch();
+  return cudaLaunchKernelEx(&cfg, router_tc_kernel, tx, tw, br, T, d, E, k, scale, idx, w, tile_counts, sb,
+                            partitions == 2 ? 2 : 1);
 }
 
 }  // namespace mova
