@@ -209,12 +209,32 @@ mova_status mova_workspace_parts(int T, int d, int E, int k, int n, size_t* offs
  *                     "Implementation pitfalls").  Where partial sums cancel,
  *                     the rounding of each half to fp32 decides the logit, and
  *                     so the selection.  Needs d % 128 == 0; other values
- *                     return MOVA_ERR_UNSUPPORTED. */
+ *                     return MOVA_ERR_UNSUPPORTED.
+ *
+ *  decode_launches    bf16 decode batches (T <= 8) on the weight-streaming
+ *                     path.  1: one persistent kernel per call -- every CTA
+ *                     first computes part of the router logits, all CTAs
+ *                     meet at a grid barrier (bounded wait), then each
+ *                     selects, groups, streams its share of the active
+ *                     experts' weights and combines.  0 or 2 (the default,
+ *                     measured 0.7 us faster per T = 8 step on B200, as the
+ *                     logits kernel overlaps the previous call's tail): the
+ *                     logits in a kernel of their own, then the streaming
+ *                     kernel (chained with programmatic dependent launch).
+ *                     Both give identical results.  The barrier words
+ *                     are library-owned device memory, a ring of 64 reused
+ *                     in turn, so calls on one stream never share one; calls
+ *                     in flight at once on different streams of one device
+ *                     may, when 64 or more are, and must then use 2.  The one
+ *                     kernel needs all its CTAs (one per SM) resident at
+ *                     once: with the device shared by other work a call may
+ *                     report MOVA_ERR_TIMEOUT instead; use 2 there. */
 typedef struct mova_options {
   mova_path path;
   void* const* events;
   long long wv_expert_stride;
   int router_partitions;
+  int decode_launches;
 } mova_options;
 
 /* mova_route with options (only router_partitions applies). */
@@ -236,7 +256,9 @@ mova_status mova_value_routed_opts(const void* x, mova_dtype x_dt, const float* 
 /* Synchronises `stream`, then returns and clears the device status word
  * held in `ws` (MOVA_OK if no device-side check fired since the last read).
  * `detail_out` (nullable) receives the first offending item (e.g. the flat
- * pair index of a bad expert index). */
+ * pair index of a bad expert index).  After a MOVA_ERR_TIMEOUT it also
+ * restores the one-launch decode kernel's grid-barrier words, which a wait
+ * that ran out leaves unbalanced. */
 mova_status mova_get_status(void* ws, int32_t* detail_out, void* stream);
 
 /* Self-test of the device-side failure detection: launches one thread that
@@ -249,13 +271,16 @@ mova_status mova_selftest_wait_timeout(void* ws, long long limit_cycles, void* s
 
 /* Self-test of the weight-streaming kernel's failure handling: arms the
  * next weight-streaming launch in this process so that its first CTA stops
- * issuing weight copies at stage `stall_stage`, and its pipeline waits give
- * up after `limit_cycles` clock cycles (at most about one second's worth).
- * That launch then records MOVA_ERR_TIMEOUT in the status word, every warp
- * leaves, the copies already issued are drained, and the context stays
- * usable.  The arming is consumed by that one launch.  Not part of the
- * method; returns MOVA_ERR_INVALID_ARG for a negative stage or a limit out of
- * range. */
+ * issuing weight copies at stage `stall_stage` (>= 0), or -- with
+ * MOVA_STALL_AT_BARRIER -- does not arrive at the one-launch decode kernel's
+ * grid barrier; its waits give up after `limit_cycles` clock cycles (at most
+ * about one second's worth).  That launch then records MOVA_ERR_TIMEOUT in
+ * the status word, every warp leaves, the copies already issued are
+ * drained, and the context stays usable (mova_get_status, reading that
+ * timeout, also restores the barrier words).  The arming is consumed by that
+ * one launch.  Not part of the method; returns MOVA_ERR_INVALID_ARG for
+ * another negative stage or a limit out of range. */
+#define MOVA_STALL_AT_BARRIER (-2)
 mova_status mova_selftest_arm_stream_stall(int stall_stage, long long limit_cycles);
 
 /* The path AUTO would pick for these sizes and dtype (for tests/benches). */

@@ -35,7 +35,8 @@ _sz = ctypes.c_size_t
 class Options(ctypes.Structure):
     """mova_options (include/mova.h)."""
     _fields_ = [("path", ctypes.c_int), ("events", ctypes.c_void_p),
-                ("wv_expert_stride", ctypes.c_longlong), ("router_partitions", ctypes.c_int)]
+                ("wv_expert_stride", ctypes.c_longlong), ("router_partitions", ctypes.c_int),
+                ("decode_launches", ctypes.c_int)]
 
 
 SIGNATURES = {

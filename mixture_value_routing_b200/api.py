@@ -85,11 +85,11 @@ def launch_count() -> int:
     return int(_lib.load().mova_launch_count())
 
 
-def _opts(path="auto", events=None, wv_stride=0, partitions=0):
+def _opts(path="auto", events=None, wv_stride=0, partitions=0, decode_launches=0):
     """A mova_options value (kept alive by the caller for the call)."""
     ev = _events(events)
     o = _lib.Options(_PATH[path], ctypes.cast(ev, ctypes.c_void_p) if ev is not None else None,
-                     int(wv_stride), int(partitions))
+                     int(wv_stride), int(partitions), int(decode_launches))
     return o, ev
 
 
@@ -194,10 +194,11 @@ def value_routed(x: torch.Tensor, Wr: torch.Tensor, br: torch.Tensor, Wv: torch.
                  k: int = 4, scale: float = 2.5, return_routing: bool = False,
                  path: str = "auto", ws: Optional[torch.Tensor] = None,
                  out: Optional[torch.Tensor] = None, events=None, rows: Optional[tuple] = None,
-                 partitions: int = 0):
+                 partitions: int = 0, decode_launches: int = 0):
     """Full value path: v (T, n) in x's dtype [, idx (T, k) int32, w (T, k) fp32].
     rows=(row0, count): only those rows of every expert (a head-parallel
-    slice, v is (T, count)); partitions=2: the router's two-partition sum."""
+    slice, v is (T, count)); partitions=2: the router's two-partition sum;
+    decode_launches=1: decode batches as one persistent kernel (default two)."""
     _need(x, "x", (torch.float32, torch.bfloat16), 2)
     _need(Wr, "Wr", (torch.float32,), 2)
     _need(br, "br", (torch.float32,), 1)
@@ -214,7 +215,7 @@ def value_routed(x: torch.Tensor, Wr: torch.Tensor, br: torch.Tensor, Wv: torch.
     if ws is None:
         ws = _workspace(nbytes, dev)
     lib = _lib.load()
-    o, _ev = _opts(path, events, stride, partitions)
+    o, _ev = _opts(path, events, stride, partitions, decode_launches)
     _lib.check(lib.mova_value_routed_opts(_ptr(x), _DT[x.dtype], _ptr(Wr), _ptr(br), _ptr(Wb),
                                           _DT[Wv.dtype], T, d, E, k, n, float(scale), _ptr(v),
                                           _ptr(idx), _ptr(w), _ptr(ws), ws.numel(), ctypes.byref(o),

@@ -51,6 +51,8 @@ cudaError_t launch_router_logits(const void* x, mova_dtype x_dt, const float* Wr
                                  StatusBlock* sb, cudaStream_t stream);
 cudaError_t launch_select_group(const float* part, int S, const float* br, int T, int E, int k, float scale,
                                 int32_t* idx, float* w, const GroupOut* g, cudaStream_t stream);
+// The number S of K ranges the decode partial logits use.
+int decode_logit_splits(int d, int E, int partitions);
 
 // Every kernel launch the library enqueues is counted (mova_launch_count).
 void note_launch();
@@ -143,7 +145,22 @@ struct RouteIn {
   int32_t* perm_out;
   int32_t* pos_out;
   int32_t* active_out;
+  // One-launch decode (Wr non-null): the kernel first computes the partial
+  // logits itself -- part[s][t][e] for the S K ranges, one (expert, range)
+  // per CTA -- into part_out (== part), resets the status and the combine
+  // tickets, and meets every other CTA at a grid barrier (slot bar_slot of
+  // the library's ring of barrier words) before it selects.
+  const float* Wr;
+  float* part_out;
+  int bar_slot;
 };
+
+// Ring of grid-barrier words of the one-launch decode kernel (library-owned
+// device memory, zero at load, left as found by every completed barrier):
+// the slot for the next launch, and a reset of the whole ring (after a
+// barrier that ran out, which leaves its word unbalanced).
+int next_grid_barrier_slot();
+cudaError_t reset_grid_barriers(cudaStream_t stream);
 
 // Test-only fault injection for the weight-streaming kernel
 // (mova_selftest_arm_stream_stall): the limit of its pipeline waits in clock
@@ -153,6 +170,7 @@ struct RouteIn {
 struct StreamFault {
   long long wait_limit;
   int stall_stage;
+  bool skip_barrier;  // the first CTA does not arrive at the one-launch grid barrier
 };
 StreamFault take_stream_fault();
 

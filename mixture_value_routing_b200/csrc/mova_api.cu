@@ -41,8 +41,9 @@ void note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 StreamFault take_stream_fault() {
   const int stage = g_fault_stage.exchange(-1);
   const long long limit = g_fault_limit.exchange(0);
-  if (stage < 0 || limit <= 0) return StreamFault{kWaitLimitCycles, -1};
-  return StreamFault{limit, stage};
+  if (stage == -1 || limit <= 0) return StreamFault{kWaitLimitCycles, -1, false};
+  if (stage == MOVA_STALL_AT_BARRIER) return StreamFault{limit, -1, true};
+  return StreamFault{limit, stage, false};
 }
 
 int sm_count() {
@@ -136,6 +137,7 @@ struct Opts {
   void* const* events = nullptr;
   long long ldw = 0;   // rows between experts in Wv (n if 0 was given)
   int partitions = 1;  // router reduction halves (1 or 2)
+  int decode_launches = 2;
 };
 
 mova_status read_opts(const mova_options* o, int d, int n, Opts* out) {
@@ -145,7 +147,9 @@ mova_status read_opts(const mova_options* o, int d, int n, Opts* out) {
     r.events = o->events;
     r.ldw = o->wv_expert_stride;
     r.partitions = o->router_partitions == 0 ? 1 : o->router_partitions;
+    r.decode_launches = o->decode_launches == 0 ? 2 : o->decode_launches;
   }
+  if (r.decode_launches != 1 && r.decode_launches != 2) return MOVA_ERR_INVALID_ARG;
   if (r.path != MOVA_PATH_AUTO && r.path != MOVA_PATH_STREAM && r.path != MOVA_PATH_TENSOR &&
       r.path != MOVA_PATH_TENSOR_1CTA)
     return MOVA_ERR_INVALID_ARG;
@@ -337,7 +341,7 @@ mova_status mova_value_ex(const void* x, mova_dtype x_dt, const void* idx, mova_
                           const void* wgt, mova_dtype w_dt, const void* Wv, mova_dtype wv_dt, int T,
                           int d, int E, int k, int n, void* v, void* ws, size_t ws_bytes,
                           mova_path path, void* const* events, void* stream) {
-  const mova_options o{path, events, 0, 0};
+  const mova_options o{path, events, 0, 0, 0};
   return mova_value_opts(x, x_dt, idx, idx_dt, wgt, w_dt, Wv, wv_dt, T, d, E, k, n, v, ws, ws_bytes, &o,
                          stream);
 }
@@ -384,11 +388,18 @@ mova_status mova_value_routed_opts(const void* x, mova_dtype x_dt, const float* 
   if (rp == MOVA_PATH_STREAM && T <= kFusedCombineMaxT && stream_resident(T, d, x_dt) &&
       stream_experts_smem(d, x_dt, T, nullptr) != 0) {
     int S = 0;
-    if (err == cudaSuccess)
-      err = launch_router_logits(x, x_dt, Wr, T, d, E, o.partitions, w.logits, &S, w.tickets, combine_tickets(T, n), w.sb, s);
+    const bool one = o.decode_launches == 1;
+    if (one) {
+      S = decode_logit_splits(d, E, o.partitions);
+    } else if (err == cudaSuccess) {
+      err = launch_router_logits(x, x_dt, Wr, T, d, E, o.partitions, w.logits, &S, w.tickets,
+                                 combine_tickets(T, n), w.sb, s);
+    }
     if (err == cudaSuccess) err = mark(events, 1, s);
     if (err == cudaSuccess) err = mark(events, 2, s);
-    const RouteIn ri{w.logits, S, br, E, scale, idx, wgt, w.counts, w.offsets, w.perm, w.pos, w.active};
+    const RouteIn ri{w.logits, S,       br,         E,        scale,   idx,   wgt,
+                     w.counts, w.offsets, w.perm, w.pos, w.active,
+                     one ? Wr : nullptr, w.logits, one ? next_grid_barrier_slot() : 0};
     if (err == cudaSuccess)
       err = launch_stream_experts(x, Wv, o.ldw, x_dt, w.counts, w.offsets, w.perm, wgt, w.active, w.sb, T, d,
                                   n, k, E, static_cast<float*>(w.P), w.tickets, v, ri, s);
@@ -431,7 +442,7 @@ mova_status mova_value_routed_ex(const void* x, mova_dtype x_dt, const float* Wr
                                  int n, float scale, void* v, int32_t* idx_out, float* w_out,
                                  void* ws, size_t ws_bytes, mova_path path, void* const* events,
                                  void* stream) {
-  const mova_options o{path, events, 0, 0};
+  const mova_options o{path, events, 0, 0, 0};
   return mova_value_routed_opts(x, x_dt, Wr, br, Wv, wv_dt, T, d, E, k, n, scale, v, idx_out, w_out, ws,
                                 ws_bytes, &o, stream);
 }
@@ -453,7 +464,9 @@ mova_status mova_selftest_wait_timeout(void* ws, long long limit_cycles, void* s
 }
 
 mova_status mova_selftest_arm_stream_stall(int stall_stage, long long limit_cycles) {
-  if (stall_stage < 0 || limit_cycles <= 0 || limit_cycles > kWaitLimitCycles) return MOVA_ERR_INVALID_ARG;
+  if ((stall_stage < 0 && stall_stage != MOVA_STALL_AT_BARRIER) || limit_cycles <= 0 ||
+      limit_cycles > kWaitLimitCycles)
+    return MOVA_ERR_INVALID_ARG;
   g_fault_limit.store(limit_cycles);
   g_fault_stage.store(stall_stage);
   return MOVA_OK;
@@ -479,6 +492,12 @@ mova_status mova_get_status(void* ws, int32_t* detail_out, void* stream) {
   err = cudaMemcpy(&sb, ws, sizeof(sb), cudaMemcpyDeviceToHost);
   if (err != cudaSuccess) return from_cuda(err);
   if (detail_out) *detail_out = sb.detail;
+  if (sb.code == MOVA_ERR_TIMEOUT) {
+    // A grid barrier that ran out leaves its word unbalanced: restore the ring.
+    err = reset_grid_barriers(s);
+    if (err == cudaSuccess) err = cudaStreamSynchronize(s);
+    if (err != cudaSuccess) return from_cuda(err);
+  }
   return static_cast<mova_status>(sb.code);
 }
 

@@ -89,6 +89,74 @@ __device__ __forceinline__ void select_token(const float* lg, const float* brs, 
   }
 }
 
+// Partial router logits of decode batches (T <= 8): 256 threads (8 warps)
+// sum one expert's router row against every token's x over a range of K.
+// Thread i takes the 8-element chunks c0 = cb + i, c0 + 256, ... < ce (the
+// first chunk's router weights w0 loaded by the caller, which may request
+// them early), 8 fused multiply-adds per token in ascending element order.
+// A transposing warp butterfly then leaves each token's warp sum in one lane
+// group, written to red[warp * 8 + token]; after a barrier of the 256
+// threads, partial_logits_final gives token t's sum (threads t < 8) with the
+// warps' sums added in warp order.  Every step has a fixed order, so the
+// partial logits do not depend on timing.
+constexpr int kPartThreads = 256;
+template <typename XT>
+__device__ __forceinline__ void partial_logits_warp(const float* __restrict__ wrow, const XT* __restrict__ x,
+                                                    int T, int d, int c0, int ce, const float (&w0)[8],
+                                                    int lane, int warp, float* red) {
+  float acc[8];
+#pragma unroll
+  for (int t = 0; t < 8; ++t) acc[t] = 0.f;
+  for (int c = c0; c < ce; c += kPartThreads) {
+    float w[8];
+    if (c == c0) {
+#pragma unroll
+      for (int q = 0; q < 8; ++q) w[q] = w0[q];
+    } else {
+      load8(wrow + 8 * c, w);
+    }
+#pragma unroll
+    for (int t = 0; t < 8; ++t) {
+      if (t < T) {
+        float xv[8];
+        load8(x + static_cast<size_t>(t) * d + 8 * c, xv);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) acc[t] = fmaf(w[q], xv[q], acc[t]);
+      }
+    }
+  }
+  // Transposing butterfly over the 8 token sums: after the steps with
+  // offsets 16, 8, 4 lane l holds token 4*b4 + 2*b3 + b2 (bits of l) summed
+  // over its 8-lane group pattern; offsets 2 and 1 finish the warp sum.
+  const bool u16 = (lane & 16) != 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float send = u16 ? acc[i] : acc[i + 4];
+    const float keep = u16 ? acc[i + 4] : acc[i];
+    acc[i] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
+  }
+  const bool u8 = (lane & 8) != 0;
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const float send = u8 ? acc[i] : acc[i + 2];
+    const float keep = u8 ? acc[i + 2] : acc[i];
+    acc[i] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+  }
+  const bool u4 = (lane & 4) != 0;
+  const float send = u4 ? acc[0] : acc[1];
+  const float keep = u4 ? acc[1] : acc[0];
+  acc[0] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
+  acc[0] += __shfl_xor_sync(0xffffffffu, acc[0], 2);
+  acc[0] += __shfl_xor_sync(0xffffffffu, acc[0], 1);
+  if ((lane & 3) == 0) red[warp * 8 + ((lane >> 4) & 1) * 4 + ((lane >> 3) & 1) * 2 + ((lane >> 2) & 1)] = acc[0];
+}
+__device__ __forceinline__ float partial_logits_final(const float* red, int t) {
+  float v = red[t];
+#pragma unroll
+  for (int w = 1; w < kPartThreads / 32; ++w) v += red[w * 8 + t];
+  return v;
+}
+
 // Grouping of N <= 64 pairs (pair f = token f / k, slot f % k, expert
 // sel[f]) by expert, by one warp: a stable counting sort.  Lane l holds pairs
 // l and l + 32; a pair's rank among the earlier pairs of its expert comes

@@ -160,7 +160,7 @@ router_kernel(const XT* __restrict__ x, const float* __restrict__ Wr, const floa
 // weight-streaming kernel, which then needs no grouping launch at all.
 // ---------------------------------------------------------------------------
 constexpr int kDecT = 8;
-constexpr int kLogitThreads = 256;
+constexpr int kLogitThreads = kPartThreads;
 
 template <typename XT>
 __global__ void __launch_bounds__(kLogitThreads)
@@ -194,61 +194,9 @@ router_logits_kernel(const float* __restrict__ Wr, const XT* __restrict__ x, int
     for (int i = tid; i < ntickets; i += kLogitThreads) tickets[i] = 0;
   }
 
-  float acc[kDecT];
-#pragma unroll
-  for (int t = 0; t < kDecT; ++t) acc[t] = 0.f;
-  for (int c = c0; c < ce; c += kLogitThreads) {
-    float w[8];
-    if (c == c0) {
-#pragma unroll
-      for (int q = 0; q < 8; ++q) w[q] = w0[q];
-    } else {
-      load8(wrow + 8 * c, w);
-    }
-#pragma unroll
-    for (int t = 0; t < kDecT; ++t) {
-      if (t < T) {
-        float xv[8];
-        load8(x + static_cast<size_t>(t) * d + 8 * c, xv);
-#pragma unroll
-        for (int q = 0; q < 8; ++q) acc[t] = fmaf(w[q], xv[q], acc[t]);
-      }
-    }
-  }
-
-  // Transposing butterfly over the 8 token sums: after the steps with
-  // offsets 16, 8, 4 lane l holds token 4*b4 + 2*b3 + b2 (bits of l) summed
-  // over its 8-lane group pattern; offsets 2 and 1 finish the warp sum.
-  {
-    const bool u16 = (lane & 16) != 0;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float send = u16 ? acc[i] : acc[i + 4];
-      const float keep = u16 ? acc[i + 4] : acc[i];
-      acc[i] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
-    }
-    const bool u8 = (lane & 8) != 0;
-#pragma unroll
-    for (int i = 0; i < 2; ++i) {
-      const float send = u8 ? acc[i] : acc[i + 2];
-      const float keep = u8 ? acc[i + 2] : acc[i];
-      acc[i] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
-    }
-    const bool u4 = (lane & 4) != 0;
-    const float send = u4 ? acc[0] : acc[1];
-    const float keep = u4 ? acc[1] : acc[0];
-    acc[0] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
-    acc[0] += __shfl_xor_sync(0xffffffffu, acc[0], 2);
-    acc[0] += __shfl_xor_sync(0xffffffffu, acc[0], 1);
-  }
-  if ((lane & 3) == 0) red[warp][((lane >> 4) & 1) * 4 + ((lane >> 3) & 1) * 2 + ((lane >> 2) & 1)] = acc[0];
+  partial_logits_warp(wrow, x, T, d, c0, ce, w0, lane, warp, &red[0][0]);
   __syncthreads();
-  if (tid < kDecT) {
-    float v = red[0][tid];
-#pragma unroll
-    for (int w = 1; w < kLogitThreads / 32; ++w) v += red[w][tid];
-    part[(s * kDecT + tid) * 64 + e] = v;
-  }
+  if (tid < kDecT) part[(s * kDecT + tid) * 64 + e] = partial_logits_final(&red[0][0], tid);
 }
 
 // Selection and grouping of a decode batch by one CTA, from the S partial
@@ -352,13 +300,15 @@ int logit_splits(int d, int E) {
   return S;
 }
 
+// Two router partitions: exactly two K ranges, the halves of d; the
+// selection adds their fp32 partial logits in range order.
+int decode_logit_splits(int d, int E, int partitions) { return partitions == 2 ? 2 : logit_splits(d, E); }
+
 cudaError_t launch_router_logits(const void* x, mova_dtype x_dt, const float* Wr, int T, int d, int E,
                                  int partitions, float* part, int* S_out, int32_t* tickets, int ntickets,
                                  StatusBlock* sb, cudaStream_t stream) {
   if (T <= 0 || T > kDecT) return cudaErrorInvalidValue;
-  // Two router partitions: exactly two K ranges, the halves of d; the
-  // selection adds their fp32 partial logits in range order.
-  const int S = partitions == 2 ? 2 : logit_splits(d, E);
+  const int S = decode_logit_splits(d, E, partitions);
   *S_out = S;
   return x_dt == MOVA_BF16 ? launch_logits_t<__nv_bfloat16>(x, Wr, T, d, E, S, part, tickets, ntickets, sb, stream)
                            : launch_logits_t<float>(x, Wr, T, d, E, S, part, tickets, ntickets, sb, stream);

@@ -25,6 +25,8 @@
 // completes a block of 8 output columns (per-block tickets) writes v there.
 // Every wait is bounded; a wait that runs out sets MOVA_ERR_TIMEOUT in the
 // status block and the CTA drains its copies and exits.
+#include <atomic>
+
 #include "common.cuh"
 #include "internal.h"
 #include "route_select.cuh"
@@ -32,6 +34,13 @@
 #include "sm100.cuh"
 
 namespace mova {
+
+// The one-launch decode kernel's grid-barrier words: library-owned device
+// memory, zero when the module loads.  Each launch takes the next slot of
+// the ring, so consecutive launches on a stream use different words, and a
+// completed barrier leaves its word as it found it (the top bit flipped).
+constexpr int kGridBarSlots = 64;
+__device__ unsigned int g_grid_bar[kGridBarSlots];
 
 namespace {
 
@@ -119,6 +128,34 @@ __device__ __forceinline__ bool consumers_any(bool v) {
   return r != 0;
 }
 
+// Grid-wide barrier of a launch whose CTAs are all resident (one per SM):
+// CTA 0 adds 2^31 - (G - 1) to the word and every other CTA adds 1, so the
+// word's top bit flips exactly when the last CTA arrives, whatever the order
+// and whatever the top bit was, and the low bits return to where they were.
+// Thread 0 of each CTA waits (bounded) for the flip; false if the wait ran
+// out.  skip_arrive (a test-only fault) keeps this CTA from arriving.
+__device__ __forceinline__ bool grid_barrier(unsigned int* word, long long limit, bool skip_arrive,
+                                             volatile int* ok_smem) {
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int ok = 1;
+    __threadfence();
+    const unsigned int add = blockIdx.x == 0 ? 0x80000000u - (gridDim.x - 1) : 1u;
+    const unsigned int old = skip_arrive ? *reinterpret_cast<volatile unsigned int*>(word) : atomicAdd(word, add);
+    const long long start = clock64();
+    while (((*reinterpret_cast<volatile unsigned int*>(word) ^ old) & 0x80000000u) == 0) {
+      if (clock64() - start > limit) {
+        ok = 0;
+        break;
+      }
+    }
+    __threadfence();
+    *ok_smem = ok;
+  }
+  __syncthreads();
+  return *ok_smem != 0;
+}
+
 template <typename DT>
 __global__ void __launch_bounds__(kThreads, 1)
 stream_experts_kernel(const DT* __restrict__ x, const DT* __restrict__ Wv,
@@ -176,7 +213,23 @@ stream_experts_kernel(const DT* __restrict__ x, const DT* __restrict__ Wv,
     *issued = 0;
     fence_barrier_init();
   }
-  pdl_wait();  // routing and grouping of this call are complete and visible
+  // One-launch decode: CTAs below E * S each compute one (expert, K range)
+  // of the partial logits; the first chunk of the router row is requested
+  // before the grid dependency wait (no kernel writes router weights).
+  const bool one_launch = route.Wr != nullptr;
+  const int lg_units = one_launch ? route.E * route.S : 0;
+  const bool lg_cta = static_cast<int>(blockIdx.x) < lg_units && threadIdx.x < kPartThreads;
+  int lg_e = 0, lg_c0 = 0, lg_ce = 0;
+  float lg_w0[8];
+  if (lg_cta) {
+    lg_e = blockIdx.x % route.E;
+    const int rs = blockIdx.x / route.E;
+    const int chunks = d / 8;
+    lg_ce = chunks * (rs + 1) / route.S;
+    lg_c0 = chunks * rs / route.S + threadIdx.x;
+    if (lg_c0 < lg_ce) load8(route.Wr + static_cast<size_t>(lg_e) * d + 8 * lg_c0, lg_w0);
+  }
+  pdl_wait();  // the previous kernel on the stream is complete (two-launch: routing of this call)
   if (resident && threadIdx.x == 0) {
     // The resident x tile: one bulk copy per token row, issued at once so its
     // latency overlaps the first weight stages.
@@ -184,6 +237,50 @@ stream_experts_kernel(const DT* __restrict__ x, const DT* __restrict__ Wv,
     mbar_arrive_expect_tx(xbar, static_cast<uint32_t>(T) * row_bytes_x);
     for (int t = 0; t < T; ++t)
       bulk_g2s(xs + t * pitch, x + static_cast<size_t>(t) * d, row_bytes_x, xbar, policy_evict_last());
+  }
+  if (one_launch) {
+    // The partial logits of this call (the part of the logits kernel of the
+    // two-launch path), then the status and tickets reset, then one grid
+    // barrier: after it every CTA reads all of them.
+    __shared__ int gb_ok;
+    float* lred = red;  // free until the weight stream starts
+    for (int unit = blockIdx.x; unit < lg_units; unit += gridDim.x) {
+      if (threadIdx.x < kPartThreads) {
+        const float* wrow = route.Wr + static_cast<size_t>(unit % route.E) * d;
+        const int rs = unit / route.E;
+        const int chunks = d / 8;
+        const int ce = chunks * (rs + 1) / route.S;
+        const int c0 = chunks * rs / route.S + threadIdx.x;
+        float w0[8];
+        if (unit == static_cast<int>(blockIdx.x) && lg_cta) {
+#pragma unroll
+          for (int q = 0; q < 8; ++q) w0[q] = lg_w0[q];
+        } else if (c0 < ce) {
+          load8(wrow + 8 * c0, w0);
+        }
+        partial_logits_warp(wrow, x, T, d, c0, ce, w0, lane, warp, lred);
+        consumers_sync();
+        if (threadIdx.x < kTok)
+          route.part_out[(rs * kTok + threadIdx.x) * 64 + unit % route.E] = partial_logits_final(lred, threadIdx.x);
+        consumers_sync();
+      }
+    }
+    if (blockIdx.x == 0) {
+      if (threadIdx.x == 0) {
+        sb->code = 0;
+        sb->detail = 0;
+        sb->work_next = 0;
+      }
+      for (int i = threadIdx.x; i < n / kRowsPerStage; i += kThreads) tickets[i] = 0;
+    }
+    if (!grid_barrier(&g_grid_bar[route.bar_slot], fault.wait_limit, fault.skip_barrier && blockIdx.x == 0,
+                      &gb_ok)) {
+      if (threadIdx.x == 0) {
+        raise_status(sb, MOVA_ERR_TIMEOUT, blockIdx.x);
+        *abort_flag = 1;
+      }
+    }
+    __syncthreads();
   }
   // Route mode: the consumer warps select and group the batch from the
   // partial logits (every CTA the same, in the same fixed order).
@@ -208,7 +305,7 @@ stream_experts_kernel(const DT* __restrict__ x, const DT* __restrict__ Wv,
 #pragma unroll
         for (int r = 0; r < kMaxLogitSplits; ++r)
           pv[h][r] = (r < route.S && threadIdx.x + h * kC < T * 64)
-                         ? route.part[r * kTok * 64 + threadIdx.x + h * kC] : 0.f;
+                         ? __ldcg(route.part + r * kTok * 64 + threadIdx.x + h * kC) : 0.f;
       const float bv = threadIdx.x < route.E ? route.br[threadIdx.x] : 0.f;
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
@@ -623,6 +720,19 @@ stream_experts_kernel(const DT* __restrict__ x, const DT* __restrict__ Wv,
 }
 
 }  // namespace
+
+namespace {
+std::atomic<unsigned int> g_bar_next{0};
+}  // namespace
+
+int next_grid_barrier_slot() { return static_cast<int>(g_bar_next.fetch_add(1) % kGridBarSlots); }
+
+cudaError_t reset_grid_barriers(cudaStream_t stream) {
+  void* p = nullptr;
+  cudaError_t err = cudaGetSymbolAddress(&p, g_grid_bar);
+  if (err != cudaSuccess) return err;
+  return cudaMemsetAsync(p, 0, sizeof(g_grid_bar), stream);
+}
 
 size_t stream_experts_smem(int d, mova_dtype dt, int T, int* stages_out) {
   const bool mma = dt == MOVA_BF16;

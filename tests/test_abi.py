@@ -145,5 +145,6 @@ def test_workspace_parts(lib):
 
 def test_stream_stall_arming_is_validated(lib):
     assert lib.mova_selftest_arm_stream_stall(-1, 1000) == _lib.ERR_INVALID_ARG
+    assert lib.mova_selftest_arm_stream_stall(-3, 1000) == _lib.ERR_INVALID_ARG
     assert lib.mova_selftest_arm_stream_stall(2, 0) == _lib.ERR_INVALID_ARG
     assert lib.mova_selftest_arm_stream_stall(2, 1 << 40) == _lib.ERR_INVALID_ARG

@@ -385,19 +385,59 @@ def test_deterministic(api):
 
 
 def test_decode_step_kernel_count(api):
-    """A bf16 decode step is two kernels: the router logits and the
-    weight-streaming experts (which also select, group and combine); fp32
-    runs selection/grouping and the combine as kernels of their own."""
-    for dtype, want in (("bf16", 2), ("f32", 4)):
+    """A bf16 decode step is one persistent kernel with decode_launches=1
+    (logits, grid barrier, selection, grouping, weight stream, combine), or
+    two by default (the logits kernel, then the streaming kernel); fp32 runs
+    selection/grouping and the combine as kernels of their own."""
+    for dtype, launches, want in (("bf16", 1, 1), ("bf16", 0, 2), ("bf16", 2, 2), ("f32", 0, 4)):
         lay = _layer(5, 2560, 64, 1024, dtype)
         bat = MI.make_batch(8, 5, dtype=dtype)
         args = (P.dev(bat.x, dtype), P.dev(lay.Wr, "f32"), P.dev(lay.br, "f32"), P.dev(lay.Wv, dtype))
-        api.value_routed(*args)
+        api.value_routed(*args, decode_launches=launches)
         torch.cuda.synchronize()
         before = api.launch_count()
-        api.value_routed(*args)
-        assert api.launch_count() - before == want, dtype
+        api.value_routed(*args, decode_launches=launches)
+        assert api.launch_count() - before == want, (dtype, launches)
     torch.cuda.synchronize()
+
+
+@pytest.mark.parametrize("T", [1, 8])
+def test_decode_two_launches(api, T):
+    """The two-launch decode path (logits kernel + streaming kernel) gives the
+    same values as the one-launch kernel, bit for bit, and passes the full
+    parity checks."""
+    lay = _layer(12, 2560, 64, 1024, "bf16")
+    bat = MI.make_batch(T, 12, dtype="bf16")
+    args = (P.dev(bat.x, "bf16"), P.dev(lay.Wr, "f32"), P.dev(lay.br, "f32"), P.dev(lay.Wv, "bf16"))
+    one = api.value_routed(*args, decode_launches=1).clone()
+    two, idx, w = api.value_routed(*args, return_routing=True, decode_launches=2)
+    torch.cuda.synchronize()
+    assert torch.equal(one, two)
+    x, ref = _routing_ref(bat, lay, 4)
+    idx_g = idx.cpu().numpy().astype(np.int64)
+    P.check_routing(idx_g, w.cpu().numpy().astype(np.float64), ref, 4, 2.5)
+    P.check_values(P.host_f64(two), O.combine(x, idx_g, O.weights_for(ref["s"], idx_g, 2.5), lay.Wv, "bf16"),
+                   "bf16")
+
+
+def test_decode_grid_barrier_timeout_and_recovery(api):
+    """The one-launch decode kernel's grid barrier is a bounded wait: with the
+    first CTA armed not to arrive and the waits limited to about a
+    millisecond, every CTA gives up, the call reports MOVA_ERR_TIMEOUT and
+    completes; reading the status restores the barrier words, and the next
+    calls (more than the ring of barrier words, so the damaged word comes
+    round again) give correct values."""
+    lay = _layer(43, 2560, 64, 1024, "bf16")
+    bat = MI.make_batch(8, 43, dtype="bf16")
+    args = (P.dev(bat.x, "bf16"), P.dev(lay.Wr, "f32"), P.dev(lay.br, "f32"), P.dev(lay.Wv, "bf16"))
+    ws = torch.empty(api.workspace_size(8, 2560, 64, 4, 1024), dtype=torch.uint8, device="cuda")
+    ref = api.value_routed(*args, decode_launches=2).clone()
+    api.arm_stream_stall(-2, 2_000_000)
+    api.value_routed(*args, ws=ws, decode_launches=1)
+    assert api.get_status(ws)[0] == "MOVA_ERR_TIMEOUT"
+    for _ in range(70):
+        assert torch.equal(api.value_routed(*args, ws=ws, decode_launches=1), ref)
+    assert api.get_status(ws)[0] == "MOVA_OK"
 
 
 # ---------------------------------------------------------------------------
@@ -441,11 +481,13 @@ def test_route_partitions_cancellation(api, T, dtype):
     if dtype == "bf16" and T <= 8:
         # The decode batches of the full path route in the logits kernel.
         Wv = _layer(3, d, E, 128, "bf16").Wv
-        _, idx2, w2 = api.value_routed(P.dev(xs, dtype), P.dev(Wr, "f32"), P.dev(br, "f32"),
-                                       P.dev(Wv, "bf16"), k, 2.5, return_routing=True, partitions=2)
-        torch.cuda.synchronize()
-        assert (idx2.cpu().numpy() == ref["idx"]).all()
-        np.testing.assert_allclose(w2.cpu().numpy(), 1.25, rtol=1e-6)
+        for launches in (1, 2):  # the one-launch kernel and the logits kernel
+            _, idx2, w2 = api.value_routed(P.dev(xs, dtype), P.dev(Wr, "f32"), P.dev(br, "f32"),
+                                           P.dev(Wv, "bf16"), k, 2.5, return_routing=True, partitions=2,
+                                           decode_launches=launches)
+            torch.cuda.synchronize()
+            assert (idx2.cpu().numpy() == ref["idx"]).all()
+            np.testing.assert_allclose(w2.cpu().numpy(), 1.25, rtol=1e-6)
 
 
 @pytest.mark.parametrize("T,d,dtype", [(8, 2560, "bf16"), (33, 2560, "bf16"), (130, 2560, "bf16"),
