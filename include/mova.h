@@ -221,7 +221,15 @@ mova_status mova_workspace_parts(int T, int d, int E, int k, int n, size_t* offs
  *                     logits kernel overlaps the previous call's tail): the
  *                     logits in a kernel of their own, then the streaming
  *                     kernel (chained with programmatic dependent launch).
- *                     Both give identical results.  The barrier words
+ *                     Both give identical results.
+ *
+ *  router_planes      NULL, or the router weight already split by
+ *                     mova_router_planes (for this Wr, E and d): bf16 batches
+ *                     routed on the tensor cores (T > 64) then skip the split
+ *                     of every call.  The planes depend on Wr only, so a
+ *                     model makes them once per layer when it loads.
+ *
+ *                     The barrier words
  *                     are library-owned device memory, a ring of 64 reused
  *                     in turn, so calls on one stream never share one; calls
  *                     in flight at once on different streams of one device
@@ -235,7 +243,23 @@ typedef struct mova_options {
   long long wv_expert_stride;
   int router_partitions;
   int decode_launches;
+  const void* router_planes;
 } mova_options;
+
+/* The fp32 router weight Wr (E, d) split exactly into three bf16 planes,
+ * Wr = hi + mid + lo (each the round-to-nearest bf16 of what the previous
+ * ones left; 8 + 8 + 8 significand bits cover fp32's 24), stored as a
+ * (3 * 64, d) bf16 matrix: row e of plane p at row 64 * p + e, rows E..63 of
+ * each plane zero.  The tensor-core router multiplies bf16 x by these planes,
+ * forming every product exactly, and adds the three fp32 accumulations
+ * (hi + mid) + lo: the logits of an fp32 dot product, accumulated in another
+ * order.  `planes` (device, 16-byte aligned) receives
+ * mova_router_planes_bytes(d) bytes; asynchronous on `stream`.  The routing
+ * calls split Wr themselves unless mova_options.router_planes is given.
+ * Errors: MOVA_ERR_INVALID_ARG for null or misaligned pointers, E outside
+ * [1, 64] or d not a positive multiple of 64. */
+size_t mova_router_planes_bytes(int d);
+mova_status mova_router_planes(const float* Wr, int E, int d, void* planes, void* stream);
 
 /* mova_route with options (only router_partitions applies). */
 mova_status mova_route_opts(const void* x, mova_dtype x_dt, const float* Wr, const float* br,

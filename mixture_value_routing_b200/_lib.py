@@ -36,7 +36,7 @@ class Options(ctypes.Structure):
     """mova_options (include/mova.h)."""
     _fields_ = [("path", ctypes.c_int), ("events", ctypes.c_void_p),
                 ("wv_expert_stride", ctypes.c_longlong), ("router_partitions", ctypes.c_int),
-                ("decode_launches", ctypes.c_int)]
+                ("decode_launches", ctypes.c_int), ("router_planes", ctypes.c_void_p)]
 
 
 SIGNATURES = {
@@ -57,6 +57,8 @@ SIGNATURES = {
     "mova_selftest_wait_timeout": (_i, [_vp, ctypes.c_longlong, _vp]),
     "mova_selftest_arm_stream_stall": (_i, [_i, ctypes.c_longlong]),
     "mova_workspace_parts": (_i, [_i, _i, _i, _i, _i, _vp]),
+    "mova_router_planes_bytes": (_sz, [_i]),
+    "mova_router_planes": (_i, [_vp, _i, _i, _vp, _vp]),
     "mova_value_routed_noalloc": (_i, [_vp, _i, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _vp,
                                        _vp]),
     "mova_route_opts": (_i, [_vp, _i, _vp, _vp, _i, _i, _i, _i, _f, _vp, _vp, _vp, _vp]),

@@ -85,12 +85,25 @@ def launch_count() -> int:
     return int(_lib.load().mova_launch_count())
 
 
-def _opts(path="auto", events=None, wv_stride=0, partitions=0, decode_launches=0):
+def _opts(path="auto", events=None, wv_stride=0, partitions=0, decode_launches=0, planes=None):
     """A mova_options value (kept alive by the caller for the call)."""
     ev = _events(events)
     o = _lib.Options(_PATH[path], ctypes.cast(ev, ctypes.c_void_p) if ev is not None else None,
-                     int(wv_stride), int(partitions), int(decode_launches))
+                     int(wv_stride), int(partitions), int(decode_launches),
+                     None if planes is None else ctypes.c_void_p(planes.data_ptr()))
     return o, ev
+
+
+def router_planes(Wr: torch.Tensor) -> torch.Tensor:
+    """The router weight split exactly into three bf16 planes (mova_router_planes),
+    to hand to value_routed(planes=...) so that calls skip the split."""
+    _need(Wr, "Wr", (torch.float32,), 2)
+    E, d = Wr.shape
+    lib = _lib.load()
+    nbytes = int(lib.mova_router_planes_bytes(d))
+    planes = torch.empty(nbytes // 2, dtype=torch.bfloat16, device=Wr.device)
+    _lib.check(lib.mova_router_planes(_ptr(Wr), E, d, _ptr(planes), _stream()), "mova_router_planes")
+    return planes
 
 
 def route(x: torch.Tensor, Wr: torch.Tensor, br: torch.Tensor, k: int = 4, scale: float = 2.5,
@@ -194,11 +207,13 @@ def value_routed(x: torch.Tensor, Wr: torch.Tensor, br: torch.Tensor, Wv: torch.
                  k: int = 4, scale: float = 2.5, return_routing: bool = False,
                  path: str = "auto", ws: Optional[torch.Tensor] = None,
                  out: Optional[torch.Tensor] = None, events=None, rows: Optional[tuple] = None,
-                 partitions: int = 0, decode_launches: int = 0):
+                 partitions: int = 0, decode_launches: int = 0,
+                 planes: Optional[torch.Tensor] = None):
     """Full value path: v (T, n) in x's dtype [, idx (T, k) int32, w (T, k) fp32].
     rows=(row0, count): only those rows of every expert (a head-parallel
     slice, v is (T, count)); partitions=2: the router's two-partition sum;
-    decode_launches=1: decode batches as one persistent kernel (default two)."""
+    decode_launches=1: decode batches as one persistent kernel (default two);
+    planes: the router's bf16 planes from router_planes(Wr), made once."""
     _need(x, "x", (torch.float32, torch.bfloat16), 2)
     _need(Wr, "Wr", (torch.float32,), 2)
     _need(br, "br", (torch.float32,), 1)
@@ -215,7 +230,11 @@ def value_routed(x: torch.Tensor, Wr: torch.Tensor, br: torch.Tensor, Wv: torch.
     if ws is None:
         ws = _workspace(nbytes, dev)
     lib = _lib.load()
-    o, _ev = _opts(path, events, stride, partitions, decode_launches)
+    if planes is not None:
+        _need(planes, "planes", (torch.bfloat16,), 1)
+        if planes.numel() * 2 < int(lib.mova_router_planes_bytes(d)):
+            raise ValueError("planes: too small for this d; make them with router_planes(Wr)")
+    o, _ev = _opts(path, events, stride, partitions, decode_launches, planes)
     _lib.check(lib.mova_value_routed_opts(_ptr(x), _DT[x.dtype], _ptr(Wr), _ptr(br), _ptr(Wb),
                                           _DT[Wv.dtype], T, d, E, k, n, float(scale), _ptr(v),
                                           _ptr(idx), _ptr(w), _ptr(ws), ws.numel(), ctypes.byref(o),

@@ -35,7 +35,10 @@ __device__ __forceinline__ void store8(__nv_bfloat16* p, const float v[8]) {
   *reinterpret_cast<uint4*>(p) = u;
 }
 
-template <typename PT, typename OT>
+// KS > 0: k == KS known at compile time -- all slots' positions, weights and
+// P vectors are loaded before the first multiply-add, so each thread keeps
+// KS independent 16-byte loads in flight.  KS == 0: any k, slot by slot.
+template <typename PT, typename OT, int KS>
 __global__ void __launch_bounds__(kThreads)
 combine_kernel(const PT* __restrict__ P, const int32_t* __restrict__ pos,
                const float* __restrict__ w32, int T, int k, int n, OT* __restrict__ v) {
@@ -52,13 +55,30 @@ combine_kernel(const PT* __restrict__ P, const int32_t* __restrict__ pos,
     float acc[8];
 #pragma unroll
     for (int q = 0; q < 8; ++q) acc[q] = 0.f;
-    for (int s = 0; s < k; ++s) {
-      const int p = pos[static_cast<size_t>(t) * k + s];
-      const float ws = w32[static_cast<size_t>(t) * k + s];
-      float pv[8];
-      load8_p(P + static_cast<size_t>(p) * n + c, pv);
+    if constexpr (KS > 0) {
+      int p[KS];
+      float ws[KS];
 #pragma unroll
-      for (int q = 0; q < 8; ++q) acc[q] = fmaf(ws, pv[q], acc[q]);
+      for (int s = 0; s < KS; ++s) {
+        p[s] = pos[static_cast<size_t>(t) * KS + s];
+        ws[s] = w32[static_cast<size_t>(t) * KS + s];
+      }
+      float pv[KS][8];
+#pragma unroll
+      for (int s = 0; s < KS; ++s) load8_p(P + static_cast<size_t>(p[s]) * n + c, pv[s]);
+#pragma unroll
+      for (int s = 0; s < KS; ++s)
+#pragma unroll
+        for (int q = 0; q < 8; ++q) acc[q] = fmaf(ws[s], pv[s][q], acc[q]);
+    } else {
+      for (int s = 0; s < k; ++s) {
+        const int p = pos[static_cast<size_t>(t) * k + s];
+        const float ws = w32[static_cast<size_t>(t) * k + s];
+        float pv[8];
+        load8_p(P + static_cast<size_t>(p) * n + c, pv);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) acc[q] = fmaf(ws, pv[q], acc[q]);
+      }
     }
     store8(v + static_cast<size_t>(t) * n + c, acc);
   }
@@ -72,7 +92,10 @@ cudaError_t launch_t(const void* P, const int32_t* pos, const float* w32, int T,
   const long long cap = static_cast<long long>(sm_count()) * 8;
   if (blocks > cap) blocks = cap;
   if (blocks < 1) blocks = 1;
-  return launch_pdl(combine_kernel<PT, OT>, dim3(static_cast<unsigned>(blocks)), dim3(kThreads), 0,
+  if (k == 4)
+    return launch_pdl(combine_kernel<PT, OT, 4>, dim3(static_cast<unsigned>(blocks)), dim3(kThreads), 0,
+                      stream, static_cast<const PT*>(P), pos, w32, T, k, n, static_cast<OT*>(v));
+  return launch_pdl(combine_kernel<PT, OT, 0>, dim3(static_cast<unsigned>(blocks)), dim3(kThreads), 0,
                     stream, static_cast<const PT*>(P), pos, w32, T, k, n, static_cast<OT*>(v));
 }
 

@@ -89,10 +89,13 @@ void* encode_tiled_fn();
 // receives each 128-token tile's expert histogram.
 constexpr int kTcRouterMinT = 64;  // bf16 batches above this many tokens use it
 size_t router_planes_bytes(int d);
+// prepared: planes made by launch_split_router beforehand (then `planes` is
+// not written), or null to split Wr into `planes` first.
 cudaError_t launch_router_tc(const void* x, const float* Wr, const float* br, int T, int d, int E,
                              int k, float scale, int partitions, int32_t* idx, float* w,
-                             int32_t* tile_counts, __nv_bfloat16* planes, StatusBlock* sb,
-                             cudaStream_t stream);
+                             int32_t* tile_counts, __nv_bfloat16* planes, const __nv_bfloat16* prepared,
+                             StatusBlock* sb, cudaStream_t stream);
+cudaError_t launch_split_router(const float* Wr, int E, int d, __nv_bfloat16* planes, cudaStream_t stream);
 
 // Stable counting sort of the pairs by expert.  idx_in has dtype idx_dt
 // (int32 or int8); when w_in is given (w_dt fp32 or fp16) it is converted to

@@ -138,6 +138,7 @@ struct Opts {
   long long ldw = 0;   // rows between experts in Wv (n if 0 was given)
   int partitions = 1;  // router reduction halves (1 or 2)
   int decode_launches = 2;
+  const void* planes = nullptr;  // prepared router planes
 };
 
 mova_status read_opts(const mova_options* o, int d, int n, Opts* out) {
@@ -148,7 +149,9 @@ mova_status read_opts(const mova_options* o, int d, int n, Opts* out) {
     r.ldw = o->wv_expert_stride;
     r.partitions = o->router_partitions == 0 ? 1 : o->router_partitions;
     r.decode_launches = o->decode_launches == 0 ? 2 : o->decode_launches;
+    r.planes = o->router_planes;
   }
+  if (r.planes != nullptr && (reinterpret_cast<uintptr_t>(r.planes) & 15) != 0) return MOVA_ERR_INVALID_ARG;
   if (r.decode_launches != 1 && r.decode_launches != 2) return MOVA_ERR_INVALID_ARG;
   if (r.path != MOVA_PATH_AUTO && r.path != MOVA_PATH_STREAM && r.path != MOVA_PATH_TENSOR &&
       r.path != MOVA_PATH_TENSOR_1CTA)
@@ -270,6 +273,15 @@ mova_status mova_route_opts(const void* x, mova_dtype x_dt, const float* Wr, con
                                  o.partitions, static_cast<cudaStream_t>(stream)));
 }
 
+size_t mova_router_planes_bytes(int d) { return d > 0 && d % 64 == 0 ? router_planes_bytes(d) : 0; }
+
+mova_status mova_router_planes(const float* Wr, int E, int d, void* planes, void* stream) {
+  if (!Wr || !planes || E < 1 || E > 64 || d <= 0 || d % 64 != 0) return MOVA_ERR_INVALID_ARG;
+  if (!aligned16(Wr) || !aligned16(planes)) return MOVA_ERR_INVALID_ARG;
+  return from_cuda(launch_split_router(Wr, E, d, static_cast<__nv_bfloat16*>(planes),
+                                       static_cast<cudaStream_t>(stream)));
+}
+
 mova_status mova_route(const void* x, mova_dtype x_dt, const float* Wr, const float* br, int T,
                        int d, int E, int k, float scale, int32_t* idx, float* w, void* stream) {
   return mova_route_opts(x, x_dt, Wr, br, T, d, E, k, scale, idx, w, nullptr, stream);
@@ -341,7 +353,7 @@ mova_status mova_value_ex(const void* x, mova_dtype x_dt, const void* idx, mova_
                           const void* wgt, mova_dtype w_dt, const void* Wv, mova_dtype wv_dt, int T,
                           int d, int E, int k, int n, void* v, void* ws, size_t ws_bytes,
                           mova_path path, void* const* events, void* stream) {
-  const mova_options o{path, events, 0, 0, 0};
+  const mova_options o{path, events, 0, 0, 0, nullptr};
   return mova_value_opts(x, x_dt, idx, idx_dt, wgt, w_dt, Wv, wv_dt, T, d, E, k, n, v, ws, ws_bytes, &o,
                          stream);
 }
@@ -413,7 +425,7 @@ mova_status mova_value_routed_opts(const void* x, mova_dtype x_dt, const float* 
   if (err == cudaSuccess) {
     if (tc_router)
       err = launch_router_tc(x, Wr, br, T, d, E, k, scale, o.partitions, idx, wgt, w.tile_counts, w.planes,
-                             w.sb, s);
+                             static_cast<const __nv_bfloat16*>(o.planes), w.sb, s);
     else
       err = launch_router(x, x_dt, Wr, br, T, d, E, k, scale, idx, wgt, &g, &grouped, o.partitions, s);
   }
@@ -442,7 +454,7 @@ mova_status mova_value_routed_ex(const void* x, mova_dtype x_dt, const float* Wr
                                  int n, float scale, void* v, int32_t* idx_out, float* w_out,
                                  void* ws, size_t ws_bytes, mova_path path, void* const* events,
                                  void* stream) {
-  const mova_options o{path, events, 0, 0, 0};
+  const mova_options o{path, events, 0, 0, 0, nullptr};
   return mova_value_routed_opts(x, x_dt, Wr, br, Wv, wv_dt, T, d, E, k, n, scale, v, idx_out, w_out, ws,
                                 ws_bytes, &o, stream);
 }

@@ -321,16 +321,25 @@ using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, 
 
 size_t router_planes_bytes(int d) { return static_cast<size_t>(RN) * d * 2; }
 
+cudaError_t launch_split_router(const float* Wr, int E, int d, __nv_bfloat16* planes, cudaStream_t stream) {
+  const int split_blocks = (64 * d / 8 + 256 * kSplitPer - 1) / (256 * kSplitPer);
+  return launch_pdl(split_router_kernel, dim3(split_blocks), dim3(256), 0, stream, Wr, E, d, planes);
+}
+
 cudaError_t launch_router_tc(const void* x, const float* Wr, const float* br, int T, int d, int E,
                              int k, float scale, int partitions, int32_t* idx, float* w,
-                             int32_t* tile_counts, __nv_bfloat16* planes, StatusBlock* sb,
-                             cudaStream_t stream) {
+                             int32_t* tile_counts, __nv_bfloat16* planes, const __nv_bfloat16* prepared,
+                             StatusBlock* sb, cudaStream_t stream) {
   void* fp = encode_tiled_fn();
   if (fp == nullptr) return cudaErrorNotSupported;
   EncodeTiled enc = reinterpret_cast<EncodeTiled>(fp);
-  const int split_blocks = (64 * d / 8 + 256 * kSplitPer - 1) / (256 * kSplitPer);
-  cudaError_t err = launch_pdl(split_router_kernel, dim3(split_blocks), dim3(256), 0, stream, Wr, E, d, planes);
-  if (err != cudaSuccess) return err;
+  cudaError_t err = cudaSuccess;
+  if (prepared == nullptr) {
+    err = launch_split_router(Wr, E, d, planes, stream);
+    if (err != cudaSuccess) return err;
+  } else {
+    planes = const_cast<__nv_bfloat16*>(prepared);
+  }
   CUtensorMap tx, tw;
   const cuuint64_t xdim[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(T)};
   const cuuint64_t wdim[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(RN)};

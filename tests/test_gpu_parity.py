@@ -331,6 +331,26 @@ def test_tensor_router_and_tile_grouping(api, T, d, E, k):
     _full(api, T, d, E, k, 256, "bf16", seed=T, path="stream")
 
 
+@pytest.mark.parametrize("E,d", [(64, 2560), (17, 512)])
+def test_router_planes_prepared(api, E, d):
+    """mova_router_planes: the three bf16 planes sum exactly to the fp32 router
+    weight (every plane's rows past E zero), and a call handed the prepared
+    planes routes and computes bit for bit what a call that splits the
+    weight itself does."""
+    lay = _layer(41, d, E, 256, "bf16")
+    Wr = P.dev(lay.Wr, "f32")
+    planes = api.router_planes(Wr)
+    torch.cuda.synchronize()
+    pl = planes[: 3 * 64 * d].view(3, 64, d).double().cpu().numpy()
+    assert np.array_equal(pl[0, :E] + pl[1, :E] + pl[2, :E], lay.Wr.astype(np.float32).astype(np.float64))
+    assert not pl[:, E:].any()
+    bat = MI.make_batch(300, 42, dtype="bf16", d=d)
+    args = (P.dev(bat.x, "bf16"), Wr, P.dev(lay.br, "f32"), P.dev(lay.Wv, "bf16"), 4, 2.5)
+    v0, i0, w0 = api.value_routed(*args, return_routing=True)
+    v1, i1, w1 = api.value_routed(*args, return_routing=True, planes=planes)
+    assert torch.equal(i0, i1) and torch.equal(w0, w1) and torch.equal(v0, v1)
+
+
 def test_bounded_wait_reports_timeout(api):
     """A device wait that can never complete gives up after its limit and
     reports MOVA_ERR_TIMEOUT; the context stays usable for a normal call."""
