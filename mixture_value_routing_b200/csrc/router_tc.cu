@@ -18,11 +18,13 @@
 //     plane tile (128-byte swizzle) through 7 stages of 28 KB, so a CTA
 //     streams 30% fewer bytes than with all plane rows in every CTA; the even
 //     CTA issues tcgen05.mma.cta_group::2 (M = 256 tokens, N = 192, K = 16),
-//     which accumulates each CTA's 128 tokens in its own tensor memory.  Four
-//     epilogue warps per CTA read one token per thread (all 192 columns),
-//     form the 64 logits, the sigmoid scores and the biased selection in
-//     registers and write idx / w, plus the 128-token tile's expert histogram
-//     for the grouping.
+//     which accumulates each CTA's 128 tokens in its own tensor memory.
+//     Sixteen epilogue warps per CTA, four per 32-token lane quarter, each
+//     over 16 experts: a thread forms its token's 16 logits, sigmoid scores
+//     and the top k of those 16 in registers; one thread per token then
+//     merges the four lists and writes idx / w, plus the 128-token tile's
+//     expert histogram for the grouping.  (With one thread per token over
+//     all 64 experts, the epilogue took twice as long as the main loop.)
 // Every wait is bounded (MOVA_ERR_TIMEOUT, then drain and free).
 #include <cuda.h>
 
@@ -41,7 +43,7 @@ constexpr int kRStages = 7;
 constexpr int kRABytes = RM * RK * 2;
 constexpr int kRBBytes = (RN / 2) * RK * 2;
 constexpr int kRStageBytes = kRABytes + kRBBytes;
-constexpr int kRThreads = 6 * 32;  // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
+constexpr int kRThreads = 18 * 32;  // warp 0 TMA, warp 1 MMA, warps 2-17 epilogue
 constexpr uint32_t kRTmemCols = 256;
 
 struct __align__(1024) RSmem {
@@ -111,7 +113,9 @@ split_router_kernel(const float* __restrict__ Wr, int E, int d, __nv_bfloat16* _
   }
 }
 
-__global__ void __launch_bounds__(kRThreads, 1)
+// 18 warps: sub-partitions 0 and 1 hold five warps each, so at most
+// 16384 / (5 * 32) -> 96 registers per thread.
+__global__ void __maxnreg__(96)
 router_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
                  const float* __restrict__ br, int T, int d, int E, int k, float scale,
                  int32_t* __restrict__ idx_out, float* __restrict__ w_out,
@@ -220,81 +224,129 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_consta
       __syncwarp();
     }
   } else {
-    // Epilogue: thread = token (TMEM lane of this CTA).
-    const int lg = warp & 3;
-    const int t = t0 + lg * 32 + lane;
+    // Epilogue: warp w reads TMEM lanes 32 * (w % 4) .. +31 (tokens) and the
+    // hi / mid / lo columns of experts 16 g .. 16 g + 15, g = (w - 2) / 4:
+    // the warps of one lane quarter split the 64 experts four ways.  Each
+    // thread forms its 16 logits and scores and the top k of its 16 experts
+    // in the selection order (highest biased score first, ties to the lower
+    // index); then one thread per token merges the four lists.
+    const int q = warp & 3;
+    const int g = (warp - 2) >> 2;
+    const int tl = q * 32 + lane;  // token within the CTA
+    // Candidate lists in the (drained) stage ring: [group][rank][token].
+    float* cb = reinterpret_cast<float*>(S.stage[0]);
+    float* cs = cb + 4 * 8 * RM;
+    int* ce = reinterpret_cast<int*>(cs + 4 * 8 * RM);
     if (mbar_wait(&S.tmem_full, 0)) {
       tc_fence_after();
-      const uint32_t tb = S.tmem_base + (static_cast<uint32_t>(lg * 32) << 16);
-      float logit[64];
-#pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        uint32_t hi[32], mid[32], lo[32];
-        tmem_ld_32(tb + c * 32, hi);
-        tmem_ld_32(tb + 64 + c * 32, mid);
-        tmem_ld_32(tb + 128 + c * 32, lo);
+      const uint32_t tb = S.tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(g * 16);
+      float sc[16];
+      {
+        uint32_t hi[16], mid[16], lo[16];
+        tmem_ld_16(tb, hi);
+        tmem_ld_16(tb + 64, mid);
+        tmem_ld_16(tb + 128, lo);
         tmem_ld_wait();
 #pragma unroll
-        for (int j = 0; j < 32; ++j)
-          logit[c * 32 + j] = (__uint_as_float(hi[j]) + __uint_as_float(mid[j])) + __uint_as_float(lo[j]);
+        for (int j = 0; j < 16; ++j)
+          sc[j] = (__uint_as_float(hi[j]) + __uint_as_float(mid[j])) + __uint_as_float(lo[j]);
         if (parts == 2) {
           // Second partition: its own fp32 partial, added after the first.
-          tmem_ld_32(tb + kRTmemCols + c * 32, hi);
-          tmem_ld_32(tb + kRTmemCols + 64 + c * 32, mid);
-          tmem_ld_32(tb + kRTmemCols + 128 + c * 32, lo);
+          tmem_ld_16(tb + kRTmemCols, hi);
+          tmem_ld_16(tb + kRTmemCols + 64, mid);
+          tmem_ld_16(tb + kRTmemCols + 128, lo);
           tmem_ld_wait();
 #pragma unroll
-          for (int j = 0; j < 32; ++j)
-            logit[c * 32 + j] +=
-                (__uint_as_float(hi[j]) + __uint_as_float(mid[j])) + __uint_as_float(lo[j]);
+          for (int j = 0; j < 16; ++j)
+            sc[j] += (__uint_as_float(hi[j]) + __uint_as_float(mid[j])) + __uint_as_float(lo[j]);
         }
       }
       tc_fence_before();
-      if (t < T) {
-        // Sigmoid scores (in place); the biased score s + br steers the
-        // selection only, NaN never wins.
+      // Sigmoid scores (in place); the biased score s + br steers the
+      // selection only, NaN never wins.
+      float bs[16];
 #pragma unroll
-        for (int e = 0; e < 64; ++e) logit[e] = sigmoidf_(logit[e]);
-        uint64_t taken = 0;
-        float ssum = 0.f;
-        int sel[8];
-        float ssel[8];
+      for (int j = 0; j < 16; ++j) {
+        sc[j] = sigmoidf_(sc[j]);
+        const float b = sc[j] + S.br[g * 16 + j];
+        bs[j] = b == b ? b : -INFINITY;
+      }
+      const int live = min(max(E - g * 16, 0), 16);  // this group's experts below E
+      uint32_t taken = 0;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          if (j < k) {
-            // Highest biased score among live experts; ties to the lower
-            // index (strict comparison in ascending expert order).
-            int be = -1;
-            float bb = 0.f, bsv = 0.f;
+      for (int r = 0; r < 8; ++r) {
+        if (r < k && r < live) {
+          int be = -1;
+          float bb = 0.f, bsv = 0.f;
 #pragma unroll
-            for (int e = 0; e < 64; ++e) {
-              float b = logit[e] + S.br[e];
-              if (!(b == b)) b = -INFINITY;
-              const bool live = e < E && !((taken >> e) & 1ull);
-              if (live && (be < 0 || b > bb)) {
-                be = e;
-                bb = b;
-                bsv = logit[e];
-              }
+          for (int j = 0; j < 16; ++j) {
+            if (j < live && !((taken >> j) & 1u) && (be < 0 || bs[j] > bb)) {
+              be = j;
+              bb = bs[j];
+              bsv = sc[j];
             }
-            taken |= 1ull << be;
-            sel[j] = be;
-            ssel[j] = bsv;
-            ssum += bsv;
           }
-        }
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          if (j < k) {
-            idx_out[static_cast<size_t>(t) * k + j] = sel[j];
-            w_out[static_cast<size_t>(t) * k + j] = scale * ssel[j] / ssum;
-            atomicAdd(&S.hist[sel[j]], 1);
-          }
+          taken |= 1u << be;
+          const int o = (g * 8 + r) * RM + tl;
+          cb[o] = bb;
+          cs[o] = bsv;
+          ce[o] = g * 16 + be;
         }
       }
     } else {
       raise_status(sb, MOVA_ERR_TIMEOUT, blockIdx.x);
       S.abort = 1;
+    }
+    asm volatile("bar.sync 1, 512;" ::: "memory");  // the 16 epilogue warps: every list is written
+    const int t = t0 + tl;
+    if (g == 0 && t < T && !*reinterpret_cast<volatile int*>(&S.abort)) {
+      // Merge: repeatedly take the best head of the four lists (strictly
+      // greater biased score; equal scores keep the lower group, i.e. the
+      // lower expert index, as the lists are in ascending expert ranges).
+      int nlen[4], head[4];
+#pragma unroll
+      for (int gg = 0; gg < 4; ++gg) {
+        nlen[gg] = min(k, min(max(E - gg * 16, 0), 16));
+        head[gg] = 0;
+      }
+      int sel[8];
+      float ssel[8];
+      float ssum = 0.f;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        if (j < k) {
+          int bg = -1;
+          float bb = 0.f;
+#pragma unroll
+          for (int gg = 0; gg < 4; ++gg) {
+            if (head[gg] < nlen[gg]) {
+              const float b = cb[(gg * 8 + head[gg]) * RM + tl];
+              if (bg < 0 || b > bb) {
+                bg = gg;
+                bb = b;
+              }
+            }
+          }
+          int o = 0;
+#pragma unroll
+          for (int gg = 0; gg < 4; ++gg)
+            if (gg == bg) {
+              o = (gg * 8 + head[gg]) * RM + tl;
+              ++head[gg];
+            }
+          sel[j] = ce[o];
+          ssel[j] = cs[o];
+          ssum += ssel[j];
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        if (j < k) {
+          idx_out[static_cast<size_t>(t) * k + j] = sel[j];
+          w_out[static_cast<size_t>(t) * k + j] = scale * ssel[j] / ssum;
+          atomicAdd(&S.hist[sel[j]], 1);
+        }
+      }
     }
   }
   __syncthreads();
