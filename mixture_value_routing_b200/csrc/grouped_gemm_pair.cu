@@ -83,9 +83,6 @@ struct __align__(1024) PSmem {
   int act_off[64];
   int act_ntt[64];
   int tile_base[65];
-  // Scratch of the ordering: the active experts in ascending order.
-  int raw_e[64];
-  int raw_cnt[64];
 };
 
 struct PTile {
@@ -159,7 +156,7 @@ constexpr int kAcc1Rows = NA / 2;               // accumulator 1's rows start he
 __global__ void __launch_bounds__(kPThreads, 1)
 grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_xp,
                          const int32_t* __restrict__ counts, const int32_t* __restrict__ offsets,
-                         const int32_t* __restrict__ active, StatusBlock* __restrict__ sb, int d, int n,
+                         int E, StatusBlock* __restrict__ sb, int d, int n,
                          int ldw, __nv_bfloat16* __restrict__ P) {
   extern __shared__ uint8_t smem_raw[];
   PSmem& S = *reinterpret_cast<PSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -188,29 +185,33 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_w, const __gri
   }
   pdl_wait();  // the grouping of this call is complete and visible
   if (threadIdx.x < 32) {
-    // Active experts, then their order by pair count (descending; equal
-    // counts keep ascending expert order), then the tile prefix.
-    const int nact = sb->num_active;
-    for (int a = lane; a < 64; a += 32) {
-      if (a < nact) {
-        const int e = active[a];
-        S.raw_e[a] = e;
-        S.raw_cnt[a] = counts[e];
-      }
+    // The active experts (count > 0) ordered by pair count, descending
+    // (equal counts keep ascending expert order), then the tile prefix.
+    // Lane l holds experts l and l + 32; all four reads go out at once.
+    const int e0 = lane, e1 = lane + 32;
+    const int c0 = e0 < E ? counts[e0] : 0;
+    const int c1 = e1 < E ? counts[e1] : 0;
+    const int f0 = e0 < E ? offsets[e0] : 0;
+    const int f1 = e1 < E ? offsets[e1] : 0;
+    int r0 = 0, r1 = 0;  // experts ahead of e0 / e1 in that order
+    for (int b = 0; b < 32; ++b) {
+      const int x0 = __shfl_sync(0xffffffffu, c0, b);  // count of expert b
+      const int x1 = __shfl_sync(0xffffffffu, c1, b);  // count of expert b + 32
+      r0 += (x0 > c0 || (x0 == c0 && b < lane)) + (x1 > c0);
+      r1 += (x0 >= c1) + (x1 > c1 || (x1 == c1 && b < lane));
     }
-    __syncwarp();
-    for (int a = lane; a < nact; a += 32) {
-      const int c = S.raw_cnt[a];
-      int rk = 0;
-      for (int b = 0; b < nact; ++b) {
-        const int cb = S.raw_cnt[b];
-        rk += (cb > c || (cb == c && b < a)) ? 1 : 0;
-      }
-      const int e = S.raw_e[a];
-      S.act_e[rk] = e;
-      S.act_cnt[rk] = c;
-      S.act_off[rk] = offsets[e];
-      S.act_ntt[rk] = (c + NT - 1) / NT;
+    const int nact = __popc(__ballot_sync(0xffffffffu, c0 > 0)) + __popc(__ballot_sync(0xffffffffu, c1 > 0));
+    if (c0 > 0) {
+      S.act_e[r0] = e0;
+      S.act_cnt[r0] = c0;
+      S.act_off[r0] = f0;
+      S.act_ntt[r0] = (c0 + NT - 1) / NT;
+    }
+    if (c1 > 0) {
+      S.act_e[r1] = e1;
+      S.act_cnt[r1] = c1;
+      S.act_off[r1] = f1;
+      S.act_ntt[r1] = (c1 + NT - 1) / NT;
     }
     __syncwarp();
     const int a0 = lane, a1 = lane + 32;
@@ -246,15 +247,17 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_w, const __gri
     int s = 0;
     uint32_t phase = 0;
     bool started = false;
-    int next = 0;
-    if (rank == 0) {
-      if (lane == 0) next = atomicAdd(&sb->work_next, 1);
-      next = __shfl_sync(0xffffffffu, next, 0);
-    }
+    // Cluster c takes tile c first, then ids ncl + (counter value).  Lane 0
+    // fetches the next id one tile ahead, so the atomic's round trip never
+    // holds up a tile's first copies.
+    const int ncl = static_cast<int>(gridDim.x) / 2;
+    int nraw = 0;
+    if (rank == 0 && lane == 0) nraw = ncl + atomicAdd(&sb->work_next, 1);
     for (int i = 0;; ++i) {
       int t;
       if (rank == 0) {
-        t = p_aborted(S) ? ntiles : next;
+        const int nxt = i == 0 ? static_cast<int>(blockIdx.x) / 2 : __shfl_sync(0xffffffffu, nraw, 0);
+        t = p_aborted(S) ? ntiles : nxt;
         if (elect_one()) {
           const int slot = i % kTileRing;
           S.tq[slot] = t;
@@ -264,8 +267,7 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_w, const __gri
         }
         __syncwarp();
         if (t >= ntiles) break;
-        if (lane == 0) next = atomicAdd(&sb->work_next, 1);  // read back at the next tile
-        next = __shfl_sync(0xffffffffu, next, 0);
+        if (i > 0 && lane == 0) nraw = ncl + atomicAdd(&sb->work_next, 1);  // read at the next tile
       } else {
         t = next_tile(S, i);
         if (t < 0) {
@@ -488,7 +490,7 @@ using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, 
 }  // namespace
 
 cudaError_t launch_tensor_experts_pair(const void* Wv, long long ldw, const int32_t* counts,
-                                       const int32_t* offsets, const int32_t* active, StatusBlock* sb, int T,
+                                       const int32_t* offsets, StatusBlock* sb, int T,
                                        int d, int n, int k, int E, const __nv_bfloat16* xp, __nv_bfloat16* P,
                                        cudaStream_t stream) {
   void* fp = encode_tiled_fn();
@@ -542,7 +544,7 @@ cudaError_t launch_tensor_experts_pair(const void* Wv, long long ldw, const int3
   }
   cfg.gridDim = dim3(2 * max_clusters);
   note_launch();
-  return cudaLaunchKernelEx(&cfg, grouped_gemm_pair_kernel, tmap_w, tmap_xp, counts, offsets, active, sb, d, n,
+  return cudaLaunchKernelEx(&cfg, grouped_gemm_pair_kernel, tmap_w, tmap_xp, counts, offsets, E, sb, d, n,
                             static_cast<int>(ldw), P);
 }
 

@@ -210,7 +210,7 @@ cudaError_t launch_gather_pairs(const void* x, const int32_t* perm, int T, int d
 // token rows already gathered into grouped order (xp, launch_gather_pairs);
 // tiles of up to 512 pairs on two accumulators.
 cudaError_t launch_tensor_experts_pair(const void* Wv, long long ldw, const int32_t* counts,
-                                       const int32_t* offsets, const int32_t* active, StatusBlock* sb, int T,
+                                       const int32_t* offsets, StatusBlock* sb, int T,
                                        int d, int n, int k, int E, const __nv_bfloat16* xp, __nv_bfloat16* P,
                                        cudaStream_t stream);
 

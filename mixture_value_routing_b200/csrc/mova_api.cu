@@ -190,7 +190,7 @@ mova_status run_experts_and_combine(const void* x, mova_dtype dt, const void* Wv
   if (err != cudaSuccess) return from_cuda(err);
   if (tensor) {
     if (pair) {
-      err = launch_tensor_experts_pair(Wv, ldw, ws.counts, ws.offsets, ws.active, ws.sb, T, d, n, k, E, ws.xp,
+      err = launch_tensor_experts_pair(Wv, ldw, ws.counts, ws.offsets, ws.sb, T, d, n, k, E, ws.xp,
                                        static_cast<__nv_bfloat16*>(ws.P), stream);
     } else {
       err = launch_tensor_experts(x, Wv, ldw, ws.counts, ws.offsets, ws.perm, w32, ws.active, ws.sb, T,
