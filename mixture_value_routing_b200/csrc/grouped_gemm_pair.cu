@@ -83,6 +83,9 @@ struct __align__(1024) PSmem {
   int act_off[64];
   int act_ntt[64];
   int tile_base[65];
+  // Per epilogue warp: a 32 x 32 bf16 block transposed for the P stores
+  // (column-major, rows paired into 32-bit words).
+  alignas(16) uint32_t epi[kEpiWarps][32 * 16];  // read as 16-byte vectors
 };
 
 struct PTile {
@@ -153,7 +156,9 @@ __device__ __forceinline__ void p_fail(PSmem& S, StatusBlock* sb) {
 constexpr int kBoxRows = 32;                    // token rows per TMA box
 constexpr int kAcc1Rows = NA / 2;               // accumulator 1's rows start here in B
 
-__global__ void __launch_bounds__(kPThreads, 1)
+// Ten warps: sub-partitions 0 and 1 hold three each, so at most
+// 16384 / (3 * 32) -> 168 registers per thread.
+__global__ void __maxnreg__(168)
 grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_xp,
                          const int32_t* __restrict__ counts, const int32_t* __restrict__ offsets,
                          int E, StatusBlock* __restrict__ sb, int d, int n,
@@ -426,9 +431,13 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_w, const __gri
       // MMA, and the second half is stored.  (Three of the ten warps share a
       // sub-partition's 16K registers, so a thread cannot hold all 256
       // columns at once.)
-      unsigned short* prow =
-          reinterpret_cast<unsigned short*>(P + static_cast<size_t>(tl.off + tl.tok0 + j0) * n + rloc);
-      const bool live = rloc < n;
+      // The warp's 32 weight rows are all below n or all at or above it (n
+      // is a multiple of 128).  Lane l stores rows rbase + 8 (l % 4) ..
+      // + 7 of a pair's P row as one 16-byte vector.
+      const int rbase = rloc - lane;
+      const bool live = rbase < n;
+      uint32_t* Tw = S.epi[warp - 2];
+      __nv_bfloat16* pseg = P + static_cast<size_t>(tl.off + tl.tok0 + j0) * n + rbase + (lane & 3) * 8;
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         uint32_t pk[4][16];
@@ -455,14 +464,27 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_w, const __gri
         if (live) {
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
+            const int cb = (4 * h + c) * 32;  // the block's first column (pair)
+            if (cb < nvalid) {
+              // Transpose the 32 rows x 32 columns block through shared
+              // memory: lanes 2i and 2i + 1 pair their rows into one word
+              // per column (even lane: column 2j, odd lane: column 2j + 1).
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              const int col = (4 * h + c) * 32 + j;
-              if (col < nvalid) {
-                const uint32_t wv = pk[c][j >> 1];
-                prow[static_cast<size_t>(col) * n] =
-                    static_cast<unsigned short>((j & 1) ? (wv >> 16) : (wv & 0xFFFFu));
+              for (int j = 0; j < 16; ++j) {
+                const uint32_t mine = pk[c][j];
+                const uint32_t other = __shfl_xor_sync(0xffffffffu, mine, 1);
+                const uint32_t w = (lane & 1) ? __byte_perm(other, mine, 0x7632) : __byte_perm(mine, other, 0x5410);
+                Tw[(2 * j + (lane & 1)) * 16 + (lane >> 1)] = w;
               }
+              __syncwarp();
+#pragma unroll
+              for (int it = 0; it < 4; ++it) {
+                const int cc = it * 8 + (lane >> 2);
+                if (cb + cc < nvalid)
+                  *reinterpret_cast<uint4*>(pseg + static_cast<size_t>(cb + cc) * n) =
+                      *reinterpret_cast<const uint4*>(&Tw[cc * 16 + (lane & 3) * 4]);
+              }
+              __syncwarp();
             }
           }
         }
