@@ -93,8 +93,13 @@ struct PTile {
 };
 
 __device__ __forceinline__ PTile decode_ptile(const PSmem& S, int t, int mtiles) {
-  int a = 0;
-  while (a + 1 < S.nact && S.tile_base[a + 1] <= t) ++a;
+  // The expert of tile t: the last a with tile_base[a] <= t (tile_base is
+  // strictly increasing over the active experts).
+  int a = 0, hi = S.nact - 1;
+  while (a < hi) {
+    const int mid = (a + hi + 1) >> 1;
+    if (S.tile_base[mid] <= t) a = mid; else hi = mid - 1;
+  }
   const int local = t - S.tile_base[a];
   const int tt = local / mtiles;
   const int cnt = S.act_cnt[a];
