@@ -254,6 +254,10 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_w, const __gri
     // producer takes the tile ids from the global counter (zeroed by this
     // call's grouping) and publishes each to both CTAs.
     const uint32_t full0_cl = mapa_shared(smem_u32(&S.full[0]), 0);  // even CTA's barriers
+    // Weights stream through once per tile: evict them first, so the
+    // gathered token rows (stored evict-last) stay in L2 for the four
+    // weight-row blocks that read them.
+    const uint64_t wpol = policy_evict_first();
     int s = 0;
     uint32_t phase = 0;
     bool started = false;
@@ -312,7 +316,7 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_w, const __gri
         uint8_t* st = S.stage[s];
         if (elect_one()) {
           if (rank == 0) mbar_arrive_expect_tx(&S.full[s], bytes);
-          tma_load_2d_pair(st, &tmap_w, kb * PK, arow, full_cl);
+          tma_load_2d_pair_hint(st, &tmap_w, kb * PK, arow, full_cl, wpol);
           uint8_t* bt = st + kPABytes;
           for (int b = 0; b < nb0; ++b)
             tma_load_2d_pair(bt + b * kBoxRows * 128, &tmap_xp, kb * PK, row0 + b * kBoxRows, full_cl);

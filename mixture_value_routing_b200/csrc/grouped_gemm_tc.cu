@@ -278,13 +278,22 @@ __global__ void __launch_bounds__(256)
 gather_pairs_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ perm, int k, int vec_per_row,
                     int N, uint4* __restrict__ xp) {
   pdl_wait();
+  // Evict-last: the rows are read again by the GEMM right after (once per
+  // 256-row weight block), while the weights stream through L2 evict-first.
+  // The same workspace rows are rewritten by every call.
+  const uint64_t pol = policy_evict_last();
   const int lane = threadIdx.x & 31;
   const long long gw = (static_cast<long long>(blockIdx.x) * 256 + threadIdx.x) >> 5;
   const long long nw = (static_cast<long long>(gridDim.x) * 256) >> 5;
   for (long long p = gw; p < N; p += nw) {
     const uint4* src = x + static_cast<size_t>(perm[p] / k) * vec_per_row;
     uint4* dst = xp + static_cast<size_t>(p) * vec_per_row;
-    for (int v = lane; v < vec_per_row; v += 32) dst[v] = src[v];
+    for (int v = lane; v < vec_per_row; v += 32) {
+      const uint4 q = src[v];
+      asm volatile("st.global.L2::cache_hint.v4.u32 [%0], {%1, %2, %3, %4}, %5;" ::"l"(dst + v), "r"(q.x),
+                   "r"(q.y), "r"(q.z), "r"(q.w), "l"(pol)
+                   : "memory");
+    }
   }
 }
 
