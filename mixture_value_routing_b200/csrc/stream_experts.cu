@@ -291,6 +291,8 @@ stream_experts_kernel(const DT* __restrict__ x, const DT* __restrict__ Wv,
   __shared__ int r_scratch[128];
   __shared__ int32_t r_cnt[64], r_off[65], r_pos[64], r_perm[64];
   __shared__ int r_nact;
+  __shared__ int p_act[64];  // the producer's own copy of the active list (route mode)
+  int p_nact = 0;
   const bool routing = route.part != nullptr;
   if (routing) {
     if (threadIdx.x < kConsumerWarps * 32) {
@@ -321,6 +323,9 @@ stream_experts_kernel(const DT* __restrict__ x, const DT* __restrict__ Wv,
         select_token(&r_lg[warp * 64], r_br, route.E, k, route.scale, warp, lane, r_sel, r_w,
                      blockIdx.x == 0 ? route.idx_out : nullptr, route.w_out);
       consumers_sync();
+      // The selection is complete: the producer warp may derive the active
+      // experts and start the weight stream while warp 0 groups the pairs.
+      asm volatile("bar.arrive 3, %0;" ::"n"((kConsumerWarps + 1) * 32) : "memory");
       if (warp == 0) {
         const int na = group_pairs_warp(r_sel, T * k, route.E, lane, r_scratch, r_cnt, r_off, r_pos,
                                         r_perm, act);
@@ -345,12 +350,33 @@ stream_experts_kernel(const DT* __restrict__ x, const DT* __restrict__ Wv,
         }
       }
     }
+    if (warp == kProducerWarp) {
+      // The active experts (ascending), from the selection alone: the same
+      // list the grouping builds.
+      asm volatile("bar.sync 3, %0;" ::"n"((kConsumerWarps + 1) * 32) : "memory");
+      uint64_t m = 0;
+      for (int i = lane; i < T * k; i += 32) m |= 1ull << r_sel[i];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) m |= __shfl_xor_sync(0xffffffffu, m, o);
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int e = lane + 32 * h;
+        if ((m >> e) & 1ull) p_act[__popcll(m & ((1ull << e) - 1ull))] = e;
+      }
+      p_nact = __popcll(m);
+      __syncwarp();
+    }
   } else {
     const int na = sb->num_active;
     if (threadIdx.x < 64) act[threadIdx.x] = (threadIdx.x < na) ? active[threadIdx.x] : 0;
   }
-  __syncthreads();
-  const int nact = routing ? r_nact : sb->num_active;
+  // Route mode: the producer goes ahead; the other warps wait for the grouping.
+  if (!routing)
+    __syncthreads();
+  else if (warp != kProducerWarp)
+    asm volatile("bar.sync 4, %0;" ::"n"((kConsumerWarps + 1) * 32) : "memory");
+  const int nact = routing ? (warp == kProducerWarp ? p_nact : r_nact) : sb->num_active;
+  const int* act_p = routing && warp == kProducerWarp ? p_act : act;
   pdl_trigger();
 
   // Rows of all active experts, in units of whole stages (n % 8 == 0, so a
@@ -391,7 +417,7 @@ stream_experts_kernel(const DT* __restrict__ x, const DT* __restrict__ Wv,
       // Test-only injection: CTA 0 stops issuing here, so the consumers'
       // wait for this stage must run out.
       if (j == fault.stall_stage && blockIdx.x == 0) break;
-      const DT* src = Wv + (static_cast<size_t>(act[a]) * ldw + rb * kRowsPerStage) * d;
+      const DT* src = Wv + (static_cast<size_t>(act_p[a]) * ldw + rb * kRowsPerStage) * d;
       uint8_t* dst = stages + s * stage_bytes;
       if (lane == 0) mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(kRowsPerStage * row_bytes));
       __syncwarp();
