@@ -14,7 +14,7 @@
 // tail waste is below 16 columns per tile.
 //
 // First, gather_pairs_kernel copies each pair's x row into grouped order
-// (xp[p] = x[token of pair p]), one bandwidth-bound pass, so that every
+// (xp[pos of pair (t, j)] = x[t], token-major), one bandwidth-bound pass, so that every
 // token tile of the GEMM is a run of consecutive rows that TMA loads as
 // plain 2-D boxes (token rows are read n/128 times, from L2, by TMA instead
 // of 16-byte gathers through the load/store units).
@@ -272,11 +272,14 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_con
   }
 }
 
-// xp[p, :] = x[perm[p] / k, :] for every pair p: one warp per row, 16-byte
-// vectors (HBM/L2-bound copy).
+// xp[pos[t * k + j], :] = x[t, :] for every token t and slot j: one warp
+// per token reads its row once (16-byte vectors, up to 8 per lane at a
+// time) and writes it to the token's k grouped positions.  Token-major, so
+// x is read once however large it is (in pair order each row would be read
+// k times, from DRAM once x outgrows L2).  HBM-bound copy.
 __global__ void __launch_bounds__(256)
-gather_pairs_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ perm, int k, int vec_per_row,
-                    int N, uint4* __restrict__ xp) {
+gather_pairs_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ pos, int k, int vec_per_row,
+                    int T, uint4* __restrict__ xp) {
   pdl_wait();
   // Evict-last: the rows are read again by the GEMM right after (once per
   // 256-row weight block), while the weights stream through L2 evict-first.
@@ -285,14 +288,28 @@ gather_pairs_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ per
   const int lane = threadIdx.x & 31;
   const long long gw = (static_cast<long long>(blockIdx.x) * 256 + threadIdx.x) >> 5;
   const long long nw = (static_cast<long long>(gridDim.x) * 256) >> 5;
-  for (long long p = gw; p < N; p += nw) {
-    const uint4* src = x + static_cast<size_t>(perm[p] / k) * vec_per_row;
-    uint4* dst = xp + static_cast<size_t>(p) * vec_per_row;
-    for (int v = lane; v < vec_per_row; v += 32) {
-      const uint4 q = src[v];
-      asm volatile("st.global.L2::cache_hint.v4.u32 [%0], {%1, %2, %3, %4}, %5;" ::"l"(dst + v), "r"(q.x),
-                   "r"(q.y), "r"(q.z), "r"(q.w), "l"(pol)
-                   : "memory");
+  for (long long t = gw; t < T; t += nw) {
+    const uint4* src = x + static_cast<size_t>(t) * vec_per_row;
+    int p = 0;
+    if (lane < k) p = pos[static_cast<size_t>(t) * k + lane];
+    for (int v0 = 0; v0 < vec_per_row; v0 += 32 * 8) {
+      uint4 q[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int v = v0 + i * 32 + lane;
+        if (v < vec_per_row) q[i] = src[v];
+      }
+      for (int j = 0; j < k; ++j) {
+        uint4* dst = xp + static_cast<size_t>(__shfl_sync(0xffffffffu, p, j)) * vec_per_row;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int v = v0 + i * 32 + lane;
+          if (v < vec_per_row)
+            asm volatile("st.global.L2::cache_hint.v4.u32 [%0], {%1, %2, %3, %4}, %5;" ::"l"(dst + v),
+                         "r"(q[i].x), "r"(q[i].y), "r"(q[i].z), "r"(q[i].w), "l"(pol)
+                         : "memory");
+        }
+      }
     }
   }
 }
@@ -306,19 +323,18 @@ using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, 
 
 size_t tensor_experts_smem() { return sizeof(Smem) + 1024; }
 
-cudaError_t launch_gather_pairs(const void* x, const int32_t* perm, int T, int d, int k,
+cudaError_t launch_gather_pairs(const void* x, const int32_t* pos, int T, int d, int k,
                                 __nv_bfloat16* xp, cudaStream_t stream) {
-  const int N = T * k;
   const int vec_per_row = d / 8;
-  long long blocks = (static_cast<long long>(N) * 32 + 255) / 256;
+  long long blocks = (static_cast<long long>(T) * 32 + 255) / 256;
   const long long cap = static_cast<long long>(sm_count()) * 8;
   if (blocks > cap) blocks = cap;
   return launch_pdl(gather_pairs_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, stream,
-                    static_cast<const uint4*>(x), perm, k, vec_per_row, N, reinterpret_cast<uint4*>(xp));
+                    static_cast<const uint4*>(x), pos, k, vec_per_row, T, reinterpret_cast<uint4*>(xp));
 }
 
 cudaError_t launch_tensor_experts(const void* x, const void* Wv, long long ldw, const int32_t* counts,
-                                  const int32_t* offsets, const int32_t* perm, const float* w32,
+                                  const int32_t* offsets, const int32_t* pos, const float* w32,
                                   const int32_t* active, StatusBlock* sb, int T, int d, int n, int k,
                                   int E, __nv_bfloat16* xp, __nv_bfloat16* P, cudaStream_t stream) {
   (void)w32;
@@ -327,7 +343,7 @@ cudaError_t launch_tensor_experts(const void* x, const void* Wv, long long ldw, 
   EncodeTiled enc = reinterpret_cast<EncodeTiled>(fp);
   const int N = T * k;
   // Rows of x in grouped order.
-  cudaError_t err = launch_gather_pairs(x, perm, T, d, k, xp, stream);
+  cudaError_t err = launch_gather_pairs(x, pos, T, d, k, xp, stream);
   if (err != cudaSuccess) return err;
   // The experts as one (E*n) x d row-major bf16 matrix; boxes of 128 rows x
   // 64 columns (128 bytes) with 128-byte swizzle.  The gathered rows: N x d,

@@ -199,12 +199,12 @@ bool stream_resident(int T, int d, mova_dtype dt);
 // tcgen05 grouped GEMM (bf16): P[p, :] = SiLU(Wv[e] x[t]) as bf16 rows.
 // xp: T*k x d bf16 scratch for the pairs' x rows in grouped order.
 cudaError_t launch_tensor_experts(const void* x, const void* Wv, long long ldw, const int32_t* counts,
-                                  const int32_t* offsets, const int32_t* perm, const float* w32,
+                                  const int32_t* offsets, const int32_t* pos, const float* w32,
                                   const int32_t* active, StatusBlock* sb, int T, int d, int n, int k,
                                   int E, __nv_bfloat16* xp, __nv_bfloat16* P, cudaStream_t stream);
 size_t tensor_experts_smem();
-// xp[p] = x[perm[p] / k] for the T*k pairs.
-cudaError_t launch_gather_pairs(const void* x, const int32_t* perm, int T, int d, int k,
+// xp[pos[t * k + j]] = x[t] for the T*k pairs (token-major: each x row read once).
+cudaError_t launch_gather_pairs(const void* x, const int32_t* pos, int T, int d, int k,
                                 __nv_bfloat16* xp, cudaStream_t stream);
 // The grouped GEMM on SM pairs (tcgen05 cta_group::2), reading the pairs'
 // token rows already gathered into grouped order (xp, launch_gather_pairs);

@@ -185,7 +185,7 @@ mova_status run_experts_and_combine(const void* x, mova_dtype dt, const void* Wv
   const bool pair = tensor && path == MOVA_PATH_TENSOR && sm_count() >= 2;
   // The pair GEMM's token rows are gathered first; the gather belongs to the
   // grouping stage, so the expert stage times the GEMM alone.
-  if (pair) err = launch_gather_pairs(x, ws.perm, T, d, k, ws.xp, stream);
+  if (pair) err = launch_gather_pairs(x, ws.pos, T, d, k, ws.xp, stream);
   if (err == cudaSuccess) err = mark(events, 2, stream);
   if (err != cudaSuccess) return from_cuda(err);
   if (tensor) {
@@ -193,7 +193,7 @@ mova_status run_experts_and_combine(const void* x, mova_dtype dt, const void* Wv
       err = launch_tensor_experts_pair(Wv, ldw, ws.counts, ws.offsets, ws.sb, T, d, n, k, E, ws.xp,
                                        static_cast<__nv_bfloat16*>(ws.P), stream);
     } else {
-      err = launch_tensor_experts(x, Wv, ldw, ws.counts, ws.offsets, ws.perm, w32, ws.active, ws.sb, T,
+      err = launch_tensor_experts(x, Wv, ldw, ws.counts, ws.offsets, ws.pos, w32, ws.active, ws.sb, T,
                                   d, n, k, E, ws.xp, static_cast<__nv_bfloat16*>(ws.P), stream);
     }
   } else {
