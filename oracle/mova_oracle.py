@@ -179,6 +179,27 @@ def as_gqa(v: np.ndarray, head_dim: int = 128) -> np.ndarray:
     return v.reshape(T, n // head_dim, head_dim)
 
 
+def attend(x: np.ndarray, idx: np.ndarray, w: np.ndarray, Wv, probs: np.ndarray,
+           wv_dtype: str = "f64", head_dim: int = 128) -> np.ndarray:
+    """The value side of one query token's attention over L cached positions
+    whose values are rematerialised from the compact cache ("IFM K2 Horizon
+    Deep Dive", Section 4, Option B: x, the top-k indices and the stored
+    weights per position; V recomputed inside attention):
+
+        V = combine(x, idx, w, Wv) viewed as (L, n / 128, 128)  (KV heads)
+        o[h] = sum over l of probs[h, l] * V[l, h // G],  G = H / (n / 128)
+
+    (query heads grouped onto KV heads as in GQA, consecutive query heads
+    sharing one).  probs: (H, L); returns o (H, head_dim) fp64."""
+    V = as_gqa(combine(x, idx, w, Wv, wv_dtype), head_dim)
+    H = probs.shape[0]
+    G = H // V.shape[1]
+    o = np.zeros((H, head_dim), dtype=np.float64)
+    for h in range(H):
+        o[h] = probs[h].astype(np.float64) @ V[:, h // G, :]
+    return o
+
+
 # ---------------------------------------------------------------------------
 # Grouping of (token, slot) pairs by expert
 # ---------------------------------------------------------------------------

@@ -376,3 +376,71 @@ def test_partitioned_logits_are_fp32_within_rounding():
     assert not (part == exact).all()  # the rounding is really there
     np.testing.assert_array_equal(O.route(x, Wr, np.zeros(8), 2, 2.5)["logits"], exact)
     np.testing.assert_array_equal(O.route(x, Wr, np.zeros(8), 2, 2.5, partitions=2)["logits"], part)
+
+
+# ---------------------------------------------------------------------------
+# Attend: the PV product over rematerialised values (Deep-dive, Section 4,
+# Option B)
+# ---------------------------------------------------------------------------
+
+
+def test_attend_brute_force_loops():
+    """attend against scalar loops written independently of combine/as_gqa:
+    every position, slot, expert row and query head summed by hand."""
+    rng = np.random.default_rng(7)
+    L, d, E, k, n, H = 3, 5, 3, 2, 256, 4  # 2 KV heads, 2 query heads each
+    x = rng.normal(size=(L, d))
+    Wv = rng.normal(size=(E, n, d)) * 0.5
+    idx = np.array([[0, 2], [1, 0], [2, 1]])
+    w = rng.uniform(0.2, 1.5, size=(L, k))
+    p = rng.uniform(size=(H, L))
+    o = O.attend(x, idx, w, Wv, p)
+    for h in range(H):
+        g = h // 2  # H / (n / 128) = 2 query heads per KV head
+        for c in range(128):
+            acc = 0.0
+            for l in range(L):
+                vl = 0.0
+                for s in range(k):
+                    hv = sum(Wv[idx[l, s], g * 128 + c, j] * x[l, j] for j in range(d))
+                    vl += w[l, s] * hv / (1.0 + math.exp(-hv))
+                acc += p[h, l] * vl
+            assert abs(o[h, c] - acc) <= 1e-12 * max(1.0, abs(acc))
+
+
+def test_attend_one_hot_reads_one_value_row():
+    """With all of a head's probability on position j, o[h] is row j of the
+    value tensor in the head's KV group; query heads 2g and 2g + 1 share KV
+    head g (a mapping h % (n/128) would swap groups and fail)."""
+    rng = np.random.default_rng(8)
+    L, d, E, k, n = 5, 6, 4, 2, 512  # 4 KV heads
+    x = rng.normal(size=(L, d))
+    Wv = rng.normal(size=(E, n, d))
+    idx = rng.integers(0, E, size=(L, k))
+    w = rng.uniform(0.1, 1.0, size=(L, k))
+    H = 8
+    p = np.zeros((H, L))
+    js = [4, 1, 3, 0, 2, 2, 1, 4]
+    for h, j in enumerate(js):
+        p[h, j] = 1.0
+    o = O.attend(x, idx, w, Wv, p)
+    V = O.combine(x, idx, w, Wv).reshape(L, 4, 128)
+    for h, j in enumerate(js):
+        np.testing.assert_allclose(o[h], V[j, h // 2], rtol=0, atol=1e-13)
+    assert not np.allclose(o[1], V[js[1], 1 % 4])  # the other mapping differs
+
+
+def test_attend_linear_in_probabilities():
+    """o is linear in probs (the attention weights enter once, outside the
+    SiLU)."""
+    rng = np.random.default_rng(9)
+    L, d, E, k, n, H = 6, 4, 3, 2, 128, 2
+    x = rng.normal(size=(L, d))
+    Wv = rng.normal(size=(E, n, d))
+    idx = rng.integers(0, E, size=(L, k))
+    w = rng.uniform(0.1, 1.0, size=(L, k))
+    a = rng.uniform(size=(H, L))
+    b = rng.uniform(size=(H, L))
+    np.testing.assert_allclose(O.attend(x, idx, w, Wv, 2.0 * a - b),
+                               2.0 * O.attend(x, idx, w, Wv, a) - O.attend(x, idx, w, Wv, b),
+                               rtol=1e-12, atol=1e-12)
