@@ -261,6 +261,31 @@ typedef struct mova_options {
 size_t mova_router_planes_bytes(int d);
 mova_status mova_router_planes(const float* Wr, int E, int d, void* planes, void* stream);
 
+/* Decode attention's value side over the compact cache, with V never
+ * written to memory ("IFM K2 Horizon Deep Dive", Section 4, Option B: the
+ * cache keeps x, the top-k indices and the fp16 weights; V is rematerialised
+ * on the fly inside the attention).  For L cached positions with hidden
+ * states x (L, d) bf16, given routing idx (L, k) int8/int32 and weights
+ * wgt (L, k) fp16/fp32, and attention probabilities probs (H, L) fp32 of one
+ * query token's H heads:
+ *
+ *   o[h, :] = sum over l of probs[h, l] * V[l, h / G, :],   G = H / (n / 128)
+ *
+ * where V[l] = sum over slots (ascending) of w[l, slot] * SiLU(Wv[idx[l, slot]] x[l]),
+ * viewed as (n / 128) KV heads of 128 ("MoVA: routing the value vectors",
+ * section "Where the routing happens": the mixture is what a GQA v_proj
+ * writes; query head h reads KV head h / G).  o: (H, 128) fp32, device.
+ * bf16 x and Wv only; 1 <= G <= 4; runs the tensor-core expert kernel with
+ * an epilogue that sums p * w * SiLU(h) per tile instead of storing V, then
+ * a fixed-order reduction (results do not depend on timing).  Workspace:
+ * mova_attend_workspace_size(L, d, E, k, n, H) bytes, 256-byte aligned.
+ * L = 0 writes zeros.  Errors as mova_value; MOVA_ERR_UNSUPPORTED for H not a
+ * multiple of n / 128 or G > 4. */
+size_t mova_attend_workspace_size(int L, int d, int E, int k, int n, int H);
+mova_status mova_value_attend(const void* x, const void* idx, mova_dtype idx_dt, const void* wgt,
+                              mova_dtype w_dt, const void* Wv, int L, int d, int E, int k, int n,
+                              const float* probs, int H, float* o, void* ws, size_t ws_bytes, void* stream);
+
 /* mova_route with options (only router_partitions applies). */
 mova_status mova_route_opts(const void* x, mova_dtype x_dt, const float* Wr, const float* br,
                             int T, int d, int E, int k, float scale, int32_t* idx, float* w,

@@ -58,6 +58,8 @@ SIGNATURES = {
     "mova_selftest_arm_stream_stall": (_i, [_i, ctypes.c_longlong]),
     "mova_workspace_parts": (_i, [_i, _i, _i, _i, _i, _vp]),
     "mova_router_planes_bytes": (_sz, [_i]),
+    "mova_attend_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i]),
+    "mova_value_attend": (_i, [_vp, _vp, _i, _vp, _i, _vp, _i, _i, _i, _i, _i, _vp, _i, _vp, _vp, _sz, _vp]),
     "mova_router_planes": (_i, [_vp, _i, _i, _vp, _vp]),
     "mova_value_routed_noalloc": (_i, [_vp, _i, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _vp,
                                        _vp]),

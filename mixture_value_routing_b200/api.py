@@ -203,6 +203,37 @@ def value(x: torch.Tensor, idx: torch.Tensor, w: torch.Tensor, Wv: torch.Tensor,
     return v
 
 
+def attend_workspace_size(L: int, d: int, E: int, k: int, n: int, H: int) -> int:
+    return int(_lib.load().mova_attend_workspace_size(L, d, E, k, n, H))
+
+
+def value_attend(x: torch.Tensor, idx: torch.Tensor, w: torch.Tensor, Wv: torch.Tensor,
+                 probs: torch.Tensor, ws: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """One query token's attention output over L cached positions whose
+    values are recomputed from the compact cache (x, idx, w) and never
+    stored: o (H, 128) fp32 = sum_l probs[h, l] * V[l, h // G]."""
+    _need(x, "x", (torch.bfloat16,), 2)
+    _need(idx, "idx", (torch.int32, torch.int8), 2)
+    _need(w, "w", (torch.float32, torch.float16), 2)
+    _need(Wv, "Wv", (torch.bfloat16,), 3)
+    _need(probs, "probs", (torch.float32,), 2)
+    L, d = x.shape
+    E, n = Wv.shape[0], Wv.shape[1]
+    k = idx.shape[1]
+    H = probs.shape[0]
+    if probs.shape[1] != L:
+        raise ValueError("probs: (H, L) for the L cached positions of x")
+    o = torch.empty((H, 128), dtype=torch.float32, device=x.device)
+    lib = _lib.load()
+    nbytes = int(lib.mova_attend_workspace_size(L, d, E, k, n, H))
+    if ws is None:
+        ws = _workspace(nbytes, x.device)
+    _lib.check(lib.mova_value_attend(_ptr(x), _ptr(idx), _DT[idx.dtype], _ptr(w), _DT[w.dtype], _ptr(Wv),
+                                     L, d, E, k, n, _ptr(probs), H, _ptr(o), _ptr(ws), ws.numel(),
+                                     _stream()), "mova_value_attend")
+    return o
+
+
 def value_routed(x: torch.Tensor, Wr: torch.Tensor, br: torch.Tensor, Wv: torch.Tensor,
                  k: int = 4, scale: float = 2.5, return_routing: bool = False,
                  path: str = "auto", ws: Optional[torch.Tensor] = None,

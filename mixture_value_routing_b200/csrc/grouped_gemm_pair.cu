@@ -82,6 +82,7 @@ struct __align__(1024) PSmem {
   int act_cnt[64];
   int act_off[64];
   int act_ntt[64];
+  int act_gbase[64];  // attend mode: the expert's first token-tile group (experts in index order)
   int tile_base[65];
   // Per epilogue warp: a 32 x 32 bf16 block transposed for the P stores
   // (column-major, rows paired into 32-bit words).
@@ -89,7 +90,7 @@ struct __align__(1024) PSmem {
 };
 
 struct PTile {
-  int e, mt, tok0, valid, N0, N1, off;
+  int e, mt, tt, tok0, valid, N0, N1, off, gbase;
 };
 
 __device__ __forceinline__ PTile decode_ptile(const PSmem& S, int t, int mtiles) {
@@ -106,6 +107,8 @@ __device__ __forceinline__ PTile decode_ptile(const PSmem& S, int t, int mtiles)
   const int ntt = S.act_ntt[a];
   PTile r;
   r.e = S.act_e[a];
+  r.tt = tt;
+  r.gbase = S.act_gbase[a];
   r.mt = local - tt * mtiles;
   r.tok0 = static_cast<int>(static_cast<long long>(tt) * cnt / ntt);
   r.valid = static_cast<int>(static_cast<long long>(tt + 1) * cnt / ntt) - r.tok0;
@@ -115,6 +118,34 @@ __device__ __forceinline__ PTile decode_ptile(const PSmem& S, int t, int mtiles)
   r.off = S.act_off[a];
   return r;
 }
+
+// Inclusive prefix over 64 values, v0 of lane l at index l and v1 at 32 + l;
+// tot0 = sum of the first 32, tot = sum of all.
+__device__ __forceinline__ void tile_prefix(int& v0, int& v1, int lane, int& tot0, int& tot) {
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y0 = __shfl_up_sync(0xffffffffu, v0, o);
+    const int y1 = __shfl_up_sync(0xffffffffu, v1, o);
+    if (lane >= o) { v0 += y0; v1 += y1; }
+  }
+  tot0 = __shfl_sync(0xffffffffu, v0, 31);
+  tot = tot0 + __shfl_sync(0xffffffffu, v1, 31);
+}
+
+// Attend mode (the PV product of decode attention with V recomputed from the
+// compact cache, never stored): per query head h and cached position l,
+// p[h * L + l] is the attention probability; query head h reads KV head
+// h / G.  Each tile leaves, per query head of its KV head and weight row,
+// the sum over its pairs of p[h, token] * w[pair] * SiLU(h_pair[row]) in
+// part[((group * 2 + accumulator) * G + head-in-group) * n + row].
+// coef[q * Hp + 4 * g + j] = p[(g * G + j) * L + token of pair q] * w[pair q]
+// for grouped position q, KV head g and head-in-group j < G (zero for
+// G <= j < 4): prepared by attend_coef_kernel.
+struct AttendArgs {
+  const float* coef;
+  float* part;
+  int Hp;  // 4 * KV heads
+};
 
 // Tensor memory holds two accumulator regions of 256 columns.  A tile of at
 // most 256 pairs takes one region, alternating between the two, so its
@@ -163,11 +194,12 @@ constexpr int kAcc1Rows = NA / 2;               // accumulator 1's rows start he
 
 // Ten warps: sub-partitions 0 and 1 hold three each, so at most
 // 16384 / (3 * 32) -> 168 registers per thread.
+template <bool kAttend>
 __global__ void __maxnreg__(168)
 grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_xp,
                          const int32_t* __restrict__ counts, const int32_t* __restrict__ offsets,
                          int E, StatusBlock* __restrict__ sb, int d, int n,
-                         int ldw, __nv_bfloat16* __restrict__ P) {
+                         int ldw, __nv_bfloat16* __restrict__ P, AttendArgs at) {
   extern __shared__ uint8_t smem_raw[];
   PSmem& S = *reinterpret_cast<PSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5;
@@ -211,6 +243,17 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_w, const __gri
       r1 += (x0 >= c1) + (x1 > c1 || (x1 == c1 && b < lane));
     }
     const int nact = __popc(__ballot_sync(0xffffffffu, c0 > 0)) + __popc(__ballot_sync(0xffffffffu, c1 > 0));
+    // Token-tile groups in expert index order (attend mode: one partial per
+    // group, accumulator, query head of the group and weight row).
+    int q0 = c0 > 0 ? (c0 + NT - 1) / NT : 0, q1 = c1 > 0 ? (c1 + NT - 1) / NT : 0;
+    {
+      int g0 = q0, g1 = q1, gt0, gt;
+      tile_prefix(g0, g1, lane, gt0, gt);
+      q0 = g0 - q0;        // exclusive: groups of experts below e0
+      q1 = gt0 + g1 - q1;  // and below e1
+    }
+    if (c0 > 0) S.act_gbase[r0] = q0;
+    if (c1 > 0) S.act_gbase[r1] = q1;
     if (c0 > 0) {
       S.act_e[r0] = e0;
       S.act_cnt[r0] = c0;
@@ -227,13 +270,8 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_w, const __gri
     const int a0 = lane, a1 = lane + 32;
     int v0 = a0 < nact ? S.act_ntt[a0] * mtiles : 0;
     int v1 = a1 < nact ? S.act_ntt[a1] * mtiles : 0;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y0 = __shfl_up_sync(0xffffffffu, v0, o);
-      const int y1 = __shfl_up_sync(0xffffffffu, v1, o);
-      if (lane >= o) { v0 += y0; v1 += y1; }
-    }
-    const int tot0 = __shfl_sync(0xffffffffu, v0, 31);
+    int tot0, tot;
+    tile_prefix(v0, v1, lane, tot0, tot);
     S.tile_base[a0 + 1] = v0;
     S.tile_base[a1 + 1] = tot0 + v1;
     if (lane == 0) {
@@ -434,6 +472,57 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_w, const __gri
       const int nvalid = min(N, tl.valid - j0);
       const int rloc = tl.mt * 2 * PM + static_cast<int>(rank) * PM + q * 32 + lane;
       const uint32_t tbase = S.tmem_base + static_cast<uint32_t>(myreg * NA) + (static_cast<uint32_t>(q * 32) << 16);
+      if constexpr (kAttend) {
+        // Attend mode: the weighted sums of SiLU(h) over the unit's pairs
+        // for the four query heads of this CTA's KV head, per weight row.
+        const int rb = rloc - lane;             // this warp's first weight row
+        const int head = (rloc - q * 32 - lane) / 128;  // the CTA's 128 rows are one KV head
+        float4* cw = reinterpret_cast<float4*>(S.epi[warp - 2]);  // 32 columns' coefficients
+        const float* cbase = at.coef + static_cast<size_t>(tl.off + tl.tok0 + j0) * at.Hp + 4 * head;
+        float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+        float4 cn = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (rb < n && lane < nvalid) cn = __ldg(reinterpret_cast<const float4*>(cbase + static_cast<size_t>(lane) * at.Hp));
+#pragma unroll 1
+        for (int cc = 0; cc < 8; ++cc) {
+          if (cc * 32 >= N) break;
+          const float4 c = cn;
+          cn = make_float4(0.f, 0.f, 0.f, 0.f);
+          const int nxt = (cc + 1) * 32 + lane;
+          if (rb < n && nxt < nvalid && (cc + 1) * 32 < N)
+            cn = __ldg(reinterpret_cast<const float4*>(cbase + static_cast<size_t>(nxt) * at.Hp));
+          uint32_t r[32];
+          tmem_ld_32(tbase + cc * 32, r);
+          cw[lane] = c;
+          tmem_ld_wait();
+          __syncwarp();
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const float4 cj = cw[j];
+            const float sv = silu_fast(__uint_as_float(r[j]));
+            a0 = fmaf(cj.x, sv, a0);
+            a1 = fmaf(cj.y, sv, a1);
+            a2 = fmaf(cj.z, sv, a2);
+            a3 = fmaf(cj.w, sv, a3);
+          }
+          __syncwarp();
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(empty_cl);
+        if (rb < n) {
+          float* pp = at.part + static_cast<size_t>((tl.gbase + tl.tt) * 2 + acc) * 4 * n + rloc;
+          pp[0] = a0;
+          pp[static_cast<size_t>(n)] = a1;
+          pp[2 * static_cast<size_t>(n)] = a2;
+          pp[3 * static_cast<size_t>(n)] = a3;
+          if (acc == 0 && tl.N1 == 0) {
+            // No second accumulator: its slot of this group holds zeros.
+#pragma unroll
+            for (int j = 0; j < 4; ++j) pp[static_cast<size_t>(4 + j) * n] = 0.f;
+          }
+        }
+        continue;
+      }
       // The accumulator's columns are read in two halves of 128 (SiLU,
       // rounded to bf16, two per word): the first half is read and stored,
       // then the second half is read, the accumulator is handed back to the
@@ -520,10 +609,12 @@ using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, 
 
 }  // namespace
 
-cudaError_t launch_tensor_experts_pair(const void* Wv, long long ldw, const int32_t* counts,
-                                       const int32_t* offsets, StatusBlock* sb, int T,
-                                       int d, int n, int k, int E, const __nv_bfloat16* xp, __nv_bfloat16* P,
-                                       cudaStream_t stream) {
+namespace {
+
+template <bool kAttend>
+cudaError_t launch_pair(const void* Wv, long long ldw, const int32_t* counts, const int32_t* offsets,
+                        StatusBlock* sb, int T, int d, int n, int k, int E, const __nv_bfloat16* xp,
+                        __nv_bfloat16* P, AttendArgs at, cudaStream_t stream) {
   void* fp = encode_tiled_fn();
   if (fp == nullptr) return cudaErrorNotSupported;
   EncodeTiled enc = reinterpret_cast<EncodeTiled>(fp);
@@ -548,7 +639,7 @@ cudaError_t launch_tensor_experts_pair(const void* Wv, long long ldw, const int3
           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
   const size_t smem = sizeof(PSmem) + 1024;
-  cudaError_t err = cudaFuncSetAttribute(grouped_gemm_pair_kernel,
+  cudaError_t err = cudaFuncSetAttribute(grouped_gemm_pair_kernel<kAttend>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (err != cudaSuccess) return err;
   // As many pairs as can be resident at once (persistent).
@@ -569,14 +660,100 @@ cudaError_t launch_tensor_experts_pair(const void* Wv, long long ldw, const int3
   if (max_clusters == 0) {
     cfg.gridDim = dim3(2 * (sm_count() / 2));
     int c = 0;
-    if (cudaOccupancyMaxActiveClusters(&c, grouped_gemm_pair_kernel, &cfg) != cudaSuccess || c <= 0)
+    if (cudaOccupancyMaxActiveClusters(&c, grouped_gemm_pair_kernel<kAttend>, &cfg) != cudaSuccess || c <= 0)
       c = sm_count() / 2;
     max_clusters = c;
   }
   cfg.gridDim = dim3(2 * max_clusters);
   note_launch();
-  return cudaLaunchKernelEx(&cfg, grouped_gemm_pair_kernel, tmap_w, tmap_xp, counts, offsets, E, sb, d, n,
-                            static_cast<int>(ldw), P);
+  return cudaLaunchKernelEx(&cfg, grouped_gemm_pair_kernel<kAttend>, tmap_w, tmap_xp, counts, offsets, E, sb, d,
+                            n, static_cast<int>(ldw), P, at);
+}
+
+// coef[q * Hp + 4 * g + j] for every grouped position q (see AttendArgs):
+// one thread per (q, KV head g), four query heads each.
+__global__ void __launch_bounds__(256)
+attend_coef_kernel(const float* __restrict__ probs, const int32_t* __restrict__ perm,
+                   const float* __restrict__ w32, int L, int k, int nkv, int G, float* __restrict__ coef) {
+  pdl_wait();
+  const long long total = static_cast<long long>(L) * k * nkv;
+  for (long long i = static_cast<long long>(blockIdx.x) * 256 + threadIdx.x; i < total;
+       i += static_cast<long long>(gridDim.x) * 256) {
+    const int q = static_cast<int>(i / nkv);
+    const int g = static_cast<int>(i % nkv);
+    const int f = perm[q];
+    const int pos = f / k;
+    const float wq = w32[f];
+    float c[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      c[j] = j < G ? probs[static_cast<size_t>(g * G + j) * L + pos] * wq : 0.f;
+    *reinterpret_cast<float4*>(coef + static_cast<size_t>(q) * 4 * nkv + 4 * g) =
+        make_float4(c[0], c[1], c[2], c[3]);
+  }
+}
+
+// o[h, c] = sum over token-tile groups (expert order, then token tile) and
+// accumulators of part[((group * 2 + acc) * 4 + h % G) * n + (h / G) * 128 + c]:
+// a fixed order, so the result does not depend on timing.  One thread per
+// (query head, column).
+__global__ void __launch_bounds__(256)
+attend_reduce_kernel(const float* __restrict__ part, const int32_t* __restrict__ counts, int E, int n,
+                     int G, int H, float* __restrict__ o) {
+  pdl_wait();
+  __shared__ int ngroups;
+  if (threadIdx.x == 0) {
+    int g = 0;
+    for (int e = 0; e < E; ++e) g += (counts[e] + NT - 1) / NT;
+    ngroups = g;
+  }
+  __syncthreads();
+  const int i = blockIdx.x * 256 + threadIdx.x;
+  if (i >= H * 128) return;
+  const int h = i / 128, c = i % 128;
+  const size_t col = static_cast<size_t>((h / G) * 128 + c);
+  const size_t hq = static_cast<size_t>(h % G);
+  float acc = 0.f;
+  for (int g = 0; g < ngroups; ++g) {
+    acc += part[((static_cast<size_t>(g) * 2) * 4 + hq) * n + col];
+    acc += part[((static_cast<size_t>(g) * 2 + 1) * 4 + hq) * n + col];
+  }
+  o[i] = acc;
+}
+
+}  // namespace
+
+cudaError_t launch_tensor_experts_pair(const void* Wv, long long ldw, const int32_t* counts,
+                                       const int32_t* offsets, StatusBlock* sb, int T,
+                                       int d, int n, int k, int E, const __nv_bfloat16* xp, __nv_bfloat16* P,
+                                       cudaStream_t stream) {
+  return launch_pair<false>(Wv, ldw, counts, offsets, sb, T, d, n, k, E, xp, P, AttendArgs{}, stream);
+}
+
+size_t attend_part_bytes(int L, int E, int k, int n) {
+  const long long groups = static_cast<long long>(L) * k / NT + E + 1;
+  return static_cast<size_t>(groups) * 2 * 4 * n * 4;
+}
+
+cudaError_t launch_tensor_attend(const void* Wv, const int32_t* counts, const int32_t* offsets,
+                                 const int32_t* perm, const float* w32, StatusBlock* sb, int L, int d, int n,
+                                 int k, int E, const float* probs, int H, const __nv_bfloat16* xp,
+                                 float* coef, float* part, float* o, cudaStream_t stream) {
+  const int nkv = n / 128;
+  const int G = H / nkv;
+  const long long total = static_cast<long long>(L) * k * nkv;
+  long long blocks = (total + 255) / 256;
+  const long long cap = static_cast<long long>(sm_count()) * 8;
+  if (blocks > cap) blocks = cap;
+  if (blocks < 1) blocks = 1;
+  cudaError_t err = launch_pdl(attend_coef_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, stream,
+                               probs, perm, w32, L, k, nkv, G, coef);
+  if (err != cudaSuccess) return err;
+  err = launch_pair<true>(Wv, n, counts, offsets, sb, L, d, n, k, E, xp, nullptr,
+                          AttendArgs{coef, part, 4 * nkv}, stream);
+  if (err != cudaSuccess) return err;
+  return launch_pdl(attend_reduce_kernel, dim3(static_cast<unsigned>((H * 128 + 255) / 256)), dim3(256), 0,
+                    stream, static_cast<const float*>(part), counts, E, n, G, H, o);
 }
 
 }  // namespace mova

@@ -203,6 +203,15 @@ cudaError_t launch_tensor_experts(const void* x, const void* Wv, long long ldw, 
                                   const int32_t* active, StatusBlock* sb, int T, int d, int n, int k,
                                   int E, __nv_bfloat16* xp, __nv_bfloat16* P, cudaStream_t stream);
 size_t tensor_experts_smem();
+// Attend mode of the pair GEMM (decode attention's PV product with V
+// recomputed from the compact cache): probs (H, L) fp32, query head h reads
+// KV head h / (H / (n / 128)), at most 4 query heads per KV head.  coef:
+// L*k*(n/32) floats; part: attend_part_bytes; o: (H, 128) fp32.
+size_t attend_part_bytes(int L, int E, int k, int n);
+cudaError_t launch_tensor_attend(const void* Wv, const int32_t* counts, const int32_t* offsets,
+                                 const int32_t* perm, const float* w32, StatusBlock* sb, int L, int d, int n,
+                                 int k, int E, const float* probs, int H, const __nv_bfloat16* xp,
+                                 float* coef, float* part, float* o, cudaStream_t stream);
 // xp[pos[t * k + j]] = x[t] for the T*k pairs (token-major: each x row read once).
 cudaError_t launch_gather_pairs(const void* x, const int32_t* pos, int T, int d, int k,
                                 __nv_bfloat16* xp, cudaStream_t stream);

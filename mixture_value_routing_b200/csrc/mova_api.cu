@@ -253,6 +253,54 @@ size_t mova_workspace_size(int T, int d, int E, int k, int n) {
 
 unsigned long long mova_launch_count(void) { return mova::g_launches.load(); }
 
+// Attend mode: the value workspace plus the per-group partials.
+static bool attend_heads_ok(int n, int H) {
+  const int nkv = n / 128;
+  return H > 0 && nkv > 0 && H % nkv == 0 && H / nkv <= 4;
+}
+
+size_t mova_attend_workspace_size(int L, int d, int E, int k, int n, int H) {
+  if (check_dims(L, d, E, k, n) != MOVA_OK || !attend_heads_ok(n, H) || L == 0) return 0;
+  return layout(nullptr, L, d, k, n).bytes + align256(attend_part_bytes(L, E, k, n));
+}
+
+mova_status mova_value_attend(const void* x, const void* idx, mova_dtype idx_dt, const void* wgt,
+                              mova_dtype w_dt, const void* Wv, int L, int d, int E, int k, int n,
+                              const float* probs, int H, float* o, void* ws, size_t ws_bytes, void* stream) {
+  mova_status st = check_dims(L, d, E, k, n);
+  if (st != MOVA_OK) return st;
+  if (H <= 0) return MOVA_ERR_INVALID_ARG;
+  if (!attend_heads_ok(n, H)) return MOVA_ERR_UNSUPPORTED;
+  if (idx_dt != MOVA_I32 && idx_dt != MOVA_I8) return MOVA_ERR_UNSUPPORTED;
+  if (w_dt != MOVA_F32 && w_dt != MOVA_F16) return MOVA_ERR_UNSUPPORTED;
+  if (!o) return MOVA_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (L == 0) return from_cuda(cudaMemsetAsync(o, 0, static_cast<size_t>(H) * 128 * sizeof(float), s));
+  if (!x || !idx || !wgt || !Wv || !probs || !ws) return MOVA_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(Wv)) return MOVA_ERR_INVALID_ARG;
+  if (sm_count() < 2) return MOVA_ERR_UNSUPPORTED;  // the pair GEMM
+  const Workspace w = layout(ws, L, d, k, n);
+  const size_t part_off = w.bytes;
+  if (ws_bytes < part_off + align256(attend_part_bytes(L, E, k, n)) || (reinterpret_cast<uintptr_t>(ws) & 255) != 0)
+    return MOVA_ERR_INVALID_ARG;
+  cudaError_t err;
+  if (L > kSmallGroupT) {
+    err = launch_tile_hist(idx, idx_dt, wgt, w_dt, L, E, k, w.idx, w.w, w.tile_counts, w.sb, s);
+    if (err == cudaSuccess)
+      err = launch_tile_group(w.idx, L, E, k, w.tile_counts, w.counts, w.offsets, w.perm, w.pos, w.active, w.sb,
+                              false, w.tickets, combine_tickets(L, n), s);
+  } else {
+    err = launch_permute(idx, idx_dt, wgt, w_dt, L * k, E, w.idx, w.w, w.counts, w.offsets, w.perm, w.pos,
+                         w.active, w.sb, w.tickets, combine_tickets(L, n), s);
+  }
+  if (err == cudaSuccess) err = launch_gather_pairs(x, w.pos, L, d, k, w.xp, s);
+  if (err == cudaSuccess)
+    err = launch_tensor_attend(Wv, w.counts, w.offsets, w.perm, w.w, w.sb, L, d, n, k, E, probs, H, w.xp,
+                               static_cast<float*>(w.P),
+                               reinterpret_cast<float*>(static_cast<char*>(ws) + part_off), o, s);
+  return from_cuda(err);
+}
+
 mova_path mova_auto_path(int T, mova_dtype x_dt) {
   return (x_dt == MOVA_BF16 && T > kStreamMaxTokens) ? MOVA_PATH_TENSOR : MOVA_PATH_STREAM;
 }

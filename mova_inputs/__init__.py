@@ -43,7 +43,7 @@ N_OUT = N_HEADS * HEAD_DIM
 SCALE = 2.5
 
 # Fixed stream ids: each tensor of a layer draws from its own child stream.
-_STREAM = {"x": 1, "wr": 2, "br": 3, "wv": 4, "idx": 5, "w": 6}
+_STREAM = {"x": 1, "wr": 2, "br": 3, "wv": 4, "idx": 5, "w": 6, "probs": 7}
 
 WORKLOADS = {
     # name: (tokens, activation dtype, routing mode, bias law)
@@ -153,6 +153,25 @@ def make_batch(T: int, seed: int = 0, step: int = 0, *, d: int = D_MODEL, dtype:
         g = _rng(seed, 1000 + step, "w").exponential(1.0, size=(T, k))
         b.w = (scale * g / g.sum(axis=1, keepdims=True)).astype(np.float16)
     return b
+
+
+def make_attention_probs(H: int, L: int, seed: int = 0, step: int = 0, *, spread: float = 2.0,
+                         support: int = 0) -> np.ndarray:
+    """Attention probabilities of one query token's H heads over L cached
+    positions, (H, L) fp32: a softmax of N(0, spread) scores per head (the
+    shape decode attention produces; no trained model is involved).  With
+    support > 0 each head puts all its probability on `support` random
+    positions (softmax over those only), the rest exactly zero."""
+    r = _rng(seed, 2000 + step, "probs")
+    z = r.standard_normal((H, L)) * spread
+    if support > 0:
+        keep = np.zeros((H, L), dtype=bool)
+        for h in range(H):
+            keep[h, r.choice(L, size=min(support, L), replace=False)] = True
+        z = np.where(keep, z, -np.inf)
+    z = z - z.max(axis=1, keepdims=True)
+    e = np.exp(z)
+    return (e / e.sum(axis=1, keepdims=True)).astype(np.float32)
 
 
 def workload(name: str, seed: int = 0, layer: int = 0, step: int = 0):

@@ -148,3 +148,17 @@ def test_stream_stall_arming_is_validated(lib):
     assert lib.mova_selftest_arm_stream_stall(-3, 1000) == _lib.ERR_INVALID_ARG
     assert lib.mova_selftest_arm_stream_stall(2, 0) == _lib.ERR_INVALID_ARG
     assert lib.mova_selftest_arm_stream_stall(2, 1 << 40) == _lib.ERR_INVALID_ARG
+
+
+def test_attend_host_side_validation(lib):
+    """mova_value_attend: head counts and sizes checked on the host."""
+    fake = ctypes.c_void_p(4096)
+    I32, F16 = _lib.I32, _lib.F16
+    args = lambda H, o: (fake, fake, I32, fake, F16, fake, 64, 2560, 64, 4, 1024, fake, H, o, fake, 1 << 30, None)
+    assert lib.mova_value_attend(*args(0, fake)) == _lib.ERR_INVALID_ARG     # no heads
+    assert lib.mova_value_attend(*args(12, fake)) == _lib.ERR_UNSUPPORTED    # not a multiple of 8 KV heads
+    assert lib.mova_value_attend(*args(48, fake)) == _lib.ERR_UNSUPPORTED    # 6 query heads per KV head
+    assert lib.mova_value_attend(*args(32, None)) == _lib.ERR_INVALID_ARG    # no output
+    assert lib.mova_attend_workspace_size(64, 2560, 64, 4, 1024, 32) > lib.mova_workspace_size(64, 2560, 64, 4, 1024)
+    assert lib.mova_attend_workspace_size(64, 2560, 64, 4, 1024, 40) == 0
+    assert lib.mova_attend_workspace_size(0, 2560, 64, 4, 1024, 32) == 0

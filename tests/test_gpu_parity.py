@@ -287,6 +287,87 @@ def test_given_32768(api):
     P.check_values(P.host_f64(v)[rows], v_ref, "bf16")
 
 
+# ---------------------------------------------------------------------------
+# Attend: the PV product with V recomputed from the compact cache
+# ---------------------------------------------------------------------------
+
+
+def _attend_ref(bat, lay, probs, rows=None):
+    x = O.to_f64(bat.x, "bf16")
+    idx = bat.idx.astype(np.int64)
+    w = bat.w.astype(np.float64)
+    p = probs.astype(np.float64)
+    if rows is not None:
+        x, idx, w, p = x[rows], idx[rows], w[rows], p[:, rows]
+    return O.attend(x, idx, w, lay.Wv, p, "bf16")
+
+
+@pytest.mark.parametrize("L,H", [(1, 32), (65, 32), (300, 8), (1000, 32), (4096, 16)])
+def test_value_attend(api, L, H):
+    """o (H, 128) against the oracle's attend: the experts' dot products and
+    SiLU in fp32, weighted by p * w in fp32, summed per tile and then over
+    tiles in a fixed order; |err| <= 1e-4 max(1, |ref|)."""
+    d, E, k, n = 2560, 64, 4, 1024
+    lay = _layer(51, d, E, n, "bf16")
+    bat = MI.make_batch(L, 51, dtype="bf16", mode="given")
+    probs = MI.make_attention_probs(H, L, 51)
+    o = api.value_attend(P.dev(bat.x, "bf16"), P.dev(bat.idx, "i8"), P.dev(bat.w, "f16"),
+                         P.dev(lay.Wv, "bf16"), torch.from_numpy(probs).cuda())
+    torch.cuda.synchronize()
+    assert o.shape == (H, 128) and o.dtype == torch.float32
+    ref = _attend_ref(bat, lay, probs)
+    err = np.abs(o.cpu().numpy().astype(np.float64) - ref)
+    assert (err <= 1e-4 * np.maximum(1.0, np.abs(ref))).all(), err.max()
+
+
+def test_value_attend_one_hot_is_the_value_row(api):
+    """All of head h's probability on position j: o[h] is row j of the value
+    tensor (the routing-given call) in KV head h // G."""
+    d, E, k, n, L, H = 2560, 64, 4, 1024, 200, 32
+    lay = _layer(52, d, E, n, "bf16")
+    bat = MI.make_batch(L, 52, dtype="bf16", mode="given")
+    js = np.random.default_rng(52).integers(0, L, size=H)
+    probs = np.zeros((H, L), dtype=np.float32)
+    probs[np.arange(H), js] = 1.0
+    args = (P.dev(bat.x, "bf16"), P.dev(bat.idx, "i8"), P.dev(bat.w, "f16"), P.dev(lay.Wv, "bf16"))
+    o = api.value_attend(*args, torch.from_numpy(probs).cuda())
+    v = api.value(*args, path="tensor")
+    torch.cuda.synchronize()
+    V = v.float().cpu().numpy().reshape(L, 8, 128)
+    G = H // 8
+    for h in range(H):
+        # v is rounded to bf16 once; o is not
+        np.testing.assert_allclose(o[h].cpu().numpy(), V[js[h], h // G], rtol=1e-2, atol=1e-2)
+
+
+def test_value_attend_32768_sparse(api):
+    """L = 32768 cached positions (the routing-given workload), every one
+    recomputed on the GPU; each head's probability on 64 random positions,
+    so the oracle needs only those."""
+    d, E, k, n, L, H = 2560, 64, 4, 1024, 32768, 32
+    lay = _layer(0, d, E, n, "bf16")
+    bat = MI.make_batch(L, 0, dtype="bf16", mode="given")
+    probs = MI.make_attention_probs(H, L, 53, support=64)
+    o = api.value_attend(P.dev(bat.x, "bf16"), P.dev(bat.idx, "i8"), P.dev(bat.w, "f16"),
+                         P.dev(lay.Wv, "bf16"), torch.from_numpy(probs).cuda())
+    torch.cuda.synchronize()
+    rows = np.nonzero(probs.any(axis=0))[0]
+    ref = _attend_ref(bat, lay, probs, rows)
+    err = np.abs(o.cpu().numpy().astype(np.float64) - ref)
+    assert (err <= 1e-4 * np.maximum(1.0, np.abs(ref))).all(), err.max()
+
+
+def test_value_attend_deterministic(api):
+    d, E, k, n, L, H = 2560, 64, 4, 1024, 3000, 32
+    lay = _layer(54, d, E, n, "bf16")
+    bat = MI.make_batch(L, 54, dtype="bf16", mode="given")
+    probs = torch.from_numpy(MI.make_attention_probs(H, L, 54)).cuda()
+    args = (P.dev(bat.x, "bf16"), P.dev(bat.idx, "i8"), P.dev(bat.w, "f16"), P.dev(lay.Wv, "bf16"), probs)
+    first = api.value_attend(*args).clone()
+    for _ in range(3):
+        assert torch.equal(api.value_attend(*args), first)
+
+
 def test_back_to_back_sizes_share_a_workspace(api):
     """A large bf16 call followed, with no synchronisation, by a smaller one on
     the same stream and the same workspace: the second call's kernels start
