@@ -42,8 +42,10 @@ WORKLOAD_TEXT = {
     "skewed": "skewed prefill T=16384 (router bias 2 ln Zipf(1.2); otherwise as prefill)",
     "given": "routing-given recompute L=32768 (int8 top-4 indices, fp16 Dirichlet(1)x2.5 weights)",
     "pr1": "PR1 reference T=128, all fp32",
+    "attend": "attend: one query token's 32 heads over L=32768 cached positions, values recomputed from the "
+              "compact cache (int8 top-4, fp16 weights) inside the PV product, never stored",
 }
-DEFAULT_STEPS = {"decode": 2000, "prefill": 300, "skewed": 60, "given": 30, "pr1": 200}
+DEFAULT_STEPS = {"decode": 2000, "prefill": 300, "skewed": 60, "given": 30, "pr1": 200, "attend": 30}
 METRIC = "MoVA value-path tokens/s at T=8 & T=4096; % of HBM / bf16 tensor roofline"
 STAGES = ("route", "group", "experts", "combine")
 KERNEL_SOURCES = {
@@ -66,7 +68,7 @@ def parse(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=8.0, help="oracle sample budget")
-    ap.add_argument("--also", default="prefill,skewed,given",
+    ap.add_argument("--also", default="prefill,skewed,given,attend",
                     help="workloads measured as sub-records of the same line (comma list; '=' for none)")
     a = ap.parse_args(argv)
     a.also = [w for w in a.also.split(",") if w and w != "="]
@@ -303,12 +305,17 @@ def measure_workload(a, name, K, layers, device, dist_on, world, rank, peaks, pe
                for l in range(L)]
     xs = [dev_of(b.x, dtype, device) for b in batches]
     routing = None
-    if mode == "given":
+    if mode in ("given", "attend"):
         routing = [(torch.from_numpy(b.idx).to(device), torch.from_numpy(b.w).to(device))
                    for b in batches]
+    probs = [torch.from_numpy(b.probs).to(device) for b in batches] if mode == "attend" else None
     tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
     v = torch.empty((T, n), dtype=tdt, device=device)
-    ws = torch.empty(api.workspace_size(T, d, E, k, n), dtype=torch.uint8, device=device)
+    if mode == "attend":
+        ws = torch.empty(api.attend_workspace_size(T, d, E, k, n, MI.ATTEND_HEADS), dtype=torch.uint8,
+                         device=device)
+    else:
+        ws = torch.empty(api.workspace_size(T, d, E, k, n), dtype=torch.uint8, device=device)
     path = api.auto_path(T, tdt)
 
     def step(i, events=None):
@@ -316,6 +323,10 @@ def measure_workload(a, name, K, layers, device, dist_on, world, rank, peaks, pe
         Wr, br, Wv = layers.get(l, cfg["bias"])
         if routing is None:
             api.value_routed(xs[l], Wr, br, Wv, k, MI.SCALE, out=v, ws=ws, events=events)
+        elif probs is not None:
+            # mova_value_attend takes no stage events: the step is timed whole.
+            idx, w = routing[l]
+            api.value_attend(xs[l], idx, w, Wv, probs[l], ws=ws)
         else:
             idx, w = routing[l]
             api.value(xs[l], idx, w, Wv, ws=ws, events=events)
@@ -405,13 +416,22 @@ def measure_workload(a, name, K, layers, device, dist_on, world, rank, peaks, pe
     del graph, pgraph
 
     ms_per_step = ms / K
+    if mode == "attend":
+        # No stage events: the whole step (coefficients, grouping, gather,
+        # GEMM with the attend epilogue, reduction) stands for the experts.
+        stage_avg_us = {s: 0.0 for s in STAGES}
+        stage_avg_us["experts"] = 1e3 * ms_per_step
+        empty_us = 0.0
     value = job_value(world, T, K, ms)
     roof = roofline(name, path, T, d, E, k, n, xs_b, distinct, stage_avg_us, empty_us, ms_per_step,
                     peaks, peak_src)
+    if mode == "attend":
+        roof["kernel"] = "whole attend step (no stage events in mova_value_attend)"
+        roof["traffic"] = None
 
     e2e = None
     if not a.no_e2e:
-        e2e = measure_e2e(a, T, L, xs, routing, layers, cfg, v, ws, k, n, tdt, dist_on, world, device)
+        e2e = measure_e2e(a, T, L, xs, routing, layers, cfg, v, ws, k, n, tdt, dist_on, world, device, probs)
 
     rec = {
         "value": round(value, 1), "unit": "tokens/s", "steps": K, "warmup": a.warmup,
@@ -475,10 +495,11 @@ def roofline(name, path, T, d, E, k, n, xs_b, distinct, stage_us, empty_us, ms_p
             "peak_source": f"{peak_src} (bf16_tflops, burst)"}
 
 
-def measure_e2e(a, T, L, xs, routing, layers, cfg, v, ws, k, n, tdt, dist_on, world, device):
+def measure_e2e(a, T, L, xs, routing, layers, cfg, v, ws, k, n, tdt, dist_on, world, device, probs=None):
     """The same metric through the public API with host buffers: per step, the
     pinned host->device copy of that step's inputs (x, and the stored routing
-    in routing-given mode), the call, and the device->host copy of v."""
+    in routing-given mode, and the attention probabilities in attend mode),
+    the call, and the device->host copy of v (of o in attend mode)."""
     import torch
 
     from mixture_value_routing_b200 import api
@@ -490,6 +511,10 @@ def measure_e2e(a, T, L, xs, routing, layers, cfg, v, ws, k, n, tdt, dist_on, wo
         rh = [(i.cpu().pin_memory(), w.cpu().pin_memory()) for i, w in routing]
         rd = [torch.empty_like(routing[0][0]), torch.empty_like(routing[0][1])]
     vh = torch.empty((T, n), dtype=tdt).pin_memory()
+    if probs is not None:
+        ph = [p.cpu().pin_memory() for p in probs]
+        pd = torch.empty_like(probs[0])
+        vh = torch.empty((probs[0].shape[0], 128), dtype=torch.float32).pin_memory()
     xd = torch.empty_like(xs[0])
     Ke = max(3, min(500, int(0.2 / max(1e-6, 2.5e-8 * T * 20))))
 
@@ -502,7 +527,11 @@ def measure_e2e(a, T, L, xs, routing, layers, cfg, v, ws, k, n, tdt, dist_on, wo
         else:
             rd[0].copy_(rh[l][0], non_blocking=True)
             rd[1].copy_(rh[l][1], non_blocking=True)
-            out = api.value(xd, rd[0], rd[1], Wv, ws=ws)
+            if probs is not None:
+                pd.copy_(ph[l], non_blocking=True)
+                out = api.value_attend(xd, rd[0], rd[1], Wv, pd, ws=ws)
+            else:
+                out = api.value(xd, rd[0], rd[1], Wv, ws=ws)
         vh.copy_(out, non_blocking=True)
 
     for i in range(a.warmup):
@@ -522,6 +551,8 @@ def measure_e2e(a, T, L, xs, routing, layers, cfg, v, ws, k, n, tdt, dist_on, wo
     h2d = xs[0].numel() * xs[0].element_size()
     if routing is not None:
         h2d += sum(t.numel() * t.element_size() for t in routing[0])
+    if probs is not None:
+        h2d += probs[0].numel() * probs[0].element_size()
     return {"value": round(job_value(world, T, Ke, ems), 1), "unit": "tokens/s",
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(vh.numel() * vh.element_size()),
             "steps": Ke, "ms_per_step": round(ems / Ke, 5)}
@@ -585,6 +616,9 @@ def _blas_threads():
 
 def _oracle_tokens(O, lay, bat, rows, mode, wv_dt, dtype):
     x = O.to_f64(bat.x[rows], dtype)
+    if mode == "attend":
+        return O.attend(x, bat.idx[rows].astype(np.int64), bat.w[rows].astype(np.float64), lay.Wv,
+                        bat.probs[:, rows].astype(np.float64), wv_dt)
     if mode == "given":
         return O.combine(x, bat.idx[rows].astype(np.int64), bat.w[rows].astype(np.float64),
                          lay.Wv, wv_dt)

@@ -694,31 +694,40 @@ attend_coef_kernel(const float* __restrict__ probs, const int32_t* __restrict__ 
 }
 
 // o[h, c] = sum over token-tile groups (expert order, then token tile) and
-// accumulators of part[((group * 2 + acc) * 4 + h % G) * n + (h / G) * 128 + c]:
-// a fixed order, so the result does not depend on timing.  One thread per
-// (query head, column).
-__global__ void __launch_bounds__(256)
+// accumulators of part[((group * 2 + acc) * 4 + h % G) * n + (h / G) * 128 + c].
+// A block of 32 warps takes query head h and 32 columns: warp w sums groups
+// w, w + 32, ... (both accumulators, in group order), lane = column; warp 0
+// then adds the 32 warps' sums in warp order.  A fixed order, so the result
+// does not depend on timing.
+__global__ void __launch_bounds__(1024)
 attend_reduce_kernel(const float* __restrict__ part, const int32_t* __restrict__ counts, int E, int n,
                      int G, int H, float* __restrict__ o) {
   pdl_wait();
   __shared__ int ngroups;
+  __shared__ float red[32][33];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     int g = 0;
     for (int e = 0; e < E; ++e) g += (counts[e] + NT - 1) / NT;
     ngroups = g;
   }
   __syncthreads();
-  const int i = blockIdx.x * 256 + threadIdx.x;
-  if (i >= H * 128) return;
-  const int h = i / 128, c = i % 128;
+  const int h = blockIdx.x / 4;
+  const int c = (blockIdx.x % 4) * 32 + lane;
   const size_t col = static_cast<size_t>((h / G) * 128 + c);
   const size_t hq = static_cast<size_t>(h % G);
   float acc = 0.f;
-  for (int g = 0; g < ngroups; ++g) {
+  for (int g = warp; g < ngroups; g += 32) {
     acc += part[((static_cast<size_t>(g) * 2) * 4 + hq) * n + col];
     acc += part[((static_cast<size_t>(g) * 2 + 1) * 4 + hq) * n + col];
   }
-  o[i] = acc;
+  red[warp][lane] = acc;
+  __syncthreads();
+  if (warp == 0) {
+    float t = 0.f;
+    for (int w = 0; w < 32; ++w) t += red[w][lane];
+    o[static_cast<size_t>(h) * 128 + c] = t;
+  }
 }
 
 }  // namespace
@@ -752,8 +761,8 @@ cudaError_t launch_tensor_attend(const void* Wv, const int32_t* counts, const in
   err = launch_pair<true>(Wv, n, counts, offsets, sb, L, d, n, k, E, xp, nullptr,
                           AttendArgs{coef, part, 4 * nkv}, stream);
   if (err != cudaSuccess) return err;
-  return launch_pdl(attend_reduce_kernel, dim3(static_cast<unsigned>((H * 128 + 255) / 256)), dim3(256), 0,
-                    stream, static_cast<const float*>(part), counts, E, n, G, H, o);
+  return launch_pdl(attend_reduce_kernel, dim3(static_cast<unsigned>(H * 4)), dim3(1024), 0, stream,
+                    static_cast<const float*>(part), counts, E, n, G, H, o);
 }
 
 }  // namespace mova

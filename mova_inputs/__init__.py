@@ -52,7 +52,11 @@ WORKLOADS = {
     "prefill": dict(T=4096, dtype="bf16", mode="routed", bias="normal"),
     "skewed": dict(T=16384, dtype="bf16", mode="routed", bias="zipf"),
     "given": dict(T=32768, dtype="bf16", mode="given", bias="normal"),
+    # one query token's attention (32 heads) over 32768 cached positions whose
+    # values are recomputed from the compact cache (the given workload's)
+    "attend": dict(T=32768, dtype="bf16", mode="attend", bias="normal"),
 }
+ATTEND_HEADS = 32
 
 
 @dataclasses.dataclass
@@ -76,6 +80,7 @@ class Batch:
     x_dtype: str
     idx: Optional[np.ndarray] = None   # (T, k) int8, routing-given mode
     w: Optional[np.ndarray] = None     # (T, k) fp16, routing-given mode
+    probs: Optional[np.ndarray] = None  # (H, T) fp32, attend mode
 
 
 def _rng(seed: int, layer: int, stream: str, sub: int = 0) -> np.random.Generator:
@@ -144,7 +149,7 @@ def make_batch(T: int, seed: int = 0, step: int = 0, *, d: int = D_MODEL, dtype:
     else:
         raise ValueError(dtype)
     b = Batch(x=x, x_dtype=dtype)
-    if mode == "given":
+    if mode in ("given", "attend"):
         # Routing of the compact cache: k distinct experts per token, the
         # first k entries of a uniform random permutation of the experts.
         r = _rng(seed, 1000 + step, "idx")
@@ -152,6 +157,8 @@ def make_batch(T: int, seed: int = 0, step: int = 0, *, d: int = D_MODEL, dtype:
         b.idx = np.argsort(keys, axis=1)[:, :k].astype(np.int8)
         g = _rng(seed, 1000 + step, "w").exponential(1.0, size=(T, k))
         b.w = (scale * g / g.sum(axis=1, keepdims=True)).astype(np.float16)
+    if mode == "attend":
+        b.probs = make_attention_probs(ATTEND_HEADS, T, seed, step)
     return b
 
 
