@@ -33,7 +33,13 @@
 //     region, one per tensor-memory lane quarter.  Each reads the region's
 //     columns into registers (SiLU, bf16) in two halves, storing the first
 //     half before reading the second, and hands the region back right after
-//     its last read.
+//     its last read; each 32 x 32 block goes through shared memory so that P
+//     rows are stored as 16-byte vectors.
+//   * Attend mode (the value side of decode attention over the compact
+//     cache, V never stored): the epilogue instead sums, per weight row,
+//     p[h, token] * w[pair] * SiLU(h) over the tile's pairs for the four
+//     query heads of the CTA's KV head, and writes one partial per
+//     token-tile group; attend_reduce_kernel adds them in a fixed order.
 //   * One persistent pair per two SMs takes tiles from a global counter;
 //     tiles are numbered largest expert first (then token tile, then the
 //     four weight-row blocks of a token tile next to each other, so pairs
