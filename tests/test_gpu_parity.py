@@ -320,6 +320,22 @@ def test_value_attend(api, L, H):
     assert (err <= 1e-4 * np.maximum(1.0, np.abs(ref))).all(), err.max()
 
 
+def test_value_attend_i32_f32_routing(api):
+    """int32 indices and fp32 weights (the other accepted compact-cache
+    formats), E = 16, k = 2, n = 512 (4 KV heads, 4 query heads each)."""
+    d, E, k, n, L, H = 1024, 16, 2, 512, 700, 16
+    lay = _layer(55, d, E, n, "bf16")
+    bat = MI.make_batch(L, 55, dtype="bf16", d=d, mode="given", E=E, k=k)
+    probs = MI.make_attention_probs(H, L, 55)
+    o = api.value_attend(P.dev(bat.x, "bf16"), P.dev(bat.idx.astype(np.int32), "i32"),
+                         P.dev(bat.w.astype(np.float32), "f32"), P.dev(lay.Wv, "bf16"),
+                         torch.from_numpy(probs).cuda())
+    torch.cuda.synchronize()
+    ref = _attend_ref(bat, lay, probs)
+    err = np.abs(o.cpu().numpy().astype(np.float64) - ref)
+    assert (err <= 1e-4 * np.maximum(1.0, np.abs(ref))).all(), err.max()
+
+
 def test_value_attend_one_hot_is_the_value_row(api):
     """All of head h's probability on position j: o[h] is row j of the value
     tensor (the routing-given call) in KV head h // G."""
