@@ -96,7 +96,7 @@ struct __align__(1024) PSmem {
 };
 
 struct PTile {
-  int e, mt, tt, tok0, valid, N0, N1, off, gbase;
+  int e, mt, tt, ntt, tok0, valid, N0, N1, off, gbase;
 };
 
 __device__ __forceinline__ PTile decode_ptile(const PSmem& S, int t, int mtiles) {
@@ -114,6 +114,7 @@ __device__ __forceinline__ PTile decode_ptile(const PSmem& S, int t, int mtiles)
   PTile r;
   r.e = S.act_e[a];
   r.tt = tt;
+  r.ntt = ntt;
   r.gbase = S.act_gbase[a];
   r.mt = local - tt * mtiles;
   r.tok0 = static_cast<int>(static_cast<long long>(tt) * cnt / ntt);
@@ -298,9 +299,11 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_w, const __gri
     // producer takes the tile ids from the global counter (zeroed by this
     // call's grouping) and publishes each to both CTAs.
     const uint32_t full0_cl = mapa_shared(smem_u32(&S.full[0]), 0);  // even CTA's barriers
-    // Weights stream through once per tile: evict them first, so the
-    // gathered token rows (stored evict-last) stay in L2 for the four
-    // weight-row blocks that read them.
+    // A weight block read by one tile only (the expert has one token tile)
+    // streams through evict-first, so the gathered token rows (stored
+    // evict-last) stay in L2 for the four weight-row blocks that read them;
+    // the blocks of experts with several token tiles keep the normal policy,
+    // as those tiles read them about together.
     const uint64_t wpol = policy_evict_first();
     int s = 0;
     uint32_t phase = 0;
@@ -360,7 +363,10 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_w, const __gri
         uint8_t* st = S.stage[s];
         if (elect_one()) {
           if (rank == 0) mbar_arrive_expect_tx(&S.full[s], bytes);
-          tma_load_2d_pair_hint(st, &tmap_w, kb * PK, arow, full_cl, wpol);
+          if (tl.ntt == 1)
+            tma_load_2d_pair_hint(st, &tmap_w, kb * PK, arow, full_cl, wpol);
+          else  // the expert's other token tiles read this weight block too
+            tma_load_2d_pair(st, &tmap_w, kb * PK, arow, full_cl);
           uint8_t* bt = st + kPABytes;
           for (int b = 0; b < nb0; ++b)
             tma_load_2d_pair(bt + b * kBoxRows * 128, &tmap_xp, kb * PK, row0 + b * kBoxRows, full_cl);
