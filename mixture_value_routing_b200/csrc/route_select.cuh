@@ -26,19 +26,21 @@ __device__ __forceinline__ uint32_t order_key(float f) {
 // attains it (ties go to the lower index), and retires that expert.  On
 // return every lane holds the same sel_e / sel_s (unbiased sigmoid scores)
 // for j < k.
-__device__ __forceinline__ void select_top_k(const float* lg, const float* brs, int E, int k,
-                                             int lane, int (&sel_e)[8], float (&sel_s)[8]) {
+// The same from the lane's two logits and biases in registers (experts
+// lane and lane + 32; values of experts >= E are ignored).
+__device__ __forceinline__ void select_top_k_regs(float lg0, float lg1, float br0, float br1, int E,
+                                                  int k, int lane, int (&sel_e)[8], float (&sel_s)[8]) {
   const int e0 = lane, e1 = lane + 32;
   float s0 = 0.f, s1 = 0.f;
   uint32_t key0 = 0, key1 = 0;
   if (e0 < E) {
-    s0 = sigmoidf_(lg[e0]);
-    const float b = s0 + brs[e0];
+    s0 = sigmoidf_(lg0);
+    const float b = s0 + br0;
     key0 = order_key(b == b ? b : -INFINITY);
   }
   if (e1 < E) {
-    s1 = sigmoidf_(lg[e1]);
-    const float b = s1 + brs[e1];
+    s1 = sigmoidf_(lg1);
+    const float b = s1 + br1;
     key1 = order_key(b == b ? b : -INFINITY);
   }
 #pragma unroll
@@ -56,6 +58,13 @@ __device__ __forceinline__ void select_top_k(const float* lg, const float* brs, 
   }
 }
 
+__device__ __forceinline__ void select_top_k(const float* lg, const float* brs, int E, int k,
+                                             int lane, int (&sel_e)[8], float (&sel_s)[8]) {
+  const int e0 = lane, e1 = lane + 32;
+  select_top_k_regs(e0 < E ? lg[e0] : 0.f, e1 < E ? lg[e1] : 0.f, e0 < E ? brs[e0] : 0.f,
+                    e1 < E ? brs[e1] : 0.f, E, k, lane, sel_e, sel_s);
+}
+
 // Sum of the k selected scores in slot order.
 __device__ __forceinline__ float sum_k(const float (&s)[8], int k) {
   float acc = 0.f;
@@ -65,15 +74,13 @@ __device__ __forceinline__ float sum_k(const float (&s)[8], int k) {
   return acc;
 }
 
-// Selection of token t by one warp, written to shared memory: sel[t*k + j]
-// (expert) and wsel[t*k + j] (renormalised, scaled weight); with idx_out /
-// w_out non-null also to global memory.
-__device__ __forceinline__ void select_token(const float* lg, const float* brs, int E, int k,
-                                             float scale, int t, int lane, int* sel, float* wsel,
-                                             int32_t* idx_out, float* w_out) {
-  int es[8];
-  float ss[8];
-  select_top_k(lg, brs, E, k, lane, es, ss);
+// Selection of token t by one warp from the selected experts and scores:
+// written to shared memory, sel[t*k + j] (expert) and wsel[t*k + j]
+// (renormalised, scaled weight); with idx_out / w_out non-null also to
+// global memory.
+__device__ __forceinline__ void store_selection(const int (&es)[8], const float (&ss)[8], int k, float scale,
+                                                int t, int lane, int* sel, float* wsel, int32_t* idx_out,
+                                                float* w_out) {
   const float ssum = sum_k(ss, k);
 #pragma unroll
   for (int j = 0; j < 8; ++j) {
@@ -87,6 +94,15 @@ __device__ __forceinline__ void select_token(const float* lg, const float* brs, 
       }
     }
   }
+}
+
+__device__ __forceinline__ void select_token(const float* lg, const float* brs, int E, int k,
+                                             float scale, int t, int lane, int* sel, float* wsel,
+                                             int32_t* idx_out, float* w_out) {
+  int es[8];
+  float ss[8];
+  select_top_k(lg, brs, E, k, lane, es, ss);
+  store_selection(es, ss, k, scale, t, lane, sel, wsel, idx_out, w_out);
 }
 
 // Partial router logits of decode batches (T <= 8): 256 threads (8 warps)

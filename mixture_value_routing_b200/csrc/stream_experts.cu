@@ -284,8 +284,6 @@ stream_experts_kernel(const DT* __restrict__ x, const DT* __restrict__ Wv,
   }
   // Route mode: the consumer warps select and group the batch from the
   // partial logits (every CTA the same, in the same fixed order).
-  __shared__ float r_lg[kTok * 64];
-  __shared__ float r_br[64];
   __shared__ int r_sel[kTok * 8];
   __shared__ float r_w[kTok * 8];
   __shared__ int r_scratch[128];
@@ -296,32 +294,34 @@ stream_experts_kernel(const DT* __restrict__ x, const DT* __restrict__ Wv,
   const bool routing = route.part != nullptr;
   if (routing) {
     if (threadIdx.x < kConsumerWarps * 32) {
-      // Every load of the partials and biases is issued before the first is
-      // used (one L2 round trip): thread i sums logits i and i + 256 over the
-      // S <= kMaxLogitSplits ranges in range order.
-      constexpr int kC = kConsumerWarps * 32;
-      static_assert(kTok * 64 == 2 * kC, "two logits per consumer thread");
-      float pv[2][kMaxLogitSplits];
+      // Warp t selects token t straight from the partials: lane l loads
+      // experts l and l + 32 of every K range (all loads issued before the
+      // first is used: one L2 round trip) and sums them in range order.
+      static_assert(kTok <= kConsumerWarps, "a warp per token");
+      if (warp < T) {
+        float p0[kMaxLogitSplits], p1[kMaxLogitSplits];
 #pragma unroll
-      for (int h = 0; h < 2; ++h)
+        for (int r = 0; r < kMaxLogitSplits; ++r) {
+          const float* pr = route.part + (r * kTok + warp) * 64;
+          p0[r] = r < route.S ? __ldcg(pr + lane) : 0.f;
+          p1[r] = r < route.S ? __ldcg(pr + lane + 32) : 0.f;
+        }
+        const float b0 = lane < route.E ? route.br[lane] : 0.f;
+        const float b1 = lane + 32 < route.E ? route.br[lane + 32] : 0.f;
+        float l0 = p0[0], l1 = p1[0];
 #pragma unroll
-        for (int r = 0; r < kMaxLogitSplits; ++r)
-          pv[h][r] = (r < route.S && threadIdx.x + h * kC < T * 64)
-                         ? __ldcg(route.part + r * kTok * 64 + threadIdx.x + h * kC) : 0.f;
-      const float bv = threadIdx.x < route.E ? route.br[threadIdx.x] : 0.f;
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        float lv = pv[h][0];
-#pragma unroll
-        for (int r = 1; r < kMaxLogitSplits; ++r)
-          if (r < route.S) lv += pv[h][r];
-        r_lg[threadIdx.x + h * kC] = lv;
+        for (int r = 1; r < kMaxLogitSplits; ++r) {
+          if (r < route.S) {
+            l0 += p0[r];
+            l1 += p1[r];
+          }
+        }
+        int es[8];
+        float ss[8];
+        select_top_k_regs(l0, l1, b0, b1, route.E, k, lane, es, ss);
+        store_selection(es, ss, k, route.scale, warp, lane, r_sel, r_w,
+                        blockIdx.x == 0 ? route.idx_out : nullptr, route.w_out);
       }
-      if (threadIdx.x < 64) r_br[threadIdx.x] = bv;
-      consumers_sync();
-      if (warp < T)
-        select_token(&r_lg[warp * 64], r_br, route.E, k, route.scale, warp, lane, r_sel, r_w,
-                     blockIdx.x == 0 ? route.idx_out : nullptr, route.w_out);
       consumers_sync();
       // The selection is complete: the producer warp may derive the active
       // experts and start the weight stream while warp 0 groups the pairs.
