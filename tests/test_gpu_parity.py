@@ -373,6 +373,17 @@ def test_value_attend_32768_sparse(api):
     assert (err <= 1e-4 * np.maximum(1.0, np.abs(ref))).all(), err.max()
 
 
+def test_value_attend_zero_positions(api):
+    """No cached positions: o is zero (nothing to attend to)."""
+    Wv = P.dev(_layer(56, 256, 8, 256, "bf16").Wv, "bf16")
+    x = torch.empty((0, 256), dtype=torch.bfloat16, device="cuda")
+    idx = torch.empty((0, 2), dtype=torch.int32, device="cuda")
+    w = torch.empty((0, 2), dtype=torch.float32, device="cuda")
+    o = api.value_attend(x, idx, w, Wv, torch.empty((8, 0), dtype=torch.float32, device="cuda"))
+    torch.cuda.synchronize()
+    assert o.shape == (8, 128) and not o.any()
+
+
 def test_value_attend_deterministic(api):
     d, E, k, n, L, H = 2560, 64, 4, 1024, 3000, 32
     lay = _layer(54, d, E, n, "bf16")
