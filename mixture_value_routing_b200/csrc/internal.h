@@ -26,8 +26,6 @@ struct GroupOut {
   int32_t* pos;
   int32_t* active;
   StatusBlock* sb;
-  int32_t* tickets;  // per-row-block completion counters of the fused combine, zeroed
-  int ntickets;
   float* logits;     // decode routing: kMaxLogitSplits x 8 x 64 partial logits
 };
 
@@ -42,13 +40,13 @@ cudaError_t launch_router(const void* x, mova_dtype x_dt, const float* Wr, const
 
 // Decode routing in parts (T <= 8): the partial logits part[s][t][e] over S
 // K ranges (S chosen here, returned in *S_out; at most 4), which also starts
-// the call's status afresh and zeroes the tickets; then selection and
+// the call's status afresh; then selection and
 // grouping by one CTA.  The weight-streaming kernel can take the place of
 // the second part (RouteIn).
 constexpr int kMaxLogitSplits = 4;
 cudaError_t launch_router_logits(const void* x, mova_dtype x_dt, const float* Wr, int T, int d, int E,
-                                 int partitions, float* part, int* S_out, int32_t* tickets, int ntickets,
-                                 StatusBlock* sb, cudaStream_t stream);
+                                 int partitions, float* part, int* S_out, StatusBlock* sb,
+                                 cudaStream_t stream);
 cudaError_t launch_select_group(const float* part, int S, const float* br, int T, int E, int k, float scale,
                                 int32_t* idx, float* w, const GroupOut* g, cudaStream_t stream);
 // The number S of K ranges the decode partial logits use.
@@ -103,8 +101,7 @@ cudaError_t launch_split_router(const float* Wr, int E, int d, __nv_bfloat16* pl
 cudaError_t launch_permute(const void* idx_in, mova_dtype idx_dt, const void* w_in,
                            mova_dtype w_dt, int N, int E, int32_t* idx32, float* w32,
                            int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* pos,
-                           int32_t* active, StatusBlock* sb, int32_t* tickets, int ntickets,
-                           cudaStream_t stream);
+                           int32_t* active, StatusBlock* sb, cudaStream_t stream);
 
 // Multi-CTA grouping (batches above kSmallGroupT tokens).  Tiles of 128
 // tokens; tile_counts holds group_tiles(T) x 64 ints.  launch_tile_hist
@@ -117,15 +114,7 @@ cudaError_t launch_tile_hist(const void* idx_in, mova_dtype idx_dt, const void* 
                              int32_t* tile_counts, StatusBlock* sb, cudaStream_t stream);
 cudaError_t launch_tile_group(const int32_t* idx32, int T, int E, int k, int32_t* tile_counts,
                               int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* pos,
-                              int32_t* active, StatusBlock* sb, bool reset_status, int32_t* tickets,
-                              int ntickets, cudaStream_t stream);
-
-// Combine tickets a value call needs (zeroed by its grouping): one per
-// 8-column block, for the weight-streaming kernel's fused combine.
-inline int combine_tickets(int T, int n) {
-  (void)T;
-  return n / 8;
-}
+                              int32_t* active, StatusBlock* sb, bool reset_status, cudaStream_t stream);
 
 // Weight-streaming expert kernel: P[p, :] = SiLU(Wv[e] x[t]) for every
 // pair p (fp32 rows in grouped order).
@@ -150,8 +139,7 @@ struct RouteIn {
   int32_t* active_out;
   // One-launch decode (Wr non-null): the kernel first computes the partial
   // logits itself -- part[s][t][e] for the S K ranges, one (expert, range)
-  // per CTA -- into part_out (== part), resets the status and the combine
-  // tickets, and meets every other CTA at a grid barrier (slot bar_slot of
+  // per CTA -- into part_out (== part), resets the status, and meets every other CTA at a grid barrier (slot bar_slot of
   // the library's ring of barrier words) before it selects.
   const float* Wr;
   float* part_out;
@@ -177,23 +165,25 @@ struct StreamFault {
 };
 StreamFault take_stream_fault();
 
-// With tickets and v given (bf16, T <= 8 only), the kernel also performs
-// the combine: the CTA that completes a block of 8 output columns computes v
-// there; the caller then skips launch_combine.  tickets: n / 8 counters,
-// zeroed by the grouping of the same call.
+// In resident mode (bf16, T <= 8; see stream_resident) v must be given and
+// the kernel also performs the combine: each CTA owns a range of output
+// columns and writes v there; the caller then skips launch_combine (P is not
+// written).  Otherwise v is null.
 // ldw: rows of Wv between consecutive experts' first rows (>= n).
 cudaError_t launch_stream_experts(const void* x, const void* Wv, long long ldw, mova_dtype dt,
                                   const int32_t* counts,
                                   const int32_t* offsets, const int32_t* perm, const float* w32,
                                   const int32_t* active, StatusBlock* sb, int T, int d, int n,
-                                  int k, int E, float* P, int32_t* tickets, void* v,
-                                  const RouteIn& route, cudaStream_t stream);
+                                  int k, int E, float* P, void* v, const RouteIn& route,
+                                  cudaStream_t stream);
 
-// Shared memory the streaming kernel needs for rows of d elements (0 if d is
-// too long for two 8-row stages).
-size_t stream_experts_smem(int d, mova_dtype dt, int T, int* stages_out);
-// Whether the weight-streaming kernel keeps x in registers for this batch
-// (the mode in which it can also perform the combine).
+// Shared memory the streaming kernel needs for rows of d elements, n
+// outputs per token and k of E experts per token (0 if d is too long for two
+// 8-row stages).
+size_t stream_experts_smem(int d, mova_dtype dt, int T, int n, int k, int E, int* stages_out);
+// Whether the weight-streaming kernel keeps every token's x in shared memory
+// for this batch (the mode in which it also performs the combine: v must be
+// given).
 bool stream_resident(int T, int d, mova_dtype dt);
 
 // tcgen05 grouped GEMM (bf16): P[p, :] = SiLU(Wv[e] x[t]) as bf16 rows.

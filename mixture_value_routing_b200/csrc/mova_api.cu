@@ -78,7 +78,6 @@ struct Workspace {
   int32_t* active;
   int32_t* perm;
   int32_t* pos;
-  int32_t* tickets;
   float* logits;
   int32_t* tile_counts;
   __nv_bfloat16* planes;
@@ -101,7 +100,6 @@ Workspace layout(void* base, int T, int d, int k, int n) {
   w.active = reinterpret_cast<int32_t*>(b + o);       o += 256;
   w.perm = reinterpret_cast<int32_t*>(b + o);         o += align256(pairs * 4);
   w.pos = reinterpret_cast<int32_t*>(b + o);          o += align256(pairs * 4);
-  w.tickets = reinterpret_cast<int32_t*>(b + o);      o += align256(static_cast<size_t>(combine_tickets(T, n)) * 4);
   w.tile_counts = reinterpret_cast<int32_t*>(b + o);  o += align256(static_cast<size_t>(group_tiles(T)) * 64 * 4);
   w.planes = reinterpret_cast<__nv_bfloat16*>(b + o); o += align256(router_planes_bytes(d));
   // The decode partial logits (T <= 8, kMaxLogitSplits x 8 x 64 floats <= 192 * d * 2 bytes for
@@ -197,12 +195,12 @@ mova_status run_experts_and_combine(const void* x, mova_dtype dt, const void* Wv
                                   d, n, k, E, ws.xp, static_cast<__nv_bfloat16*>(ws.P), stream);
     }
   } else {
-    if (stream_experts_smem(d, dt, T, nullptr) == 0) return MOVA_ERR_UNSUPPORTED;
+    if (stream_experts_smem(d, dt, T, n, k, E, nullptr) == 0) return MOVA_ERR_UNSUPPORTED;
     // Decode-sized bf16 batches fold the combine into the expert kernel.
     fused_combine = T <= kFusedCombineMaxT && stream_resident(T, d, dt);
     err = launch_stream_experts(x, Wv, ldw, dt, ws.counts, ws.offsets, ws.perm, w32, ws.active, ws.sb,
                                 T, d, n, k, E, static_cast<float*>(ws.P),
-                                fused_combine ? ws.tickets : nullptr, fused_combine ? v : nullptr,
+                                fused_combine ? v : nullptr,
                                 RouteIn{}, stream);
   }
   if (err == cudaSuccess) err = mark(events, 3, stream);
@@ -288,10 +286,10 @@ mova_status mova_value_attend(const void* x, const void* idx, mova_dtype idx_dt,
     err = launch_tile_hist(idx, idx_dt, wgt, w_dt, L, E, k, w.idx, w.w, w.tile_counts, w.sb, s);
     if (err == cudaSuccess)
       err = launch_tile_group(w.idx, L, E, k, w.tile_counts, w.counts, w.offsets, w.perm, w.pos, w.active, w.sb,
-                              false, w.tickets, combine_tickets(L, n), s);
+                              false, s);
   } else {
     err = launch_permute(idx, idx_dt, wgt, w_dt, L * k, E, w.idx, w.w, w.counts, w.offsets, w.perm, w.pos,
-                         w.active, w.sb, w.tickets, combine_tickets(L, n), s);
+                         w.active, w.sb, s);
   }
   if (err == cudaSuccess) err = launch_gather_pairs(x, w.pos, L, d, k, w.xp, s);
   if (err == cudaSuccess)
@@ -350,11 +348,11 @@ mova_status mova_permute(const int32_t* idx, int T, int E, int k, int32_t* count
                                        w.tile_counts, w.sb, s);
     if (err == cudaSuccess)
       err = launch_tile_group(idx, T, E, k, w.tile_counts, counts, offsets, perm, pos, w.active, w.sb,
-                              false, nullptr, 0, s);
+                              false, s);
     return from_cuda(err);
   }
   return from_cuda(launch_permute(idx, MOVA_I32, nullptr, MOVA_F32, T * k, E, nullptr, nullptr,
-                                  counts, offsets, perm, pos, w.active, w.sb, nullptr, 0, s));
+                                  counts, offsets, perm, pos, w.active, w.sb, s));
 }
 
 mova_status mova_value_opts(const void* x, mova_dtype x_dt, const void* idx, mova_dtype idx_dt,
@@ -387,10 +385,10 @@ mova_status mova_value_opts(const void* x, mova_dtype x_dt, const void* idx, mov
       err = launch_tile_hist(idx, idx_dt, wgt, w_dt, T, E, k, w.idx, w.w, w.tile_counts, w.sb, s);
       if (err == cudaSuccess)
         err = launch_tile_group(w.idx, T, E, k, w.tile_counts, w.counts, w.offsets, w.perm, w.pos,
-                                w.active, w.sb, false, w.tickets, combine_tickets(T, n), s);
+                                w.active, w.sb, false, s);
     } else {
       err = launch_permute(idx, idx_dt, wgt, w_dt, T * k, E, w.idx, w.w, w.counts, w.offsets, w.perm,
-                           w.pos, w.active, w.sb, w.tickets, combine_tickets(T, n), s);
+                           w.pos, w.active, w.sb, s);
     }
   }
   if (err != cudaSuccess) return from_cuda(err);
@@ -439,21 +437,20 @@ mova_status mova_value_routed_opts(const void* x, mova_dtype x_dt, const float* 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   int32_t* idx = idx_out ? idx_out : w.idx;
   float* wgt = w_out ? w_out : w.w;
-  const GroupOut g{w.counts, w.offsets, w.perm, w.pos, w.active, w.sb, w.tickets, combine_tickets(T, n), w.logits};
+  const GroupOut g{w.counts, w.offsets, w.perm, w.pos, w.active, w.sb, w.logits};
   bool grouped = false;
   cudaError_t err = mark(events, 0, s);
   // Decode batches on the weight-streaming path: the router computes the
   // logits only; the streaming kernel selects, groups and combines.
   const mova_path rp = path == MOVA_PATH_AUTO ? mova_auto_path(T, x_dt) : path;
   if (rp == MOVA_PATH_STREAM && T <= kFusedCombineMaxT && stream_resident(T, d, x_dt) &&
-      stream_experts_smem(d, x_dt, T, nullptr) != 0) {
+      stream_experts_smem(d, x_dt, T, n, k, E, nullptr) != 0) {
     int S = 0;
     const bool one = o.decode_launches == 1;
     if (one) {
       S = decode_logit_splits(d, E, o.partitions);
     } else if (err == cudaSuccess) {
-      err = launch_router_logits(x, x_dt, Wr, T, d, E, o.partitions, w.logits, &S, w.tickets,
-                                 combine_tickets(T, n), w.sb, s);
+      err = launch_router_logits(x, x_dt, Wr, T, d, E, o.partitions, w.logits, &S, w.sb, s);
     }
     if (err == cudaSuccess) err = mark(events, 1, s);
     if (err == cudaSuccess) err = mark(events, 2, s);
@@ -462,7 +459,7 @@ mova_status mova_value_routed_opts(const void* x, mova_dtype x_dt, const float* 
                      one ? Wr : nullptr, w.logits, one ? next_grid_barrier_slot() : 0};
     if (err == cudaSuccess)
       err = launch_stream_experts(x, Wv, o.ldw, x_dt, w.counts, w.offsets, w.perm, wgt, w.active, w.sb, T, d,
-                                  n, k, E, static_cast<float*>(w.P), w.tickets, v, ri, s);
+                                  n, k, E, static_cast<float*>(w.P), v, ri, s);
     if (err == cudaSuccess) err = mark(events, 3, s);
     if (err == cudaSuccess) err = mark(events, 4, s);
     return from_cuda(err);
@@ -481,16 +478,16 @@ mova_status mova_value_routed_opts(const void* x, mova_dtype x_dt, const float* 
   if (err == cudaSuccess && !grouped) {
     if (tc_router) {
       err = launch_tile_group(idx, T, E, k, w.tile_counts, w.counts, w.offsets, w.perm, w.pos, w.active,
-                              w.sb, true, w.tickets, combine_tickets(T, n), s);
+                              w.sb, true, s);
     } else if (T > kSmallGroupT) {
       err = launch_tile_hist(idx, MOVA_I32, nullptr, MOVA_F32, T, E, k, nullptr, nullptr, w.tile_counts,
                              w.sb, s);
       if (err == cudaSuccess)
         err = launch_tile_group(idx, T, E, k, w.tile_counts, w.counts, w.offsets, w.perm, w.pos,
-                                w.active, w.sb, false, w.tickets, combine_tickets(T, n), s);
+                                w.active, w.sb, false, s);
     } else {
       err = launch_permute(idx, MOVA_I32, nullptr, MOVA_F32, T * k, E, nullptr, nullptr, w.counts,
-                           w.offsets, w.perm, w.pos, w.active, w.sb, w.tickets, combine_tickets(T, n), s);
+                           w.offsets, w.perm, w.pos, w.active, w.sb, s);
     }
   }
   if (err != cudaSuccess) return from_cuda(err);

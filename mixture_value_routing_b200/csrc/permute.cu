@@ -28,8 +28,7 @@ __global__ void __launch_bounds__(kPermThreads)
 permute_kernel(const IT* __restrict__ idx_in, const WT* __restrict__ w_in, int N, int E,
                int32_t* __restrict__ idx32, float* __restrict__ w32, int32_t* __restrict__ counts,
                int32_t* __restrict__ offsets, int32_t* __restrict__ perm, int32_t* __restrict__ pos,
-               int32_t* __restrict__ active, StatusBlock* sb, int32_t* __restrict__ tickets,
-               int ntickets) {
+               int32_t* __restrict__ active, StatusBlock* sb) {
   extern __shared__ uint8_t codes[];  // N expert codes
   __shared__ int hist[kPermWarps][64];
   __shared__ int tot[64];
@@ -46,7 +45,6 @@ permute_kernel(const IT* __restrict__ idx_in, const WT* __restrict__ w_in, int N
     sb->detail = 0;
     sb->work_next = 0;
   }
-  for (int i = tid; i < ntickets; i += kPermThreads) tickets[i] = 0;
   __syncthreads();
 
   const int seg = (N + kPermWarps - 1) / kPermWarps;
@@ -135,8 +133,7 @@ permute_kernel(const IT* __restrict__ idx_in, const WT* __restrict__ w_in, int N
 template <typename IT, typename WT>
 cudaError_t launch_t(const void* idx_in, const void* w_in, int N, int E, int32_t* idx32, float* w32,
                      int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* pos,
-                     int32_t* active, StatusBlock* sb, int32_t* tickets, int ntickets,
-                     cudaStream_t stream) {
+                     int32_t* active, StatusBlock* sb, cudaStream_t stream) {
   auto kern = permute_kernel<IT, WT>;
   const size_t smem = static_cast<size_t>(N);
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -145,8 +142,7 @@ cudaError_t launch_t(const void* idx_in, const void* w_in, int N, int E, int32_t
   note_launch();
   kern<<<1, kPermThreads, smem, stream>>>(static_cast<const IT*>(idx_in),
                                           static_cast<const WT*>(w_in), N, E, idx32, w32, counts,
-                                          offsets, perm, pos, active, sb, tickets,
-                                          tickets ? ntickets : 0);
+                                          offsets, perm, pos, active, sb);
   return cudaGetLastError();
 }
 
@@ -198,11 +194,8 @@ __global__ void __launch_bounds__(128)
 tile_scatter_kernel(const int32_t* __restrict__ idx32, int N, int k, int E,
                     const int32_t* __restrict__ tile_counts, int ntiles, int32_t* __restrict__ counts,
                     int32_t* __restrict__ offsets, int32_t* __restrict__ active, StatusBlock* sb,
-                    bool reset_status, int32_t* __restrict__ perm, int32_t* __restrict__ pos,
-                    int32_t* __restrict__ tickets, int ntickets) {
+                    bool reset_status, int32_t* __restrict__ perm, int32_t* __restrict__ pos) {
   pdl_wait();
-  // The combine tickets of this call start at zero.
-  for (int i = blockIdx.x * 128 + threadIdx.x; i < ntickets; i += gridDim.x * 128) tickets[i] = 0;
   __shared__ int hist[4][64];
   __shared__ int base[64];
   __shared__ int tot_s[64];
@@ -306,22 +299,21 @@ cudaError_t launch_hist_t(const void* idx_in, const void* w_in, int N, int E, in
 cudaError_t launch_permute(const void* idx_in, mova_dtype idx_dt, const void* w_in,
                            mova_dtype w_dt, int N, int E, int32_t* idx32, float* w32,
                            int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* pos,
-                           int32_t* active, StatusBlock* sb, int32_t* tickets, int ntickets,
-                           cudaStream_t stream) {
+                           int32_t* active, StatusBlock* sb, cudaStream_t stream) {
   if (N <= 0 || N > kMaxPairs) return cudaErrorInvalidValue;
   if (w_in == nullptr) w32 = nullptr;
   if (idx_dt == MOVA_I8) {
     if (w_dt == MOVA_F16)
       return launch_t<int8_t, __half>(idx_in, w_in, N, E, idx32, w32, counts, offsets, perm, pos,
-                                      active, sb, tickets, ntickets, stream);
+                                      active, sb, stream);
     return launch_t<int8_t, float>(idx_in, w_in, N, E, idx32, w32, counts, offsets, perm, pos,
-                                   active, sb, tickets, ntickets, stream);
+                                   active, sb, stream);
   }
   if (w_dt == MOVA_F16)
     return launch_t<int32_t, __half>(idx_in, w_in, N, E, idx32, w32, counts, offsets, perm, pos,
-                                     active, sb, tickets, ntickets, stream);
+                                     active, sb, stream);
   return launch_t<int32_t, float>(idx_in, w_in, N, E, idx32, w32, counts, offsets, perm, pos,
-                                  active, sb, tickets, ntickets, stream);
+                                  active, sb, stream);
 }
 
 }  // namespace mova
@@ -350,13 +342,12 @@ cudaError_t launch_tile_hist(const void* idx_in, mova_dtype idx_dt, const void* 
 
 cudaError_t launch_tile_group(const int32_t* idx32, int T, int E, int k, int32_t* tile_counts,
                               int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* pos,
-                              int32_t* active, StatusBlock* sb, bool reset_status, int32_t* tickets,
-                              int ntickets, cudaStream_t stream) {
+                              int32_t* active, StatusBlock* sb, bool reset_status, cudaStream_t stream) {
   const int N = T * k;
   const int ntiles = group_tiles(T);
   return launch_pdl(tile_scatter_kernel, dim3(ntiles), dim3(128), 0, stream, idx32, N, k, E,
                     static_cast<const int32_t*>(tile_counts), ntiles, counts, offsets, active, sb,
-                    reset_status, perm, pos, tickets, tickets ? ntickets : 0);
+                    reset_status, perm, pos);
 }
 
 }  // namespace mova

@@ -152,8 +152,7 @@ router_kernel(const XT* __restrict__ x, const float* __restrict__ Wr, const floa
 // warp butterfly leaves each token's warp sum in one lane group; the warps'
 // sums are added in warp order and stored as part[s][t][e].  Every step has a
 // fixed order, so the logits do not depend on timing.  The CTA of (expert 0,
-// range 0) also starts the call's status afresh and zeroes the fused
-// combine's row-block tickets.
+// range 0) also starts the call's status afresh.
 //
 // The selection and grouping that follow (select_token, group_pairs_warp)
 // run either in select_group_kernel (one CTA) or at the start of the
@@ -165,8 +164,7 @@ constexpr int kLogitThreads = kPartThreads;
 template <typename XT>
 __global__ void __launch_bounds__(kLogitThreads)
 router_logits_kernel(const float* __restrict__ Wr, const XT* __restrict__ x, int T, int d, int E,
-                     float* __restrict__ part, int32_t* __restrict__ tickets, int ntickets,
-                     StatusBlock* __restrict__ sb) {
+                     float* __restrict__ part, StatusBlock* __restrict__ sb) {
   __shared__ float red[kLogitThreads / 32][kDecT];
   const int e = blockIdx.x % E;
   const int s = blockIdx.x / E;
@@ -185,13 +183,10 @@ router_logits_kernel(const float* __restrict__ Wr, const XT* __restrict__ x, int
   if (c0 < ce) load8(wrow + 8 * c0, w0);
   pdl_wait();  // x may come from the previous kernel; every output is written after this
   pdl_trigger();
-  if (blockIdx.x == 0) {
-    if (tid == 0 && sb != nullptr) {
-      sb->code = 0;
-      sb->detail = 0;
-      sb->work_next = 0;
-    }
-    for (int i = tid; i < ntickets; i += kLogitThreads) tickets[i] = 0;
+  if (blockIdx.x == 0 && tid == 0 && sb != nullptr) {
+    sb->code = 0;
+    sb->detail = 0;
+    sb->work_next = 0;
   }
 
   partial_logits_warp(wrow, x, T, d, c0, ce, w0, lane, warp, &red[0][0]);
@@ -255,9 +250,9 @@ cudaError_t launch_router_t(const void* x, const float* Wr, const float* br, int
 
 template <typename XT>
 cudaError_t launch_logits_t(const void* x, const float* Wr, int T, int d, int E, int S, float* part,
-                            int32_t* tickets, int ntickets, StatusBlock* sb, cudaStream_t stream) {
+                            StatusBlock* sb, cudaStream_t stream) {
   return launch_pdl(router_logits_kernel<XT>, dim3(static_cast<unsigned>(E * S)), dim3(kLogitThreads), 0,
-                    stream, Wr, static_cast<const XT*>(x), T, d, E, part, tickets, ntickets, sb);
+                    stream, Wr, static_cast<const XT*>(x), T, d, E, part, sb);
 }
 
 }  // namespace
@@ -269,8 +264,7 @@ cudaError_t launch_router(const void* x, mova_dtype x_dt, const float* Wr, const
   if (T <= 0) return cudaSuccess;
   if (T <= kFusedRouterMaxT && g != nullptr && g->logits != nullptr) {
     int S = 0;
-    cudaError_t err = launch_router_logits(x, x_dt, Wr, T, d, E, partitions, g->logits, &S, g->tickets,
-                                           g->ntickets, g->sb, stream);
+    cudaError_t err = launch_router_logits(x, x_dt, Wr, T, d, E, partitions, g->logits, &S, g->sb, stream);
     if (err != cudaSuccess) return err;
     if (grouped) *grouped = true;
     return launch_select_group(g->logits, S, br, T, E, k, scale, idx, w, g, stream);
@@ -305,13 +299,13 @@ int logit_splits(int d, int E) {
 int decode_logit_splits(int d, int E, int partitions) { return partitions == 2 ? 2 : logit_splits(d, E); }
 
 cudaError_t launch_router_logits(const void* x, mova_dtype x_dt, const float* Wr, int T, int d, int E,
-                                 int partitions, float* part, int* S_out, int32_t* tickets, int ntickets,
-                                 StatusBlock* sb, cudaStream_t stream) {
+                                 int partitions, float* part, int* S_out, StatusBlock* sb,
+                                 cudaStream_t stream) {
   if (T <= 0 || T > kDecT) return cudaErrorInvalidValue;
   const int S = decode_logit_splits(d, E, partitions);
   *S_out = S;
-  return x_dt == MOVA_BF16 ? launch_logits_t<__nv_bfloat16>(x, Wr, T, d, E, S, part, tickets, ntickets, sb, stream)
-                           : launch_logits_t<float>(x, Wr, T, d, E, S, part, tickets, ntickets, sb, stream);
+  return x_dt == MOVA_BF16 ? launch_logits_t<__nv_bfloat16>(x, Wr, T, d, E, S, part, sb, stream)
+                           : launch_logits_t<float>(x, Wr, T, d, E, S, part, sb, stream);
 }
 
 cudaError_t launch_select_group(const float* part, int S, const float* br, int T, int E, int k, float scale,

@@ -9,22 +9,29 @@
 //
 // At a few tokens per expert this is a matrix-vector product per active
 // expert and HBM-bound: each active expert's n x d weight is read exactly
-// once.  The rows of all active experts, concatenated, are split evenly over
-// one persistent CTA per SM.  In each CTA a producer warp streams 8-row slabs
-// (contiguous bytes of one expert) into a ring of 4 shared-memory stages with
-// 1-D bulk (TMA) copies completing on mbarriers (lanes 0-7 issue a stage's
-// eight row copies together), so each SM keeps ~160 KB of weights in flight
-// without spending registers on it.  Eight consumer warps split K, run
-// mma.sync m16n8k16 on (8 weight rows) x (8 token columns), and reduce the
-// partial tiles in warp order; a slab's 8 x 8 results go to P.
+// once, by one persistent CTA per SM.  In each CTA a producer warp streams
+// 8-row slabs into a ring of 4 shared-memory stages with 1-D bulk (TMA)
+// copies completing on mbarriers (lanes 0-7 issue a stage's eight row copies
+// together), so each SM keeps ~160 KB of weights in flight without spending
+// registers on it.  Eight consumer warps split K and run mma.sync m16n8k16
+// on (8 weight rows) x (8 token columns).
 //
-// Decode batches (bf16, T <= 8) keep every token's x in shared memory, and
-// with RouteIn the kernel also routes them itself: each CTA sums the router's
-// partial logits, selects (route_select.cuh) and groups in shared memory.
-// With the combine fused in, slabs run row-block-major and the CTA that
-// completes a block of 8 output columns (per-block tickets) writes v there.
+// Decode batches (bf16, T <= 8; resident mode) keep every token's x in
+// shared memory, and with RouteIn the kernel also routes them itself: each
+// CTA sums the router's partial logits, selects (route_select.cuh) and
+// groups in shared memory.  The combine is fused in: each CTA owns a range
+// of output columns (about n / CTAs) and streams those rows of every active
+// expert, concatenated, in full 8-row slabs (a slab may span two experts:
+// the mma computes every row against every token anyway).  A reducer warp
+// sums the consumers' partial tiles in warp order and keeps the slab's
+// SiLU(8 x 8) tile in shared memory as it is; at the end it sums the slots
+// of every token for its columns, so nothing leaves the CTA but v.
+// Otherwise (fp32, or more tokens) the rows of all active experts, in whole
+// slabs of one expert, are split evenly over the CTAs, the consumers reduce
+// each slab's partial tiles themselves and its results go to P.
 // Every wait is bounded; a wait that runs out sets MOVA_ERR_TIMEOUT in the
 // status block and the CTA drains its copies and exits.
+#include <algorithm>
 #include <atomic>
 
 #include "common.cuh"
@@ -116,18 +123,6 @@ __device__ __forceinline__ void consumers_sync() {
   asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");
 }
 
-// Consumer-group barrier that also ORs a predicate over the group's threads.
-__device__ __forceinline__ bool consumers_any(bool v) {
-  uint32_t r;
-  asm volatile(
-      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.or.pred q, 1, %2, p;\n\t"
-      "selp.u32 %0, 1, 0, q;\n\t}"
-      : "=r"(r)
-      : "r"(static_cast<uint32_t>(v)), "n"(kConsumerWarps * 32)
-      : "memory");
-  return r != 0;
-}
-
 // Grid-wide barrier of a launch whose CTAs are all resident (one per SM):
 // CTA 0 adds 2^31 - (G - 1) to the word and every other CTA adds 1, so the
 // word's top bit flips exactly when the last CTA arrives, whatever the order
@@ -163,7 +158,7 @@ stream_experts_kernel(const DT* __restrict__ x, const DT* __restrict__ Wv,
                       const int32_t* __restrict__ perm, const float* __restrict__ w32,
                       const int32_t* __restrict__ active, StatusBlock* __restrict__ sb, int T,
                       int d, int n, int k, float* __restrict__ P, int NS,
-                      int32_t* __restrict__ tickets, DT* __restrict__ v, RouteIn route,
+                      DT* __restrict__ v, RouteIn route,
                       StreamFault fault, long long ldw) {
   constexpr bool kMma = sizeof(DT) == 2;
   constexpr int EL = Vec<DT>::EL;
@@ -183,21 +178,19 @@ stream_experts_kernel(const DT* __restrict__ x, const DT* __restrict__ Wv,
   // kernel (the mma computes all 8 token columns for every expert; each pair
   // reads its token's column), and the pair tables below replace all global
   // loads of the grouping in the loop.
-  int* pair_tok = tok_p + kTok;          // [64] token of each grouped position
-  float* pair_w = reinterpret_cast<float*>(pair_tok + 64);  // [64] its weight
-  int* act_cnt = reinterpret_cast<int*>(pair_w + 64);       // [64] pairs per active expert
+  int* slot_act = tok_p + kTok;                             // [64] active-list index of pair f's expert
+  int* act_cnt = slot_act + 64;                             // [64] pairs per active expert
   int* act_off = act_cnt + 64;                              // [64] first position
-  int* slot_pos = act_off + 64;                             // [64] grouped position of pair f
-  float* slot_w = reinterpret_cast<float*>(slot_pos + 64);  // [64] weight of pair f
+  float* slot_w = reinterpret_cast<float*>(act_off + 64);  // [64] weight of pair f
   uint64_t* full = reinterpret_cast<uint64_t*>(slot_w + 64);
   uint64_t* empty = full + kMaxStages;
   uint64_t* xbar = empty + kMaxStages;  // resident x rows landed
   uint64_t* partb = xbar + 2;           // [kMaxStages] resident: a stage's 8 partial tiles are in red
-  float* hred = reinterpret_cast<float*>(partb + kMaxStages);  // [8][8] the reducer's summed tile
-  int* act = reinterpret_cast<int*>(hred + 64);
+  int* act = reinterpret_cast<int*>(partb + kMaxStages);
   volatile int* abort_flag = act + 64;
   int* issued = act + 65;
-  int* blk_tick = act + 66;  // [64] completion counts of this CTA's row blocks (fused combine)
+  // Resident mode: the SiLU values of this CTA's rows, [flat row][token].
+  float* hv = reinterpret_cast<float*>(act + 68);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -240,7 +233,7 @@ stream_experts_kernel(const DT* __restrict__ x, const DT* __restrict__ Wv,
   }
   if (one_launch) {
     // The partial logits of this call (the part of the logits kernel of the
-    // two-launch path), then the status and tickets reset, then one grid
+    // two-launch path), then the status reset, then one grid
     // barrier: after it every CTA reads all of them.
     __shared__ int gb_ok;
     float* lred = red;  // free until the weight stream starts
@@ -265,13 +258,10 @@ stream_experts_kernel(const DT* __restrict__ x, const DT* __restrict__ Wv,
         consumers_sync();
       }
     }
-    if (blockIdx.x == 0) {
-      if (threadIdx.x == 0) {
-        sb->code = 0;
-        sb->detail = 0;
-        sb->work_next = 0;
-      }
-      for (int i = threadIdx.x; i < n / kRowsPerStage; i += kThreads) tickets[i] = 0;
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+      sb->code = 0;
+      sb->detail = 0;
+      sb->work_next = 0;
     }
     if (!grid_barrier(&g_grid_bar[route.bar_slot], fault.wait_limit, fault.skip_barrier && blockIdx.x == 0,
                       &gb_ok)) {
@@ -379,19 +369,21 @@ stream_experts_kernel(const DT* __restrict__ x, const DT* __restrict__ Wv,
   const int* act_p = routing && warp == kProducerWarp ? p_act : act;
   pdl_trigger();
 
-  // Rows of all active experts, in units of whole stages (n % 8 == 0, so a
-  // stage never straddles two experts), split evenly over the CTAs.  With
-  // the combine fused in (v given; only in resident mode), units run
-  // row-block-major -- unit u is row block u / nact of active expert
-  // u % nact -- so a row block's units sit in one or two neighbouring CTAs
-  // and the one that completes it last also combines it: it owns every
-  // slot's expert row for those 8 output columns.  Otherwise units run
-  // expert-major, so the staged x rows change only with the expert.
-  const bool fused = v != nullptr;
+  // Resident mode (the combine fused in): this CTA owns output columns
+  // [r_lo, r_lo + nr).  Its rows are those columns of every active expert in
+  // turn -- flat row f is column r_lo + f % nr of active expert f / nr --
+  // and stage j holds flat rows 8j .. 8j + 7.
+  // Otherwise the rows of all active experts, in units of whole stages
+  // (n % 8 == 0, so a stage never straddles two experts), are split evenly
+  // over the CTAs, expert-major, so the staged x rows change only with the
+  // expert.
   const int units_per_expert = n / kRowsPerStage;
-  const int units = nact * units_per_expert;
-  const int u0 = static_cast<int>(static_cast<long long>(units) * blockIdx.x / gridDim.x);
-  const int u1 = static_cast<int>(static_cast<long long>(units) * (blockIdx.x + 1) / gridDim.x);
+  const int r_lo = static_cast<int>(static_cast<long long>(n) * blockIdx.x / gridDim.x);
+  const int nr = static_cast<int>(static_cast<long long>(n) * (blockIdx.x + 1) / gridDim.x) - r_lo;
+  const int rows_total = nact * nr;
+  const int units = resident ? (rows_total + kRowsPerStage - 1) / kRowsPerStage : nact * units_per_expert;
+  const int u0 = resident ? 0 : static_cast<int>(static_cast<long long>(units) * blockIdx.x / gridDim.x);
+  const int u1 = resident ? units : static_cast<int>(static_cast<long long>(units) * (blockIdx.x + 1) / gridDim.x);
   const int nstages = u1 - u0;
 
   if (warp == kProducerWarp) {
@@ -399,8 +391,6 @@ stream_experts_kernel(const DT* __restrict__ x, const DT* __restrict__ Wv,
     // bytes, then lanes 0-7 issue one row copy each, so a stage's eight
     // copies leave at once.  The unit's expert and row advance incrementally.
     const uint64_t pol = policy_evict_first();
-    int a = fused ? u0 % max(nact, 1) : u0 / units_per_expert;
-    int rb = fused ? u0 / max(nact, 1) : u0 - a * units_per_expert;  // row block
     int s = 0;
     uint32_t phase = 0;
     int j = 0;
@@ -417,19 +407,25 @@ stream_experts_kernel(const DT* __restrict__ x, const DT* __restrict__ Wv,
       // Test-only injection: CTA 0 stops issuing here, so the consumers'
       // wait for this stage must run out.
       if (j == fault.stall_stage && blockIdx.x == 0) break;
-      const DT* src = Wv + (static_cast<size_t>(act_p[a]) * ldw + rb * kRowsPerStage) * d;
-      uint8_t* dst = stages + s * stage_bytes;
-      if (lane == 0) mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(kRowsPerStage * row_bytes));
-      __syncwarp();
-      if (lane < kRowsPerStage)
-        bulk_g2s(dst + lane * pitch, src + static_cast<size_t>(lane) * d, static_cast<uint32_t>(row_bytes),
-                 &full[s], pol);
-      __syncwarp();
-      if (fused) {
-        if (++a == nact) { a = 0; ++rb; }
+      // This lane's row of the stage: active expert a, row r.
+      int nrows = kRowsPerStage, a, r;
+      if (resident) {
+        const int f = j * kRowsPerStage + lane;
+        nrows = min(kRowsPerStage, rows_total - j * kRowsPerStage);
+        a = f / max(nr, 1);
+        r = r_lo + (f - a * nr);
       } else {
-        if (++rb == units_per_expert) { rb = 0; ++a; }
+        const int u = u0 + j;
+        a = u / units_per_expert;
+        r = (u - a * units_per_expert) * kRowsPerStage + lane;
       }
+      uint8_t* dst = stages + s * stage_bytes;
+      if (lane == 0) mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(nrows * row_bytes));
+      __syncwarp();
+      if (lane < nrows)
+        bulk_g2s(dst + lane * pitch, Wv + (static_cast<size_t>(act_p[a]) * ldw + r) * d,
+                 static_cast<uint32_t>(row_bytes), &full[s], pol);
+      __syncwarp();
       if (++s == NS) { s = 0; phase ^= 1; }
     }
     if (lane == 0) *issued = j;
@@ -438,11 +434,10 @@ stream_experts_kernel(const DT* __restrict__ x, const DT* __restrict__ Wv,
       // Resident mode: the consumer warps hand each stage's partial tiles
       // (their K slices of 8 weight rows x 8 token columns) over through an
       // mbarrier instead of meeting at a block barrier; this warp sums them
-      // in warp order, applies SiLU, stores the rows of every pair of the
-      // stage's expert, and frees the stage.  It takes every stage, even
-      // after a failure (then storing nothing), so the stage ring stays in
-      // step.
-      int cur_a = -1, cnt = 0, off = 0;
+      // in warp order, applies SiLU, keeps the stage's rows of every pair of
+      // its expert, and frees the stage.  It takes every stage, even after a
+      // failure (then keeping nothing), so the stage ring stays in step.
+      bool all_ok = true;
       for (int j = 0; j < nstages; ++j) {
         const int s = j % NS;
         bool ok = *abort_flag == 0;
@@ -454,15 +449,9 @@ stream_experts_kernel(const DT* __restrict__ x, const DT* __restrict__ Wv,
           }
         }
         ok = __all_sync(0xffffffffu, ok);
-        const int u = u0 + j;
-        const int a = fused ? u % nact : u / units_per_expert;
-        const int r0 = (fused ? u / nact : u - a * units_per_expert) * kRowsPerStage;
-        if (a != cur_a) {
-          cur_a = a;
-          cnt = act_cnt[a];
-          off = act_off[a];
-        }
+        all_ok = all_ok && ok;
         if (ok) {
+          // Stage row q (flat row 8j + q), token column c: hv[(8j + q) * 8 + c].
           const float* rb = red + s * (kConsumerWarps * 64);
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
@@ -470,22 +459,29 @@ stream_experts_kernel(const DT* __restrict__ x, const DT* __restrict__ Wv,
             float acc = 0.f;
 #pragma unroll
             for (int w = 0; w < kConsumerWarps; ++w) acc += rb[w * 64 + e];
-            hred[e] = siluf_(acc);
+            hv[j * 64 + e] = siluf_(acc);
           }
-          __syncwarp();
-          for (int e = lane; e < cnt * kRowsPerStage; e += 32) {
-            const int p = off + e / kRowsPerStage;
-            const int row = e % kRowsPerStage;
-            P[static_cast<size_t>(p) * n + r0 + row] = hred[row * 8 + pair_tok[p]];
-          }
-          __syncwarp();
         }
+        __syncwarp();
         if (lane == 0) mbar_arrive(&empty[s]);
       }
-      // This warp's rows of P are complete: the consumers' fused combine
-      // reads them after the barrier below.
-      __threadfence();
-      asm volatile("bar.sync 2, %0;" ::"n"((kConsumerWarps + 1) * 32) : "memory");
+      // Every stage of every active expert is in (a role that failed set the
+      // abort flag before its last arrival, so it is seen here): the combine
+      // for this CTA's columns,
+      //   v[t, r] = sum over slots (ascending) of w[t, slot] * SiLU value,
+      // the same fmaf chain as the separate combine pass.
+      if (all_ok && *abort_flag == 0) {
+        for (int i = lane; i < T * nr; i += 32) {
+          const int t = i / nr;
+          const int r = i - t * nr;
+          float acc = 0.f;
+          for (int sl = 0; sl < k; ++sl) {
+            const int f = t * k + sl;
+            acc = fmaf(slot_w[f], hv[(slot_act[f] * nr + r) * 8 + t], acc);
+          }
+          v[static_cast<size_t>(t) * n + r_lo + r] = from_f32<DT>(acc);
+        }
+      }
     }
   } else {
     int cur_a = -1, cnt = 0, off = 0;
@@ -497,17 +493,14 @@ stream_experts_kernel(const DT* __restrict__ x, const DT* __restrict__ Wv,
     if (resident) {
       // Pair tables, while x and the first weight stages are in flight.
       const int N = T * k;
-      if (threadIdx.x < N) {
-        const int f = routing ? r_perm[threadIdx.x] : perm[threadIdx.x];
-        const float wf = routing ? r_w[f] : w32[f];
-        pair_tok[threadIdx.x] = f / k;
-        pair_w[threadIdx.x] = wf;
-        slot_pos[f] = threadIdx.x;
-        slot_w[f] = wf;
-      }
+      if (threadIdx.x < N) slot_w[threadIdx.x] = routing ? r_w[threadIdx.x] : w32[threadIdx.x];
       if (threadIdx.x < nact) {
-        act_cnt[threadIdx.x] = routing ? r_cnt[act[threadIdx.x]] : counts[act[threadIdx.x]];
-        act_off[threadIdx.x] = routing ? r_off[act[threadIdx.x]] : offsets[act[threadIdx.x]];
+        const int e = act[threadIdx.x];
+        const int cnt_e = routing ? r_cnt[e] : counts[e];
+        const int off_e = routing ? r_off[e] : offsets[e];
+        act_cnt[threadIdx.x] = cnt_e;
+        act_off[threadIdx.x] = off_e;
+        for (int i = 0; i < cnt_e; ++i) slot_act[routing ? r_perm[off_e + i] : perm[off_e + i]] = threadIdx.x;
       }
       if (!mbar_wait_or_abort(xbar, 0, abort_flag, fault.wait_limit)) {
         raise_status(sb, MOVA_ERR_TIMEOUT, blockIdx.x);
@@ -531,14 +524,6 @@ stream_experts_kernel(const DT* __restrict__ x, const DT* __restrict__ Wv,
         }
       }
       ok = __all_sync(0xffffffffu, ok);
-      const int u = u0 + j;
-      const int a = fused ? u % nact : u / units_per_expert;
-      const int r0 = (fused ? u / nact : u - a * units_per_expert) * kRowsPerStage;
-      if (a != cur_a) {
-        cur_a = a;
-        cnt = resident ? act_cnt[a] : counts[act[a]];
-        off = resident ? act_off[a] : offsets[act[a]];
-      }
       const uint8_t* wst = stages + s * stage_bytes;
       if constexpr (kMma) {
         if (resident) {
@@ -585,6 +570,13 @@ stream_experts_kernel(const DT* __restrict__ x, const DT* __restrict__ Wv,
           if (lane == 0) mbar_arrive(&partb[s]);
           continue;  // the reducer frees the stage
         }
+      }
+      const int a = (u0 + j) / units_per_expert;
+      const int r0 = (u0 + j - a * units_per_expert) * kRowsPerStage;
+      if (a != cur_a) {
+        cur_a = a;
+        cnt = counts[act[a]];
+        off = offsets[act[a]];
       }
       for (int c0 = 0; c0 < cnt; c0 += kTok) {
         const int nt = min(kTok, cnt - c0);
@@ -641,7 +633,7 @@ stream_experts_kernel(const DT* __restrict__ x, const DT* __restrict__ Wv,
             const int row = threadIdx.x >> 3;
             const int t = threadIdx.x & 7;
             if (t < nt) {
-              const int col = resident ? pair_tok[off + c0 + t] : t;  // the pair's token column
+              const int col = t;  // the pair's token column
               float h = 0.f;
 #pragma unroll
               for (int w = 0; w < kConsumerWarps; ++w) h += rb[(w * 8 + row) * 8 + col];
@@ -694,46 +686,6 @@ stream_experts_kernel(const DT* __restrict__ x, const DT* __restrict__ Wv,
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[s]);
     }
-    // Resident mode: wait until the reducer has stored this CTA's rows of P.
-    if (resident) asm volatile("bar.sync 2, %0;" ::"n"((kConsumerWarps + 1) * 32) : "memory");
-    // The consumer warps agree (one bar.red) on whether any role failed: if
-    // so, nothing is combined; otherwise every warp takes the same path.
-    if (fused && nstages > 0 && !consumers_any(*abort_flag != 0)) {
-      // Fused combine.  This CTA's rows of P are complete: publish them, then
-      // count them on the tickets of the row blocks they belong to; the CTA
-      // that completes a block's count sums the slots of every token for its
-      // 8 columns,
-      //   v[t, r] = sum over slots (ascending) of w[t, slot] * P[pos[t, slot], r].
-      // Done once at the end, so the weight stream never waits for it.
-      __threadfence();
-      consumers_sync();
-      const int jb = u0 / nact;
-      const int je = (u1 - 1) / nact;
-      for (int j0 = jb; j0 <= je; j0 += 64) {
-        const int nb = min(64, je - j0 + 1);
-        if (threadIdx.x < nb) {
-          const int jj = j0 + threadIdx.x;
-          const int done = min(u1, (jj + 1) * nact) - max(u0, jj * nact);
-          blk_tick[threadIdx.x] = atomicAdd(&tickets[jj], done) + done;
-        }
-        consumers_sync();
-        __threadfence();
-        for (int i = threadIdx.x; i < nb * kTok * kRowsPerStage; i += kConsumerWarps * 32) {
-          const int bi = i / (kTok * kRowsPerStage);
-          const int t = (i / kRowsPerStage) % kTok;
-          const int row = i % kRowsPerStage;
-          if (blk_tick[bi] != nact || t >= T) continue;
-          const int col = (j0 + bi) * kRowsPerStage + row;
-          float acc = 0.f;
-          for (int sl = 0; sl < k; ++sl) {
-            const float pv = __ldcg(P + static_cast<size_t>(slot_pos[t * k + sl]) * n + col);
-            acc = fmaf(slot_w[t * k + sl], pv, acc);
-          }
-          v[static_cast<size_t>(t) * n + col] = from_f32<DT>(acc);
-        }
-        consumers_sync();
-      }
-    }
   }
   __syncthreads();
   // No bulk copy may still be writing this CTA's shared memory at exit: wait
@@ -760,18 +712,26 @@ cudaError_t reset_grid_barriers(cudaStream_t stream) {
   return cudaMemsetAsync(p, 0, sizeof(g_grid_bar), stream);
 }
 
-size_t stream_experts_smem(int d, mova_dtype dt, int T, int* stages_out) {
+size_t stream_experts_smem(int d, mova_dtype dt, int T, int n, int k, int E, int* stages_out) {
   const bool mma = dt == MOVA_BF16;
-  (void)T;
+  // Resident mode: the SiLU values of a CTA's rows (its ceil(n / CTAs)
+  // columns of each of at most min(E, T k) active experts, in whole
+  // stages) for all 8 token columns.
+  const int G = sm_count();
+  const size_t rows = static_cast<size_t>(std::min(E, T * k)) * ((n + G - 1) / G);
+  const size_t hv_bytes =
+      is_resident(mma, T) ? (rows + kRowsPerStage - 1) / kRowsPerStage * kRowsPerStage * kTok * sizeof(float) : 0;
   const size_t pitch = static_cast<size_t>(d) * (mma ? 2 : 4) + 16;
   const size_t stage_bytes = pitch * kRowsPerStage;
-  const size_t budget = 220 * 1024;
+  // With the kernel's ~2.4 KB of static arrays, under the 227 KB a block
+  // may opt in to.
+  const size_t budget = 222 * 1024;
   // The most stages (up to kStreamStages) that fit next to the fixed parts,
   // whose partial-tile buffers grow with the stage count.
   for (int NS = kStreamStages; NS >= 2; --NS) {
     const size_t fixed = (mma ? kTok * pitch + red_slots(NS) * kConsumerWarps * 64 * sizeof(float) : 0) +
-                         2 * kTok * sizeof(float) + 6 * 64 * sizeof(int) +
-                         (3 * kMaxStages + 2) * sizeof(uint64_t) + 64 * sizeof(float) + 130 * sizeof(int);
+                         2 * kTok * sizeof(float) + 4 * 64 * sizeof(int) +
+                         (3 * kMaxStages + 2) * sizeof(uint64_t) + 68 * sizeof(int) + hv_bytes;
     if (NS * stage_bytes + fixed <= budget) {
       if (stages_out) *stages_out = NS;
       return NS * stage_bytes + fixed;
@@ -790,12 +750,13 @@ cudaError_t launch_stream_experts(const void* x, const void* Wv, long long ldw, 
                                   const int32_t* counts,
                                   const int32_t* offsets, const int32_t* perm, const float* w32,
                                   const int32_t* active, StatusBlock* sb, int T, int d, int n,
-                                  int k, int E, float* P, int32_t* tickets, void* v,
-                                  const RouteIn& route, cudaStream_t stream) {
-  (void)E;
+                                  int k, int E, float* P, void* v, const RouteIn& route,
+                                  cudaStream_t stream) {
   int NS = 0;
-  const size_t smem = stream_experts_smem(d, dt, T, &NS);
+  const size_t smem = stream_experts_smem(d, dt, T, n, k, E, &NS);
   if (smem == 0) return cudaErrorInvalidValue;
+  // Resident mode always combines inside the kernel.
+  if (is_resident(dt == MOVA_BF16, T) && v == nullptr) return cudaErrorInvalidValue;
   const dim3 grid(sm_count());
   const StreamFault fault = take_stream_fault();
   if (dt == MOVA_BF16) {
@@ -805,7 +766,7 @@ cudaError_t launch_stream_experts(const void* x, const void* Wv, long long ldw, 
     if (err != cudaSuccess) return err;
     return launch_pdl(kern, grid, dim3(kThreads), smem, stream,
                       static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(Wv),
-                      counts, offsets, perm, w32, active, sb, T, d, n, k, P, NS, tickets,
+                      counts, offsets, perm, w32, active, sb, T, d, n, k, P, NS,
                       static_cast<__nv_bfloat16*>(v), route, fault, ldw);
   }
   auto kern = stream_experts_kernel<float>;
@@ -814,7 +775,7 @@ cudaError_t launch_stream_experts(const void* x, const void* Wv, long long ldw, 
   if (err != cudaSuccess) return err;
   return launch_pdl(kern, grid, dim3(kThreads), smem, stream, static_cast<const float*>(x),
                     static_cast<const float*>(Wv), counts, offsets, perm, w32, active, sb, T, d, n,
-                    k, P, NS, tickets, static_cast<float*>(v), route, fault, ldw);
+                    k, P, NS, static_cast<float*>(v), route, fault, ldw);
 }
 
 }  // namespace mova
