@@ -201,7 +201,6 @@ stream_experts_kernel(const DT* __restrict__ x, const DT* __restrict__ Wv,
       mbar_init(&empty[s], resident ? 1 : kConsumerWarps);
       mbar_init(&partb[s], kConsumerWarps);
     }
-    mbar_init(xbar, 1);
     *abort_flag = 0;
     *issued = 0;
     fence_barrier_init();
@@ -223,9 +222,14 @@ stream_experts_kernel(const DT* __restrict__ x, const DT* __restrict__ Wv,
     if (lg_c0 < lg_ce) load8(route.Wr + static_cast<size_t>(lg_e) * d + 8 * lg_c0, lg_w0);
   }
   pdl_wait();  // the previous kernel on the stream is complete (two-launch: routing of this call)
-  if (resident && threadIdx.x == 0) {
+  if (resident && threadIdx.x == kReducerWarp * 32) {
     // The resident x tile: one bulk copy per token row, issued at once so its
-    // latency overlaps the first weight stages.
+    // latency overlaps the first weight stages.  The reducer warp, idle until
+    // the first stage, initialises its barrier and issues the copies, so the
+    // selecting warps do not wait for the issue; the consumers wait on the
+    // barrier only after the grouping barrier, which this warp joins later.
+    mbar_init(xbar, 1);
+    fence_barrier_init();
     const uint32_t row_bytes_x = static_cast<uint32_t>(row_bytes);
     mbar_arrive_expect_tx(xbar, static_cast<uint32_t>(T) * row_bytes_x);
     for (int t = 0; t < T; ++t)
