@@ -215,6 +215,16 @@ def test_full_edge_shapes(api, T, E, k, n):
     _full(api, T, 256, E, k, n, "bf16", seed=T)
 
 
+@pytest.mark.parametrize("T,d,E,k,n", [(8, 256, 16, 4, 2048), (8, 2560, 64, 8, 1024), (7, 512, 64, 8, 128)])
+def test_full_decode_column_ranges(api, T, d, E, k, n):
+    """Decode batches whose CTAs own more than 8 output columns (n = 2048:
+    13 or 14 per CTA), whose SiLU tiles need the largest buffer (k = 8 of 64
+    experts: up to 64 active, which leaves room for three weight stages), and
+    whose slabs each span up to 8 experts (n = 128: one column per CTA, some
+    CTAs none)."""
+    _full(api, T, d, E, k, n, "bf16", seed=n + k, path="stream")
+
+
 @pytest.mark.parametrize("T,d", [(8, 3072), (4, 4096), (3, 4544)])
 def test_full_stream_resident_boundary(api, T, d):
     """Decode batches at and near the widest rows the weight-streaming
