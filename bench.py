@@ -496,55 +496,59 @@ def roofline(name, path, T, d, E, k, n, xs_b, distinct, stage_us, empty_us, ms_p
 
 
 def measure_e2e(a, T, L, xs, routing, layers, cfg, v, ws, k, n, tdt, dist_on, world, device, probs=None):
-    """The same metric through the public API with host buffers: per step, the
-    pinned host->device copy of that step's inputs (x, and the stored routing
-    in routing-given mode, and the attention probabilities in attend mode),
-    the call, and the device->host copy of v (of o in attend mode)."""
+    """The same metric through the C ABI's host-buffer calls (mova_value_routed_host,
+    mova_value_host, mova_value_attend_host): every step copies its inputs from
+    pinned host memory (x; the stored int8 indices and fp16 weights in
+    routing-given and attend mode; the attention probabilities in attend mode)
+    into the device workspace, runs the path, and copies v (o in attend mode)
+    back to pinned host memory.  Two steps are in flight, on two streams with a
+    workspace each, so that one step's copies overlap the other's kernels."""
     import torch
 
     from mixture_value_routing_b200 import api
-    xh = [torch.empty_like(x, device="cpu").pin_memory() for x in xs]
-    for i, x in enumerate(xs):
-        xh[i].copy_(x)
-    rh = None
-    if routing is not None:
-        rh = [(i.cpu().pin_memory(), w.cpu().pin_memory()) for i, w in routing]
-        rd = [torch.empty_like(routing[0][0]), torch.empty_like(routing[0][1])]
-    vh = torch.empty((T, n), dtype=tdt).pin_memory()
-    if probs is not None:
-        ph = [p.cpu().pin_memory() for p in probs]
-        pd = torch.empty_like(probs[0])
-        vh = torch.empty((probs[0].shape[0], 128), dtype=torch.float32).pin_memory()
-    xd = torch.empty_like(xs[0])
+    xh = [x.cpu().pin_memory() for x in xs]
+    rh = None if routing is None else [(i.cpu().pin_memory(), w.cpu().pin_memory()) for i, w in routing]
+    ph = None if probs is None else [p.cpu().pin_memory() for p in probs]
+    d = xs[0].shape[1]
+    E = layers.get(0, cfg["bias"])[2].shape[0]
+    if ph is not None:
+        H = probs[0].shape[0]
+        nbytes = api.attend_workspace_size_host(T, d, E, k, n, H)
+        outs = [torch.empty((H, 128), dtype=torch.float32).pin_memory() for _ in range(2)]
+    else:
+        nbytes = api.workspace_size_host(T, d, E, k, n)
+        outs = [torch.empty((T, n), dtype=tdt).pin_memory() for _ in range(2)]
+    wss = [torch.empty(nbytes, dtype=torch.uint8, device=device) for _ in range(2)]
+    streams = [torch.cuda.Stream(device) for _ in range(2)]
     Ke = max(3, min(500, int(0.2 / max(1e-6, 2.5e-8 * T * 20))))
 
     def e2e_step(i):
-        l = i % L
-        xd.copy_(xh[l], non_blocking=True)
+        l, j = i % L, i % 2
         Wr, br, Wv = layers.get(l, cfg["bias"])
         if rh is None:
-            out = api.value_routed(xd, Wr, br, Wv, k, MI.SCALE, ws=ws)
+            api.value_routed_host(xh[l], Wr, br, Wv, k, MI.SCALE, out=outs[j], ws=wss[j], stream=streams[j])
+        elif ph is None:
+            api.value_host(xh[l], rh[l][0], rh[l][1], Wv, out=outs[j], ws=wss[j], stream=streams[j])
         else:
-            rd[0].copy_(rh[l][0], non_blocking=True)
-            rd[1].copy_(rh[l][1], non_blocking=True)
-            if probs is not None:
-                pd.copy_(ph[l], non_blocking=True)
-                out = api.value_attend(xd, rd[0], rd[1], Wv, pd, ws=ws)
-            else:
-                out = api.value(xd, rd[0], rd[1], Wv, ws=ws)
-        vh.copy_(out, non_blocking=True)
+            api.value_attend_host(xh[l], rh[l][0], rh[l][1], Wv, ph[l], out=outs[j], ws=wss[j],
+                                  stream=streams[j])
 
     for i in range(a.warmup):
         e2e_step(i)
     torch.cuda.synchronize()
+    cur = torch.cuda.current_stream(device)
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     barrier(dist_on)
     torch.cuda.synchronize()
-    e0.record()
+    e0.record(cur)
+    for s in streams:
+        s.wait_event(e0)
     for i in range(Ke):
         e2e_step(i)
-    e1.record()
+    for s in streams:
+        cur.wait_stream(s)
+    e1.record(cur)
     torch.cuda.synchronize()
     barrier(dist_on)
     ems = allmax(e0.elapsed_time(e1), dist_on, device)
@@ -554,8 +558,9 @@ def measure_e2e(a, T, L, xs, routing, layers, cfg, v, ws, k, n, tdt, dist_on, wo
     if probs is not None:
         h2d += probs[0].numel() * probs[0].element_size()
     return {"value": round(job_value(world, T, Ke, ems), 1), "unit": "tokens/s",
-            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(vh.numel() * vh.element_size()),
-            "steps": Ke, "ms_per_step": round(ems / Ke, 5)}
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(outs[0].numel() * outs[0].element_size()),
+            "steps": Ke, "ms_per_step": round(ems / Ke, 5),
+            "api": "C-ABI host-buffer calls; two steps in flight on two streams"}
 
 
 def run_mova(a):

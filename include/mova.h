@@ -286,6 +286,41 @@ mova_status mova_value_attend(const void* x, const void* idx, mova_dtype idx_dt,
                               mova_dtype w_dt, const void* Wv, int L, int d, int E, int k, int n,
                               const float* probs, int H, float* o, void* ws, size_t ws_bytes, void* stream);
 
+/* Host-buffer forms of mova_value_routed, mova_value and mova_value_attend,
+ * for callers whose batch lives in host memory.  The same computation and
+ * arguments, except that the batch's inputs (x; idx and w of a given routing;
+ * probs) are HOST pointers, read by cudaMemcpyAsync into staging space at the
+ * end of the device workspace, and the result (v, or o; with
+ * mova_value_routed_host also the optional idx_out / w_out copies of the
+ * routing) is written to HOST memory by cudaMemcpyAsync.  The weights (Wr,
+ * br, Wv) stay DEVICE pointers.  Order on `stream`: input copies, the device
+ * call, output copies.
+ *  - Host buffers: page-locked (cudaHostAlloc / pinned) memory makes both
+ *    copies asynchronous; pageable memory works, with the driver's
+ *    synchronous staging.  The caller keeps the inputs unchanged and does not
+ *    read the outputs until the stream has passed the call (e.g. after
+ *    cudaStreamSynchronize or an event).
+ *  - Workspace: mova_workspace_size_host(T, d, E, k, n) bytes for the two
+ *    value forms, mova_attend_workspace_size_host(L, d, E, k, n, H) for the
+ *    attend form (also > 0 for L = 0, which writes zeros to o), 256-byte
+ *    aligned device memory; the device call uses its first part, the staging
+ *    the rest.  Two calls in flight on different streams need two workspaces.
+ *  - Errors: as the device forms, all detected before anything is enqueued
+ *    (a CUDA error from a copy returns MOVA_ERR_CUDA). */
+size_t mova_workspace_size_host(int T, int d, int E, int k, int n);
+size_t mova_attend_workspace_size_host(int L, int d, int E, int k, int n, int H);
+mova_status mova_value_routed_host(const void* x_host, mova_dtype x_dt, const float* Wr, const float* br,
+                                   const void* Wv, mova_dtype wv_dt, int T, int d, int E, int k, int n,
+                                   float scale, void* v_host, int32_t* idx_host, float* w_host, void* ws,
+                                   size_t ws_bytes, void* stream);
+mova_status mova_value_host(const void* x_host, mova_dtype x_dt, const void* idx_host, mova_dtype idx_dt,
+                            const void* w_host, mova_dtype w_dt, const void* Wv, mova_dtype wv_dt, int T, int d,
+                            int E, int k, int n, void* v_host, void* ws, size_t ws_bytes, void* stream);
+mova_status mova_value_attend_host(const void* x_host, const void* idx_host, mova_dtype idx_dt,
+                                   const void* w_host, mova_dtype w_dt, const void* Wv, int L, int d, int E,
+                                   int k, int n, const float* probs_host, int H, float* o_host, void* ws,
+                                   size_t ws_bytes, void* stream);
+
 /* mova_route with options (only router_partitions applies). */
 mova_status mova_route_opts(const void* x, mova_dtype x_dt, const float* Wr, const float* br,
                             int T, int d, int E, int k, float scale, int32_t* idx, float* w,

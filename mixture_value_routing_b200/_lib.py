@@ -61,6 +61,13 @@ SIGNATURES = {
     "mova_attend_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i]),
     "mova_value_attend": (_i, [_vp, _vp, _i, _vp, _i, _vp, _i, _i, _i, _i, _i, _vp, _i, _vp, _vp, _sz, _vp]),
     "mova_router_planes": (_i, [_vp, _i, _i, _vp, _vp]),
+    "mova_workspace_size_host": (_sz, [_i, _i, _i, _i, _i]),
+    "mova_attend_workspace_size_host": (_sz, [_i, _i, _i, _i, _i, _i]),
+    "mova_value_routed_host": (_i, [_vp, _i, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _vp, _vp, _vp,
+                                    _vp, _sz, _vp]),
+    "mova_value_host": (_i, [_vp, _i, _vp, _i, _vp, _i, _vp, _i, _i, _i, _i, _i, _i, _vp, _vp, _sz, _vp]),
+    "mova_value_attend_host": (_i, [_vp, _vp, _i, _vp, _i, _vp, _i, _i, _i, _i, _i, _vp, _i, _vp, _vp, _sz,
+                                    _vp]),
     "mova_value_routed_noalloc": (_i, [_vp, _i, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _vp,
                                        _vp]),
     "mova_route_opts": (_i, [_vp, _i, _vp, _vp, _i, _i, _i, _i, _f, _vp, _vp, _vp, _vp]),

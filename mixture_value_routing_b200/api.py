@@ -11,6 +11,7 @@ synchronising.  Device-side checks are read with get_status().
 from __future__ import annotations
 
 import ctypes
+import functools
 from typing import Optional
 
 import torch
@@ -27,7 +28,18 @@ def _ptr(t: Optional[torch.Tensor]):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
-def _stream():
+try:
+    _raw_stream = torch._C._cuda_getCurrentRawStream  # the current stream's handle, without a Stream object
+except AttributeError:  # pragma: no cover - older torch
+    _raw_stream = None
+
+
+def _stream(stream: Optional["torch.cuda.Stream"] = None):
+    """The handle of `stream`, else of the current stream of the current device."""
+    if stream is not None:
+        return ctypes.c_void_p(stream.cuda_stream)
+    if _raw_stream is not None:
+        return ctypes.c_void_p(_raw_stream(torch.cuda.current_device()))
     return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
 
 
@@ -71,8 +83,21 @@ def _workspace(nbytes: int, device) -> torch.Tensor:
     return _WS[dev].get(nbytes, dev)
 
 
+@functools.lru_cache(maxsize=256)
 def workspace_size(T: int, d: int, E: int, k: int, n: int) -> int:
     return int(_lib.load().mova_workspace_size(T, d, E, k, n))
+
+
+@functools.lru_cache(maxsize=256)
+def workspace_size_host(T: int, d: int, E: int, k: int, n: int) -> int:
+    """Device workspace of the host-buffer value calls (value_routed_host, value_host)."""
+    return int(_lib.load().mova_workspace_size_host(T, d, E, k, n))
+
+
+@functools.lru_cache(maxsize=256)
+def attend_workspace_size_host(L: int, d: int, E: int, k: int, n: int, H: int) -> int:
+    """Device workspace of value_attend_host."""
+    return int(_lib.load().mova_attend_workspace_size_host(L, d, E, k, n, H))
 
 
 def auto_path(T: int, dtype: torch.dtype) -> str:
@@ -273,6 +298,98 @@ def value_routed(x: torch.Tensor, Wr: torch.Tensor, br: torch.Tensor, Wv: torch.
     if return_routing:
         return v, idx, w
     return v
+
+
+def _need_host(t: torch.Tensor, name: str, dtypes=None, ndim=None):
+    if t.is_cuda:
+        raise ValueError(f"{name} must be a host (CPU) tensor; pinned memory makes the copy asynchronous")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtypes is not None and t.dtype not in dtypes:
+        raise ValueError(f"{name}: dtype {t.dtype} not in {dtypes}")
+    if ndim is not None and t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dims")
+
+
+def _host_out(out, shape, dtype, name="out"):
+    if out is None:
+        return torch.empty(shape, dtype=dtype, pin_memory=True)
+    _need_host(out, name, (dtype,), len(shape))
+    if tuple(out.shape) != tuple(shape):
+        raise ValueError(f"{name}: shape {tuple(out.shape)}, expected {tuple(shape)}")
+    return out
+
+
+def value_routed_host(x: torch.Tensor, Wr: torch.Tensor, br: torch.Tensor, Wv: torch.Tensor,
+                      k: int = 4, scale: float = 2.5, out: Optional[torch.Tensor] = None,
+                      ws: Optional[torch.Tensor] = None, stream=None, return_routing: bool = False):
+    """value_routed for a batch in host memory (mova_value_routed_host): x is a
+    CPU tensor (pinned for an asynchronous copy), the weights are on the
+    device, and v (and the routing) come back in host tensors, valid once the
+    stream has passed the call."""
+    _need_host(x, "x", (torch.float32, torch.bfloat16), 2)
+    _need(Wr, "Wr", (torch.float32,), 2)
+    _need(br, "br", (torch.float32,), 1)
+    _need(Wv, "Wv", (x.dtype,), 3)
+    T, d = x.shape
+    E, n = Wv.shape[0], Wv.shape[1]
+    v = _host_out(out, (T, n), x.dtype)
+    idx = w = None
+    if return_routing:
+        idx = torch.empty((T, k), dtype=torch.int32, pin_memory=True)
+        w = torch.empty((T, k), dtype=torch.float32, pin_memory=True)
+    if ws is None:
+        ws = _workspace(workspace_size_host(T, d, E, k, n), Wv.device)
+    _lib.check(_lib.load().mova_value_routed_host(
+        _ptr(x), _DT[x.dtype], _ptr(Wr), _ptr(br), _ptr(Wv), _DT[Wv.dtype], T, d, E, k, n, float(scale),
+        _ptr(v), _ptr(idx), _ptr(w), _ptr(ws), ws.numel(), _stream(stream)), "mova_value_routed_host")
+    return (v, idx, w) if return_routing else v
+
+
+def value_host(x: torch.Tensor, idx: torch.Tensor, w: torch.Tensor, Wv: torch.Tensor,
+               out: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None, stream=None):
+    """value for a batch and stored routing in host memory (mova_value_host);
+    v comes back in a host tensor, valid once the stream has passed the call."""
+    _need_host(x, "x", (torch.float32, torch.bfloat16), 2)
+    _need_host(idx, "idx", (torch.int32, torch.int8), 2)
+    _need_host(w, "w", (torch.float32, torch.float16), 2)
+    _need(Wv, "Wv", (x.dtype,), 3)
+    T, d = x.shape
+    E, n = Wv.shape[0], Wv.shape[1]
+    k = idx.shape[1]
+    v = _host_out(out, (T, n), x.dtype)
+    if ws is None:
+        ws = _workspace(workspace_size_host(T, d, E, k, n), Wv.device)
+    _lib.check(_lib.load().mova_value_host(
+        _ptr(x), _DT[x.dtype], _ptr(idx), _DT[idx.dtype], _ptr(w), _DT[w.dtype], _ptr(Wv), _DT[Wv.dtype],
+        T, d, E, k, n, _ptr(v), _ptr(ws), ws.numel(), _stream(stream)), "mova_value_host")
+    return v
+
+
+def value_attend_host(x: torch.Tensor, idx: torch.Tensor, w: torch.Tensor, Wv: torch.Tensor,
+                      probs: torch.Tensor, out: Optional[torch.Tensor] = None,
+                      ws: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """value_attend for a compact cache and probabilities in host memory
+    (mova_value_attend_host); o (H, 128) fp32 comes back in a host tensor,
+    valid once the stream has passed the call."""
+    _need_host(x, "x", (torch.bfloat16,), 2)
+    _need_host(idx, "idx", (torch.int32, torch.int8), 2)
+    _need_host(w, "w", (torch.float32, torch.float16), 2)
+    _need_host(probs, "probs", (torch.float32,), 2)
+    _need(Wv, "Wv", (torch.bfloat16,), 3)
+    L, d = x.shape
+    E, n = Wv.shape[0], Wv.shape[1]
+    k = idx.shape[1]
+    H = probs.shape[0]
+    if probs.shape[1] != L:
+        raise ValueError("probs: (H, L) for the L cached positions of x")
+    o = _host_out(out, (H, 128), torch.float32)
+    if ws is None:
+        ws = _workspace(attend_workspace_size_host(L, d, E, k, n, H), Wv.device)
+    _lib.check(_lib.load().mova_value_attend_host(
+        _ptr(x), _ptr(idx), _DT[idx.dtype], _ptr(w), _DT[w.dtype], _ptr(Wv), L, d, E, k, n, _ptr(probs), H,
+        _ptr(o), _ptr(ws), ws.numel(), _stream(stream)), "mova_value_attend_host")
+    return o
 
 
 def workspace_parts(T: int, d: int, E: int, k: int, n: int) -> dict:

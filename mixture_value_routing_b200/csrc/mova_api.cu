@@ -540,6 +540,139 @@ mova_status mova_workspace_parts(int T, int d, int E, int k, int n, size_t* offs
   return MOVA_OK;
 }
 
+// ---- Host-buffer forms ------------------------------------------------------
+// The batch's inputs are copied from host memory into staging space that
+// follows the device call's workspace, the device call runs on it, and the
+// result is copied back to host memory: three steps on the caller's stream.
+
+static size_t act_size(mova_dtype dt) { return dt == MOVA_BF16 ? 2 : 4; }
+static size_t idx_size(mova_dtype dt) { return dt == MOVA_I8 ? 1 : 4; }
+static size_t wgt_size(mova_dtype dt) { return dt == MOVA_F16 ? 2 : 4; }
+
+// Staging of a value call: x (at most 4 B an element), v, idx and w.
+static size_t value_staging_bytes(int T, int d, int k, int n) {
+  const size_t Tz = static_cast<size_t>(T);
+  return align256(Tz * d * 4) + align256(Tz * n * 4) + 2 * align256(Tz * k * 4);
+}
+
+size_t mova_workspace_size_host(int T, int d, int E, int k, int n) {
+  const size_t base = mova_workspace_size(T, d, E, k, n);
+  if (base == 0) return 0;
+  return align256(base) + value_staging_bytes(T, d, k, n);
+}
+
+static bool host_ws_ok(const void* ws, size_t ws_bytes, size_t need) {
+  return need != 0 && ws_bytes >= need && (reinterpret_cast<uintptr_t>(ws) & 255) == 0;
+}
+
+mova_status mova_value_routed_host(const void* x_host, mova_dtype x_dt, const float* Wr, const float* br,
+                                   const void* Wv, mova_dtype wv_dt, int T, int d, int E, int k, int n,
+                                   float scale, void* v_host, int32_t* idx_host, float* w_host, void* ws,
+                                   size_t ws_bytes, void* stream) {
+  mova_status st = check_dims(T, d, E, k, n);
+  if (st != MOVA_OK) return st;
+  if (!valid_act_dtype(x_dt) || wv_dt != x_dt) return MOVA_ERR_UNSUPPORTED;
+  if (T == 0) return MOVA_OK;
+  if (!x_host || !Wr || !br || !Wv || !v_host || !ws) return MOVA_ERR_INVALID_ARG;
+  if (!aligned16(Wr) || !aligned16(Wv)) return MOVA_ERR_INVALID_ARG;
+  if (!host_ws_ok(ws, ws_bytes, mova_workspace_size_host(T, d, E, k, n))) return MOVA_ERR_INVALID_ARG;
+  const size_t base = align256(mova_workspace_size(T, d, E, k, n));
+  const size_t Tz = static_cast<size_t>(T), es = act_size(x_dt);
+  char* x_dev = static_cast<char*>(ws) + base;
+  char* v_dev = x_dev + align256(Tz * d * 4);
+  int32_t* idx_dev = reinterpret_cast<int32_t*>(v_dev + align256(Tz * n * 4));
+  float* w_dev = reinterpret_cast<float*>(reinterpret_cast<char*>(idx_dev) + align256(Tz * k * 4));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t err = cudaMemcpyAsync(x_dev, x_host, Tz * d * es, cudaMemcpyHostToDevice, s);
+  if (err != cudaSuccess) return from_cuda(err);
+  st = mova_value_routed(x_dev, x_dt, Wr, br, Wv, wv_dt, T, d, E, k, n, scale, v_dev,
+                         idx_host ? idx_dev : nullptr, w_host ? w_dev : nullptr, ws, base, stream);
+  if (st != MOVA_OK) return st;
+  err = cudaMemcpyAsync(v_host, v_dev, Tz * n * es, cudaMemcpyDeviceToHost, s);
+  if (err == cudaSuccess && idx_host) err = cudaMemcpyAsync(idx_host, idx_dev, Tz * k * 4, cudaMemcpyDeviceToHost, s);
+  if (err == cudaSuccess && w_host) err = cudaMemcpyAsync(w_host, w_dev, Tz * k * 4, cudaMemcpyDeviceToHost, s);
+  return from_cuda(err);
+}
+
+mova_status mova_value_host(const void* x_host, mova_dtype x_dt, const void* idx_host, mova_dtype idx_dt,
+                            const void* w_host, mova_dtype w_dt, const void* Wv, mova_dtype wv_dt, int T, int d,
+                            int E, int k, int n, void* v_host, void* ws, size_t ws_bytes, void* stream) {
+  mova_status st = check_dims(T, d, E, k, n);
+  if (st != MOVA_OK) return st;
+  if (!valid_act_dtype(x_dt) || wv_dt != x_dt) return MOVA_ERR_UNSUPPORTED;
+  if (idx_dt != MOVA_I32 && idx_dt != MOVA_I8) return MOVA_ERR_UNSUPPORTED;
+  if (w_dt != MOVA_F32 && w_dt != MOVA_F16) return MOVA_ERR_UNSUPPORTED;
+  if (T == 0) return MOVA_OK;
+  if (!x_host || !idx_host || !w_host || !Wv || !v_host || !ws) return MOVA_ERR_INVALID_ARG;
+  if (!aligned16(Wv)) return MOVA_ERR_INVALID_ARG;
+  if (!host_ws_ok(ws, ws_bytes, mova_workspace_size_host(T, d, E, k, n))) return MOVA_ERR_INVALID_ARG;
+  const size_t base = align256(mova_workspace_size(T, d, E, k, n));
+  const size_t Tz = static_cast<size_t>(T), es = act_size(x_dt);
+  char* x_dev = static_cast<char*>(ws) + base;
+  char* v_dev = x_dev + align256(Tz * d * 4);
+  char* idx_dev = v_dev + align256(Tz * n * 4);
+  char* w_dev = idx_dev + align256(Tz * k * 4);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t err = cudaMemcpyAsync(x_dev, x_host, Tz * d * es, cudaMemcpyHostToDevice, s);
+  if (err == cudaSuccess)
+    err = cudaMemcpyAsync(idx_dev, idx_host, Tz * k * idx_size(idx_dt), cudaMemcpyHostToDevice, s);
+  if (err == cudaSuccess) err = cudaMemcpyAsync(w_dev, w_host, Tz * k * wgt_size(w_dt), cudaMemcpyHostToDevice, s);
+  if (err != cudaSuccess) return from_cuda(err);
+  st = mova_value(x_dev, x_dt, idx_dev, idx_dt, w_dev, w_dt, Wv, wv_dt, T, d, E, k, n, v_dev, ws, base, stream);
+  if (st != MOVA_OK) return st;
+  return from_cuda(cudaMemcpyAsync(v_host, v_dev, Tz * n * es, cudaMemcpyDeviceToHost, s));
+}
+
+// Staging of an attend call: x (bf16), idx and w (at most 4 B), probs, o.
+static size_t attend_staging_bytes(int L, int d, int k, int H) {
+  const size_t Lz = static_cast<size_t>(L);
+  return align256(Lz * d * 2) + 2 * align256(Lz * k * 4) + align256(static_cast<size_t>(H) * Lz * 4) +
+         align256(static_cast<size_t>(H) * 128 * 4);
+}
+
+size_t mova_attend_workspace_size_host(int L, int d, int E, int k, int n, int H) {
+  if (check_dims(L, d, E, k, n) != MOVA_OK || !attend_heads_ok(n, H)) return 0;
+  return align256(mova_attend_workspace_size(L, d, E, k, n, H)) + attend_staging_bytes(L, d, k, H);
+}
+
+mova_status mova_value_attend_host(const void* x_host, const void* idx_host, mova_dtype idx_dt,
+                                   const void* w_host, mova_dtype w_dt, const void* Wv, int L, int d, int E,
+                                   int k, int n, const float* probs_host, int H, float* o_host, void* ws,
+                                   size_t ws_bytes, void* stream) {
+  mova_status st = check_dims(L, d, E, k, n);
+  if (st != MOVA_OK) return st;
+  if (H <= 0) return MOVA_ERR_INVALID_ARG;
+  if (!attend_heads_ok(n, H)) return MOVA_ERR_UNSUPPORTED;
+  if (idx_dt != MOVA_I32 && idx_dt != MOVA_I8) return MOVA_ERR_UNSUPPORTED;
+  if (w_dt != MOVA_F32 && w_dt != MOVA_F16) return MOVA_ERR_UNSUPPORTED;
+  if (!o_host || !ws) return MOVA_ERR_INVALID_ARG;
+  if (L > 0 && (!x_host || !idx_host || !w_host || !Wv || !probs_host)) return MOVA_ERR_INVALID_ARG;
+  if (L > 0 && !aligned16(Wv)) return MOVA_ERR_INVALID_ARG;
+  if (L > 0 && sm_count() < 2) return MOVA_ERR_UNSUPPORTED;  // the pair GEMM
+  if (!host_ws_ok(ws, ws_bytes, mova_attend_workspace_size_host(L, d, E, k, n, H))) return MOVA_ERR_INVALID_ARG;
+  const size_t base = align256(mova_attend_workspace_size(L, d, E, k, n, H));
+  const size_t Lz = static_cast<size_t>(L), Hz = static_cast<size_t>(H);
+  char* x_dev = static_cast<char*>(ws) + base;
+  char* idx_dev = x_dev + align256(Lz * d * 2);
+  char* w_dev = idx_dev + align256(Lz * k * 4);
+  float* p_dev = reinterpret_cast<float*>(w_dev + align256(Lz * k * 4));
+  float* o_dev = reinterpret_cast<float*>(reinterpret_cast<char*>(p_dev) + align256(Hz * Lz * 4));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t err = cudaSuccess;
+  if (L > 0) {
+    err = cudaMemcpyAsync(x_dev, x_host, Lz * d * 2, cudaMemcpyHostToDevice, s);
+    if (err == cudaSuccess)
+      err = cudaMemcpyAsync(idx_dev, idx_host, Lz * k * idx_size(idx_dt), cudaMemcpyHostToDevice, s);
+    if (err == cudaSuccess) err = cudaMemcpyAsync(w_dev, w_host, Lz * k * wgt_size(w_dt), cudaMemcpyHostToDevice, s);
+    if (err == cudaSuccess) err = cudaMemcpyAsync(p_dev, probs_host, Hz * Lz * 4, cudaMemcpyHostToDevice, s);
+    if (err != cudaSuccess) return from_cuda(err);
+  }
+  st = mova_value_attend(x_dev, idx_dev, idx_dt, w_dev, w_dt, Wv, L, d, E, k, n, p_dev, H, o_dev, ws, base,
+                         stream);
+  if (st != MOVA_OK) return st;
+  return from_cuda(cudaMemcpyAsync(o_host, o_dev, Hz * 128 * 4, cudaMemcpyDeviceToHost, s));
+}
+
 mova_status mova_get_status(void* ws, int32_t* detail_out, void* stream) {
   if (!ws) return MOVA_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);

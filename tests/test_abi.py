@@ -162,3 +162,40 @@ def test_attend_host_side_validation(lib):
     assert lib.mova_attend_workspace_size(64, 2560, 64, 4, 1024, 32) > lib.mova_workspace_size(64, 2560, 64, 4, 1024)
     assert lib.mova_attend_workspace_size(64, 2560, 64, 4, 1024, 40) == 0
     assert lib.mova_attend_workspace_size(0, 2560, 64, 4, 1024, 32) == 0
+
+
+def test_host_buffer_forms_validation(lib):
+    """The host-buffer value calls check their arguments and workspace on the
+    host before enqueueing any copy; their workspace is the device call's plus
+    aligned staging for the batch and the result."""
+    fake = ctypes.c_void_p(4096)
+    BF16, F32, I8, F16 = _lib.BF16, _lib.F32, _lib.I8, _lib.F16
+    T, d, E, k, n = 8, 2560, 64, 4, 1024
+    base = lib.mova_workspace_size(T, d, E, k, n)
+    host = lib.mova_workspace_size_host(T, d, E, k, n)
+    staging = 2560 * 8 * 4 + 1024 * 8 * 4 + 2 * 256  # x and v at 4 B an element, idx and w rounded up
+    assert host == ((base + 255) & ~255) + staging
+    assert lib.mova_workspace_size_host(0, d, E, k, n) == 0
+    assert lib.mova_workspace_size_host(T, d + 1, E, k, n) == 0
+    routed = lambda x_dt, wv_dt, T_, ws_bytes, v: lib.mova_value_routed_host(
+        fake, x_dt, fake, fake, fake, wv_dt, T_, d, E, k, n, 2.5, v, None, None, fake, ws_bytes, None)
+    assert routed(BF16, BF16, 0, 0, None) == _lib.OK                       # T == 0: nothing to do
+    assert routed(BF16, F32, T, host, fake) == _lib.ERR_UNSUPPORTED         # Wv dtype must equal x's
+    assert routed(BF16, BF16, T, host, None) == _lib.ERR_INVALID_ARG        # no output buffer
+    assert routed(BF16, BF16, T, base, fake) == _lib.ERR_INVALID_ARG        # room for the call, not the staging
+    assert lib.mova_value_host(fake, BF16, fake, F32, fake, F16, fake, BF16, T, d, E, k, n, fake, fake,
+                               host, None) == _lib.ERR_UNSUPPORTED        # idx must be int32 or int8
+    assert lib.mova_value_host(fake, BF16, fake, I8, fake, F16, fake, BF16, T, d, E, k, n, fake, fake,
+                               host - 256, None) == _lib.ERR_INVALID_ARG  # workspace too small
+    assert lib.mova_value_host(fake, BF16, fake, I8, fake, F16, ctypes.c_void_p(4100), BF16, T, d, E, k, n,
+                               fake, fake, host, None) == _lib.ERR_INVALID_ARG  # misaligned Wv
+    # attend: staging for o even at L == 0 (zeros are written through it)
+    assert lib.mova_attend_workspace_size_host(0, d, E, k, n, 32) == 32 * 128 * 4
+    assert lib.mova_attend_workspace_size_host(64, d, E, k, n, 40) == 0
+    assert lib.mova_attend_workspace_size_host(64, d, E, k, n, 32) > lib.mova_attend_workspace_size(64, d, E, k, n, 32)
+    attend = lambda H, o, ws_bytes: lib.mova_value_attend_host(fake, fake, I8, fake, F16, fake, 64, d, E, k, n,
+                                                               fake, H, o, fake, ws_bytes, None)
+    assert attend(0, fake, 1 << 30) == _lib.ERR_INVALID_ARG
+    assert attend(12, fake, 1 << 30) == _lib.ERR_UNSUPPORTED
+    assert attend(32, None, 1 << 30) == _lib.ERR_INVALID_ARG
+    assert attend(32, fake, 4096) == _lib.ERR_INVALID_ARG

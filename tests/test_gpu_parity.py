@@ -713,3 +713,84 @@ def test_head_parallel_given(api):
     v_ref = O.combine(O.to_f64(bat.x, "bf16"), bat.idx.astype(np.int64), bat.w.astype(np.float64),
                       lay.Wv, "bf16")
     P.check_values(P.host_f64(v), v_ref[:, 256:640], "bf16")
+
+
+# ---------------------------------------------------------------------------
+# Host-buffer forms (batch and result in pinned host memory)
+# ---------------------------------------------------------------------------
+
+def _pinned(t):
+    return t.cpu().pin_memory()
+
+
+@pytest.mark.parametrize("T", [8, 300])
+def test_value_routed_host_buffers(api, T):
+    """mova_value_routed_host (copy in, the device call, copy out on one
+    stream) gives the device form's v and routing bit for bit, and v against
+    the oracle."""
+    d, E, k, n = 2560, 64, 4, 1024
+    lay = _layer(T + 3, d, E, n, "bf16")
+    bat = MI.make_batch(T, T + 3, dtype="bf16", d=d)
+    Wr, br, Wv = P.dev(lay.Wr, "f32"), P.dev(lay.br, "f32"), P.dev(lay.Wv, "bf16")
+    xd = P.dev(bat.x, "bf16")
+    v_dev, idx_dev, w_dev = api.value_routed(xd, Wr, br, Wv, k, 2.5, return_routing=True)
+    ws = torch.empty(api.workspace_size_host(T, d, E, k, n), dtype=torch.uint8, device="cuda")
+    v, idx, w = api.value_routed_host(_pinned(xd), Wr, br, Wv, k, 2.5, ws=ws, return_routing=True)
+    torch.cuda.synchronize()
+    assert not v.is_cuda and v.shape == (T, n) and v.dtype == torch.bfloat16
+    assert torch.equal(v, v_dev.cpu()) and torch.equal(idx, idx_dev.cpu()) and torch.equal(w, w_dev.cpu())
+    x, ref = _routing_ref(bat, lay, k)
+    idx_g = idx.numpy().astype(np.int64)
+    P.check_routing(idx_g, w.numpy().astype(np.float64), ref, k, 2.5)
+    rows = np.arange(min(T, 64))
+    v_ref = O.combine(x[rows], idx_g[rows], O.weights_for(ref["s"][rows], idx_g[rows], 2.5), lay.Wv, "bf16")
+    P.check_values(P.host_f64(v)[rows], v_ref, "bf16")
+
+
+@pytest.mark.parametrize("T,path", [(37, "stream"), (1000, "auto")])
+def test_value_host_buffers(api, T, path):
+    """mova_value_host with int8 indices and fp16 weights in host memory gives
+    the device form's v bit for bit, and v against the oracle."""
+    d, E, k, n = 512, 16, 4, 256
+    lay = _layer(T, d, E, n, "bf16")
+    rng = np.random.default_rng(T)
+    idx = np.argsort(rng.random((T, E)), axis=1)[:, :k].astype(np.int8)
+    g = rng.exponential(1.0, size=(T, k))
+    w = (2.5 * g / g.sum(axis=1, keepdims=True)).astype(np.float16)
+    bat = MI.make_batch(T, T, dtype="bf16", d=d)
+    xd, idxd, wd, Wv = P.dev(bat.x, "bf16"), P.dev(idx, "i8"), P.dev(w, "f16"), P.dev(lay.Wv, "bf16")
+    v_dev = api.value(xd, idxd, wd, Wv, path=path)
+    v = api.value_host(_pinned(xd), _pinned(idxd), _pinned(wd), Wv)
+    torch.cuda.synchronize()
+    assert torch.equal(v, v_dev.cpu())
+    v_ref = O.combine(O.to_f64(bat.x, "bf16"), idx.astype(np.int64), w.astype(np.float64), lay.Wv, "bf16")
+    P.check_values(P.host_f64(v), v_ref, "bf16")
+
+
+@pytest.mark.parametrize("L", [0, 65])
+def test_value_attend_host_buffers(api, L):
+    """mova_value_attend_host: o equals the device form's bit for bit (zeros
+    for L = 0, written through the workspace's staging)."""
+    d, E, k, n, H = 2560, 64, 4, 1024, 32
+    lay = _layer(52, d, E, n, "bf16")
+    Wv = P.dev(lay.Wv, "bf16")
+    if L == 0:
+        x = torch.empty((0, d), dtype=torch.bfloat16).pin_memory()
+        idx = torch.empty((0, k), dtype=torch.int8).pin_memory()
+        w = torch.empty((0, k), dtype=torch.float16).pin_memory()
+        p = torch.empty((H, 0), dtype=torch.float32).pin_memory()
+        o = api.value_attend_host(x, idx, w, Wv, p, out=torch.full((H, 128), 7.0).pin_memory())
+        torch.cuda.synchronize()
+        assert torch.equal(o, torch.zeros((H, 128)))
+        return
+    bat = MI.make_batch(L, 52, dtype="bf16", mode="given")
+    probs = MI.make_attention_probs(H, L, 52)
+    xd, idxd, wd = P.dev(bat.x, "bf16"), P.dev(bat.idx, "i8"), P.dev(bat.w, "f16")
+    pd = torch.from_numpy(probs).cuda()
+    o_dev = api.value_attend(xd, idxd, wd, Wv, pd)
+    o = api.value_attend_host(_pinned(xd), _pinned(idxd), _pinned(wd), Wv, _pinned(pd))
+    torch.cuda.synchronize()
+    assert torch.equal(o, o_dev.cpu())
+    ref = _attend_ref(bat, lay, probs)
+    err = np.abs(o.numpy().astype(np.float64) - ref)
+    assert (err <= 1e-4 * np.maximum(1.0, np.abs(ref))).all(), err.max()
