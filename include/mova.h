@@ -24,7 +24,9 @@
  *
  * Conventions for every entry point:
  *  - All tensor pointers are DEVICE pointers owned by the caller, row-major
- *    and contiguous, 16-byte aligned.  The library never allocates.
+ *    and contiguous, 16-byte aligned, except the batch and result buffers of
+ *    the *_host entry points, which are HOST pointers.  The library never
+ *    allocates.
  *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default
  *    stream).  Every compute call is asynchronous on it; outputs are valid
  *    once the stream has reached that point.
