@@ -21,7 +21,9 @@
 //   * Per 64-wide K step a CTA loads 16 KB of weights (one 2-D box) and up to
 //     32 KB of token rows (its half of the tile's pairs: accumulator 0's rows
 //     at the start of the stage's B area, accumulator 1's 16 KB further);
-//     four 48 KB stages.
+//     four 48 KB stages.  Batches of at most 256 pairs per expert on
+//     average take tiles of up to 384 pairs instead (accumulator 1 at most
+//     128), so a stage is 40 KB and five fit: more weight bytes in flight.
 //     Both CTAs' copies complete on the even CTA's stage barrier (no
 //     multicast).  The even CTA's MMA warp issues tcgen05.mma.cta_group::2
 //     (M = 256, N = 16..256, K = 16) into accumulator 0 (pairs 0..255 of the
@@ -60,21 +62,37 @@ namespace {
 
 constexpr int PM = 128;         // weight rows per CTA (256 per pair)
 constexpr int NA = 256;         // pairs per accumulator
-constexpr int NT = 2 * NA;      // pairs per tile
+constexpr int NT = 2 * NA;      // pairs per tile (the configuration of larger batches)
+constexpr int NT_SMALL = NA + NA / 2;  // pairs per tile at <= 256 pairs per expert on average
 constexpr int PK = 64;
-constexpr int kPStages = 4;
 constexpr int kTileRing = 16;
 constexpr int kPABytes = PM * PK * 2;           // 16 KB of weights per stage
-constexpr int kPBBytes = (NT / 2) * PK * 2;     // up to 32 KB of token rows
-constexpr int kPStageBytes = kPABytes + kPBBytes;
+// The stage ring, in one of two configurations over the same shared-memory
+// area: tiles of up to 512 pairs with four 48 KB stages (16 KB of weights and
+// 32 KB of token rows per CTA), or tiles of up to 384 pairs with five 40 KB
+// stages.  The second keeps more weight bytes in flight per SM; it is taken
+// when the batch has at most 256 pairs per expert on average, where experts
+// rarely need a second token tile (with 512-pair tiles fewer experts split,
+// which matters at larger batches).
+template <int kNT>
+struct Ring {
+  static constexpr int kStages = kNT > NT_SMALL ? 4 : 5;
+  static constexpr int kBBytes = (kNT / 2) * PK * 2;
+  static constexpr int kStageBytes = kPABytes + kBBytes;
+};
+constexpr int kPStagesMax = 5;
+constexpr int kStageArea = Ring<NT_SMALL>::kStages * Ring<NT_SMALL>::kStageBytes;
+static_assert(Ring<NT>::kStages * Ring<NT>::kStageBytes <= kStageArea, "both rings fit the stage area");
+static_assert(Ring<NT_SMALL>::kStageBytes % 1024 == 0 && Ring<NT>::kStageBytes % 1024 == 0,
+              "stages stay 1024-byte aligned (128-byte swizzle atoms)");
 constexpr int kEpiWarps = 8;
 constexpr int kPThreads = (2 + kEpiWarps) * 32;  // warp 0 TMA, warp 1 MMA, 2-9 epilogue
 constexpr uint32_t kPTmemCols = 512;
 
 struct __align__(1024) PSmem {
-  uint8_t stage[kPStages][kPStageBytes];
-  uint64_t full[kPStages];      // even CTA: both CTAs' copies of the stage landed
-  uint64_t empty[kPStages];     // both CTAs: the pair's MMAs on the stage are done
+  uint8_t stage_area[kStageArea];  // Ring<kNT>::kStages stages of Ring<kNT>::kStageBytes
+  uint64_t full[kPStagesMax];   // even CTA: both CTAs' copies of the stage landed
+  uint64_t empty[kPStagesMax];  // both CTAs: the pair's MMAs on the stage are done
   uint64_t reg_full[2];         // both CTAs: tensor-memory region r holds a finished accumulator
   uint64_t reg_empty[2];        // even CTA: region r read out by its 4 epilogue warps x 2 CTAs
   uint64_t tq_full[kTileRing];  // both CTAs: tile id i of this cluster published
@@ -201,7 +219,7 @@ constexpr int kAcc1Rows = NA / 2;               // accumulator 1's rows start he
 
 // Ten warps: sub-partitions 0 and 1 hold three each, so at most
 // 16384 / (3 * 32) -> 168 registers per thread.
-template <bool kAttend>
+template <bool kAttend, int kNT>
 __global__ void __maxnreg__(168)
 grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_xp,
                          const int32_t* __restrict__ counts, const int32_t* __restrict__ offsets,
@@ -209,6 +227,8 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_w, const __gri
                          int ldw, __nv_bfloat16* __restrict__ P, AttendArgs at) {
   extern __shared__ uint8_t smem_raw[];
   PSmem& S = *reinterpret_cast<PSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  using R = Ring<kNT>;
+  static_assert(!kAttend || kNT == NT, "attend partials are laid out for 512-pair tiles");
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const uint32_t rank = cluster_rank();
@@ -216,7 +236,7 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_w, const __gri
   const int nk = d / PK;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kPStages; ++s) {
+    for (int s = 0; s < R::kStages; ++s) {
       mbar_init(&S.full[s], 1);
       mbar_init(&S.empty[s], 1);
     }
@@ -252,7 +272,7 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_w, const __gri
     const int nact = __popc(__ballot_sync(0xffffffffu, c0 > 0)) + __popc(__ballot_sync(0xffffffffu, c1 > 0));
     // Token-tile groups in expert index order (attend mode: one partial per
     // group, accumulator, query head of the group and weight row).
-    int q0 = c0 > 0 ? (c0 + NT - 1) / NT : 0, q1 = c1 > 0 ? (c1 + NT - 1) / NT : 0;
+    int q0 = c0 > 0 ? (c0 + kNT - 1) / kNT : 0, q1 = c1 > 0 ? (c1 + kNT - 1) / kNT : 0;
     {
       int g0 = q0, g1 = q1, gt0, gt;
       tile_prefix(g0, g1, lane, gt0, gt);
@@ -265,13 +285,13 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_w, const __gri
       S.act_e[r0] = e0;
       S.act_cnt[r0] = c0;
       S.act_off[r0] = f0;
-      S.act_ntt[r0] = (c0 + NT - 1) / NT;
+      S.act_ntt[r0] = (c0 + kNT - 1) / kNT;
     }
     if (c1 > 0) {
       S.act_e[r1] = e1;
       S.act_cnt[r1] = c1;
       S.act_off[r1] = f1;
-      S.act_ntt[r1] = (c1 + NT - 1) / NT;
+      S.act_ntt[r1] = (c1 + kNT - 1) / kNT;
     }
     __syncwarp();
     const int a0 = lane, a1 = lane + 32;
@@ -360,7 +380,7 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_w, const __gri
           break;
         }
         const uint32_t full_cl = full0_cl + static_cast<uint32_t>(s) * 8u;
-        uint8_t* st = S.stage[s];
+        uint8_t* st = S.stage_area + s * R::kStageBytes;
         if (elect_one()) {
           if (rank == 0) mbar_arrive_expect_tx(&S.full[s], bytes);
           if (tl.ntt == 1)
@@ -375,7 +395,7 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_w, const __gri
                              full_cl);
         }
         __syncwarp();
-        if (++s == kPStages) {
+        if (++s == R::kStages) {
           s = 0;
           phase ^= 1;
           started = true;
@@ -388,9 +408,9 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_w, const __gri
       // The whole warp runs the loop; one elected lane issues the MMAs and
       // commits.  Stage descriptors are built once and advanced by adding
       // offsets (start address in 16-byte units).
-      const uint64_t adesc0 = smem_desc_sw128(smem_u32(S.stage[0]));
-      const uint64_t bdesc0 = smem_desc_sw128(smem_u32(S.stage[0]) + kPABytes);
-      constexpr uint32_t kStageDesc = kPStageBytes >> 4;
+      const uint64_t adesc0 = smem_desc_sw128(smem_u32(S.stage_area));
+      const uint64_t bdesc0 = smem_desc_sw128(smem_u32(S.stage_area) + kPABytes);
+      constexpr uint32_t kStageDesc = R::kStageBytes >> 4;
       int s = 0;
       uint32_t phase = 0;
       Regions reg;
@@ -445,7 +465,7 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_w, const __gri
             tc_commit_pair_both(&S.empty[s]);
           }
           __syncwarp();
-          if (++s == kPStages) {
+          if (++s == R::kStages) {
             s = 0;
             phase ^= 1;
           }
@@ -605,7 +625,7 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_w, const __gri
   tc_fence_before();
   cluster_sync_all();  // neither CTA leaves while the pair may still touch its memory
   if (S.abort && threadIdx.x == 0) {
-    for (int s = 0; s < kPStages; ++s) mbar_wait(&S.empty[s], 0);
+    for (int s = 0; s < R::kStages; ++s) mbar_wait(&S.empty[s], 0);
   }
   __syncthreads();
   if (warp == 1) {
@@ -623,7 +643,7 @@ using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, 
 
 namespace {
 
-template <bool kAttend>
+template <bool kAttend, int kNT>
 cudaError_t launch_pair(const void* Wv, long long ldw, const int32_t* counts, const int32_t* offsets,
                         StatusBlock* sb, int T, int d, int n, int k, int E, const __nv_bfloat16* xp,
                         __nv_bfloat16* P, AttendArgs at, cudaStream_t stream) {
@@ -651,7 +671,7 @@ cudaError_t launch_pair(const void* Wv, long long ldw, const int32_t* counts, co
           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
   const size_t smem = sizeof(PSmem) + 1024;
-  cudaError_t err = cudaFuncSetAttribute(grouped_gemm_pair_kernel<kAttend>,
+  cudaError_t err = cudaFuncSetAttribute(grouped_gemm_pair_kernel<kAttend, kNT>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (err != cudaSuccess) return err;
   // As many pairs as can be resident at once (persistent).
@@ -672,13 +692,13 @@ cudaError_t launch_pair(const void* Wv, long long ldw, const int32_t* counts, co
   if (max_clusters == 0) {
     cfg.gridDim = dim3(2 * (sm_count() / 2));
     int c = 0;
-    if (cudaOccupancyMaxActiveClusters(&c, grouped_gemm_pair_kernel<kAttend>, &cfg) != cudaSuccess || c <= 0)
+    if (cudaOccupancyMaxActiveClusters(&c, grouped_gemm_pair_kernel<kAttend, kNT>, &cfg) != cudaSuccess || c <= 0)
       c = sm_count() / 2;
     max_clusters = c;
   }
   cfg.gridDim = dim3(2 * max_clusters);
   note_launch();
-  return cudaLaunchKernelEx(&cfg, grouped_gemm_pair_kernel<kAttend>, tmap_w, tmap_xp, counts, offsets, E, sb, d,
+  return cudaLaunchKernelEx(&cfg, grouped_gemm_pair_kernel<kAttend, kNT>, tmap_w, tmap_xp, counts, offsets, E, sb, d,
                             n, static_cast<int>(ldw), P, at);
 }
 
@@ -748,7 +768,11 @@ cudaError_t launch_tensor_experts_pair(const void* Wv, long long ldw, const int3
                                        const int32_t* offsets, StatusBlock* sb, int T,
                                        int d, int n, int k, int E, const __nv_bfloat16* xp, __nv_bfloat16* P,
                                        cudaStream_t stream) {
-  return launch_pair<false>(Wv, ldw, counts, offsets, sb, T, d, n, k, E, xp, P, AttendArgs{}, stream);
+  // At most 256 pairs per expert on average: the 384-pair tiles and the
+  // deeper ring; otherwise the 512-pair tiles.
+  if (static_cast<long long>(T) * k <= 256LL * E)
+    return launch_pair<false, NT_SMALL>(Wv, ldw, counts, offsets, sb, T, d, n, k, E, xp, P, AttendArgs{}, stream);
+  return launch_pair<false, NT>(Wv, ldw, counts, offsets, sb, T, d, n, k, E, xp, P, AttendArgs{}, stream);
 }
 
 size_t attend_part_bytes(int L, int E, int k, int n) {
@@ -770,7 +794,7 @@ cudaError_t launch_tensor_attend(const void* Wv, const int32_t* counts, const in
   cudaError_t err = launch_pdl(attend_coef_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, stream,
                                probs, perm, w32, L, k, nkv, G, coef);
   if (err != cudaSuccess) return err;
-  err = launch_pair<true>(Wv, n, counts, offsets, sb, L, d, n, k, E, xp, nullptr,
+  err = launch_pair<true, NT>(Wv, n, counts, offsets, sb, L, d, n, k, E, xp, nullptr,
                           AttendArgs{coef, part, 4 * nkv}, stream);
   if (err != cudaSuccess) return err;
   return launch_pdl(attend_reduce_kernel, dim3(static_cast<unsigned>(H * 4)), dim3(1024), 0, stream,
