@@ -182,9 +182,10 @@ cudaError_t launch_stream_experts(const void* x, const void* Wv, long long ldw, 
 // 8-row stages).
 size_t stream_experts_smem(int d, mova_dtype dt, int T, int n, int k, int E, int* stages_out);
 // Whether the weight-streaming kernel keeps every token's x in shared memory
-// for this batch (the mode in which it also performs the combine: v must be
-// given).
-bool stream_resident(int T, int d, mova_dtype dt);
+// for this batch (bf16, T <= 8, and its buffers fit; the mode in which it
+// also performs the combine and may route: v must be given).  Otherwise the
+// batch runs the per-chunk mode with a separate combine.
+bool stream_resident(int T, int d, int n, int k, int E, mova_dtype dt);
 
 // tcgen05 grouped GEMM (bf16): P[p, :] = SiLU(Wv[e] x[t]) as bf16 rows.
 // xp: T*k x d bf16 scratch for the pairs' x rows in grouped order.

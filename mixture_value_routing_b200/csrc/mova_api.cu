@@ -197,7 +197,7 @@ mova_status run_experts_and_combine(const void* x, mova_dtype dt, const void* Wv
   } else {
     if (stream_experts_smem(d, dt, T, n, k, E, nullptr) == 0) return MOVA_ERR_UNSUPPORTED;
     // Decode-sized bf16 batches fold the combine into the expert kernel.
-    fused_combine = T <= kFusedCombineMaxT && stream_resident(T, d, dt);
+    fused_combine = T <= kFusedCombineMaxT && stream_resident(T, d, n, k, E, dt);
     err = launch_stream_experts(x, Wv, ldw, dt, ws.counts, ws.offsets, ws.perm, w32, ws.active, ws.sb,
                                 T, d, n, k, E, static_cast<float*>(ws.P),
                                 fused_combine ? v : nullptr,
@@ -443,7 +443,7 @@ mova_status mova_value_routed_opts(const void* x, mova_dtype x_dt, const float* 
   // Decode batches on the weight-streaming path: the router computes the
   // logits only; the streaming kernel selects, groups and combines.
   const mova_path rp = path == MOVA_PATH_AUTO ? mova_auto_path(T, x_dt) : path;
-  if (rp == MOVA_PATH_STREAM && T <= kFusedCombineMaxT && stream_resident(T, d, x_dt) &&
+  if (rp == MOVA_PATH_STREAM && T <= kFusedCombineMaxT && stream_resident(T, d, n, k, E, x_dt) &&
       stream_experts_smem(d, x_dt, T, n, k, E, nullptr) != 0) {
     int S = 0;
     const bool one = o.decode_launches == 1;

@@ -159,14 +159,13 @@ stream_experts_kernel(const DT* __restrict__ x, const DT* __restrict__ Wv,
                       const int32_t* __restrict__ active, StatusBlock* __restrict__ sb, int T,
                       int d, int n, int k, float* __restrict__ P, int NS,
                       DT* __restrict__ v, RouteIn route,
-                      StreamFault fault, long long ldw) {
+                      StreamFault fault, long long ldw, bool resident) {
   constexpr bool kMma = sizeof(DT) == 2;
   constexpr int EL = Vec<DT>::EL;
   extern __shared__ __align__(128) uint8_t smem[];
   const size_t row_bytes = static_cast<size_t>(d) * sizeof(DT);
   const size_t pitch = row_bytes + 16;
   const size_t stage_bytes = pitch * kRowsPerStage;
-  const bool resident = is_resident(kMma, T);
   uint8_t* stages = smem;
   uint8_t* xs = smem + NS * stage_bytes;  // bf16: kTok padded x rows
   // Partial tiles of the consumer warps: one [warps][8][8] buffer per stage
@@ -716,22 +715,26 @@ cudaError_t reset_grid_barriers(cudaStream_t stream) {
   return cudaMemsetAsync(p, 0, sizeof(g_grid_bar), stream);
 }
 
-size_t stream_experts_smem(int d, mova_dtype dt, int T, int n, int k, int E, int* stages_out) {
-  const bool mma = dt == MOVA_BF16;
-  // Resident mode: the SiLU values of a CTA's rows (its ceil(n / CTAs)
-  // columns of each of at most min(E, T k) active experts, in whole
-  // stages) for all 8 token columns.
+namespace {
+
+// Resident mode's buffer of SiLU values: a CTA's rows (its ceil(n / CTAs)
+// columns of each of at most min(E, T k) active experts, in whole stages)
+// for all 8 token columns.
+size_t hv_bytes_for(int T, int n, int k, int E) {
   const int G = sm_count();
   const size_t rows = static_cast<size_t>(std::min(E, T * k)) * ((n + G - 1) / G);
-  const size_t hv_bytes =
-      is_resident(mma, T) ? (rows + kRowsPerStage - 1) / kRowsPerStage * kRowsPerStage * kTok * sizeof(float) : 0;
+  return (rows + kRowsPerStage - 1) / kRowsPerStage * kRowsPerStage * kTok * sizeof(float);
+}
+
+// Shared memory of a launch in the given mode: the most stages (up to
+// kStreamStages) that fit next to the fixed parts, whose partial-tile buffers
+// grow with the stage count; 0 if not even two fit.
+size_t smem_bytes(int d, bool mma, size_t hv_bytes, int* stages_out) {
   const size_t pitch = static_cast<size_t>(d) * (mma ? 2 : 4) + 16;
   const size_t stage_bytes = pitch * kRowsPerStage;
   // With the kernel's ~2.4 KB of static arrays, under the 227 KB a block
   // may opt in to.
   const size_t budget = 222 * 1024;
-  // The most stages (up to kStreamStages) that fit next to the fixed parts,
-  // whose partial-tile buffers grow with the stage count.
   for (int NS = kStreamStages; NS >= 2; --NS) {
     const size_t fixed = (mma ? kTok * pitch + red_slots(NS) * kConsumerWarps * 64 * sizeof(float) : 0) +
                          2 * kTok * sizeof(float) + 4 * 64 * sizeof(int) +
@@ -745,9 +748,16 @@ size_t stream_experts_smem(int d, mova_dtype dt, int T, int n, int k, int E, int
   return 0;
 }
 
-bool stream_resident(int T, int d, mova_dtype dt) {
-  (void)d;
-  return is_resident(dt == MOVA_BF16, T);
+}  // namespace
+
+bool stream_resident(int T, int d, int n, int k, int E, mova_dtype dt) {
+  const bool mma = dt == MOVA_BF16;
+  return is_resident(mma, T) && smem_bytes(d, mma, hv_bytes_for(T, n, k, E), nullptr) != 0;
+}
+
+size_t stream_experts_smem(int d, mova_dtype dt, int T, int n, int k, int E, int* stages_out) {
+  const bool res = stream_resident(T, d, n, k, E, dt);
+  return smem_bytes(d, dt == MOVA_BF16, res ? hv_bytes_for(T, n, k, E) : 0, stages_out);
 }
 
 cudaError_t launch_stream_experts(const void* x, const void* Wv, long long ldw, mova_dtype dt,
@@ -759,8 +769,9 @@ cudaError_t launch_stream_experts(const void* x, const void* Wv, long long ldw, 
   int NS = 0;
   const size_t smem = stream_experts_smem(d, dt, T, n, k, E, &NS);
   if (smem == 0) return cudaErrorInvalidValue;
-  // Resident mode always combines inside the kernel.
-  if (is_resident(dt == MOVA_BF16, T) && v == nullptr) return cudaErrorInvalidValue;
+  // Resident mode always combines inside the kernel, and only it routes.
+  const bool resident = stream_resident(T, d, n, k, E, dt);
+  if (resident != (v != nullptr) || (!resident && route.part != nullptr)) return cudaErrorInvalidValue;
   const dim3 grid(sm_count());
   const StreamFault fault = take_stream_fault();
   if (dt == MOVA_BF16) {
@@ -771,7 +782,7 @@ cudaError_t launch_stream_experts(const void* x, const void* Wv, long long ldw, 
     return launch_pdl(kern, grid, dim3(kThreads), smem, stream,
                       static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(Wv),
                       counts, offsets, perm, w32, active, sb, T, d, n, k, P, NS,
-                      static_cast<__nv_bfloat16*>(v), route, fault, ldw);
+                      static_cast<__nv_bfloat16*>(v), route, fault, ldw, resident);
   }
   auto kern = stream_experts_kernel<float>;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -779,7 +790,7 @@ cudaError_t launch_stream_experts(const void* x, const void* Wv, long long ldw, 
   if (err != cudaSuccess) return err;
   return launch_pdl(kern, grid, dim3(kThreads), smem, stream, static_cast<const float*>(x),
                     static_cast<const float*>(Wv), counts, offsets, perm, w32, active, sb, T, d, n,
-                    k, P, NS, static_cast<float*>(v), route, fault, ldw);
+                    k, P, NS, static_cast<float*>(v), route, fault, ldw, resident);
 }
 
 }  // namespace mova

@@ -225,6 +225,14 @@ def test_full_decode_column_ranges(api, T, d, E, k, n):
     _full(api, T, d, E, k, n, "bf16", seed=n + k, path="stream")
 
 
+def test_full_stream_widest_rows_many_experts(api):
+    """Decode batch at the widest rows (d = 4544) with k = 8 of 64 experts
+    and n = 1024: the resident mode's buffers do not fit next to its x tile
+    and two stages, so the batch takes the per-chunk mode with a separate
+    combine, and is still supported."""
+    _full(api, 8, 4544, 64, 8, 1024, "bf16", seed=4544, path="stream")
+
+
 @pytest.mark.parametrize("T,d", [(8, 3072), (4, 4096), (3, 4544)])
 def test_full_stream_resident_boundary(api, T, d):
     """Decode batches at and near the widest rows the weight-streaming
