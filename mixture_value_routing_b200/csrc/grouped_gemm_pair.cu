@@ -175,9 +175,11 @@ struct AttendArgs {
 // Tensor memory holds two accumulator regions of 256 columns.  A tile of at
 // most 256 pairs takes one region, alternating between the two, so its
 // epilogue overlaps the next tile's MMAs; a larger tile takes both (pairs
-// 0..255 in the next region, the rest in the other).  Every role walks the
-// cluster's tile sequence and applies this rule, so they agree on which
-// region holds what, and on each region's use count (its barrier parity).
+// 0..255 in the next region, the rest in the other), and the tile after it
+// starts in the region of that smaller second accumulator, which its
+// epilogue hands back first.  Every role walks the cluster's tile sequence
+// and applies this rule, so they agree on which region holds what, and on
+// each region's use count (its barrier parity).
 struct Regions {
   int next = 0;
   int uses0 = 0, uses1 = 0;
@@ -189,12 +191,8 @@ struct Regions {
   // if none).
   __device__ __forceinline__ void take(const PTile& tl, int& r0, int& r1) {
     r0 = next;
-    if (tl.N1 > 0) {
-      r1 = next ^ 1;
-    } else {
-      r1 = -1;
-      next ^= 1;
-    }
+    r1 = tl.N1 > 0 ? next ^ 1 : -1;
+    next ^= 1;
   }
 };
 
@@ -558,7 +556,8 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_w, const __gri
       // The accumulator's columns are read in two halves of 128 (SiLU,
       // rounded to bf16, two per word): the first half is read and stored,
       // then the second half is read, the accumulator is handed back to the
-      // MMA, and the second half is stored.  (Three of the ten warps share a
+      // MMA, and the second half is stored.  An accumulator of at most 128
+      // columns is handed back right after its only read.  (Three of the ten warps share a
       // sub-partition's 16K registers, so a thread cannot hold all 256
       // columns at once.)
       // The warp's 32 weight rows are all below n or all at or above it (n
@@ -586,7 +585,7 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_w, const __gri
             }
           }
         }
-        if (h == 1) {
+        if (h == (N > 128 ? 1 : 0)) {  // after the last read of the accumulator
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive_cluster(empty_cl);
