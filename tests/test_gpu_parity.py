@@ -802,3 +802,29 @@ def test_value_attend_host_buffers(api, L):
     ref = _attend_ref(bat, lay, probs)
     err = np.abs(o.numpy().astype(np.float64) - ref)
     assert (err <= 1e-4 * np.maximum(1.0, np.abs(ref))).all(), err.max()
+
+
+def test_host_buffer_calls_on_two_streams(api):
+    """Two host-buffer calls in flight on two streams, each with its own
+    workspace (as the benchmark's end-to-end loop runs them), give the same
+    results as the same calls one after another: the library keeps no state
+    between calls that two streams could share."""
+    d, E, k, n = 2560, 64, 4, 1024
+    lay = _layer(77, d, E, n, "bf16")
+    Wr, br, Wv = P.dev(lay.Wr, "f32"), P.dev(lay.br, "f32"), P.dev(lay.Wv, "bf16")
+    batches = [MI.make_batch(T, 77, step=s, dtype="bf16", d=d) for s, T in enumerate((8, 8, 300, 300))]
+    xs = [_pinned(P.dev(b.x, "bf16")) for b in batches]
+    ref = [api.value_routed_host(x, Wr, br, Wv, k, 2.5) for x in xs]
+    torch.cuda.synchronize()
+    streams = [torch.cuda.Stream() for _ in range(2)]
+    wss = [torch.empty(api.workspace_size_host(300, d, E, k, n), dtype=torch.uint8, device="cuda")
+           for _ in range(2)]
+    for rep in range(3):
+        outs = []
+        for i, x in enumerate(xs):
+            out = torch.empty((x.shape[0], n), dtype=torch.bfloat16).pin_memory()
+            outs.append(api.value_routed_host(x, Wr, br, Wv, k, 2.5, out=out, ws=wss[i % 2],
+                                              stream=streams[i % 2]))
+        torch.cuda.synchronize()
+        for i in range(len(xs)):
+            assert torch.equal(outs[i], ref[i]), f"call {i} of round {rep} differs"
