@@ -331,8 +331,9 @@ def measure_workload(a, name, K, layers, device, dist_on, world, rank, peaks, pe
             idx, w = routing[l]
             api.value(xs[l], idx, w, Wv, ws=ws, events=events)
 
-    # Distinct experts each layer's step streams, and the busiest expert's load.
-    distinct, max_load = [], []
+    # Distinct experts each layer's step streams, the busiest expert's load,
+    # and the first step's loads of its active experts (descending).
+    distinct, max_load, loads0 = [], [], []
     for l in range(L):
         if routing is None:
             _, idx_l, _ = api.value_routed(xs[l], *layers.get(l, cfg["bias"]), k, MI.SCALE,
@@ -342,6 +343,8 @@ def measure_workload(a, name, K, layers, device, dist_on, world, rank, peaks, pe
         cnt = torch.bincount(idx_l.long().flatten(), minlength=E)
         distinct.append(int((cnt > 0).sum().item()))
         max_load.append(int(cnt.max().item()))
+        if l == 0:
+            loads0 = sorted((int(c) for c in cnt.tolist() if c > 0), reverse=True)
 
     for i in range(a.warmup):
         step(i)
@@ -441,6 +444,7 @@ def measure_workload(a, name, K, layers, device, dist_on, world, rank, peaks, pe
                    "l2": f"weights rotate over {L} layers ({L * E * n * d * xs_b / 1e9:.2f} GB) "
                          f"> 126 MB L2; no flush",
                    "distinct_experts_per_step": distinct, "max_expert_load_per_step": max_load,
+                   "expert_loads_first_step": loads0,
                    "timing": "one CUDA graph of the K steps, replayed once between barrier + "
                              "synchronize; CUDA events on the replaying stream"},
         "stage_us": {s: round(u, 3) for s, u in stage_avg_us.items()},
