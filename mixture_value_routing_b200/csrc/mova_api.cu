@@ -565,6 +565,13 @@ static bool host_ws_ok(const void* ws, size_t ws_bytes, size_t need) {
   return need != 0 && ws_bytes >= need && (reinterpret_cast<uintptr_t>(ws) & 255) == 0;
 }
 
+// The one support condition the device call checks only on its chosen path:
+// the weight-streaming kernel's shared memory for this d.  Checked here
+// first, so that nothing is enqueued when the call would be refused.
+static bool host_path_supported(int T, int d, int E, int k, int n, mova_dtype dt) {
+  return mova_auto_path(T, dt) != MOVA_PATH_STREAM || stream_experts_smem(d, dt, T, n, k, E, nullptr) != 0;
+}
+
 mova_status mova_value_routed_host(const void* x_host, mova_dtype x_dt, const float* Wr, const float* br,
                                    const void* Wv, mova_dtype wv_dt, int T, int d, int E, int k, int n,
                                    float scale, void* v_host, int32_t* idx_host, float* w_host, void* ws,
@@ -576,6 +583,7 @@ mova_status mova_value_routed_host(const void* x_host, mova_dtype x_dt, const fl
   if (!x_host || !Wr || !br || !Wv || !v_host || !ws) return MOVA_ERR_INVALID_ARG;
   if (!aligned16(Wr) || !aligned16(Wv)) return MOVA_ERR_INVALID_ARG;
   if (!host_ws_ok(ws, ws_bytes, mova_workspace_size_host(T, d, E, k, n))) return MOVA_ERR_INVALID_ARG;
+  if (!host_path_supported(T, d, E, k, n, x_dt)) return MOVA_ERR_UNSUPPORTED;
   const size_t base = align256(mova_workspace_size(T, d, E, k, n));
   const size_t Tz = static_cast<size_t>(T), es = act_size(x_dt);
   char* x_dev = static_cast<char*>(ws) + base;
@@ -606,6 +614,7 @@ mova_status mova_value_host(const void* x_host, mova_dtype x_dt, const void* idx
   if (!x_host || !idx_host || !w_host || !Wv || !v_host || !ws) return MOVA_ERR_INVALID_ARG;
   if (!aligned16(Wv)) return MOVA_ERR_INVALID_ARG;
   if (!host_ws_ok(ws, ws_bytes, mova_workspace_size_host(T, d, E, k, n))) return MOVA_ERR_INVALID_ARG;
+  if (!host_path_supported(T, d, E, k, n, x_dt)) return MOVA_ERR_UNSUPPORTED;
   const size_t base = align256(mova_workspace_size(T, d, E, k, n));
   const size_t Tz = static_cast<size_t>(T), es = act_size(x_dt);
   char* x_dev = static_cast<char*>(ws) + base;

@@ -174,9 +174,9 @@ stream_experts_kernel(const DT* __restrict__ x, const DT* __restrict__ Wv,
   float* tok_w = red + (kMma ? red_slots(NS) * kConsumerWarps * 64 : 0);  // weights of the staged pairs
   int* tok_p = reinterpret_cast<int*>(tok_w + kTok);           // their grouped positions
   // Resident mode: every token's x row stays in the x tile for the whole
-  // kernel (the mma computes all 8 token columns for every expert; each pair
-  // reads its token's column), and the pair tables below replace all global
-  // loads of the grouping in the loop.
+  // kernel (the mma computes all 8 token columns for every expert; the final
+  // combine reads each pair's token column), and the tables below replace
+  // all global loads of the grouping.
   int* slot_act = tok_p + kTok;                             // [64] active-list index of pair f's expert
   int* act_cnt = slot_act + 64;                             // [64] pairs per active expert
   int* act_off = act_cnt + 64;                              // [64] first position
