@@ -41,7 +41,7 @@
  *  - Supported on the GPU: 1 <= E <= 64, 1 <= k <= min(E, 8), d % 64 == 0,
  *    n % 128 == 0, T * k <= 131072; dtypes x/Wv/v all fp32, or all bf16
  *    (router Wr/br always fp32).  The weight-streaming expert kernel also
- *    needs d <= 4544 (bf16) or d <= 3456 (fp32).  Anything else returns
+ *    needs d <= 4608 (bf16) or d <= 3456 (fp32).  Anything else returns
  *    MOVA_ERR_UNSUPPORTED; there is no fallback path.
  */
 #ifndef MOVA_H_

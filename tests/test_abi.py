@@ -183,9 +183,9 @@ def test_host_buffer_forms_validation(lib):
     assert routed(BF16, F32, T, host, fake) == _lib.ERR_UNSUPPORTED         # Wv dtype must equal x's
     assert routed(BF16, BF16, T, host, None) == _lib.ERR_INVALID_ARG        # no output buffer
     assert routed(BF16, BF16, T, base, fake) == _lib.ERR_INVALID_ARG        # room for the call, not the staging
-    # rows wider than the streaming kernel holds (d = 4608 at T = 8): refused before any copy is enqueued
-    wide = lib.mova_workspace_size_host(T, 4608, E, k, n)
-    assert lib.mova_value_routed_host(fake, BF16, fake, fake, fake, BF16, T, 4608, E, k, n, 2.5, fake, None, None,
+    # rows wider than the streaming kernel holds (d = 4672 at T = 8): refused before any copy is enqueued
+    wide = lib.mova_workspace_size_host(T, 4672, E, k, n)
+    assert lib.mova_value_routed_host(fake, BF16, fake, fake, fake, BF16, T, 4672, E, k, n, 2.5, fake, None, None,
                                       fake, wide, None) == _lib.ERR_UNSUPPORTED
     assert lib.mova_value_host(fake, BF16, fake, F32, fake, F16, fake, BF16, T, d, E, k, n, fake, fake,
                                host, None) == _lib.ERR_UNSUPPORTED        # idx must be int32 or int8

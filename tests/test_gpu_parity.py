@@ -226,17 +226,18 @@ def test_full_decode_column_ranges(api, T, d, E, k, n):
 
 
 def test_full_stream_widest_rows_many_experts(api):
-    """Decode batch at the widest rows (d = 4544) with k = 8 of 64 experts
-    and n = 1024: the resident mode's buffers do not fit next to its x tile
-    and two stages, so the batch takes the per-chunk mode with a separate
-    combine, and is still supported."""
+    """Decode batch with wide rows (d = 4544) and k = 8 of 64 experts, n =
+    1024: the resident mode's buffers do not fit next to its x tile and two
+    stages, so the batch takes the per-chunk mode with a separate combine,
+    and is still supported."""
     _full(api, 8, 4544, 64, 8, 1024, "bf16", seed=4544, path="stream")
 
 
-@pytest.mark.parametrize("T,d", [(8, 3072), (4, 4096), (3, 4544)])
+@pytest.mark.parametrize("T,d", [(8, 3072), (4, 4096), (3, 4544), (8, 4608)])
 def test_full_stream_resident_boundary(api, T, d):
     """Decode batches at and near the widest rows the weight-streaming
-    kernel holds (two stages of 8 rows plus the resident x tile)."""
+    kernel holds: two stages of 8 rows plus the x tile (resident up to
+    d = 4544 here; d = 4608 runs the per-chunk mode)."""
     _full(api, T, d, 16, 4, 256, "bf16", seed=d, path="stream")
 
 
