@@ -193,6 +193,11 @@ stream_experts_kernel(const DT* __restrict__ x, const DT* __restrict__ Wv,
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  // Resident mode: this CTA's output columns [r_lo, r_lo + nr), formed here,
+  // off the path from the selection to the first weight copy (n * CTAs
+  // stays far below 2^32).
+  const int r_lo = static_cast<int>(static_cast<unsigned>(n) * blockIdx.x / gridDim.x);
+  const int nr = static_cast<int>(static_cast<unsigned>(n) * (blockIdx.x + 1) / gridDim.x) - r_lo;
   if (threadIdx.x == 0) {
     for (int s = 0; s < NS; ++s) {
       mbar_init(&full[s], 1);
@@ -381,8 +386,6 @@ stream_experts_kernel(const DT* __restrict__ x, const DT* __restrict__ Wv,
   // over the CTAs, expert-major, so the staged x rows change only with the
   // expert.
   const int units_per_expert = n / kRowsPerStage;
-  const int r_lo = static_cast<int>(static_cast<long long>(n) * blockIdx.x / gridDim.x);
-  const int nr = static_cast<int>(static_cast<long long>(n) * (blockIdx.x + 1) / gridDim.x) - r_lo;
   const int rows_total = nact * nr;
   const int units = resident ? (rows_total + kRowsPerStage - 1) / kRowsPerStage : nact * units_per_expert;
   const int u0 = resident ? 0 : static_cast<int>(static_cast<long long>(units) * blockIdx.x / gridDim.x);
