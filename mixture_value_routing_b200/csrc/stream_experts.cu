@@ -352,10 +352,16 @@ stream_experts_kernel(const DT* __restrict__ x, const DT* __restrict__ Wv,
       // The active experts (ascending), from the selection alone: the same
       // list the grouping builds.
       asm volatile("bar.sync 3, %0;" ::"n"((kConsumerWarps + 1) * 32) : "memory");
-      uint64_t m = 0;
-      for (int i = lane; i < T * k; i += 32) m |= 1ull << r_sel[i];
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) m |= __shfl_xor_sync(0xffffffffu, m, o);
+      // Experts 0-31 and 32-63 as two 32-bit masks, each OR-reduced over
+      // the warp in one instruction.
+      uint32_t m_lo = 0, m_hi = 0;
+      for (int i = lane; i < T * k; i += 32) {
+        const int e = r_sel[i];
+        if (e < 32) m_lo |= 1u << e; else m_hi |= 1u << (e - 32);
+      }
+      m_lo = __reduce_or_sync(0xffffffffu, m_lo);
+      m_hi = __reduce_or_sync(0xffffffffu, m_hi);
+      const uint64_t m = (static_cast<uint64_t>(m_hi) << 32) | m_lo;
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         const int e = lane + 32 * h;
