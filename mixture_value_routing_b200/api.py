@@ -5,8 +5,11 @@ torch CUDA tensors (torch only provides device memory and the stream).
     idx, w = route(x, Wr, br)
     v = value(x, idx, w, Wv)                    # routing given (compact cache)
 
-Every function enqueues on torch's current CUDA stream and returns without
-synchronising.  Device-side checks are read with get_status().
+Every function enqueues on torch's current CUDA stream (the host-buffer forms:
+on `stream` if given) and returns without synchronising.  Device-side checks
+are read with get_status().  A call given no `ws` uses the workspace this
+module keeps for its device and stream, so calls on different streams may
+overlap on the GPU.  Calls that share a `ws` must run on one stream.
 """
 from __future__ import annotations
 
@@ -34,13 +37,18 @@ except AttributeError:  # pragma: no cover - older torch
     _raw_stream = None
 
 
+def _current_stream_handle() -> int:
+    """The handle of the current stream of the current device."""
+    if _raw_stream is not None:
+        return int(_raw_stream(torch.cuda.current_device()))
+    return int(torch.cuda.current_stream().cuda_stream)
+
+
 def _stream(stream: Optional["torch.cuda.Stream"] = None):
     """The handle of `stream`, else of the current stream of the current device."""
     if stream is not None:
         return ctypes.c_void_p(stream.cuda_stream)
-    if _raw_stream is not None:
-        return ctypes.c_void_p(_raw_stream(torch.cuda.current_device()))
-    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    return ctypes.c_void_p(_current_stream_handle())
 
 
 def _need(t: torch.Tensor, name: str, dtypes=None, ndim=None):
@@ -55,7 +63,7 @@ def _need(t: torch.Tensor, name: str, dtypes=None, ndim=None):
 
 
 class Workspace:
-    """A device workspace that grows on demand (one per device)."""
+    """A device workspace that grows on demand."""
 
     def __init__(self):
         self.buf: Optional[torch.Tensor] = None
@@ -66,21 +74,36 @@ class Workspace:
         return self.buf
 
 
+# The workspaces of calls made without `ws`: one per (device, stream).  A call
+# leaves its routing, grouping and expert rows in its workspace until its last
+# kernel has run, so calls that may overlap on the GPU -- calls on different
+# streams -- must not share one.  Calls on one stream run in order and share
+# that stream's workspace.
 _WS = {}
 
 
 def _devkey(device) -> torch.device:
     dev = torch.device(device)
-    if dev.index is None:
+    if dev.type == "cuda" and dev.index is None:
         dev = torch.device(dev.type, torch.cuda.current_device())
     return dev
 
 
-def _workspace(nbytes: int, device) -> torch.Tensor:
+def _workspace(nbytes: int, device, stream: Optional["torch.cuda.Stream"] = None) -> torch.Tensor:
+    """The default workspace of `stream` (else of the current stream) on
+    `device`, grown to at least `nbytes`.  It is allocated while that stream is
+    current: torch's caching allocator then keeps the memory of a buffer that
+    a later, larger call replaces from every other stream's allocations until
+    this stream has passed its last use."""
     dev = _devkey(device)
-    if dev not in _WS:
-        _WS[dev] = Workspace()
-    return _WS[dev].get(nbytes, dev)
+    handle = int(stream.cuda_stream) if stream is not None else _current_stream_handle()
+    key = (dev, handle)
+    if key not in _WS:
+        _WS[key] = Workspace()
+    if stream is None:
+        return _WS[key].get(nbytes, dev)
+    with torch.cuda.stream(stream):
+        return _WS[key].get(nbytes, dev)
 
 
 @functools.lru_cache(maxsize=256)
@@ -339,7 +362,7 @@ def value_routed_host(x: torch.Tensor, Wr: torch.Tensor, br: torch.Tensor, Wv: t
         idx = torch.empty((T, k), dtype=torch.int32, pin_memory=True)
         w = torch.empty((T, k), dtype=torch.float32, pin_memory=True)
     if ws is None:
-        ws = _workspace(workspace_size_host(T, d, E, k, n), Wv.device)
+        ws = _workspace(workspace_size_host(T, d, E, k, n), Wv.device, stream)
     _lib.check(_lib.load().mova_value_routed_host(
         _ptr(x), _DT[x.dtype], _ptr(Wr), _ptr(br), _ptr(Wv), _DT[Wv.dtype], T, d, E, k, n, float(scale),
         _ptr(v), _ptr(idx), _ptr(w), _ptr(ws), ws.numel(), _stream(stream)), "mova_value_routed_host")
@@ -359,7 +382,7 @@ def value_host(x: torch.Tensor, idx: torch.Tensor, w: torch.Tensor, Wv: torch.Te
     k = idx.shape[1]
     v = _host_out(out, (T, n), x.dtype)
     if ws is None:
-        ws = _workspace(workspace_size_host(T, d, E, k, n), Wv.device)
+        ws = _workspace(workspace_size_host(T, d, E, k, n), Wv.device, stream)
     _lib.check(_lib.load().mova_value_host(
         _ptr(x), _DT[x.dtype], _ptr(idx), _DT[idx.dtype], _ptr(w), _DT[w.dtype], _ptr(Wv), _DT[Wv.dtype],
         T, d, E, k, n, _ptr(v), _ptr(ws), ws.numel(), _stream(stream)), "mova_value_host")
@@ -385,7 +408,7 @@ def value_attend_host(x: torch.Tensor, idx: torch.Tensor, w: torch.Tensor, Wv: t
         raise ValueError("probs: (H, L) for the L cached positions of x")
     o = _host_out(out, (H, 128), torch.float32)
     if ws is None:
-        ws = _workspace(attend_workspace_size_host(L, d, E, k, n, H), Wv.device)
+        ws = _workspace(attend_workspace_size_host(L, d, E, k, n, H), Wv.device, stream)
     _lib.check(_lib.load().mova_value_attend_host(
         _ptr(x), _ptr(idx), _DT[idx.dtype], _ptr(w), _DT[w.dtype], _ptr(Wv), L, d, E, k, n, _ptr(probs), H,
         _ptr(o), _ptr(ws), ws.numel(), _stream(stream)), "mova_value_attend_host")
@@ -421,10 +444,17 @@ def arm_stream_stall(stall_stage: int, limit_cycles: int) -> None:
                "mova_selftest_arm_stream_stall")
 
 
-def get_status(ws: Optional[torch.Tensor] = None, device=None):
-    """(status name, detail) of the last value call on this workspace."""
+def get_status(ws: Optional[torch.Tensor] = None, device=None, stream=None):
+    """(status name, detail) of the last value call on this workspace; without
+    `ws`, on the default workspace of `stream` (else of the current stream),
+    i.e. of the last call made there without `ws`.  Waits for that stream."""
     if ws is None:
-        ws = _WS[_devkey(device if device is not None else "cuda")].buf
+        dev = _devkey(device if device is not None else "cuda")
+        handle = int(stream.cuda_stream) if stream is not None else _current_stream_handle()
+        entry = _WS.get((dev, handle))
+        if entry is None or entry.buf is None:
+            raise ValueError(f"no call on {dev} has used the default workspace of this stream")
+        ws = entry.buf
     detail = ctypes.c_int32(0)
-    code = _lib.load().mova_get_status(_ptr(ws), ctypes.byref(detail), _stream())
+    code = _lib.load().mova_get_status(_ptr(ws), ctypes.byref(detail), _stream(stream))
     return _lib.STATUS_NAMES.get(code, str(code)), int(detail.value)

@@ -829,3 +829,33 @@ def test_host_buffer_calls_on_two_streams(api):
         torch.cuda.synchronize()
         for i in range(len(xs)):
             assert torch.equal(outs[i], ref[i]), f"call {i} of round {rep} differs"
+
+
+def test_default_workspaces_on_two_streams(api):
+    """Calls given no workspace, in flight on two streams at once -- the
+    host-buffer form with `stream=` and the device form under a stream
+    context -- give the results of the same calls made one after another:
+    each stream has a default workspace of its own, so no call reads another
+    stream's routing, grouping or expert rows."""
+    d, E, k, n = 2560, 64, 4, 1024
+    lay = _layer(78, d, E, n, "bf16")
+    Wr, br, Wv = P.dev(lay.Wr, "f32"), P.dev(lay.br, "f32"), P.dev(lay.Wv, "bf16")
+    batches = [MI.make_batch(T, 78, step=s, dtype="bf16", d=d) for s, T in enumerate((8, 300, 8, 300))]
+    xd = [P.dev(b.x, "bf16") for b in batches]
+    xs = [_pinned(x) for x in xd]
+    ref = [api.value_routed(x, Wr, br, Wv, k, 2.5).cpu() for x in xd]  # serial, current stream
+    streams = [torch.cuda.Stream() for _ in range(2)]
+    for s in streams:
+        s.wait_stream(torch.cuda.current_stream())
+    for rep in range(3):
+        host_out = [api.value_routed_host(x, Wr, br, Wv, k, 2.5, stream=streams[i % 2]) for i, x in enumerate(xs)]
+        dev_out = []
+        for i, x in enumerate(xd):
+            with torch.cuda.stream(streams[i % 2]):
+                dev_out.append(api.value_routed(x, Wr, br, Wv, k, 2.5))
+        torch.cuda.synchronize()
+        for i in range(len(xs)):
+            assert torch.equal(host_out[i], ref[i]), f"host-buffer call {i} of round {rep} differs"
+            assert torch.equal(dev_out[i].cpu(), ref[i]), f"device call {i} of round {rep} differs"
+    for s in streams:
+        assert api.get_status(stream=s)[0] == "MOVA_OK"
