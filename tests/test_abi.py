@@ -203,3 +203,94 @@ def test_host_buffer_forms_validation(lib):
     assert attend(12, fake, 1 << 30) == _lib.ERR_UNSUPPORTED
     assert attend(32, None, 1 << 30) == _lib.ERR_INVALID_ARG
     assert attend(32, fake, 4096) == _lib.ERR_INVALID_ARG
+
+
+def _c_type_to_ctypes(decl: str):
+    """The ctypes type that marshals a C parameter or return type of the header."""
+    t = " ".join(decl.replace("const", " ").split())
+    if "*" in t:
+        return ctypes.c_char_p if t.startswith("char") else ctypes.c_void_p
+    base = re.sub(r"\s*\b[A-Za-z_]\w*$", "", t) if len(t.split()) > 1 else t
+    return {"size_t": ctypes.c_size_t, "long long": ctypes.c_longlong,
+            "unsigned long long": ctypes.c_ulonglong, "float": ctypes.c_float, "int": ctypes.c_int,
+            "int32_t": ctypes.c_int32, "mova_dtype": ctypes.c_int, "mova_path": ctypes.c_int,
+            "mova_status": ctypes.c_int}[base]
+
+
+def _prototypes():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    src = re.sub(r"//[^\n]*", "", src)
+    out = {}
+    for m in re.finditer(r"([A-Za-z_][\w \t\*]*?)\s*\b(mova_[a-z_]+)\s*\(([^()]*)\)\s*;", src):
+        ret, name, params = m.group(1).strip(), m.group(2), m.group(3).strip()
+        ret = ret.split("\n")[-1].strip()
+        args = [] if params in ("", "void") else [p.strip() for p in params.split(",")]
+        out[name] = (_c_type_to_ctypes(ret + " r"), [_c_type_to_ctypes(a) for a in args])
+    return out
+
+
+def test_binding_signatures_match_the_header():
+    """Every ctypes prototype of the binding has the header's return type and
+    parameter types, one for one: a dropped, swapped or mistyped argument
+    would otherwise reach the library as garbage without any error."""
+    protos = _prototypes()
+    assert set(protos) == set(_lib.SIGNATURES)
+    for name, (ret, args) in protos.items():
+        b_ret, b_args = _lib.SIGNATURES[name]
+        assert b_ret == ret, (name, "return", b_ret, ret)
+        assert len(b_args) == len(args), (name, len(b_args), len(args))
+        for i, (b, h) in enumerate(zip(b_args, args)):
+            assert b == h or (ctypes.sizeof(b) == ctypes.sizeof(h) and b not in (ctypes.c_float,)
+                              and h not in (ctypes.c_float,) and (b is ctypes.c_void_p) == (h is ctypes.c_void_p)), \
+                (name, i, b, h)
+
+
+def test_options_struct_matches_the_header():
+    src = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    body = re.search(r"typedef struct mova_options \{(.*?)\} mova_options;", src, re.S).group(1)
+    fields = [f.strip() for f in body.split(";") if f.strip()]
+    names = [re.search(r"(\w+)$", f).group(1) for f in fields]
+    assert names == [n for n, _ in _lib.Options._fields_]
+    for f, (_, ct) in zip(fields, _lib.Options._fields_):
+        assert ctypes.sizeof(ct) == ctypes.sizeof(_c_type_to_ctypes(f)), f
+
+
+def test_header_is_plain_c_and_links(lib, tmp_path):
+    """The header compiles as C11 with warnings as errors, and a C program
+    linked against libmova.so makes host-only calls: the library is usable
+    without Python or C++."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    prog = tmp_path / "abi.c"
+    prog.write_text(r'''
+#include <stdio.h>
+#include <string.h>
+#include "mova.h"
+int main(void) {
+  if (strcmp(mova_status_str(MOVA_ERR_TIMEOUT), "MOVA_ERR_TIMEOUT") != 0) return 1;
+  if (mova_workspace_size(8, 2560, 64, 4, 1024) == 0) return 2;
+  if (mova_workspace_size(8, 2560, 65, 4, 1024) != 0) return 3;      /* E > 64 unsupported */
+  if (mova_auto_path(4096, MOVA_BF16) != MOVA_PATH_TENSOR) return 4;
+  if (mova_value_routed(NULL, MOVA_BF16, NULL, NULL, NULL, MOVA_BF16, 8, 2560, 64, 4, 1024, 2.5f,
+                        NULL, NULL, NULL, NULL, 0, NULL) != MOVA_ERR_INVALID_ARG) return 5;
+  mova_options o;
+  memset(&o, 0, sizeof o);
+  o.router_partitions = 3;                                          /* unsupported */
+  if (mova_route_opts(NULL, MOVA_BF16, NULL, NULL, 8, 2560, 64, 4, 2.5f, NULL, NULL, &o, NULL)
+      != MOVA_ERR_UNSUPPORTED) return 6;
+  puts("ok");
+  return 0;
+}
+''')
+    exe = tmp_path / "abi"
+    libdir = os.path.dirname(_lib.LIB_PATH)
+    r = subprocess.run([cc, "-std=c11", "-Wall", "-Wextra", "-Werror", "-I", os.path.join(ROOT, "include"),
+                        str(prog), "-o", str(exe), "-L", libdir, "-lmova", f"-Wl,-rpath,{libdir}"],
+                       capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert r.returncode == 0 and r.stdout.strip() == "ok", (r.returncode, r.stdout, r.stderr)
