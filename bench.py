@@ -287,6 +287,19 @@ def _replay_for(graph, seconds, step_s, K):
     return reps
 
 
+def workload_config(a, name, world):
+    """The `config` of a workload's record: what the workload is and how L2 is
+    kept from serving the weights, the same on the reference arm's line as on
+    this one.  What a run measured (the routing's expert counts) and how it
+    was timed go under the record's "run" key."""
+    cfg = MI.WORKLOADS[name]
+    T, xs_b = cfg["T"], 2 if cfg["dtype"] == "bf16" else 4
+    L, d, E, n = max(1, a.layers), MI.D_MODEL, MI.N_EXPERTS, MI.N_OUT
+    return {"workload": WORKLOAD_TEXT[name], "tokens_per_step_per_gpu": T, "layers_rotated": L,
+            "l2": f"weights rotate over {L} layers ({L * E * n * d * xs_b / 1e9:.2f} GB) > 126 MB L2; no flush",
+            "parallelism": f"dp{world} (independent batches, no collective)"}
+
+
 def measure_workload(a, name, K, layers, device, dist_on, world, rank, peaks, peak_src):
     """One workload: W warm-up steps, then exactly K steps in one CUDA graph
     timed with CUDA events between barrier + synchronize (max over ranks);
@@ -439,14 +452,11 @@ def measure_workload(a, name, K, layers, device, dist_on, world, rank, peaks, pe
     rec = {
         "value": round(value, 1), "unit": "tokens/s", "steps": K, "warmup": a.warmup,
         "ms_per_step": round(ms_per_step, 5), "dtype": dtype,
-        "config": {"workload": WORKLOAD_TEXT[name], "tokens_per_step_per_gpu": T,
-                   "layers_rotated": L, "expert_path": path,
-                   "l2": f"weights rotate over {L} layers ({L * E * n * d * xs_b / 1e9:.2f} GB) "
-                         f"> 126 MB L2; no flush",
-                   "distinct_experts_per_step": distinct, "max_expert_load_per_step": max_load,
-                   "expert_loads_first_step": loads0,
-                   "timing": "one CUDA graph of the K steps, replayed once between barrier + "
-                             "synchronize; CUDA events on the replaying stream"},
+        "config": workload_config(a, name, world),
+        "run": {"expert_path": path, "distinct_experts_per_step": distinct,
+                "max_expert_load_per_step": max_load, "expert_loads_first_step": loads0,
+                "timing": "one CUDA graph of the K steps, replayed once between barrier + "
+                          "synchronize; CUDA events on the replaying stream"},
         "stage_us": {s: round(u, 3) for s, u in stage_avg_us.items()},
         "event_pair_us": round(empty_us, 3),
         "stage_timing": f"second replay of the K steps with stage events ({prof_ms / K * 1e3:.2f} us/step); "
@@ -598,7 +608,7 @@ def run_mova(a):
         "steps": a.steps, "warmup": a.warmup, "ms_per_step": h["ms_per_step"],
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": h["dtype"],
         "data": "synthetic (seeded; mova_inputs)",
-        "config": dict(h["config"], parallelism=f"dp{world} (independent batches, no collective)"),
+        "config": h["config"], "run": h["run"],
         "stage_us": h["stage_us"], "event_pair_us": h["event_pair_us"], "stage_timing": h["stage_timing"],
         "roofline": h["roofline"], "e2e": h["e2e"], "gpu_launches": h["gpu_launches"], "clocks": h["clocks"],
     }
@@ -722,7 +732,7 @@ def run_reference(a):
             "ms_per_step": round(1e3 * cb["seconds"] / max(1, cb["steps_timed"]), 3),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "f64", "data": "synthetic (seeded; mova_inputs)",
-            "config": {"workload": WORKLOAD_TEXT[a.workload]},
+            "config": workload_config(a, a.workload, world),
             "cpu_baseline": cb,
             "e2e": {"value": cb["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}

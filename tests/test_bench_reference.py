@@ -30,6 +30,13 @@ def test_reference_arm_line_on_rank0():
     assert d["e2e"] == {"value": d["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0,
                         "d2h_bytes_per_step": 0}
     assert d["config"]["workload"].startswith("decode step T=8")
+    # The reference arm describes the workload exactly as the GPU arm's line
+    # does (both build it with bench.workload_config), so the two lines' configs
+    # compare equal.
+    sys.path.insert(0, ROOT)
+    import bench
+    assert d["config"] == bench.workload_config(bench.parse(["--steps", "1", "--warmup", "3"]), "decode", 1)
+    assert set(d["config"]) == {"workload", "tokens_per_step_per_gpu", "layers_rotated", "l2", "parallelism"}
 
 
 def test_reference_arm_other_ranks_print_nothing():
