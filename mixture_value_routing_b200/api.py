@@ -106,6 +106,14 @@ def _workspace(nbytes: int, device, stream: Optional["torch.cuda.Stream"] = None
         return _WS[key].get(nbytes, dev)
 
 
+def release_workspaces() -> None:
+    """Drop the default workspaces (each stream that ran a call without `ws`
+    keeps one, sized for its largest call, until this is called).  Safe with
+    calls still in flight: torch's caching allocator reuses a freed buffer
+    only for later work on the stream that used it."""
+    _WS.clear()
+
+
 @functools.lru_cache(maxsize=256)
 def workspace_size(T: int, d: int, E: int, k: int, n: int) -> int:
     return int(_lib.load().mova_workspace_size(T, d, E, k, n))

@@ -69,3 +69,15 @@ def test_status_without_a_call_on_this_stream_is_an_error(fresh):
     current["handle"] = 0x5000
     with pytest.raises(ValueError, match="default workspace"):
         api.get_status(device="cpu")
+
+
+def test_release_drops_every_default_workspace(fresh):
+    current, _ = fresh
+    api._workspace(1000, "cpu")
+    current["handle"] = 0x2000
+    api._workspace(1000, "cpu")
+    assert len(api._WS) == 2
+    api.release_workspaces()
+    assert api._WS == {}
+    with pytest.raises(ValueError):
+        api.get_status(device="cpu")
