@@ -38,6 +38,15 @@
  *    mova_get_status().  Offending entries are clamped so that no access
  *    leaves its buffer.
  *  - T == 0 is a valid no-op and returns MOVA_OK.
+ *  - The weights (Wr, br, Wv and prepared router planes) are read as
+ *    constants.  A call's first kernel is chained to the kernel before it
+ *    on the stream with programmatic dependent launch, and the router
+ *    kernels start reading Wr and br before they wait for that kernel.
+ *    Inputs and outputs (x, idx, w, v, the workspace) are touched only after
+ *    the wait.  A caller that writes router weights with a kernel (an online
+ *    bias update, say) must let it complete before the call: write them on
+ *    another stream and make this one wait on an event recorded after the
+ *    write, or synchronize.
  *  - Supported on the GPU: 1 <= E <= 64, 1 <= k <= min(E, 8), d % 64 == 0,
  *    n % 128 == 0, T * k <= 131072; dtypes x/Wv/v all fp32, or all bf16
  *    (router Wr/br always fp32).  The weight-streaming expert kernel also
