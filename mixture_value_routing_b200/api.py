@@ -62,6 +62,14 @@ def _need(t: torch.Tensor, name: str, dtypes=None, ndim=None):
         raise ValueError(f"{name} must have {ndim} dims")
 
 
+def _shape(t: torch.Tensor, name: str, want) -> None:
+    """The library sees only pointers and the sizes passed with them, so a
+    tensor of the wrong shape would be read or written out of bounds: refuse
+    it here."""
+    if t.shape != want:
+        raise ValueError(f"{name}: shape {tuple(t.shape)}, expected {tuple(want)}")
+
+
 class Workspace:
     """A device workspace that grows on demand."""
 
@@ -171,6 +179,8 @@ def route(x: torch.Tensor, Wr: torch.Tensor, br: torch.Tensor, k: int = 4, scale
     _need(br, "br", (torch.float32,), 1)
     T, d = x.shape
     E = Wr.shape[0]
+    _shape(Wr, "Wr", (E, d))
+    _shape(br, "br", (E,))
     idx = torch.empty((T, k), dtype=torch.int32, device=x.device)
     w = torch.empty((T, k), dtype=torch.float32, device=x.device)
     lib = _lib.load()
@@ -246,6 +256,9 @@ def value(x: torch.Tensor, idx: torch.Tensor, w: torch.Tensor, Wv: torch.Tensor,
     T, d = x.shape
     E, n, stride, Wb = _expert_view(Wv, rows)
     k = idx.shape[1]
+    _shape(idx, "idx", (T, k))
+    _shape(w, "w", (T, k))
+    _shape(Wv, "Wv", (E, Wv.shape[1], d))
     v = torch.empty((T, n), dtype=x.dtype, device=x.device)
     nbytes = workspace_size(T, d, E, k, n)
     if ws is None:
@@ -279,6 +292,9 @@ def value_attend(x: torch.Tensor, idx: torch.Tensor, w: torch.Tensor, Wv: torch.
     H = probs.shape[0]
     if probs.shape[1] != L:
         raise ValueError("probs: (H, L) for the L cached positions of x")
+    _shape(idx, "idx", (L, k))
+    _shape(w, "w", (L, k))
+    _shape(Wv, "Wv", (E, n, d))
     o = torch.empty((H, 128), dtype=torch.float32, device=x.device)
     lib = _lib.load()
     nbytes = int(lib.mova_attend_workspace_size(L, d, E, k, n, H))
@@ -307,7 +323,13 @@ def value_routed(x: torch.Tensor, Wr: torch.Tensor, br: torch.Tensor, Wv: torch.
     _need(Wv, "Wv", (x.dtype,), 3)
     T, d = x.shape
     E, n, stride, Wb = _expert_view(Wv, rows)
+    _shape(Wr, "Wr", (E, d))
+    _shape(br, "br", (E,))
+    _shape(Wv, "Wv", (E, Wv.shape[1], d))
     dev = x.device
+    if out is not None:
+        _need(out, "out", (x.dtype,), 2)
+        _shape(out, "out", (T, n))
     v = out if out is not None else torch.empty((T, n), dtype=x.dtype, device=dev)
     idx = w = None
     if return_routing:
@@ -364,6 +386,9 @@ def value_routed_host(x: torch.Tensor, Wr: torch.Tensor, br: torch.Tensor, Wv: t
     _need(Wv, "Wv", (x.dtype,), 3)
     T, d = x.shape
     E, n = Wv.shape[0], Wv.shape[1]
+    _shape(Wr, "Wr", (E, d))
+    _shape(br, "br", (E,))
+    _shape(Wv, "Wv", (E, n, d))
     v = _host_out(out, (T, n), x.dtype)
     idx = w = None
     if return_routing:
@@ -388,6 +413,9 @@ def value_host(x: torch.Tensor, idx: torch.Tensor, w: torch.Tensor, Wv: torch.Te
     T, d = x.shape
     E, n = Wv.shape[0], Wv.shape[1]
     k = idx.shape[1]
+    _shape(idx, "idx", (T, k))
+    _shape(w, "w", (T, k))
+    _shape(Wv, "Wv", (E, n, d))
     v = _host_out(out, (T, n), x.dtype)
     if ws is None:
         ws = _workspace(workspace_size_host(T, d, E, k, n), Wv.device, stream)
@@ -414,6 +442,9 @@ def value_attend_host(x: torch.Tensor, idx: torch.Tensor, w: torch.Tensor, Wv: t
     H = probs.shape[0]
     if probs.shape[1] != L:
         raise ValueError("probs: (H, L) for the L cached positions of x")
+    _shape(idx, "idx", (L, k))
+    _shape(w, "w", (L, k))
+    _shape(Wv, "Wv", (E, n, d))
     o = _host_out(out, (H, 128), torch.float32)
     if ws is None:
         ws = _workspace(attend_workspace_size_host(L, d, E, k, n, H), Wv.device, stream)

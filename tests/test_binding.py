@@ -81,3 +81,54 @@ def test_release_drops_every_default_workspace(fresh):
     assert api._WS == {}
     with pytest.raises(ValueError):
         api.get_status(device="cpu")
+
+
+class _Tensor:
+    """Shape-only stand-in for a device tensor: the device checks are
+    skipped below, so the shape checks run without a GPU."""
+
+    def __init__(self, *shape, dtype=torch.bfloat16):
+        self.shape = torch.Size(shape)
+        self.dtype = dtype
+        self.device = torch.device("cpu")
+
+    def dim(self):
+        return len(self.shape)
+
+
+@pytest.mark.parametrize("case", ["Wr rows", "Wr width", "br", "Wv width", "out"])
+def test_value_routed_refuses_mismatched_shapes(monkeypatch, case):
+    """A tensor whose shape disagrees with x's and Wv's is refused before
+    the library sees its pointer (which it would read or write out of bounds)."""
+    monkeypatch.setattr(api, "_need", lambda *a, **k: None)
+    T, d, E, n = 8, 2560, 64, 1024
+    x, Wv = _Tensor(T, d), _Tensor(E, n, d)
+    Wr, br, out = _Tensor(E, d, dtype=torch.float32), _Tensor(E, dtype=torch.float32), _Tensor(T, n)
+    if case == "Wr rows":
+        Wr = _Tensor(E - 1, d, dtype=torch.float32)
+    elif case == "Wr width":
+        Wr = _Tensor(E, d - 64, dtype=torch.float32)
+    elif case == "br":
+        br = _Tensor(E + 1, dtype=torch.float32)
+    elif case == "Wv width":
+        Wv = _Tensor(E, n, d - 64)
+    else:
+        out = _Tensor(T - 1, n)
+    with pytest.raises(ValueError, match="shape"):
+        api.value_routed(x, Wr, br, Wv, out=out)
+
+
+@pytest.mark.parametrize("case", ["idx rows", "w shape", "Wv width"])
+def test_value_refuses_mismatched_shapes(monkeypatch, case):
+    monkeypatch.setattr(api, "_need", lambda *a, **k: None)
+    T, d, E, n, k = 8, 2560, 64, 1024, 4
+    x, Wv = _Tensor(T, d), _Tensor(E, n, d)
+    idx, w = _Tensor(T, k, dtype=torch.int8), _Tensor(T, k, dtype=torch.float16)
+    if case == "idx rows":
+        idx = _Tensor(T - 1, k, dtype=torch.int8)
+    elif case == "w shape":
+        w = _Tensor(T, k + 1, dtype=torch.float16)
+    else:
+        Wv = _Tensor(E, n, d + 64)
+    with pytest.raises(ValueError, match="shape"):
+        api.value(x, idx, w, Wv)
