@@ -39,8 +39,8 @@
  *    leaves its buffer.
  *  - T == 0 is a valid no-op and returns MOVA_OK.
  *  - The weights (Wr, br, Wv and prepared router planes) are read as
- *    constants.  A call's first kernel is chained to the kernel before it
- *    on the stream with programmatic dependent launch, and the router
+ *    constants.  A call's first kernel may be chained to the kernel before
+ *    it on the stream with programmatic dependent launch, and the router
  *    kernels start reading Wr and br before they wait for that kernel.
  *    Inputs and outputs (x, idx, w, v, the workspace) are touched only after
  *    the wait.  A caller that writes router weights with a kernel (an online
@@ -121,7 +121,9 @@ mova_status mova_route(const void* x, mova_dtype x_dt, const float* Wr, const fl
  *   pos     (T*k)  int32 out: inverse of perm
  * Bit-exact and deterministic.  An index outside [0, E) is clamped and
  * raises MOVA_ERR_DEVICE_CHECK in the status word held by `ws`
- * (ws_bytes >= mova_workspace_size(T, 64, E, k, 128) suffices). */
+ * (ws_bytes >= mova_workspace_size(T, 64, E, k, 128) suffices).
+ * Source: "So what does it cost?" (the released combine visits each touched
+ * expert once with its tokens; this is that grouping, made deterministic). */
 mova_status mova_permute(const int32_t* idx, int T, int E, int k,
                          int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* pos,
                          void* ws, size_t ws_bytes, void* stream);
@@ -133,7 +135,10 @@ mova_status mova_permute(const int32_t* idx, int T, int E, int k,
  *   w   (T, k)    w_dt in {MOVA_F32, MOVA_F16}; used as given (no renormalisation)
  *   Wv  (E, n, d) wv_dt == x_dt; expert e's weight is output-major (n rows of d)
  *   v   (T, n)    same dtype as x; equals (T, n/128, 128) GQA value heads
- *   ws  device workspace of ws_bytes >= mova_workspace_size(T, d, E, k, n) */
+ *   ws  device workspace of ws_bytes >= mova_workspace_size(T, d, E, k, n)
+ * Source: "IFM K2 Horizon Deep Dive ...", Section 4, Option B (the cache
+ * keeps x, the top-4 indices and fp16 weights; V is recomputed), with the
+ * mixture of "Where the routing happens". */
 mova_status mova_value(const void* x, mova_dtype x_dt, const void* idx, mova_dtype idx_dt,
                        const void* w, mova_dtype w_dt, const void* Wv, mova_dtype wv_dt,
                        int T, int d, int E, int k, int n, void* v,
@@ -142,7 +147,9 @@ mova_status mova_value(const void* x, mova_dtype x_dt, const void* idx, mova_dty
 /* Full value path: route, group, expert projections with SiLU x weight,
  * fixed-order combine.  Arguments as in mova_route and mova_value; idx_out
  * (T, k) int32 and w_out (T, k) fp32 are optional copies of the routing
- * (pass NULL to skip). */
+ * (pass NULL to skip).  Source: "Where the routing happens" (the forward:
+ * router, gate with the bias, top-4, scale 2.5, SiLU mixture, reshape to
+ * 128-wide heads). */
 mova_status mova_value_routed(const void* x, mova_dtype x_dt, const float* Wr, const float* br,
                               const void* Wv, mova_dtype wv_dt,
                               int T, int d, int E, int k, int n, float scale, void* v,
