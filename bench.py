@@ -287,6 +287,21 @@ def _replay_for(graph, seconds, step_s, K):
     return reps
 
 
+# About 2 ms of spinning at the B200's clocks: longer than the host takes to
+# record an event and submit the largest timed graph.
+COVER_CYCLES = 4_000_000
+
+
+def _cover_submission():
+    """Keep the stream busy while the host records the start event and
+    submits the timed graph: the start event then fires only when the spin
+    ends, with the graph's kernels already queued, so the timed region holds
+    the K steps' device work and not the host's submission latency (which
+    otherwise adds tens of microseconds to a region of a few hundred)."""
+    import torch
+    torch.cuda._sleep(COVER_CYCLES)
+
+
 def workload_config(a, name, world):
     """The `config` of a workload's record: what the workload is and how L2 is
     kept from serving the weights, the same on the reference arm's line as on
@@ -404,6 +419,7 @@ def measure_workload(a, name, K, layers, device, dist_on, world, rank, peaks, pe
         _replay_for(graph, 0.25, est_step_s, K)
         barrier(dist_on)
         torch.cuda.synchronize()
+        _cover_submission()
         t0.record()
         graph.replay()
         t1.record()
@@ -416,6 +432,7 @@ def measure_workload(a, name, K, layers, device, dist_on, world, rank, peaks, pe
     assert status == "MOVA_OK", status
     p0 = torch.cuda.Event(enable_timing=True)
     p1 = torch.cuda.Event(enable_timing=True)
+    _cover_submission()
     p0.record()
     pgraph.replay()
     p1.record()
