@@ -6,7 +6,9 @@
 
 A step is one pass of the whole value path over one batch of synthetic tokens
 (seeded, see mova_inputs).  The timed region is one CUDA graph holding all K
-steps, launched once between a barrier + synchronize on both sides; the expert
+steps, launched once between a barrier + synchronize on both sides (a short
+spin kernel before the start event hides the host's submission of the graph,
+so the events bracket only the K steps' device work); the expert
 weights rotate over several layers (each layer's weights are read once per
 step, as in a real forward pass), so the weights a step reads are far larger
 than L2.  Per-kernel durations come from a second replay with stage events
@@ -14,8 +16,9 @@ recorded inside the graph, less the measured cost of an empty event pair.
 Rank 0 prints one JSON line: the headline workload (--workload, decode T=8 by
 default) and, as sub-records of the same line, the other workloads of the
 metric and scope (--also: prefill T=4096, skewed prefill T=16384,
-routing-given L=32768), each with its own steps, roofline, end-to-end rate and
-CPU baseline.  Multi-GPU: one process per GPU, each on its own batch (weak
+routing-given L=32768, attend), each with its own steps, roofline, end-to-end
+rate and CPU baseline; `config` describes the workload (the same on the
+reference arm's line), `run` what the run measured.  Multi-GPU: one process per GPU, each on its own batch (weak
 scaling, no collective in the data path).
 """
 from __future__ import annotations
