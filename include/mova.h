@@ -422,9 +422,11 @@ unsigned long long mova_launch_count(void);
  *    ids, every call looks the address up.
  *  - All calls share the one array and it keeps the last call's contents;
  *    each call's first kernel resets the status fields it relies on, and
- *    every other part is fully rewritten.  Calls that overlap on the GPU
- *    (different streams, or other devices' work is unaffected) race: order
- *    them on one stream.  The device status word is not exposed. */
+ *    every other part is fully rewritten.  Calls on one device that may
+ *    overlap on the GPU (calls on different streams) race: order them on one
+ *    stream.  Each device holds its own copy of the array, so calls on
+ *    different devices do not interfere.  The device status word is not
+ *    exposed. */
 mova_status mova_value_routed_noalloc(const void* x, mova_dtype x_dt, const float* Wr,
                                       const float* br, const void* Wv, mova_dtype wv_dt,
                                       int T, int d, int E, int k, int n, float scale, void* v,
