@@ -241,6 +241,15 @@ def test_full_stream_resident_boundary(api, T, d):
     _full(api, T, d, 16, 4, 256, "bf16", seed=d, path="stream")
 
 
+@pytest.mark.parametrize("T,n", [(8, 128), (1, 128), (5, 384)])
+def test_full_stream_fewer_columns_than_ctas(api, T, n):
+    """Decode batches whose n output columns are fewer than, or not a
+    multiple of, the CTAs the streaming kernel runs (one per SM): at n = 128
+    some CTAs own no column at all and must leave without work, the others
+    one; every value still matches the oracle."""
+    _full(api, T, 2560, 64, 4, n, "bf16", seed=n + T, path="stream")
+
+
 @pytest.mark.parametrize("T", [24, 64])
 def test_full_stream_mid(api, T):
     """Weight-streaming path with more than 8 tokens on some experts."""
